@@ -1,0 +1,131 @@
+"""CPU oracle of the Engram N-gram Embedding path (hash, gather, backward).
+
+TEST INFRASTRUCTURE ONLY. Only `tests/`, `__graft_entry__.smoke()` and the
+CPU-baseline / reference legs of `bench.py` may import this package. The
+product path (`hashed_gram_embedding_raw_b200`) never imports it and shares no
+code with it.
+
+`engram_oracle.c` is the oracle proper (scalar C, fp64 accumulation);
+`bruteforce.py` is an independent exact-integer statement of the hash that
+pins it on tiny inputs. This module compiles the C file with gcc (`build()`)
+and wraps it with ctypes over NumPy arrays.
+
+Parity of the hash against the released checkpoint is unpinned: the engram
+page prints no worked example. What pins each function is listed in the
+oracle tests.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "engram_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+F32, BF16, F16 = 0, 1, 2
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc into oracle/liboracle.so."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-Wall", "-Wextra", "-shared",
+                               "-fPIC", "-o", tmp, _SRC])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def build_mutant(mutant: int, outdir: str):
+    """Build a copy of the oracle with one planted mistake (tests only) and
+    return it loaded; see ORACLE_MUTANT in engram_oracle.c."""
+    path = os.path.join(outdir, f"liboracle_mutant{mutant}.so")
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-shared", "-fPIC",
+                           f"-DORACLE_MUTANT={int(mutant)}", "-o", path, _SRC])
+    return _declare(ctypes.CDLL(path))
+
+
+def _declare(L):
+    P = ctypes.c_void_p
+    i32, i64 = ctypes.c_int32, ctypes.c_int64
+    L.oracle_hash.argtypes = [i32, i32, P, P, P, i64, i32, P, P, i32, i64, P]
+    L.oracle_hash.restype = ctypes.c_int
+    L.oracle_gather.argtypes = [P, i64, i64, P, i64, P]
+    L.oracle_gather.restype = ctypes.c_int
+    L.oracle_backward.argtypes = [P, i64, P, ctypes.c_int, i32, P, P, P]
+    L.oracle_backward.restype = ctypes.c_int
+    return L
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        build()
+        _lib = _declare(ctypes.CDLL(_LIB))
+    return _lib
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def hash_ids(ids, cu, params) -> np.ndarray:
+    """Global row IDs [T, H] (int64) of every head for every token."""
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    T = ids.shape[0]
+    N, K = params["ngram_size"], params["heads_per_ngram"]
+    H = (N - 1) * K
+    mult = np.asarray(params["multipliers"], dtype=np.int64)
+    vocab = np.asarray(params["vocab_sizes"], dtype=np.int64)
+    off = np.asarray(params["offsets"], dtype=np.int64)
+    out = np.empty((T, H), dtype=np.int64)
+    if cu is None:
+        cu_arr, nseq, cu_p = None, 1, None
+    else:
+        cu_arr = np.ascontiguousarray(cu, dtype=np.int32)
+        nseq, cu_p = cu_arr.shape[0] - 1, _ptr(cu_arr)
+    rc = lib().oracle_hash(N, K, _ptr(mult), _ptr(vocab), _ptr(off),
+                           int(params["fill_id"]), int(params["eos_id"]),
+                           _ptr(ids), cu_p, nseq, T, _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle_hash: invalid arguments")
+    return out
+
+
+def gather(table: np.ndarray, idx) -> np.ndarray:
+    """out[i, :] = table[idx[i], :] bit for bit; table is any [R, D] array."""
+    table = np.ascontiguousarray(table)
+    idx = np.ascontiguousarray(np.asarray(idx).reshape(-1), dtype=np.int64)
+    out = np.empty((idx.shape[0],) + table.shape[1:], dtype=table.dtype)
+    row_bytes = table.strides[0] if table.ndim > 1 else table.itemsize
+    rc = lib().oracle_gather(_ptr(table), table.shape[0], row_bytes, _ptr(idx),
+                             idx.shape[0], _ptr(out))
+    if rc != 0:
+        raise IndexError("oracle_gather: row index out of range")
+    return out
+
+
+def backward(idx, dout: np.ndarray, dtype: int):
+    """(uniq_rows int64 [U], row_grads fp32 [U, D]) of the row-gradient sum.
+
+    `dout` holds raw values of `dtype` (F32: float32 array; BF16/F16: uint16
+    bit patterns), shape [n, D].
+    """
+    idx = np.ascontiguousarray(np.asarray(idx).reshape(-1), dtype=np.int64)
+    dout = np.ascontiguousarray(dout)
+    n, D = dout.shape
+    assert n == idx.shape[0]
+    uniq = np.empty(max(n, 1), dtype=np.int64)
+    grads = np.empty((max(n, 1), D), dtype=np.float32)
+    nu = np.zeros(1, dtype=np.int64)
+    rc = lib().oracle_backward(_ptr(idx), n, _ptr(dout), dtype, D, _ptr(uniq),
+                               _ptr(grads), _ptr(nu))
+    if rc != 0:
+        raise ValueError("oracle_backward: invalid arguments")
+    U = int(nu[0])
+    return uniq[:U].copy(), grads[:U].copy()

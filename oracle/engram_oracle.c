@@ -1,0 +1,255 @@
+/*
+ * engram_oracle.c -- CPU oracle for the Engram N-gram Embedding ("ple") path.
+ *
+ * TEST INFRASTRUCTURE ONLY. Plain, slow, scalar C that the parity tests, the
+ * smoke check and the CPU-baseline leg of the benchmark compare the CUDA path
+ * against. It shares no code, header, table or constant with the CUDA library
+ * and is never called by the product path.
+ *
+ * Source: the Qwen3.8-Flash-Next engram API page (NeMo AutoModel docs),
+ * class Qwen3_8_FlashNextNGramEmbedding and its methods
+ * _shift_right_after_eos, _hash_input_ids, _lookup_ngram_ids and forward,
+ * and class Qwen3_8_FlashNextOwnerShardedEmbedding (an owner accumulates each
+ * row's gradient). Readings taken where the page is silent or cut short:
+ *   - per-token terms are combined by XOR of wrapped int64 products
+ *     (the page's "original DeepSeek Engram" lineage; not printed);
+ *   - multiplier k multiplies the token k positions back (k = 0: current);
+ *   - all heads of one order share that order's mix; heads differ only in
+ *     their prime modulus and global offset;
+ *   - positions lacking valid context read the value `fill` (0 by default;
+ *     the page's sentence is cut off);
+ *   - context also resets at every sequence start given by cu_seqlens;
+ *   - backward: one fp64 sum per distinct row over its lookups in ascending
+ *     lookup order, rounded once to fp32; rows reported in ascending order.
+ *
+ * Parity of the hash against the released checkpoint is unpinned: the page
+ * prints no worked example (see the tests for what does pin each function).
+ */
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ORACLE_MUTANT (tests only) plants one known mistake so the tests can show
+ * that their pins catch it; the default build defines none. */
+#ifndef ORACLE_MUTANT
+#define ORACLE_MUTANT 0
+#endif
+
+#define ORACLE_OK 0
+#define ORACLE_EINVAL (-1)
+
+/* dtype codes of the raw buffers handed to the oracle */
+#define ORACLE_F32 0
+#define ORACLE_BF16 1
+#define ORACLE_F16 2
+
+/* ------------------------------------------------------------------ hash */
+
+/*
+ * _shift_right_after_eos(input_ids, shift), one position: read the token
+ * `shift` places before t without crossing an EOS boundary. An EOS ends the
+ * segment it closes, so reading across position p (p in t-shift .. t-1) is
+ * forbidden when ids[p] is EOS. Positions before the sequence start also lack
+ * valid context. Either way the result is `fill`.
+ */
+static int64_t shift_right_after_eos(const int32_t *ids, int64_t seq_begin,
+                                     int64_t t, int shift, int32_t eos,
+                                     int64_t fill)
+{
+    if (ORACLE_MUTANT == 5)
+        seq_begin = 0; /* mutant: no reset at sequence starts */
+    if (t - shift < seq_begin)
+        return fill;
+    for (int64_t p = t - shift; p < t + (ORACLE_MUTANT == 2); ++p)
+        if (ids[p] == eos)
+            return fill;
+    return (int64_t)ids[t - shift];
+}
+
+/* Signed int64 product with two's-complement wrap ("signed int64 overflow"). */
+static int64_t wrap_mul(int64_t a, int64_t b)
+{
+    return (int64_t)((uint64_t)a * (uint64_t)b);
+}
+
+/* Remainder in [0, m) for m > 0 ("positive remainders"). */
+static int64_t positive_mod(int64_t a, int64_t m)
+{
+    int64_t r = a % m;
+    if (r < 0 && ORACLE_MUTANT != 4)
+        r += m;
+    return r;
+}
+
+/*
+ * _hash_input_ids: global table row of every head for every token.
+ *   ids        [T] raw token IDs, cu [nseq+1] sequence bounds (NULL: one sequence)
+ *   mult       [ngram_size]
+ *   vocab, off [(ngram_size-1) * heads_per_ngram]
+ *   out        [T, (ngram_size-1) * heads_per_ngram] int64
+ * Heads 0..K-1 hash bigrams, K..2K-1 trigrams, and so on.
+ */
+int oracle_hash(int32_t ngram_size, int32_t heads_per_ngram,
+                const int64_t *mult, const int64_t *vocab, const int64_t *off,
+                int64_t fill, int32_t eos,
+                const int32_t *ids, const int32_t *cu, int32_t nseq, int64_t T,
+                int64_t *out)
+{
+    if (ngram_size < 2 || heads_per_ngram < 1 || T < 0)
+        return ORACLE_EINVAL;
+    const int H = (ngram_size - 1) * heads_per_ngram;
+    for (int h = 0; h < H; ++h)
+        if (vocab[h] <= 0)
+            return ORACLE_EINVAL;
+
+    /* shifted[k][t] = _shift_right_after_eos(ids, k)[t] for k = 1..ngram_size-1 */
+    int64_t *shifted = (int64_t *)malloc(sizeof(int64_t) * (size_t)(T > 0 ? T : 1) *
+                                         (size_t)ngram_size);
+    if (!shifted)
+        return ORACLE_EINVAL;
+    int32_t ns = cu ? nseq : 1;
+    for (int32_t s = 0; s < ns; ++s) {
+        int64_t b = cu ? cu[s] : 0, e = cu ? cu[s + 1] : T;
+        if (b < 0 || e < b || e > T) {
+            free(shifted);
+            return ORACLE_EINVAL;
+        }
+        for (int64_t t = b; t < e; ++t) {
+            shifted[t * ngram_size + 0] = ids[t];
+            for (int k = 1; k < ngram_size; ++k)
+                shifted[t * ngram_size + k] =
+                    shift_right_after_eos(ids, b, t, k, eos, fill);
+        }
+    }
+
+    for (int64_t t = 0; t < T; ++t) {
+        const int64_t *x = &shifted[t * ngram_size];
+        for (int n = 2; n <= ngram_size; ++n) {
+            /* order-n mix: XOR of x_k * m_k over the n most recent tokens */
+            int64_t mix = 0;
+            for (int k = 0; k < n; ++k) {
+                if (ORACLE_MUTANT == 1)
+                    mix += wrap_mul(x[k], mult[k]);
+                else if (ORACLE_MUTANT == 3)
+                    mix ^= wrap_mul(x[k], mult[n - 1 - k]);
+                else
+                    mix ^= wrap_mul(x[k], mult[k]);
+            }
+            for (int i = 0; i < heads_per_ngram; ++i) {
+                int h = (n - 2) * heads_per_ngram + i;
+                out[t * H + h] = off[h] + positive_mod(mix, vocab[h]);
+            }
+        }
+    }
+    free(shifted);
+    return ORACLE_OK;
+}
+
+/* ---------------------------------------------------------------- gather */
+
+/*
+ * _lookup_ngram_ids / OwnerShardedEmbedding.forward on a single-rank table:
+ * out[i, :] = table[idx[i], :], copied bit for bit. Rows are `row_bytes` wide.
+ */
+int oracle_gather(const void *table, int64_t rows, int64_t row_bytes,
+                  const int64_t *idx, int64_t n, void *out)
+{
+    const char *src = (const char *)table;
+    char *dst = (char *)out;
+    for (int64_t i = 0; i < n; ++i) {
+        if (idx[i] < 0 || idx[i] >= rows)
+            return ORACLE_EINVAL;
+        memcpy(dst + i * row_bytes, src + idx[i] * row_bytes, (size_t)row_bytes);
+    }
+    return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------- backward */
+
+static double load_value(const void *buf, int dtype, int64_t i)
+{
+    if (dtype == ORACLE_F32) {
+        return (double)((const float *)buf)[i];
+    } else if (dtype == ORACLE_BF16) {
+        /* bfloat16: the upper 16 bits of an IEEE binary32 */
+        uint32_t bits = (uint32_t)((const uint16_t *)buf)[i] << 16;
+        float f;
+        memcpy(&f, &bits, sizeof f);
+        return (double)f;
+    } else {
+        /* IEEE binary16: 1 sign, 5 exponent (bias 15), 10 fraction bits */
+        uint16_t h = ((const uint16_t *)buf)[i];
+        int sign = h >> 15, ex = (h >> 10) & 0x1f, fr = h & 0x3ff;
+        double v;
+        if (ex == 0)
+            v = (double)fr * (1.0 / 16777216.0); /* fr * 2^-24 */
+        else if (ex == 31)
+            v = fr ? (0.0 / 0.0) : (1.0 / 0.0);
+        else {
+            v = 1.0 + fr / 1024.0;
+            int e = ex - 15;
+            while (e > 0) { v *= 2.0; --e; }
+            while (e < 0) { v *= 0.5; ++e; }
+        }
+        return sign ? -v : v;
+    }
+}
+
+typedef struct { int64_t row; int64_t j; } lookup_t;
+
+static int cmp_lookup(const void *a, const void *b)
+{
+    const lookup_t *x = (const lookup_t *)a, *y = (const lookup_t *)b;
+    if (x->row != y->row)
+        return x->row < y->row ? -1 : 1;
+    return x->j < y->j ? -1 : (x->j > y->j);
+}
+
+/*
+ * Row-gradient accumulation of the lookup (the owner side of the page's
+ * backward): for every distinct row r among idx[0..n), in ascending order,
+ *   grads[u, :] = fp32( sum over j with idx[j] == r, ascending j, of dout[j, :] )
+ * with the sum taken in fp64. uniq[u] = r; *num_unique = number of rows.
+ */
+int oracle_backward(const int64_t *idx, int64_t n, const void *dout, int dtype,
+                    int32_t dim, int64_t *uniq, float *grads, int64_t *num_unique)
+{
+    if (n < 0 || dim <= 0)
+        return ORACLE_EINVAL;
+    lookup_t *l = (lookup_t *)malloc(sizeof(lookup_t) * (size_t)(n > 0 ? n : 1));
+    double *acc = (double *)malloc(sizeof(double) * (size_t)dim);
+    if (!l || !acc) {
+        free(l);
+        free(acc);
+        return ORACLE_EINVAL;
+    }
+    for (int64_t j = 0; j < n; ++j) {
+        l[j].row = idx[j];
+        l[j].j = j;
+    }
+    qsort(l, (size_t)n, sizeof(lookup_t), cmp_lookup);
+
+    int64_t u = 0;
+    for (int64_t a = 0; a < n;) {
+        int64_t b = a;
+        for (int d = 0; d < dim; ++d)
+            acc[d] = 0.0;
+        while (b < n && (l[b].row == l[a].row ||
+                         (ORACLE_MUTANT == 7 && l[b].row == l[a].row + 1))) {
+            for (int d = 0; d < dim; ++d)
+                acc[d] = ORACLE_MUTANT == 6
+                    ? (double)((float)acc[d] + (float)load_value(dout, dtype, l[b].j * dim + d))
+                    : acc[d] + load_value(dout, dtype, l[b].j * dim + d);
+            ++b;
+        }
+        uniq[u] = l[a].row;
+        for (int d = 0; d < dim; ++d)
+            grads[u * dim + d] = (float)acc[d];
+        ++u;
+        a = b;
+    }
+    *num_unique = u;
+    free(l);
+    free(acc);
+    return ORACLE_OK;
+}

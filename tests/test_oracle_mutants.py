@@ -1,0 +1,53 @@
+"""Planted mistakes in the oracle must be caught by its pins (CPU only).
+
+Each mutant is the oracle rebuilt with one known mistake (ORACLE_MUTANT in
+engram_oracle.c): a plausible slip in the hash (operator, reset position,
+multiplier pairing, remainder sign, sequence reset) or in the backward
+(accumulation precision, grouping). The pins of test_oracle_hash.py and
+test_oracle_gather_backward.py are run against each; at least one must fail.
+"""
+
+import pytest
+
+import oracle
+from tests import test_oracle_gather_backward as GB
+from tests import test_oracle_hash as TH
+
+HASH_PINS = [
+    TH.test_hand_worked_example,
+    lambda: [TH.test_bruteforce_adversarial(c, f) for c in range(len(TH.ADVERSARIAL))
+             for f in (0, 17)],
+    lambda: [TH.test_bruteforce_random(s, 3, 8) for s in range(6)],
+    TH.test_single_term_multipliers_isolate_positions,
+    TH.test_token_after_eos_hashes_like_sequence_start,
+    TH.test_eos_token_keeps_its_own_left_context,
+]
+BACKWARD_PINS = [
+    lambda: [GB.test_backward_matches_add_at(s) for s in range(4)],
+    GB.test_backward_bf16_and_f16_decode,
+    GB.test_backward_adjoint_identity,
+    lambda: GB.test_backward_per_head_mass_and_counts("tiny"),
+]
+
+MUTANTS = {
+    1: ("add instead of xor", HASH_PINS),
+    2: ("reset before EOS instead of after", HASH_PINS),
+    3: ("multipliers paired in reverse", HASH_PINS),
+    4: ("truncating remainder", HASH_PINS),
+    5: ("no reset at cu_seqlens starts", HASH_PINS),
+    6: ("fp32 accumulation", BACKWARD_PINS),
+    7: ("adjacent rows merged", BACKWARD_PINS),
+}
+
+
+@pytest.mark.parametrize("mutant", sorted(MUTANTS))
+def test_pins_catch_planted_mistake(mutant, tmp_path, monkeypatch):
+    what, pins = MUTANTS[mutant]
+    monkeypatch.setattr(oracle, "_lib", oracle.build_mutant(mutant, str(tmp_path)))
+    caught = []
+    for pin in pins:
+        try:
+            pin()
+        except AssertionError:
+            caught.append(pin)
+    assert caught, f"no pin caught mutant {mutant} ({what})"
