@@ -1,0 +1,25 @@
+"""B200-native Engram N-gram Embedding: hash, gather and compact backward.
+
+Python face of the C ABI in include/engram.h (libengram_b200.so, sm_100a).
+Every step runs in the library's CUDA kernels; this package only marshals
+arguments and allocates buffers with torch. Importing it fails if the library
+has not been built (`python hashed_gram_embedding_raw_b200/build.py`).
+"""
+
+from ._binding import (ENGRAM_BF16, ENGRAM_DEVERR_CU_SEQLENS, ENGRAM_DEVERR_ROW_RANGE,
+                       ENGRAM_EINVAL, ENGRAM_ECUDA, ENGRAM_ENOSPC, ENGRAM_F16, ENGRAM_F32,
+                       ENGRAM_OK, EXPORTED, LIB_PATH, EngramError, EngramParams,
+                       engram_abi_version, engram_backward, engram_backward_reduce,
+                       engram_backward_sort, engram_backward_workspace_size, engram_gather,
+                       engram_get_device_error, engram_hash, engram_hash_gather,
+                       engram_host_floor_mod, engram_launch_count, lib, make_params,
+                       status_string)
+
+__all__ = [
+    "ENGRAM_BF16", "ENGRAM_DEVERR_CU_SEQLENS", "ENGRAM_DEVERR_ROW_RANGE", "ENGRAM_EINVAL",
+    "ENGRAM_ECUDA", "ENGRAM_ENOSPC", "ENGRAM_F16", "ENGRAM_F32", "ENGRAM_OK", "EXPORTED",
+    "LIB_PATH", "EngramError", "EngramParams", "engram_abi_version", "engram_backward",
+    "engram_backward_reduce", "engram_backward_sort", "engram_backward_workspace_size",
+    "engram_gather", "engram_get_device_error", "engram_hash", "engram_hash_gather",
+    "engram_host_floor_mod", "engram_launch_count", "lib", "make_params", "status_string",
+]

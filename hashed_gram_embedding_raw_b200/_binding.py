@@ -1,0 +1,312 @@
+"""ctypes binding of libengram_b200.so (include/engram.h).
+
+Argument marshalling only: every function checks tensor devices, dtypes and
+shapes, allocates outputs with torch when the caller passes none, and hands
+raw pointers plus the current CUDA stream to the C ABI. All computation runs
+in the library's sm_100a kernels; there is no fallback path. Importing this
+module fails loudly when the library has not been built.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "_lib", "libengram_b200.so")
+
+ENGRAM_OK, ENGRAM_EINVAL, ENGRAM_ENOSPC, ENGRAM_ECUDA = 0, 1, 2, 3
+ENGRAM_F32, ENGRAM_BF16, ENGRAM_F16 = 0, 1, 2
+ENGRAM_DEVERR_ROW_RANGE, ENGRAM_DEVERR_CU_SEQLENS = 1, 2
+ENGRAM_MAX_NGRAM, ENGRAM_MAX_HEADS = 4, 32
+
+_DTYPE_CODE = {torch.float32: ENGRAM_F32, torch.bfloat16: ENGRAM_BF16,
+               torch.float16: ENGRAM_F16}
+
+EXPORTED = (
+    "engram_hash", "engram_gather", "engram_hash_gather",
+    "engram_backward_workspace_size", "engram_backward", "engram_backward_sort",
+    "engram_backward_reduce", "engram_get_device_error", "engram_status_string",
+    "engram_abi_version", "engram_params_size", "engram_launch_count",
+    "engram_host_floor_mod",
+)
+
+
+class EngramError(RuntimeError):
+    """A C-ABI call returned a non-zero status."""
+
+    def __init__(self, what: str, status: int):
+        super().__init__(f"{what}: {status_string(status)}")
+        self.status = status
+
+
+class EngramParams(ctypes.Structure):
+    """Mirror of engram_params_t."""
+    _fields_ = [
+        ("ngram_size", ctypes.c_int32),
+        ("heads_per_ngram", ctypes.c_int32),
+        ("multipliers", ctypes.c_int64 * ENGRAM_MAX_NGRAM),
+        ("vocab_sizes", ctypes.c_int64 * ENGRAM_MAX_HEADS),
+        ("offsets", ctypes.c_int64 * ENGRAM_MAX_HEADS),
+        ("fill_id", ctypes.c_int64),
+        ("table_rows", ctypes.c_int64),
+        ("dim", ctypes.c_int32),
+        ("eos_id", ctypes.c_int32),
+    ]
+
+    @property
+    def heads(self) -> int:
+        return (self.ngram_size - 1) * self.heads_per_ngram
+
+
+def make_params(cfg: dict) -> EngramParams:
+    """EngramParams from a dict with the NGramEmbedding constructor fields
+    (ngram_size, heads_per_ngram, multipliers, vocab_sizes, offsets, eos_id,
+    fill_id) and the table shape (table_rows, dim)."""
+    p = EngramParams()
+    p.ngram_size = int(cfg["ngram_size"])
+    p.heads_per_ngram = int(cfg["heads_per_ngram"])
+    for k, m in enumerate(cfg["multipliers"]):
+        p.multipliers[k] = int(m)
+    for h, (v, o) in enumerate(zip(cfg["vocab_sizes"], cfg["offsets"])):
+        p.vocab_sizes[h] = int(v)
+        p.offsets[h] = int(o)
+    p.fill_id = int(cfg.get("fill_id", 0))
+    p.table_rows = int(cfg["table_rows"])
+    p.dim = int(cfg["dim"])
+    p.eos_id = int(cfg["eos_id"])
+    return p
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"Engram CUDA library not found at {LIB_PATH}; build it with "
+            "`python hashed_gram_embedding_raw_b200/build.py` (needs nvcc)")
+    L = ctypes.CDLL(LIB_PATH)
+    P, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    sig = {
+        "engram_hash": [P, P, P, i32, i64, P, P],
+        "engram_gather": [P, i32, i64, i32, P, i64, P, P],
+        "engram_hash_gather": [P, P, P, i32, i64, P, i32, P, P, P],
+        "engram_backward_workspace_size": [i64, i64, i32, ctypes.POINTER(sz)],
+        "engram_backward": [P, i64, i64, i32, P, i32, P, P, P, P, sz, P],
+        "engram_backward_sort": [P, i64, i64, i32, P, sz, P],
+        "engram_backward_reduce": [i64, i64, i32, P, i32, P, P, P, P, sz, P],
+        "engram_get_device_error": [ctypes.POINTER(ctypes.c_uint32), P],
+        "engram_status_string": [ctypes.c_int],
+        "engram_abi_version": [],
+        "engram_params_size": [],
+        "engram_launch_count": [],
+        "engram_host_floor_mod": [i64, i64, ctypes.POINTER(ctypes.c_int)],
+    }
+    for name, args in sig.items():
+        fn = getattr(L, name)
+        fn.argtypes = args
+        fn.restype = ctypes.c_int
+    L.engram_status_string.restype = ctypes.c_char_p
+    L.engram_params_size.restype = sz
+    L.engram_launch_count.restype = ctypes.c_uint64
+    L.engram_host_floor_mod.restype = i64
+    if L.engram_params_size() != ctypes.sizeof(EngramParams):
+        raise ImportError("engram_params_t layout differs between library and binding")
+    return L
+
+
+lib = _load()
+
+
+def status_string(status: int) -> str:
+    return lib.engram_status_string(int(status)).decode()
+
+
+def _check(rc: int, what: str):
+    if rc != ENGRAM_OK:
+        raise EngramError(what, rc)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _cuda(t: torch.Tensor, name: str, dtype=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    return t
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    try:
+        return _DTYPE_CODE[t.dtype]
+    except KeyError:
+        raise ValueError(f"unsupported dtype {t.dtype}") from None
+
+
+def _cu_args(cu_seqlens):
+    if cu_seqlens is None:
+        return None, 1
+    _cuda(cu_seqlens, "cu_seqlens", torch.int32)
+    return cu_seqlens, cu_seqlens.numel() - 1
+
+
+# ------------------------------------------------------------------ forward
+
+def engram_hash(params: EngramParams, ids: torch.Tensor, cu_seqlens=None, out_idx=None,
+                stream=None) -> torch.Tensor:
+    """Row indices [T, H] int32 of every hash head for every token."""
+    _cuda(ids, "ids", torch.int32)
+    T = ids.numel()
+    cu, nseq = _cu_args(cu_seqlens)
+    if out_idx is None:
+        out_idx = torch.empty((T, params.heads), dtype=torch.int32, device=ids.device)
+    _cuda(out_idx, "out_idx", torch.int32)
+    if out_idx.numel() != T * params.heads:
+        raise ValueError("out_idx must hold T * H elements")
+    _check(lib.engram_hash(ctypes.byref(params), _ptr(ids), _ptr(cu), nseq, T,
+                           _ptr(out_idx), _stream(stream)), "engram_hash")
+    return out_idx
+
+
+def engram_gather(table: torch.Tensor, idx: torch.Tensor, out=None, stream=None) -> torch.Tensor:
+    """out[i, :] = table[idx[i], :] for an int32 index tensor of any shape."""
+    _cuda(table, "table")
+    _cuda(idx, "idx", torch.int32)
+    rows, dim = table.shape
+    n = idx.numel()
+    if out is None:
+        out = torch.empty(tuple(idx.shape) + (dim,), dtype=table.dtype, device=table.device)
+    _cuda(out, "out", table.dtype)
+    if out.numel() != n * dim:
+        raise ValueError("out must hold n * dim elements")
+    _check(lib.engram_gather(_ptr(table), _dtype_code(table), rows, dim, _ptr(idx), n,
+                             _ptr(out), _stream(stream)), "engram_gather")
+    return out
+
+
+def engram_hash_gather(params: EngramParams, ids: torch.Tensor, table: torch.Tensor,
+                       cu_seqlens=None, out=None, out_idx=None, want_idx: bool = True,
+                       stream=None):
+    """Fused hash + gather: returns (out [T, H * dim], out_idx [T, H] or None)."""
+    _cuda(ids, "ids", torch.int32)
+    _cuda(table, "table")
+    if table.shape != (params.table_rows, params.dim):
+        raise ValueError("table shape must be (params.table_rows, params.dim)")
+    T, H = ids.numel(), params.heads
+    cu, nseq = _cu_args(cu_seqlens)
+    if out is None:
+        out = torch.empty((T, H * params.dim), dtype=table.dtype, device=table.device)
+    _cuda(out, "out", table.dtype)
+    if out.numel() != T * H * params.dim:
+        raise ValueError("out must hold T * H * dim elements")
+    if out_idx is None and want_idx:
+        out_idx = torch.empty((T, H), dtype=torch.int32, device=ids.device)
+    if out_idx is not None:
+        _cuda(out_idx, "out_idx", torch.int32)
+        if out_idx.numel() != T * H:
+            raise ValueError("out_idx must hold T * H elements")
+    _check(lib.engram_hash_gather(ctypes.byref(params), _ptr(ids), _ptr(cu), nseq, T,
+                                  _ptr(table), _dtype_code(table), _ptr(out_idx), _ptr(out),
+                                  _stream(stream)), "engram_hash_gather")
+    return out, out_idx
+
+
+# ----------------------------------------------------------------- backward
+
+def engram_backward_workspace_size(n: int, table_rows: int, dim: int) -> int:
+    b = ctypes.c_size_t(0)
+    _check(lib.engram_backward_workspace_size(n, table_rows, dim, ctypes.byref(b)),
+           "engram_backward_workspace_size")
+    return b.value
+
+
+def _bwd_buffers(n, dim, device, uniq_rows, row_grads, num_unique, workspace, table_rows):
+    if uniq_rows is None:
+        uniq_rows = torch.empty(max(n, 1), dtype=torch.int32, device=device)
+    if row_grads is None:
+        row_grads = torch.empty((max(n, 1), dim), dtype=torch.float32, device=device)
+    if num_unique is None:
+        num_unique = torch.empty(1, dtype=torch.int32, device=device)
+    if workspace is None:
+        workspace = torch.empty(engram_backward_workspace_size(n, table_rows, dim),
+                                dtype=torch.uint8, device=device)
+    _cuda(uniq_rows, "uniq_rows", torch.int32)
+    _cuda(row_grads, "row_grads", torch.float32)
+    _cuda(num_unique, "num_unique", torch.int32)
+    _cuda(workspace, "workspace", torch.uint8)
+    if uniq_rows.numel() < n or row_grads.numel() < n * dim:
+        raise ValueError("uniq_rows / row_grads must hold n rows")
+    return uniq_rows, row_grads, num_unique, workspace
+
+
+def engram_backward(idx: torch.Tensor, dout: torch.Tensor, table_rows: int, uniq_rows=None,
+                    row_grads=None, num_unique=None, workspace=None, stream=None):
+    """Compact table gradient: (uniq_rows [cap], row_grads [cap, dim] fp32,
+    num_unique [1]); the first num_unique entries are valid."""
+    _cuda(idx, "idx", torch.int32)
+    _cuda(dout, "dout")
+    n = idx.numel()
+    dim = dout.shape[-1]
+    if dout.numel() != n * dim:
+        raise ValueError("dout must be [n, dim] for n = idx.numel()")
+    uniq_rows, row_grads, num_unique, workspace = _bwd_buffers(
+        n, dim, idx.device, uniq_rows, row_grads, num_unique, workspace, table_rows)
+    _check(lib.engram_backward(_ptr(idx), n, table_rows, dim, _ptr(dout), _dtype_code(dout),
+                               _ptr(uniq_rows), _ptr(row_grads), _ptr(num_unique),
+                               _ptr(workspace), workspace.numel(), _stream(stream)),
+           "engram_backward")
+    return uniq_rows, row_grads, num_unique
+
+
+def engram_backward_sort(idx: torch.Tensor, table_rows: int, dim: int, workspace,
+                         stream=None) -> None:
+    _cuda(idx, "idx", torch.int32)
+    _cuda(workspace, "workspace", torch.uint8)
+    _check(lib.engram_backward_sort(_ptr(idx), idx.numel(), table_rows, dim, _ptr(workspace),
+                                    workspace.numel(), _stream(stream)), "engram_backward_sort")
+
+
+def engram_backward_reduce(n: int, table_rows: int, dout: torch.Tensor, uniq_rows, row_grads,
+                           num_unique, workspace, stream=None) -> None:
+    _cuda(dout, "dout")
+    dim = dout.shape[-1]
+    _bwd_buffers(n, dim, dout.device, uniq_rows, row_grads, num_unique, workspace, table_rows)
+    _check(lib.engram_backward_reduce(n, table_rows, dim, _ptr(dout), _dtype_code(dout),
+                                      _ptr(uniq_rows), _ptr(row_grads), _ptr(num_unique),
+                                      _ptr(workspace), workspace.numel(), _stream(stream)),
+           "engram_backward_reduce")
+
+
+# -------------------------------------------------------------------- misc
+
+def engram_get_device_error(stream=None) -> int:
+    """ENGRAM_DEVERR_* bits set since the last call (synchronises the stream)."""
+    v = ctypes.c_uint32(0)
+    _check(lib.engram_get_device_error(ctypes.byref(v), _stream(stream)),
+           "engram_get_device_error")
+    return int(v.value)
+
+
+def engram_launch_count() -> int:
+    return int(lib.engram_launch_count())
+
+
+def engram_abi_version() -> int:
+    return int(lib.engram_abi_version())
+
+
+def engram_host_floor_mod(a: int, m: int) -> int:
+    st = ctypes.c_int(0)
+    r = lib.engram_host_floor_mod(int(a), int(m), ctypes.byref(st))
+    _check(st.value, "engram_host_floor_mod")
+    return int(r)

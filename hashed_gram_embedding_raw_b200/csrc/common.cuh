@@ -1,0 +1,130 @@
+// common.cuh -- helpers shared by the Engram kernels (sm_100a).
+#pragma once
+
+#include <cstdint>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "engram.h"
+
+namespace engram {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+// Per-device error word (ENGRAM_DEVERR_* bits); zero when the module loads.
+// Kernels OR bits into it instead of trapping.
+__device__ unsigned int g_device_error;
+
+__device__ __forceinline__ void raise_device_error(unsigned bits)
+{
+    atomicOr(&g_device_error, bits);
+}
+
+__host__ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
+
+// ------------------------------------------------------------- modular math
+
+__host__ __device__ __forceinline__ uint64_t mulhi64(uint64_t a, uint64_t b)
+{
+#ifdef __CUDA_ARCH__
+    return __umul64hi(a, b);
+#else
+    return (uint64_t)(((unsigned __int128)a * b) >> 64);
+#endif
+}
+
+// Barrett reduction: n mod p for any 64-bit n and 1 <= p < 2^63, where
+// magic = floor((2^64 - 1) / p) >= 2^64 / p - 1. The estimate
+// q = floor(n * magic / 2^64) then satisfies n/p - 1 < n*magic/2^64 <= n/p,
+// so q is floor(n/p) or one less and r = n - q*p lies in [0, 2p): a single
+// conditional subtraction completes the remainder.
+__host__ __device__ __forceinline__ uint64_t barrett_mod(uint64_t n, uint64_t p, uint64_t magic)
+{
+    const uint64_t q = mulhi64(n, magic);
+    const uint64_t r = n - q * p;
+    return r >= p ? r - p : r;
+}
+
+// Remainder of a signed a by p > 0 in [0, p) ("positive remainder").
+// For a < 0 write a = -(u + 1) with u = ~a >= 0; then a mod p = p - 1 - (u mod p).
+__host__ __device__ __forceinline__ int64_t floor_mod(int64_t a, uint64_t p, uint64_t magic)
+{
+    const bool neg = a < 0;
+    const uint64_t u = neg ? ~(uint64_t)a : (uint64_t)a;
+    const uint64_t r = barrett_mod(u, p, magic);
+    return (int64_t)(neg ? p - 1 - r : r);
+}
+
+// --------------------------------------------------------- memory helpers
+
+// 16-byte read-only load that does not allocate in L1 (table rows and
+// gradients are touched once per launch).
+__device__ __forceinline__ uint4 ld_stream(const uint4 *p)
+{
+    uint4 v;
+    asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+        : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+        : "l"(p));
+    return v;
+}
+
+// 16-byte streaming store (evict-first): outputs are written once.
+__device__ __forceinline__ void st_stream(uint4 *p, uint4 v)
+{
+    asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y),
+                 "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+__device__ __forceinline__ void st_stream(float4 *p, float4 v)
+{
+    asm volatile("st.global.cs.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(v.x), "f"(v.y),
+                 "f"(v.z), "f"(v.w)
+                 : "memory");
+}
+
+__device__ __forceinline__ uint32_t lanemask_lt()
+{
+    uint32_t m;
+    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+    return m;
+}
+
+// Exclusive scan of one value per thread over the block (blockDim.x a
+// multiple of 32, at most 1024). s_warp holds 32 words of shared scratch.
+// Every thread gets the block total in *total when total != nullptr.
+__device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t *s_warp,
+                                                         uint32_t *total)
+{
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int nw = blockDim.x >> 5;
+    uint32_t x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(kFull, x, o);
+        if (lane >= o)
+            x += y;
+    }
+    if (lane == 31)
+        s_warp[wid] = x;
+    __syncthreads();
+    if (wid == 0) {
+        uint32_t s = lane < nw ? s_warp[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(kFull, s, o);
+            if (lane >= o)
+                s += y;
+        }
+        if (lane < nw)
+            s_warp[lane] = s;
+    }
+    __syncthreads();
+    const uint32_t before = wid ? s_warp[wid - 1] : 0u;
+    if (total)
+        *total = s_warp[nw - 1];
+    __syncthreads();
+    return before + x - v;
+}
+
+} // namespace engram

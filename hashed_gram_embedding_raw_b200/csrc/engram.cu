@@ -1,0 +1,498 @@
+// engram.cu -- C ABI of the Engram N-gram Embedding library (include/engram.h).
+//
+// Host side: argument checks (ENGRAM_EINVAL before anything is launched),
+// launch planning (grid sized to the resident warps of the current device,
+// work cut into balanced contiguous per-warp ranges), workspace layout of the
+// backward, and the device error word. All arithmetic runs in the kernels of
+// hash_gather.cuh and backward.cuh.
+#include <atomic>
+#include <climits>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <tuple>
+
+#include "engram.h"
+
+#include "backward.cuh"
+#include "common.cuh"
+#include "hash_gather.cuh"
+
+using namespace engram;
+
+namespace {
+
+std::atomic<uint64_t> g_launches{0};
+
+int after_launch()
+{
+    if (cudaGetLastError() != cudaSuccess)
+        return ENGRAM_ECUDA;
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return ENGRAM_OK;
+}
+
+#define ENGRAM_TRY(expr)                                                                   \
+    do {                                                                                   \
+        const int rc_ = (expr);                                                            \
+        if (rc_ != ENGRAM_OK)                                                              \
+            return rc_;                                                                    \
+    } while (0)
+
+int device_sms(int *sms)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return ENGRAM_ECUDA;
+    static std::atomic<int> cache[128];
+    if (dev >= 0 && dev < 128) {
+        const int c = cache[dev].load(std::memory_order_relaxed);
+        if (c > 0) {
+            *sms = c;
+            return ENGRAM_OK;
+        }
+    }
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+        return ENGRAM_ECUDA;
+    if (dev >= 0 && dev < 128)
+        cache[dev].store(v, std::memory_order_relaxed);
+    *sms = v;
+    return ENGRAM_OK;
+}
+
+// Resident warps of `fn` on the current device with the given block shape.
+template <typename F>
+int resident_warps(F fn, int threads, size_t smem, int64_t *warps)
+{
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return ENGRAM_ECUDA;
+    ENGRAM_TRY(device_sms(&sms));
+    static std::mutex mu;
+    static std::map<std::tuple<const void *, int, int, size_t>, int> cache;
+    const auto key = std::make_tuple((const void *)fn, dev, threads, smem);
+    int nb = 0;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        auto it = cache.find(key);
+        if (it != cache.end())
+            nb = it->second;
+    }
+    if (nb == 0) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fn, threads, smem) != cudaSuccess)
+            return ENGRAM_ECUDA;
+        if (nb < 1)
+            nb = 1;
+        std::lock_guard<std::mutex> lock(mu);
+        cache[key] = nb;
+    }
+    *warps = (int64_t)sms * nb * (threads / 32);
+    return ENGRAM_OK;
+}
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+int elem_bytes(int32_t dtype)
+{
+    switch (dtype) {
+    case ENGRAM_F32:
+        return 4;
+    case ENGRAM_BF16:
+    case ENGRAM_F16:
+        return 2;
+    default:
+        return 0;
+    }
+}
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+int make_hash_args(const engram_params_t *p, HashArgs *a)
+{
+    if (p == nullptr)
+        return ENGRAM_EINVAL;
+    const int N = p->ngram_size, K = p->heads_per_ngram;
+    if (N < 2 || N > ENGRAM_MAX_NGRAM || K < 1 || K > ENGRAM_MAX_HEADS ||
+        (N - 1) * K > ENGRAM_MAX_HEADS)
+        return ENGRAM_EINVAL;
+    if (p->table_rows < 1 || p->table_rows > (int64_t(1) << 31) || p->dim < 1)
+        return ENGRAM_EINVAL;
+    std::memset(a, 0, sizeof(*a));
+    a->N = N;
+    a->K = K;
+    a->H = (N - 1) * K;
+    a->eos = p->eos_id;
+    a->fill = p->fill_id;
+    for (int k = 0; k < N; ++k)
+        a->mult[k] = p->multipliers[k];
+    for (int h = 0; h < a->H; ++h) {
+        const int64_t v = p->vocab_sizes[h], o = p->offsets[h];
+        if (v < 1 || o < 0 || o > p->table_rows - v)
+            return ENGRAM_EINVAL;
+        a->p[h] = (uint64_t)v;
+        a->magic[h] = UINT64_MAX / (uint64_t)v;
+        a->off[h] = (int32_t)o;
+    }
+    return ENGRAM_OK;
+}
+
+// ---------------------------------------------------------------- forward
+
+int launch_hash(const HashArgs &a, const int32_t *ids, const int32_t *cu, int32_t nseq,
+                int64_t T, int32_t *out_idx, cudaStream_t stream)
+{
+    const size_t smem = (size_t)(kHashThreads / 32) * 32 * (a.H + 1) * sizeof(int32_t);
+    const bool page_shape = a.N == 3 && a.K == 8;
+    auto fn = page_shape ? hash_kernel<3, 8> : hash_kernel<0, 0>;
+    int64_t res = 0;
+    ENGRAM_TRY(resident_warps(fn, kHashThreads, smem, &res));
+    const int64_t nwarps = std::min<int64_t>(res, ceil_div(T, 32));
+    const int64_t blocks = ceil_div(nwarps, kHashThreads / 32);
+    fn<<<(unsigned)blocks, kHashThreads, smem, stream>>>(a, ids, cu, nseq, T, nwarps, out_idx);
+    return after_launch();
+}
+
+int launch_hash_gather(const HashArgs &a, const int32_t *ids, const int32_t *cu, int32_t nseq,
+                       int64_t T, const void *table, int V, int32_t *out_idx, void *out,
+                       cudaStream_t stream)
+{
+    const size_t smem = (size_t)(kHashThreads / 32) * 32 * (a.H + 1) * sizeof(int32_t);
+    const bool page_shape = a.N == 3 && a.K == 8;
+    auto fn = hash_gather_kernel<0, 0, 0>;
+    if (page_shape && V == 20)
+        fn = hash_gather_kernel<3, 8, 20>;
+    else if (page_shape && V == 40)
+        fn = hash_gather_kernel<3, 8, 40>;
+    int64_t res = 0;
+    ENGRAM_TRY(resident_warps(fn, kHashThreads, smem, &res));
+    const int64_t nwarps = std::min<int64_t>(res, ceil_div(T, 8));
+    const int64_t blocks = ceil_div(nwarps, kHashThreads / 32);
+    fn<<<(unsigned)blocks, kHashThreads, smem, stream>>>(
+        a, ids, cu, nseq, T, nwarps, (const uint4 *)table, V, out_idx, (uint4 *)out);
+    return after_launch();
+}
+
+// --------------------------------------------------------------- backward
+
+struct BwdPlan {
+    int passes = 0, ntiles = 0, W = 0, G = 0;
+    size_t a = 0, b = 0, hist = 0, totals = 0, wcount = 0, wbase = 0, pb = 0, pe = 0,
+           meta = 0, total = 0;
+};
+
+int bwd_plan(int64_t n, int64_t rows, int32_t dim, BwdPlan *P)
+{
+    if (n < 0 || n > INT32_MAX || rows < 1 || rows > (int64_t(1) << 31) || dim < 8 ||
+        dim % 8 != 0 || dim > 512)
+        return ENGRAM_EINVAL;
+    int bits = 0;
+    while ((int64_t(1) << bits) < rows)
+        ++bits;
+    P->passes = std::max(1, (bits + bwd::kRadixBits - 1) / bwd::kRadixBits);
+    P->ntiles = (int)std::max<int64_t>(1, ceil_div(n, bwd::kSortTile));
+    int sms = 0;
+    ENGRAM_TRY(device_sms(&sms));
+    const int64_t wmax = (int64_t)sms * 32;
+    P->W = (int)std::max<int64_t>(1, std::min<int64_t>(wmax, ceil_div(n, 32)));
+    P->G = (dim / 8 + 31) / 32;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = off;
+        off += (bytes + 255) & ~size_t(255);
+        return at;
+    };
+    const size_t nn = (size_t)std::max<int64_t>(n, 1);
+    P->a = take(nn * 8);
+    P->b = take(nn * 8);
+    P->hist = take((size_t)bwd::kRadix * P->ntiles * 4);
+    P->totals = take(bwd::kRadix * 4);
+    P->wcount = take((size_t)P->W * 4);
+    P->wbase = take((size_t)P->W * 4);
+    P->pb = take((size_t)P->W * dim * 8);
+    P->pe = take((size_t)P->W * dim * 8);
+    P->meta = take((size_t)P->W * sizeof(bwd::SegMeta));
+    P->total = off;
+    return ENGRAM_OK;
+}
+
+int check_workspace(const BwdPlan &P, void *ws, size_t ws_bytes)
+{
+    if (ws == nullptr || ((uintptr_t)ws & 255u) != 0)
+        return ENGRAM_EINVAL;
+    if (ws_bytes < P.total)
+        return ENGRAM_ENOSPC;
+    return ENGRAM_OK;
+}
+
+int launch_sort(const int32_t *idx, int64_t n, int64_t rows, const BwdPlan &P, char *ws,
+                cudaStream_t stream)
+{
+    using namespace bwd;
+    auto *A = (unsigned long long *)(ws + P.a);
+    auto *B = (unsigned long long *)(ws + P.b);
+    auto *hist = (uint32_t *)(ws + P.hist);
+    auto *totals = (uint32_t *)(ws + P.totals);
+    const void *src = idx;
+    for (int pass = 0; pass < P.passes; ++pass) {
+        unsigned long long *dst = (pass % 2 == 0) ? A : B;
+        const int shift = pass * kRadixBits;
+        if (pass == 0)
+            radix_upsweep<true><<<P.ntiles, kSortThreads, 0, stream>>>(src, n, shift,
+                                                                         (uint32_t)rows,
+                                                                         hist, P.ntiles);
+        else
+            radix_upsweep<false><<<P.ntiles, kSortThreads, 0, stream>>>(src, n, shift,
+                                                                          (uint32_t)rows,
+                                                                          hist, P.ntiles);
+        ENGRAM_TRY(after_launch());
+        radix_scan<<<kRadix, kSortThreads, 0, stream>>>(hist, P.ntiles, totals);
+        ENGRAM_TRY(after_launch());
+        if (pass == 0)
+            radix_downsweep<true><<<P.ntiles, kSortThreads, 0, stream>>>(src, dst, n, shift,
+                                                                           hist, totals,
+                                                                           P.ntiles);
+        else
+            radix_downsweep<false><<<P.ntiles, kSortThreads, 0, stream>>>(src, dst, n, shift,
+                                                                            hist, totals,
+                                                                            P.ntiles);
+        ENGRAM_TRY(after_launch());
+        src = dst;
+    }
+    return ENGRAM_OK;
+}
+
+template <int DT, int G>
+int launch_seg_reduce(const unsigned long long *items, int64_t n, const BwdPlan &P,
+                      const uint32_t *wbase, const void *dout, int dim, int32_t *uniq,
+                      float *grads, char *ws, cudaStream_t stream)
+{
+    using namespace bwd;
+    const int blocks = (int)ceil_div((int64_t)P.W * 32, kSegThreads);
+    seg_reduce<DT, G><<<blocks, kSegThreads, 0, stream>>>(
+        items, n, P.W, wbase, dout, dim, uniq, grads, (double *)(ws + P.pb),
+        (double *)(ws + P.pe), (SegMeta *)(ws + P.meta));
+    ENGRAM_TRY(after_launch());
+    seg_fixup<G><<<blocks, kSegThreads, 0, stream>>>(P.W, dim, (const double *)(ws + P.pb),
+                                                     (const double *)(ws + P.pe),
+                                                     (const SegMeta *)(ws + P.meta), uniq,
+                                                     grads);
+    return after_launch();
+}
+
+int launch_reduce(int64_t n, int32_t dim, const void *dout, int32_t dtype, int32_t *uniq,
+                  float *grads, int32_t *num_unique, const BwdPlan &P, char *ws,
+                  cudaStream_t stream)
+{
+    using namespace bwd;
+    if (n == 0) {
+        if (cudaMemsetAsync(num_unique, 0, sizeof(int32_t), stream) != cudaSuccess)
+            return ENGRAM_ECUDA;
+        return ENGRAM_OK;
+    }
+    const auto *items = (const unsigned long long *)(ws + ((P.passes % 2 == 1) ? P.a : P.b));
+    auto *wcount = (uint32_t *)(ws + P.wcount);
+    auto *wbase = (uint32_t *)(ws + P.wbase);
+    const int blocks = (int)ceil_div((int64_t)P.W * 32, kSegThreads);
+    seg_count<<<blocks, kSegThreads, 0, stream>>>(items, n, P.W, wcount);
+    ENGRAM_TRY(after_launch());
+    seg_scan<<<1, 1024, 0, stream>>>(wcount, P.W, wbase, num_unique);
+    ENGRAM_TRY(after_launch());
+#define ENGRAM_SEG(DT)                                                                     \
+    return P.G == 1 ? launch_seg_reduce<DT, 1>(items, n, P, wbase, dout, dim, uniq, grads,  \
+                                               ws, stream)                                 \
+                    : launch_seg_reduce<DT, 2>(items, n, P, wbase, dout, dim, uniq, grads,  \
+                                               ws, stream)
+    switch (dtype) {
+    case ENGRAM_F32:
+        ENGRAM_SEG(ENGRAM_F32);
+    case ENGRAM_BF16:
+        ENGRAM_SEG(ENGRAM_BF16);
+    default:
+        ENGRAM_SEG(ENGRAM_F16);
+    }
+#undef ENGRAM_SEG
+}
+
+int check_reduce_args(int64_t n, const void *dout, int32_t dtype, int32_t *uniq, float *grads,
+                      int32_t *num_unique)
+{
+    if (elem_bytes(dtype) == 0 || num_unique == nullptr)
+        return ENGRAM_EINVAL;
+    if (n > 0 && (dout == nullptr || uniq == nullptr || grads == nullptr ||
+                  !aligned16(dout) || !aligned16(grads)))
+        return ENGRAM_EINVAL;
+    return ENGRAM_OK;
+}
+
+} // namespace
+
+// =============================================================== C ABI
+
+extern "C" {
+
+int engram_hash(const engram_params_t *params, const int32_t *ids, const int32_t *cu_seqlens,
+                int32_t nseq, int64_t T, int32_t *out_idx, engram_stream_t stream)
+{
+    HashArgs a;
+    ENGRAM_TRY(make_hash_args(params, &a));
+    if (T < 0 || T > INT32_MAX || (cu_seqlens != nullptr && nseq < 1))
+        return ENGRAM_EINVAL;
+    if (T == 0)
+        return ENGRAM_OK;
+    if (ids == nullptr || out_idx == nullptr)
+        return ENGRAM_EINVAL;
+    return launch_hash(a, ids, cu_seqlens, nseq, T, out_idx, (cudaStream_t)stream);
+}
+
+int engram_gather(const void *table, int32_t dtype, int64_t table_rows, int32_t dim,
+                  const int32_t *idx, int64_t n, void *out, engram_stream_t stream)
+{
+    const int eb = elem_bytes(dtype);
+    if (eb == 0 || dim < 1 || ((int64_t)dim * eb) % 16 != 0 || table_rows < 1 || n < 0)
+        return ENGRAM_EINVAL;
+    if (n == 0)
+        return ENGRAM_OK;
+    if (table == nullptr || idx == nullptr || out == nullptr || !aligned16(table) ||
+        !aligned16(out))
+        return ENGRAM_EINVAL;
+    const int V = (int)((int64_t)dim * eb / 16);
+    auto fn = V == 20 ? gather_kernel<20> : V == 40 ? gather_kernel<40> : gather_kernel<0>;
+    int64_t res = 0;
+    ENGRAM_TRY(resident_warps(fn, kHashThreads, 0, &res));
+    const int64_t nwarps = std::min<int64_t>(res, ceil_div(n, 32));
+    const int64_t blocks = ceil_div(nwarps, kHashThreads / 32);
+    fn<<<(unsigned)blocks, kHashThreads, 0, (cudaStream_t)stream>>>(
+        (const uint4 *)table, table_rows, V, idx, n, nwarps, (uint4 *)out);
+    return after_launch();
+}
+
+int engram_hash_gather(const engram_params_t *params, const int32_t *ids,
+                       const int32_t *cu_seqlens, int32_t nseq, int64_t T, const void *table,
+                       int32_t dtype, int32_t *out_idx, void *out, engram_stream_t stream)
+{
+    HashArgs a;
+    ENGRAM_TRY(make_hash_args(params, &a));
+    const int eb = elem_bytes(dtype);
+    if (eb == 0 || ((int64_t)params->dim * eb) % 16 != 0)
+        return ENGRAM_EINVAL;
+    if (T < 0 || T > INT32_MAX || (cu_seqlens != nullptr && nseq < 1))
+        return ENGRAM_EINVAL;
+    if (T == 0)
+        return ENGRAM_OK;
+    if (ids == nullptr || table == nullptr || out == nullptr || !aligned16(table) ||
+        !aligned16(out))
+        return ENGRAM_EINVAL;
+    const int V = (int)((int64_t)params->dim * eb / 16);
+    return launch_hash_gather(a, ids, cu_seqlens, nseq, T, table, V, out_idx, out,
+                              (cudaStream_t)stream);
+}
+
+int engram_backward_workspace_size(int64_t n, int64_t table_rows, int32_t dim, size_t *bytes)
+{
+    if (bytes == nullptr)
+        return ENGRAM_EINVAL;
+    BwdPlan P;
+    ENGRAM_TRY(bwd_plan(n, table_rows, dim, &P));
+    *bytes = P.total;
+    return ENGRAM_OK;
+}
+
+int engram_backward_sort(const int32_t *idx, int64_t n, int64_t table_rows, int32_t dim,
+                         void *workspace, size_t workspace_bytes, engram_stream_t stream)
+{
+    BwdPlan P;
+    ENGRAM_TRY(bwd_plan(n, table_rows, dim, &P));
+    ENGRAM_TRY(check_workspace(P, workspace, workspace_bytes));
+    if (n == 0)
+        return ENGRAM_OK;
+    if (idx == nullptr)
+        return ENGRAM_EINVAL;
+    return launch_sort(idx, n, table_rows, P, (char *)workspace, (cudaStream_t)stream);
+}
+
+int engram_backward_reduce(int64_t n, int64_t table_rows, int32_t dim, const void *dout,
+                           int32_t dtype, int32_t *uniq_rows, float *row_grads,
+                           int32_t *num_unique, void *workspace, size_t workspace_bytes,
+                           engram_stream_t stream)
+{
+    BwdPlan P;
+    ENGRAM_TRY(bwd_plan(n, table_rows, dim, &P));
+    ENGRAM_TRY(check_workspace(P, workspace, workspace_bytes));
+    ENGRAM_TRY(check_reduce_args(n, dout, dtype, uniq_rows, row_grads, num_unique));
+    return launch_reduce(n, dim, dout, dtype, uniq_rows, row_grads, num_unique, P,
+                         (char *)workspace, (cudaStream_t)stream);
+}
+
+int engram_backward(const int32_t *idx, int64_t n, int64_t table_rows, int32_t dim,
+                    const void *dout, int32_t dtype, int32_t *uniq_rows, float *row_grads,
+                    int32_t *num_unique, void *workspace, size_t workspace_bytes,
+                    engram_stream_t stream)
+{
+    BwdPlan P;
+    ENGRAM_TRY(bwd_plan(n, table_rows, dim, &P));
+    ENGRAM_TRY(check_workspace(P, workspace, workspace_bytes));
+    ENGRAM_TRY(check_reduce_args(n, dout, dtype, uniq_rows, row_grads, num_unique));
+    if (n > 0 && idx == nullptr)
+        return ENGRAM_EINVAL;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (n > 0)
+        ENGRAM_TRY(launch_sort(idx, n, table_rows, P, (char *)workspace, s));
+    return launch_reduce(n, dim, dout, dtype, uniq_rows, row_grads, num_unique, P,
+                         (char *)workspace, s);
+}
+
+int engram_get_device_error(uint32_t *flags, engram_stream_t stream)
+{
+    if (flags == nullptr)
+        return ENGRAM_EINVAL;
+    cudaStream_t s = (cudaStream_t)stream;
+    void *addr = nullptr;
+    unsigned int v = 0;
+    if (cudaGetSymbolAddress(&addr, g_device_error) != cudaSuccess)
+        return ENGRAM_ECUDA;
+    if (cudaMemcpyAsync(&v, addr, sizeof(v), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return ENGRAM_ECUDA;
+    if (cudaMemsetAsync(addr, 0, sizeof(v), s) != cudaSuccess)
+        return ENGRAM_ECUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess)
+        return ENGRAM_ECUDA;
+    *flags = v;
+    return ENGRAM_OK;
+}
+
+const char *engram_status_string(int status)
+{
+    switch (status) {
+    case ENGRAM_OK:
+        return "ENGRAM_OK: success";
+    case ENGRAM_EINVAL:
+        return "ENGRAM_EINVAL: invalid argument (nothing launched)";
+    case ENGRAM_ENOSPC:
+        return "ENGRAM_ENOSPC: workspace too small (nothing launched)";
+    case ENGRAM_ECUDA:
+        return "ENGRAM_ECUDA: CUDA launch or runtime call failed";
+    default:
+        return "unknown engram status";
+    }
+}
+
+int engram_abi_version(void) { return ENGRAM_ABI_VERSION; }
+
+size_t engram_params_size(void) { return sizeof(engram_params_t); }
+
+uint64_t engram_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int64_t engram_host_floor_mod(int64_t a, int64_t m, int *status)
+{
+    if (m < 1 || m > (int64_t)UINT32_MAX) {
+        if (status)
+            *status = ENGRAM_EINVAL;
+        return 0;
+    }
+    if (status)
+        *status = ENGRAM_OK;
+    return floor_mod(a, (uint64_t)m, UINT64_MAX / (uint64_t)m);
+}
+
+} // extern "C"

@@ -1,0 +1,220 @@
+/*
+ * engram.h -- C ABI of the B200 (sm_100a) Engram N-gram Embedding library.
+ *
+ * The operations are those of the Qwen3.8-Flash-Next Engram N-gram Embedding
+ * ("ple" in the checkpoint config), NeMo AutoModel engram API page:
+ *   class Qwen3_8_FlashNextNGramEmbedding      -- hash raw token IDs into the
+ *        packed multi-head table and concatenate the looked-up rows;
+ *   class Qwen3_8_FlashNextOwnerShardedEmbedding -- row lookup on a table held
+ *        by one rank (process_group=None), and the owner-side accumulation of
+ *        each row's gradient in the backward pass.
+ * Here the whole table lives on one GPU; the library never communicates.
+ *
+ * Conventions for every entry point:
+ *   - Pointers named as device pointers must point to device memory of the
+ *     current CUDA device, owned by the caller. The library never allocates;
+ *     scratch space is passed in by the caller (see engram_backward).
+ *   - Calls are asynchronous on `stream` (NULL = the legacy default stream).
+ *     The return code reports host-side argument checks and launch errors
+ *     only; results are ready when the stream reaches the call's end.
+ *   - Return codes: ENGRAM_OK, ENGRAM_EINVAL (argument rejected on the host,
+ *     nothing launched), ENGRAM_ENOSPC (workspace too small, nothing
+ *     launched), ENGRAM_ECUDA (a CUDA launch failed). engram_status_string
+ *     names each one.
+ *   - Faults found on the device (a row index outside the table, malformed
+ *     cu_seqlens) never trap: the kernel skips the offending access, records
+ *     a bit in a per-device error word, and carries on. Read and clear it
+ *     with engram_get_device_error.
+ */
+#ifndef ENGRAM_B200_H
+#define ENGRAM_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define ENGRAM_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define ENGRAM_API __attribute__((visibility("default")))
+#else
+#define ENGRAM_API
+#endif
+
+#define ENGRAM_MAX_NGRAM 4   /* largest supported ngram_size */
+#define ENGRAM_MAX_HEADS 32  /* largest (ngram_size - 1) * heads_per_ngram */
+
+/* return codes */
+#define ENGRAM_OK 0
+#define ENGRAM_EINVAL 1
+#define ENGRAM_ENOSPC 2
+#define ENGRAM_ECUDA 3
+
+/* element types of tables and gradients */
+#define ENGRAM_F32 0
+#define ENGRAM_BF16 1
+#define ENGRAM_F16 2
+
+/* bits of the device error word */
+#define ENGRAM_DEVERR_ROW_RANGE 1u   /* a row index outside [0, table_rows) */
+#define ENGRAM_DEVERR_CU_SEQLENS 2u  /* cu_seqlens not non-decreasing from 0 to T */
+
+/* Same type as cudaStream_t, without requiring the CUDA headers. */
+typedef struct CUstream_st *engram_stream_t;
+
+/*
+ * Hash configuration: the constructor arguments of the page's
+ * Qwen3_8_FlashNextNGramEmbedding (ngram_size, heads_per_ngram,
+ * eos_token_id, layer_multipliers, ngram_heads_vocab_sizes,
+ * ngram_heads_offsets) plus the table shape of
+ * Qwen3_8_FlashNextEngramTableConfig (num_embeddings, embedding_dim).
+ *   H = (ngram_size - 1) * heads_per_ngram heads; head h in group
+ *   g = h / heads_per_ngram hashes the order-(g + 2) n-gram ending at each
+ *   token. Only the first ngram_size multipliers and the first H moduli and
+ *   offsets are read. Requirements (else ENGRAM_EINVAL):
+ *   2 <= ngram_size <= ENGRAM_MAX_NGRAM, heads_per_ngram >= 1,
+ *   H <= ENGRAM_MAX_HEADS, vocab_sizes[h] >= 1, offsets[h] >= 0,
+ *   offsets[h] + vocab_sizes[h] <= table_rows <= 2^31, dim >= 1.
+ *   fill_id is the raw ID read where a token lacks valid earlier context
+ *   (the page's sentence on it is cut off; 0 is the documented default).
+ */
+typedef struct engram_params {
+    int32_t ngram_size;                      /* N, page default 3 */
+    int32_t heads_per_ngram;                 /* K, page default 8 */
+    int64_t multipliers[ENGRAM_MAX_NGRAM];   /* signed int64, [N] */
+    int64_t vocab_sizes[ENGRAM_MAX_HEADS];   /* prime modulus per head, [H] */
+    int64_t offsets[ENGRAM_MAX_HEADS];       /* global row offset per head, [H] */
+    int64_t fill_id;                         /* ID used for missing context */
+    int64_t table_rows;                      /* padded rows R of the table */
+    int32_t dim;                             /* row width D (160) */
+    int32_t eos_id;                          /* raw EOS token ID (248044) */
+} engram_params_t;
+
+/*
+ * engram_hash -- NGramEmbedding._hash_input_ids with _shift_right_after_eos.
+ * For token t of sequence s (cu_seqlens[s] <= t < cu_seqlens[s+1]) let x_k be
+ * the token k places back, or fill_id if that position lies before the
+ * sequence start or an EOS lies at any of positions t-k .. t-1 (context
+ * resets after EOS; an EOS keeps its own left context). The order-n mix is
+ * XOR_{k<n} (x_k * multipliers[k]) in wrapping signed int64 arithmetic and
+ *   out_idx[t, h] = offsets[h] + floor_mod(mix_{g+2}, vocab_sizes[h]).
+ *   ids        device, int32 [T] raw token IDs (any value; negative IDs are
+ *              sign-extended to int64 before the multiply)
+ *   cu_seqlens device, int32 [nseq + 1], cu[0] = 0, non-decreasing, cu[nseq]
+ *              = T; NULL means one sequence [0, T). A [B, S] batch is
+ *              cu = {0, S, 2S, ..., B*S}. Malformed bounds set
+ *              ENGRAM_DEVERR_CU_SEQLENS (memory safety is unaffected).
+ *   T          tokens, 0 <= T < 2^31
+ *   out_idx    device, int32 [T, H] row-major
+ */
+ENGRAM_API int engram_hash(const engram_params_t *params, const int32_t *ids,
+                const int32_t *cu_seqlens, int32_t nseq, int64_t T,
+                int32_t *out_idx, engram_stream_t stream);
+
+/*
+ * engram_gather -- NGramEmbedding._lookup_ngram_ids on a single-rank table:
+ *   out[i, :] = table[idx[i], :] for 0 <= i < n, bit for bit.
+ *   table  device, [table_rows, dim] of dtype, 16-byte aligned
+ *   dtype  ENGRAM_F32 | ENGRAM_BF16 | ENGRAM_F16; dim * sizeof(dtype) must be
+ *          a multiple of 16 bytes
+ *   idx    device, int32 [n]
+ *   out    device, [n, dim] of dtype, 16-byte aligned
+ * An index outside [0, table_rows) writes a zero row and sets
+ * ENGRAM_DEVERR_ROW_RANGE.
+ */
+ENGRAM_API int engram_gather(const void *table, int32_t dtype, int64_t table_rows, int32_t dim,
+                  const int32_t *idx, int64_t n, void *out, engram_stream_t stream);
+
+/*
+ * engram_hash_gather -- NGramEmbedding.forward: hash and lookup fused in one
+ * kernel. out is [T, H, dim] of dtype (= [T, H * dim], heads concatenated in
+ * head order: bigram heads first). out_idx may be NULL; if given it receives
+ * the [T, H] row indices exactly as engram_hash writes them (the backward
+ * needs them). Table requirements as engram_gather, table_rows and dim taken
+ * from params.
+ */
+ENGRAM_API int engram_hash_gather(const engram_params_t *params, const int32_t *ids,
+                       const int32_t *cu_seqlens, int32_t nseq, int64_t T,
+                       const void *table, int32_t dtype, int32_t *out_idx,
+                       void *out, engram_stream_t stream);
+
+/*
+ * engram_backward_workspace_size -- bytes of scratch engram_backward needs for
+ * n lookups into a table of table_rows rows of width dim, on the current
+ * device (the size depends on its SM count).
+ */
+ENGRAM_API int engram_backward_workspace_size(int64_t n, int64_t table_rows, int32_t dim,
+                                   size_t *bytes);
+
+/*
+ * engram_backward -- gradient of the lookup with respect to the table, in
+ * compact form (the owner-side row-gradient accumulation of the page's
+ * OwnerShardedEmbedding; no dense [table_rows, dim] gradient is formed):
+ *   uniq_rows[u]    = the u-th distinct value of idx[0..n), ascending
+ *   row_grads[u, :] = sum over j with idx[j] == uniq_rows[u] of dout[j, :],
+ *                     accumulated in fp64 and rounded once to fp32 (no
+ *                     atomics; deterministic for a given device type)
+ *   *num_unique     = U, the number of distinct rows
+ *   idx        device, int32 [n], 0 <= n < 2^31; out-of-range values set
+ *              ENGRAM_DEVERR_ROW_RANGE (results are then unspecified, memory
+ *              accesses stay in bounds)
+ *   dout       device, [n, dim] of dtype, 16-byte aligned; dim % 8 == 0 and
+ *              dim <= 512
+ *   uniq_rows  device, int32, capacity n
+ *   row_grads  device, fp32 [n, dim] capacity, 16-byte aligned
+ *   num_unique device, int32 scalar
+ *   workspace  device, >= engram_backward_workspace_size bytes, 256-byte
+ *              aligned; contents on entry are ignored
+ * engram_backward = engram_backward_sort followed by engram_backward_reduce
+ * with the same n, table_rows, dim and workspace.
+ */
+ENGRAM_API int engram_backward(const int32_t *idx, int64_t n, int64_t table_rows, int32_t dim,
+                    const void *dout, int32_t dtype, int32_t *uniq_rows,
+                    float *row_grads, int32_t *num_unique, void *workspace,
+                    size_t workspace_bytes, engram_stream_t stream);
+
+/* First stage: stable LSD radix sort of the (idx[j], j) pairs into the workspace. */
+ENGRAM_API int engram_backward_sort(const int32_t *idx, int64_t n, int64_t table_rows, int32_t dim,
+                         void *workspace, size_t workspace_bytes, engram_stream_t stream);
+
+/* Second stage: distinct rows and segmented fp32 sums from the sorted pairs
+ * that engram_backward_sort left in the workspace. */
+ENGRAM_API int engram_backward_reduce(int64_t n, int64_t table_rows, int32_t dim, const void *dout,
+                           int32_t dtype, int32_t *uniq_rows, float *row_grads,
+                           int32_t *num_unique, void *workspace, size_t workspace_bytes,
+                           engram_stream_t stream);
+
+/*
+ * engram_get_device_error -- copy the current device's error word
+ * (ENGRAM_DEVERR_* bits set since the last call) into *flags and clear it.
+ * Synchronises `stream`. Calls on several streams share one word.
+ */
+ENGRAM_API int engram_get_device_error(uint32_t *flags, engram_stream_t stream);
+
+/* Static description of a return code. */
+ENGRAM_API const char *engram_status_string(int status);
+
+/* ENGRAM_ABI_VERSION of the loaded library. */
+ENGRAM_API int engram_abi_version(void);
+
+/* sizeof(engram_params_t) as compiled into the library (binding layout check). */
+ENGRAM_API size_t engram_params_size(void);
+
+/* Number of kernels this library has launched in this process. */
+ENGRAM_API uint64_t engram_launch_count(void);
+
+/*
+ * Host-side check of the device modular reduction: floor_mod(a, m) for
+ * 1 <= m < 2^32, computed on the CPU by the same Barrett routine the kernels
+ * use (result in [0, m); 0 with ENGRAM_EINVAL in *status otherwise).
+ */
+ENGRAM_API int64_t engram_host_floor_mod(int64_t a, int64_t m, int *status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ENGRAM_B200_H */

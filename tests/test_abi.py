@@ -1,0 +1,145 @@
+"""The C-ABI library loads and exports what include/engram.h declares (CPU only).
+
+No kernel runs here: these checks cover symbol export, the parameter layout,
+status strings, host-side argument rejection (which returns before any CUDA
+call), and the Barrett modular reduction the kernels use, run on the host.
+"""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+from tests.conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "engram.h")
+
+
+@pytest.fixture(scope="session")
+def E():
+    import __graft_entry__
+    __graft_entry__._build_module().build()
+    import hashed_gram_embedding_raw_b200 as E
+    return E
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"^ENGRAM_API\s+[\w\s\*]*?\b(engram_\w+)\(", src, re.M)))
+
+
+def test_header_declares_expected_entry_points():
+    names = declared_functions()
+    for must in ("engram_hash", "engram_gather", "engram_hash_gather", "engram_backward",
+                 "engram_backward_workspace_size", "engram_get_device_error"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(E):
+    out = subprocess.check_output(["nm", "-D", "--defined-only", E.LIB_PATH], text=True)
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, missing
+    # and nothing else of ours leaks out of the library
+    assert sorted(n for n in exported if n.startswith("engram")) == declared_functions()
+    assert set(E.EXPORTED) == set(declared_functions())
+
+
+def test_params_layout_and_version(E):
+    assert E.lib.engram_params_size() == ctypes.sizeof(E.EngramParams) == 576
+    assert E.engram_abi_version() == 1
+    for rc in range(4):
+        assert E.status_string(rc).startswith("ENGRAM_")
+    assert "unknown" in E.status_string(99)
+
+
+def test_host_floor_mod_matches_python(E):
+    rng = np.random.Generator(np.random.PCG64(0))
+    mods = [1, 2, 3, 7, 1000003, 20000003, 20000171, 2 ** 31 - 1, 2 ** 32 - 1]
+    vals = [0, 1, -1, 2 ** 63 - 1, -(2 ** 63), -(2 ** 63) + 1, 2 ** 62, -(2 ** 62)]
+    vals += [int(v) for v in rng.integers(-(2 ** 63), 2 ** 63 - 1, size=400, dtype=np.int64)]
+    for m in mods:
+        for a in vals:
+            assert E.engram_host_floor_mod(a, m) == a % m, (a, m)
+        # values next to multiples of m, where a one-off quotient would show
+        for k in (1, 2, 12345, 2 ** 31):
+            for d in (-1, 0, 1):
+                a = k * m + d
+                if a < 2 ** 63:
+                    assert E.engram_host_floor_mod(a, m) == a % m
+                    assert E.engram_host_floor_mod(-a, m) == (-a) % m
+    with pytest.raises(E.EngramError):
+        E.engram_host_floor_mod(5, 0)
+
+
+def _page_params(E):
+    from workloads import head_params
+    return E.make_params(head_params("full"))
+
+
+def test_host_rejects_bad_params(E):
+    L = E.lib
+    bad = []
+    p = _page_params(E)
+    p.ngram_size = 5
+    bad.append(p)
+    p = _page_params(E)
+    p.heads_per_ngram = 0
+    bad.append(p)
+    p = _page_params(E)
+    p.vocab_sizes[3] = 0
+    bad.append(p)
+    p = _page_params(E)
+    p.offsets[15] = p.table_rows - p.vocab_sizes[15] + 1    # slice past the table end
+    bad.append(p)
+    p = _page_params(E)
+    p.table_rows = 2 ** 31 + 1
+    bad.append(p)
+    dummy = ctypes.c_void_p(16)
+    for p in bad:
+        assert L.engram_hash(ctypes.byref(p), dummy, None, 1, 10, dummy, None) == E.ENGRAM_EINVAL
+        assert L.engram_hash_gather(ctypes.byref(p), dummy, None, 1, 10, dummy, 1, None, dummy,
+                                    None) == E.ENGRAM_EINVAL
+    assert L.engram_hash(None, dummy, None, 1, 10, dummy, None) == E.ENGRAM_EINVAL
+    p = _page_params(E)
+    assert L.engram_hash(ctypes.byref(p), dummy, None, 1, -1, dummy, None) == E.ENGRAM_EINVAL
+    assert L.engram_hash(ctypes.byref(p), dummy, dummy, 0, 10, dummy, None) == E.ENGRAM_EINVAL
+    assert L.engram_hash(ctypes.byref(p), None, None, 1, 10, dummy, None) == E.ENGRAM_EINVAL
+    # T = 0 is a no-op
+    assert L.engram_hash(ctypes.byref(p), None, None, 1, 0, None, None) == E.ENGRAM_OK
+
+
+def test_host_rejects_bad_gather_and_backward_args(E):
+    L = E.lib
+    al = ctypes.c_void_p(256)
+    mis = ctypes.c_void_p(264)
+    # row bytes not a multiple of 16, bad dtype, misaligned table or output
+    assert L.engram_gather(al, 1, 100, 12, al, 5, al, None) == E.ENGRAM_EINVAL
+    assert L.engram_gather(al, 7, 100, 160, al, 5, al, None) == E.ENGRAM_EINVAL
+    assert L.engram_gather(mis, 1, 100, 160, al, 5, al, None) == E.ENGRAM_EINVAL
+    assert L.engram_gather(al, 1, 100, 160, al, 5, mis, None) == E.ENGRAM_EINVAL
+    assert L.engram_gather(al, 1, 100, 160, al, 0, al, None) == E.ENGRAM_OK
+    # backward: dim must be a multiple of 8 up to 512; n below 2^31
+    size = ctypes.c_size_t(0)
+    assert L.engram_backward_workspace_size(10, 100, 12, ctypes.byref(size)) == E.ENGRAM_EINVAL
+    assert L.engram_backward_workspace_size(10, 100, 520, ctypes.byref(size)) == E.ENGRAM_EINVAL
+    assert L.engram_backward_workspace_size(2 ** 31, 100, 160,
+                                            ctypes.byref(size)) == E.ENGRAM_EINVAL
+    assert L.engram_backward_workspace_size(10, 0, 160, ctypes.byref(size)) == E.ENGRAM_EINVAL
+    assert L.engram_backward_workspace_size(10, 100, 160, None) == E.ENGRAM_EINVAL
+
+
+def test_package_import_fails_loudly_without_library(tmp_path):
+    # a copy of the binding pointed at a directory with no library must raise
+    import importlib.util
+    src = os.path.join(ROOT, "hashed_gram_embedding_raw_b200", "_binding.py")
+    pkg = tmp_path / "fakepkg"
+    pkg.mkdir()
+    (pkg / "_binding.py").write_text(open(src).read())
+    spec = importlib.util.spec_from_file_location("fake_binding", pkg / "_binding.py")
+    mod = importlib.util.module_from_spec(spec)
+    with pytest.raises(ImportError, match="not found"):
+        spec.loader.exec_module(mod)

@@ -1,0 +1,314 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle, on a B200.
+
+Bar: hash indices and gathered rows bit-exact; row gradients within
+|g - o| <= 1e-6 + 1e-5 |o| per element, distinct rows and their count exact.
+Sizes: small streams spanning several warp ranges with ragged tails and edge
+cases, then every workload at full size. On the 320,001,536-row table the
+oracle cannot hold the table on the host, so gathered rows are compared on a
+sample of tokens (all indices are still compared in full), and the expected
+rows are the input table's rows at the oracle's indices.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests.test_oracle_hash import ADVERSARIAL, small_params
+from workloads import (WORKLOADS, fill_device_table, head_params, host_dout, host_table,
+                       random_stream, token_stream)
+
+pytestmark = pytest.mark.gpu
+
+RTOL, ATOL = 1e-5, 1e-6
+
+
+@pytest.fixture(scope="module")
+def E():
+    import hashed_gram_embedding_raw_b200 as E
+    torch.cuda.set_device(0)
+    E.engram_get_device_error()        # start from a clean error word
+    return E
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def bits16(t: torch.Tensor) -> np.ndarray:
+    return t.contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+def assert_grads_close(got: np.ndarray, want: np.ndarray):
+    err = np.abs(got.astype(np.float64) - want.astype(np.float64))
+    bound = ATOL + RTOL * np.abs(want.astype(np.float64))
+    bad = err > bound
+    assert not bad.any(), f"{bad.sum()} elements out of tolerance, max err {err.max()}"
+
+
+# =================================================================== hash
+
+@pytest.mark.parametrize("case", range(len(ADVERSARIAL)))
+def test_hash_adversarial(E, case):
+    ids, cu = ADVERSARIAL[case]
+    if not ids:
+        return
+    cfg = small_params(seed=case, eos=999, fill=17 if case % 2 else 0)
+    p = E.make_params(cfg)
+    ids = np.array(ids, np.int32)
+    cu_a = None if cu is None else np.array(cu, np.int32)
+    got = E.engram_hash(p, dev(ids), None if cu_a is None else dev(cu_a))
+    want = oracle.hash_ids(ids, cu_a, cfg)
+    np.testing.assert_array_equal(got.cpu().numpy(), want)
+
+
+@pytest.mark.parametrize("N,K", [(3, 8), (2, 3), (4, 2), (3, 1), (2, 32)])
+@pytest.mark.parametrize("T,nseq", [(1, 1), (31, 1), (33, 2), (1000, 7), (20011, 40), (5003, 5003)])
+def test_hash_random_streams(E, N, K, T, nseq):
+    seed = T * 7 + N * 3 + K
+    cfg = small_params(seed=seed % 97, N=N, K=K, eos=13, fill=seed % 3)
+    ids, cu = random_stream(seed, T, [50, 100_000, 2 ** 31 - 1][seed % 3], 13, 0.05, nseq=nseq)
+    ids = ids.copy()
+    ids[::7] = -ids[::7]
+    got = E.engram_hash(E.make_params(cfg), dev(ids), dev(cu))
+    np.testing.assert_array_equal(got.cpu().numpy(), oracle.hash_ids(ids, cu, cfg))
+    got = E.engram_hash(E.make_params(cfg), dev(ids), None)     # one sequence
+    np.testing.assert_array_equal(got.cpu().numpy(), oracle.hash_ids(ids, None, cfg))
+
+
+@pytest.mark.parametrize("name", list(WORKLOADS))
+def test_hash_full_workloads(E, name):
+    cfg = head_params(name)
+    ids, cu = token_stream(name)
+    got = E.engram_hash(E.make_params(cfg), dev(ids), dev(cu)).cpu().numpy()
+    np.testing.assert_array_equal(got, oracle.hash_ids(ids, cu, cfg))
+    assert E.engram_get_device_error() == 0
+
+
+def test_hash_flags_malformed_cu_seqlens(E):
+    cfg = small_params(seed=1)
+    ids, _ = random_stream(1, 100, 1000, 999, 0.0)
+    for cu in ([0, 50, 40, 100], [1, 50, 100], [0, 50, 99]):
+        E.engram_hash(E.make_params(cfg), dev(ids), dev(np.array(cu, np.int32)))
+        assert E.engram_get_device_error() & E.ENGRAM_DEVERR_CU_SEQLENS
+    E.engram_hash(E.make_params(cfg), dev(ids), dev(np.array([0, 50, 100], np.int32)))
+    assert E.engram_get_device_error() == 0
+
+
+# ================================================================= gather
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("dim", [160, 8, 96, 264])
+@pytest.mark.parametrize("n", [1, 33, 4099])
+def test_gather_random(E, dtype, dim, n):
+    if (dim * torch.finfo(dtype).bits // 8) % 16:
+        pytest.skip("row bytes must be a multiple of 16")
+    rng = np.random.Generator(np.random.PCG64(n + dim))
+    rows = 3001
+    table = torch.from_numpy(rng.standard_normal((rows, dim)).astype(np.float32)).to(dtype)
+    idx = rng.integers(0, rows, size=n).astype(np.int32)
+    idx[: min(n, 3)] = [0, rows - 1, 7][: min(n, 3)]
+    got = E.engram_gather(table.cuda(), dev(idx)).cpu()
+    host = table.view(torch.int16 if dtype != torch.float32 else torch.int32).numpy()
+    want = oracle.gather(host, idx)
+    assert got.view(torch.int16 if dtype != torch.float32 else torch.int32).numpy().tobytes() \
+        == want.tobytes()
+
+
+def test_gather_out_of_range_rows(E):
+    table = torch.randn(100, 160, dtype=torch.bfloat16, device="cuda")
+    idx = dev(np.array([5, 100, -1, 99], np.int32))
+    out = E.engram_gather(table, idx)
+    assert E.engram_get_device_error() & E.ENGRAM_DEVERR_ROW_RANGE
+    assert torch.equal(out[0], table[5]) and torch.equal(out[3], table[99])
+    assert not out[1].any() and not out[2].any()
+
+
+# =========================================================== fused forward
+
+def check_forward(E, cfg, ids, cu, table_dev, out, idx, sample=None):
+    """Indices in full; rows on all tokens, or on `sample` token positions."""
+    want_idx = oracle.hash_ids(ids, cu, cfg)
+    np.testing.assert_array_equal(idx.cpu().numpy(), want_idx)
+    toks = np.arange(len(ids)) if sample is None else np.asarray(sample)
+    rows = want_idx[toks].reshape(-1)
+    # expected rows: the input table's rows at the oracle's indices
+    uniq, inv = np.unique(rows, return_inverse=True)
+    compact = table_dev[torch.from_numpy(uniq).cuda()].cpu()
+    if compact.dtype != torch.float32:
+        compact_np = compact.view(torch.int16).numpy()
+        got = out[torch.from_numpy(toks).cuda()].cpu().view(torch.int16).numpy()
+    else:
+        compact_np = compact.numpy()
+        got = out[torch.from_numpy(toks).cuda()].cpu().numpy()
+    want = oracle.gather(compact_np, inv).reshape(len(toks), -1)
+    assert got.tobytes() == want.tobytes()
+
+
+def test_forward_tiny_fp32(E):
+    cfg = head_params("tiny")
+    ids, cu = token_stream("tiny")
+    table = dev(host_table("tiny"))
+    out, idx = E.engram_hash_gather(E.make_params(cfg), dev(ids), table, cu_seqlens=dev(cu))
+    check_forward(E, cfg, ids, cu, table, out, idx)
+
+
+@pytest.mark.parametrize("N,K,dim,dtype", [(3, 8, 160, torch.bfloat16), (3, 8, 160, torch.float16),
+                                           (2, 3, 64, torch.bfloat16), (4, 2, 160, torch.float32),
+                                           (3, 8, 24, torch.float32)])
+@pytest.mark.parametrize("T", [1, 77, 6007])
+def test_forward_shapes(E, N, K, dim, dtype, T):
+    cfg = dict(small_params(seed=T % 11, N=N, K=K, eos=3), dim=dim)
+    ids, cu = random_stream(T, T, 40, 3, 0.1, nseq=1 + T // 500)
+    table = torch.randn(cfg["table_rows"], dim, dtype=torch.float32).to(dtype).cuda()
+    out, idx = E.engram_hash_gather(E.make_params(cfg), dev(ids), table, cu_seqlens=dev(cu))
+    check_forward(E, cfg, ids, cu, table, out, idx)
+    out2, none = E.engram_hash_gather(E.make_params(cfg), dev(ids), table, cu_seqlens=dev(cu),
+                                      want_idx=False)
+    assert none is None and torch.equal(out, out2)
+
+
+@pytest.fixture(scope="module")
+def page_table():
+    """The full 320,001,536 x 160 bf16 table (102.4 GB), filled once."""
+    cfg = head_params("full")
+    t = torch.empty(cfg["table_rows"], cfg["dim"], dtype=torch.bfloat16, device="cuda")
+    fill_device_table(t, WORKLOADS["full"].seed)
+    yield t
+    del t
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("name", ["b4x4096", "thd64k"])
+def test_forward_seeded_tables_full_size(E, name):
+    cfg = head_params(name)
+    ids, cu = token_stream(name)
+    table = torch.empty(cfg["table_rows"], cfg["dim"], dtype=torch.bfloat16, device="cuda")
+    fill_device_table(table, WORKLOADS[name].seed)
+    out, idx = E.engram_hash_gather(E.make_params(cfg), dev(ids), table, cu_seqlens=dev(cu))
+    check_forward(E, cfg, ids, cu, table, out, idx)
+    assert E.engram_get_device_error() == 0
+
+
+@pytest.mark.parametrize("name", ["full", "long256k"])
+def test_forward_page_table_full_size(E, page_table, name):
+    cfg = head_params(name)
+    ids, cu = token_stream(name)
+    out, idx = E.engram_hash_gather(E.make_params(cfg), dev(ids), page_table, cu_seqlens=dev(cu))
+    rng = np.random.Generator(np.random.PCG64(5))
+    T = len(ids)
+    sample = np.unique(np.concatenate([rng.integers(0, T, 4096), [0, 1, T - 1],
+                                       np.nonzero(ids == cfg["eos_id"])[0][:64] + 1]))
+    check_forward(E, cfg, ids, cu, page_table, out, idx, sample=sample[sample < T])
+    assert E.engram_get_device_error() == 0
+
+
+# ================================================================ backward
+
+def check_backward(E, idx_np, dout_t, rows, dtype_code):
+    n = len(idx_np)
+    uniq, grads, nu = E.engram_backward(dev(idx_np.astype(np.int32)), dout_t.cuda(), rows)
+    U = int(nu.item())
+    raw = dout_t.numpy() if dout_t.dtype == torch.float32 else bits16(dout_t)
+    want_u, want_g = oracle.backward(idx_np, raw.reshape(n, -1), dtype_code)
+    assert U == len(want_u)
+    np.testing.assert_array_equal(uniq[:U].cpu().numpy(), want_u)
+    assert_grads_close(grads[:U].cpu().numpy(), want_g)
+    return uniq[:U].clone(), grads[:U].clone()
+
+
+def test_backward_tiny_fp32(E):
+    cfg = head_params("tiny")
+    ids, cu = token_stream("tiny")
+    idx = oracle.hash_ids(ids, cu, cfg).reshape(-1)
+    dout = host_dout("tiny", len(idx), cfg["dim"], "f32")
+    check_backward(E, idx, dout, cfg["table_rows"], oracle.F32)
+
+
+@pytest.mark.parametrize("pattern", ["one_row", "two_rows", "hot_and_cold", "ascending",
+                                     "descending", "max_row"])
+@pytest.mark.parametrize("n", [1, 31, 1000, 250_007])
+def test_backward_patterns(E, pattern, n):
+    rng = np.random.Generator(np.random.PCG64(n))
+    rows = 320_001_536
+    if pattern == "one_row":
+        idx = np.full(n, 12345)
+    elif pattern == "two_rows":
+        idx = np.where(np.arange(n) % 2 == 0, 7, 2 ** 28 + 3)
+    elif pattern == "hot_and_cold":
+        idx = np.where(rng.random(n) < 0.5, rng.integers(0, 3, n), rng.integers(0, rows, n))
+    elif pattern == "ascending":
+        idx = np.arange(n) * 3
+    elif pattern == "descending":
+        idx = (n - np.arange(n)) * 1000
+    else:
+        idx = np.where(rng.random(n) < 0.5, rows - 1, 0)
+    dout = torch.randn(n, 160, generator=torch.Generator().manual_seed(n)).to(torch.bfloat16)
+    check_backward(E, idx.astype(np.int64), dout, rows, oracle.BF16)
+
+
+@pytest.mark.parametrize("dim,dtype", [(8, torch.float32), (264, torch.bfloat16),
+                                       (512, torch.float16), (160, torch.float16),
+                                       (160, torch.float32)])
+def test_backward_dims_dtypes(E, dim, dtype):
+    rng = np.random.Generator(np.random.PCG64(dim))
+    n, rows = 20_000, 5000
+    idx = rng.integers(0, rows, n)
+    dout = torch.randn(n, dim, generator=torch.Generator().manual_seed(dim)).to(dtype)
+    code = {torch.float32: oracle.F32, torch.bfloat16: oracle.BF16, torch.float16: oracle.F16}[dtype]
+    check_backward(E, idx, dout, rows, code)
+
+
+@pytest.mark.parametrize("rows", [1, 2, 255, 256, 257, 65536, 2 ** 24 + 1, 2 ** 31])
+def test_backward_radix_pass_counts(E, rows):
+    rng = np.random.Generator(np.random.PCG64(rows % 1000))
+    n = 9000
+    idx = rng.integers(0, rows, n)
+    dout = torch.randn(n, 16, generator=torch.Generator().manual_seed(1))
+    check_backward(E, idx, dout, rows, oracle.F32)
+
+
+def test_backward_empty(E):
+    uniq, grads, nu = E.engram_backward(torch.empty(0, dtype=torch.int32, device="cuda"),
+                                        torch.empty(0, 160, device="cuda"), 100)
+    assert int(nu.item()) == 0
+
+
+def test_backward_flags_out_of_range(E):
+    idx = dev(np.array([3, 100, 5, -2], np.int32))
+    E.engram_backward(idx, torch.randn(4, 16, device="cuda"), 100)
+    assert E.engram_get_device_error() & E.ENGRAM_DEVERR_ROW_RANGE
+
+
+@pytest.mark.parametrize("name", list(WORKLOADS))
+def test_backward_full_workloads(E, name):
+    cfg = head_params(name)
+    ids, cu = token_stream(name)
+    idx = oracle.hash_ids(ids, cu, cfg).reshape(-1)
+    w = WORKLOADS[name]
+    dout = host_dout(name, len(idx), cfg["dim"], w.dtype)
+    code = oracle.F32 if w.dtype == "f32" else oracle.BF16
+    u1, g1 = check_backward(E, idx, dout, cfg["table_rows"], code)
+    # deterministic: a second run gives the same bits
+    u2, g2, nu = E.engram_backward(dev(idx.astype(np.int32)), dout.cuda(), cfg["table_rows"])
+    U = int(nu.item())
+    assert torch.equal(u1, u2[:U]) and torch.equal(g1, g2[:U])
+    assert E.engram_get_device_error() == 0
+
+
+def test_backward_stages_equal_whole(E):
+    cfg = head_params("b4x4096")
+    ids, cu = token_stream("b4x4096")
+    idx = dev(oracle.hash_ids(ids, cu, cfg).reshape(-1).astype(np.int32))
+    n, D, R = idx.numel(), cfg["dim"], cfg["table_rows"]
+    dout = torch.randn(n, D, device="cuda").to(torch.bfloat16)
+    u1, g1, nu1 = E.engram_backward(idx, dout, R)
+    ws = torch.empty(E.engram_backward_workspace_size(n, R, D), dtype=torch.uint8, device="cuda")
+    u2 = torch.empty(n, dtype=torch.int32, device="cuda")
+    g2 = torch.empty(n, D, device="cuda")
+    nu2 = torch.empty(1, dtype=torch.int32, device="cuda")
+    E.engram_backward_sort(idx, R, D, ws)
+    E.engram_backward_reduce(n, R, dout, u2, g2, nu2, ws)
+    U = int(nu1.item())
+    assert U == int(nu2.item())
+    assert torch.equal(u1[:U], u2[:U]) and torch.equal(g1[:U], g2[:U])
