@@ -1,0 +1,448 @@
+"""Benchmark of the Engram N-gram Embedding hot path on B200.
+
+One step = the fused hash+gather forward (engram_hash_gather, writing the
+[T, 16*160] rows and the [T, 16] indices) followed by the compact backward
+(engram_backward_sort + engram_backward_reduce: distinct rows and fp32 row
+gradients) over one batch of the named workload, all inputs resident in HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload full]
+    python bench.py --impl reference ...   # the CPU oracle, timed on this host
+
+Multi-GPU (torchrun, one rank per GPU): every rank holds its own table
+replica and processes its own batch; no data-path collective exists, so the
+run is weak scaling and the reported value is all ranks' tokens over the
+slowest rank's device time. Prints one JSON line on rank 0.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "Engram tokens/s (fused hash+gather fwd, scatter bwd); achieved HBM GB/s vs peak"
+UNIT = "tokens/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ------------------------------------------------------------------ ranks
+
+def rank_env():
+    """(rank, local_rank, world_size) from the torchrun environment."""
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)),
+            int(os.environ.get("WORLD_SIZE", 1)))
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    """Maximum of a per-rank float over the process group (identity alone)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ------------------------------------------------------------- peaks, clocks
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str, interval_ms: int = 50):
+        self.gpu_id, self.interval_ms, self.proc = gpu_id, interval_ms, None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_id}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", f"-lms={self.interval_ms}"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=10)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def gpu_smi_id(torch, device) -> str:
+    props = torch.cuda.get_device_properties(device)
+    bus = getattr(props, "pci_bus_id", None)
+    if bus is not None:
+        dom = getattr(props, "pci_domain_id", 0)
+        dev = getattr(props, "pci_device_id", 0)
+        return f"{dom:08x}:{bus:02x}:{dev:02x}.0"
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    return vis.split(",")[device.index] if vis else str(device.index)
+
+
+# -------------------------------------------------------- committed traffic
+
+def csrc_digest() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "hashed_gram_embedding_raw_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(kernel: str, units: float):
+    """DRAM bytes per launch from profiles/dram_traffic.json, scaled to `units`
+    (lookups or tokens), or None if absent or taken on other kernel sources."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if rec.get("csrc_digest") != csrc_digest():
+        return None
+    k = rec.get("kernels", {}).get(kernel)
+    if not k:
+        return None
+    return k["dram_bytes_per_unit"] * units
+
+
+# ------------------------------------------------------------ CPU oracle leg
+
+def oracle_run(name: str, S: int, reps_seconds: float = 0.0, max_reps: int = 1):
+    """Time the CPU oracle on the first S tokens of a workload: hash, gather from
+    a host table holding the rows those lookups touch (staged untimed), and the
+    row-gradient backward. Returns (tokens/s, seconds, reps, description)."""
+    import torch
+    import oracle
+    from workloads import WORKLOADS, head_params, host_dout, token_stream
+
+    cfg = head_params(name)
+    ids, cu = token_stream(name)
+    S = min(S, len(ids))
+    ids = np.ascontiguousarray(ids[:S])
+    cu = np.concatenate([cu[cu < S], [S]]).astype(np.int32)
+    H, D = 16, cfg["dim"]
+    w = WORKLOADS[name]
+    # untimed staging: the rows this sample touches, and its output gradient
+    idx0 = oracle.hash_ids(ids, cu, cfg)
+    uniq = np.unique(idx0)
+    rng = np.random.Generator(np.random.PCG64(7))
+    esize = 4 if w.dtype == "f32" else 2
+    compact = rng.integers(0, 2 ** 16, size=(len(uniq), D * esize // 2), dtype=np.uint16)
+    remap = np.searchsorted(uniq, idx0.reshape(-1))
+    dout = host_dout(name, S * H, D, w.dtype)
+    dout_raw = dout.numpy() if w.dtype == "f32" else \
+        dout.view(torch.int16).numpy().view(np.uint16)
+    code = oracle.F32 if w.dtype == "f32" else oracle.BF16
+    oracle.lib()
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        idx = oracle.hash_ids(ids, cu, cfg)
+        out = oracle.gather(compact, remap)
+        u, g = oracle.backward(idx.reshape(-1), dout_raw, code)
+        reps += 1
+        el = time.perf_counter() - t0
+        if reps >= max_reps or el >= reps_seconds:
+            break
+    assert out.shape[0] == S * H and len(u) == len(uniq)
+    desc = (f"first {S} of {len(token_stream(name)[0])} tokens of workload '{name}' "
+            f"x {reps} rep(s); gather from a host table of the {len(uniq)} rows the "
+            f"sample touches (staged before timing); single-threaded C oracle")
+    return S * reps / el, el, reps, desc
+
+
+def run_reference(args):
+    """--impl reference: the oracle, as it stands, on this host's cores."""
+    rank, _, world = rank_env()
+    if rank != 0:
+        return 0
+    name = args.workload
+    # calibrate, then size each step's sample so W + K steps take ~2 minutes
+    rate, _, _, _ = oracle_run(name, 4096)
+    budget = float(os.environ.get("ENGRAM_REFERENCE_BUDGET_S", "120"))
+    S = int(max(256, min(65536 * 4, rate * budget / max(1, args.steps + args.warmup))))
+    for _ in range(args.warmup):
+        oracle_run(name, S)
+    times = []
+    for _ in range(args.steps):
+        _, el, _, desc = oracle_run(name, S)
+        times.append(el)
+    total = sum(times)
+    value = S * len(times) / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / len(times), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int64/f64", "data": "synthetic",
+        "config": {"workload": name, "tokens_per_step": S},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------- GPU leg
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import hashed_gram_embedding_raw_b200 as E
+    from workloads import WORKLOADS, fill_device_table, head_params, host_dout, token_stream
+
+    rank, local_rank, world = rank_env()
+    assert torch.cuda.is_available(), "bench.py needs a CUDA device"
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", device_id=device,
+                                timeout=datetime.timedelta(seconds=300))
+
+    name = args.workload
+    w = WORKLOADS[name]
+    cfg = head_params(name)
+    params = E.make_params(cfg)
+    ids_np, cu_np = token_stream(name)
+    T, H, D, R = len(ids_np), params.heads, cfg["dim"], cfg["table_rows"]
+    n = T * H
+    tdtype = {"bf16": torch.bfloat16, "f32": torch.float32}[w.dtype]
+    esize = 2 if w.dtype == "bf16" else 4
+
+    # inputs resident in HBM
+    table = torch.empty(R, D, dtype=tdtype, device=device)
+    fill_device_table(table, w.seed)
+    ids = torch.from_numpy(ids_np).to(device)
+    cu = torch.from_numpy(cu_np).to(device)
+    dout_h = host_dout(name, n, D, w.dtype).pin_memory()
+    dout = dout_h.to(device)
+    out = torch.empty(T, H * D, dtype=tdtype, device=device)
+    idx = torch.empty(T, H, dtype=torch.int32, device=device)
+    ws = torch.empty(E.engram_backward_workspace_size(n, R, D), dtype=torch.uint8,
+                     device=device)
+    uniq = torch.empty(n, dtype=torch.int32, device=device)
+    grads = torch.empty(n, D, dtype=torch.float32, device=device)
+    nu = torch.empty(1, dtype=torch.int32, device=device)
+    stream = torch.cuda.Stream(device)
+    idx_flat = idx.view(-1)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        E.engram_hash_gather(params, ids, table, cu_seqlens=cu, out=out, out_idx=idx,
+                             stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        E.engram_backward_sort(idx_flat, R, D, ws, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+        E.engram_backward_reduce(n, R, dout, uniq, grads, nu, ws, stream=stream)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    if E.engram_get_device_error(stream):
+        raise RuntimeError("device error flag set during warm-up")
+    U = int(nu.item())
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = E.engram_launch_count()
+    barrier(device)
+    torch.cuda.synchronize(device)
+    with ClockSampler(gpu_smi_id(torch, device)) as clk:
+        t_start.record(stream)
+        for k in range(K):
+            step(evs[k])
+        t_end.record(stream)
+        torch.cuda.synchronize(device)
+    barrier(device)
+    launches = E.engram_launch_count() - launches0
+    local_ms = t_start.elapsed_time(t_end)
+    total_ms = max_over_ranks(local_ms, device)
+    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    sort_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    red_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+
+    # ---- end to end through the public API with host buffers
+    e2e_steps = max(1, min(K, args.e2e_steps))
+    ids_h = torch.from_numpy(ids_np.copy()).pin_memory()
+    cu_h = torch.from_numpy(cu_np.copy()).pin_memory()
+    out_h = torch.empty(T, H * D, dtype=tdtype).pin_memory()
+    uniq_h = torch.empty(n, dtype=torch.int32).pin_memory()
+    grads_h = torch.empty(n, D, dtype=torch.float32).pin_memory()
+    nu_h = torch.empty(1, dtype=torch.int32).pin_memory()
+    h2d = ids_h.numel() * 4 + cu_h.numel() * 4 + dout_h.numel() * esize
+    d2h_bytes = []
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            ids.copy_(ids_h, non_blocking=True)
+            cu.copy_(cu_h, non_blocking=True)
+            dout.copy_(dout_h, non_blocking=True)
+            step()
+            out_h.copy_(out, non_blocking=True)
+            nu_h.copy_(nu, non_blocking=True)
+            stream.synchronize()
+            u = int(nu_h.item())
+            uniq_h[:u].copy_(uniq[:u], non_blocking=True)
+            grads_h[:u].copy_(grads[:u], non_blocking=True)
+            d2h_bytes.append(out_h.numel() * esize + 4 + u * 4 + u * D * 4)
+        e1.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), device)
+    barrier(device)
+
+    if E.engram_get_device_error(stream):
+        raise RuntimeError("device error flag set during timing")
+
+    # ---- numbers
+    value = world * T * K / (total_ms / 1e3)
+    peak, peak_kind = hbm_peak()
+    fwd_bytes = T * (4 + 2 * H * D * esize + H * 4)
+    red_bytes = n * D * esize + U * (4 + D * 4)
+    bwd_bytes = n * 4 + red_bytes
+    stages = {
+        "fwd_hash_gather": {"ms": fwd_ms, "alg_bytes": fwd_bytes,
+                            "gbs": fwd_bytes / fwd_ms / 1e6,
+                            "frac": fwd_bytes / fwd_ms / 1e6 / peak},
+        "bwd_sort": {"ms": sort_ms, "kernels": None},
+        "bwd_reduce": {"ms": red_ms, "alg_bytes": red_bytes,
+                       "gbs": red_bytes / red_ms / 1e6,
+                       "frac": red_bytes / red_ms / 1e6 / peak},
+        "bwd_total": {"ms": sort_ms + red_ms, "alg_bytes": bwd_bytes,
+                      "gbs": bwd_bytes / (sort_ms + red_ms) / 1e6,
+                      "frac": bwd_bytes / (sort_ms + red_ms) / 1e6 / peak},
+        "num_unique": U,
+    }
+    # dominant kernel: the fused forward unless the reduce stage takes longer
+    if fwd_ms >= red_ms:
+        dom, dom_ms, dom_bytes, tkey, tunits = ("hash_gather_kernel", fwd_ms, fwd_bytes,
+                                               "hash_gather_kernel", T)
+    else:
+        dom, dom_ms, dom_bytes, tkey, tunits = ("segment reduce stage (seg_count + seg_scan "
+                                               "+ seg_reduce + seg_fixup)", red_ms,
+                                               red_bytes, "seg_reduce", n)
+    achieved = dom_bytes / dom_ms / 1e6
+    clocks = clk.summary()
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": name, "tokens_per_step_per_gpu": T, "heads": H, "dim": D,
+                   "table_rows": R, "table_dtype": w.dtype, "num_unique": U,
+                   "parallelism": f"replicas x{world} (own table and batch per GPU)",
+                   "l2": "inputs larger than L2 (102.4 GB table; 336 MB out and dout)"
+                   if R > 1e8 else "per-step working set vs 126 MB L2: see table_rows",
+                   "head_constants": "page" if w.heads == "page" else "seeded primes"},
+        "roofline": {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peak,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": committed_traffic(tkey, tunits)},
+        "stages": stages,
+        "e2e": {"value": world * T * e2e_steps / (e2e_ms / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": int(statistics.mean(d2h_bytes)),
+                "steps": e2e_steps},
+        "gpu_launches": launches,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        v, el, reps, desc = oracle_run(name, T, reps_seconds=args.cpu_seconds, max_reps=8)
+        line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
+                                "sample": desc, "seconds": el}
+    else:
+        line["cpu_baseline"] = None
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="full",
+                    choices=["tiny", "b4x4096", "thd64k", "full", "long256k"])
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    args.warmup = max(3, args.warmup)      # at least 3 untimed warm-up steps
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())
