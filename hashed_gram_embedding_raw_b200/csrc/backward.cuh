@@ -8,23 +8,28 @@
 //
 // Stage 1 (sort): the pairs (idx[j], j) are packed as 64-bit items
 // key << 32 | j and sorted by key with a stable least-significant-digit radix
-// sort, 8 bits per pass, ceil(bits(table_rows - 1) / 8) passes. Each pass is
-// reduce-then-scan: per-tile digit counts (upsweep), an exclusive scan of the
-// counts of each digit over tiles (scan), and a stable in-tile ranking with
-// warp match/ballot, staged through shared memory so the scatter writes
-// contiguous runs (downsweep). No block ever waits on another block.
+// sort, 8 bits per pass, ceil(bits(table_rows - 1) / 8) passes, onesweep
+// style: one kernel counts the digits of every pass at once (the counts do not
+// depend on the order), then one kernel per pass ranks a 4096-item tile
+// stably in shared memory and finds the tile's global offsets by decoupled
+// look-back over the tiles before it. Tiles are handed out in launch order by
+// an atomic ticket, so every tile a block waits on belongs to a block that is
+// already running; each wait is bounded and raises ENGRAM_DEVERR_TIMEOUT
+// instead of hanging.
 //
 // Stage 2 (reduce): the sorted items are cut into one contiguous range per
-// warp. A segment is a run of equal keys. Warps count segment heads in their
-// ranges, a single-block scan turns the counts into each range's first
-// segment index, and each warp then sums dout rows along its range in fp64
-// (rounded once to fp32 on output, so hot rows with thousands of terms stay
-// within a few fp32 ulps of the exact sum):
-// segments that start and end inside the range are written directly; the
-// pieces of segments that cross range boundaries are written as partial sums
-// and combined, in range order, by one warp per crossing segment. Hot rows
-// (thousands of lookups of one row) are thereby spread over many warps with
-// no atomics, and the result is deterministic.
+// resident warp. A segment is a run of equal keys. seg_count counts segment
+// heads per range and per block; seg_reduce turns those counts into each
+// range's first segment index, then streams the dout rows of its range through
+// a shared-memory ring filled by cp.async (several rows in flight per warp,
+// independent of registers) and sums each segment in fp64 (rounded once to
+// fp32 on output, so hot rows with thousands of terms stay at fp32-rounding
+// distance from the exact sum). Segments that start and end inside a range are
+// written directly, with each store instruction covering contiguous bytes; the
+// pieces of segments that cross range boundaries are written as fp64 partial
+// sums and combined, in range order, by seg_fixup (one warp per crossing
+// segment). No atomics touch the sums, so the result is deterministic and hot
+// rows spread over many warps.
 #pragma once
 
 #include "common.cuh"
@@ -37,13 +42,76 @@ constexpr int kSortItems = 16;
 constexpr int kSortTile = kSortThreads * kSortItems; // 4096 pairs per tile
 constexpr int kRadixBits = 8;
 constexpr int kRadix = 1 << kRadixBits;
+constexpr int kMaxPasses = 4; // keys below 2^32
 constexpr int kSortWarps = kSortThreads / 32;
 static_assert(kRadix == kSortThreads, "one thread per digit");
 
+// look-back status word: flag in the high half, count in the low half
+constexpr unsigned long long kFlagAggregate = 1ull << 32;
+constexpr unsigned long long kFlagPrefix = 2ull << 32;
+constexpr uint32_t kMaxSpin = 1u << 22; // ~0.1-1 s of polling before giving up
+constexpr int kLookback = 8;            // predecessor tiles read per look-back step
+
 constexpr int kSegThreads = 256;
-constexpr int kSegPrefetch = 8; // dout rows in flight per warp
+constexpr int kSegWarps = kSegThreads / 32;
+constexpr int kSegStages = 3;      // cp.async ring depth per warp
+constexpr int kSegMaxBatch = 8;    // rows per stage
+constexpr int kSegStageBytes = 4096;
 
 __device__ __forceinline__ uint32_t item_key(uint64_t it) { return (uint32_t)(it >> 32); }
+
+// Status words carry the flag and the count in one 64-bit word, so a reader
+// that sees the flag sees the count: relaxed (fence-free) accesses suffice.
+__device__ __forceinline__ void st_status(unsigned long long *p, unsigned long long v)
+{
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ unsigned long long ld_status(const unsigned long long *p)
+{
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// ------------------------------------------------------------------- sort
+
+// Digit counts of every pass over all keys: ghist[pass * 256 + digit].
+__global__ void __launch_bounds__(kSortThreads)
+    radix_histogram(const int32_t *__restrict__ idx, int64_t n, int passes, uint32_t rows,
+                    uint32_t *__restrict__ ghist)
+{
+    __shared__ uint32_t s[kMaxPasses][kRadix];
+    for (int k = threadIdx.x; k < kMaxPasses * kRadix; k += kSortThreads)
+        (&s[0][0])[k] = 0;
+    __syncthreads();
+    bool bad = false;
+    const int64_t stride = (int64_t)gridDim.x * kSortThreads;
+    for (int64_t i0 = (int64_t)blockIdx.x * kSortThreads + threadIdx.x; i0 < n; i0 += 8 * stride) {
+        uint32_t key[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const int64_t i = i0 + q * stride;
+            key[q] = i < n ? (uint32_t)__ldg(idx + i) : 0u;
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            if (i0 + q * stride < n) {
+                bad |= key[q] >= rows;
+                for (int p = 0; p < passes; ++p)
+                    atomicAdd(&s[p][(key[q] >> (p * kRadixBits)) & (kRadix - 1)], 1u);
+            }
+        }
+    }
+    if (bad)
+        raise_device_error(ENGRAM_DEVERR_ROW_RANGE);
+    __syncthreads();
+    for (int k = threadIdx.x; k < passes * kRadix; k += kSortThreads) {
+        const uint32_t c = (&s[0][0])[k];
+        if (c)
+            atomicAdd(ghist + k, c);
+    }
+}
 
 // Pass 0 reads the int32 indices and forms the items; later passes read items.
 template <bool FIRST>
@@ -57,90 +125,31 @@ __device__ __forceinline__ uint64_t load_item(const void *__restrict__ src, int6
     }
 }
 
-// Per-tile digit counts, stored digit-major: hist[d * ntiles + tile].
+// One stable pass: rank a tile by digit, find its global offsets by look-back,
+// scatter through shared memory.
 template <bool FIRST>
 __global__ void __launch_bounds__(kSortThreads)
-    radix_upsweep(const void *__restrict__ src, int64_t n, int shift, uint32_t rows,
-                  uint32_t *__restrict__ hist, int ntiles)
-{
-    __shared__ uint32_t s_cnt[kRadix];
-    s_cnt[threadIdx.x] = 0;
-    __syncthreads();
-    const int lane = threadIdx.x & 31;
-    const int64_t base = (int64_t)blockIdx.x * kSortTile;
-    bool bad = false;
-#pragma unroll 4
-    for (int r = 0; r < kSortItems; ++r) {
-        const int64_t i = base + (int64_t)r * kSortThreads + threadIdx.x;
-        const bool valid = i < n;
-        uint32_t d = kRadix; // sentinel shared by the lanes past the end
-        if (valid) {
-            const uint32_t key = item_key(load_item<FIRST>(src, i));
-            if (FIRST && key >= rows)
-                bad = true;
-            d = (key >> shift) & (kRadix - 1);
-        }
-        const uint32_t peers = __match_any_sync(kFull, d);
-        if (valid && lane == __ffs(peers) - 1)
-            atomicAdd(&s_cnt[d], (uint32_t)__popc(peers));
-    }
-    if (bad)
-        raise_device_error(ENGRAM_DEVERR_ROW_RANGE);
-    __syncthreads();
-    hist[(size_t)threadIdx.x * ntiles + blockIdx.x] = s_cnt[threadIdx.x];
-}
-
-// One block per digit: exclusive scan of that digit's counts over the tiles
-// (in place) and the digit's total.
-__global__ void __launch_bounds__(kSortThreads)
-    radix_scan(uint32_t *__restrict__ hist, int ntiles, uint32_t *__restrict__ totals)
-{
-    __shared__ uint32_t s_warp[32];
-    uint32_t *row = hist + (size_t)blockIdx.x * ntiles;
-    uint32_t carry = 0;
-    for (int t0 = 0; t0 < ntiles; t0 += kSortThreads * 4) {
-        uint32_t v[4], sum = 0;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int t = t0 + threadIdx.x * 4 + q;
-            v[q] = t < ntiles ? row[t] : 0u;
-            sum += v[q];
-        }
-        uint32_t tot;
-        uint32_t run = carry + block_exclusive_scan(sum, s_warp, &tot);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int t = t0 + threadIdx.x * 4 + q;
-            if (t < ntiles)
-                row[t] = run;
-            run += v[q];
-        }
-        carry += tot;
-    }
-    if (threadIdx.x == 0)
-        totals[blockIdx.x] = carry;
-}
-
-// Stable scatter of one tile to its sorted positions.
-template <bool FIRST>
-__global__ void __launch_bounds__(kSortThreads)
-    radix_downsweep(const void *__restrict__ src, unsigned long long *__restrict__ dst,
-                    int64_t n, int shift, const uint32_t *__restrict__ hist,
-                    const uint32_t *__restrict__ totals, int ntiles)
+    radix_pass(const void *__restrict__ src, unsigned long long *__restrict__ dst, int64_t n,
+               int shift, const uint32_t *__restrict__ ghist, unsigned long long *status,
+               uint32_t *ticket)
 {
     __shared__ uint32_t s_whist[kSortWarps][kRadix];
     __shared__ uint32_t s_tstart[kRadix];
     __shared__ uint32_t s_gbase[kRadix];
     __shared__ uint32_t s_warp[32];
     __shared__ unsigned long long s_items[kSortTile];
+    __shared__ int s_tile;
 
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    if (tid == 0)
+        s_tile = (int)atomicAdd(ticket, 1u);
     for (int k = tid; k < kSortWarps * kRadix; k += kSortThreads)
         (&s_whist[0][0])[k] = 0;
     __syncthreads();
+    const int tile = s_tile;
 
     // Each warp ranks its own 32 * kSortItems consecutive items, in order.
-    const int64_t base = (int64_t)blockIdx.x * kSortTile;
+    const int64_t base = (int64_t)tile * kSortTile;
     const int64_t wbase = base + (int64_t)wid * (32 * kSortItems);
     const uint32_t lt = lanemask_lt();
     uint64_t it[kSortItems];
@@ -148,8 +157,12 @@ __global__ void __launch_bounds__(kSortThreads)
 #pragma unroll
     for (int r = 0; r < kSortItems; ++r) {
         const int64_t i = wbase + r * 32 + lane;
+        it[r] = i < n ? load_item<FIRST>(src, i) : 0ull;
+    }
+#pragma unroll
+    for (int r = 0; r < kSortItems; ++r) {
+        const int64_t i = wbase + r * 32 + lane;
         const bool valid = i < n;
-        it[r] = valid ? load_item<FIRST>(src, i) : 0ull;
         const uint32_t d = valid ? (item_key(it[r]) >> shift) & (kRadix - 1) : kRadix;
         const uint32_t peers = __match_any_sync(kFull, d);
         const int leader = __ffs(peers) - 1;
@@ -164,35 +177,83 @@ __global__ void __launch_bounds__(kSortThreads)
     }
     __syncthreads();
 
-    // Thread d: offsets of digit d for every warp (in warp order), the
-    // digit's start inside the tile, and its global base.
+    // Thread d: offsets of digit d per warp (warp order) and in the tile.
+    const int d = tid;
     uint32_t tcount = 0;
 #pragma unroll
     for (int w = 0; w < kSortWarps; ++w) {
-        const uint32_t c = s_whist[w][tid];
-        s_whist[w][tid] = tcount;
+        const uint32_t c = s_whist[w][d];
+        s_whist[w][d] = tcount;
         tcount += c;
     }
-    const uint32_t tstart = block_exclusive_scan(tcount, s_warp, nullptr);
-    const uint32_t dbase = block_exclusive_scan(totals[tid], s_warp, nullptr);
-    s_tstart[tid] = tstart;
-    s_gbase[tid] = dbase + hist[(size_t)tid * ntiles + blockIdx.x] - tstart;
-    __syncthreads();
+    // Publish this tile's count at once so the tiles after it can proceed.
+    unsigned long long *mine = status + (size_t)tile * kRadix + d;
+    st_status(mine, (tile == 0 ? kFlagPrefix : kFlagAggregate) | tcount);
 
+    // Stable order inside the tile, staged in shared memory.
+    const uint32_t tstart = block_exclusive_scan(tcount, s_warp, nullptr);
+    s_tstart[d] = tstart;
+    __syncthreads();
 #pragma unroll
     for (int r = 0; r < kSortItems; ++r) {
         const int64_t i = wbase + r * 32 + lane;
         if (i < n) {
-            const uint32_t d = (item_key(it[r]) >> shift) & (kRadix - 1);
-            s_items[s_tstart[d] + s_whist[wid][d] + rank[r]] = it[r];
+            const uint32_t dd = (item_key(it[r]) >> shift) & (kRadix - 1);
+            s_items[s_tstart[dd] + s_whist[wid][dd] + rank[r]] = it[r];
         }
     }
+
+    // Decoupled look-back: add up the counts of the tiles before this one,
+    // kLookback at a time, back to the nearest one that already carries its
+    // inclusive prefix; then publish this tile's inclusive prefix.
+    uint32_t excl = 0;
+    if (tile > 0) {
+        int t = tile - 1;
+        uint32_t spins = 0;
+        while (t >= 0) {
+            unsigned long long w[kLookback];
+#pragma unroll
+            for (int q = 0; q < kLookback; ++q)
+                w[q] = t - q >= 0 ? ld_status(status + (size_t)(t - q) * kRadix + d)
+                                  : kFlagPrefix;
+            int q = 0; // predecessors consumed in this step
+            bool done = false, found = false;
+#pragma unroll
+            for (int k = 0; k < kLookback; ++k) {
+                if (!done) {
+                    const unsigned long long flag = w[k] & ~0xffffffffull;
+                    if (flag == 0) {
+                        done = true; // not published yet: reload from here
+                    } else {
+                        excl += (uint32_t)w[k];
+                        ++q;
+                        if (flag == kFlagPrefix)
+                            done = found = true;
+                    }
+                }
+            }
+            if (found)
+                break;
+            t -= q;
+            if (q == 0) {
+                if (++spins > kMaxSpin) {
+                    raise_device_error(ENGRAM_DEVERR_TIMEOUT);
+                    break;
+                }
+                __nanosleep(32);
+            }
+        }
+        st_status(mine, kFlagPrefix | (excl + tcount));
+    }
+
+    const uint32_t dbase = block_exclusive_scan(ghist[d], s_warp, nullptr);
+    s_gbase[d] = dbase + excl - tstart;
     __syncthreads();
     const int tile_n = (int)min64(kSortTile, n - base);
     for (int p = tid; p < tile_n; p += kSortThreads) {
         const unsigned long long x = s_items[p];
-        const uint32_t d = (item_key(x) >> shift) & (kRadix - 1);
-        dst[(uint32_t)(s_gbase[d] + (uint32_t)p)] = x;
+        const uint32_t dd = (item_key(x) >> shift) & (kRadix - 1);
+        dst[(uint32_t)(s_gbase[dd] + (uint32_t)p)] = x;
     }
 }
 
@@ -212,236 +273,296 @@ __device__ __forceinline__ void range_of(int64_t n, int64_t w, int64_t W, int64_
     b = n * (w + 1) / W;
 }
 
-// Number of segment heads (first item, or key differs from the previous) per range.
+// Segment heads (first item, or key differs from the previous one) per range
+// (wcount) and per block of kSegWarps ranges (bcount).
 __global__ void __launch_bounds__(kSegThreads)
     seg_count(const unsigned long long *__restrict__ items, int64_t n, int W,
-              uint32_t *__restrict__ wcount)
+              uint32_t *__restrict__ wcount, uint32_t *__restrict__ bcount)
 {
-    const int lane = threadIdx.x & 31;
-    const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    if (w >= W)
-        return;
-    int64_t a, b;
-    range_of(n, w, W, a, b);
+    __shared__ uint32_t s_cnt[kSegWarps];
+    const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+    const int64_t w = (int64_t)blockIdx.x * kSegWarps + wib;
     uint32_t cnt = 0;
-    for (int64_t c0 = a; c0 < b; c0 += 32) {
-        const int64_t i = c0 + lane;
-        const bool live = i < b;
-        const uint32_t key = live ? item_key(__ldg(items + i)) : 0u;
-        const uint32_t prev = (live && i > 0) ? item_key(__ldg(items + i - 1)) : ~key;
-        cnt += __popc(__ballot_sync(kFull, live && key != prev));
+    if (w < W) {
+        int64_t a, b;
+        range_of(n, w, W, a, b);
+        for (int64_t c0 = a; c0 < b; c0 += 128) {
+            uint32_t key[4], prev[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int64_t i = c0 + 32 * q + lane;
+                key[q] = i < b ? item_key(__ldg(items + i)) : 0u;
+                prev[q] = (i < b && i > 0) ? item_key(__ldg(items + i - 1)) : ~key[q];
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int64_t i = c0 + 32 * q + lane;
+                cnt += __popc(__ballot_sync(kFull, i < b && key[q] != prev[q]));
+            }
+        }
+        if (lane == 0)
+            wcount[w] = cnt;
     }
     if (lane == 0)
-        wcount[w] = cnt;
-}
-
-// Exclusive scan of the per-range head counts (one block); total = U.
-__global__ void __launch_bounds__(1024)
-    seg_scan(const uint32_t *__restrict__ wcount, int W, uint32_t *__restrict__ wbase,
-             int32_t *__restrict__ num_unique)
-{
-    __shared__ uint32_t s_warp[32];
-    uint32_t carry = 0;
-    for (int w0 = 0; w0 < W; w0 += 1024) {
-        const int w = w0 + threadIdx.x;
-        const uint32_t v = w < W ? wcount[w] : 0u;
-        uint32_t tot;
-        const uint32_t ex = block_exclusive_scan(v, s_warp, &tot);
-        if (w < W)
-            wbase[w] = carry + ex;
-        carry += tot;
-    }
-    if (threadIdx.x == 0)
-        *num_unique = (int32_t)carry;
-}
-
-// 8 consecutive values of row j, group col (8 * col .. 8 * col + 7), as fp32.
-template <int DT>
-__device__ __forceinline__ void load_group(const void *__restrict__ dout, uint32_t j, int dim,
-                                           int col, uint4 &lo, uint4 &hi)
-{
-    if constexpr (DT == ENGRAM_F32) {
-        const uint4 *p = (const uint4 *)((const float *)dout + (size_t)j * dim) + 2 * col;
-        lo = ld_stream(p);
-        hi = ld_stream(p + 1);
-    } else {
-        const uint4 *p = (const uint4 *)((const uint16_t *)dout + (size_t)j * dim) + col;
-        lo = ld_stream(p);
+        s_cnt[wib] = w < W ? cnt : 0u;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t t = 0;
+        for (int k = 0; k < kSegWarps; ++k)
+            t += s_cnt[k];
+        bcount[blockIdx.x] = t;
     }
 }
 
+// Four consecutive columns (float4 group f) of one staged row, as fp32.
 template <int DT>
-__device__ __forceinline__ void add_group(double (&acc)[8], const uint4 &lo, const uint4 &hi)
+__device__ __forceinline__ float4 load_quad(const unsigned char *row, int f)
 {
     if constexpr (DT == ENGRAM_F32) {
-        acc[0] += (double)__uint_as_float(lo.x);
-        acc[1] += (double)__uint_as_float(lo.y);
-        acc[2] += (double)__uint_as_float(lo.z);
-        acc[3] += (double)__uint_as_float(lo.w);
-        acc[4] += (double)__uint_as_float(hi.x);
-        acc[5] += (double)__uint_as_float(hi.y);
-        acc[6] += (double)__uint_as_float(hi.z);
-        acc[7] += (double)__uint_as_float(hi.w);
+        return *(const float4 *)(row + 16 * f);
     } else if constexpr (DT == ENGRAM_BF16) {
-        const uint32_t w[4] = {lo.x, lo.y, lo.z, lo.w};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            acc[2 * q] += (double)__uint_as_float(w[q] << 16);
-            acc[2 * q + 1] += (double)__uint_as_float(w[q] & 0xffff0000u);
-        }
+        const uint2 v = *(const uint2 *)(row + 8 * f);
+        return make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u),
+                           __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xffff0000u));
     } else {
-        const uint32_t w[4] = {lo.x, lo.y, lo.z, lo.w};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            __half2 h2;
-            memcpy(&h2, &w[q], 4);
-            const float2 f = __half22float2(h2);
-            acc[2 * q] += (double)f.x;
-            acc[2 * q + 1] += (double)f.y;
-        }
+        const uint2 v = *(const uint2 *)(row + 8 * f);
+        __half2 a, b;
+        memcpy(&a, &v.x, 4);
+        memcpy(&b, &v.y, 4);
+        const float2 fa = __half22float2(a), fb = __half22float2(b);
+        return make_float4(fa.x, fa.y, fb.x, fb.y);
     }
 }
 
-// Row gradient: the fp64 sums rounded once to fp32.
-template <int G>
-__device__ __forceinline__ void store_groups(float *__restrict__ dst, const double (&acc)[G][8],
-                                             int lane, int CV)
+// Running sum of one segment on one lane's column groups. A segment of one
+// lookup is its fp32 row, copied exactly; from the second lookup on the sum
+// is kept in fp64 (the first two terms added exactly) and rounded once.
+template <int GF>
+struct SegAcc {
+    float4 first[GF];
+    double acc[GF][4];
+    int cnt; // lookups in the segment, saturating at 2
+
+    __device__ __forceinline__ void add(int g, const float4 &v)
+    {
+        if (cnt == 0) {
+            first[g] = v;
+        } else if (cnt == 1) {
+            acc[g][0] = (double)first[g].x + (double)v.x;
+            acc[g][1] = (double)first[g].y + (double)v.y;
+            acc[g][2] = (double)first[g].z + (double)v.z;
+            acc[g][3] = (double)first[g].w + (double)v.w;
+        } else {
+            acc[g][0] += (double)v.x;
+            acc[g][1] += (double)v.y;
+            acc[g][2] += (double)v.z;
+            acc[g][3] += (double)v.w;
+        }
+    }
+
+    __device__ __forceinline__ float4 rounded(int g) const
+    {
+        if (cnt <= 1)
+            return first[g];
+        return make_float4((float)acc[g][0], (float)acc[g][1], (float)acc[g][2],
+                           (float)acc[g][3]);
+    }
+
+    __device__ __forceinline__ double exact(int g, int q) const
+    {
+        if (cnt <= 1) {
+            const float4 f = first[g];
+            return (double)(q == 0 ? f.x : q == 1 ? f.y : q == 2 ? f.z : f.w);
+        }
+        return acc[g][q];
+    }
+};
+
+// Row gradient: lane owns float4 groups f = lane + 32 g, so each store
+// instruction covers contiguous bytes.
+template <int GF>
+__device__ __forceinline__ void store_row(float *__restrict__ dst, const SegAcc<GF> &s,
+                                          int lane, int F)
 {
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-        const int col = lane + 32 * g;
-        if (col < CV) {
-            float4 *p = (float4 *)(dst + 8 * col);
-            st_stream(p, make_float4((float)acc[g][0], (float)acc[g][1], (float)acc[g][2],
-                                     (float)acc[g][3]));
-            st_stream(p + 1, make_float4((float)acc[g][4], (float)acc[g][5], (float)acc[g][6],
-                                         (float)acc[g][7]));
-        }
+    for (int g = 0; g < GF; ++g) {
+        const int f = lane + 32 * g;
+        if (f < F)
+            st_stream((float4 *)dst + f, s.rounded(g));
     }
 }
 
 // Partial sum of a segment piece, kept in fp64.
-template <int G>
-__device__ __forceinline__ void store_partial(double *__restrict__ dst, const double (&acc)[G][8],
-                                              int lane, int CV)
+template <int GF>
+__device__ __forceinline__ void store_partial(double *__restrict__ dst, const SegAcc<GF> &s,
+                                              int lane, int F)
 {
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-        const int col = lane + 32 * g;
-        if (col < CV) {
-            double2 *p = (double2 *)(dst + 8 * col);
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-                p[k] = make_double2(acc[g][2 * k], acc[g][2 * k + 1]);
+    for (int g = 0; g < GF; ++g) {
+        const int f = lane + 32 * g;
+        if (f < F) {
+            double2 *p = (double2 *)(dst + 4 * f);
+            p[0] = make_double2(s.exact(g, 0), s.exact(g, 1));
+            p[1] = make_double2(s.exact(g, 2), s.exact(g, 3));
         }
     }
 }
 
-// Segmented fp32 sums over one contiguous range of sorted items per warp.
-// G = 8-value column groups per lane (dim <= 256 * G).
-template <int DT, int G>
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem)
+{
+    const uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit()
+{
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+template <int N>
+__device__ __forceinline__ void cp_async_wait()
+{
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Segmented sums over one contiguous range of sorted items per warp.
+// DT: dout dtype; GF: float4 column groups per lane (dim <= 128 * GF);
+// RVT: 16-byte vectors per dout row when fixed at compile time (0: runtime).
+// Dynamic shared memory: kSegWarps * kSegStages * (stage bytes + batch items).
+template <int DT, int GF, int RVT>
 __global__ void __launch_bounds__(kSegThreads)
     seg_reduce(const unsigned long long *__restrict__ items, int64_t n, int W,
-               const uint32_t *__restrict__ wbase, const void *__restrict__ dout, int dim,
-               int32_t *__restrict__ uniq, float *__restrict__ grads, double *__restrict__ pb,
-               double *__restrict__ pe, SegMeta *__restrict__ meta)
+               const uint32_t *__restrict__ wcount, const uint32_t *__restrict__ bcount,
+               const void *__restrict__ dout, int dim, int batch, int stage_bytes,
+               int32_t *__restrict__ uniq, float *__restrict__ grads,
+               double *__restrict__ pb, double *__restrict__ pe, SegMeta *__restrict__ meta,
+               int32_t *__restrict__ num_unique)
 {
-    const int lane = threadIdx.x & 31;
-    const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    extern __shared__ __align__(16) unsigned char smem[];
+    __shared__ uint32_t s_warp[32];
+    const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+    const int64_t w = (int64_t)blockIdx.x * kSegWarps + wib;
+    const int F = dim >> 2; // float4 groups per row
+    const int rvec = RVT ? RVT : dim * (DT == ENGRAM_F32 ? 4 : 2) / 16;
+
+    // First segment index of each range: heads in earlier blocks + earlier warps.
+    uint32_t before = 0;
+    for (int k = threadIdx.x; k < (int)blockIdx.x; k += kSegThreads)
+        before += bcount[k];
+    uint32_t block_before;
+    (void)block_exclusive_scan(before, s_warp, &block_before);
+    uint32_t warp_before = 0;
+    for (int k = 0; k < wib; ++k) {
+        const int64_t wk = (int64_t)blockIdx.x * kSegWarps + k;
+        warp_before += wk < W ? wcount[wk] : 0u;
+    }
+    if (blockIdx.x == gridDim.x - 1 && threadIdx.x == 0)
+        *num_unique = (int32_t)(block_before + bcount[blockIdx.x]);
     if (w >= W)
         return;
+
     int64_t a, b;
     range_of(n, w, W, a, b);
-    const int CV = dim >> 3;
+    const int len = (int)(b - a);
+    const unsigned long long *wit = items + a;
+    const int stage_stride = stage_bytes + kSegMaxBatch * 8;
+    unsigned char *ring = smem + (size_t)wib * kSegStages * stage_stride;
+    const uint4 *drows = (const uint4 *)dout;
 
-    double acc[G][8];
-#pragma unroll
-    for (int g = 0; g < G; ++g)
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-            acc[g][q] = 0.0;
-
-    // If the range opens in the middle of a segment that began earlier, its
-    // first head (if any) closes that piece, which goes to pb.
-    int32_t u = (int32_t)wbase[w] - 1; // index of the open segment
-    uint32_t cur_key = 0;
-    bool open_here = false; // the open segment's head lies in this range
-    int32_t pb_ends = 0;
-
-    for (int64_t c0 = a; c0 < b; c0 += 32) {
-        const int64_t i = c0 + lane;
-        const bool live = i < b;
-        const unsigned long long it = live ? __ldg(items + i) : 0ull;
-        const uint32_t key = item_key(it);
-        const uint32_t j = (uint32_t)it;
-        uint32_t prev = __shfl_up_sync(kFull, key, 1);
-        if (lane == 0)
-            prev = c0 > 0 ? item_key(__ldg(items + c0 - 1)) : ~key;
-        const uint32_t heads = __ballot_sync(kFull, live && key != prev);
-        const int nlive = (int)min64(32, b - c0);
-
-        for (int e0 = 0; e0 < nlive; e0 += kSegPrefetch) {
-            uint4 lo[kSegPrefetch][G], hi[kSegPrefetch][G];
-#pragma unroll
-            for (int q = 0; q < kSegPrefetch; ++q) {
-                const int e = e0 + q;
-                const uint32_t jj = __shfl_sync(kFull, j, e);
-#pragma unroll
-                for (int g = 0; g < G; ++g) {
-                    const int col = lane + 32 * g;
-                    lo[q][g] = hi[q][g] = make_uint4(0, 0, 0, 0);
-                    if (e < nlive && col < CV)
-                        load_group<DT>(dout, jj, dim, col, lo[q][g], hi[q][g]);
-                }
+    // Copies of batch k (range offsets k*batch ...) into stage k % kSegStages.
+    auto issue = [&](int k) {
+        const int e0 = k * batch;
+        if (e0 < len) {
+            unsigned char *stage = ring + (k % kSegStages) * stage_stride;
+            unsigned long long *smeta = (unsigned long long *)(stage + stage_bytes);
+            const int rows = min(batch, len - e0);
+            unsigned long long my = 0;
+            if (lane < rows) {
+                my = __ldg(wit + e0 + lane);
+                smeta[lane] = my;
             }
-#pragma unroll
-            for (int q = 0; q < kSegPrefetch; ++q) {
-                const int e = e0 + q;
-                if (e < nlive) {
-                    if ((heads >> e) & 1u) {
-                        if (c0 + e > a) {
-                            // close the segment that ends just before this head
-                            if (open_here) {
-                                store_groups<G>(grads + (size_t)u * dim, acc, lane, CV);
-                                if (lane == 0)
-                                    uniq[u] = (int32_t)cur_key;
-                            } else {
-                                store_partial<G>(pb + (size_t)w * dim, acc, lane, CV);
-                                pb_ends = 1;
-                            }
-                        }
-                        ++u;
-                        cur_key = __shfl_sync(kFull, key, e);
-                        open_here = true;
-#pragma unroll
-                        for (int g = 0; g < G; ++g)
-#pragma unroll
-                            for (int k = 0; k < 8; ++k)
-                                acc[g][k] = 0.0;
-                    }
-#pragma unroll
-                    for (int g = 0; g < G; ++g)
-                        add_group<DT>(acc[g], lo[q][g], hi[q][g]);
-                }
+            const int nvec = rows * rvec;
+            // uniform trip count across the warp (the shuffle needs every lane)
+            for (int v0 = 0; v0 < nvec; v0 += 32) {
+                const int v = v0 + lane;
+                const int r = min(v / rvec, rows - 1), c = v - r * rvec;
+                const uint32_t j = (uint32_t)__shfl_sync(kFull, my, r);
+                if (v < nvec)
+                    cp_async16(stage + 16 * v, drows + (size_t)j * rvec + c);
             }
         }
+        cp_async_commit();
+    };
+
+    SegAcc<GF> sa;
+    sa.cnt = 0;
+    int32_t u = (int32_t)(block_before + warp_before) - 1; // open segment's index
+    uint32_t cur_key = 0;
+    uint32_t prev_key = a > 0 ? item_key(__ldg(items + a - 1)) : ~item_key(__ldg(items + a));
+    bool open_here = false; // the open segment's head lies in this range
+    bool started = false;   // some lookup of this range has been added
+    int32_t pb_ends = 0;
+
+    const int nb = (len + batch - 1) / batch;
+#pragma unroll
+    for (int k = 0; k < kSegStages; ++k)
+        issue(k);
+    for (int k = 0; k < nb; ++k) {
+        cp_async_wait<kSegStages - 1>();
+        __syncwarp();
+        const unsigned char *stage = ring + (k % kSegStages) * stage_stride;
+        const unsigned long long *smeta = (const unsigned long long *)(stage + stage_bytes);
+        const int rows = min(batch, len - k * batch);
+        for (int r = 0; r < rows; ++r) {
+            const uint32_t key = item_key(smeta[r]);
+            if (key != prev_key) {
+                if (started) {
+                    // close the segment that ends just before this head
+                    if (open_here) {
+                        store_row<GF>(grads + (size_t)u * dim, sa, lane, F);
+                        if (lane == 0)
+                            uniq[u] = (int32_t)cur_key;
+                    } else {
+                        store_partial<GF>(pb + (size_t)w * dim, sa, lane, F);
+                        pb_ends = 1;
+                    }
+                }
+                ++u;
+                cur_key = key;
+                open_here = true;
+                sa.cnt = 0;
+            }
+            prev_key = key;
+            started = true;
+            const unsigned char *row = stage + r * rvec * 16;
+#pragma unroll
+            for (int g = 0; g < GF; ++g) {
+                const int f = lane + 32 * g;
+                if (f < F)
+                    sa.add(g, load_quad<DT>(row, f));
+            }
+            sa.cnt = min(sa.cnt + 1, 2);
+        }
+        __syncwarp();
+        issue(k + kSegStages);
     }
+    cp_async_wait<0>();
 
     // The range's last segment: does it go on past b?
-    const bool cont = b < n && item_key(__ldg(items + b)) == item_key(__ldg(items + b - 1));
+    const bool cont = b < n && item_key(__ldg(items + b)) == prev_key;
     int32_t pe_valid = 0;
     if (open_here) {
         if (cont) {
-            store_partial<G>(pe + (size_t)w * dim, acc, lane, CV);
+            store_partial<GF>(pe + (size_t)w * dim, sa, lane, F);
             pe_valid = 1;
         } else {
-            store_groups<G>(grads + (size_t)u * dim, acc, lane, CV);
+            store_row<GF>(grads + (size_t)u * dim, sa, lane, F);
             if (lane == 0)
                 uniq[u] = (int32_t)cur_key;
         }
     } else {
         // no head in the range: it is one piece of a segment begun earlier
-        store_partial<G>(pb + (size_t)w * dim, acc, lane, CV);
+        store_partial<GF>(pb + (size_t)w * dim, sa, lane, F);
         pb_ends = cont ? 0 : 1;
     }
     if (lane == 0)
@@ -450,7 +571,7 @@ __global__ void __launch_bounds__(kSegThreads)
 
 // One warp per segment that crosses range boundaries: its head piece plus the
 // following ranges' pieces, in range order.
-template <int G>
+template <int GF>
 __global__ void __launch_bounds__(kSegThreads)
     seg_fixup(int W, int dim, const double *__restrict__ pb, const double *__restrict__ pe,
               const SegMeta *__restrict__ meta, int32_t *__restrict__ uniq,
@@ -463,29 +584,36 @@ __global__ void __launch_bounds__(kSegThreads)
     const SegMeta m = meta[w];
     if (!m.pe_valid)
         return;
-    const int CV = dim >> 3;
-    double acc[G][8];
+    const int F = dim >> 2;
+    double acc[GF][4];
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-        const int col = lane + 32 * g;
+    for (int g = 0; g < GF; ++g) {
+        const int f = lane + 32 * g;
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
-            acc[g][k] = col < CV ? pe[(size_t)w * dim + 8 * col + k] : 0.0;
+        for (int q = 0; q < 4; ++q)
+            acc[g][q] = f < F ? pe[(size_t)w * dim + 4 * f + q] : 0.0;
     }
     for (int64_t w2 = w + 1; w2 < W; ++w2) {
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-            const int col = lane + 32 * g;
-            if (col < CV) {
+        for (int g = 0; g < GF; ++g) {
+            const int f = lane + 32 * g;
+            if (f < F) {
 #pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    acc[g][k] += pb[(size_t)w2 * dim + 8 * col + k];
+                for (int q = 0; q < 4; ++q)
+                    acc[g][q] += pb[(size_t)w2 * dim + 4 * f + q];
             }
         }
         if (meta[w2].pb_ends)
             break;
     }
-    store_groups<G>(grads + (size_t)m.pe_u * dim, acc, lane, CV);
+#pragma unroll
+    for (int g = 0; g < GF; ++g) {
+        const int f = lane + 32 * g;
+        if (f < F)
+            st_stream((float4 *)(grads + (size_t)m.pe_u * dim) + f,
+                      make_float4((float)acc[g][0], (float)acc[g][1], (float)acc[g][2],
+                                  (float)acc[g][3]));
+    }
     if (lane == 0)
         uniq[m.pe_u] = m.pe_key;
 }

@@ -176,9 +176,9 @@ int launch_hash_gather(const HashArgs &a, const int32_t *ids, const int32_t *cu,
 // --------------------------------------------------------------- backward
 
 struct BwdPlan {
-    int passes = 0, ntiles = 0, W = 0, G = 0;
-    size_t a = 0, b = 0, hist = 0, totals = 0, wcount = 0, wbase = 0, pb = 0, pe = 0,
-           meta = 0, total = 0;
+    int passes = 0, ntiles = 0, wmax = 0, GF = 0;
+    size_t a = 0, b = 0, ctl = 0, ctl_bytes = 0, status = 0, ghist = 0, tickets = 0;
+    size_t wcount = 0, bcount = 0, pb = 0, pe = 0, meta = 0, total = 0;
 };
 
 int bwd_plan(int64_t n, int64_t rows, int32_t dim, BwdPlan *P)
@@ -193,9 +193,8 @@ int bwd_plan(int64_t n, int64_t rows, int32_t dim, BwdPlan *P)
     P->ntiles = (int)std::max<int64_t>(1, ceil_div(n, bwd::kSortTile));
     int sms = 0;
     ENGRAM_TRY(device_sms(&sms));
-    const int64_t wmax = (int64_t)sms * 32;
-    P->W = (int)std::max<int64_t>(1, std::min<int64_t>(wmax, ceil_div(n, 32)));
-    P->G = (dim / 8 + 31) / 32;
+    P->wmax = sms * 32; // upper bound on resident warps of seg_reduce
+    P->GF = (dim / 4 + 31) / 32;
     size_t off = 0;
     auto take = [&](size_t bytes) {
         const size_t at = off;
@@ -205,13 +204,18 @@ int bwd_plan(int64_t n, int64_t rows, int32_t dim, BwdPlan *P)
     const size_t nn = (size_t)std::max<int64_t>(n, 1);
     P->a = take(nn * 8);
     P->b = take(nn * 8);
-    P->hist = take((size_t)bwd::kRadix * P->ntiles * 4);
-    P->totals = take(bwd::kRadix * 4);
-    P->wcount = take((size_t)P->W * 4);
-    P->wbase = take((size_t)P->W * 4);
-    P->pb = take((size_t)P->W * dim * 8);
-    P->pe = take((size_t)P->W * dim * 8);
-    P->meta = take((size_t)P->W * sizeof(bwd::SegMeta));
+    // sort control block, zeroed once per sort: look-back status words of
+    // every pass, digit counts of every pass, tile tickets of every pass
+    P->ctl = off;
+    P->status = take((size_t)P->passes * P->ntiles * bwd::kRadix * 8);
+    P->ghist = take((size_t)P->passes * bwd::kRadix * 4);
+    P->tickets = take((size_t)P->passes * 4);
+    P->ctl_bytes = off - P->ctl;
+    P->wcount = take((size_t)P->wmax * 4);
+    P->bcount = take((size_t)ceil_div(P->wmax, bwd::kSegWarps) * 4);
+    P->pb = take((size_t)P->wmax * dim * 8);
+    P->pe = take((size_t)P->wmax * dim * 8);
+    P->meta = take((size_t)P->wmax * sizeof(bwd::SegMeta));
     P->total = off;
     return ENGRAM_OK;
 }
@@ -231,87 +235,109 @@ int launch_sort(const int32_t *idx, int64_t n, int64_t rows, const BwdPlan &P, c
     using namespace bwd;
     auto *A = (unsigned long long *)(ws + P.a);
     auto *B = (unsigned long long *)(ws + P.b);
-    auto *hist = (uint32_t *)(ws + P.hist);
-    auto *totals = (uint32_t *)(ws + P.totals);
+    auto *status = (unsigned long long *)(ws + P.status);
+    auto *ghist = (uint32_t *)(ws + P.ghist);
+    auto *tickets = (uint32_t *)(ws + P.tickets);
+    if (cudaMemsetAsync(ws + P.ctl, 0, P.ctl_bytes, stream) != cudaSuccess)
+        return ENGRAM_ECUDA;
+    int sms = 0;
+    ENGRAM_TRY(device_sms(&sms));
+    const int hblocks = (int)std::max<int64_t>(
+        1, std::min<int64_t>((int64_t)sms * 2, ceil_div(n, kSortThreads * 8)));
+    radix_histogram<<<hblocks, kSortThreads, 0, stream>>>(idx, n, P.passes, (uint32_t)rows,
+                                                          ghist);
+    ENGRAM_TRY(after_launch());
     const void *src = idx;
     for (int pass = 0; pass < P.passes; ++pass) {
         unsigned long long *dst = (pass % 2 == 0) ? A : B;
-        const int shift = pass * kRadixBits;
+        unsigned long long *st = status + (size_t)pass * P.ntiles * kRadix;
         if (pass == 0)
-            radix_upsweep<true><<<P.ntiles, kSortThreads, 0, stream>>>(src, n, shift,
-                                                                         (uint32_t)rows,
-                                                                         hist, P.ntiles);
+            radix_pass<true><<<P.ntiles, kSortThreads, 0, stream>>>(
+                src, dst, n, pass * kRadixBits, ghist + pass * kRadix, st, tickets + pass);
         else
-            radix_upsweep<false><<<P.ntiles, kSortThreads, 0, stream>>>(src, n, shift,
-                                                                          (uint32_t)rows,
-                                                                          hist, P.ntiles);
-        ENGRAM_TRY(after_launch());
-        radix_scan<<<kRadix, kSortThreads, 0, stream>>>(hist, P.ntiles, totals);
-        ENGRAM_TRY(after_launch());
-        if (pass == 0)
-            radix_downsweep<true><<<P.ntiles, kSortThreads, 0, stream>>>(src, dst, n, shift,
-                                                                           hist, totals,
-                                                                           P.ntiles);
-        else
-            radix_downsweep<false><<<P.ntiles, kSortThreads, 0, stream>>>(src, dst, n, shift,
-                                                                            hist, totals,
-                                                                            P.ntiles);
+            radix_pass<false><<<P.ntiles, kSortThreads, 0, stream>>>(
+                src, dst, n, pass * kRadixBits, ghist + pass * kRadix, st, tickets + pass);
         ENGRAM_TRY(after_launch());
         src = dst;
     }
     return ENGRAM_OK;
 }
 
-template <int DT, int G>
-int launch_seg_reduce(const unsigned long long *items, int64_t n, const BwdPlan &P,
-                      const uint32_t *wbase, const void *dout, int dim, int32_t *uniq,
-                      float *grads, char *ws, cudaStream_t stream)
+template <int DT, int GF, int RVT>
+int launch_seg(const unsigned long long *items, int64_t n, const BwdPlan &P, const void *dout,
+               int dim, int32_t *uniq, float *grads, int32_t *num_unique, char *ws,
+               cudaStream_t stream)
 {
     using namespace bwd;
-    const int blocks = (int)ceil_div((int64_t)P.W * 32, kSegThreads);
-    seg_reduce<DT, G><<<blocks, kSegThreads, 0, stream>>>(
-        items, n, P.W, wbase, dout, dim, uniq, grads, (double *)(ws + P.pb),
-        (double *)(ws + P.pe), (SegMeta *)(ws + P.meta));
+    const int row_bytes = dim * (DT == ENGRAM_F32 ? 4 : 2);
+    const int batch = std::max(1, std::min(kSegMaxBatch, kSegStageBytes / row_bytes));
+    const int stage_bytes = batch * row_bytes;
+    const size_t smem = (size_t)kSegWarps * kSegStages * (stage_bytes + kSegMaxBatch * 8);
+    auto fn = seg_reduce<DT, GF, RVT>;
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+        return ENGRAM_ECUDA;
+    int64_t res = 0;
+    ENGRAM_TRY(resident_warps(fn, kSegThreads, smem, &res));
+    const int W = (int)std::max<int64_t>(
+        1, std::min<int64_t>(std::min<int64_t>(res, P.wmax), ceil_div(n, 32)));
+    const int blocks = (int)ceil_div(W, kSegWarps);
+    auto *wcount = (uint32_t *)(ws + P.wcount);
+    auto *bcount = (uint32_t *)(ws + P.bcount);
+    auto *pb = (double *)(ws + P.pb);
+    auto *pe = (double *)(ws + P.pe);
+    auto *meta = (SegMeta *)(ws + P.meta);
+    seg_count<<<blocks, kSegThreads, 0, stream>>>(items, n, W, wcount, bcount);
     ENGRAM_TRY(after_launch());
-    seg_fixup<G><<<blocks, kSegThreads, 0, stream>>>(P.W, dim, (const double *)(ws + P.pb),
-                                                     (const double *)(ws + P.pe),
-                                                     (const SegMeta *)(ws + P.meta), uniq,
-                                                     grads);
+    fn<<<blocks, kSegThreads, smem, stream>>>(items, n, W, wcount, bcount, dout, dim, batch,
+                                              stage_bytes, uniq, grads, pb, pe, meta,
+                                              num_unique);
+    ENGRAM_TRY(after_launch());
+    seg_fixup<GF><<<blocks, kSegThreads, 0, stream>>>(W, dim, pb, pe, meta, uniq, grads);
     return after_launch();
+}
+
+template <int DT>
+int launch_seg_dt(const unsigned long long *items, int64_t n, const BwdPlan &P,
+                  const void *dout, int dim, int32_t *uniq, float *grads, int32_t *num_unique,
+                  char *ws, cudaStream_t stream)
+{
+    // the page's 160-wide rows get a compile-time row width
+    constexpr int kRow160 = 160 * (DT == ENGRAM_F32 ? 4 : 2) / 16;
+    if (dim == 160)
+        return launch_seg<DT, 2, kRow160>(items, n, P, dout, dim, uniq, grads, num_unique, ws,
+                                          stream);
+    switch (P.GF) {
+    case 1:
+        return launch_seg<DT, 1, 0>(items, n, P, dout, dim, uniq, grads, num_unique, ws, stream);
+    case 2:
+        return launch_seg<DT, 2, 0>(items, n, P, dout, dim, uniq, grads, num_unique, ws, stream);
+    default:
+        return launch_seg<DT, 4, 0>(items, n, P, dout, dim, uniq, grads, num_unique, ws, stream);
+    }
 }
 
 int launch_reduce(int64_t n, int32_t dim, const void *dout, int32_t dtype, int32_t *uniq,
                   float *grads, int32_t *num_unique, const BwdPlan &P, char *ws,
                   cudaStream_t stream)
 {
-    using namespace bwd;
     if (n == 0) {
         if (cudaMemsetAsync(num_unique, 0, sizeof(int32_t), stream) != cudaSuccess)
             return ENGRAM_ECUDA;
         return ENGRAM_OK;
     }
     const auto *items = (const unsigned long long *)(ws + ((P.passes % 2 == 1) ? P.a : P.b));
-    auto *wcount = (uint32_t *)(ws + P.wcount);
-    auto *wbase = (uint32_t *)(ws + P.wbase);
-    const int blocks = (int)ceil_div((int64_t)P.W * 32, kSegThreads);
-    seg_count<<<blocks, kSegThreads, 0, stream>>>(items, n, P.W, wcount);
-    ENGRAM_TRY(after_launch());
-    seg_scan<<<1, 1024, 0, stream>>>(wcount, P.W, wbase, num_unique);
-    ENGRAM_TRY(after_launch());
-#define ENGRAM_SEG(DT)                                                                     \
-    return P.G == 1 ? launch_seg_reduce<DT, 1>(items, n, P, wbase, dout, dim, uniq, grads,  \
-                                               ws, stream)                                 \
-                    : launch_seg_reduce<DT, 2>(items, n, P, wbase, dout, dim, uniq, grads,  \
-                                               ws, stream)
     switch (dtype) {
     case ENGRAM_F32:
-        ENGRAM_SEG(ENGRAM_F32);
+        return launch_seg_dt<ENGRAM_F32>(items, n, P, dout, dim, uniq, grads, num_unique, ws,
+                                         stream);
     case ENGRAM_BF16:
-        ENGRAM_SEG(ENGRAM_BF16);
+        return launch_seg_dt<ENGRAM_BF16>(items, n, P, dout, dim, uniq, grads, num_unique, ws,
+                                          stream);
     default:
-        ENGRAM_SEG(ENGRAM_F16);
+        return launch_seg_dt<ENGRAM_F16>(items, n, P, dout, dim, uniq, grads, num_unique, ws,
+                                         stream);
     }
-#undef ENGRAM_SEG
 }
 
 int check_reduce_args(int64_t n, const void *dout, int32_t dtype, int32_t *uniq, float *grads,
