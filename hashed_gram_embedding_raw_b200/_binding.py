@@ -30,8 +30,10 @@ EXPORTED = (
     "engram_backward_workspace_size", "engram_backward", "engram_backward_sort",
     "engram_backward_reduce", "engram_get_device_error", "engram_status_string",
     "engram_abi_version", "engram_params_size", "engram_launch_count",
-    "engram_host_floor_mod",
+    "engram_host_floor_mod", "engram_backward_noalloc",
 )
+
+ENGRAM_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 class EngramError(RuntimeError):
@@ -101,6 +103,7 @@ def _load():
         "engram_params_size": [],
         "engram_launch_count": [],
         "engram_host_floor_mod": [i64, i64, ctypes.POINTER(ctypes.c_int)],
+        "engram_backward_noalloc": [P, i64, i64, i32, P, i32, P, P, P, P],
     }
     for name, args in sig.items():
         fn = getattr(L, name)
@@ -266,6 +269,29 @@ def engram_backward(idx: torch.Tensor, dout: torch.Tensor, table_rows: int, uniq
                                _ptr(workspace), workspace.numel(), _stream(stream)),
            "engram_backward")
     return uniq_rows, row_grads, num_unique
+
+
+def engram_backward_noalloc(idx: torch.Tensor, dout: torch.Tensor, table_rows: int,
+                            uniq_rows, row_grads, num_unique, stream=None) -> None:
+    """engram_backward for callers that cannot allocate device memory: the
+    library uses its own fixed device scratch array (ENGRAM_NOALLOC_SCRATCH_BYTES)
+    instead of a workspace, and the caller passes preallocated outputs. Calls
+    that overlap on the GPU share that array and race; serialise them."""
+    _cuda(idx, "idx", torch.int32)
+    _cuda(dout, "dout")
+    n = idx.numel()
+    dim = dout.shape[-1]
+    if dout.numel() != n * dim:
+        raise ValueError("dout must be [n, dim] for n = idx.numel()")
+    _cuda(uniq_rows, "uniq_rows", torch.int32)
+    _cuda(row_grads, "row_grads", torch.float32)
+    _cuda(num_unique, "num_unique", torch.int32)
+    if uniq_rows.numel() < n or row_grads.numel() < n * dim:
+        raise ValueError("uniq_rows / row_grads must hold n rows")
+    _check(lib.engram_backward_noalloc(_ptr(idx), n, table_rows, dim, _ptr(dout),
+                                       _dtype_code(dout), _ptr(uniq_rows), _ptr(row_grads),
+                                       _ptr(num_unique), _stream(stream)),
+           "engram_backward_noalloc")
 
 
 def engram_backward_sort(idx: torch.Tensor, table_rows: int, dim: int, workspace,

@@ -468,6 +468,61 @@ int engram_backward(const int32_t *idx, int64_t n, int64_t table_rows, int32_t d
                          (char *)workspace, s);
 }
 
+} // extern "C"
+
+// ------------------------------------------------- allocation-free backward
+
+namespace {
+
+// Scratch of engram_backward_noalloc: one array per device, loaded with the
+// library and held until the process exits. In host code this name only
+// stands for the array; its device address comes from cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[ENGRAM_NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_noalloc_scratch on the current device, looked up on the
+// first call per device (with that device current) and cached.
+int noalloc_scratch(char **ptr)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128)
+        return ENGRAM_ECUDA;
+    static std::mutex mu;
+    static char *cache[128] = {};
+    std::lock_guard<std::mutex> lock(mu);
+    if (cache[dev] == nullptr) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+            return ENGRAM_ECUDA;
+        cache[dev] = (char *)p;
+    }
+    *ptr = cache[dev];
+    return ENGRAM_OK;
+}
+
+} // namespace
+
+extern "C" {
+
+int engram_backward_noalloc(const int32_t *idx, int64_t n, int64_t table_rows, int32_t dim,
+                            const void *dout, int32_t dtype, int32_t *uniq_rows,
+                            float *row_grads, int32_t *num_unique, engram_stream_t stream)
+{
+    BwdPlan P;
+    ENGRAM_TRY(bwd_plan(n, table_rows, dim, &P));
+    if (P.total > ENGRAM_NOALLOC_SCRATCH_BYTES)
+        return ENGRAM_ENOSPC;
+    ENGRAM_TRY(check_reduce_args(n, dout, dtype, uniq_rows, row_grads, num_unique));
+    if (n > 0 && idx == nullptr)
+        return ENGRAM_EINVAL;
+    char *ws = nullptr;
+    ENGRAM_TRY(noalloc_scratch(&ws));
+    cudaStream_t s = (cudaStream_t)stream;
+    // launch_sort clears the sort's control block in the array on every call
+    if (n > 0)
+        ENGRAM_TRY(launch_sort(idx, n, table_rows, P, ws, s));
+    return launch_reduce(n, dim, dout, dtype, uniq_rows, row_grads, num_unique, P, ws, s);
+}
+
 int engram_get_device_error(uint32_t *flags, engram_stream_t stream)
 {
     if (flags == nullptr)

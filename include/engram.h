@@ -188,6 +188,36 @@ ENGRAM_API int engram_backward_reduce(int64_t n, int64_t table_rows, int32_t dim
                            int32_t *num_unique, void *workspace, size_t workspace_bytes,
                            engram_stream_t stream);
 
+/* Size of the library's own device scratch array used by engram_backward_noalloc. */
+#define ENGRAM_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20) /* 32 MiB per device */
+
+/*
+ * engram_backward_noalloc -- engram_backward for callers that cannot allocate
+ * device memory: a plugin or kernel library inside a host application that
+ * owns all device memory and offers no workspace hook, or a latency-critical
+ * path that must not call cudaMalloc (which may synchronise the device). The
+ * pages describe no such entry point; it is a convenience of this library.
+ *
+ * Same arguments and results as engram_backward, without the workspace: the
+ * scratch lives in one file-scope device array of ENGRAM_NOALLOC_SCRATCH_BYTES
+ * inside the library. Every GPU that loads the library holds that array until
+ * the process exits. The call allocates nothing (no cudaMalloc, no cudaFree).
+ *   - Sizes whose workspace (engram_backward_workspace_size) exceeds
+ *     ENGRAM_NOALLOC_SCRATCH_BYTES are rejected with ENGRAM_ENOSPC before
+ *     anything is launched.
+ *   - The first call on a device looks up the array's device address on that
+ *     device (cudaGetSymbolAddress); make that first call before any stream
+ *     capture on the device.
+ *   - All calls on a device share the one array and it keeps the last call's
+ *     contents (each call clears what must start at zero). Calls that overlap
+ *     on the GPU -- on different streams, or from several host threads --
+ *     race on it; serialise them, e.g. on one stream.
+ */
+ENGRAM_API int engram_backward_noalloc(const int32_t *idx, int64_t n, int64_t table_rows,
+                                       int32_t dim, const void *dout, int32_t dtype,
+                                       int32_t *uniq_rows, float *row_grads,
+                                       int32_t *num_unique, engram_stream_t stream);
+
 /*
  * engram_get_device_error -- copy the current device's error word
  * (ENGRAM_DEVERR_* bits set since the last call) into *flags and clear it.
