@@ -270,36 +270,48 @@ def run_ours(args):
     tdtype = {"bf16": torch.bfloat16, "f32": torch.float32}[w.dtype]
     esize = 2 if w.dtype == "bf16" else 4
 
-    # inputs resident in HBM
-    table = torch.empty(R, D, dtype=tdtype, device=device)
-    fill_device_table(table, w.seed)
-    ids = torch.from_numpy(ids_np).to(device)
-    cu = torch.from_numpy(cu_np).to(device)
+    # inputs resident in HBM; two sets of per-step buffers for the e2e pipeline
+    fwd = args.stage == "all"
+    table = None
+    if fwd:
+        table = torch.empty(R, D, dtype=tdtype, device=device)
+        fill_device_table(table, w.seed)
     dout_h = host_dout(name, n, D, w.dtype).pin_memory()
-    dout = dout_h.to(device)
-    out = torch.empty(T, H * D, dtype=tdtype, device=device)
-    idx = torch.empty(T, H, dtype=torch.int32, device=device)
     ws = torch.empty(E.engram_backward_workspace_size(n, R, D), dtype=torch.uint8,
                      device=device)
-    uniq = torch.empty(n, dtype=torch.int32, device=device)
-    grads = torch.empty(n, D, dtype=torch.float32, device=device)
-    nu = torch.empty(1, dtype=torch.int32, device=device)
+    nbuf = 2 if fwd else 1
+    bufs = [{
+        "ids": torch.from_numpy(ids_np.copy()).to(device),
+        "cu": torch.from_numpy(cu_np.copy()).to(device),
+        "dout": dout_h.to(device),
+        "out": torch.empty(T, H * D, dtype=tdtype, device=device) if fwd else None,
+        "idx": torch.empty(T, H, dtype=torch.int32, device=device),
+        "uniq": torch.empty(n, dtype=torch.int32, device=device),
+        "grads": torch.empty(n, D, dtype=torch.float32, device=device),
+        "nu": torch.empty(1, dtype=torch.int32, device=device),
+    } for _ in range(nbuf)]
     stream = torch.cuda.Stream(device)
-    idx_flat = idx.view(-1)
+    if not fwd:  # backward alone: the indices come from the hash, no table needed
+        E.engram_hash(params, bufs[0]["ids"], bufs[0]["cu"], out_idx=bufs[0]["idx"],
+                      stream=stream)
 
-    def step(ev=None):
+    def step(ev=None, b=None):
+        b = bufs[0] if b is None else b
         if ev is not None:
             ev[0].record(stream)
-        E.engram_hash_gather(params, ids, table, cu_seqlens=cu, out=out, out_idx=idx,
-                             stream=stream)
+        if fwd:
+            E.engram_hash_gather(params, b["ids"], table, cu_seqlens=b["cu"], out=b["out"],
+                                 out_idx=b["idx"], stream=stream)
         if ev is not None:
             ev[1].record(stream)
-        E.engram_backward_sort(idx_flat, R, D, ws, stream=stream)
+        E.engram_backward_sort(b["idx"].view(-1), R, D, ws, stream=stream)
         if ev is not None:
             ev[2].record(stream)
-        E.engram_backward_reduce(n, R, dout, uniq, grads, nu, ws, stream=stream)
+        E.engram_backward_reduce(n, R, b["dout"], b["uniq"], b["grads"], b["nu"], ws,
+                                 stream=stream)
         if ev is not None:
             ev[3].record(stream)
+    nu = bufs[0]["nu"]
 
     for _ in range(args.warmup):
         step()
@@ -328,37 +340,75 @@ def run_ours(args):
     sort_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     red_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
 
-    # ---- end to end through the public API with host buffers
-    e2e_steps = max(1, min(K, args.e2e_steps))
-    ids_h = torch.from_numpy(ids_np.copy()).pin_memory()
-    cu_h = torch.from_numpy(cu_np.copy()).pin_memory()
-    out_h = torch.empty(T, H * D, dtype=tdtype).pin_memory()
-    uniq_h = torch.empty(n, dtype=torch.int32).pin_memory()
-    grads_h = torch.empty(n, D, dtype=torch.float32).pin_memory()
-    nu_h = torch.empty(1, dtype=torch.int32).pin_memory()
-    h2d = ids_h.numel() * 4 + cu_h.numel() * 4 + dout_h.numel() * esize
-    d2h_bytes = []
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(device)
-    torch.cuda.synchronize(device)
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        for _ in range(e2e_steps):
-            ids.copy_(ids_h, non_blocking=True)
-            cu.copy_(cu_h, non_blocking=True)
-            dout.copy_(dout_h, non_blocking=True)
-            step()
-            out_h.copy_(out, non_blocking=True)
-            nu_h.copy_(nu, non_blocking=True)
-            stream.synchronize()
-            u = int(nu_h.item())
-            uniq_h[:u].copy_(uniq[:u], non_blocking=True)
-            grads_h[:u].copy_(grads[:u], non_blocking=True)
-            d2h_bytes.append(out_h.numel() * esize + 4 + u * 4 + u * D * 4)
-        e1.record(stream)
-    torch.cuda.synchronize(device)
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), device)
-    barrier(device)
+    # ---- end to end through the public API with host buffers: every step
+    # copies its inputs in from pinned host memory and its results out. Three
+    # streams pipeline consecutive steps (copy-in, compute, copy-out, with two
+    # sets of device buffers), so step k's results travel to the host while
+    # step k+1 computes and PCIe carries both directions at once.
+    e2e = None
+    if fwd:
+        e2e_steps = max(1, min(K, args.e2e_steps))
+        ids_h = torch.from_numpy(ids_np.copy()).pin_memory()
+        cu_h = torch.from_numpy(cu_np.copy()).pin_memory()
+        host = [{"out": torch.empty(T, H * D, dtype=tdtype).pin_memory(),
+                 "uniq": torch.empty(n, dtype=torch.int32).pin_memory(),
+                 "grads": torch.empty(n, D, dtype=torch.float32).pin_memory(),
+                 "nu": torch.empty(1, dtype=torch.int32).pin_memory()} for _ in range(2)]
+        s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
+        ev = lambda: torch.cuda.Event()  # noqa: E731
+        in_done = [ev() for _ in range(e2e_steps)]
+        comp_done = [ev() for _ in range(e2e_steps)]
+        nu_done = [ev() for _ in range(e2e_steps)]
+        out_done = [ev() for _ in range(e2e_steps)]
+        h2d = ids_h.numel() * 4 + cu_h.numel() * 4 + dout_h.numel() * esize
+        d2h_bytes = [0] * e2e_steps
+
+        def drain(k):
+            # rows of step k: the host needs num_unique before copying them out
+            nu_done[k].synchronize()
+            hb, b = host[k % 2], bufs[k % 2]
+            u = int(hb["nu"].item())
+            with torch.cuda.stream(s_out):
+                hb["uniq"][:u].copy_(b["uniq"][:u], non_blocking=True)
+                hb["grads"][:u].copy_(b["grads"][:u], non_blocking=True)
+                out_done[k].record(s_out)
+            d2h_bytes[k] = hb["out"].numel() * esize + 4 + u * 4 + u * D * 4
+
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(device)
+        torch.cuda.synchronize(device)
+        e0.record(s_in)
+        for k in range(e2e_steps):
+            b, hb = bufs[k % 2], host[k % 2]
+            with torch.cuda.stream(s_in):
+                if k >= 2:
+                    s_in.wait_event(comp_done[k - 2])  # inputs of buffer set k%2 free
+                b["ids"].copy_(ids_h, non_blocking=True)
+                b["cu"].copy_(cu_h, non_blocking=True)
+                b["dout"].copy_(dout_h, non_blocking=True)
+                in_done[k].record(s_in)
+            stream.wait_event(in_done[k])
+            if k >= 2:
+                stream.wait_event(out_done[k - 2])     # outputs of buffer set k%2 copied out
+            step(b=b)
+            comp_done[k].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(comp_done[k])
+                hb["out"].copy_(b["out"], non_blocking=True)
+                hb["nu"].copy_(b["nu"], non_blocking=True)
+                nu_done[k].record(s_out)
+            if k >= 1:
+                drain(k - 1)
+        drain(e2e_steps - 1)
+        e1.record(s_out)
+        torch.cuda.synchronize(device)
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), device)
+        barrier(device)
+        e2e = {"value": world * T * e2e_steps / (e2e_ms / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": int(statistics.mean(d2h_bytes)),
+               "steps": e2e_steps,
+               "pipeline": "copy-in / compute / copy-out streams, two buffer sets"}
 
     if E.engram_get_device_error(stream):
         raise RuntimeError("device error flag set during timing")
@@ -371,8 +421,8 @@ def run_ours(args):
     bwd_bytes = n * 4 + red_bytes
     stages = {
         "fwd_hash_gather": {"ms": fwd_ms, "alg_bytes": fwd_bytes,
-                            "gbs": fwd_bytes / fwd_ms / 1e6,
-                            "frac": fwd_bytes / fwd_ms / 1e6 / peak},
+                            "gbs": fwd_bytes / max(fwd_ms, 1e-9) / 1e6,
+                            "frac": fwd_bytes / max(fwd_ms, 1e-9) / 1e6 / peak},
         "bwd_sort": {"ms": sort_ms, "kernels": None},
         "bwd_reduce": {"ms": red_ms, "alg_bytes": red_bytes,
                        "gbs": red_bytes / red_ms / 1e6,
@@ -383,20 +433,23 @@ def run_ours(args):
         "num_unique": U,
     }
     # dominant kernel: the fused forward unless the reduce stage takes longer
-    if fwd_ms >= red_ms:
+    if fwd and fwd_ms >= red_ms:
         dom, dom_ms, dom_bytes, tkey, tunits = ("hash_gather_kernel", fwd_ms, fwd_bytes,
                                                "hash_gather_kernel", T)
     else:
-        dom, dom_ms, dom_bytes, tkey, tunits = ("segment reduce stage (seg_count + seg_scan "
-                                               "+ seg_reduce + seg_fixup)", red_ms,
+        dom, dom_ms, dom_bytes, tkey, tunits = ("segment reduce stage (seg_count + seg_reduce "
+                                               "+ seg_fixup; seg_reduce dominates)", red_ms,
                                                red_bytes, "seg_reduce", n)
+    if not fwd:
+        stages.pop("fwd_hash_gather")
     achieved = dom_bytes / dom_ms / 1e6
     clocks = clk.summary()
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-        "config": {"workload": name, "tokens_per_step_per_gpu": T, "heads": H, "dim": D,
+        "config": {"workload": name, "stage": "forward + backward" if fwd else "backward only",
+                   "tokens_per_step_per_gpu": T, "heads": H, "dim": D,
                    "table_rows": R, "table_dtype": w.dtype, "num_unique": U,
                    "parallelism": f"replicas x{world} (own table and batch per GPU)",
                    "l2": "inputs larger than L2 (102.4 GB table; 336 MB out and dout)"
@@ -406,14 +459,11 @@ def run_ours(args):
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": committed_traffic(tkey, tunits)},
         "stages": stages,
-        "e2e": {"value": world * T * e2e_steps / (e2e_ms / 1e3), "unit": UNIT,
-                "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": int(statistics.mean(d2h_bytes)),
-                "steps": e2e_steps},
+        "e2e": e2e,
         "gpu_launches": launches,
         "clocks": clocks,
     }
-    if world == 1 and not args.no_cpu_baseline:
+    if world == 1 and fwd and not args.no_cpu_baseline:
         v, el, reps, desc = oracle_run(name, T, reps_seconds=args.cpu_seconds, max_reps=8)
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
                                 "sample": desc, "seconds": el}
@@ -437,6 +487,9 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--stage", choices=["all", "bwd"], default="all",
+                    help="all: forward + backward (the step); bwd: the backward alone "
+                         "(indices from engram_hash, no table allocated)")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)      # at least 3 untimed warm-up steps
     if args.impl == "reference":

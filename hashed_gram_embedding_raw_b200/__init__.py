@@ -7,21 +7,19 @@ has not been built (`python hashed_gram_embedding_raw_b200/build.py`).
 """
 
 from ._binding import (ENGRAM_BF16, ENGRAM_DEVERR_CU_SEQLENS, ENGRAM_DEVERR_ROW_RANGE,
-                       ENGRAM_DEVERR_TIMEOUT,
                        ENGRAM_EINVAL, ENGRAM_ECUDA, ENGRAM_ENOSPC, ENGRAM_F16, ENGRAM_F32,
-                       ENGRAM_OK, EXPORTED, LIB_PATH, EngramError, EngramParams,
-                       ENGRAM_NOALLOC_SCRATCH_BYTES, engram_abi_version, engram_backward,
-                       engram_backward_noalloc, engram_backward_reduce,
-                       engram_backward_sort, engram_backward_workspace_size, engram_gather,
-                       engram_get_device_error, engram_hash, engram_hash_gather,
-                       engram_host_floor_mod, engram_launch_count, lib, make_params,
-                       status_string)
+                       ENGRAM_NOALLOC_SCRATCH_BYTES, ENGRAM_OK, EXPORTED, LIB_PATH,
+                       EngramError, EngramParams, engram_abi_version, engram_backward,
+                       engram_backward_noalloc, engram_backward_reduce, engram_backward_sort,
+                       engram_backward_workspace_size, engram_gather, engram_get_device_error,
+                       engram_hash, engram_hash_gather, engram_host_floor_mod,
+                       engram_launch_count, lib, make_params, status_string)
 
 __all__ = [
-    "ENGRAM_BF16", "ENGRAM_DEVERR_CU_SEQLENS", "ENGRAM_DEVERR_ROW_RANGE", "ENGRAM_DEVERR_TIMEOUT", "ENGRAM_EINVAL",
-    "ENGRAM_ECUDA", "ENGRAM_ENOSPC", "ENGRAM_F16", "ENGRAM_F32", "ENGRAM_OK", "EXPORTED",
-    "LIB_PATH", "EngramError", "EngramParams", "ENGRAM_NOALLOC_SCRATCH_BYTES",
-    "engram_abi_version", "engram_backward", "engram_backward_noalloc",
+    "ENGRAM_BF16", "ENGRAM_DEVERR_CU_SEQLENS", "ENGRAM_DEVERR_ROW_RANGE", "ENGRAM_EINVAL",
+    "ENGRAM_ECUDA", "ENGRAM_ENOSPC", "ENGRAM_F16", "ENGRAM_F32",
+    "ENGRAM_NOALLOC_SCRATCH_BYTES", "ENGRAM_OK", "EXPORTED", "LIB_PATH", "EngramError",
+    "EngramParams", "engram_abi_version", "engram_backward", "engram_backward_noalloc",
     "engram_backward_reduce", "engram_backward_sort", "engram_backward_workspace_size",
     "engram_gather", "engram_get_device_error", "engram_hash", "engram_hash_gather",
     "engram_host_floor_mod", "engram_launch_count", "lib", "make_params", "status_string",

@@ -6,16 +6,7 @@
 // owner is this GPU, and the gradient is kept compact: the distinct rows in
 // ascending order and one fp32 sum per row, never a dense table gradient.
 //
-// Stage 1 (sort): the pairs (idx[j], j) are packed as 64-bit items
-// key << 32 | j and sorted by key with a stable least-significant-digit radix
-// sort, 8 bits per pass, ceil(bits(table_rows - 1) / 8) passes, onesweep
-// style: one kernel counts the digits of every pass at once (the counts do not
-// depend on the order), then one kernel per pass ranks a 4096-item tile
-// stably in shared memory and finds the tile's global offsets by decoupled
-// look-back over the tiles before it. Tiles are handed out in launch order by
-// an atomic ticket, so every tile a block waits on belongs to a block that is
-// already running; each wait is bounded and raises ENGRAM_DEVERR_TIMEOUT
-// instead of hanging.
+// Stage 1 (sort): radix_sort.cuh orders the (row, lookup) pairs by row.
 //
 // Stage 2 (reduce): the sorted items are cut into one contiguous range per
 // resident warp. A segment is a run of equal keys. seg_count counts segment
@@ -33,229 +24,16 @@
 #pragma once
 
 #include "common.cuh"
+#include "radix_sort.cuh"
 
 namespace engram {
 namespace bwd {
-
-constexpr int kSortThreads = 256;
-constexpr int kSortItems = 16;
-constexpr int kSortTile = kSortThreads * kSortItems; // 4096 pairs per tile
-constexpr int kRadixBits = 8;
-constexpr int kRadix = 1 << kRadixBits;
-constexpr int kMaxPasses = 4; // keys below 2^32
-constexpr int kSortWarps = kSortThreads / 32;
-static_assert(kRadix == kSortThreads, "one thread per digit");
-
-// look-back status word: flag in the high half, count in the low half
-constexpr unsigned long long kFlagAggregate = 1ull << 32;
-constexpr unsigned long long kFlagPrefix = 2ull << 32;
-constexpr uint32_t kMaxSpin = 1u << 22; // ~0.1-1 s of polling before giving up
-constexpr int kLookback = 8;            // predecessor tiles read per look-back step
 
 constexpr int kSegThreads = 256;
 constexpr int kSegWarps = kSegThreads / 32;
 constexpr int kSegStages = 3;      // cp.async ring depth per warp
 constexpr int kSegMaxBatch = 8;    // rows per stage
 constexpr int kSegStageBytes = 4096;
-
-__device__ __forceinline__ uint32_t item_key(uint64_t it) { return (uint32_t)(it >> 32); }
-
-// Status words carry the flag and the count in one 64-bit word, so a reader
-// that sees the flag sees the count: relaxed (fence-free) accesses suffice.
-__device__ __forceinline__ void st_status(unsigned long long *p, unsigned long long v)
-{
-    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
-
-__device__ __forceinline__ unsigned long long ld_status(const unsigned long long *p)
-{
-    unsigned long long v;
-    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-    return v;
-}
-
-// ------------------------------------------------------------------- sort
-
-// Digit counts of every pass over all keys: ghist[pass * 256 + digit].
-__global__ void __launch_bounds__(kSortThreads)
-    radix_histogram(const int32_t *__restrict__ idx, int64_t n, int passes, uint32_t rows,
-                    uint32_t *__restrict__ ghist)
-{
-    __shared__ uint32_t s[kMaxPasses][kRadix];
-    for (int k = threadIdx.x; k < kMaxPasses * kRadix; k += kSortThreads)
-        (&s[0][0])[k] = 0;
-    __syncthreads();
-    bool bad = false;
-    const int64_t stride = (int64_t)gridDim.x * kSortThreads;
-    for (int64_t i0 = (int64_t)blockIdx.x * kSortThreads + threadIdx.x; i0 < n; i0 += 8 * stride) {
-        uint32_t key[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            const int64_t i = i0 + q * stride;
-            key[q] = i < n ? (uint32_t)__ldg(idx + i) : 0u;
-        }
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            if (i0 + q * stride < n) {
-                bad |= key[q] >= rows;
-                for (int p = 0; p < passes; ++p)
-                    atomicAdd(&s[p][(key[q] >> (p * kRadixBits)) & (kRadix - 1)], 1u);
-            }
-        }
-    }
-    if (bad)
-        raise_device_error(ENGRAM_DEVERR_ROW_RANGE);
-    __syncthreads();
-    for (int k = threadIdx.x; k < passes * kRadix; k += kSortThreads) {
-        const uint32_t c = (&s[0][0])[k];
-        if (c)
-            atomicAdd(ghist + k, c);
-    }
-}
-
-// Pass 0 reads the int32 indices and forms the items; later passes read items.
-template <bool FIRST>
-__device__ __forceinline__ uint64_t load_item(const void *__restrict__ src, int64_t i)
-{
-    if constexpr (FIRST) {
-        const uint32_t key = (uint32_t)__ldg((const int32_t *)src + i);
-        return ((uint64_t)key << 32) | (uint32_t)i;
-    } else {
-        return __ldg((const unsigned long long *)src + i);
-    }
-}
-
-// One stable pass: rank a tile by digit, find its global offsets by look-back,
-// scatter through shared memory.
-template <bool FIRST>
-__global__ void __launch_bounds__(kSortThreads)
-    radix_pass(const void *__restrict__ src, unsigned long long *__restrict__ dst, int64_t n,
-               int shift, const uint32_t *__restrict__ ghist, unsigned long long *status,
-               uint32_t *ticket)
-{
-    __shared__ uint32_t s_whist[kSortWarps][kRadix];
-    __shared__ uint32_t s_tstart[kRadix];
-    __shared__ uint32_t s_gbase[kRadix];
-    __shared__ uint32_t s_warp[32];
-    __shared__ unsigned long long s_items[kSortTile];
-    __shared__ int s_tile;
-
-    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    if (tid == 0)
-        s_tile = (int)atomicAdd(ticket, 1u);
-    for (int k = tid; k < kSortWarps * kRadix; k += kSortThreads)
-        (&s_whist[0][0])[k] = 0;
-    __syncthreads();
-    const int tile = s_tile;
-
-    // Each warp ranks its own 32 * kSortItems consecutive items, in order.
-    const int64_t base = (int64_t)tile * kSortTile;
-    const int64_t wbase = base + (int64_t)wid * (32 * kSortItems);
-    const uint32_t lt = lanemask_lt();
-    uint64_t it[kSortItems];
-    uint32_t rank[kSortItems];
-#pragma unroll
-    for (int r = 0; r < kSortItems; ++r) {
-        const int64_t i = wbase + r * 32 + lane;
-        it[r] = i < n ? load_item<FIRST>(src, i) : 0ull;
-    }
-#pragma unroll
-    for (int r = 0; r < kSortItems; ++r) {
-        const int64_t i = wbase + r * 32 + lane;
-        const bool valid = i < n;
-        const uint32_t d = valid ? (item_key(it[r]) >> shift) & (kRadix - 1) : kRadix;
-        const uint32_t peers = __match_any_sync(kFull, d);
-        const int leader = __ffs(peers) - 1;
-        uint32_t cnt = 0;
-        if (valid && lane == leader) {
-            cnt = s_whist[wid][d];
-            s_whist[wid][d] = cnt + __popc(peers);
-        }
-        cnt = __shfl_sync(kFull, cnt, leader);
-        rank[r] = cnt + __popc(peers & lt);
-        __syncwarp();
-    }
-    __syncthreads();
-
-    // Thread d: offsets of digit d per warp (warp order) and in the tile.
-    const int d = tid;
-    uint32_t tcount = 0;
-#pragma unroll
-    for (int w = 0; w < kSortWarps; ++w) {
-        const uint32_t c = s_whist[w][d];
-        s_whist[w][d] = tcount;
-        tcount += c;
-    }
-    // Publish this tile's count at once so the tiles after it can proceed.
-    unsigned long long *mine = status + (size_t)tile * kRadix + d;
-    st_status(mine, (tile == 0 ? kFlagPrefix : kFlagAggregate) | tcount);
-
-    // Stable order inside the tile, staged in shared memory.
-    const uint32_t tstart = block_exclusive_scan(tcount, s_warp, nullptr);
-    s_tstart[d] = tstart;
-    __syncthreads();
-#pragma unroll
-    for (int r = 0; r < kSortItems; ++r) {
-        const int64_t i = wbase + r * 32 + lane;
-        if (i < n) {
-            const uint32_t dd = (item_key(it[r]) >> shift) & (kRadix - 1);
-            s_items[s_tstart[dd] + s_whist[wid][dd] + rank[r]] = it[r];
-        }
-    }
-
-    // Decoupled look-back: add up the counts of the tiles before this one,
-    // kLookback at a time, back to the nearest one that already carries its
-    // inclusive prefix; then publish this tile's inclusive prefix.
-    uint32_t excl = 0;
-    if (tile > 0) {
-        int t = tile - 1;
-        uint32_t spins = 0;
-        while (t >= 0) {
-            unsigned long long w[kLookback];
-#pragma unroll
-            for (int q = 0; q < kLookback; ++q)
-                w[q] = t - q >= 0 ? ld_status(status + (size_t)(t - q) * kRadix + d)
-                                  : kFlagPrefix;
-            int q = 0; // predecessors consumed in this step
-            bool done = false, found = false;
-#pragma unroll
-            for (int k = 0; k < kLookback; ++k) {
-                if (!done) {
-                    const unsigned long long flag = w[k] & ~0xffffffffull;
-                    if (flag == 0) {
-                        done = true; // not published yet: reload from here
-                    } else {
-                        excl += (uint32_t)w[k];
-                        ++q;
-                        if (flag == kFlagPrefix)
-                            done = found = true;
-                    }
-                }
-            }
-            if (found)
-                break;
-            t -= q;
-            if (q == 0) {
-                if (++spins > kMaxSpin) {
-                    raise_device_error(ENGRAM_DEVERR_TIMEOUT);
-                    break;
-                }
-                __nanosleep(32);
-            }
-        }
-        st_status(mine, kFlagPrefix | (excl + tcount));
-    }
-
-    const uint32_t dbase = block_exclusive_scan(ghist[d], s_warp, nullptr);
-    s_gbase[d] = dbase + excl - tstart;
-    __syncthreads();
-    const int tile_n = (int)min64(kSortTile, n - base);
-    for (int p = tid; p < tile_n; p += kSortThreads) {
-        const unsigned long long x = s_items[p];
-        const uint32_t dd = (item_key(x) >> shift) & (kRadix - 1);
-        dst[(uint32_t)(s_gbase[dd] + (uint32_t)p)] = x;
-    }
-}
 
 // ------------------------------------------------------------------ reduce
 
@@ -513,35 +291,84 @@ __global__ void __launch_bounds__(kSegThreads)
         const unsigned char *stage = ring + (k % kSegStages) * stage_stride;
         const unsigned long long *smeta = (const unsigned long long *)(stage + stage_bytes);
         const int rows = min(batch, len - k * batch);
-        for (int r = 0; r < rows; ++r) {
-            const uint32_t key = item_key(smeta[r]);
-            if (key != prev_key) {
-                if (started) {
-                    // close the segment that ends just before this head
-                    if (open_here) {
-                        store_row<GF>(grads + (size_t)u * dim, sa, lane, F);
-                        if (lane == 0)
-                            uniq[u] = (int32_t)cur_key;
-                    } else {
-                        store_partial<GF>(pb + (size_t)w * dim, sa, lane, F);
-                        pb_ends = 1;
-                    }
+
+        // Close the open segment (it ends just before the current row).
+        auto close = [&]() {
+            if (open_here) {
+                store_row<GF>(grads + (size_t)u * dim, sa, lane, F);
+                if (lane == 0)
+                    uniq[u] = (int32_t)cur_key;
+            } else {
+                store_partial<GF>(pb + (size_t)w * dim, sa, lane, F);
+                pb_ends = 1;
+            }
+        };
+
+        bool all_heads = false;
+        if constexpr (RVT != 0) {
+            // Fast path: every row of a full batch starts its own segment (the
+            // common case when rows are nearly all distinct). Rows 0..rows-2
+            // are then complete one-lookup segments whose gradients are the
+            // rows themselves, and their outputs are contiguous in grads:
+            // convert and copy with fully coalesced stores.
+            const uint32_t mykey = lane < rows ? item_key(smeta[lane]) : 0u;
+            uint32_t up = __shfl_up_sync(kFull, mykey, 1);
+            if (lane == 0)
+                up = prev_key;
+            const uint32_t repeats = __ballot_sync(kFull, lane < rows && mykey == up);
+            all_heads = rows == batch && repeats == 0;
+            if (all_heads) {
+                if (started)
+                    close();
+                constexpr int FT = RVT * 16 / (DT == ENGRAM_F32 ? 16 : 8); // float4 groups per row
+                const int32_t ub = u + 1; // segment index of row 0
+                const int nv = (rows - 1) * FT;
+                float4 *gdst = (float4 *)(grads + (size_t)ub * dim);
+                for (int v = lane; v < nv; v += 32) {
+                    const int r = v / FT, f = v - r * FT;
+                    st_stream(gdst + v, load_quad<DT>(stage + r * RVT * 16, f));
                 }
-                ++u;
-                cur_key = key;
-                open_here = true;
+                if (lane < rows - 1)
+                    uniq[ub + lane] = (int32_t)mykey;
+                // the last row opens the next segment
+                const int rl = rows - 1;
                 sa.cnt = 0;
-            }
-            prev_key = key;
-            started = true;
-            const unsigned char *row = stage + r * rvec * 16;
 #pragma unroll
-            for (int g = 0; g < GF; ++g) {
-                const int f = lane + 32 * g;
-                if (f < F)
-                    sa.add(g, load_quad<DT>(row, f));
+                for (int g = 0; g < GF; ++g) {
+                    const int f = lane + 32 * g;
+                    if (f < F)
+                        sa.add(g, load_quad<DT>(stage + rl * RVT * 16, f));
+                }
+                sa.cnt = 1;
+                u = ub + rl;
+                cur_key = __shfl_sync(kFull, mykey, rl);
+                prev_key = cur_key;
+                open_here = true;
+                started = true;
             }
-            sa.cnt = min(sa.cnt + 1, 2);
+        }
+        if (!all_heads) {
+            for (int r = 0; r < rows; ++r) {
+                const uint32_t key = item_key(smeta[r]);
+                if (key != prev_key) {
+                    if (started)
+                        close();
+                    ++u;
+                    cur_key = key;
+                    open_here = true;
+                    sa.cnt = 0;
+                }
+                prev_key = key;
+                started = true;
+                const unsigned char *row = stage + r * rvec * 16;
+#pragma unroll
+                for (int g = 0; g < GF; ++g) {
+                    const int f = lane + 32 * g;
+                    if (f < F)
+                        sa.add(g, load_quad<DT>(row, f));
+                }
+                sa.cnt = min(sa.cnt + 1, 2);
+            }
         }
         __syncwarp();
         issue(k + kSegStages);

@@ -83,6 +83,14 @@ __device__ __forceinline__ void st_stream(float4 *p, float4 v)
                  : "memory");
 }
 
+// Load with acquire semantics at device scope (pairs with a releasing write).
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned *p)
+{
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
 __device__ __forceinline__ uint32_t lanemask_lt()
 {
     uint32_t m;

@@ -176,8 +176,8 @@ int launch_hash_gather(const HashArgs &a, const int32_t *ids, const int32_t *cu,
 // --------------------------------------------------------------- backward
 
 struct BwdPlan {
-    int passes = 0, ntiles = 0, wmax = 0, GF = 0;
-    size_t a = 0, b = 0, ctl = 0, ctl_bytes = 0, status = 0, ghist = 0, tickets = 0;
+    int passes = 0, ntiles = 0, ngroups = 0, wmax = 0, GF = 0;
+    size_t a = 0, b = 0, tile_cnt = 0, ctl = 0, ctl_bytes = 0, group_cnt = 0, barrier = 0;
     size_t wcount = 0, bcount = 0, pb = 0, pe = 0, meta = 0, total = 0;
 };
 
@@ -204,12 +204,13 @@ int bwd_plan(int64_t n, int64_t rows, int32_t dim, BwdPlan *P)
     const size_t nn = (size_t)std::max<int64_t>(n, 1);
     P->a = take(nn * 8);
     P->b = take(nn * 8);
-    // sort control block, zeroed once per sort: look-back status words of
-    // every pass, digit counts of every pass, tile tickets of every pass
+    // per-tile digit counts (rewritten by every pass), and per-group digit
+    // sums of every pass (accumulated with atomic adds, zeroed once per sort)
+    P->ngroups = (int)ceil_div(P->ntiles, bwd::kTilesPerGroup);
+    P->tile_cnt = take((size_t)bwd::kRadix * P->ntiles * 4);
     P->ctl = off;
-    P->status = take((size_t)P->passes * P->ntiles * bwd::kRadix * 8);
-    P->ghist = take((size_t)P->passes * bwd::kRadix * 4);
-    P->tickets = take((size_t)P->passes * 4);
+    P->group_cnt = take((size_t)P->passes * bwd::kRadix * P->ngroups * 4);
+    P->barrier = take(2 * sizeof(unsigned)); // grid barrier of the one-launch sort
     P->ctl_bytes = off - P->ctl;
     P->wcount = take((size_t)P->wmax * 4);
     P->bcount = take((size_t)ceil_div(P->wmax, bwd::kSegWarps) * 4);
@@ -235,28 +236,49 @@ int launch_sort(const int32_t *idx, int64_t n, int64_t rows, const BwdPlan &P, c
     using namespace bwd;
     auto *A = (unsigned long long *)(ws + P.a);
     auto *B = (unsigned long long *)(ws + P.b);
-    auto *status = (unsigned long long *)(ws + P.status);
-    auto *ghist = (uint32_t *)(ws + P.ghist);
-    auto *tickets = (uint32_t *)(ws + P.tickets);
+    auto *tile_cnt = (uint32_t *)(ws + P.tile_cnt);
+    auto *group_cnt = (uint32_t *)(ws + P.group_cnt);
     if (cudaMemsetAsync(ws + P.ctl, 0, P.ctl_bytes, stream) != cudaSuccess)
         return ENGRAM_ECUDA;
-    int sms = 0;
-    ENGRAM_TRY(device_sms(&sms));
-    const int hblocks = (int)std::max<int64_t>(
-        1, std::min<int64_t>((int64_t)sms * 2, ceil_div(n, kSortThreads * 8)));
-    radix_histogram<<<hblocks, kSortThreads, 0, stream>>>(idx, n, P.passes, (uint32_t)rows,
-                                                          ghist);
-    ENGRAM_TRY(after_launch());
+
+    // One cooperative launch for every pass when the device supports it: the
+    // grid is at most the co-resident blocks, which the launch itself checks.
+    int dev = 0, coop = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) == cudaSuccess &&
+        coop) {
+        int64_t res = 0;
+        ENGRAM_TRY(resident_warps(radix_sort_coop, kSortThreads, 0, &res));
+        const int grid = (int)std::min<int64_t>(P.ntiles, res / (kSortThreads / 32));
+        SortArgs args{idx, A, B, n, (uint32_t)rows, P.passes, P.ntiles, P.ngroups,
+                      tile_cnt, group_cnt, (unsigned *)(ws + P.barrier)};
+        void *params[] = {&args};
+        if (cudaLaunchCooperativeKernel((const void *)radix_sort_coop, dim3(grid),
+                                        dim3(kSortThreads), params, 0, stream) == cudaSuccess) {
+            g_launches.fetch_add(1, std::memory_order_relaxed);
+            return ENGRAM_OK;
+        }
+        (void)cudaGetLastError(); // not launched: run the phases as separate launches
+    }
+
     const void *src = idx;
     for (int pass = 0; pass < P.passes; ++pass) {
         unsigned long long *dst = (pass % 2 == 0) ? A : B;
-        unsigned long long *st = status + (size_t)pass * P.ntiles * kRadix;
-        if (pass == 0)
-            radix_pass<true><<<P.ntiles, kSortThreads, 0, stream>>>(
-                src, dst, n, pass * kRadixBits, ghist + pass * kRadix, st, tickets + pass);
-        else
-            radix_pass<false><<<P.ntiles, kSortThreads, 0, stream>>>(
-                src, dst, n, pass * kRadixBits, ghist + pass * kRadix, st, tickets + pass);
+        uint32_t *gc = group_cnt + (size_t)pass * kRadix * P.ngroups;
+        const int shift = pass * kRadixBits;
+        if (pass == 0) {
+            radix_count<true><<<P.ntiles, kSortThreads, 0, stream>>>(src, n, shift,
+                                                                    (uint32_t)rows, tile_cnt, gc);
+            ENGRAM_TRY(after_launch());
+            radix_scatter<true><<<P.ntiles, kSortThreads, 0, stream>>>(src, dst, n, shift,
+                                                                      tile_cnt, gc, P.ngroups);
+        } else {
+            radix_count<false><<<P.ntiles, kSortThreads, 0, stream>>>(src, n, shift,
+                                                                     (uint32_t)rows, tile_cnt, gc);
+            ENGRAM_TRY(after_launch());
+            radix_scatter<false><<<P.ntiles, kSortThreads, 0, stream>>>(src, dst, n, shift,
+                                                                       tile_cnt, gc, P.ngroups);
+        }
         ENGRAM_TRY(after_launch());
         src = dst;
     }

@@ -1,0 +1,328 @@
+// radix_sort.cuh -- stable LSD radix sort of the backward's (row, lookup) pairs.
+//
+// The pairs (idx[j], j) are packed as 64-bit items key << 32 | j and sorted by
+// key, 8 bits per pass, ceil(bits(table_rows - 1) / 8) passes. Because the
+// items start in j order and every pass is stable, equal keys end up in
+// ascending j.
+//
+// Each pass has two phases over 2048-item tiles:
+//   count    a tile's digit counts are stored (tile-major, tile_cnt[tile][d])
+//            and added into per-group sums (group_cnt[group][d], 32 tiles per
+//            group; the adds commute, so the sums are deterministic);
+//   scatter  a tile ranks its items stably in shared memory (per-warp digit
+//            counters, peers found with one ballot per digit bit), takes each
+//            digit's global offset as
+//              sum of all earlier digits' totals
+//              + that digit's group sums before the tile's group
+//              + that digit's tile counts earlier in the group
+//            (a few dozen independent, coalesced loads per thread), and writes
+//            the tile out in contiguous runs staged through shared memory.
+// No tile ever waits on another tile's result, so there is no serial prefix
+// chain across tiles.
+//
+// radix_sort_coop runs every phase of every pass in one cooperative launch:
+// each resident block takes tiles blockIdx.x, blockIdx.x + gridDim.x, ... and
+// the phases are separated by a grid barrier (bounded wait; a timeout raises
+// ENGRAM_DEVERR_SORT_TIMEOUT instead of hanging). Data written by other blocks
+// in the same launch is read through L2 (ld.global.cg), never through the
+// non-coherent load path. radix_count / radix_scatter run the same phases as
+// separate launches where cooperative launch is unavailable.
+#pragma once
+
+#include "common.cuh"
+
+namespace engram {
+namespace bwd {
+
+constexpr int kSortThreads = 256;
+constexpr int kSortItems = 8;
+constexpr int kSortTile = kSortThreads * kSortItems; // 2048 pairs per tile
+constexpr int kRadixBits = 8;
+constexpr int kRadix = 1 << kRadixBits;
+constexpr int kMaxPasses = 4; // keys below 2^32
+constexpr int kSortWarps = kSortThreads / 32;
+constexpr int kTilesPerGroup = 32;
+constexpr uint32_t kBarrierSpin = 1u << 22; // polls (~64 ns apart) before a barrier gives up
+static_assert(kRadix == kSortThreads, "one thread per digit");
+
+__device__ __forceinline__ uint32_t item_key(uint64_t it) { return (uint32_t)(it >> 32); }
+
+struct SortSmem {
+    uint32_t whist[kSortWarps][kRadix];
+    uint32_t tstart[kRadix];
+    uint32_t gbase[kRadix];
+    uint32_t cnt[kRadix];
+    uint32_t warp[32];
+    unsigned long long items[kSortTile];
+    int flag;
+};
+
+// Item i of a pass: pass 0 forms it from the int32 index, later passes read it.
+// COHERENT loads go through L2 only (needed when another block of the same
+// launch wrote the data); otherwise the read-only path is used.
+template <bool COHERENT>
+__device__ __forceinline__ uint64_t load_item(const void *__restrict__ src, bool first, int64_t i)
+{
+    if (first) {
+        const int32_t *p = (const int32_t *)src + i;
+        const uint32_t key = (uint32_t)(COHERENT ? __ldcg(p) : __ldg(p));
+        return ((uint64_t)key << 32) | (uint32_t)i;
+    }
+    const unsigned long long *p = (const unsigned long long *)src + i;
+    return COHERENT ? __ldcg(p) : __ldg(p);
+}
+
+template <bool COHERENT>
+__device__ __forceinline__ uint32_t load_u32(const uint32_t *p)
+{
+    return COHERENT ? __ldcg(p) : __ldg(p);
+}
+
+// Lanes of the warp whose digit equals this lane's (valid lanes only).
+__device__ __forceinline__ uint32_t digit_peers(uint32_t dg, bool valid)
+{
+    uint32_t peers = __ballot_sync(kFull, valid);
+#pragma unroll
+    for (int bit = 0; bit < kRadixBits; ++bit) {
+        const bool on = (dg >> bit) & 1u;
+        const uint32_t bal = __ballot_sync(kFull, on);
+        peers &= on ? bal : ~bal;
+    }
+    return peers;
+}
+
+// Count phase of one tile. Pass 0 also flags keys outside [0, rows).
+template <bool COHERENT>
+__device__ __forceinline__ void count_tile(SortSmem &sm, const void *src, bool first, int64_t n,
+                                           int shift, uint32_t rows, int tile,
+                                           uint32_t *tile_cnt, uint32_t *group_cnt)
+{
+    const int tid = threadIdx.x, lane = tid & 31;
+    sm.cnt[tid] = 0;
+    __syncthreads();
+    const int64_t base = (int64_t)tile * kSortTile;
+    uint32_t key[kSortItems];
+#pragma unroll
+    for (int r = 0; r < kSortItems; ++r) {
+        const int64_t i = base + r * kSortThreads + tid;
+        key[r] = i < n ? item_key(load_item<COHERENT>(src, first, i)) : 0u;
+    }
+    bool bad = false;
+#pragma unroll
+    for (int r = 0; r < kSortItems; ++r) {
+        const bool valid = base + r * kSortThreads + tid < n;
+        if (first && valid && key[r] >= rows)
+            bad = true;
+        // one shared-memory add per distinct digit in the warp, so runs of a
+        // hot key do not serialise on one counter
+        const uint32_t dg = (key[r] >> shift) & (kRadix - 1);
+        const uint32_t peers = digit_peers(dg, valid);
+        if (valid && lane == __ffs(peers) - 1)
+            atomicAdd(&sm.cnt[dg], (uint32_t)__popc(peers));
+    }
+    if (bad)
+        raise_device_error(ENGRAM_DEVERR_ROW_RANGE);
+    __syncthreads();
+    const uint32_t c = sm.cnt[tid];
+    tile_cnt[(size_t)tile * kRadix + tid] = c;
+    if (c)
+        atomicAdd(&group_cnt[(size_t)(tile / kTilesPerGroup) * kRadix + tid], c);
+    __syncthreads(); // sm.cnt free for the next tile
+}
+
+// Scatter phase of one tile (after every tile of the pass has been counted).
+template <bool COHERENT>
+__device__ __forceinline__ void scatter_tile(SortSmem &sm, const void *src, bool first,
+                                             unsigned long long *dst, int64_t n, int shift,
+                                             int tile, const uint32_t *tile_cnt,
+                                             const uint32_t *group_cnt, int ngroups)
+{
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    for (int k = tid; k < kSortWarps * kRadix; k += kSortThreads)
+        (&sm.whist[0][0])[k] = 0;
+
+    // Global offset of digit d = tid for this tile. Counts are tile- and
+    // group-major, so each load instruction reads 32 consecutive digits; the
+    // loops are unrolled so the loads are in flight together (and overlap the
+    // item loads below).
+    const int d = tid;
+    const int grp = tile / kTilesPerGroup;
+    uint32_t excl = 0, total = 0;
+    for (int g0 = 0; g0 < ngroups; g0 += 8) {
+        uint32_t c[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+            c[q] = g0 + q < ngroups
+                       ? load_u32<COHERENT>(group_cnt + (size_t)(g0 + q) * kRadix + d)
+                       : 0u;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            total += c[q];
+            if (g0 + q < grp)
+                excl += c[q];
+        }
+    }
+    {
+        const int t0 = grp * kTilesPerGroup;
+        uint32_t c[kTilesPerGroup];
+#pragma unroll
+        for (int q = 0; q < kTilesPerGroup; ++q)
+            c[q] = t0 + q < tile ? load_u32<COHERENT>(tile_cnt + (size_t)(t0 + q) * kRadix + d)
+                                 : 0u;
+#pragma unroll
+        for (int q = 0; q < kTilesPerGroup; ++q)
+            excl += c[q];
+    }
+
+    // Each warp ranks its own 32 * kSortItems consecutive items, in order.
+    const int64_t base = (int64_t)tile * kSortTile;
+    const int64_t wbase = base + (int64_t)wid * (32 * kSortItems);
+    const uint32_t lt = lanemask_lt();
+    uint64_t it[kSortItems];
+    uint32_t rank[kSortItems];
+#pragma unroll
+    for (int r = 0; r < kSortItems; ++r) {
+        const int64_t i = wbase + r * 32 + lane;
+        it[r] = i < n ? load_item<COHERENT>(src, first, i) : 0ull;
+    }
+    __syncthreads(); // whist zeroed
+#pragma unroll
+    for (int r = 0; r < kSortItems; ++r) {
+        const bool valid = wbase + r * 32 + lane < n;
+        const uint32_t dg = (item_key(it[r]) >> shift) & (kRadix - 1);
+        const uint32_t peers = digit_peers(dg, valid);
+        const int leader = valid ? __ffs(peers) - 1 : lane;
+        uint32_t cnt = 0;
+        if (valid && lane == leader) {
+            cnt = sm.whist[wid][dg];
+            sm.whist[wid][dg] = cnt + __popc(peers);
+        }
+        cnt = __shfl_sync(kFull, cnt, leader);
+        rank[r] = cnt + __popc(peers & lt);
+        __syncwarp();
+    }
+    __syncthreads();
+
+    // Thread d: offsets of digit d per warp (warp order) and in the tile.
+    uint32_t tcount = 0;
+#pragma unroll
+    for (int w = 0; w < kSortWarps; ++w) {
+        const uint32_t c = sm.whist[w][d];
+        sm.whist[w][d] = tcount;
+        tcount += c;
+    }
+    const uint32_t tstart = block_exclusive_scan(tcount, sm.warp, nullptr);
+    const uint32_t dbase = block_exclusive_scan(total, sm.warp, nullptr);
+    sm.tstart[d] = tstart;
+    sm.gbase[d] = dbase + excl - tstart;
+    __syncthreads();
+
+#pragma unroll
+    for (int r = 0; r < kSortItems; ++r) {
+        if (wbase + r * 32 + lane < n) {
+            const uint32_t dg = (item_key(it[r]) >> shift) & (kRadix - 1);
+            sm.items[sm.tstart[dg] + sm.whist[wid][dg] + rank[r]] = it[r];
+        }
+    }
+    __syncthreads();
+    const int tile_n = (int)min64(kSortTile, n - base);
+    for (int p = tid; p < tile_n; p += kSortThreads) {
+        const unsigned long long x = sm.items[p];
+        const uint32_t dg = (item_key(x) >> shift) & (kRadix - 1);
+        dst[(uint32_t)(sm.gbase[dg] + (uint32_t)p)] = x;
+    }
+    __syncthreads(); // shared memory free for the next tile
+}
+
+// ----------------------------------------------- one launch per phase
+
+template <bool FIRST>
+__global__ void __launch_bounds__(kSortThreads)
+    radix_count(const void *__restrict__ src, int64_t n, int shift, uint32_t rows,
+                uint32_t *__restrict__ tile_cnt, uint32_t *__restrict__ group_cnt)
+{
+    __shared__ SortSmem sm;
+    count_tile<false>(sm, src, FIRST, n, shift, rows, blockIdx.x, tile_cnt, group_cnt);
+}
+
+template <bool FIRST>
+__global__ void __launch_bounds__(kSortThreads)
+    radix_scatter(const void *__restrict__ src, unsigned long long *__restrict__ dst,
+                  int64_t n, int shift, const uint32_t *__restrict__ tile_cnt,
+                  const uint32_t *__restrict__ group_cnt, int ngroups)
+{
+    __shared__ SortSmem sm;
+    scatter_tile<false>(sm, src, FIRST, dst, n, shift, blockIdx.x, tile_cnt, group_cnt,
+                        ngroups);
+}
+
+// ------------------------------------------------ one cooperative launch
+
+struct SortArgs {
+    const int32_t *idx;
+    unsigned long long *a, *b; // ping-pong item buffers; pass p writes (p even ? a : b)
+    int64_t n;
+    uint32_t rows;
+    int passes, ntiles, ngroups;
+    uint32_t *tile_cnt;  // [ntiles][256], rewritten every pass
+    uint32_t *group_cnt; // [passes][ngroups][256], zero on entry
+    unsigned *barrier;   // [2]: arrival count, generation; zero on entry
+};
+
+// Grid-wide barrier among co-resident blocks. The last block to arrive resets
+// the count and advances the generation; the others poll it with a bound.
+// Returns false (and raises ENGRAM_DEVERR_SORT_TIMEOUT) if the wait gave up.
+__device__ __forceinline__ bool grid_barrier(unsigned *bar, unsigned &gen, int &flag)
+{
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const unsigned target = gen + 1;
+        bool ok = true;
+        __threadfence();
+        if (atomicAdd(&bar[0], 1u) == gridDim.x - 1) {
+            atomicExch(&bar[0], 0u);
+            __threadfence();
+            atomicExch(&bar[1], target);
+        } else {
+            uint32_t spins = 0;
+            while (ld_acquire_u32(&bar[1]) != target) {
+                if (++spins > kBarrierSpin) {
+                    raise_device_error(ENGRAM_DEVERR_SORT_TIMEOUT);
+                    ok = false;
+                    break;
+                }
+                __nanosleep(64);
+            }
+        }
+        __threadfence();
+        flag = ok;
+    }
+    __syncthreads();
+    gen += 1;
+    return flag != 0;
+}
+
+__global__ void __launch_bounds__(kSortThreads) radix_sort_coop(SortArgs a)
+{
+    __shared__ SortSmem sm;
+    unsigned gen = 0;
+    for (int pass = 0; pass < a.passes; ++pass) {
+        const bool first = pass == 0;
+        const void *src = first ? (const void *)a.idx : (pass % 2 == 1 ? a.a : a.b);
+        unsigned long long *dst = pass % 2 == 0 ? a.a : a.b;
+        uint32_t *gc = a.group_cnt + (size_t)pass * a.ngroups * kRadix;
+        const int shift = pass * kRadixBits;
+        for (int tile = blockIdx.x; tile < a.ntiles; tile += gridDim.x)
+            count_tile<true>(sm, src, first, a.n, shift, a.rows, tile, a.tile_cnt, gc);
+        if (!grid_barrier(a.barrier, gen, sm.flag))
+            return;
+        for (int tile = blockIdx.x; tile < a.ntiles; tile += gridDim.x)
+            scatter_tile<true>(sm, src, first, dst, a.n, shift, tile, a.tile_cnt, gc,
+                               a.ngroups);
+        if (pass + 1 < a.passes && !grid_barrier(a.barrier, gen, sm.flag))
+            return;
+    }
+}
+
+} // namespace bwd
+} // namespace engram

@@ -61,8 +61,8 @@ extern "C" {
 /* bits of the device error word */
 #define ENGRAM_DEVERR_ROW_RANGE 1u   /* a row index outside [0, table_rows) */
 #define ENGRAM_DEVERR_CU_SEQLENS 2u  /* cu_seqlens not non-decreasing from 0 to T */
-#define ENGRAM_DEVERR_TIMEOUT 4u     /* a bounded wait between blocks gave up (results invalid) */
-
+#define ENGRAM_DEVERR_SORT_TIMEOUT 4u /* the backward sort's grid barrier gave up waiting
+                                         (results of that call are invalid) */
 /* Same type as cudaStream_t, without requiring the CUDA headers. */
 typedef struct CUstream_st *engram_stream_t;
 
