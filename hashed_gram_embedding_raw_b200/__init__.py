@@ -12,7 +12,8 @@ from ._binding import (ENGRAM_BF16, ENGRAM_DEVERR_CU_SEQLENS, ENGRAM_DEVERR_ROW_
                        EngramError, EngramParams, engram_abi_version, engram_backward,
                        engram_backward_noalloc, engram_backward_reduce, engram_backward_sort,
                        engram_backward_workspace_size, engram_gather, engram_get_device_error,
-                       engram_hash, engram_hash_gather, engram_host_floor_mod,
+                       engram_hash, engram_hash_gather, engram_hash_gather_slice,
+                       engram_host_floor_mod,
                        engram_launch_count, lib, make_params, status_string)
 
 __all__ = [
@@ -22,5 +23,6 @@ __all__ = [
     "EngramParams", "engram_abi_version", "engram_backward", "engram_backward_noalloc",
     "engram_backward_reduce", "engram_backward_sort", "engram_backward_workspace_size",
     "engram_gather", "engram_get_device_error", "engram_hash", "engram_hash_gather",
+    "engram_hash_gather_slice",
     "engram_host_floor_mod", "engram_launch_count", "lib", "make_params", "status_string",
 ]

@@ -30,7 +30,7 @@ EXPORTED = (
     "engram_backward_workspace_size", "engram_backward", "engram_backward_sort",
     "engram_backward_reduce", "engram_get_device_error", "engram_status_string",
     "engram_abi_version", "engram_params_size", "engram_launch_count",
-    "engram_host_floor_mod", "engram_backward_noalloc",
+    "engram_host_floor_mod", "engram_backward_noalloc", "engram_hash_gather_slice",
 )
 
 ENGRAM_NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -104,6 +104,7 @@ def _load():
         "engram_launch_count": [],
         "engram_host_floor_mod": [i64, i64, ctypes.POINTER(ctypes.c_int)],
         "engram_backward_noalloc": [P, i64, i64, i32, P, i32, P, P, P, P],
+        "engram_hash_gather_slice": [P, P, P, i32, i64, i64, i64, i64, P, i32, P, P, P],
     }
     for name, args in sig.items():
         fn = getattr(L, name)
@@ -221,6 +222,40 @@ def engram_hash_gather(params: EngramParams, ids: torch.Tensor, table: torch.Ten
     _check(lib.engram_hash_gather(ctypes.byref(params), _ptr(ids), _ptr(cu), nseq, T,
                                   _ptr(table), _dtype_code(table), _ptr(out_idx), _ptr(out),
                                   _stream(stream)), "engram_hash_gather")
+    return out, out_idx
+
+
+def engram_hash_gather_slice(params: EngramParams, ids: torch.Tensor, table: torch.Tensor,
+                             start: int, end: int, row_len: int = 0, cu_seqlens=None,
+                             out=None, out_idx=None, want_idx: bool = True, stream=None):
+    """_forward_global_slice: hash the whole stream, look up positions
+    [start, end) of every row of row_len tokens (0: one row). Returns
+    (out [rows, end - start, H * dim], out_idx [rows, end - start, H] or None)."""
+    _cuda(ids, "ids", torch.int32)
+    _cuda(table, "table")
+    if table.shape != (params.table_rows, params.dim):
+        raise ValueError("table shape must be (params.table_rows, params.dim)")
+    T, H = ids.numel(), params.heads
+    row = row_len or T
+    if row <= 0 or T % row or not 0 <= start <= end <= row:
+        raise ValueError("need 0 <= start <= end <= row_len and T divisible by row_len")
+    nrows, ln = T // row, end - start
+    cu, nseq = _cu_args(cu_seqlens)
+    if out is None:
+        out = torch.empty((nrows, ln, H * params.dim), dtype=table.dtype, device=table.device)
+    _cuda(out, "out", table.dtype)
+    if out.numel() != nrows * ln * H * params.dim:
+        raise ValueError("out must hold rows * (end - start) * H * dim elements")
+    if out_idx is None and want_idx:
+        out_idx = torch.empty((nrows, ln, H), dtype=torch.int32, device=ids.device)
+    if out_idx is not None:
+        _cuda(out_idx, "out_idx", torch.int32)
+        if out_idx.numel() != nrows * ln * H:
+            raise ValueError("out_idx must hold rows * (end - start) * H elements")
+    _check(lib.engram_hash_gather_slice(ctypes.byref(params), _ptr(ids), _ptr(cu), nseq, T,
+                                        row_len, start, end, _ptr(table), _dtype_code(table),
+                                        _ptr(out_idx), _ptr(out), _stream(stream)),
+           "engram_hash_gather_slice")
     return out, out_idx
 
 

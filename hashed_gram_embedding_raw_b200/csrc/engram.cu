@@ -153,23 +153,28 @@ int launch_hash(const HashArgs &a, const int32_t *ids, const int32_t *cu, int32_
     return after_launch();
 }
 
+// slice == nullptr: the whole stream; else only the slice's nlog tokens.
 int launch_hash_gather(const HashArgs &a, const int32_t *ids, const int32_t *cu, int32_t nseq,
                        int64_t T, const void *table, int V, int32_t *out_idx, void *out,
-                       cudaStream_t stream)
+                       cudaStream_t stream, const SliceMap *slice = nullptr, int64_t nlog = 0)
 {
     const size_t smem = (size_t)(kHashThreads / 32) * 32 * (a.H + 1) * sizeof(int32_t);
     const bool page_shape = a.N == 3 && a.K == 8;
-    auto fn = hash_gather_kernel<0, 0, 0>;
+    const bool mapped = slice != nullptr;
+    auto fn = mapped ? hash_gather_kernel<0, 0, 0, true> : hash_gather_kernel<0, 0, 0, false>;
     if (page_shape && V == 20)
-        fn = hash_gather_kernel<3, 8, 20>;
+        fn = mapped ? hash_gather_kernel<3, 8, 20, true> : hash_gather_kernel<3, 8, 20, false>;
     else if (page_shape && V == 40)
-        fn = hash_gather_kernel<3, 8, 40>;
+        fn = mapped ? hash_gather_kernel<3, 8, 40, true> : hash_gather_kernel<3, 8, 40, false>;
     int64_t res = 0;
     ENGRAM_TRY(resident_warps(fn, kHashThreads, smem, &res));
-    const int64_t nwarps = std::min<int64_t>(res, ceil_div(T, 8));
+    const int64_t units = mapped ? nlog : T;
+    const int64_t nwarps = std::max<int64_t>(1, std::min<int64_t>(res, ceil_div(units, 8)));
     const int64_t blocks = ceil_div(nwarps, kHashThreads / 32);
-    fn<<<(unsigned)blocks, kHashThreads, smem, stream>>>(
-        a, ids, cu, nseq, T, nwarps, (const uint4 *)table, V, out_idx, (uint4 *)out);
+    const SliceMap m = mapped ? *slice : SliceMap{0, 0, 1};
+    fn<<<(unsigned)blocks, kHashThreads, smem, stream>>>(a, ids, cu, nseq, T, nwarps,
+                                                         (const uint4 *)table, V, out_idx,
+                                                         (uint4 *)out, m, nlog);
     return after_launch();
 }
 
@@ -434,6 +439,33 @@ int engram_hash_gather(const engram_params_t *params, const int32_t *ids,
     const int V = (int)((int64_t)params->dim * eb / 16);
     return launch_hash_gather(a, ids, cu_seqlens, nseq, T, table, V, out_idx, out,
                               (cudaStream_t)stream);
+}
+
+int engram_hash_gather_slice(const engram_params_t *params, const int32_t *ids,
+                             const int32_t *cu_seqlens, int32_t nseq, int64_t T, int64_t row_len,
+                             int64_t start, int64_t end, const void *table, int32_t dtype,
+                             int32_t *out_idx, void *out, engram_stream_t stream)
+{
+    HashArgs a;
+    ENGRAM_TRY(make_hash_args(params, &a));
+    const int eb = elem_bytes(dtype);
+    if (eb == 0 || ((int64_t)params->dim * eb) % 16 != 0)
+        return ENGRAM_EINVAL;
+    if (T < 0 || T > INT32_MAX || (cu_seqlens != nullptr && nseq < 1))
+        return ENGRAM_EINVAL;
+    const int64_t row = row_len == 0 ? T : row_len;
+    if (row < 0 || (row > 0 && T % row != 0) || start < 0 || end < start || end > row)
+        return ENGRAM_EINVAL;
+    const int64_t len = end - start;
+    if (T == 0 || len == 0)
+        return ENGRAM_OK;
+    if (ids == nullptr || table == nullptr || out == nullptr || !aligned16(table) ||
+        !aligned16(out))
+        return ENGRAM_EINVAL;
+    const int V = (int)((int64_t)params->dim * eb / 16);
+    const SliceMap m{row, start, len};
+    return launch_hash_gather(a, ids, cu_seqlens, nseq, T, table, V, out_idx, out,
+                              (cudaStream_t)stream, &m, (T / row) * len);
 }
 
 int engram_backward_workspace_size(int64_t n, int64_t table_rows, int32_t dim, size_t *bytes)

@@ -64,27 +64,47 @@ __device__ __forceinline__ void check_cu_seqlens(const int32_t *__restrict__ cu,
     }
 }
 
-// Hashes tokens t0 .. t0+31 below t_end (lane l owns t0 + l) and writes their
-// H row indices to s_idx[l * HP + h]. `s` is the warp's cursor into
-// cu_seqlens: on entry cu[s] <= t0; on exit s is the largest index below nseq
-// whose bound is <= the chunk's last token.
-template <int NT, int KT>
+// A slice of the stream (_forward_global_slice): positions [start, start+len)
+// of every row of `row` tokens. Logical token L of the slice is stream
+// position (L / len) * row + start + L % len; the identity map has row = len
+// = 1 << 62, start = 0.
+struct SliceMap {
+    int64_t row, start, len;
+};
+
+__device__ __forceinline__ int64_t slice_token(const SliceMap &m, int64_t L)
+{
+    return (L / m.len) * m.row + m.start + L % m.len;
+}
+
+// Hashes logical tokens l0 .. l0+31 below l_end (lane i owns l0 + i) and
+// writes their H row indices to s_idx[i * HP + h]. Without MAPPED the logical
+// token is the stream position and the earlier tokens come from neighbouring
+// lanes; with MAPPED the position comes from the slice map and earlier tokens
+// are read from global memory (the whole stream is there, so context from
+// before the slice is kept). `s` is the warp's cursor into cu_seqlens: on
+// entry cu[s] <= the chunk's first position; on exit s is the largest index
+// below nseq whose bound is <= the chunk's last position.
+template <int NT, int KT, bool MAPPED = false>
 __device__ __forceinline__ void hash_chunk(const HashArgs &a, const int32_t *__restrict__ ids,
                                            const int32_t *__restrict__ cu, int32_t nseq,
-                                           int64_t T, int64_t t0, int64_t t_end, int32_t &s,
-                                           int32_t *s_idx, int HP, int lane)
+                                           int64_t T, int64_t l0, int64_t l_end, int32_t &s,
+                                           int32_t *s_idx, int HP, int lane,
+                                           const SliceMap &m = SliceMap{0, 0, 1})
 {
     const int N = NT ? NT : a.N;
     const int K = KT ? KT : a.K;
-    const int64_t t = t0 + lane;
-    const int32_t x0 = t < t_end ? __ldg(ids + t) : 0;
+    const int64_t L = l0 + lane;
+    const int64_t t = MAPPED ? slice_token(m, min(L, l_end - 1)) : L;
+    const int32_t x0 = L < l_end ? __ldg(ids + t) : 0;
 
     // Start of the lane's sequence: sequence bounds inside this chunk are
     // visited in order, each lane keeping the last one at or before its token.
     int64_t S = 0;
     if (cu != nullptr) {
         S = __ldg(cu + s);
-        const int64_t last = min(t0 + 31, t_end - 1);
+        const int64_t llast = min(l0 + 31, l_end - 1);
+        const int64_t last = MAPPED ? slice_token(m, llast) : llast;
         while (s + 1 < nseq) {
             const int64_t b = __ldg(cu + s + 1);
             if (b > last)
@@ -103,9 +123,14 @@ __device__ __forceinline__ void hash_chunk(const HashArgs &a, const int32_t *__r
 #pragma unroll
     for (int k = 1; k < ENGRAM_MAX_NGRAM; ++k) {
         if (k < N) {
-            int32_t prev = __shfl_up_sync(kFull, x0, k);
-            if (lane < k)
-                prev = (t - k >= 0 && t - k < T) ? __ldg(ids + t - k) : 0;
+            int32_t prev;
+            if constexpr (MAPPED) {
+                prev = t - k >= 0 ? __ldg(ids + t - k) : 0;
+            } else {
+                prev = __shfl_up_sync(kFull, x0, k);
+                if (lane < k)
+                    prev = (t - k >= 0 && t - k < T) ? __ldg(ids + t - k) : 0;
+            }
             ok = ok && (t - k >= S) && (prev != a.eos);
             x[k] = ok ? (int64_t)prev : a.fill;
         }
@@ -173,12 +198,15 @@ __global__ void __launch_bounds__(kHashThreads)
 
 // engram_hash_gather: hash a chunk, then stream its rows.
 // VT = 16-byte vectors per row (20 for bf16 x 160, 40 for fp32 x 160); 0 = runtime.
-template <int NT, int KT, int VT>
+// MAPPED: hash and gather only the slice described by m (nlog logical tokens
+// of the T-token stream); outputs are indexed by logical token.
+template <int NT, int KT, int VT, bool MAPPED = false>
 __global__ void __launch_bounds__(kHashThreads)
     hash_gather_kernel(HashArgs a, const int32_t *__restrict__ ids,
                        const int32_t *__restrict__ cu, int32_t nseq, int64_t T, int64_t nwarps,
                        const uint4 *__restrict__ table, int v_rt,
-                       int32_t *__restrict__ out_idx, uint4 *__restrict__ out)
+                       int32_t *__restrict__ out_idx, uint4 *__restrict__ out,
+                       SliceMap m = SliceMap{0, 0, 1}, int64_t nlog = 0)
 {
     extern __shared__ int32_t smem[];
     if (cu != nullptr)
@@ -193,11 +221,13 @@ __global__ void __launch_bounds__(kHashThreads)
     if (w >= nwarps)
         return;
     int64_t tb, te;
-    warp_range(T, w, nwarps, tb, te);
-    int32_t s = cu != nullptr ? find_sequence(cu, nseq, tb) : 0;
+    warp_range(MAPPED ? nlog : T, w, nwarps, tb, te);
+    if (tb >= te)
+        return;
+    int32_t s = cu != nullptr ? find_sequence(cu, nseq, MAPPED ? slice_token(m, tb) : tb) : 0;
 
     for (int64_t t0 = tb; t0 < te; t0 += 32) {
-        hash_chunk<NT, KT>(a, ids, cu, nseq, T, t0, te, s, s_idx, HP, lane);
+        hash_chunk<NT, KT, MAPPED>(a, ids, cu, nseq, T, t0, te, s, s_idx, HP, lane, m);
         __syncwarp();
         const int ntok = (int)min64(32, te - t0);
         if (out_idx != nullptr)

@@ -143,6 +143,27 @@ ENGRAM_API int engram_hash_gather(const engram_params_t *params, const int32_t *
                        void *out, engram_stream_t stream);
 
 /*
+ * engram_hash_gather_slice -- NGramEmbedding._forward_global_slice: hash the
+ * complete stream but look up only positions [start, end) of every row, so
+ * the earlier tokens and the EOS / sequence resets that a slice boundary cuts
+ * off still shape the slice's first tokens (the page hashes the replicated
+ * global IDs for this reason when context parallelism shards the sequence).
+ *   ids, cu_seqlens, nseq, T  the whole stream, as for engram_hash
+ *   row_len    tokens per row of a [T / row_len, row_len] batch (T must be a
+ *              multiple); 0 means one row of T tokens
+ *   start, end 0 <= start <= end <= row length
+ *   out_idx    device, int32 [T / row_len, end - start, H] (may be NULL)
+ *   out        device, [T / row_len, end - start, H * dim] of dtype
+ * Equal to engram_hash_gather over the whole stream followed by taking
+ * positions [start, end) of every row, without computing the rest.
+ */
+ENGRAM_API int engram_hash_gather_slice(const engram_params_t *params, const int32_t *ids,
+                                        const int32_t *cu_seqlens, int32_t nseq, int64_t T,
+                                        int64_t row_len, int64_t start, int64_t end,
+                                        const void *table, int32_t dtype, int32_t *out_idx,
+                                        void *out, engram_stream_t stream);
+
+/*
  * engram_backward_workspace_size -- bytes of scratch engram_backward needs for
  * n lookups into a table of table_rows rows of width dim, on the current
  * device (the size depends on its SM count).

@@ -110,6 +110,13 @@ def test_host_rejects_bad_params(E):
     assert L.engram_hash(ctypes.byref(p), None, None, 1, 10, dummy, None) == E.ENGRAM_EINVAL
     # T = 0 is a no-op
     assert L.engram_hash(ctypes.byref(p), None, None, 1, 0, None, None) == E.ENGRAM_OK
+    # slices: start > end, end past the row, T not a multiple of the row length
+    for row_len, start, end in [(64, 10, 5), (64, 0, 65), (60, 0, 10), (-5, 0, 1)]:
+        assert L.engram_hash_gather_slice(ctypes.byref(p), dummy, None, 1, 128, row_len, start,
+                                          end, dummy, 1, None, dummy, None) == E.ENGRAM_EINVAL
+    # an empty slice is a no-op
+    assert L.engram_hash_gather_slice(ctypes.byref(p), dummy, None, 1, 128, 64, 7, 7, dummy,
+                                      1, None, dummy, None) == E.ENGRAM_OK
 
 
 def test_host_rejects_bad_gather_and_backward_args(E):
