@@ -135,4 +135,37 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t *s
     return before + x - v;
 }
 
+// The same scan over 64-bit values (no total); s_warp holds 32 words.
+__device__ __forceinline__ unsigned long long block_exclusive_scan64(unsigned long long v,
+                                                                    unsigned long long *s_warp)
+{
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int nw = blockDim.x >> 5;
+    unsigned long long x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned long long y = __shfl_up_sync(kFull, x, o);
+        if (lane >= o)
+            x += y;
+    }
+    if (lane == 31)
+        s_warp[wid] = x;
+    __syncthreads();
+    if (wid == 0) {
+        unsigned long long s = lane < nw ? s_warp[lane] : 0ull;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned long long y = __shfl_up_sync(kFull, s, o);
+            if (lane >= o)
+                s += y;
+        }
+        if (lane < nw)
+            s_warp[lane] = s;
+    }
+    __syncthreads();
+    const unsigned long long before = wid ? s_warp[wid - 1] : 0ull;
+    __syncthreads();
+    return before + x - v;
+}
+
 } // namespace engram

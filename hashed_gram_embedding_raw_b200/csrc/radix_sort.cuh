@@ -53,6 +53,7 @@ struct SortSmem {
     uint32_t gbase[kRadix];
     uint32_t cnt[kRadix];
     uint32_t warp[32];
+    unsigned long long warp2[32];
     unsigned long long items[kSortTile];
     int flag;
 };
@@ -130,21 +131,88 @@ __device__ __forceinline__ void count_tile(SortSmem &sm, const void *src, bool f
     __syncthreads(); // sm.cnt free for the next tile
 }
 
-// Scatter phase of one tile (after every tile of the pass has been counted).
+// Loads the tile's items and ranks them stably: rank[r] is item r's position
+// among the items of its digit in its warp, and sm.whist[w][d] ends up as the
+// number of items of digit d in warp w. Pass 0 also flags keys outside the table.
 template <bool COHERENT>
-__device__ __forceinline__ void scatter_tile(SortSmem &sm, const void *src, bool first,
-                                             unsigned long long *dst, int64_t n, int shift,
-                                             int tile, const uint32_t *tile_cnt,
-                                             const uint32_t *group_cnt, int ngroups)
+__device__ __forceinline__ void rank_tile(SortSmem &sm, const void *src, bool first, int64_t n,
+                                          int shift, uint32_t rows, int tile,
+                                          uint64_t (&it)[kSortItems],
+                                          uint32_t (&rank)[kSortItems])
 {
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     for (int k = tid; k < kSortWarps * kRadix; k += kSortThreads)
         (&sm.whist[0][0])[k] = 0;
+    const int64_t wbase = (int64_t)tile * kSortTile + (int64_t)wid * (32 * kSortItems);
+    const uint32_t lt = lanemask_lt();
+#pragma unroll
+    for (int r = 0; r < kSortItems; ++r) {
+        const int64_t i = wbase + r * 32 + lane;
+        it[r] = i < n ? load_item<COHERENT>(src, first, i) : 0ull;
+    }
+    __syncthreads(); // whist zeroed
+    bool bad = false;
+#pragma unroll
+    for (int r = 0; r < kSortItems; ++r) {
+        const bool valid = wbase + r * 32 + lane < n;
+        if (first && valid && item_key(it[r]) >= rows)
+            bad = true;
+        const uint32_t dg = (item_key(it[r]) >> shift) & (kRadix - 1);
+        const uint32_t peers = digit_peers(dg, valid);
+        const int leader = valid ? __ffs(peers) - 1 : lane;
+        uint32_t cnt = 0;
+        if (valid && lane == leader) {
+            cnt = sm.whist[wid][dg];
+            sm.whist[wid][dg] = cnt + __popc(peers);
+        }
+        cnt = __shfl_sync(kFull, cnt, leader);
+        rank[r] = cnt + __popc(peers & lt);
+        __syncwarp();
+    }
+    if (bad)
+        raise_device_error(ENGRAM_DEVERR_ROW_RANGE);
+    __syncthreads();
+}
 
+// Thread d: turns sm.whist[.][d] into per-warp exclusive offsets and returns
+// the tile's count of digit d.
+__device__ __forceinline__ uint32_t tile_digit_count(SortSmem &sm)
+{
+    const int d = threadIdx.x;
+    uint32_t tcount = 0;
+#pragma unroll
+    for (int w = 0; w < kSortWarps; ++w) {
+        const uint32_t c = sm.whist[w][d];
+        sm.whist[w][d] = tcount;
+        tcount += c;
+    }
+    return tcount;
+}
+
+// Stores a tile's digit counts (tile-major) and adds them into its group's sums.
+__device__ __forceinline__ void publish_counts(int tile, uint32_t tcount, uint32_t *tile_cnt,
+                                               uint32_t *group_cnt)
+{
+    const int d = threadIdx.x;
+    tile_cnt[(size_t)tile * kRadix + d] = tcount;
+    if (tcount)
+        atomicAdd(&group_cnt[(size_t)(tile / kTilesPerGroup) * kRadix + d], tcount);
+}
+
+// Writes a ranked tile to its sorted positions, once every tile of the pass
+// has published its counts. tcount is digit threadIdx.x's count in the tile.
+template <bool COHERENT>
+__device__ __forceinline__ void place_tile(SortSmem &sm, unsigned long long *dst, int64_t n,
+                                           int shift, int tile, uint32_t tcount,
+                                           const uint64_t (&it)[kSortItems],
+                                           const uint32_t (&rank)[kSortItems],
+                                           const uint32_t *tile_cnt, const uint32_t *group_cnt,
+                                           int ngroups)
+{
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     // Global offset of digit d = tid for this tile. Counts are tile- and
     // group-major, so each load instruction reads 32 consecutive digits; the
-    // loops are unrolled so the loads are in flight together (and overlap the
-    // item loads below).
+    // loops are unrolled so the loads are in flight together.
     const int d = tid;
     const int grp = tile / kTilesPerGroup;
     uint32_t excl = 0, total = 0;
@@ -174,49 +242,16 @@ __device__ __forceinline__ void scatter_tile(SortSmem &sm, const void *src, bool
             excl += c[q];
     }
 
-    // Each warp ranks its own 32 * kSortItems consecutive items, in order.
-    const int64_t base = (int64_t)tile * kSortTile;
-    const int64_t wbase = base + (int64_t)wid * (32 * kSortItems);
-    const uint32_t lt = lanemask_lt();
-    uint64_t it[kSortItems];
-    uint32_t rank[kSortItems];
-#pragma unroll
-    for (int r = 0; r < kSortItems; ++r) {
-        const int64_t i = wbase + r * 32 + lane;
-        it[r] = i < n ? load_item<COHERENT>(src, first, i) : 0ull;
-    }
-    __syncthreads(); // whist zeroed
-#pragma unroll
-    for (int r = 0; r < kSortItems; ++r) {
-        const bool valid = wbase + r * 32 + lane < n;
-        const uint32_t dg = (item_key(it[r]) >> shift) & (kRadix - 1);
-        const uint32_t peers = digit_peers(dg, valid);
-        const int leader = valid ? __ffs(peers) - 1 : lane;
-        uint32_t cnt = 0;
-        if (valid && lane == leader) {
-            cnt = sm.whist[wid][dg];
-            sm.whist[wid][dg] = cnt + __popc(peers);
-        }
-        cnt = __shfl_sync(kFull, cnt, leader);
-        rank[r] = cnt + __popc(peers & lt);
-        __syncwarp();
-    }
-    __syncthreads();
-
-    // Thread d: offsets of digit d per warp (warp order) and in the tile.
-    uint32_t tcount = 0;
-#pragma unroll
-    for (int w = 0; w < kSortWarps; ++w) {
-        const uint32_t c = sm.whist[w][d];
-        sm.whist[w][d] = tcount;
-        tcount += c;
-    }
-    const uint32_t tstart = block_exclusive_scan(tcount, sm.warp, nullptr);
-    const uint32_t dbase = block_exclusive_scan(total, sm.warp, nullptr);
+    // One scan over digits gives both the tile-local start (low half) and the
+    // start of the digit among all digits (high half).
+    const unsigned long long both = block_exclusive_scan64(
+        ((unsigned long long)total << 32) | tcount, (unsigned long long *)sm.warp2);
+    const uint32_t tstart = (uint32_t)both, dbase = (uint32_t)(both >> 32);
     sm.tstart[d] = tstart;
     sm.gbase[d] = dbase + excl - tstart;
     __syncthreads();
 
+    const int64_t wbase = (int64_t)tile * kSortTile + (int64_t)wid * (32 * kSortItems);
 #pragma unroll
     for (int r = 0; r < kSortItems; ++r) {
         if (wbase + r * 32 + lane < n) {
@@ -225,6 +260,7 @@ __device__ __forceinline__ void scatter_tile(SortSmem &sm, const void *src, bool
         }
     }
     __syncthreads();
+    const int64_t base = (int64_t)tile * kSortTile;
     const int tile_n = (int)min64(kSortTile, n - base);
     for (int p = tid; p < tile_n; p += kSortThreads) {
         const unsigned long long x = sm.items[p];
@@ -232,6 +268,22 @@ __device__ __forceinline__ void scatter_tile(SortSmem &sm, const void *src, bool
         dst[(uint32_t)(sm.gbase[dg] + (uint32_t)p)] = x;
     }
     __syncthreads(); // shared memory free for the next tile
+}
+
+// Scatter phase of one tile after a separate count phase: rank, then place.
+template <bool COHERENT>
+__device__ __forceinline__ void scatter_tile(SortSmem &sm, const void *src, bool first,
+                                             unsigned long long *dst, int64_t n, int shift,
+                                             int tile, const uint32_t *tile_cnt,
+                                             const uint32_t *group_cnt, int ngroups)
+{
+    uint64_t it[kSortItems];
+    uint32_t rank[kSortItems];
+    // (the count phase has already checked the keys against the table)
+    rank_tile<COHERENT>(sm, src, first, n, shift, 0xffffffffu, tile, it, rank);
+    const uint32_t tcount = tile_digit_count(sm);
+    place_tile<COHERENT>(sm, dst, n, shift, tile, tcount, it, rank, tile_cnt, group_cnt,
+                         ngroups);
 }
 
 // ----------------------------------------------- one launch per phase
@@ -302,10 +354,41 @@ __device__ __forceinline__ bool grid_barrier(unsigned *bar, unsigned &gen, int &
     return flag != 0;
 }
 
-__global__ void __launch_bounds__(kSortThreads) radix_sort_coop(SortArgs a)
+// Four blocks per SM keep 592 tiles (1.2M pairs) resident on a 148-SM B200.
+__global__ void __launch_bounds__(kSortThreads, 4) radix_sort_coop(SortArgs a)
 {
     __shared__ SortSmem sm;
     unsigned gen = 0;
+    if (a.ntiles <= (int)gridDim.x) {
+        // One tile per block: rank once, keep the items and their ranks in
+        // registers (and the per-warp offsets in shared memory) across the
+        // barrier, then place them.
+        const int tile = blockIdx.x;
+        const bool has = tile < a.ntiles;
+        for (int pass = 0; pass < a.passes; ++pass) {
+            const bool first = pass == 0;
+            const void *src = first ? (const void *)a.idx : (pass % 2 == 1 ? a.a : a.b);
+            unsigned long long *dst = pass % 2 == 0 ? a.a : a.b;
+            uint32_t *gc = a.group_cnt + (size_t)pass * a.ngroups * kRadix;
+            const int shift = pass * kRadixBits;
+            uint64_t it[kSortItems];
+            uint32_t rank[kSortItems];
+            uint32_t tcount = 0;
+            if (has) {
+                rank_tile<true>(sm, src, first, a.n, shift, a.rows, tile, it, rank);
+                tcount = tile_digit_count(sm);
+                publish_counts(tile, tcount, a.tile_cnt, gc);
+            }
+            if (!grid_barrier(a.barrier, gen, sm.flag))
+                return;
+            if (has)
+                place_tile<true>(sm, dst, a.n, shift, tile, tcount, it, rank, a.tile_cnt, gc,
+                                 a.ngroups);
+            if (pass + 1 < a.passes && !grid_barrier(a.barrier, gen, sm.flag))
+                return;
+        }
+        return;
+    }
     for (int pass = 0; pass < a.passes; ++pass) {
         const bool first = pass == 0;
         const void *src = first ? (const void *)a.idx : (pass % 2 == 1 ? a.a : a.b);
