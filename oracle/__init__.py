@@ -1,4 +1,5 @@
-"""CPU oracle of the Engram N-gram Embedding path (hash, gather, backward).
+"""CPU oracle of the Engram N-gram Embedding path (hash, gather, backward,
+and the PLE layer's grouped RMS norm and causal short convolution).
 
 TEST INFRASTRUCTURE ONLY. Only `tests/`, `__graft_entry__.smoke()` and the
 CPU-baseline / reference legs of `bench.py` may import this package. The
@@ -36,7 +37,7 @@ def build(force: bool = False) -> str:
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
         tmp = _LIB + f".tmp{os.getpid()}"
         subprocess.check_call(["gcc", "-O2", "-std=c11", "-Wall", "-Wextra", "-shared",
-                               "-fPIC", "-o", tmp, _SRC])
+                               "-fPIC", "-o", tmp, _SRC, "-lm"])
         os.replace(tmp, _LIB)
     return _LIB
 
@@ -46,7 +47,7 @@ def build_mutant(mutant: int, outdir: str):
     return it loaded; see ORACLE_MUTANT in engram_oracle.c."""
     path = os.path.join(outdir, f"liboracle_mutant{mutant}.so")
     subprocess.check_call(["gcc", "-O2", "-std=c11", "-shared", "-fPIC",
-                           f"-DORACLE_MUTANT={int(mutant)}", "-o", path, _SRC])
+                           f"-DORACLE_MUTANT={int(mutant)}", "-o", path, _SRC, "-lm"])
     return _declare(ctypes.CDLL(path))
 
 
@@ -59,6 +60,13 @@ def _declare(L):
     L.oracle_gather.restype = ctypes.c_int
     L.oracle_backward.argtypes = [P, i64, P, ctypes.c_int, i32, P, P, P]
     L.oracle_backward.restype = ctypes.c_int
+    L.oracle_grouped_rms_norm.argtypes = [P, ctypes.c_int, i64, i32, i32, P, ctypes.c_int,
+                                          ctypes.c_double, P]
+    L.oracle_grouped_rms_norm.restype = ctypes.c_int
+    L.oracle_short_conv.argtypes = [P, ctypes.c_int, P, i32, i64, i32, i32, P, ctypes.c_double,
+                                    P, P, ctypes.c_int, i32, i32, ctypes.c_int, ctypes.c_int,
+                                    ctypes.c_int, P]
+    L.oracle_short_conv.restype = ctypes.c_int
     return L
 
 
@@ -129,3 +137,57 @@ def backward(idx, dout: np.ndarray, dtype: int):
         raise ValueError("oracle_backward: invalid arguments")
     U = int(nu[0])
     return uniq[:U].copy(), grads[:U].copy()
+
+
+def _raw(a, dtype):
+    """Contiguous raw buffer of `dtype` (F32: float32 values; BF16/F16: uint16
+    bit patterns, or float16 values for F16)."""
+    if a is None:
+        return None
+    a = np.ascontiguousarray(a)
+    if dtype == F32:
+        return np.ascontiguousarray(a, dtype=np.float32)
+    if a.dtype == np.float16:
+        return a.view(np.uint16)
+    assert a.dtype == np.uint16, "BF16/F16 buffers are passed as uint16 bit patterns"
+    return a
+
+
+def grouped_rms_norm(x, dtype, group, weight=None, wdtype=F32, eps=1e-6) -> np.ndarray:
+    """fp64 [rows, C] Gemma-style norm of every group of `group` features."""
+    xr = _raw(x, dtype)
+    rows, C = xr.shape
+    wr = _raw(weight, wdtype)
+    out = np.empty((rows, C), dtype=np.float64)
+    rc = lib().oracle_grouped_rms_norm(_ptr(xr), dtype, rows, C, group,
+                                       None if wr is None else _ptr(wr), wdtype, float(eps),
+                                       _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle_grouped_rms_norm: invalid arguments")
+    return out
+
+
+def short_conv(x, dtype, cu, conv_w, *, dilation, group=None, norm_w=None, eps=1e-6,
+               bias=None, wdtype=F32, norm=True, silu=True, residual=True) -> np.ndarray:
+    """fp64 [T, C] output of the PLE tail x + SiLU(conv(norm(x))) (each of
+    norm, SiLU and residual optional); conv_w is [C, K]."""
+    xr = _raw(x, dtype)
+    T, C = xr.shape
+    wr = _raw(conv_w, wdtype)
+    K = wr.shape[1]
+    nw, br = _raw(norm_w, wdtype), _raw(bias, wdtype)
+    if cu is None:
+        cu_arr, nseq, cu_p = None, 1, None
+    else:
+        cu_arr = np.ascontiguousarray(cu, dtype=np.int32)
+        nseq, cu_p = cu_arr.shape[0] - 1, _ptr(cu_arr)
+    out = np.empty((T, C), dtype=np.float64)
+    rc = lib().oracle_short_conv(_ptr(xr), dtype, cu_p, nseq, T, C,
+                                 int(group if group else C),
+                                 None if nw is None else _ptr(nw), float(eps), _ptr(wr),
+                                 None if br is None else _ptr(br), wdtype, K, int(dilation),
+                                 int(bool(norm)), int(bool(silu)), int(bool(residual)),
+                                 _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle_short_conv: invalid arguments")
+    return out

@@ -22,12 +22,23 @@
  *   - backward: one fp64 sum per distinct row over its lookups in ascending
  *     lookup order, rounded once to fp32; rows reported in ascending order.
  *
+ * The PLE section follows the same page's Qwen3_8_FlashNextPLELayer
+ * (norm_conv, conv1d with short_conv_dilation = ngram_size, _causal_short_conv
+ * with left zero history, init_weights' zero-start convolution) and the layers
+ * page's Qwen3_8_FlashNextGroupedRMSNorm (Gemma-style, additive scale that
+ * starts at zero, groups of group_size features). Readings taken there:
+ *   - norm_conv normalises the convolution's input;
+ *   - the convolution's history is zero before every start in cu_seqlens;
+ *   - the optional SiLU and residual follow the Engram paper the page cites
+ *     (output = x + SiLU(conv(norm(x)))); the page itself prints neither.
+ *
  * Parity of the hash against the released checkpoint is unpinned: the page
  * prints no worked example (see the tests for what does pin each function).
  */
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#include <math.h>
 
 /* ORACLE_MUTANT (tests only) plants one known mistake so the tests can show
  * that their pins catch it; the default build defines none. */
@@ -251,5 +262,110 @@ int oracle_backward(const int64_t *idx, int64_t n, const void *dout, int dtype,
     *num_unique = u;
     free(l);
     free(acc);
+    return ORACLE_OK;
+}
+
+/* -------------------------------------------------- PLE short convolution */
+
+/*
+ * Branch-local Gemma RMS norm (layers page, Qwen3_8_FlashNextGroupedRMSNorm):
+ * each row of C features is cut into C / G groups of G consecutive features
+ * (one HyperConnection branch each) and every group is normalised on its own,
+ *   n[c] = x[c] / sqrt(mean over the group of x^2 + eps) * (1 + w[c]),
+ * where w is the additive scale that starts at zero (weight NULL = zeros).
+ * All in fp64; out is fp64 [rows, C].
+ */
+int oracle_grouped_rms_norm(const void *x, int dtype, int64_t rows, int32_t C, int32_t G,
+                            const void *weight, int wdtype, double eps, double *out)
+{
+    if (rows < 0 || C <= 0 || G <= 0 || C % G != 0 || eps < 0.0)
+        return ORACLE_EINVAL;
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int32_t g0 = 0; g0 < C; g0 += G) {
+            double ss = 0.0;
+            for (int32_t c = g0; c < g0 + G; ++c) {
+                const double v = load_value(x, dtype, r * C + c);
+                ss += v * v;
+            }
+            double ms = ss / (double)G;
+            if (ORACLE_MUTANT == 9)
+                ms = ss / (double)C; /* mutant: mean over the whole row's width */
+            const double inv = ORACLE_MUTANT == 10 ? 1.0 / (sqrt(ms) + eps)
+                                                   : 1.0 / sqrt(ms + eps);
+            for (int32_t c = g0; c < g0 + G; ++c) {
+                const double w = weight ? load_value(weight, wdtype, c) : 0.0;
+                const double scale = ORACLE_MUTANT == 8 ? w : 1.0 + w;
+                out[r * C + c] = load_value(x, dtype, r * C + c) * inv * scale;
+            }
+        }
+    }
+    return ORACLE_OK;
+}
+
+/*
+ * The PLE layer's contextualising tail (engram page,
+ * Qwen3_8_FlashNextPLELayer: norm_conv, conv1d, _causal_short_conv), taken
+ * step by step over a [T, C] tensor of branch-flattened values:
+ *   1. n = grouped RMS norm of x with norm_w (when do_norm; else n = x);
+ *   2. causal depthwise convolution of width K and dilation dil with zero
+ *      history before each sequence start: for token t of sequence s,
+ *        y[t, c] = bias[c] + sum over k = 0 .. K-1 with t - k*dil >= cu[s] of
+ *                  conv_w[c, K-1-k] * n[t - k*dil, c]
+ *      (conv_w is [C, K] row-major, the [C, 1, K] weight of a depthwise
+ *      conv1d whose last tap meets the current token; bias NULL = zeros);
+ *   3. y = y * sigmoid(y) when do_silu;
+ *   4. y = y + x when do_residual.
+ * cu NULL means one sequence [0, T). out is fp64 [T, C].
+ */
+int oracle_short_conv(const void *x, int dtype, const int32_t *cu, int32_t nseq, int64_t T,
+                      int32_t C, int32_t G, const void *norm_w, double eps,
+                      const void *conv_w, const void *bias, int wdtype, int32_t K,
+                      int32_t dil, int do_norm, int do_silu, int do_residual, double *out)
+{
+    if (T < 0 || C <= 0 || K < 1 || dil < 1 || (do_norm && (G <= 0 || C % G != 0)))
+        return ORACLE_EINVAL;
+    if (cu && (nseq < 0 || cu[0] != 0 || cu[nseq] != T))
+        return ORACLE_EINVAL;
+    double *n = (double *)malloc(sizeof(double) * (size_t)(T * C > 0 ? T * C : 1));
+    if (!n)
+        return ORACLE_EINVAL;
+    if (do_norm) {
+        const int rc = oracle_grouped_rms_norm(x, dtype, T, C, G, norm_w, wdtype, eps, n);
+        if (rc != ORACLE_OK) {
+            free(n);
+            return rc;
+        }
+    } else {
+        for (int64_t i = 0; i < T * C; ++i)
+            n[i] = load_value(x, dtype, i);
+    }
+    const int32_t ns = cu ? nseq : 1;
+    for (int32_t s = 0; s < ns; ++s) {
+        int64_t begin = cu ? cu[s] : 0, end = cu ? cu[s + 1] : T;
+        if (begin > end)
+            continue;
+        if (ORACLE_MUTANT == 13)
+            begin = 0; /* mutant: history runs across sequence starts */
+        for (int64_t t = cu ? cu[s] : 0; t < end; ++t) {
+            for (int32_t c = 0; c < C; ++c) {
+                double y = bias ? load_value(bias, wdtype, c) : 0.0;
+                for (int32_t k = 0; k < K; ++k) {
+                    const int64_t step = ORACLE_MUTANT == 11 ? (int64_t)k * (dil + 1)
+                                                             : (int64_t)k * dil;
+                    const int64_t src = t - step;
+                    if (src < begin)
+                        break;
+                    const int32_t tap = ORACLE_MUTANT == 12 ? k : K - 1 - k;
+                    y += load_value(conv_w, wdtype, (int64_t)c * K + tap) * n[src * C + c];
+                }
+                if (do_silu)
+                    y = y / (1.0 + exp(-y));
+                if (do_residual)
+                    y += ORACLE_MUTANT == 14 ? n[t * C + c] : load_value(x, dtype, t * C + c);
+                out[t * C + c] = y;
+            }
+        }
+    }
+    free(n);
     return ORACLE_OK;
 }

@@ -2,9 +2,11 @@
 
 Each mutant is the oracle rebuilt with one known mistake (ORACLE_MUTANT in
 engram_oracle.c): a plausible slip in the hash (operator, reset position,
-multiplier pairing, remainder sign, sequence reset) or in the backward
-(accumulation precision, grouping). The pins of test_oracle_hash.py and
-test_oracle_gather_backward.py are run against each; at least one must fail.
+multiplier pairing, remainder sign, sequence reset), in the backward
+(accumulation precision, grouping) or in the PLE norm and convolution (scale,
+group width, epsilon, dilation, tap order, history reset, residual). The pins
+of test_oracle_hash.py, test_oracle_gather_backward.py and test_oracle_ple.py
+are run against each; at least one must fail.
 """
 
 import pytest
@@ -12,6 +14,7 @@ import pytest
 import oracle
 from tests import test_oracle_gather_backward as GB
 from tests import test_oracle_hash as TH
+from tests import test_oracle_ple as PL
 
 HASH_PINS = [
     TH.test_hand_worked_example,
@@ -29,6 +32,20 @@ BACKWARD_PINS = [
     lambda: GB.test_backward_per_head_mass_and_counts("tiny"),
 ]
 
+PLE_PINS = [
+    lambda: [PL.test_norm_matches_torch_rms_norm(g) for g in (4, 8, 16)],
+    PL.test_norm_constant_group_closed_form,
+    PL.test_norm_unit_rms_and_branch_scale_invariance,
+    PL.test_norm_zero_scale_is_plain_rms_norm,
+    lambda: [PL.test_conv_matches_torch_conv1d(K, d, cu) for K, d in ((4, 3), (3, 5))
+             for cu in (None, [0, 13, 13, 40])],
+    PL.test_conv_impulse_response,
+    PL.test_full_tail_matches_torch_chain,
+    PL.test_zero_start_convolution_leaves_the_residual,
+    PL.test_causal_branch_local_and_sequence_local,
+    PL.test_sequences_are_independent,
+]
+
 MUTANTS = {
     1: ("add instead of xor", HASH_PINS),
     2: ("reset before EOS instead of after", HASH_PINS),
@@ -37,6 +54,13 @@ MUTANTS = {
     5: ("no reset at cu_seqlens starts", HASH_PINS),
     6: ("fp32 accumulation", BACKWARD_PINS),
     7: ("adjacent rows merged", BACKWARD_PINS),
+    8: ("norm scale w instead of 1 + w", PLE_PINS),
+    9: ("norm mean over the whole row", PLE_PINS),
+    10: ("eps added after the square root", PLE_PINS),
+    11: ("dilation off by one", PLE_PINS),
+    12: ("conv taps reversed", PLE_PINS),
+    13: ("conv history crosses sequence starts", PLE_PINS),
+    14: ("residual of the normalised input", PLE_PINS),
 }
 
 
