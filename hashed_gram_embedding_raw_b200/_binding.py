@@ -20,6 +20,8 @@ LIB_PATH = os.path.join(_PKG, "_lib", "libengram_b200.so")
 ENGRAM_OK, ENGRAM_EINVAL, ENGRAM_ENOSPC, ENGRAM_ECUDA = 0, 1, 2, 3
 ENGRAM_F32, ENGRAM_BF16, ENGRAM_F16 = 0, 1, 2
 ENGRAM_DEVERR_ROW_RANGE, ENGRAM_DEVERR_CU_SEQLENS, ENGRAM_DEVERR_SORT_TIMEOUT = 1, 2, 4
+ENGRAM_DEVERR_COPY_TIMEOUT = 8
+ENGRAM_CONV_NORM, ENGRAM_CONV_SILU, ENGRAM_CONV_RESIDUAL = 1, 2, 4
 ENGRAM_MAX_NGRAM, ENGRAM_MAX_HEADS = 4, 32
 
 _DTYPE_CODE = {torch.float32: ENGRAM_F32, torch.bfloat16: ENGRAM_BF16,
@@ -31,6 +33,7 @@ EXPORTED = (
     "engram_backward_reduce", "engram_get_device_error", "engram_status_string",
     "engram_abi_version", "engram_params_size", "engram_launch_count",
     "engram_host_floor_mod", "engram_backward_noalloc", "engram_hash_gather_slice",
+    "engram_ple_short_conv", "engram_grouped_rms_norm",
 )
 
 ENGRAM_NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -61,6 +64,20 @@ class EngramParams(ctypes.Structure):
     @property
     def heads(self) -> int:
         return (self.ngram_size - 1) * self.heads_per_ngram
+
+
+class ConvParams(ctypes.Structure):
+    """Mirror of engram_conv_params_t."""
+    _fields_ = [
+        ("channels", ctypes.c_int32),
+        ("group_size", ctypes.c_int32),
+        ("kernel_size", ctypes.c_int32),
+        ("dilation", ctypes.c_int32),
+        ("eps", ctypes.c_float),
+        ("flags", ctypes.c_uint32),
+        ("weight_dtype", ctypes.c_int32),
+        ("reserved", ctypes.c_int32),
+    ]
 
 
 def make_params(cfg: dict) -> EngramParams:
@@ -105,6 +122,8 @@ def _load():
         "engram_host_floor_mod": [i64, i64, ctypes.POINTER(ctypes.c_int)],
         "engram_backward_noalloc": [P, i64, i64, i32, P, i32, P, P, P, P],
         "engram_hash_gather_slice": [P, P, P, i32, i64, i64, i64, i64, P, i32, P, P, P],
+        "engram_ple_short_conv": [P, P, i32, P, i32, i64, P, P, P, P, i32, P],
+        "engram_grouped_rms_norm": [P, i32, i64, i32, i32, P, i32, ctypes.c_float, P, i32, P],
     }
     for name, args in sig.items():
         fn = getattr(L, name)
@@ -346,6 +365,72 @@ def engram_backward_reduce(n: int, table_rows: int, dout: torch.Tensor, uniq_row
                                       _ptr(uniq_rows), _ptr(row_grads), _ptr(num_unique),
                                       _ptr(workspace), workspace.numel(), _stream(stream)),
            "engram_backward_reduce")
+
+
+# ----------------------------------------------------------- PLE layer tail
+
+def _out_like(x: torch.Tensor, out, out_dtype):
+    dt = x.dtype if out_dtype is None else out_dtype
+    if out is None:
+        out = torch.empty(x.shape, dtype=dt, device=x.device)
+    _cuda(out, "out", dt)
+    if out.shape != x.shape:
+        raise ValueError("out must have the shape of x")
+    return out
+
+
+def engram_ple_short_conv(x: torch.Tensor, conv_weight: torch.Tensor, *, dilation: int,
+                          group_size: int, cu_seqlens=None, norm_weight=None, conv_bias=None,
+                          eps: float = 1e-6, norm: bool = True, silu: bool = True,
+                          residual: bool = True, out=None, out_dtype=None,
+                          stream=None) -> torch.Tensor:
+    """PLE tail over x [T, C]: x + SiLU(causal depthwise conv(grouped RMS norm(x)))
+    with each of norm, SiLU and residual optional; conv_weight is [C, K] (or
+    the conv1d layout [C, 1, K]); all weights share one dtype."""
+    _cuda(x, "x")
+    if x.dim() != 2:
+        raise ValueError("x must be [T, C]")
+    T, C = x.shape
+    w = conv_weight.reshape(C, -1) if conv_weight.dim() == 3 else conv_weight
+    _cuda(w, "conv_weight")
+    if w.shape[0] != C:
+        raise ValueError("conv_weight must be [C, K]")
+    for name, t in (("norm_weight", norm_weight), ("conv_bias", conv_bias)):
+        if t is not None:
+            _cuda(t, name, w.dtype)
+            if t.numel() != C:
+                raise ValueError(f"{name} must hold C elements")
+    cu, nseq = _cu_args(cu_seqlens)
+    out = _out_like(x, out, out_dtype)
+    p = ConvParams(C, int(group_size), w.shape[1], int(dilation), float(eps),
+                   (ENGRAM_CONV_NORM if norm else 0) | (ENGRAM_CONV_SILU if silu else 0)
+                   | (ENGRAM_CONV_RESIDUAL if residual else 0), _dtype_code(w), 0)
+    _check(lib.engram_ple_short_conv(ctypes.byref(p), _ptr(x), _dtype_code(x), _ptr(cu), nseq,
+                                     T, _ptr(norm_weight), _ptr(w), _ptr(conv_bias), _ptr(out),
+                                     _dtype_code(out), _stream(stream)),
+           "engram_ple_short_conv")
+    return out
+
+
+def engram_grouped_rms_norm(x: torch.Tensor, group_size: int, weight=None, eps: float = 1e-6,
+                            out=None, out_dtype=None, stream=None) -> torch.Tensor:
+    """Branch-local Gemma RMS norm of x [..., C] over groups of group_size
+    features, scale (1 + weight); out may be x itself (in place)."""
+    _cuda(x, "x")
+    C = x.shape[-1]
+    rows = x.numel() // C if C else 0
+    wdt = ENGRAM_F32
+    if weight is not None:
+        _cuda(weight, "weight")
+        if weight.numel() != C:
+            raise ValueError("weight must hold C elements")
+        wdt = _dtype_code(weight)
+    out = _out_like(x, out, out_dtype)
+    _check(lib.engram_grouped_rms_norm(_ptr(x), _dtype_code(x), rows, C, int(group_size),
+                                       _ptr(weight), wdt, float(eps), _ptr(out),
+                                       _dtype_code(out), _stream(stream)),
+           "engram_grouped_rms_norm")
+    return out
 
 
 # -------------------------------------------------------------------- misc

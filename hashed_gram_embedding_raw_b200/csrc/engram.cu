@@ -7,9 +7,11 @@
 // hash_gather.cuh and backward.cuh.
 #include <atomic>
 #include <climits>
+#include <cmath>
 #include <cstring>
 #include <map>
 #include <mutex>
+#include <set>
 #include <tuple>
 
 #include "engram.h"
@@ -17,6 +19,7 @@
 #include "backward.cuh"
 #include "common.cuh"
 #include "hash_gather.cuh"
+#include "ple_conv.cuh"
 
 using namespace engram;
 
@@ -628,6 +631,205 @@ int64_t engram_host_floor_mod(int64_t a, int64_t m, int *status)
     if (status)
         *status = ENGRAM_OK;
     return floor_mod(a, (uint64_t)m, UINT64_MAX / (uint64_t)m);
+}
+
+} // extern "C"
+
+// ------------------------------------------------------ PLE layer tail
+
+namespace {
+
+struct ConvPlan {
+    ple::ConvArgs a;
+    size_t smem = 0;
+    int grid = 0, threads = 0;
+};
+
+bool overlaps(const void *a, size_t na, const void *b, size_t nb)
+{
+    const uintptr_t x = (uintptr_t)a, y = (uintptr_t)b;
+    return na > 0 && nb > 0 && x < y + nb && y < x + na;
+}
+
+// Checks the shape (host only) and picks the block layout: the landing ring
+// as deep as shared memory allows after the private rings of the normalised
+// history. conv_grid adds the grid: one block per (branch, range), sms /
+// branches blocks per branch.
+int conv_plan(const engram_conv_params_t *p, int32_t dtype, int32_t out_dtype, int64_t T,
+              ConvPlan *P)
+{
+    if (p == nullptr)
+        return ENGRAM_EINVAL;
+    const int eb = elem_bytes(dtype);
+    if (eb == 0 || elem_bytes(out_dtype) == 0 || elem_bytes(p->weight_dtype) == 0 ||
+        (out_dtype != dtype && out_dtype != ENGRAM_F32))
+        return ENGRAM_EINVAL;
+    const int C = p->channels, G = p->group_size, K = p->kernel_size, d = p->dilation;
+    if (C < 1 || G < 1 || C % G != 0 || G % ple::kChan != 0 ||
+        G / ple::kChan > ple::kMaxThreads)
+        return ENGRAM_EINVAL;
+    if (K < 1 || K > ple::kMaxTaps || d < 1 || d > 4096 || p->reserved != 0)
+        return ENGRAM_EINVAL;
+    if (!std::isfinite(p->eps) || p->eps < 0.f || (p->flags & ~7u) != 0)
+        return ENGRAM_EINVAL;
+    if (T < 0 || T > INT32_MAX)
+        return ENGRAM_EINVAL;
+    const int halo = (K - 1) * d;
+    const int nth = G / ple::kChan;
+    const int pitch = (G * eb + 127) / 128 * 128;
+    const int norm_slots = halo + ple::kRows;
+    int raw = ple::kMaxRawSlots;
+    while (raw >= ple::kMinRawSlots &&
+           ple::smem_bytes(raw, pitch, norm_slots, nth) > ple::kSmemLimit)
+        --raw;
+    if (raw < ple::kMinRawSlots)
+        return ENGRAM_EINVAL;
+    ple::ConvArgs &a = P->a;
+    std::memset(&a, 0, sizeof(a));
+    a.T = T;
+    a.C = C;
+    a.G = G;
+    a.nth = nth;
+    a.wdtype = p->weight_dtype;
+    a.eps = p->eps;
+    a.inv_G = 1.f / (float)G;
+    a.K = K;
+    a.dil = d;
+    a.halo = halo;
+    a.raw_slots = raw;
+    a.raw_pitch = pitch;
+    a.norm_slots = norm_slots;
+    a.flags = p->flags;
+    P->threads = (nth + 31) / 32 * 32;
+    P->smem = ple::smem_bytes(raw, pitch, norm_slots, nth);
+    return ENGRAM_OK;
+}
+
+// Grid of a checked plan on the current device (T > 0).
+int conv_grid(ConvPlan *P)
+{
+    int sms = 0;
+    ENGRAM_TRY(device_sms(&sms));
+    const int groups = P->a.C / P->a.G;
+    int64_t bpg = std::max(1, sms / groups);
+    bpg = std::min<int64_t>(bpg, std::max<int64_t>(1, ceil_div(P->a.T, 64)));
+    if ((int64_t)groups * bpg > INT32_MAX)
+        return ENGRAM_EINVAL;
+    P->a.bpg = (int32_t)bpg;
+    P->grid = (int)(groups * bpg);
+    return ENGRAM_OK;
+}
+
+// Raises the dynamic shared-memory limit of `fn` to the block maximum, once
+// per device (the limit only gates launches; it reserves nothing).
+template <typename F>
+int allow_smem(F fn)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return ENGRAM_ECUDA;
+    static std::mutex mu;
+    static std::set<std::pair<const void *, int>> done;
+    const auto key = std::make_pair((const void *)fn, dev);
+    std::lock_guard<std::mutex> lock(mu);
+    if (done.count(key) == 0) {
+        if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)ple::kSmemLimit) != cudaSuccess)
+            return ENGRAM_ECUDA;
+        done.insert(key);
+    }
+    return ENGRAM_OK;
+}
+
+template <typename XT, typename OT>
+int launch_conv_t(const ConvPlan &P, cudaStream_t s)
+{
+    auto fn = P.a.K == 4   ? ple::short_conv_kernel<XT, OT, 4>
+              : P.a.K == 1 ? ple::short_conv_kernel<XT, OT, 1>
+                           : ple::short_conv_kernel<XT, OT, 0>;
+    ENGRAM_TRY(allow_smem(fn));
+    fn<<<P.grid, P.threads, P.smem, s>>>(P.a);
+    return after_launch();
+}
+
+int launch_conv(ConvPlan &P, int32_t dtype, int32_t out_dtype, cudaStream_t s)
+{
+    ENGRAM_TRY(conv_grid(&P));
+    const bool f32_out = out_dtype == ENGRAM_F32;
+    switch (dtype) {
+    case ENGRAM_F32:
+        return launch_conv_t<float, float>(P, s);
+    case ENGRAM_BF16:
+        return f32_out ? launch_conv_t<__nv_bfloat16, float>(P, s)
+                       : launch_conv_t<__nv_bfloat16, __nv_bfloat16>(P, s);
+    default:
+        return f32_out ? launch_conv_t<__half, float>(P, s) : launch_conv_t<__half, __half>(P, s);
+    }
+}
+
+} // namespace
+
+extern "C" {
+
+int engram_ple_short_conv(const engram_conv_params_t *params, const void *x, int32_t dtype,
+                          const int32_t *cu_seqlens, int32_t nseq, int64_t T,
+                          const void *norm_weight, const void *conv_weight,
+                          const void *conv_bias, void *out, int32_t out_dtype,
+                          engram_stream_t stream)
+{
+    ConvPlan P;
+    ENGRAM_TRY(conv_plan(params, dtype, out_dtype, T, &P));
+    if (cu_seqlens != nullptr && nseq < 1)
+        return ENGRAM_EINVAL;
+    if (T == 0)
+        return ENGRAM_OK;
+    if (x == nullptr || out == nullptr || conv_weight == nullptr || !aligned16(x) ||
+        !aligned16(out))
+        return ENGRAM_EINVAL;
+    const size_t n = (size_t)T * params->channels;
+    if (overlaps(x, n * elem_bytes(dtype), out, n * elem_bytes(out_dtype)))
+        return ENGRAM_EINVAL;
+    P.a.x = x;
+    P.a.out = out;
+    P.a.cu = cu_seqlens;
+    P.a.nseq = cu_seqlens != nullptr ? nseq : 1;
+    P.a.norm_w = norm_weight;
+    P.a.conv_w = conv_weight;
+    P.a.bias = conv_bias;
+    return launch_conv(P, dtype, out_dtype, (cudaStream_t)stream);
+}
+
+int engram_grouped_rms_norm(const void *x, int32_t dtype, int64_t rows, int32_t channels,
+                            int32_t group_size, const void *weight, int32_t weight_dtype,
+                            float eps, void *out, int32_t out_dtype, engram_stream_t stream)
+{
+    engram_conv_params_t p;
+    std::memset(&p, 0, sizeof(p));
+    p.channels = channels;
+    p.group_size = group_size;
+    p.kernel_size = 1;
+    p.dilation = 1;
+    p.eps = eps;
+    p.flags = ENGRAM_CONV_NORM;
+    p.weight_dtype = weight_dtype;
+    ConvPlan P;
+    ENGRAM_TRY(conv_plan(&p, dtype, out_dtype, rows, &P));
+    if (rows == 0)
+        return ENGRAM_OK;
+    if (x == nullptr || out == nullptr || !aligned16(x) || !aligned16(out))
+        return ENGRAM_EINVAL;
+    // in place is allowed: a block writes a row only after reading it, and no
+    // other block reads that row
+    const size_t n = (size_t)rows * channels;
+    if (out != x && overlaps(x, n * elem_bytes(dtype), out, n * elem_bytes(out_dtype)))
+        return ENGRAM_EINVAL;
+    if (out == x && out_dtype != dtype)
+        return ENGRAM_EINVAL;
+    P.a.x = x;
+    P.a.out = out;
+    P.a.nseq = 1;
+    P.a.norm_w = weight;
+    return launch_conv(P, dtype, out_dtype, (cudaStream_t)stream);
 }
 
 } // extern "C"

@@ -35,35 +35,6 @@ struct HashArgs {
 
 constexpr int kHashThreads = 256;
 
-// Largest s < nseq with cu[s] <= t (cu[0] = 0 <= t for well-formed bounds).
-__device__ __forceinline__ int32_t find_sequence(const int32_t *__restrict__ cu, int32_t nseq,
-                                                 int64_t t)
-{
-    int32_t lo = 0, hi = nseq - 1;
-    while (lo < hi) {
-        const int32_t mid = (lo + hi + 1) >> 1;
-        if (__ldg(cu + mid) <= t)
-            lo = mid;
-        else
-            hi = mid - 1;
-    }
-    return lo;
-}
-
-// Flags malformed cu_seqlens (not 0 .. T, or decreasing). Grid-strided.
-__device__ __forceinline__ void check_cu_seqlens(const int32_t *__restrict__ cu, int32_t nseq,
-                                                 int64_t T)
-{
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i <= nseq; i += stride) {
-        const int64_t c = __ldg(cu + i);
-        const bool bad = (i == 0 && c != 0) || (i == nseq && c != T) ||
-                         (i < nseq && c > __ldg(cu + i + 1));
-        if (bad)
-            raise_device_error(ENGRAM_DEVERR_CU_SEQLENS);
-    }
-}
-
 // A slice of the stream (_forward_global_slice): positions [start, start+len)
 // of every row of `row` tokens. Logical token L of the slice is stream
 // position (L / len) * row + start + L % len; the identity map has row = len

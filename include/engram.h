@@ -63,6 +63,8 @@ extern "C" {
 #define ENGRAM_DEVERR_CU_SEQLENS 2u  /* cu_seqlens not non-decreasing from 0 to T */
 #define ENGRAM_DEVERR_SORT_TIMEOUT 4u /* the backward sort's grid barrier gave up waiting
                                          (results of that call are invalid) */
+#define ENGRAM_DEVERR_COPY_TIMEOUT 8u /* a bulk copy into shared memory did not complete in
+                                         time (results of that call are invalid) */
 /* Same type as cudaStream_t, without requiring the CUDA headers. */
 typedef struct CUstream_st *engram_stream_t;
 
@@ -238,6 +240,79 @@ ENGRAM_API int engram_backward_noalloc(const int32_t *idx, int64_t n, int64_t ta
                                        int32_t dim, const void *dout, int32_t dtype,
                                        int32_t *uniq_rows, float *row_grads,
                                        int32_t *num_unique, engram_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * PLE layer tail: the consumer of the embedding inside
+ * Qwen3_8_FlashNextPLELayer (engram page), after its key/value projections.
+ * The page lists a branch-local Gemma RMS norm (norm_conv, and norm_key /
+ * norm_query of the same kind: Qwen3_8_FlashNextGroupedRMSNorm, layers page)
+ * and a causal depthwise convolution of width conv_kernel_size = 4 and
+ * dilation short_conv_dilation = ngram_size = 3 with zero history
+ * (_causal_short_conv; its context-parallel halo is (4 - 1) * 3 = 9 tokens).
+ * The page prints neither an activation nor a residual for the convolution;
+ * the Engram paper it cites applies x + SiLU(conv(norm(x))), which the
+ * ENGRAM_CONV_* flags select step by step.
+ * ------------------------------------------------------------------------ */
+
+#define ENGRAM_CONV_NORM 1u     /* normalise each branch slice before the convolution */
+#define ENGRAM_CONV_SILU 2u     /* y * sigmoid(y) after the convolution */
+#define ENGRAM_CONV_RESIDUAL 4u /* add the (unnormalised) input */
+
+typedef struct engram_conv_params {
+    int32_t channels;     /* C = hc_count * hidden_size (page: 4 * 2560) */
+    int32_t group_size;   /* G = hidden_size: features normalised together; C % G == 0,
+                             G % 8 == 0, G <= 4096 */
+    int32_t kernel_size;  /* K, 1 .. 8 (page: 4) */
+    int32_t dilation;     /* d >= 1 (page: ngram_size = 3) */
+    float eps;            /* rms_norm_eps (page default 1e-6), >= 0 */
+    uint32_t flags;       /* ENGRAM_CONV_* bits */
+    int32_t weight_dtype; /* ENGRAM_F32 | ENGRAM_BF16 | ENGRAM_F16 of the weights */
+    int32_t reserved;     /* must be 0 */
+} engram_conv_params_t;
+
+/*
+ * engram_ple_short_conv -- over x = [T, C] (C / G branch slices of G
+ * features per token), for every token t of sequence s and channel c:
+ *   n[t, c] = x[t, c] * rsqrt(mean over c's slice of x[t, .]^2 + eps)
+ *             * (1 + norm_weight[c])        (ENGRAM_CONV_NORM; else n = x)
+ *   y[t, c] = conv_bias[c] + sum over k < K with t - k*d >= cu_seqlens[s] of
+ *             conv_weight[c, K - 1 - k] * n[t - k*d, c]
+ *   out     = y * sigmoid(y) (ENGRAM_CONV_SILU), then + x (ENGRAM_CONV_RESIDUAL)
+ * computed in fp32 and rounded once to out_dtype.
+ *   x           device, [T, C] of dtype (F32 | BF16 | F16), 16-byte aligned
+ *   cu_seqlens  device, int32 [nseq + 1] as for engram_hash (NULL = one
+ *               sequence): the convolution's history is zero before each start
+ *   norm_weight device, [C] of weight_dtype (NULL = zeros; read only with
+ *               ENGRAM_CONV_NORM) -- the additive Gemma scale
+ *   conv_weight device, [C, K] of weight_dtype (the [C, 1, K] depthwise
+ *               conv1d weight; its last tap meets the current token)
+ *   conv_bias   device, [C] of weight_dtype, or NULL
+ *   out         device, [T, C] of out_dtype (dtype or ENGRAM_F32), 16-byte
+ *               aligned, not overlapping x
+ * Limits (else ENGRAM_EINVAL): those of engram_conv_params_t and
+ * 4 * G * ((K - 1) * d + 4) + 8 * G * sizeof(dtype) + 2 KB <= 227 KB of shared
+ * memory per block (the page's shape, G = 2560, K = 4, d = 3: 133 KB + ring).
+ */
+ENGRAM_API int engram_ple_short_conv(const engram_conv_params_t *params, const void *x,
+                                     int32_t dtype, const int32_t *cu_seqlens, int32_t nseq,
+                                     int64_t T, const void *norm_weight,
+                                     const void *conv_weight, const void *conv_bias,
+                                     void *out, int32_t out_dtype, engram_stream_t stream);
+
+/*
+ * engram_grouped_rms_norm -- Qwen3_8_FlashNextGroupedRMSNorm.forward over
+ * `rows` rows of `channels` features: every group of group_size consecutive
+ * features is normalised on its own,
+ *   out[r, c] = x[r, c] * rsqrt(mean over c's group of x[r, .]^2 + eps)
+ *               * (1 + weight[c])
+ * in fp32, rounded once to out_dtype (dtype or ENGRAM_F32). weight [channels]
+ * of weight_dtype, NULL = zeros (the page's reset value). Same layout limits
+ * as engram_ple_short_conv with K = 1.
+ */
+ENGRAM_API int engram_grouped_rms_norm(const void *x, int32_t dtype, int64_t rows,
+                                       int32_t channels, int32_t group_size,
+                                       const void *weight, int32_t weight_dtype, float eps,
+                                       void *out, int32_t out_dtype, engram_stream_t stream);
 
 /*
  * engram_get_device_error -- copy the current device's error word

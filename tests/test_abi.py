@@ -139,6 +139,47 @@ def test_host_rejects_bad_gather_and_backward_args(E):
     assert L.engram_backward_workspace_size(10, 100, 160, None) == E.ENGRAM_EINVAL
 
 
+def test_host_rejects_bad_conv_args(E):
+    L = E.lib
+    al, al2, mis = ctypes.c_void_p(256), ctypes.c_void_p(1 << 30), ctypes.c_void_p(264)
+
+    def params(**kw):
+        base = dict(channels=10240, group_size=2560, kernel_size=4, dilation=3, eps=1e-6,
+                    flags=7, weight_dtype=1, reserved=0)
+        base.update(kw)
+        return E.ConvParams(**base)
+
+    def conv(p, x=al, dtype=1, cu=None, nseq=1, T=100, out=al2, out_dtype=1):
+        return L.engram_ple_short_conv(ctypes.byref(p), x, dtype, cu, nseq, T, None, al, None,
+                                       out, out_dtype, None)
+
+    for bad in (dict(group_size=12), dict(group_size=3000), dict(channels=7680 + 100),
+                dict(group_size=8192, channels=8192), dict(kernel_size=0),
+                dict(kernel_size=9), dict(dilation=0), dict(eps=-1.0),
+                dict(eps=float("nan")), dict(flags=8), dict(weight_dtype=5), dict(reserved=1),
+                dict(kernel_size=8, dilation=4096)):
+        assert conv(params(**bad)) == E.ENGRAM_EINVAL, bad
+    p = params()
+    assert L.engram_ple_short_conv(None, al, 1, None, 1, 100, None, al, None, al2, 1,
+                                   None) == E.ENGRAM_EINVAL
+    assert conv(p, dtype=7) == E.ENGRAM_EINVAL
+    assert conv(p, out_dtype=2) == E.ENGRAM_EINVAL          # bf16 in, f16 out
+    assert conv(p, dtype=0, out_dtype=1) == E.ENGRAM_EINVAL  # f32 in, bf16 out
+    assert conv(p, T=-1) == E.ENGRAM_EINVAL
+    assert conv(p, cu=al, nseq=0) == E.ENGRAM_EINVAL
+    assert conv(p, x=mis) == E.ENGRAM_EINVAL
+    assert conv(p, out=mis) == E.ENGRAM_EINVAL
+    assert conv(p, x=None) == E.ENGRAM_EINVAL
+    assert conv(p, out=ctypes.c_void_p(256 + 4096)) == E.ENGRAM_EINVAL  # overlaps x
+    assert conv(p, T=0, x=None, out=None) == E.ENGRAM_OK                # empty: no-op
+    # the norm alone: groups must divide the row, in place needs one dtype
+    N = L.engram_grouped_rms_norm
+    assert N(al, 1, 10, 100, 30, None, 0, 1e-6, al2, 1, None) == E.ENGRAM_EINVAL
+    assert N(al, 1, 10, 96, 0, None, 0, 1e-6, al2, 1, None) == E.ENGRAM_EINVAL
+    assert N(al, 1, 10, 96, 32, None, 0, 1e-6, al, 0, None) == E.ENGRAM_EINVAL
+    assert N(al, 1, 0, 96, 32, None, 0, 1e-6, al, 1, None) == E.ENGRAM_OK
+
+
 def test_package_import_fails_loudly_without_library(tmp_path):
     # a copy of the binding pointed at a directory with no library must raise
     import importlib.util

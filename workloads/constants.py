@@ -33,6 +33,13 @@ EMBEDDING_DIM = 160            # row width of the [320001536, 160] table
 INITIALIZER_RANGE = 0.02       # EngramTableConfig default std
 TOKENIZER_VOCAB = 248320       # raw token ID range used by the workloads
 
+# PLE layer (engram page, Qwen3_8_FlashNextPLELayer; model overview page,
+# Architecture: four persistent HyperConnection streams of width 2,560).
+HC_COUNT = 4                   # HyperConnection branches
+HIDDEN_SIZE = 2560             # width of one branch (the norm group)
+PLE_CONV_KERNEL = 4            # conv_kernel_size default
+PLE_RMS_EPS = 1e-6             # rms_norm_eps default
+
 # Printed prefix of the truncated tuples.
 PRINTED_VOCAB_SIZES = (20000003, 20000023, 20000033, 20000047,
                        20000059, 20000063, 20000069, 20000077)

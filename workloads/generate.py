@@ -216,3 +216,67 @@ def host_dout(name: str, n_lookups: int, dim: int, dtype: str, seed_offset: int 
     g.manual_seed(4000 + w.seed + seed_offset)
     tdt = {"f32": torch.float32, "bf16": torch.bfloat16, "f16": torch.float16}[dtype]
     return torch.randn(n_lookups, dim, generator=g, dtype=torch.float32).to(tdt)
+
+
+# ------------------------------------------------------------ PLE layer tail
+
+@dataclasses.dataclass(frozen=True)
+class PleShape:
+    """Shape of the PLE convolution tail: T tokens of C = branches * G channels."""
+    name: str
+    seed: int
+    batch: int          # rows of the [batch, seq_len] token batch (cu_seqlens per row)
+    seq_len: int
+    branches: int       # hc_count
+    group: int          # hidden_size, features normalised together
+    kernel: int         # conv_kernel_size
+    dilation: int       # short_conv_dilation = ngram_size
+    dtype: str
+    description: str = ""
+
+    @property
+    def tokens(self) -> int:
+        return self.batch * self.seq_len
+
+    @property
+    def channels(self) -> int:
+        return self.branches * self.group
+
+
+PLE_SHAPES = {
+    "ple_small": PleShape(
+        "ple_small", 10, 3, 700, 4, 256, C.PLE_CONV_KERNEL, C.NGRAM_SIZE, "bf16",
+        "3 x 700 tokens, 4 branches of 256 channels, kernel 4, dilation 3"),
+    "ple_full": PleShape(
+        "ple_full", 11, 16, 4096, C.HC_COUNT, C.HIDDEN_SIZE, C.PLE_CONV_KERNEL, C.NGRAM_SIZE,
+        "bf16",
+        "16 x 4,096 tokens (the full workload's batch), 4 HyperConnection branches "
+        "of 2,560 channels (C = 10,240), kernel 4, dilation 3, bf16"),
+}
+
+
+def ple_inputs(T: int, channels: int, kernel: int, seed: int, dtype: str = "bf16"):
+    """Host inputs of the PLE tail: x [T, C] ~ N(0, 1), norm scale [C] ~
+    N(0, 0.1^2), conv weight [C, K] ~ N(0, 0.5^2), bias [C] ~ N(0, 0.1^2).
+
+    Returns float32 arrays for "f32", else uint16 bit patterns of the dtype
+    (rounded to nearest even by torch)."""
+    import torch
+    g = torch.Generator().manual_seed(5000 + int(seed))
+    x = torch.randn((T, channels), generator=g, dtype=torch.float32)
+    nw = 0.1 * torch.randn(channels, generator=g, dtype=torch.float32)
+    w = 0.5 * torch.randn((channels, kernel), generator=g, dtype=torch.float32)
+    b = 0.1 * torch.randn(channels, generator=g, dtype=torch.float32)
+
+    def cast(t):
+        if dtype == "f32":
+            return t.numpy()
+        tt = torch.bfloat16 if dtype == "bf16" else torch.float16
+        return t.to(tt).view(torch.int16).numpy().view(np.uint16)
+
+    return cast(x), cast(nw), cast(w), cast(b)
+
+
+def row_bounds(batch: int, seq_len: int) -> np.ndarray:
+    """cu_seqlens of a [batch, seq_len] batch: 0, S, 2S, ..., batch * S."""
+    return (np.arange(batch + 1, dtype=np.int64) * seq_len).astype(np.int32)
