@@ -7,6 +7,7 @@ gradients) over one batch of the named workload, all inputs resident in HBM.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload full]
     python bench.py --impl reference ...   # the CPU oracle, timed on this host
+    python bench.py --stage ple ...        # the PLE tail kernel on its own workload
 
 Multi-GPU (torchrun, one rank per GPU): every rank holds its own table
 replica and processes its own batch; no data-path collective exists, so the
@@ -215,24 +216,29 @@ def run_reference(args):
     if rank != 0:
         return 0
     name = args.workload
+    ple = args.stage == "ple"
+    run = (lambda S: ple_oracle_run(S)) if ple else (lambda S: oracle_run(name, S))
     # calibrate, then size each step's sample so W + K steps take ~2 minutes
-    rate, _, _, _ = oracle_run(name, 4096)
+    rate, _, _, _ = run(256 if ple else 4096)
     budget = float(os.environ.get("ENGRAM_REFERENCE_BUDGET_S", "120"))
     S = int(max(256, min(65536 * 4, rate * budget / max(1, args.steps + args.warmup))))
     for _ in range(args.warmup):
-        oracle_run(name, S)
+        run(S)
     times = []
     for _ in range(args.steps):
-        _, el, _, desc = oracle_run(name, S)
+        _, el, _, desc = run(S)
         times.append(el)
     total = sum(times)
     value = S * len(times) / total
+    if ple:
+        name = "ple_full"
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "impl": "reference", "metric": PLE_METRIC if ple else METRIC, "value": value,
+        "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * total / len(times), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "int64/f64", "data": "synthetic",
-        "config": {"workload": name, "tokens_per_step": S},
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64" if ple else "int64/f64",
+        "data": "synthetic", "config": {"workload": name, "tokens_per_step": S},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
                          "sample": desc},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -476,6 +482,172 @@ def run_ours(args):
     return 0
 
 
+# --------------------------------------------------------- PLE tail stage
+
+PLE_METRIC = ("PLE tail tokens/s (grouped RMS norm + causal depthwise conv + SiLU + residual "
+              "over hc_count x hidden channels); achieved HBM GB/s vs peak")
+
+
+def ple_oracle_run(S: int, reps_seconds: float = 0.0, max_reps: int = 1):
+    """Time the CPU oracle of the PLE tail on S tokens (one sequence) of the
+    page's channel shape. Returns (tokens/s, seconds, reps, description)."""
+    import oracle
+    from workloads import PLE_SHAPES, ple_inputs
+
+    s = PLE_SHAPES["ple_full"]
+    x, nw, w, b = ple_inputs(S, s.channels, s.kernel, s.seed, s.dtype)
+    oracle.lib()
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        out = oracle.short_conv(x, oracle.BF16, None, w, dilation=s.dilation, group=s.group,
+                                norm_w=nw, bias=b, wdtype=oracle.BF16)
+        reps += 1
+        el = time.perf_counter() - t0
+        if reps >= max_reps or el >= reps_seconds:
+            break
+    assert out.shape == (S, s.channels)
+    desc = (f"{S} tokens x {s.channels} channels (one sequence, the page's 4 x 2,560 "
+            f"branches, kernel {s.kernel}, dilation {s.dilation}) x {reps} rep(s); "
+            f"single-threaded C oracle in fp64")
+    return S * reps / el, el, reps, desc
+
+
+def run_ple(args):
+    """--stage ple: engram_ple_short_conv on the page's PLE shape at the full
+    workload's batch (16 x 4,096 tokens, C = 4 x 2,560 bf16)."""
+    import torch
+
+    import hashed_gram_embedding_raw_b200 as E
+    from workloads import PLE_SHAPES, ple_inputs, row_bounds
+
+    rank, local_rank, world = rank_env()
+    assert torch.cuda.is_available(), "bench.py needs a CUDA device"
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", device_id=device,
+                                timeout=datetime.timedelta(seconds=300))
+    s = PLE_SHAPES["ple_full"]
+    T, C, G, K, d = s.tokens, s.channels, s.group, s.kernel, s.dilation
+    g = torch.Generator(device=device).manual_seed(5000 + s.seed)
+    x = torch.randn((T, C), generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+    _, nw_h, w_h, b_h = ple_inputs(1, C, K, s.seed, s.dtype)
+
+    def bf(a):
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(device)
+
+    nw, w, b = bf(nw_h), bf(w_h), bf(b_h)
+    cu = torch.from_numpy(row_bounds(s.batch, s.seq_len)).to(device)
+    out = torch.empty_like(x)
+    stream = torch.cuda.Stream(device)
+
+    def step(xx=x, oo=out):
+        E.engram_ple_short_conv(xx, w, dilation=d, group_size=G, cu_seqlens=cu,
+                                norm_weight=nw, conv_bias=b, out=oo, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    if E.engram_get_device_error(stream):
+        raise RuntimeError("device error flag set during warm-up")
+    Ksteps = args.steps
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(Ksteps)]
+    launches0 = E.engram_launch_count()
+    barrier(device)
+    torch.cuda.synchronize(device)
+    with ClockSampler(gpu_smi_id(torch, device)) as clk:
+        for e in evs:
+            e[0].record(stream)
+            step()
+            e[1].record(stream)
+        torch.cuda.synchronize(device)
+    barrier(device)
+    launches = E.engram_launch_count() - launches0
+    per = [e[0].elapsed_time(e[1]) for e in evs]
+    total_ms = max_over_ranks(evs[0][0].elapsed_time(evs[-1][1]), device)
+    kern_ms = statistics.mean(per)
+
+    # end to end through the public call with host buffers: x in from pinned
+    # memory, out back, copy-in / compute / copy-out overlapped on three streams
+    e2e_steps = max(1, min(Ksteps, args.e2e_steps))
+    x_h = x.cpu().pin_memory()
+    out_h = [torch.empty_like(x_h).pin_memory() for _ in range(2)]
+    xd = [x, torch.empty_like(x)]
+    od = [out, torch.empty_like(out)]
+    s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    in_done = [torch.cuda.Event() for _ in range(e2e_steps)]
+    comp_done = [torch.cuda.Event() for _ in range(e2e_steps)]
+    out_done = [torch.cuda.Event() for _ in range(e2e_steps)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    e0.record(s_in)
+    for k in range(e2e_steps):
+        with torch.cuda.stream(s_in):
+            if k >= 2:
+                s_in.wait_event(comp_done[k - 2])
+            xd[k % 2].copy_(x_h, non_blocking=True)
+            in_done[k].record(s_in)
+        stream.wait_event(in_done[k])
+        if k >= 2:
+            stream.wait_event(out_done[k - 2])
+        step(xd[k % 2], od[k % 2])
+        comp_done[k].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(comp_done[k])
+            out_h[k % 2].copy_(od[k % 2], non_blocking=True)
+            out_done[k].record(s_out)
+    e1.record(s_out)
+    torch.cuda.synchronize(device)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), device)
+    if E.engram_get_device_error(stream):
+        raise RuntimeError("device error flag set during timing")
+
+    peak, peak_kind = hbm_peak()
+    alg = T * C * 2 * 2 + C * (K + 2) * 2 + cu.numel() * 4
+    achieved = alg / kern_ms / 1e6
+    line = {
+        "metric": PLE_METRIC, "value": world * T * Ksteps / (total_ms / 1e3), "unit": UNIT,
+        "n_gpus": world, "steps": Ksteps, "warmup": args.warmup,
+        "ms_per_step": total_ms / Ksteps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "ple_full", "tokens_per_step_per_gpu": T, "channels": C,
+                   "branches": s.branches, "group": G, "kernel": K, "dilation": d,
+                   "flags": "norm + silu + residual", "cu_seqlens": f"{s.batch} rows",
+                   "l2": "inputs larger than L2 (1.34 GB in, 1.34 GB out)"},
+        "roofline": {"kernel": "short_conv_reg_kernel<bf16,bf16,4,3>", "bound": "hbm",
+                     "achieved": achieved, "peak": peak, "peak_kind": peak_kind,
+                     "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": committed_traffic("short_conv_reg_kernel", T)},
+        "stages": {"ple_short_conv": {"ms": kern_ms, "alg_bytes": alg, "gbs": achieved,
+                                      "frac": achieved / peak,
+                                      "ms_min": min(per), "ms_max": max(per)}},
+        "e2e": {"value": world * T * e2e_steps / (e2e_ms / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": x_h.numel() * 2, "d2h_bytes_per_step": x_h.numel() * 2,
+                "steps": e2e_steps,
+                "pipeline": "copy-in / compute / copy-out streams, two buffer sets"},
+        "gpu_launches": launches,
+        "clocks": clk.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        rate, _, _, _ = ple_oracle_run(256)
+        S = int(max(256, min(16384, rate * args.cpu_seconds)))
+        v, el, reps, desc = ple_oracle_run(S)
+        line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
+                                "sample": desc, "seconds": el}
+    else:
+        line["cpu_baseline"] = None
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -487,13 +659,16 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--stage", choices=["all", "bwd"], default="all",
+    ap.add_argument("--stage", choices=["all", "bwd", "ple"], default="all",
                     help="all: forward + backward (the step); bwd: the backward alone "
-                         "(indices from engram_hash, no table allocated)")
+                         "(indices from engram_hash, no table allocated); ple: the PLE "
+                         "tail (norm + short conv) on its own workload")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)      # at least 3 untimed warm-up steps
     if args.impl == "reference":
         return run_reference(args)
+    if args.stage == "ple":
+        return run_ple(args)
     return run_ours(args)
 
 

@@ -22,7 +22,8 @@ from ._binding import (ENGRAM_BF16, ENGRAM_CONV_NORM, ENGRAM_CONV_RESIDUAL, ENGR
 
 __all__ = [
     "ENGRAM_BF16", "ENGRAM_CONV_NORM", "ENGRAM_CONV_RESIDUAL", "ENGRAM_CONV_SILU",
-    "ENGRAM_DEVERR_COPY_TIMEOUT", "ENGRAM_DEVERR_CU_SEQLENS", "ENGRAM_DEVERR_ROW_RANGE", "ENGRAM_EINVAL",
+    "ENGRAM_DEVERR_COPY_TIMEOUT", "ENGRAM_DEVERR_CU_SEQLENS", "ENGRAM_DEVERR_ROW_RANGE",
+    "ENGRAM_EINVAL",
     "ENGRAM_ECUDA", "ENGRAM_ENOSPC", "ENGRAM_F16", "ENGRAM_F32",
     "ENGRAM_NOALLOC_SCRATCH_BYTES", "ENGRAM_OK", "EXPORTED", "LIB_PATH", "ConvParams",
     "EngramError", "EngramParams", "engram_abi_version", "engram_backward", "engram_backward_noalloc",

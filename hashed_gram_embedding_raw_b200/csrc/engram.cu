@@ -20,6 +20,7 @@
 #include "common.cuh"
 #include "hash_gather.cuh"
 #include "ple_conv.cuh"
+#include "ple_conv_reg.cuh"
 
 using namespace engram;
 
@@ -642,7 +643,8 @@ namespace {
 struct ConvPlan {
     ple::ConvArgs a;
     size_t smem = 0;
-    int grid = 0, threads = 0;
+    int grid = 0, threads = 0, chan = 4;
+    bool reg = false;  // kernel width 4, dilation 3: history in registers
 };
 
 bool overlaps(const void *a, size_t na, const void *b, size_t nb)
@@ -651,10 +653,10 @@ bool overlaps(const void *a, size_t na, const void *b, size_t nb)
     return na > 0 && nb > 0 && x < y + nb && y < x + na;
 }
 
-// Checks the shape (host only) and picks the block layout: the landing ring
-// as deep as shared memory allows after the private rings of the normalised
-// history. conv_grid adds the grid: one block per (branch, range), sms /
-// branches blocks per branch.
+// Checks the shape (host only) and sizes the block: G / 4 threads of 4
+// channels (G / 8 of 8 for branches wider than 2,560) and the private rings
+// of the normalised history. conv_grid adds the grid: one block per (branch,
+// range), sms / branches blocks per branch.
 int conv_plan(const engram_conv_params_t *p, int32_t dtype, int32_t out_dtype, int64_t T,
               ConvPlan *P)
 {
@@ -665,8 +667,7 @@ int conv_plan(const engram_conv_params_t *p, int32_t dtype, int32_t out_dtype, i
         (out_dtype != dtype && out_dtype != ENGRAM_F32))
         return ENGRAM_EINVAL;
     const int C = p->channels, G = p->group_size, K = p->kernel_size, d = p->dilation;
-    if (C < 1 || G < 1 || C % G != 0 || G % ple::kChan != 0 ||
-        G / ple::kChan > ple::kMaxThreads)
+    if (C < 1 || G < 8 || C % G != 0 || G % 8 != 0 || G / 8 > ple::kWideThreads)
         return ENGRAM_EINVAL;
     if (K < 1 || K > ple::kMaxTaps || d < 1 || d > 4096 || p->reserved != 0)
         return ENGRAM_EINVAL;
@@ -675,14 +676,10 @@ int conv_plan(const engram_conv_params_t *p, int32_t dtype, int32_t out_dtype, i
     if (T < 0 || T > INT32_MAX)
         return ENGRAM_EINVAL;
     const int halo = (K - 1) * d;
-    const int nth = G / ple::kChan;
-    const int pitch = (G * eb + 127) / 128 * 128;
+    const int chan = G / 4 <= ple::kNarrowThreads ? 4 : 8;  // channels per thread
+    const int nth = G / chan;
     const int norm_slots = halo + ple::kRows;
-    int raw = ple::kMaxRawSlots;
-    while (raw >= ple::kMinRawSlots &&
-           ple::smem_bytes(raw, pitch, norm_slots, nth) > ple::kSmemLimit)
-        --raw;
-    if (raw < ple::kMinRawSlots)
+    if (ple::smem_bytes(norm_slots, nth, chan) > ple::kSmemLimit)
         return ENGRAM_EINVAL;
     ple::ConvArgs &a = P->a;
     std::memset(&a, 0, sizeof(a));
@@ -696,12 +693,23 @@ int conv_plan(const engram_conv_params_t *p, int32_t dtype, int32_t out_dtype, i
     a.K = K;
     a.dil = d;
     a.halo = halo;
-    a.raw_slots = raw;
-    a.raw_pitch = pitch;
     a.norm_slots = norm_slots;
     a.flags = p->flags;
+    P->chan = chan;
     P->threads = (nth + 31) / 32 * 32;
-    P->smem = ple::smem_bytes(raw, pitch, norm_slots, nth);
+    P->smem = ple::smem_bytes(norm_slots, nth, chan);
+    // kernel width 4, dilation 3: blocks of 9 rows buffered in shared memory
+    const int pitch_reg = (G * eb + 127) / 128 * 128;
+    const int bufs = (int)std::min<size_t>(
+        ple::kRegMaxBufs, (ple::kSmemLimit - ple::kRegDataOffset) / ((size_t)9 * pitch_reg));
+    P->reg = K == 4 && d == 3 && G / 8 <= 32 * ple::kRegMaxConvWarps && bufs >= 2;
+    if (P->reg) {
+        a.nth = G / 8;
+        a.reg_bufs = bufs;
+        a.pitch = pitch_reg;
+        P->threads = 32 * ((a.nth + 31) / 32 + ple::kRegRmsWarps);
+        P->smem = ple::reg_smem_bytes(bufs, 9, pitch_reg);
+    }
     return ENGRAM_OK;
 }
 
@@ -741,12 +749,23 @@ int allow_smem(F fn)
     return ENGRAM_OK;
 }
 
+// The page's kernel width and dilation (4, 3) on branches up to 2,560
+// channels: the register-history kernel. Otherwise branches up to 2,560
+// channels take 4 channels per thread (kernel width 4 and the norm alone
+// specialised), wider branches 8.
 template <typename XT, typename OT>
 int launch_conv_t(const ConvPlan &P, cudaStream_t s)
 {
-    auto fn = P.a.K == 4   ? ple::short_conv_kernel<XT, OT, 4>
-              : P.a.K == 1 ? ple::short_conv_kernel<XT, OT, 1>
-                           : ple::short_conv_kernel<XT, OT, 0>;
+    if (P.reg) {
+        auto fr = ple::short_conv_reg_kernel<XT, OT, 4, 3>;
+        ENGRAM_TRY(allow_smem(fr));
+        fr<<<P.grid, P.threads, P.smem, s>>>(P.a);
+        return after_launch();
+    }
+    auto fn = P.chan == 8      ? ple::short_conv_kernel<XT, OT, 0, 8>
+              : P.a.K == 4 ? ple::short_conv_kernel<XT, OT, 4, 4>
+              : P.a.K == 1 ? ple::short_conv_kernel<XT, OT, 1, 4>
+                           : ple::short_conv_kernel<XT, OT, 0, 4>;
     ENGRAM_TRY(allow_smem(fn));
     fn<<<P.grid, P.threads, P.smem, s>>>(P.a);
     return after_launch();

@@ -290,8 +290,8 @@ typedef struct engram_conv_params {
  *   out         device, [T, C] of out_dtype (dtype or ENGRAM_F32), 16-byte
  *               aligned, not overlapping x
  * Limits (else ENGRAM_EINVAL): those of engram_conv_params_t and
- * 4 * G * ((K - 1) * d + 4) + 8 * G * sizeof(dtype) + 2 KB <= 227 KB of shared
- * memory per block (the page's shape, G = 2560, K = 4, d = 3: 133 KB + ring).
+ * 4 * G * ((K - 1) * d + 4) + 1152 <= 227 KB of shared memory per block (the
+ * page's shape, G = 2560, K = 4, d = 3: 134 KB).
  */
 ENGRAM_API int engram_ple_short_conv(const engram_conv_params_t *params, const void *x,
                                      int32_t dtype, const int32_t *cu_seqlens, int32_t nseq,
