@@ -139,10 +139,11 @@ def gpu_smi_id(torch, device) -> str:
 
 # -------------------------------------------------------- committed traffic
 
-def csrc_digest() -> str:
+def source_digest(files) -> str:
+    """Digest of the named kernel sources (file names under csrc/)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "hashed_gram_embedding_raw_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in sorted(files):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -150,17 +151,16 @@ def csrc_digest() -> str:
 
 def committed_traffic(kernel: str, units: float):
     """DRAM bytes per launch from profiles/dram_traffic.json, scaled to `units`
-    (lookups or tokens), or None if absent or taken on other kernel sources."""
+    (lookups or tokens), or None if absent or taken on other kernel sources
+    (each record carries the digest of the sources its kernel is built from)."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f)
-    except (OSError, ValueError):
-        return None
-    if rec.get("csrc_digest") != csrc_digest():
-        return None
-    k = rec.get("kernels", {}).get(kernel)
-    if not k:
+        k = rec["kernels"][kernel]
+        if k["digest"] != source_digest(k["sources"]):
+            return None
+    except (OSError, ValueError, KeyError):
         return None
     return k["dram_bytes_per_unit"] * units
 
