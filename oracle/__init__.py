@@ -1,5 +1,6 @@
 """CPU oracle of the Engram N-gram Embedding path (hash, gather, backward,
-and the PLE layer's grouped RMS norm and causal short convolution).
+the PLE layer's grouped RMS norm and causal short convolution, and the sparse
+optimizer step on the touched rows).
 
 TEST INFRASTRUCTURE ONLY. Only `tests/`, `__graft_entry__.smoke()` and the
 CPU-baseline / reference legs of `bench.py` may import this package. The
@@ -67,6 +68,9 @@ def _declare(L):
                                     P, P, ctypes.c_int, i32, i32, ctypes.c_int, ctypes.c_int,
                                     ctypes.c_int, P]
     L.oracle_short_conv.restype = ctypes.c_int
+    d = ctypes.c_double
+    L.oracle_sparse_adam.argtypes = [P, P, P, i64, i32, P, P, i64, d, d, d, d, d, i64]
+    L.oracle_sparse_adam.restype = ctypes.c_int
     return L
 
 
@@ -191,3 +195,23 @@ def short_conv(x, dtype, cu, conv_w, *, dilation, group=None, norm_w=None, eps=1
     if rc != 0:
         raise ValueError("oracle_short_conv: invalid arguments")
     return out
+
+
+def sparse_adam(p, m, v, rows, grads, *, lr, betas=(0.9, 0.999), eps=1e-8, weight_decay=0.0,
+                step=1):
+    """One lazy AdamW step on `rows` (int64 [U]) with row gradients `grads`
+    (fp32 [U, D]); p, m, v are fp64 [R, D] arrays, returned updated copies."""
+    p = np.array(p, dtype=np.float64, order="C")
+    m = np.array(m, dtype=np.float64, order="C")
+    v = np.array(v, dtype=np.float64, order="C")
+    rows = np.ascontiguousarray(rows, dtype=np.int64).reshape(-1)
+    grads = np.ascontiguousarray(grads, dtype=np.float32)
+    R, D = p.shape
+    U = rows.shape[0]
+    assert grads.shape == (U, D)
+    rc = lib().oracle_sparse_adam(_ptr(p), _ptr(m), _ptr(v), R, D, _ptr(rows),
+                                  _ptr(grads) if U else None, U, float(lr), float(betas[0]),
+                                  float(betas[1]), float(eps), float(weight_decay), int(step))
+    if rc != 0:
+        raise ValueError("oracle_sparse_adam: invalid arguments")
+    return p, m, v

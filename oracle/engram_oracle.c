@@ -369,3 +369,55 @@ int oracle_short_conv(const void *x, int dtype, const int32_t *cu, int32_t nseq,
     free(n);
     return ORACLE_OK;
 }
+
+/* ----------------------------------------------- sparse optimizer step */
+
+/*
+ * One AdamW step applied only to the rows a backward produced (the owner
+ * "stores and updates each row's gradient", model card; the table's
+ * optimizer tensors live in the checkpoint, model card §Current Scope). The
+ * pages name no formula; this is AdamW updated lazily, with the step counter
+ * global to the table. For u < U, r = rows[u], g = grads[u, :] and every
+ * column c:
+ *   p[r,c] *= 1 - lr * wd                          (decoupled weight decay)
+ *   m[r,c]  = b1 * m[r,c] + (1 - b1) * g[c]
+ *   v[r,c]  = b2 * v[r,c] + (1 - b2) * g[c]^2
+ *   p[r,c] -= lr / (1 - b1^step) * m[r,c] / (sqrt(v[r,c] / (1 - b2^step)) + eps)
+ * Rows not listed keep p, m and v. p, m, v are fp64 [rows, dim] in and out;
+ * rows listed twice are updated twice, in order.
+ */
+int oracle_sparse_adam(double *p, double *m, double *v, int64_t rows, int32_t dim,
+                       const int64_t *uniq, const float *grads, int64_t U, double lr,
+                       double b1, double b2, double eps, double wd, int64_t step)
+{
+    if (rows < 0 || dim <= 0 || U < 0 || step < 1)
+        return ORACLE_EINVAL;
+    double bc1 = 1.0, bc2 = 1.0;
+    for (int64_t s = 0; s < step; ++s) {
+        bc1 *= b1;
+        bc2 *= b2;
+    }
+    bc1 = 1.0 - bc1;
+    bc2 = 1.0 - bc2;
+    if (ORACLE_MUTANT == 15)
+        bc1 = bc2 = 1.0; /* mutant: no bias correction */
+    for (int64_t u = 0; u < U; ++u) {
+        const int64_t r = uniq[u];
+        if (r < 0 || r >= rows)
+            return ORACLE_EINVAL;
+        for (int32_t c = 0; c < dim; ++c) {
+            const int64_t i = r * dim + c;
+            double g = (double)grads[u * dim + c];
+            if (ORACLE_MUTANT == 17)
+                g += wd * p[i]; /* mutant: L2 penalty in the gradient, not decoupled */
+            else
+                p[i] *= 1.0 - lr * wd;
+            m[i] = b1 * m[i] + (1.0 - b1) * g;
+            v[i] = b2 * v[i] + (1.0 - b2) * g * g;
+            const double denom = ORACLE_MUTANT == 16 ? sqrt(v[i] / bc2 + eps)
+                                                     : sqrt(v[i] / bc2) + eps;
+            p[i] -= lr / bc1 * m[i] / denom;
+        }
+    }
+    return ORACLE_OK;
+}

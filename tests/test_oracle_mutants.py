@@ -4,14 +4,16 @@ Each mutant is the oracle rebuilt with one known mistake (ORACLE_MUTANT in
 engram_oracle.c): a plausible slip in the hash (operator, reset position,
 multiplier pairing, remainder sign, sequence reset), in the backward
 (accumulation precision, grouping) or in the PLE norm and convolution (scale,
-group width, epsilon, dilation, tap order, history reset, residual). The pins
-of test_oracle_hash.py, test_oracle_gather_backward.py and test_oracle_ple.py
-are run against each; at least one must fail.
+group width, epsilon, dilation, tap order, history reset, residual) or in the
+optimizer step (bias correction, epsilon, weight decay). The pins of
+test_oracle_hash.py, test_oracle_gather_backward.py, test_oracle_ple.py and
+test_oracle_adam.py are run against each; at least one must fail.
 """
 
 import pytest
 
 import oracle
+from tests import test_oracle_adam as AD
 from tests import test_oracle_gather_backward as GB
 from tests import test_oracle_hash as TH
 from tests import test_oracle_ple as PL
@@ -46,6 +48,12 @@ PLE_PINS = [
     PL.test_sequences_are_independent,
 ]
 
+ADAM_PINS = [
+    AD.test_first_step_closed_form,
+    lambda: [AD.test_matches_torch_adamw_when_all_rows_present(wd) for wd in (0.0, 0.05)],
+    AD.test_matches_torch_sparse_adam_over_changing_rows,
+]
+
 MUTANTS = {
     1: ("add instead of xor", HASH_PINS),
     2: ("reset before EOS instead of after", HASH_PINS),
@@ -61,6 +69,9 @@ MUTANTS = {
     12: ("conv taps reversed", PLE_PINS),
     13: ("conv history crosses sequence starts", PLE_PINS),
     14: ("residual of the normalised input", PLE_PINS),
+    15: ("no bias correction", ADAM_PINS),
+    16: ("eps inside the square root", ADAM_PINS),
+    17: ("L2 penalty instead of decoupled decay", ADAM_PINS),
 }
 
 
