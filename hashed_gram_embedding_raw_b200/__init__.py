@@ -1,5 +1,6 @@
-"""B200-native Engram N-gram Embedding: hash, gather, compact backward, and
-the PLE layer's grouped RMS norm and causal short convolution.
+"""B200-native Engram N-gram Embedding: hash, gather, compact backward, the
+sparse optimizer step on the touched rows, and the PLE layer's grouped RMS
+norm and causal short convolution.
 
 Python face of the C ABI in include/engram.h (libengram_b200.so, sm_100a).
 Every step runs in the library's CUDA kernels; this package only marshals
@@ -12,12 +13,13 @@ from ._binding import (ENGRAM_BF16, ENGRAM_CONV_NORM, ENGRAM_CONV_RESIDUAL, ENGR
                        ENGRAM_DEVERR_ROW_RANGE,
                        ENGRAM_EINVAL, ENGRAM_ECUDA, ENGRAM_ENOSPC, ENGRAM_F16, ENGRAM_F32,
                        ENGRAM_NOALLOC_SCRATCH_BYTES, ENGRAM_OK, EXPORTED, LIB_PATH,
-                       ConvParams, EngramError, EngramParams, engram_abi_version,
+                       AdamParams, ConvParams, EngramError, EngramParams, engram_abi_version,
                        engram_backward,
                        engram_backward_noalloc, engram_backward_reduce, engram_backward_sort,
                        engram_backward_workspace_size, engram_gather, engram_get_device_error,
                        engram_grouped_rms_norm, engram_hash, engram_hash_gather,
                        engram_hash_gather_slice, engram_host_floor_mod, engram_ple_short_conv,
+                       engram_sparse_adam,
                        engram_launch_count, lib, make_params, status_string)
 
 __all__ = [
@@ -25,10 +27,11 @@ __all__ = [
     "ENGRAM_DEVERR_COPY_TIMEOUT", "ENGRAM_DEVERR_CU_SEQLENS", "ENGRAM_DEVERR_ROW_RANGE",
     "ENGRAM_EINVAL",
     "ENGRAM_ECUDA", "ENGRAM_ENOSPC", "ENGRAM_F16", "ENGRAM_F32",
-    "ENGRAM_NOALLOC_SCRATCH_BYTES", "ENGRAM_OK", "EXPORTED", "LIB_PATH", "ConvParams",
+    "ENGRAM_NOALLOC_SCRATCH_BYTES", "ENGRAM_OK", "EXPORTED", "LIB_PATH", "AdamParams", "ConvParams",
     "EngramError", "EngramParams", "engram_abi_version", "engram_backward", "engram_backward_noalloc",
     "engram_backward_reduce", "engram_backward_sort", "engram_backward_workspace_size",
     "engram_gather", "engram_get_device_error", "engram_hash", "engram_hash_gather",
     "engram_hash_gather_slice", "engram_grouped_rms_norm", "engram_ple_short_conv",
+    "engram_sparse_adam",
     "engram_host_floor_mod", "engram_launch_count", "lib", "make_params", "status_string",
 ]

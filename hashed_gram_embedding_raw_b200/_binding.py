@@ -33,7 +33,7 @@ EXPORTED = (
     "engram_backward_reduce", "engram_get_device_error", "engram_status_string",
     "engram_abi_version", "engram_params_size", "engram_launch_count",
     "engram_host_floor_mod", "engram_backward_noalloc", "engram_hash_gather_slice",
-    "engram_ple_short_conv", "engram_grouped_rms_norm",
+    "engram_ple_short_conv", "engram_grouped_rms_norm", "engram_sparse_adam",
 )
 
 ENGRAM_NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -77,6 +77,19 @@ class ConvParams(ctypes.Structure):
         ("flags", ctypes.c_uint32),
         ("weight_dtype", ctypes.c_int32),
         ("reserved", ctypes.c_int32),
+    ]
+
+
+class AdamParams(ctypes.Structure):
+    """Mirror of engram_adam_params_t."""
+    _fields_ = [
+        ("lr", ctypes.c_float),
+        ("beta1", ctypes.c_float),
+        ("beta2", ctypes.c_float),
+        ("eps", ctypes.c_float),
+        ("weight_decay", ctypes.c_float),
+        ("reserved", ctypes.c_int32),
+        ("step", ctypes.c_int64),
     ]
 
 
@@ -124,6 +137,7 @@ def _load():
         "engram_hash_gather_slice": [P, P, P, i32, i64, i64, i64, i64, P, i32, P, P, P],
         "engram_ple_short_conv": [P, P, i32, P, i32, i64, P, P, P, P, i32, P],
         "engram_grouped_rms_norm": [P, i32, i64, i32, i32, P, i32, ctypes.c_float, P, i32, P],
+        "engram_sparse_adam": [P, P, i32, i64, i32, P, P, P, P, P, i64, P],
     }
     for name, args in sig.items():
         fn = getattr(L, name)
@@ -431,6 +445,35 @@ def engram_grouped_rms_norm(x: torch.Tensor, group_size: int, weight=None, eps: 
                                        _dtype_code(out), _stream(stream)),
            "engram_grouped_rms_norm")
     return out
+
+
+# ---------------------------------------------------------- optimizer step
+
+def engram_sparse_adam(table: torch.Tensor, exp_avg: torch.Tensor, exp_avg_sq: torch.Tensor,
+                       uniq_rows: torch.Tensor, row_grads: torch.Tensor, num_unique: torch.Tensor,
+                       *, lr: float, betas=(0.9, 0.999), eps: float = 1e-8,
+                       weight_decay: float = 0.0, step: int, stream=None) -> None:
+    """Lazy AdamW step, in place, on the rows uniq_rows[:num_unique] of
+    `table` [R, D] (fp32 / bf16 / fp16) with fp32 moments [R, D];
+    num_unique is the device scalar the backward wrote."""
+    _cuda(table, "table")
+    _cuda(exp_avg, "exp_avg", torch.float32)
+    _cuda(exp_avg_sq, "exp_avg_sq", torch.float32)
+    _cuda(uniq_rows, "uniq_rows", torch.int32)
+    _cuda(row_grads, "row_grads", torch.float32)
+    _cuda(num_unique, "num_unique", torch.int32)
+    R, D = table.shape
+    if exp_avg.shape != table.shape or exp_avg_sq.shape != table.shape:
+        raise ValueError("moments must have the table's shape")
+    cap = uniq_rows.numel()
+    if row_grads.numel() < cap * D:
+        raise ValueError("row_grads must hold capacity x D values")
+    p = AdamParams(float(lr), float(betas[0]), float(betas[1]), float(eps), float(weight_decay),
+                   0, int(step))
+    _check(lib.engram_sparse_adam(ctypes.byref(p), _ptr(table), _dtype_code(table), R, D,
+                                  _ptr(exp_avg), _ptr(exp_avg_sq), _ptr(uniq_rows),
+                                  _ptr(row_grads), _ptr(num_unique), cap, _stream(stream)),
+           "engram_sparse_adam")
 
 
 # -------------------------------------------------------------------- misc

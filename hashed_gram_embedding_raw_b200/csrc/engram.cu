@@ -21,6 +21,7 @@
 #include "hash_gather.cuh"
 #include "ple_conv.cuh"
 #include "ple_conv_reg.cuh"
+#include "optim.cuh"
 
 using namespace engram;
 
@@ -849,6 +850,79 @@ int engram_grouped_rms_norm(const void *x, int32_t dtype, int64_t rows, int32_t 
     P.a.nseq = 1;
     P.a.norm_w = weight;
     return launch_conv(P, dtype, out_dtype, (cudaStream_t)stream);
+}
+
+} // extern "C"
+
+// ------------------------------------------------------ optimizer step
+
+extern "C" {
+
+int engram_sparse_adam(const engram_adam_params_t *params, void *table, int32_t dtype,
+                       int64_t table_rows, int32_t dim, float *exp_avg, float *exp_avg_sq,
+                       const int32_t *uniq_rows, const float *row_grads,
+                       const int32_t *num_unique, int64_t max_rows, engram_stream_t stream)
+{
+    if (params == nullptr)
+        return ENGRAM_EINVAL;
+    const engram_adam_params_t &p = *params;
+    const int eb = elem_bytes(dtype);
+    if (eb == 0 || dim < 4 || dim % 4 != 0 || table_rows < 1 || table_rows > INT32_MAX ||
+        max_rows < 0 || max_rows > INT32_MAX || p.reserved != 0 || p.step < 1)
+        return ENGRAM_EINVAL;
+    if (!std::isfinite(p.lr) || p.lr < 0.f || !(p.beta1 >= 0.f && p.beta1 < 1.f) ||
+        !(p.beta2 >= 0.f && p.beta2 < 1.f) || !std::isfinite(p.eps) || p.eps < 0.f ||
+        !std::isfinite(p.weight_decay) || p.weight_decay < 0.f)
+        return ENGRAM_EINVAL;
+    if (max_rows == 0)
+        return ENGRAM_OK;
+    if (table == nullptr || exp_avg == nullptr || exp_avg_sq == nullptr ||
+        uniq_rows == nullptr || row_grads == nullptr || num_unique == nullptr)
+        return ENGRAM_EINVAL;
+    if (((uintptr_t)table & (dtype == ENGRAM_F32 ? 15u : 7u)) != 0 || !aligned16(exp_avg) ||
+        !aligned16(exp_avg_sq) || !aligned16(row_grads))
+        return ENGRAM_EINVAL;
+    optim::AdamArgs a;
+    a.table = table;
+    a.m = exp_avg;
+    a.v = exp_avg_sq;
+    a.rows = uniq_rows;
+    a.grads = row_grads;
+    a.num_unique = num_unique;
+    a.table_rows = table_rows;
+    a.max_rows = max_rows;
+    a.dim = dim;
+    a.b1 = p.beta1;
+    a.b2 = p.beta2;
+    a.one_b1 = (float)(1.0 - (double)p.beta1);
+    a.one_b2 = (float)(1.0 - (double)p.beta2);
+    const double bc1 = 1.0 - std::pow((double)p.beta1, (double)p.step);
+    const double bc2 = 1.0 - std::pow((double)p.beta2, (double)p.step);
+    a.step_size = (float)((double)p.lr / bc1);
+    a.inv_sqrt_bc2 = (float)(1.0 / std::sqrt(bc2));
+    a.eps = p.eps;
+    a.decay = (float)(1.0 - (double)p.lr * (double)p.weight_decay);
+    int sms = 0;
+    ENGRAM_TRY(device_sms(&sms));
+    const int64_t work = max_rows * (dim / 4);
+    const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(ceil_div(work, 256), (int64_t)sms * 8));
+    cudaStream_t s = (cudaStream_t)stream;
+    const bool d160 = dim == 160;
+    switch (dtype) {
+    case ENGRAM_F32:
+        (d160 ? optim::sparse_adam_kernel<float, 40> : optim::sparse_adam_kernel<float, 0>)
+            <<<(unsigned)blocks, 256, 0, s>>>(a);
+        break;
+    case ENGRAM_BF16:
+        (d160 ? optim::sparse_adam_kernel<__nv_bfloat16, 40>
+              : optim::sparse_adam_kernel<__nv_bfloat16, 0>)<<<(unsigned)blocks, 256, 0, s>>>(a);
+        break;
+    default:
+        (d160 ? optim::sparse_adam_kernel<__half, 40> : optim::sparse_adam_kernel<__half, 0>)
+            <<<(unsigned)blocks, 256, 0, s>>>(a);
+        break;
+    }
+    return after_launch();
 }
 
 } // extern "C"

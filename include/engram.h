@@ -314,6 +314,49 @@ ENGRAM_API int engram_grouped_rms_norm(const void *x, int32_t dtype, int64_t row
                                        const void *weight, int32_t weight_dtype, float eps,
                                        void *out, int32_t out_dtype, engram_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * Optimizer step on the rows a backward produced. The pages say that the
+ * owner stores and updates each row's gradient and that the Engram table
+ * carries optimizer tensors in the checkpoint; they name no formula. This is
+ * AdamW with per-row moments, applied lazily (only the listed rows change)
+ * with the step count global to the table.
+ * ------------------------------------------------------------------------ */
+
+typedef struct engram_adam_params {
+    float lr;            /* learning rate, >= 0 */
+    float beta1, beta2;  /* in [0, 1) */
+    float eps;           /* >= 0 */
+    float weight_decay;  /* decoupled decay, >= 0 */
+    int32_t reserved;    /* must be 0 */
+    int64_t step;        /* 1 for the first update */
+} engram_adam_params_t;
+
+/*
+ * engram_sparse_adam -- for u < U = min(*num_unique, max_rows), row
+ * r = uniq_rows[u], gradient g = row_grads[u, :]:
+ *   p[r] *= 1 - lr * weight_decay
+ *   m[r]  = beta1 * m[r] + (1 - beta1) * g
+ *   v[r]  = beta2 * v[r] + (1 - beta2) * g^2
+ *   p[r] -= lr / (1 - beta1^step) * m[r] / (sqrt(v[r]) / sqrt(1 - beta2^step) + eps)
+ * in fp32, p rounded once to dtype. Other rows are untouched.
+ *   table      device, [table_rows, dim] of dtype (F32 | BF16 | F16), updated in
+ *              place; 16-byte aligned (F32) or 8-byte aligned (BF16 / F16)
+ *   exp_avg, exp_avg_sq  device, fp32 [table_rows, dim], 16-byte aligned, updated
+ *   uniq_rows  device, int32 [>= U], distinct rows (the backward's output);
+ *              a row outside the table is skipped and sets ENGRAM_DEVERR_ROW_RANGE
+ *   row_grads  device, fp32 [>= U, dim], 16-byte aligned
+ *   num_unique device, int32 scalar (read on the device: no host round trip
+ *              after engram_backward)
+ *   max_rows   capacity of uniq_rows / row_grads
+ * dim % 4 == 0. Rows listed twice race (the backward lists each row once).
+ */
+ENGRAM_API int engram_sparse_adam(const engram_adam_params_t *params, void *table,
+                                  int32_t dtype, int64_t table_rows, int32_t dim,
+                                  float *exp_avg, float *exp_avg_sq,
+                                  const int32_t *uniq_rows, const float *row_grads,
+                                  const int32_t *num_unique, int64_t max_rows,
+                                  engram_stream_t stream);
+
 /*
  * engram_get_device_error -- copy the current device's error word
  * (ENGRAM_DEVERR_* bits set since the last call) into *flags and clear it.

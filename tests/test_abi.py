@@ -180,6 +180,28 @@ def test_host_rejects_bad_conv_args(E):
     assert N(al, 1, 0, 96, 32, None, 0, 1e-6, al, 1, None) == E.ENGRAM_OK
 
 
+def test_host_rejects_bad_adam_args(E):
+    L = E.lib
+    a16, a8 = ctypes.c_void_p(1 << 20), ctypes.c_void_p((1 << 21) + 8)
+
+    def adam(dtype=1, rows=100, dim=160, table=a16, m=a16, cap=10, **kw):
+        base = dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0, reserved=0,
+                    step=1)
+        base.update(kw)
+        p = E.AdamParams(**base)
+        return L.engram_sparse_adam(ctypes.byref(p), table, dtype, rows, dim, m, a16, a16, a16,
+                                    a16, cap, None)
+
+    for kw in (dict(dim=6), dict(dim=0), dict(dtype=9), dict(rows=0), dict(step=0),
+               dict(lr=-1.0), dict(beta1=1.0), dict(beta2=-0.1), dict(eps=-1e-8),
+               dict(weight_decay=float("inf")), dict(reserved=3), dict(cap=-1),
+               dict(m=a8), dict(dtype=0, table=a8)):
+        assert adam(**kw) == E.ENGRAM_EINVAL, kw
+    assert adam(cap=0) == E.ENGRAM_OK                            # nothing to update
+    assert L.engram_sparse_adam(None, a16, 1, 100, 160, a16, a16, a16, a16, a16, 10,
+                                None) == E.ENGRAM_EINVAL
+
+
 def test_package_import_fails_loudly_without_library(tmp_path):
     # a copy of the binding pointed at a directory with no library must raise
     import importlib.util
