@@ -8,6 +8,7 @@ gradients) over one batch of the named workload, all inputs resident in HBM.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload full]
     python bench.py --impl reference ...   # the CPU oracle, timed on this host
     python bench.py --stage ple ...        # the PLE tail kernel on its own workload
+    python bench.py --stage adam ...       # the sparse optimizer step on a table shard
 
 Multi-GPU (torchrun, one rank per GPU): every rank holds its own table
 replica and processes its own batch; no data-path collective exists, so the
@@ -216,8 +217,13 @@ def run_reference(args):
     if rank != 0:
         return 0
     name = args.workload
-    ple = args.stage == "ple"
-    run = (lambda S: ple_oracle_run(S)) if ple else (lambda S: oracle_run(name, S))
+    ple, adam = args.stage == "ple", args.stage == "adam"
+    if adam:
+        run = adam_oracle_run
+    elif ple:
+        run = ple_oracle_run
+    else:
+        run = lambda S: oracle_run(name, S)  # noqa: E731
     # calibrate, then size each step's sample so W + K steps take ~2 minutes
     rate, _, _, _ = run(256 if ple else 4096)
     budget = float(os.environ.get("ENGRAM_REFERENCE_BUDGET_S", "120"))
@@ -232,16 +238,18 @@ def run_reference(args):
     value = S * len(times) / total
     if ple:
         name = "ple_full"
+    if adam:
+        name = "adam_shard"
     line = {
-        "impl": "reference", "metric": PLE_METRIC if ple else METRIC, "value": value,
-        "unit": UNIT,
+        "impl": "reference", "metric": ADAM_METRIC if adam else PLE_METRIC if ple else METRIC,
+        "value": value, "unit": "rows/s" if adam else UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * total / len(times), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64" if ple else "int64/f64",
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64" if ple or adam else "int64/f64",
         "data": "synthetic", "config": {"workload": name, "tokens_per_step": S},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": desc},
-        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+        "cpu_baseline": {"value": value, "unit": "rows/s" if adam else UNIT, "cores": 1,
+                         "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "rows/s" if adam else UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -648,6 +656,184 @@ def run_ple(args):
     return 0
 
 
+# ------------------------------------------------------ optimizer stage
+
+ADAM_METRIC = ("Sparse AdamW rows/s (lazy update of the touched rows of a 40,000,192 x 160 bf16 "
+               "table shard with fp32 moments); achieved HBM GB/s vs peak")
+ADAM_ROWS = 40_000_192        # one eighth of the 320,001,536 padded rows: an 8-way owner shard
+ADAM_TOUCHED = 1 << 20        # rows one step updates (about one full-workload backward)
+ADAM_DIM = 160
+ADAM_BYTES_PER_ROW = 4 + 640 + 2 * 2 * 640 + 2 * 320   # id, grad, m and v r/w, bf16 p r/w
+
+
+def adam_oracle_run(U: int, reps_seconds: float = 0.0, max_reps: int = 1):
+    """Time the CPU oracle's optimizer step on U rows (a U-row table with every
+    row touched). Returns (rows/s, seconds, reps, description)."""
+    import oracle
+    rng = np.random.default_rng(9)
+    p = rng.standard_normal((U, ADAM_DIM))
+    m = np.zeros_like(p)
+    v = np.zeros_like(p)
+    rows = np.arange(U, dtype=np.int64)
+    g = rng.standard_normal((U, ADAM_DIM)).astype(np.float32)
+    oracle.lib()
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        p, m, v = oracle.sparse_adam(p, m, v, rows, g, lr=1e-3, weight_decay=0.01,
+                                     step=reps + 1)
+        reps += 1
+        el = time.perf_counter() - t0
+        if reps >= max_reps or el >= reps_seconds:
+            break
+    desc = (f"{U} rows x {ADAM_DIM} columns, all touched, x {reps} rep(s) (array copies "
+            f"included); single-threaded C oracle in fp64")
+    return U * reps / el, el, reps, desc
+
+
+def run_adam(args):
+    """--stage adam: engram_sparse_adam on an 8-way owner shard of the page's
+    table with a full backward's worth of touched rows."""
+    import torch
+
+    import hashed_gram_embedding_raw_b200 as E
+
+    rank, local_rank, world = rank_env()
+    assert torch.cuda.is_available(), "bench.py needs a CUDA device"
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", device_id=device,
+                                timeout=datetime.timedelta(seconds=300))
+    R, D, U = args.adam_rows, ADAM_DIM, args.adam_touched
+    if not 0 < U <= R:
+        raise ValueError("need 0 < --adam-touched <= --adam-rows")
+    g = torch.Generator(device=device).manual_seed(8000 + rank)
+    table = torch.empty((R, D), dtype=torch.bfloat16, device=device)
+    for r0 in range(0, R, 1 << 22):  # chunked fill keeps the fp32 temporary small
+        r1 = min(R, r0 + (1 << 22))
+        table[r0:r1] = (0.02 * torch.randn((r1 - r0, D), generator=g, device=device)).to(
+            torch.bfloat16)
+    m = torch.zeros((R, D), dtype=torch.float32, device=device)
+    v = torch.zeros((R, D), dtype=torch.float32, device=device)
+    rows = torch.randperm(R, generator=g, device=device)[:U].sort().values.to(torch.int32)
+    grads = torch.randn((U, D), generator=g, device=device)
+    nu = torch.tensor([U], dtype=torch.int32, device=device)
+    stream = torch.cuda.Stream(device)
+    step_no = [0]
+
+    def step(rr=rows, gg=grads, n=nu):
+        step_no[0] += 1
+        E.engram_sparse_adam(table, m, v, rr, gg, n, lr=1e-3, weight_decay=0.01,
+                             step=step_no[0], stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    if E.engram_get_device_error(stream):
+        raise RuntimeError("device error flag set during warm-up")
+    K = args.steps
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(K)]
+    launches0 = E.engram_launch_count()
+    barrier(device)
+    torch.cuda.synchronize(device)
+    with ClockSampler(gpu_smi_id(torch, device)) as clk:
+        for e in evs:
+            e[0].record(stream)
+            step()
+            e[1].record(stream)
+        torch.cuda.synchronize(device)
+    barrier(device)
+    launches = E.engram_launch_count() - launches0
+    per = [e[0].elapsed_time(e[1]) for e in evs]
+    total_ms = max_over_ranks(evs[0][0].elapsed_time(evs[-1][1]), device)
+    kern_ms = statistics.mean(per)
+
+    # end to end: the step's rows and gradients in from pinned memory, the step,
+    # and the updated rows (engram_gather) back out, over three streams
+    e2e_steps = max(1, min(K, args.e2e_steps))
+    rows_h = rows.cpu().pin_memory()
+    grads_h = grads.cpu().pin_memory()
+    out_h = [torch.empty((U, D), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    rd = [rows, torch.empty_like(rows)]
+    gd = [grads, torch.empty_like(grads)]
+    od = [torch.empty((U, D), dtype=torch.bfloat16, device=device) for _ in range(2)]
+    s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    in_done = [torch.cuda.Event() for _ in range(e2e_steps)]
+    comp_done = [torch.cuda.Event() for _ in range(e2e_steps)]
+    out_done = [torch.cuda.Event() for _ in range(e2e_steps)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    e0.record(s_in)
+    for k in range(e2e_steps):
+        b = k % 2
+        with torch.cuda.stream(s_in):
+            if k >= 2:
+                s_in.wait_event(comp_done[k - 2])
+            rd[b].copy_(rows_h, non_blocking=True)
+            gd[b].copy_(grads_h, non_blocking=True)
+            in_done[k].record(s_in)
+        stream.wait_event(in_done[k])
+        if k >= 2:
+            stream.wait_event(out_done[k - 2])
+        step(rd[b], gd[b])
+        E.engram_gather(table, rd[b], out=od[b], stream=stream)
+        comp_done[k].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(comp_done[k])
+            out_h[b].copy_(od[b], non_blocking=True)
+            out_done[k].record(s_out)
+    e1.record(s_out)
+    torch.cuda.synchronize(device)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), device)
+    if E.engram_get_device_error(stream):
+        raise RuntimeError("device error flag set during timing")
+
+    peak, peak_kind = hbm_peak()
+    alg = U * ADAM_BYTES_PER_ROW
+    achieved = alg / kern_ms / 1e6
+    line = {
+        "metric": ADAM_METRIC, "value": world * U * K / (total_ms / 1e3), "unit": "rows/s",
+        "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": total_ms / K,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16/f32",
+        "data": "synthetic",
+        "config": {"workload": "adam_shard" if (R, U) == (ADAM_ROWS, ADAM_TOUCHED)
+                   else f"adam_{R}x{D}_touch{U}", "table_rows": R, "dim": D, "touched_rows": U,
+                   "table_dtype": "bf16", "moments": "f32", "lr": 1e-3, "weight_decay": 0.01,
+                   "l2": "inputs larger than L2 (12.8 GB table, 51.2 GB moments, random rows)"},
+        "roofline": {"kernel": "sparse_adam_kernel<bf16,40>", "bound": "hbm",
+                     "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": achieved / peak,
+                     "traffic": committed_traffic("sparse_adam_kernel", U)},
+        "stages": {"sparse_adam": {"ms": kern_ms, "alg_bytes": alg, "gbs": achieved,
+                                   "frac": achieved / peak, "ms_min": min(per),
+                                   "ms_max": max(per)}},
+        "e2e": {"value": world * U * e2e_steps / (e2e_ms / 1e3), "unit": "rows/s",
+                "h2d_bytes_per_step": rows_h.numel() * 4 + grads_h.numel() * 4,
+                "d2h_bytes_per_step": U * D * 2, "steps": e2e_steps,
+                "pipeline": "copy-in / step + gather of the updated rows / copy-out streams"},
+        "gpu_launches": launches,
+        "clocks": clk.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        rate, _, _, _ = adam_oracle_run(2048)
+        n = int(max(2048, min(1 << 18, rate * args.cpu_seconds)))
+        val, el, reps, desc = adam_oracle_run(n)
+        line["cpu_baseline"] = {"value": val, "unit": "rows/s", "cores": 1, "kind": "oracle",
+                                "sample": desc, "seconds": el}
+    else:
+        line["cpu_baseline"] = None
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -657,18 +843,25 @@ def main(argv=None):
     ap.add_argument("--workload", default="full",
                     choices=["tiny", "b4x4096", "thd64k", "full", "long256k"])
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--adam-rows", type=int, default=ADAM_ROWS,
+                    help="--stage adam: table rows (default: an 8-way shard of the page table)")
+    ap.add_argument("--adam-touched", type=int, default=ADAM_TOUCHED,
+                    help="--stage adam: rows one step updates")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--stage", choices=["all", "bwd", "ple"], default="all",
+    ap.add_argument("--stage", choices=["all", "bwd", "ple", "adam"], default="all",
                     help="all: forward + backward (the step); bwd: the backward alone "
                          "(indices from engram_hash, no table allocated); ple: the PLE "
-                         "tail (norm + short conv) on its own workload")
+                         "tail (norm + short conv) on its own workload; adam: the sparse "
+                         "optimizer step on an 8-way owner shard of the table")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)      # at least 3 untimed warm-up steps
     if args.impl == "reference":
         return run_reference(args)
     if args.stage == "ple":
         return run_ple(args)
+    if args.stage == "adam":
+        return run_adam(args)
     return run_ours(args)
 
 
