@@ -22,6 +22,7 @@
 #include "ple_conv.cuh"
 #include "ple_conv_reg.cuh"
 #include "optim.cuh"
+#include "norm.cuh"
 
 using namespace engram;
 
@@ -845,6 +846,63 @@ int engram_grouped_rms_norm(const void *x, int32_t dtype, int64_t rows, int32_t 
         return ENGRAM_EINVAL;
     if (out == x && out_dtype != dtype)
         return ENGRAM_EINVAL;
+    const int eb = elem_bytes(dtype);
+    const int nvec = group_size * eb / 16;  // 16-byte vectors per group slice
+    if (nvec <= 32 * norm::kMaxVec) {
+        // the streaming kernel: a warp per group slice, scales in shared memory
+        int sms = 0;
+        ENGRAM_TRY(device_sms(&sms));
+        const int groups = channels / group_size;
+        int64_t bpg = std::max<int64_t>(1, ceil_div((int64_t)sms * 4, groups));
+        bpg = std::min<int64_t>(bpg, std::max<int64_t>(1, ceil_div(rows, 16)));
+        if ((int64_t)groups * bpg > INT32_MAX)
+            return ENGRAM_EINVAL;
+        norm::NormArgs na;
+        na.x = x;
+        na.out = out;
+        na.w = weight;
+        na.wdtype = weight_dtype;
+        na.rows = rows;
+        na.C = channels;
+        na.G = group_size;
+        na.bpg = (int32_t)bpg;
+        na.eps = eps;
+        na.inv_G = 1.f / (float)group_size;
+        const int need = (nvec + 31) / 32;
+        const size_t smem = (size_t)group_size * sizeof(float);
+        const unsigned grid = (unsigned)(groups * bpg);
+        cudaStream_t st = (cudaStream_t)stream;
+        auto go = [&](auto fn) {
+            ENGRAM_TRY(allow_smem(fn));
+            fn<<<grid, norm::kThreads, smem, st>>>(na);
+            return after_launch();
+        };
+        auto pick = [&](auto xt, auto ot) {
+            using XT = decltype(xt);
+            using OT = decltype(ot);
+            if (need <= 1)
+                return go(norm::norm_kernel<XT, OT, 1>);
+            if (need <= 2)
+                return go(norm::norm_kernel<XT, OT, 2>);
+            if (need <= 4)
+                return go(norm::norm_kernel<XT, OT, 4>);
+            if (need <= 8)
+                return go(norm::norm_kernel<XT, OT, 8>);
+            if (need <= 10)
+                return go(norm::norm_kernel<XT, OT, 10>);
+            return go(norm::norm_kernel<XT, OT, 16>);
+        };
+        const bool f32_out = out_dtype == ENGRAM_F32;
+        switch (dtype) {
+        case ENGRAM_F32:
+            return pick(float(), float());
+        case ENGRAM_BF16:
+            return f32_out ? pick(__nv_bfloat16(), float())
+                           : pick(__nv_bfloat16(), __nv_bfloat16());
+        default:
+            return f32_out ? pick(__half(), float()) : pick(__half(), __half());
+        }
+    }
     P.a.x = x;
     P.a.out = out;
     P.a.nseq = 1;

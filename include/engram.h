@@ -306,8 +306,9 @@ ENGRAM_API int engram_ple_short_conv(const engram_conv_params_t *params, const v
  *   out[r, c] = x[r, c] * rsqrt(mean over c's group of x[r, .]^2 + eps)
  *               * (1 + weight[c])
  * in fp32, rounded once to out_dtype (dtype or ENGRAM_F32). weight [channels]
- * of weight_dtype, NULL = zeros (the page's reset value). Same layout limits
- * as engram_ple_short_conv with K = 1.
+ * of weight_dtype, NULL = zeros (the page's reset value). out may be x itself
+ * (same dtype). Limits: channels % group_size == 0, group_size % 8 == 0,
+ * group_size <= 4096; x and out 16-byte aligned.
  */
 ENGRAM_API int engram_grouped_rms_norm(const void *x, int32_t dtype, int64_t rows,
                                        int32_t channels, int32_t group_size,
