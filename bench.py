@@ -359,14 +359,22 @@ def run_ours(args):
     # streams pipeline consecutive steps (copy-in, compute, copy-out, with two
     # sets of device buffers), so step k's results travel to the host while
     # step k+1 computes and PCIe carries both directions at once.
-    e2e = None
-    if fwd:
+    def run_e2e(full_readback: bool):
+        """End to end through the public API with host buffers: every step
+        copies its inputs (ids, cu_seqlens, dout) in from pinned host memory
+        and reads its result back: num_unique (the step's metric) or, with
+        full_readback, also out, uniq_rows[:U] and row_grads[:U]. Three
+        streams pipeline consecutive steps (copy-in, compute, copy-out, two
+        sets of device buffers)."""
         e2e_steps = max(1, min(K, args.e2e_steps))
         ids_h = torch.from_numpy(ids_np.copy()).pin_memory()
         cu_h = torch.from_numpy(cu_np.copy()).pin_memory()
-        host = [{"out": torch.empty(T, H * D, dtype=tdtype).pin_memory(),
-                 "uniq": torch.empty(n, dtype=torch.int32).pin_memory(),
-                 "grads": torch.empty(n, D, dtype=torch.float32).pin_memory(),
+        host = [{"out": torch.empty(T, H * D, dtype=tdtype).pin_memory() if full_readback
+                 else None,
+                 "uniq": torch.empty(n, dtype=torch.int32).pin_memory() if full_readback
+                 else None,
+                 "grads": torch.empty(n, D, dtype=torch.float32).pin_memory() if full_readback
+                 else None,
                  "nu": torch.empty(1, dtype=torch.int32).pin_memory()} for _ in range(2)]
         s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
         ev = lambda: torch.cuda.Event()  # noqa: E731
@@ -375,11 +383,15 @@ def run_ours(args):
         nu_done = [ev() for _ in range(e2e_steps)]
         out_done = [ev() for _ in range(e2e_steps)]
         h2d = ids_h.numel() * 4 + cu_h.numel() * 4 + dout_h.numel() * esize
-        d2h_bytes = [0] * e2e_steps
+        d2h_bytes = [4] * e2e_steps
 
         def drain(k):
             # rows of step k: the host needs num_unique before copying them out
             nu_done[k].synchronize()
+            if not full_readback:
+                with torch.cuda.stream(s_out):
+                    out_done[k].record(s_out)
+                return
             hb, b = host[k % 2], bufs[k % 2]
             u = int(hb["nu"].item())
             with torch.cuda.stream(s_out):
@@ -408,7 +420,8 @@ def run_ours(args):
             comp_done[k].record(stream)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(comp_done[k])
-                hb["out"].copy_(b["out"], non_blocking=True)
+                if full_readback:
+                    hb["out"].copy_(b["out"], non_blocking=True)
                 hb["nu"].copy_(b["nu"], non_blocking=True)
                 nu_done[k].record(s_out)
             if k >= 1:
@@ -418,11 +431,18 @@ def run_ours(args):
         torch.cuda.synchronize(device)
         e2e_ms = max_over_ranks(e0.elapsed_time(e1), device)
         barrier(device)
-        e2e = {"value": world * T * e2e_steps / (e2e_ms / 1e3), "unit": UNIT,
-               "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": int(statistics.mean(d2h_bytes)),
-               "steps": e2e_steps,
-               "pipeline": "copy-in / compute / copy-out streams, two buffer sets"}
+        return {"value": world * T * e2e_steps / (e2e_ms / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": int(statistics.mean(d2h_bytes)),
+                "steps": e2e_steps,
+                "readback": "out, uniq_rows[:U], row_grads[:U], num_unique" if full_readback
+                else "num_unique (the step's metric; out and the row gradients stay resident)",
+                "pipeline": "copy-in / compute / copy-out streams, two buffer sets"}
+
+    e2e = e2e_full = None
+    if fwd:
+        e2e = run_e2e(False)
+        e2e_full = run_e2e(True)
 
     if E.engram_get_device_error(stream):
         raise RuntimeError("device error flag set during timing")
@@ -474,6 +494,7 @@ def run_ours(args):
                      "traffic": committed_traffic(tkey, tunits)},
         "stages": stages,
         "e2e": e2e,
+        "e2e_full_readback": e2e_full,
         "gpu_launches": launches,
         "clocks": clocks,
     }
