@@ -1,6 +1,6 @@
 """CPU oracle of the Engram N-gram Embedding path (hash, gather, backward,
-the PLE layer's grouped RMS norm and causal short convolution, and the sparse
-optimizer step on the touched rows).
+the PLE layer's grouped RMS norm and causal short convolution with its
+backward, and the sparse optimizer step on the touched rows).
 
 TEST INFRASTRUCTURE ONLY. Only `tests/`, `__graft_entry__.smoke()` and the
 CPU-baseline / reference legs of `bench.py` may import this package. The
@@ -71,6 +71,10 @@ def _declare(L):
     d = ctypes.c_double
     L.oracle_sparse_adam.argtypes = [P, P, P, i64, i32, P, P, i64, d, d, d, d, d, i64]
     L.oracle_sparse_adam.restype = ctypes.c_int
+    L.oracle_short_conv_backward.argtypes = [P, ctypes.c_int, P, i32, i64, i32, i32, P, d, P, P,
+                                             ctypes.c_int, i32, i32, ctypes.c_int, ctypes.c_int,
+                                             ctypes.c_int, P, P, P, P, P]
+    L.oracle_short_conv_backward.restype = ctypes.c_int
     return L
 
 
@@ -215,3 +219,29 @@ def sparse_adam(p, m, v, rows, grads, *, lr, betas=(0.9, 0.999), eps=1e-8, weigh
     if rc != 0:
         raise ValueError("oracle_sparse_adam: invalid arguments")
     return p, m, v
+
+
+def short_conv_backward(x, dtype, cu, conv_w, dout, *, dilation, group=None, norm_w=None,
+                        eps=1e-6, bias=None, wdtype=F32, norm=True, silu=True, residual=True):
+    """Gradients of short_conv's output given dout (fp64 [T, C]): returns
+    (dx [T, C], dnorm_w [C], dconv_w [C, K], dbias [C]), all fp64."""
+    xr = _raw(x, dtype)
+    T, C = xr.shape
+    wr = _raw(conv_w, wdtype)
+    K = wr.shape[1]
+    nw, br = _raw(norm_w, wdtype), _raw(bias, wdtype)
+    if cu is None:
+        cu_arr, nseq, cu_p = None, 1, None
+    else:
+        cu_arr = np.ascontiguousarray(cu, dtype=np.int32)
+        nseq, cu_p = cu_arr.shape[0] - 1, _ptr(cu_arr)
+    g = np.ascontiguousarray(dout, dtype=np.float64)
+    dx = np.empty((T, C)); dnw = np.empty(C); dw = np.empty((C, K)); db = np.empty(C)
+    rc = lib().oracle_short_conv_backward(
+        _ptr(xr), dtype, cu_p, nseq, T, C, int(group if group else C),
+        None if nw is None else _ptr(nw), float(eps), _ptr(wr), None if br is None else _ptr(br),
+        wdtype, K, int(dilation), int(bool(norm)), int(bool(silu)), int(bool(residual)),
+        _ptr(g), _ptr(dx), _ptr(dnw), _ptr(dw), _ptr(db))
+    if rc != 0:
+        raise ValueError("oracle_short_conv_backward: invalid arguments")
+    return dx, dnw, dw, db

@@ -30,7 +30,10 @@
  *   - norm_conv normalises the convolution's input;
  *   - the convolution's history is zero before every start in cu_seqlens;
  *   - the optional SiLU and residual follow the Engram paper the page cites
- *     (output = x + SiLU(conv(norm(x)))); the page itself prints neither.
+ *     (output = x + SiLU(conv(norm(x)))); the page itself prints neither;
+ *   - the tail's backward (for training the layer) is the chain rule through
+ *     those same steps; the pages print no backward, so it has no reading of
+ *     its own beyond the forward's.
  *
  * Parity of the hash against the released checkpoint is unpinned: the page
  * prints no worked example (see the tests for what does pin each function).
@@ -419,5 +422,130 @@ int oracle_sparse_adam(double *p, double *m, double *v, int64_t rows, int32_t di
             p[i] -= lr / bc1 * m[i] / denom;
         }
     }
+    return ORACLE_OK;
+}
+
+/*
+ * Gradients of oracle_short_conv's output, given dout = dL/dout [T, C] (fp64),
+ * by the chain rule through the same steps in reverse:
+ *   dy[t,c]  = dout[t,c] * (do_silu ? s(y) (1 + y (1 - s(y))) : 1),  s = sigmoid
+ *   dbias[c] = sum_t dy[t,c]
+ *   for every tap k of row t that reads row src = t - k*dil (same sequence):
+ *     dconv_w[c, K-1-k] += dy[t,c] * n[src,c]
+ *     dn[src,c]         += conv_w[c, K-1-k] * dy[t,c]
+ *   norm on (n = xh * (1 + norm_w), xh = x * inv over each group of G):
+ *     dnorm_w[c] = sum_t dn[t,c] * xh[t,c]
+ *     dxh = dn * (1 + norm_w);  dx = inv * (dxh - xh * mean over the group(dxh * xh))
+ *   norm off: dx = dn;  residual: dx += dout.
+ * Outputs are fp64: dx [T, C], dnorm_w [C], dconv_w [C, K], dbias [C].
+ */
+int oracle_short_conv_backward(const void *x, int dtype, const int32_t *cu, int32_t nseq,
+                               int64_t T, int32_t C, int32_t G, const void *norm_w, double eps,
+                               const void *conv_w, const void *bias, int wdtype, int32_t K,
+                               int32_t dil, int do_norm, int do_silu, int do_residual,
+                               const double *dout, double *dx, double *dnorm_w, double *dconv_w,
+                               double *dbias)
+{
+    if (T < 0 || C <= 0 || K < 1 || dil < 1 || (do_norm && (G <= 0 || C % G != 0)))
+        return ORACLE_EINVAL;
+    if (cu && (nseq < 0 || cu[0] != 0 || cu[nseq] != T))
+        return ORACLE_EINVAL;
+    const size_t TC = (size_t)(T * C > 0 ? T * C : 1);
+    double *n = (double *)calloc(TC, sizeof(double));
+    double *xh = (double *)calloc(TC, sizeof(double));
+    double *dy = (double *)calloc(TC, sizeof(double));
+    double *dn = (double *)calloc(TC, sizeof(double));
+    double *inv = (double *)calloc((size_t)(T > 0 ? T : 1) * (size_t)(do_norm ? C / G : 1),
+                                   sizeof(double));
+    if (!n || !xh || !dy || !dn || !inv) {
+        free(n); free(xh); free(dy); free(dn); free(inv);
+        return ORACLE_EINVAL;
+    }
+    /* forward again: xh, n */
+    for (int64_t t = 0; t < T; ++t) {
+        if (do_norm) {
+            for (int32_t g0 = 0; g0 < C; g0 += G) {
+                double ss = 0.0;
+                for (int32_t c = g0; c < g0 + G; ++c) {
+                    const double v = load_value(x, dtype, t * C + c);
+                    ss += v * v;
+                }
+                const double iv = 1.0 / sqrt(ss / (double)G + eps);
+                inv[t * (C / G) + g0 / G] = iv;
+                for (int32_t c = g0; c < g0 + G; ++c) {
+                    xh[t * C + c] = load_value(x, dtype, t * C + c) * iv;
+                    n[t * C + c] = xh[t * C + c] *
+                                   (1.0 + (norm_w ? load_value(norm_w, wdtype, c) : 0.0));
+                }
+            }
+        } else {
+            for (int32_t c = 0; c < C; ++c)
+                n[t * C + c] = xh[t * C + c] = load_value(x, dtype, t * C + c);
+        }
+    }
+    for (int32_t c = 0; c < C; ++c) {
+        dbias[c] = 0.0;
+        dnorm_w[c] = 0.0;
+        for (int32_t k = 0; k < K; ++k)
+            dconv_w[c * K + k] = 0.0;
+    }
+    /* y, dy, and the convolution's gradients */
+    const int32_t ns = cu ? nseq : 1;
+    for (int32_t s = 0; s < ns; ++s) {
+        const int64_t begin = cu ? cu[s] : 0, end = cu ? cu[s + 1] : T;
+        for (int64_t t = begin; t < end; ++t) {
+            for (int32_t c = 0; c < C; ++c) {
+                double y = bias ? load_value(bias, wdtype, c) : 0.0;
+                for (int32_t k = 0; k < K && t - (int64_t)k * dil >= begin; ++k)
+                    y += load_value(conv_w, wdtype, (int64_t)c * K + K - 1 - k) *
+                         n[(t - (int64_t)k * dil) * C + c];
+                double g = dout[t * C + c];
+                if (do_silu) {
+                    const double sg = 1.0 / (1.0 + exp(-y));
+                    g *= ORACLE_MUTANT == 18 ? sg : sg * (1.0 + y * (1.0 - sg));
+                }
+                dy[t * C + c] = g;
+                dbias[c] += g;
+                for (int32_t k = 0; k < K && t - (int64_t)k * dil >= begin; ++k) {
+                    const int64_t src = t - (int64_t)k * dil;
+                    const double w = load_value(conv_w, wdtype, (int64_t)c * K + K - 1 - k);
+                    dconv_w[(int64_t)c * K + K - 1 - k] += g * n[src * C + c];
+                    if (ORACLE_MUTANT == 19) {
+                        /* mutant: the taps' gradient sent forward instead of back */
+                        if (t + (int64_t)k * dil < end)
+                            dn[(t + (int64_t)k * dil) * C + c] += w * g;
+                    } else {
+                        dn[src * C + c] += w * g;
+                    }
+                }
+            }
+        }
+    }
+    /* the norm's gradients, then the residual */
+    for (int64_t t = 0; t < T; ++t) {
+        if (do_norm) {
+            for (int32_t g0 = 0; g0 < C; g0 += G) {
+                double dot = 0.0;
+                for (int32_t c = g0; c < g0 + G; ++c) {
+                    const double sc = 1.0 + (norm_w ? load_value(norm_w, wdtype, c) : 0.0);
+                    dnorm_w[c] += dn[t * C + c] * xh[t * C + c];
+                    dot += dn[t * C + c] * sc * xh[t * C + c];
+                }
+                const double mean = ORACLE_MUTANT == 20 ? 0.0 : dot / (double)G;
+                const double iv = inv[t * (C / G) + g0 / G];
+                for (int32_t c = g0; c < g0 + G; ++c) {
+                    const double sc = 1.0 + (norm_w ? load_value(norm_w, wdtype, c) : 0.0);
+                    dx[t * C + c] = iv * (dn[t * C + c] * sc - xh[t * C + c] * mean);
+                }
+            }
+        } else {
+            for (int32_t c = 0; c < C; ++c)
+                dx[t * C + c] = dn[t * C + c];
+        }
+        if (do_residual)
+            for (int32_t c = 0; c < C; ++c)
+                dx[t * C + c] += dout[t * C + c];
+    }
+    free(n); free(xh); free(dy); free(dn); free(inv);
     return ORACLE_OK;
 }

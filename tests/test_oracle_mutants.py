@@ -4,10 +4,12 @@ Each mutant is the oracle rebuilt with one known mistake (ORACLE_MUTANT in
 engram_oracle.c): a plausible slip in the hash (operator, reset position,
 multiplier pairing, remainder sign, sequence reset), in the backward
 (accumulation precision, grouping) or in the PLE norm and convolution (scale,
-group width, epsilon, dilation, tap order, history reset, residual) or in the
+group width, epsilon, dilation, tap order, history reset, residual), in its
+backward (SiLU derivative, tap direction, the norm's mean term) or in the
 optimizer step (bias correction, epsilon, weight decay). The pins of
-test_oracle_hash.py, test_oracle_gather_backward.py, test_oracle_ple.py and
-test_oracle_adam.py are run against each; at least one must fail.
+test_oracle_hash.py, test_oracle_gather_backward.py, test_oracle_ple.py,
+test_oracle_ple_backward.py and test_oracle_adam.py are run against each; at
+least one must fail.
 """
 
 import pytest
@@ -17,6 +19,7 @@ from tests import test_oracle_adam as AD
 from tests import test_oracle_gather_backward as GB
 from tests import test_oracle_hash as TH
 from tests import test_oracle_ple as PL
+from tests import test_oracle_ple_backward as PB
 
 HASH_PINS = [
     TH.test_hand_worked_example,
@@ -48,6 +51,14 @@ PLE_PINS = [
     PL.test_sequences_are_independent,
 ]
 
+PLE_BWD_PINS = [
+    lambda: [PB.test_matches_torch_autograd(*c) for c in PB.CASES],
+    lambda: [PB.test_finite_differences(s) for s in range(3)],
+    PB.test_linear_convolution_adjoint_and_bilinear_form,
+    PB.test_transposed_impulse_response,
+    PB.test_norm_input_gradient_orthogonal_to_each_group,
+]
+
 ADAM_PINS = [
     AD.test_first_step_closed_form,
     lambda: [AD.test_matches_torch_adamw_when_all_rows_present(wd) for wd in (0.0, 0.05)],
@@ -72,6 +83,9 @@ MUTANTS = {
     15: ("no bias correction", ADAM_PINS),
     16: ("eps inside the square root", ADAM_PINS),
     17: ("L2 penalty instead of decoupled decay", ADAM_PINS),
+    18: ("SiLU derivative taken as the sigmoid", PLE_BWD_PINS),
+    19: ("conv gradient sent forward along the taps", PLE_BWD_PINS),
+    20: ("norm backward without the mean term", PLE_BWD_PINS),
 }
 
 
