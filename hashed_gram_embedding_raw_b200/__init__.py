@@ -1,6 +1,6 @@
 """B200-native Engram N-gram Embedding: hash, gather, compact backward, the
 sparse optimizer step on the touched rows, and the PLE layer's grouped RMS
-norm and causal short convolution.
+norm and causal short convolution with its backward.
 
 Python face of the C ABI in include/engram.h (libengram_b200.so, sm_100a).
 Every step runs in the library's CUDA kernels; this package only marshals
@@ -19,7 +19,8 @@ from ._binding import (ENGRAM_BF16, ENGRAM_CONV_NORM, ENGRAM_CONV_RESIDUAL, ENGR
                        engram_backward_workspace_size, engram_gather, engram_get_device_error,
                        engram_grouped_rms_norm, engram_hash, engram_hash_gather,
                        engram_hash_gather_slice, engram_host_floor_mod, engram_ple_short_conv,
-                       engram_sparse_adam,
+                       engram_ple_short_conv_backward,
+                       engram_ple_short_conv_backward_workspace_size, engram_sparse_adam,
                        engram_launch_count, lib, make_params, status_string)
 
 __all__ = [
@@ -32,6 +33,7 @@ __all__ = [
     "engram_backward_reduce", "engram_backward_sort", "engram_backward_workspace_size",
     "engram_gather", "engram_get_device_error", "engram_hash", "engram_hash_gather",
     "engram_hash_gather_slice", "engram_grouped_rms_norm", "engram_ple_short_conv",
+    "engram_ple_short_conv_backward", "engram_ple_short_conv_backward_workspace_size",
     "engram_sparse_adam",
     "engram_host_floor_mod", "engram_launch_count", "lib", "make_params", "status_string",
 ]

@@ -34,6 +34,7 @@ EXPORTED = (
     "engram_abi_version", "engram_params_size", "engram_launch_count",
     "engram_host_floor_mod", "engram_backward_noalloc", "engram_hash_gather_slice",
     "engram_ple_short_conv", "engram_grouped_rms_norm", "engram_sparse_adam",
+    "engram_ple_short_conv_backward", "engram_ple_short_conv_backward_workspace_size",
 )
 
 ENGRAM_NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -138,6 +139,9 @@ def _load():
         "engram_ple_short_conv": [P, P, i32, P, i32, i64, P, P, P, P, i32, P],
         "engram_grouped_rms_norm": [P, i32, i64, i32, i32, P, i32, ctypes.c_float, P, i32, P],
         "engram_sparse_adam": [P, P, i32, i64, i32, P, P, P, P, P, i64, P],
+        "engram_ple_short_conv_backward": [P, P, i32, P, i32, i64, P, P, P, P, i32, P, P, P, P,
+                                           P, sz, P],
+        "engram_ple_short_conv_backward_workspace_size": [P, i64, ctypes.POINTER(sz)],
     }
     for name, args in sig.items():
         fn = getattr(L, name)
@@ -424,6 +428,75 @@ def engram_ple_short_conv(x: torch.Tensor, conv_weight: torch.Tensor, *, dilatio
                                      _dtype_code(out), _stream(stream)),
            "engram_ple_short_conv")
     return out
+
+
+def _conv_params(C, group_size, w, dilation, eps, norm, silu, residual):
+    return ConvParams(C, int(group_size), w.shape[1], int(dilation), float(eps),
+                      (ENGRAM_CONV_NORM if norm else 0) | (ENGRAM_CONV_SILU if silu else 0)
+                      | (ENGRAM_CONV_RESIDUAL if residual else 0), _dtype_code(w), 0)
+
+
+def engram_ple_short_conv_backward_workspace_size(channels: int, group_size: int,
+                                                  kernel_size: int, dilation: int,
+                                                  tokens: int) -> int:
+    """Workspace bytes of engram_ple_short_conv_backward on the current device."""
+    p = ConvParams(int(channels), int(group_size), int(kernel_size), int(dilation), 1e-6,
+                   ENGRAM_CONV_NORM | ENGRAM_CONV_SILU | ENGRAM_CONV_RESIDUAL, ENGRAM_F32, 0)
+    n = ctypes.c_size_t(0)
+    _check(lib.engram_ple_short_conv_backward_workspace_size(ctypes.byref(p), int(tokens),
+                                                             ctypes.byref(n)),
+           "engram_ple_short_conv_backward_workspace_size")
+    return n.value
+
+
+def engram_ple_short_conv_backward(x: torch.Tensor, conv_weight: torch.Tensor,
+                                   dout: torch.Tensor, *, dilation: int, group_size: int,
+                                   cu_seqlens=None, norm_weight=None, conv_bias=None,
+                                   eps: float = 1e-6, norm: bool = True, silu: bool = True,
+                                   residual: bool = True, dx=None, dnorm_weight=None,
+                                   dconv_weight=None, dconv_bias=None, workspace=None,
+                                   stream=None):
+    """Gradients of engram_ple_short_conv's output given dout [T, C]:
+    returns (dx [T, C] of dout's dtype, dnorm_weight [C], dconv_weight [C, K],
+    dconv_bias [C]), the weight gradients fp32. Optional outputs and the
+    workspace (uint8) may be passed in; they are allocated otherwise."""
+    _cuda(x, "x")
+    _cuda(dout, "dout")
+    if x.dim() != 2 or dout.shape != x.shape:
+        raise ValueError("x and dout must both be [T, C]")
+    T, C = x.shape
+    w = conv_weight.reshape(C, -1) if conv_weight.dim() == 3 else conv_weight
+    _cuda(w, "conv_weight")
+    if w.shape[0] != C:
+        raise ValueError("conv_weight must be [C, K]")
+    K = w.shape[1]
+    for name, t in (("norm_weight", norm_weight), ("conv_bias", conv_bias)):
+        if t is not None:
+            _cuda(t, name, w.dtype)
+            if t.numel() != C:
+                raise ValueError(f"{name} must hold C elements")
+    cu, nseq = _cu_args(cu_seqlens)
+    dev = x.device
+    dx = _out_like(dout, dx, None)
+    dnorm_weight = torch.empty(C, device=dev) if dnorm_weight is None else dnorm_weight
+    dconv_weight = torch.empty((C, K), device=dev) if dconv_weight is None else dconv_weight
+    dconv_bias = torch.empty(C, device=dev) if dconv_bias is None else dconv_bias
+    for name, t, n in (("dnorm_weight", dnorm_weight, C), ("dconv_weight", dconv_weight, C * K),
+                       ("dconv_bias", dconv_bias, C)):
+        _cuda(t, name, torch.float32)
+        if t.numel() != n:
+            raise ValueError(f"{name} must hold {n} elements")
+    p = _conv_params(C, group_size, w, dilation, eps, norm, silu, residual)
+    if workspace is None:
+        need = engram_ple_short_conv_backward_workspace_size(C, group_size, K, dilation, T)
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    _cuda(workspace, "workspace", torch.uint8)
+    _check(lib.engram_ple_short_conv_backward(
+        ctypes.byref(p), _ptr(x), _dtype_code(x), _ptr(cu), nseq, T, _ptr(norm_weight), _ptr(w),
+        _ptr(conv_bias), _ptr(dout), _dtype_code(dout), _ptr(dx), _ptr(dnorm_weight),
+        _ptr(dconv_weight), _ptr(dconv_bias), _ptr(workspace), workspace.numel(),
+        _stream(stream)), "engram_ple_short_conv_backward")
+    return dx, dnorm_weight, dconv_weight, dconv_bias
 
 
 def engram_grouped_rms_norm(x: torch.Tensor, group_size: int, weight=None, eps: float = 1e-6,

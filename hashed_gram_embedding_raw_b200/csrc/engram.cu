@@ -21,6 +21,7 @@
 #include "hash_gather.cuh"
 #include "ple_conv.cuh"
 #include "ple_conv_reg.cuh"
+#include "ple_conv_bwd.cuh"
 #include "optim.cuh"
 #include "norm.cuh"
 
@@ -908,6 +909,186 @@ int engram_grouped_rms_norm(const void *x, int32_t dtype, int64_t rows, int32_t 
     P.a.nseq = 1;
     P.a.norm_w = weight;
     return launch_conv(P, dtype, out_dtype, (cudaStream_t)stream);
+}
+
+} // extern "C"
+
+// ------------------------------------------------- PLE layer tail backward
+
+namespace {
+
+struct ConvBwdPlan {
+    ple::ConvBwdArgs a;
+    size_t smem = 0, ws = 0;
+    int grid = 0, threads = 0, npart = 0;
+};
+
+// Checks the shape (host only) and sizes the launch: G / 8 threads, a ring of
+// row slots as deep as shared memory allows (at most 32, at least 11), and
+// one block per (branch, residue, chunk) with chunks chosen so that one wave
+// covers the multiprocessors.
+int conv_bwd_plan(const engram_conv_params_t *p, int32_t dtype, int32_t grad_dtype, int64_t T,
+                  ConvBwdPlan *P)
+{
+    if (p == nullptr)
+        return ENGRAM_EINVAL;
+    const int ex = elem_bytes(dtype), eg = elem_bytes(grad_dtype);
+    if (ex == 0 || eg == 0 || elem_bytes(p->weight_dtype) == 0)
+        return ENGRAM_EINVAL;
+    const int C = p->channels, G = p->group_size, K = p->kernel_size, d = p->dilation;
+    if (C < 1 || G < 8 || C % G != 0 || G % 8 != 0 || G / 8 > ple::kBwdThreads)
+        return ENGRAM_EINVAL;
+    if (K < 1 || K > ple::kBwdTaps || d < 1 || d > 4096 || p->reserved != 0)
+        return ENGRAM_EINVAL;
+    if (!std::isfinite(p->eps) || p->eps < 0.f || (p->flags & ~7u) != 0)
+        return ENGRAM_EINVAL;
+    if (T < 0 || T > INT32_MAX)
+        return ENGRAM_EINVAL;
+    const int pitch_x = (G * ex + 127) / 128 * 128, pitch_g = (G * eg + 127) / 128 * 128;
+    const int fit = (int)((ple::kSmemLimit - ple::kBwdDataOffset) / (size_t)(pitch_x + pitch_g));
+    const int slots_max = std::min(fit, ple::kBwdMaxSlots);
+    const int ahead = std::min((slots_max - ple::kBwdLag) / ple::kBwdRows - 1, ple::kBwdBars - 2);
+    if (ahead < 1)
+        return ENGRAM_EINVAL;
+    ple::ConvBwdArgs &a = P->a;
+    std::memset(&a, 0, sizeof(a));
+    a.T = T;
+    a.C = C;
+    a.G = G;
+    a.nth = G / 8;
+    a.dil = d;
+    a.K = K;
+    a.wdtype = p->weight_dtype;
+    a.eps = p->eps;
+    a.inv_G = 1.f / (float)G;
+    a.flags = p->flags;
+    a.ahead = ahead;
+    a.slots = ple::kBwdLag + (ahead + 1) * ple::kBwdRows;
+    a.pitch_x = pitch_x;
+    a.pitch_g = pitch_g;
+    P->smem = ple::bwd_smem_bytes(a.slots, pitch_x, pitch_g);
+    P->threads = (a.nth + 31) / 32 * 32;
+    return ENGRAM_OK;
+}
+
+// Grid and workspace of a checked plan on the current device.
+int conv_bwd_grid(ConvBwdPlan *P)
+{
+    ple::ConvBwdArgs &a = P->a;
+    int sms = 0;
+    ENGRAM_TRY(device_sms(&sms));
+    const int groups = a.C / a.G;
+    const int classes = (int)std::max<int64_t>(1, std::min<int64_t>(a.dil, a.T));
+    const int64_t rows = std::max<int64_t>(1, ceil_div(a.T, a.dil));  // rows of residue 0
+    int64_t chunks = std::max<int64_t>(1, sms / ((int64_t)groups * classes));
+    chunks = std::min<int64_t>(chunks, std::max<int64_t>(1, ceil_div(rows, 16)));
+    const int64_t grid = (int64_t)groups * classes * chunks;
+    if (grid > INT32_MAX)
+        return ENGRAM_EINVAL;
+    a.chunks = (int32_t)chunks;
+    P->grid = (int)grid;
+    P->npart = (int)(classes * chunks);
+    P->ws = (size_t)P->npart * ple::kBwdQuantities * (size_t)a.C * sizeof(float);
+    return ENGRAM_OK;
+}
+
+template <typename XT, typename GT>
+int launch_conv_bwd_t(const ConvBwdPlan &P, cudaStream_t s)
+{
+    auto fn = ple::short_conv_bwd_kernel<XT, GT>;
+    ENGRAM_TRY(allow_smem(fn));
+    fn<<<P.grid, P.threads, P.smem, s>>>(P.a);
+    return after_launch();
+}
+
+template <typename XT>
+int launch_conv_bwd_x(const ConvBwdPlan &P, int32_t grad_dtype, cudaStream_t s)
+{
+    switch (grad_dtype) {
+    case ENGRAM_F32:
+        return launch_conv_bwd_t<XT, float>(P, s);
+    case ENGRAM_BF16:
+        return launch_conv_bwd_t<XT, __nv_bfloat16>(P, s);
+    default:
+        return launch_conv_bwd_t<XT, __half>(P, s);
+    }
+}
+
+} // namespace
+
+extern "C" {
+
+int engram_ple_short_conv_backward_workspace_size(const engram_conv_params_t *params, int64_t T,
+                                                  size_t *bytes)
+{
+    if (bytes == nullptr)
+        return ENGRAM_EINVAL;
+    ConvBwdPlan P;
+    ENGRAM_TRY(conv_bwd_plan(params, ENGRAM_BF16, ENGRAM_BF16, T, &P));
+    ENGRAM_TRY(conv_bwd_grid(&P));
+    *bytes = P.ws;
+    return ENGRAM_OK;
+}
+
+int engram_ple_short_conv_backward(const engram_conv_params_t *params, const void *x,
+                                   int32_t dtype, const int32_t *cu_seqlens, int32_t nseq,
+                                   int64_t T, const void *norm_weight, const void *conv_weight,
+                                   const void *conv_bias, const void *dout, int32_t grad_dtype,
+                                   void *dx, float *dnorm_weight, float *dconv_weight,
+                                   float *dconv_bias, void *workspace, size_t workspace_bytes,
+                                   engram_stream_t stream)
+{
+    ConvBwdPlan P;
+    ENGRAM_TRY(conv_bwd_plan(params, dtype, grad_dtype, T, &P));
+    if (cu_seqlens != nullptr && nseq < 1)
+        return ENGRAM_EINVAL;
+    if (conv_weight == nullptr || dconv_weight == nullptr)
+        return ENGRAM_EINVAL;
+    const int C = params->channels, K = params->kernel_size;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (T > 0) {
+        if (x == nullptr || dout == nullptr || dx == nullptr || !aligned16(x) ||
+            !aligned16(dout) || !aligned16(dx))
+            return ENGRAM_EINVAL;
+        const size_t n = (size_t)T * C;
+        const size_t nx = n * elem_bytes(dtype), ng = n * elem_bytes(grad_dtype);
+        if (overlaps(dx, ng, x, nx) || overlaps(dx, ng, dout, ng))
+            return ENGRAM_EINVAL;
+        if (workspace == nullptr || !aligned16(workspace))
+            return ENGRAM_EINVAL;
+        ENGRAM_TRY(conv_bwd_grid(&P));
+        if (workspace_bytes < P.ws)
+            return ENGRAM_ENOSPC;
+        P.a.x = x;
+        P.a.dout = dout;
+        P.a.dx = dx;
+        P.a.partial = static_cast<float *>(workspace);
+        P.a.cu = cu_seqlens;
+        P.a.nseq = cu_seqlens != nullptr ? nseq : 1;
+        P.a.norm_w = norm_weight;
+        P.a.conv_w = conv_weight;
+        P.a.bias = conv_bias;
+        switch (dtype) {
+        case ENGRAM_F32:
+            ENGRAM_TRY(launch_conv_bwd_x<float>(P, grad_dtype, s));
+            break;
+        case ENGRAM_BF16:
+            ENGRAM_TRY(launch_conv_bwd_x<__nv_bfloat16>(P, grad_dtype, s));
+            break;
+        default:
+            ENGRAM_TRY(launch_conv_bwd_x<__half>(P, grad_dtype, s));
+            break;
+        }
+    }
+    // weight gradients: sum of the blocks' partials (zeros when T = 0)
+    int sms = 0;
+    ENGRAM_TRY(device_sms(&sms));
+    const int64_t work = (int64_t)ple::kBwdQuantities * C;
+    const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>(ceil_div(work, 256), sms * 4));
+    ple::conv_bwd_reduce_kernel<<<blocks, 256, 0, s>>>(
+        static_cast<const float *>(workspace), T > 0 ? P.npart : 0, C, K, dconv_weight,
+        dconv_bias, dnorm_weight);
+    return after_launch();
 }
 
 } // extern "C"

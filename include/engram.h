@@ -300,6 +300,50 @@ ENGRAM_API int engram_ple_short_conv(const engram_conv_params_t *params, const v
                                      void *out, int32_t out_dtype, engram_stream_t stream);
 
 /*
+ * engram_ple_short_conv_backward -- gradients of engram_ple_short_conv's
+ * output (same params, x, cu_seqlens and weights) for training the layer. The
+ * pages print no backward; it is the chain rule through the forward's steps.
+ * With xh = x * inv (inv the slice's rsqrt as above), s = 1 + norm_weight,
+ * n = s * xh, and dout = dL/dout:
+ *   dy      = dout * (sg + y * sg * (1 - sg)), sg = sigmoid(y)
+ *             (ENGRAM_CONV_SILU; else dy = dout)
+ *   dn[t]   = sum over k < K with t + k*d in t's sequence of
+ *             conv_weight[c, K - 1 - k] * dy[t + k*d]
+ *   dx      = inv * (s * dn - xh * mean over the slice of (s * dn * xh))
+ *             (ENGRAM_CONV_NORM; else dx = dn), then + dout (ENGRAM_CONV_RESIDUAL)
+ *   dconv_weight[c, K - 1 - k] = sum over t of dy[t + k*d] * n[t]   (same pairs)
+ *   dconv_bias[c]   = sum over t of dy[t]
+ *   dnorm_weight[c] = sum over t of dn[t] * xh[t]    (0 without ENGRAM_CONV_NORM)
+ * computed in fp32; dx rounded once to grad_dtype, the weight gradients
+ * summed per block and then over blocks in a fixed order (results do not
+ * depend on timing).
+ *   dout          device, [T, C] of grad_dtype (F32 | BF16 | F16), 16-byte aligned
+ *   dx            device, [T, C] of grad_dtype, 16-byte aligned, overlapping
+ *                 neither x nor dout
+ *   dconv_weight  device, fp32 [C, K]
+ *   dconv_bias    device, fp32 [C], or NULL (not wanted)
+ *   dnorm_weight  device, fp32 [C], or NULL (not wanted)
+ *   workspace     device, >= engram_ple_short_conv_backward_workspace_size
+ *                 bytes, 16-byte aligned (per-block partial sums; overwritten)
+ * Limits (else ENGRAM_EINVAL): those of engram_conv_params_t, K <= 4,
+ * G <= 2560, and a ring of 11 row slots -- G elements of dtype plus G of
+ * grad_dtype, each rounded up to 128 bytes -- within 227 KB of shared memory
+ * (every dtype pair fits up to G = 2560). Two launches; T = 0 writes zero
+ * weight gradients.
+ */
+ENGRAM_API int engram_ple_short_conv_backward(
+    const engram_conv_params_t *params, const void *x, int32_t dtype,
+    const int32_t *cu_seqlens, int32_t nseq, int64_t T, const void *norm_weight,
+    const void *conv_weight, const void *conv_bias, const void *dout, int32_t grad_dtype,
+    void *dx, float *dnorm_weight, float *dconv_weight, float *dconv_bias, void *workspace,
+    size_t workspace_bytes, engram_stream_t stream);
+
+/* Workspace bytes engram_ple_short_conv_backward needs for T tokens on the
+ * current device (it depends on the device's multiprocessor count). */
+ENGRAM_API int engram_ple_short_conv_backward_workspace_size(
+    const engram_conv_params_t *params, int64_t T, size_t *bytes);
+
+/*
  * engram_grouped_rms_norm -- Qwen3_8_FlashNextGroupedRMSNorm.forward over
  * `rows` rows of `channels` features: every group of group_size consecutive
  * features is normalised on its own,

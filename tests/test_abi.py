@@ -180,6 +180,47 @@ def test_host_rejects_bad_conv_args(E):
     assert N(al, 1, 0, 96, 32, None, 0, 1e-6, al, 1, None) == E.ENGRAM_OK
 
 
+def test_host_rejects_bad_conv_backward_args(E):
+    L = E.lib
+    al, al2, al3 = ctypes.c_void_p(256), ctypes.c_void_p(1 << 30), ctypes.c_void_p(1 << 31)
+    mis = ctypes.c_void_p(264)
+    ws = ctypes.c_void_p(1 << 32)
+
+    def params(**kw):
+        base = dict(channels=10240, group_size=2560, kernel_size=4, dilation=3, eps=1e-6,
+                    flags=7, weight_dtype=1, reserved=0)
+        base.update(kw)
+        return E.ConvParams(**base)
+
+    def bwd(p, x=al, dtype=1, cu=None, nseq=1, T=100, dout=al2, gdt=1, dx=al3, dw=al,
+            work=ws):
+        return L.engram_ple_short_conv_backward(ctypes.byref(p), x, dtype, cu, nseq, T, None,
+                                                al, None, dout, gdt, dx, None, dw, None, work,
+                                                1 << 30, None)
+
+    for bad in (dict(group_size=12), dict(group_size=2568, channels=2568),
+                dict(channels=7680 + 100), dict(kernel_size=0), dict(kernel_size=5),
+                dict(dilation=0), dict(eps=-1.0), dict(eps=float("nan")), dict(flags=8),
+                dict(weight_dtype=5), dict(reserved=1)):
+        assert bwd(params(**bad)) == E.ENGRAM_EINVAL, bad
+    p = params()
+    assert bwd(p, dtype=7) == E.ENGRAM_EINVAL
+    assert bwd(p, gdt=7) == E.ENGRAM_EINVAL
+    assert bwd(p, T=-1) == E.ENGRAM_EINVAL
+    assert bwd(p, cu=al, nseq=0) == E.ENGRAM_EINVAL
+    assert bwd(p, x=mis) == E.ENGRAM_EINVAL
+    assert bwd(p, dout=mis) == E.ENGRAM_EINVAL
+    assert bwd(p, dx=mis) == E.ENGRAM_EINVAL
+    assert bwd(p, x=None) == E.ENGRAM_EINVAL
+    assert bwd(p, dw=None) == E.ENGRAM_EINVAL
+    assert bwd(p, work=None) == E.ENGRAM_EINVAL
+    assert bwd(p, dx=ctypes.c_void_p((1 << 30) + 4096)) == E.ENGRAM_EINVAL  # overlaps dout
+    assert bwd(p, dx=ctypes.c_void_p(256 + 4096)) == E.ENGRAM_EINVAL        # overlaps x
+    assert L.engram_ple_short_conv_backward_workspace_size(
+        ctypes.byref(params(kernel_size=5)), 100, ctypes.byref(ctypes.c_size_t())) == \
+        E.ENGRAM_EINVAL
+
+
 def test_host_rejects_bad_adam_args(E):
     L = E.lib
     a16, a8 = ctypes.c_void_p(1 << 20), ctypes.c_void_p((1 << 21) + 8)
