@@ -8,6 +8,7 @@ gradients) over one batch of the named workload, all inputs resident in HBM.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload full]
     python bench.py --impl reference ...   # the CPU oracle, timed on this host
     python bench.py --stage ple ...        # the PLE tail kernel on its own workload
+    python bench.py --stage ple_bwd ...    # the PLE tail's backward on the same workload
     python bench.py --stage adam ...       # the sparse optimizer step on a table shard
 
 Multi-GPU (torchrun, one rank per GPU): every rank holds its own table
@@ -217,11 +218,12 @@ def run_reference(args):
     if rank != 0:
         return 0
     name = args.workload
-    ple, adam = args.stage == "ple", args.stage == "adam"
+    ple, adam = args.stage in ("ple", "ple_bwd"), args.stage == "adam"
+    ple_bwd = args.stage == "ple_bwd"
     if adam:
         run = adam_oracle_run
     elif ple:
-        run = ple_oracle_run
+        run = lambda S: ple_oracle_run(S, backward=ple_bwd)  # noqa: E731
     else:
         run = lambda S: oracle_run(name, S)  # noqa: E731
     # calibrate, then size each step's sample so W + K steps take ~2 minutes
@@ -237,11 +239,13 @@ def run_reference(args):
     total = sum(times)
     value = S * len(times) / total
     if ple:
-        name = "ple_full"
+        name = "ple_full_bwd" if ple_bwd else "ple_full"
     if adam:
         name = "adam_shard"
+    metric = (ADAM_METRIC if adam else PLE_BWD_METRIC if ple_bwd else PLE_METRIC if ple
+              else METRIC)
     line = {
-        "impl": "reference", "metric": ADAM_METRIC if adam else PLE_METRIC if ple else METRIC,
+        "impl": "reference", "metric": metric,
         "value": value, "unit": "rows/s" if adam else UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * total / len(times), "higher_is_better": True,
@@ -543,19 +547,32 @@ PLE_METRIC = ("PLE tail tokens/s (grouped RMS norm + causal depthwise conv + SiL
               "over hc_count x hidden channels); achieved HBM GB/s vs peak")
 
 
-def ple_oracle_run(S: int, reps_seconds: float = 0.0, max_reps: int = 1):
-    """Time the CPU oracle of the PLE tail on S tokens (one sequence) of the
-    page's channel shape. Returns (tokens/s, seconds, reps, description)."""
+PLE_BWD_METRIC = ("PLE tail backward tokens/s (dx and the norm-scale, conv-weight and bias "
+                  "gradients of norm + causal depthwise conv + SiLU + residual over hc_count x "
+                  "hidden channels); achieved HBM GB/s vs peak")
+
+
+def ple_oracle_run(S: int, reps_seconds: float = 0.0, max_reps: int = 1,
+                   backward: bool = False):
+    """Time the CPU oracle of the PLE tail (or of its backward) on S tokens (one
+    sequence) of the page's channel shape. Returns (tokens/s, seconds, reps,
+    description)."""
     import oracle
     from workloads import PLE_SHAPES, ple_inputs
 
     s = PLE_SHAPES["ple_full"]
     x, nw, w, b = ple_inputs(S, s.channels, s.kernel, s.seed, s.dtype)
+    dout = np.random.default_rng(s.seed).standard_normal((S, s.channels)) if backward else None
     oracle.lib()
     reps, t0 = 0, time.perf_counter()
     while True:
-        out = oracle.short_conv(x, oracle.BF16, None, w, dilation=s.dilation, group=s.group,
-                                norm_w=nw, bias=b, wdtype=oracle.BF16)
+        if backward:
+            out = oracle.short_conv_backward(x, oracle.BF16, None, w, dout, dilation=s.dilation,
+                                             group=s.group, norm_w=nw, bias=b,
+                                             wdtype=oracle.BF16)[0]
+        else:
+            out = oracle.short_conv(x, oracle.BF16, None, w, dilation=s.dilation,
+                                    group=s.group, norm_w=nw, bias=b, wdtype=oracle.BF16)
         reps += 1
         el = time.perf_counter() - t0
         if reps >= max_reps or el >= reps_seconds:
@@ -563,13 +580,15 @@ def ple_oracle_run(S: int, reps_seconds: float = 0.0, max_reps: int = 1):
     assert out.shape == (S, s.channels)
     desc = (f"{S} tokens x {s.channels} channels (one sequence, the page's 4 x 2,560 "
             f"branches, kernel {s.kernel}, dilation {s.dilation}) x {reps} rep(s); "
-            f"single-threaded C oracle in fp64")
+            f"single-threaded C oracle in fp64{' (backward)' if backward else ''}")
     return S * reps / el, el, reps, desc
 
 
-def run_ple(args):
+def run_ple(args, backward: bool = False):
     """--stage ple: engram_ple_short_conv on the page's PLE shape at the full
-    workload's batch (16 x 4,096 tokens, C = 4 x 2,560 bf16)."""
+    workload's batch (16 x 4,096 tokens, C = 4 x 2,560 bf16); --stage ple_bwd:
+    engram_ple_short_conv_backward (dx and the weight gradients, two launches)
+    on the same shape with a bf16 dout."""
     import torch
 
     import hashed_gram_embedding_raw_b200 as E
@@ -586,6 +605,10 @@ def run_ple(args):
                                 timeout=datetime.timedelta(seconds=300))
     s = PLE_SHAPES["ple_full"]
     T, C, G, K, d = s.tokens, s.channels, s.group, s.kernel, s.dilation
+    batch = s.batch
+    if args.ple_tokens:      # a smaller case of the same shape (whole rows), for profiling
+        batch = max(1, args.ple_tokens // s.seq_len)
+        T = batch * s.seq_len
     g = torch.Generator(device=device).manual_seed(5000 + s.seed)
     x = torch.randn((T, C), generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
     _, nw_h, w_h, b_h = ple_inputs(1, C, K, s.seed, s.dtype)
@@ -594,13 +617,25 @@ def run_ple(args):
         return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(device)
 
     nw, w, b = bf(nw_h), bf(w_h), bf(b_h)
-    cu = torch.from_numpy(row_bounds(s.batch, s.seq_len)).to(device)
+    cu = torch.from_numpy(row_bounds(batch, s.seq_len)).to(device)
     out = torch.empty_like(x)
     stream = torch.cuda.Stream(device)
+    if backward:
+        dout = torch.randn((T, C), generator=g, device=device).to(torch.bfloat16)
+        dnw, db = torch.empty(C, device=device), torch.empty(C, device=device)
+        dw = torch.empty((C, K), device=device)
+        ws = torch.empty(E.engram_ple_short_conv_backward_workspace_size(C, G, K, d, T),
+                         dtype=torch.uint8, device=device)
 
-    def step(xx=x, oo=out):
-        E.engram_ple_short_conv(xx, w, dilation=d, group_size=G, cu_seqlens=cu,
-                                norm_weight=nw, conv_bias=b, out=oo, stream=stream)
+    def step(xx=x, oo=out, gg=None):
+        if backward:
+            E.engram_ple_short_conv_backward(
+                xx, w, dout if gg is None else gg, dilation=d, group_size=G, cu_seqlens=cu,
+                norm_weight=nw, conv_bias=b, dx=oo, dnorm_weight=dnw, dconv_weight=dw,
+                dconv_bias=db, workspace=ws, stream=stream)
+        else:
+            E.engram_ple_short_conv(xx, w, dilation=d, group_size=G, cu_seqlens=cu,
+                                    norm_weight=nw, conv_bias=b, out=oo, stream=stream)
 
     for _ in range(args.warmup):
         step()
@@ -625,12 +660,15 @@ def run_ple(args):
     total_ms = max_over_ranks(evs[0][0].elapsed_time(evs[-1][1]), device)
     kern_ms = statistics.mean(per)
 
-    # end to end through the public call with host buffers: x in from pinned
-    # memory, out back, copy-in / compute / copy-out overlapped on three streams
+    # end to end through the public call with host buffers: x (and dout) in
+    # from pinned memory, out (dx) back, copy-in / compute / copy-out overlapped
+    # on three streams
     e2e_steps = max(1, min(Ksteps, args.e2e_steps))
     x_h = x.cpu().pin_memory()
+    g_h = dout.cpu().pin_memory() if backward else None
     out_h = [torch.empty_like(x_h).pin_memory() for _ in range(2)]
     xd = [x, torch.empty_like(x)]
+    gd = [dout, torch.empty_like(dout)] if backward else [None, None]
     od = [out, torch.empty_like(out)]
     s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
     in_done = [torch.cuda.Event() for _ in range(e2e_steps)]
@@ -645,11 +683,13 @@ def run_ple(args):
             if k >= 2:
                 s_in.wait_event(comp_done[k - 2])
             xd[k % 2].copy_(x_h, non_blocking=True)
+            if backward:
+                gd[k % 2].copy_(g_h, non_blocking=True)
             in_done[k].record(s_in)
         stream.wait_event(in_done[k])
         if k >= 2:
             stream.wait_event(out_done[k - 2])
-        step(xd[k % 2], od[k % 2])
+        step(xd[k % 2], od[k % 2], gd[k % 2])
         comp_done[k].record(stream)
         with torch.cuda.stream(s_out):
             s_out.wait_event(comp_done[k])
@@ -662,35 +702,46 @@ def run_ple(args):
         raise RuntimeError("device error flag set during timing")
 
     peak, peak_kind = hbm_peak()
-    alg = T * C * 2 * 2 + C * (K + 2) * 2 + cu.numel() * 4
+    if backward:   # x, dout in; dx out; weights in; fp32 weight gradients out
+        alg = T * C * 2 * 3 + C * (K + 2) * 2 + C * (K + 2) * 4 + cu.numel() * 4
+        kname = "short_conv_bwd_kernel<bf16,bf16> + conv_bwd_reduce_kernel (one call)"
+        tname = "short_conv_bwd_kernel"
+    else:
+        alg = T * C * 2 * 2 + C * (K + 2) * 2 + cu.numel() * 4
+        kname = "short_conv_reg_kernel<bf16,bf16,4,3>"
+        tname = "short_conv_reg_kernel"
     achieved = alg / kern_ms / 1e6
     line = {
-        "metric": PLE_METRIC, "value": world * T * Ksteps / (total_ms / 1e3), "unit": UNIT,
+        "metric": PLE_BWD_METRIC if backward else PLE_METRIC,
+        "value": world * T * Ksteps / (total_ms / 1e3), "unit": UNIT,
         "n_gpus": world, "steps": Ksteps, "warmup": args.warmup,
         "ms_per_step": total_ms / Ksteps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": "ple_full", "tokens_per_step_per_gpu": T, "channels": C,
+        "config": {"workload": "ple_full_bwd" if backward else "ple_full",
+                   "tokens_per_step_per_gpu": T, "channels": C,
                    "branches": s.branches, "group": G, "kernel": K, "dilation": d,
-                   "flags": "norm + silu + residual", "cu_seqlens": f"{s.batch} rows",
-                   "l2": "inputs larger than L2 (1.34 GB in, 1.34 GB out)"},
-        "roofline": {"kernel": "short_conv_reg_kernel<bf16,bf16,4,3>", "bound": "hbm",
+                   "flags": "norm + silu + residual", "cu_seqlens": f"{batch} rows",
+                   "l2": (f"inputs larger than L2 ({T * C * 2 * (2 if backward else 1) / 1e9:.2f} "
+                          f"GB in, {T * C * 2 / 1e9:.2f} GB out)")},
+        "roofline": {"kernel": kname, "bound": "hbm",
                      "achieved": achieved, "peak": peak, "peak_kind": peak_kind,
                      "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": committed_traffic("short_conv_reg_kernel", T)},
-        "stages": {"ple_short_conv": {"ms": kern_ms, "alg_bytes": alg, "gbs": achieved,
-                                      "frac": achieved / peak,
-                                      "ms_min": min(per), "ms_max": max(per)}},
+                     "traffic": committed_traffic(tname, T)},
+        "stages": {("ple_short_conv_backward" if backward else "ple_short_conv"): {
+            "ms": kern_ms, "alg_bytes": alg, "gbs": achieved, "frac": achieved / peak,
+            "ms_min": min(per), "ms_max": max(per)}},
         "e2e": {"value": world * T * e2e_steps / (e2e_ms / 1e3), "unit": UNIT,
-                "h2d_bytes_per_step": x_h.numel() * 2, "d2h_bytes_per_step": x_h.numel() * 2,
+                "h2d_bytes_per_step": x_h.numel() * 2 * (2 if backward else 1),
+                "d2h_bytes_per_step": x_h.numel() * 2,
                 "steps": e2e_steps,
                 "pipeline": "copy-in / compute / copy-out streams, two buffer sets"},
         "gpu_launches": launches,
         "clocks": clk.summary(),
     }
     if world == 1 and not args.no_cpu_baseline:
-        rate, _, _, _ = ple_oracle_run(256)
+        rate, _, _, _ = ple_oracle_run(256, backward=backward)
         S = int(max(256, min(16384, rate * args.cpu_seconds)))
-        v, el, reps, desc = ple_oracle_run(S)
+        v, el, reps, desc = ple_oracle_run(S, backward=backward)
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
                                 "sample": desc, "seconds": el}
     else:
@@ -894,16 +945,20 @@ def main(argv=None):
                     help="--stage adam: table rows (default: an 8-way shard of the page table)")
     ap.add_argument("--adam-touched", type=int, default=ADAM_TOUCHED,
                     help="--stage adam: rows one step updates")
+    ap.add_argument("--ple-tokens", type=int, default=0,
+                    help="--stage ple / ple_bwd: whole 4,096-token rows to use instead of "
+                         "the workload's 16 (a smaller case for profiling)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--graph", dest="graph", action="store_true", default=True,
                     help="time the step as a replayed CUDA graph (default)")
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="time eager launches instead")
-    ap.add_argument("--stage", choices=["all", "bwd", "ple", "adam"], default="all",
+    ap.add_argument("--stage", choices=["all", "bwd", "ple", "ple_bwd", "adam"], default="all",
                     help="all: forward + backward (the step); bwd: the backward alone "
                          "(indices from engram_hash, no table allocated); ple: the PLE "
-                         "tail (norm + short conv) on its own workload; adam: the sparse "
+                         "tail (norm + short conv) on its own workload; ple_bwd: its "
+                         "backward on the same workload; adam: the sparse "
                          "optimizer step on an 8-way owner shard of the table")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)      # at least 3 untimed warm-up steps
@@ -911,6 +966,8 @@ def main(argv=None):
         return run_reference(args)
     if args.stage == "ple":
         return run_ple(args)
+    if args.stage == "ple_bwd":
+        return run_ple(args, backward=True)
     if args.stage == "adam":
         return run_adam(args)
     return run_ours(args)

@@ -936,7 +936,8 @@ int conv_bwd_plan(const engram_conv_params_t *p, int32_t dtype, int32_t grad_dty
     if (ex == 0 || eg == 0 || elem_bytes(p->weight_dtype) == 0)
         return ENGRAM_EINVAL;
     const int C = p->channels, G = p->group_size, K = p->kernel_size, d = p->dilation;
-    if (C < 1 || G < 8 || C % G != 0 || G % 8 != 0 || G / 8 > ple::kBwdThreads)
+    if (C < 1 || G < 8 || C % G != 0 || G % 8 != 0 ||
+        G / 8 > ple::kBwdThreads * ple::kBwdMaxCluster)
         return ENGRAM_EINVAL;
     if (K < 1 || K > ple::kBwdTaps || d < 1 || d > 4096 || p->reserved != 0)
         return ENGRAM_EINVAL;
@@ -944,7 +945,13 @@ int conv_bwd_plan(const engram_conv_params_t *p, int32_t dtype, int32_t grad_dty
         return ENGRAM_EINVAL;
     if (T < 0 || T > INT32_MAX)
         return ENGRAM_EINVAL;
-    const int pitch_x = (G * ex + 127) / 128 * 128, pitch_g = (G * eg + 127) / 128 * 128;
+    // branches wider than one block's 160 threads x 8 channels: two blocks of a
+    // cluster, one half each (G / 2 stays a multiple of 8)
+    const int csize = G / 8 > ple::kBwdThreads ? 2 : 1;
+    if (G % (8 * csize) != 0)
+        return ENGRAM_EINVAL;
+    const int gc = G / csize;
+    const int pitch_x = (gc * ex + 127) / 128 * 128, pitch_g = (gc * eg + 127) / 128 * 128;
     const int fit = (int)((ple::kSmemLimit - ple::kBwdDataOffset) / (size_t)(pitch_x + pitch_g));
     const int slots_max = std::min(fit, ple::kBwdMaxSlots);
     const int ahead = std::min((slots_max - ple::kBwdLag) / ple::kBwdRows - 1, ple::kBwdBars - 2);
@@ -955,7 +962,7 @@ int conv_bwd_plan(const engram_conv_params_t *p, int32_t dtype, int32_t grad_dty
     a.T = T;
     a.C = C;
     a.G = G;
-    a.nth = G / 8;
+    a.nth = gc / 8;
     a.dil = d;
     a.K = K;
     a.wdtype = p->weight_dtype;
@@ -966,6 +973,7 @@ int conv_bwd_plan(const engram_conv_params_t *p, int32_t dtype, int32_t grad_dty
     a.slots = ple::kBwdLag + (ahead + 1) * ple::kBwdRows;
     a.pitch_x = pitch_x;
     a.pitch_g = pitch_g;
+    a.csize = csize;
     P->smem = ple::bwd_smem_bytes(a.slots, pitch_x, pitch_g);
     P->threads = (a.nth + 31) / 32 * 32;
     return ENGRAM_OK;
@@ -980,9 +988,9 @@ int conv_bwd_grid(ConvBwdPlan *P)
     const int groups = a.C / a.G;
     const int classes = (int)std::max<int64_t>(1, std::min<int64_t>(a.dil, a.T));
     const int64_t rows = std::max<int64_t>(1, ceil_div(a.T, a.dil));  // rows of residue 0
-    int64_t chunks = std::max<int64_t>(1, sms / ((int64_t)groups * classes));
+    int64_t chunks = std::max<int64_t>(1, sms / ((int64_t)groups * classes * a.csize));
     chunks = std::min<int64_t>(chunks, std::max<int64_t>(1, ceil_div(rows, 16)));
-    const int64_t grid = (int64_t)groups * classes * chunks;
+    const int64_t grid = (int64_t)groups * classes * chunks * a.csize;
     if (grid > INT32_MAX)
         return ENGRAM_EINVAL;
     a.chunks = (int32_t)chunks;
@@ -997,7 +1005,21 @@ int launch_conv_bwd_t(const ConvBwdPlan &P, cudaStream_t s)
 {
     auto fn = ple::short_conv_bwd_kernel<XT, GT>;
     ENGRAM_TRY(allow_smem(fn));
-    fn<<<P.grid, P.threads, P.smem, s>>>(P.a);
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3((unsigned)P.grid);
+    cfg.blockDim = dim3((unsigned)P.threads);
+    cfg.dynamicSmemBytes = P.smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)P.a.csize;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, fn, P.a) != cudaSuccess)
+        return ENGRAM_ECUDA;
     return after_launch();
 }
 

@@ -14,29 +14,36 @@
 //   dnorm_w = sum_t dn xh
 // where back(t) / fwd(t) count the taps that stay inside t's sequence.
 //
-// The convolution only couples rows of one residue modulo d, so a block owns
-// one branch, one residue r and a range [ja, jb) of that residue's rows
-// j (token t = r + j d): along them the convolution has dilation 1. It walks
-// the rows in batches of B = 4, with the kernel width fixed at 4 (narrower
-// kernels run with zero taps) so that the lag of the transposed convolution
-// is 3 rows:
+// The convolution only couples rows of one residue modulo d, so a unit of
+// work is one branch, one residue r and a range [ja, jb) of that residue's
+// rows j (token t = r + j d): along them the convolution has dilation 1. A
+// thread owns 8 channels and keeps about 250 registers of state (the dy ring,
+// weights, weight-gradient sums), so a block has at most 5 warps (two per
+// scheduler) and a branch wider than 1,280 channels is split between the two
+// blocks of a cluster, which exchange their per-row partial sums through
+// distributed shared memory. The unit walks its rows in batches of B = 4,
+// with the kernel width fixed at 4 (narrower kernels run with zero taps) so
+// that the lag of the transposed convolution is 3 rows:
 //   stage 1  every thread sums the squares of its 8 channels of the batch's
-//            rows (one warp sum for four rows), warps post partial sums;
-//   barrier
-//   stage 2  inverse RMS of the four rows; y from the rows' normalised
-//            history (read again from shared memory), dy into a register
-//            ring holding rows j0 - 3 .. j0 + 3;
+//            rows (one warp sum for four rows); warps post partial sums to
+//            both blocks;
+//   barrier (over the cluster)
+//   stage 2  inverse RMS of the four rows; every row of the ring (j0 - 3 ..
+//            j0 + 3) is read and normalised once and added into the y of the
+//            batch rows it is a tap of; dy into a register ring;
 //   stage 3  for the lagged rows j0 - 3 .. j0: dn from the ring, the weight
-//            gradients, and per-warp partials of sum(s dn xh);
-//   barrier
+//            gradients, and partials of sum(s dn xh), posted to both blocks;
+//   barrier (over the cluster)
 //   stage 4  dx of the lagged rows (streaming stores), then the ring shifts.
-// Rows reach shared memory through a ring of row slots filled by cp.async.bulk
-// (one copy per row of x and of dout, issued `ahead` batches early by thread
-// 0, completion on a per-batch mbarrier waited on with a time bound). Halo
-// rows (3 before ja for history, 3 after jb for dy) are read but own no
-// output. Each block writes its weight-gradient partials to a workspace,
-// [d * chunks][4 + 2][C] fp32, that conv_bwd_reduce_kernel sums in a fixed
-// order, so results do not depend on timing.
+// Rows whose taps all stay inside their sequence (nearly all) take a path
+// without per-tap masks. Rows reach shared memory through a ring of row
+// slots filled by cp.async.bulk (one copy per row of x and of dout, issued
+// `ahead` batches early by four lanes of warp 0, completion on a per-batch
+// mbarrier waited on with a time bound). Halo rows (3 before ja for history,
+// 3 after jb for dy) are read but own no output. Each block writes its
+// weight-gradient partials to a workspace, [d * chunks][4 + 2][C] fp32, that
+// conv_bwd_reduce_kernel sums in a fixed order, so results do not depend on
+// timing.
 #pragma once
 
 #include "ple_conv_reg.cuh"
@@ -47,14 +54,16 @@ namespace ple {
 constexpr int kBwdRows = 4;                    // rows per batch
 constexpr int kBwdTaps = 4;                    // kernel widths 1..4
 constexpr int kBwdLag = kBwdTaps - 1;
-constexpr int kBwdWarps = 10;                  // 8 channels per thread: G <= 2560
-constexpr int kBwdThreads = 32 * kBwdWarps;
+constexpr int kBwdCtaWarps = 5;                // per block of a cluster
+constexpr int kBwdThreads = 32 * kBwdCtaWarps; // 8 channels per thread
+constexpr int kBwdMaxCluster = 2;              // blocks sharing a branch: G <= 2560
 constexpr int kBwdPartStride = 12;             // per-row partials, padded for float4 reads
 constexpr int kBwdMaxSlots = 32;
 constexpr int kBwdBars = 8;
 constexpr int kBwdQuantities = kBwdTaps + 2;   // weight taps, bias, norm scale
 
-// Shared memory: square-sum and dot partials [B][12] float each, inverse RMS
+// Shared memory: square-sum and dot partials [B][12] float each (column
+// rank * 5 + warp; the pads stay zero), inverse RMS
 // [32] float and tap counts [32] int32 per row slot, mbarriers [8]; then the
 // row slots of x [slots][pitch_x] and of dout [slots][pitch_g].
 constexpr int kBwdOffDot = kBwdRows * kBwdPartStride * 4;
@@ -84,7 +93,32 @@ struct ConvBwdArgs {
     uint32_t flags;
     int32_t slots, ahead;   // row slots; batches in flight ahead of the current one
     int32_t pitch_x, pitch_g;
+    int32_t csize;          // blocks per cluster sharing one branch slice (1 or 2)
 };
+
+__device__ __forceinline__ uint32_t cluster_rank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Barrier over every thread of the cluster, ordering shared-memory accesses
+// (local and remote) before it against those after it.
+__device__ __forceinline__ void cluster_barrier()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+                 "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// A float into the same offset of block `rank`'s shared memory.
+__device__ __forceinline__ void st_cluster(const float *local, uint32_t rank, float v)
+{
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)),
+                 "r"(rank));
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(remote), "f"(v) : "memory");
+}
 
 // 8 channels of one row in a shared-memory slot, as floats.
 template <typename T>
@@ -132,14 +166,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const bool active = tid < a.nth;
     const int d = a.dil;
+    const bool pair = a.csize == 2;
+    const uint32_t q_cta = pair ? cluster_rank() : 0u;  // half of the branch slice
+    const int unit = blockIdx.x / a.csize;
     const int per_branch = d * a.chunks;
-    const int m = blockIdx.x / per_branch;
-    const int rem = blockIdx.x - m * per_branch;
+    const int m = unit / per_branch;
+    const int rem = unit - m * per_branch;
     const int r = rem / a.chunks, p = rem - r * a.chunks;
     const int64_t nr = a.T > r ? (a.T - r + d - 1) / d : 0;  // rows of residue r
     const int64_t ja = nr * p / a.chunks, jb = nr * (p + 1) / a.chunks;
-    const int64_t c0 = (int64_t)m * a.G + (int64_t)tid * CH;  // first channel of this thread
+    const int gc = a.G / a.csize;                               // channels of this block
+    const int64_t cb = (int64_t)m * a.G + (int64_t)q_cta * gc;  // first channel of this block
+    const int64_t c0 = cb + (int64_t)tid * CH;                  // first channel of this thread
     float *part = a.partial + (size_t)(r * a.chunks + p) * kBwdQuantities * a.C + c0;
+    const int pslot = (int)q_cta * kBwdCtaWarps + wid;         // this warp's partial column
 
     if (ja >= jb) {  // no rows: the block's partials are zero
         if (active)
@@ -154,27 +194,28 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
     const int64_t je = min64(nr, jb + L);
     const int nbatch = (int)((jb + L - js + B - 1) / B);
     const int S = a.slots;
-    const uint32_t xbytes = (uint32_t)a.G * sizeof(XT), gbytes = (uint32_t)a.G * sizeof(GT);
-    const char *xb = static_cast<const char *>(a.x) + (int64_t)m * a.G * sizeof(XT);
-    const char *gb = static_cast<const char *>(a.dout) + (int64_t)m * a.G * sizeof(GT);
+    const uint32_t xbytes = (uint32_t)gc * sizeof(XT), gbytes = (uint32_t)gc * sizeof(GT);
+    const char *xb = static_cast<const char *>(a.x) + cb * sizeof(XT);
+    const char *gb = static_cast<const char *>(a.dout) + cb * sizeof(GT);
     const int64_t xrow = (int64_t)a.C * sizeof(XT), grow = (int64_t)a.C * sizeof(GT);
     const bool do_norm = a.flags & ENGRAM_CONV_NORM;
     const bool do_silu = a.flags & ENGRAM_CONV_SILU;
     const bool do_res = a.flags & ENGRAM_CONV_RESIDUAL;
 
-    // sequence frontier of the loading thread: [seq_lo, seq_hi) holds the
-    // last row it described
+    // warp 0, lane i < B: rows j0 + i of every batch; each such lane keeps
+    // the bounds [seq_lo, seq_hi) of the sequence holding its last row
     int32_t seq = 0;
     int64_t seq_lo = 0, seq_hi = a.T;
+    if (wid == 0 && lane < B && a.cu != nullptr) {
+        const int64_t t = r + min64(js + lane, nr - 1) * d;
+        seq = find_sequence(a.cu, a.nseq, t);
+        seq_lo = __ldg(a.cu + seq);
+        seq_hi = __ldg(a.cu + seq + 1);
+    }
     if (tid == 0) {
         for (int b = 0; b < kBwdBars; ++b)
             mbar_init(bars + b, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        if (a.cu != nullptr) {
-            seq = find_sequence(a.cu, a.nseq, r + js * d);
-            seq_lo = __ldg(a.cu + seq);
-            seq_hi = __ldg(a.cu + seq + 1);
-        }
     }
     for (int i = tid; i < 2 * B * kBwdPartStride; i += blockDim.x)
         ss_part[i] = 0.f;  // (and dot_part) pads of absent warps stay zero
@@ -182,30 +223,47 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
         inv_s[i] = 0.f;
         meta_s[i] = 0;
     }
-    __syncthreads();
+    // (every block of the cluster has started and zeroed its partials before
+    // any block writes into another's)
+    auto sync_all = [&]() {
+        if (pair)
+            cluster_barrier();
+        else
+            __syncthreads();
+    };
+    // one row sum of each warp, into this block's and the partner's partials
+    auto post = [&](float *partials, float tot) {
+        if ((lane & 7) == 0) {
+            float *dst = partials + (lane >> 3) * kBwdPartStride + pslot;
+            *dst = tot;
+            if (pair)
+                st_cluster(dst, q_cta ^ 1u, tot);
+        }
+    };
+    sync_all();
 
-    // thread 0: rows of batch b into their slots, and their tap counts
+    // warp 0: rows of batch b into their slots (lane i: row j0 + i), and
+    // their in-sequence tap counts
     auto issue = [&](int b) {
         const int64_t j0 = js + (int64_t)b * B;
-        uint32_t bytes = 0;
-#pragma unroll
-        for (int i = 0; i < B; ++i) {
-            const int64_t j = j0 + i;
-            if (j < je)
-                bytes += xbytes + (j >= ja ? gbytes : 0u);
-        }
-        if (bytes == 0)
+        if (j0 >= je)
             return;
         uint64_t *bar = bars + b % kBwdBars;
-        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
-                     "r"(bytes)
-                     : "memory");
-        int slot = (int)((j0 - js) % S);
+        if (lane == 0) {
+            uint32_t bytes = 0;
 #pragma unroll
-        for (int i = 0; i < B; ++i, slot = slot + 1 == S ? 0 : slot + 1) {
-            const int64_t j = j0 + i;
-            if (j >= je)
-                break;
+            for (int i = 0; i < B; ++i)
+                if (j0 + i < je)
+                    bytes += xbytes + (j0 + i >= ja ? gbytes : 0u);
+            asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(
+                             smem_u32(bar)),
+                         "r"(bytes)
+                         : "memory");
+        }
+        __syncwarp();
+        const int64_t j = j0 + lane;
+        if (lane < B && j < je) {
+            const int slot = (int)((j - js) % S);
             const int64_t t = r + j * d;
             bulk_load(xs + (size_t)slot * a.pitch_x, xb + t * xrow, xbytes, bar);
             if (j >= ja)
@@ -222,7 +280,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
             meta_s[slot] = nb | nf << 8;
         }
     };
-    if (tid == 0)
+    if (wid == 0)
         for (int b = 0; b < a.ahead && b < nbatch; ++b)
             issue(b);
 
@@ -259,16 +317,30 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
     }
 
     const size_t xoff = (size_t)tid * CH * sizeof(XT), goff = (size_t)tid * CH * sizeof(GT);
-    char *dxb = static_cast<char *>(a.dx) + (int64_t)m * a.G * sizeof(GT) + goff;
+    char *dxb = static_cast<char *>(a.dx) + cb * sizeof(GT) + goff;
     bool timed_out = false;
+
+    // x of ring row q (rows j0 - L .. j0 + B - 1) of the batch, normalised
+    auto load_xh = [&](int slot, float iv, float2 *xh) {
+        float f[CH];
+        load_slot8<XT>(xs + (size_t)slot * a.pitch_x + xoff, f);
+        const float2 iv2 = make_float2(iv, iv);
+#pragma unroll
+        for (int pp = 0; pp < NP; ++pp)
+            xh[pp] = __fmul2_rn(make_float2(f[2 * pp], f[2 * pp + 1]), iv2);
+    };
 
     for (int b = 0; b < nbatch; ++b) {
         const int64_t j0 = js + (int64_t)b * B;
-        int slot[B];
-        slot[0] = (int)((j0 - js) % S);
+        // slots of ring rows j0 - L .. j0 + B - 1
+        int slot[RING];
+        slot[L] = (int)((j0 - js) % S);
 #pragma unroll
-        for (int i = 1; i < B; ++i)
-            slot[i] = slot[i - 1] + 1 == S ? 0 : slot[i - 1] + 1;
+        for (int q = L - 1; q >= 0; --q)
+            slot[q] = slot[q + 1] == 0 ? S - 1 : slot[q + 1] - 1;
+#pragma unroll
+        for (int q = L + 1; q < RING; ++q)
+            slot[q] = slot[q - 1] + 1 == S ? 0 : slot[q - 1] + 1;
         if (j0 < je && !timed_out &&
             !mbar_wait(bars + b % kBwdBars, (uint32_t)(b / kBwdBars) & 1u))
             timed_out = true;
@@ -281,7 +353,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
                 float2 acc = zero2;
                 if (active && j0 + i < je) {
                     float f[CH];
-                    load_slot8<XT>(xs + (size_t)slot[i] * a.pitch_x + xoff, f);
+                    load_slot8<XT>(xs + (size_t)slot[L + i] * a.pitch_x + xoff, f);
 #pragma unroll
                     for (int pp = 0; pp < NP; ++pp) {
                         const float2 x2 = make_float2(f[2 * pp], f[2 * pp + 1]);
@@ -290,54 +362,69 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
                 }
                 ss[i] = acc.x + acc.y;
             }
-            const float tot = warp_sum4(ss[0], ss[1], ss[2], ss[3], lane);
-            if ((lane & 7) == 0)
-                ss_part[(lane >> 3) * kBwdPartStride + wid] = tot;
+            post(ss_part, warp_sum4(ss[0], ss[1], ss[2], ss[3], lane));
         }
-        __syncthreads();
-        if (tid == 0 && b + a.ahead < nbatch)
+        sync_all();
+        if (wid == 0 && b + a.ahead < nbatch)
             issue(b + a.ahead);
 
         // ---- stage 2: inverse RMS, y and dy of the batch's rows
-        float inv[B];
+        float inv[RING];  // of the ring rows: earlier batches' from shared memory
+#pragma unroll
+        for (int q = 0; q < L; ++q)
+            inv[q] = inv_s[slot[q]];
 #pragma unroll
         for (int i = 0; i < B; ++i) {
-            inv[i] = do_norm ? rsqrtf(fmaf(sum_parts(ss_part, i), a.inv_G, a.eps)) : 1.f;
+            inv[L + i] = do_norm ? rsqrtf(fmaf(sum_parts(ss_part, i), a.inv_G, a.eps)) : 1.f;
             if (tid == 0)
-                inv_s[slot[i]] = inv[i];
+                inv_s[slot[L + i]] = inv[L + i];
+        }
+        // taps: a row of the ring feeds rows i = q - L + k of the batch, tap k
+        int back[B];
+        bool full_back = true;
+#pragma unroll
+        for (int i = 0; i < B; ++i) {
+            back[i] = meta_s[slot[L + i]] & 0xff;
+            full_back = full_back && back[i] == L;
+        }
+        full_back = full_back && j0 + B <= je && j0 >= ja;
+        float2 acc[B][NP];
+#pragma unroll
+        for (int i = 0; i < B; ++i)
+#pragma unroll
+            for (int pp = 0; pp < NP; ++pp)
+                acc[i][pp] = zero2;
+        if (active) {
+#pragma unroll
+            for (int q = 0; q < RING; ++q) {
+                const int64_t jr = j0 - L + q;
+                if (jr < js || jr >= je)
+                    continue;  // not loaded (no batch row reads it: its tap is out of range)
+                float2 xh[NP];
+                load_xh(slot[q], inv[q], xh);
+#pragma unroll
+                for (int i = 0; i < B; ++i) {
+                    const int k = L + i - q;
+                    if (k < 0 || k >= KT)
+                        continue;
+                    if (full_back || k <= back[i]) {
+#pragma unroll
+                        for (int pp = 0; pp < NP; ++pp)
+                            acc[i][pp] = __ffma2_rn(w[k][pp], xh[pp], acc[i][pp]);
+                    }
+                }
+            }
         }
 #pragma unroll
         for (int i = 0; i < B; ++i) {
             const int64_t j = j0 + i;
-#pragma unroll
-            for (int pp = 0; pp < NP; ++pp)
-                dy[L + i][pp] = zero2;
-            if (!active || j >= je || j < ja)
-                continue;
-            const int back = meta_s[slot[i]] & 0xff;
-            float2 acc[NP];
-#pragma unroll
-            for (int pp = 0; pp < NP; ++pp)
-                acc[pp] = zero2;
-#pragma unroll
-            for (int k = 0; k < KT; ++k) {
-                if (k > back)
-                    break;
-                const int sk = slot[i] - k < 0 ? slot[i] - k + S : slot[i] - k;
-                const float ik = i - k >= 0 ? inv[i - k >= 0 ? i - k : 0] : inv_s[sk];
-                float f[CH];
-                load_slot8<XT>(xs + (size_t)sk * a.pitch_x + xoff, f);
-                const float2 ik2 = make_float2(ik, ik);
-#pragma unroll
-                for (int pp = 0; pp < NP; ++pp)
-                    acc[pp] = __ffma2_rn(
-                        w[k][pp], __fmul2_rn(make_float2(f[2 * pp], f[2 * pp + 1]), ik2), acc[pp]);
-            }
+            const bool need = active && j < je && j >= ja;
             float g[CH];
-            load_slot8<GT>(gs + (size_t)slot[i] * a.pitch_g + goff, g);
+            if (need)
+                load_slot8<GT>(gs + (size_t)slot[L + i] * a.pitch_g + goff, g);
 #pragma unroll
             for (int pp = 0; pp < NP; ++pp) {
-                const float2 y = __ffma2_rn(sc[pp], acc[pp], bias[pp]);
+                const float2 y = __ffma2_rn(sc[pp], acc[i][pp], bias[pp]);
                 float2 f = make_float2(1.f, 1.f);
                 if (do_silu) {
                     // SiLU'(y) = sg + y sg (1 - sg), sg = 1 / (1 + 2^(-y log2 e))
@@ -350,48 +437,49 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
                                                  make_float2(1.f, 1.f));
                     f = __ffma2_rn(y, __fmul2_rn(sg, om), sg);
                 }
-                dy[L + i][pp] = __fmul2_rn(make_float2(g[2 * pp], g[2 * pp + 1]), f);
+                dy[L + i][pp] = need ? __fmul2_rn(make_float2(g[2 * pp], g[2 * pp + 1]), f)
+                                     : zero2;
             }
         }
 
         // ---- stage 3: dn, weight gradients and dot partials of the lagged rows
+        // (ring rows 0 .. B - 1)
+        int fwd[B];
+        bool full_fwd = j0 - L >= ja && j0 - L + B <= jb;
+#pragma unroll
+        for (int i = 0; i < B; ++i) {
+            fwd[i] = meta_s[slot[i]] >> 8;
+            full_fwd = full_fwd && fwd[i] == L;
+        }
         {
             float dotv[B];
 #pragma unroll
             for (int i = 0; i < B; ++i) {
                 const int64_t jj = j0 - L + i;
-                float2 acc = zero2;
+                float2 accd = zero2;
                 if (active && jj >= ja && jj < jb) {
-                    const int sl = slot[i] - L < 0 ? slot[i] - L + S : slot[i] - L;
-                    const int fwd = meta_s[sl] >> 8;
-                    const float ij = i - L >= 0 ? inv[i - L >= 0 ? i - L : 0] : inv_s[sl];
-                    float f[CH];
-                    load_slot8<XT>(xs + (size_t)sl * a.pitch_x + xoff, f);
-                    const float2 ij2 = make_float2(ij, ij);
+                    float2 xh[NP];
+                    load_xh(slot[i], inv[i], xh);
 #pragma unroll
                     for (int pp = 0; pp < NP; ++pp) {
-                        const float2 xh = __fmul2_rn(make_float2(f[2 * pp], f[2 * pp + 1]), ij2);
                         float2 dn = zero2;
 #pragma unroll
                         for (int k = 0; k < KT; ++k) {
-                            const float2 g = k <= fwd ? dy[i + k][pp] : zero2;
+                            const float2 g = full_fwd || k <= fwd[i] ? dy[i + k][pp] : zero2;
                             dn = __ffma2_rn(w[k][pp], g, dn);
-                            dw[k][pp] = __ffma2_rn(xh, g, dw[k][pp]);
+                            dw[k][pp] = __ffma2_rn(xh[pp], g, dw[k][pp]);
                         }
                         db[pp] = __fadd2_rn(db[pp], dy[i][pp]);
-                        dnw[pp] = __ffma2_rn(dn, xh, dnw[pp]);
-                        acc = __ffma2_rn(__fmul2_rn(sc[pp], dn), xh, acc);
+                        dnw[pp] = __ffma2_rn(dn, xh[pp], dnw[pp]);
+                        accd = __ffma2_rn(__fmul2_rn(sc[pp], dn), xh[pp], accd);
                     }
                 }
-                dotv[i] = acc.x + acc.y;
+                dotv[i] = accd.x + accd.y;
             }
-            if (do_norm) {
-                const float tot = warp_sum4(dotv[0], dotv[1], dotv[2], dotv[3], lane);
-                if ((lane & 7) == 0)
-                    dot_part[(lane >> 3) * kBwdPartStride + wid] = tot;
-            }
+            if (do_norm)
+                post(dot_part, warp_sum4(dotv[0], dotv[1], dotv[2], dotv[3], lane));
         }
-        __syncthreads();
+        sync_all();
 
         // ---- stage 4: dx of the lagged rows
 #pragma unroll
@@ -399,28 +487,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
             const int64_t jj = j0 - L + i;
             if (!active || jj < ja || jj >= jb)
                 continue;
-            const int sl = slot[i] - L < 0 ? slot[i] - L + S : slot[i] - L;
-            const int fwd = meta_s[sl] >> 8;
-            const float ij = i - L >= 0 ? inv[i - L >= 0 ? i - L : 0] : inv_s[sl];
             const float mean = do_norm ? sum_parts(dot_part, i) * a.inv_G : 0.f;
-            float f[CH], g[CH], o[CH];
-            load_slot8<XT>(xs + (size_t)sl * a.pitch_x + xoff, f);
+            float g[CH], o[CH];
+            float2 xh[NP];
+            load_xh(slot[i], inv[i], xh);
             if (do_res)
-                load_slot8<GT>(gs + (size_t)sl * a.pitch_g + goff, g);
-            const float2 ij2 = make_float2(ij, ij), mean2 = make_float2(-mean, -mean);
+                load_slot8<GT>(gs + (size_t)slot[i] * a.pitch_g + goff, g);
+            const float2 ij2 = make_float2(inv[i], inv[i]), mean2 = make_float2(-mean, -mean);
 #pragma unroll
             for (int pp = 0; pp < NP; ++pp) {
                 float2 dn = zero2;
 #pragma unroll
                 for (int k = 0; k < KT; ++k)
-                    dn = __ffma2_rn(w[k][pp], k <= fwd ? dy[i + k][pp] : zero2, dn);
-                float2 v;
-                if (do_norm) {
-                    const float2 xh = __fmul2_rn(make_float2(f[2 * pp], f[2 * pp + 1]), ij2);
-                    v = __fmul2_rn(ij2, __ffma2_rn(xh, mean2, __fmul2_rn(sc[pp], dn)));
-                } else {
-                    v = dn;
-                }
+                    dn = __ffma2_rn(w[k][pp], full_fwd || k <= fwd[i] ? dy[i + k][pp] : zero2,
+                                    dn);
+                float2 v = do_norm ? __fmul2_rn(ij2, __ffma2_rn(xh[pp], mean2,
+                                                                __fmul2_rn(sc[pp], dn)))
+                                   : dn;
                 if (do_res)
                     v = __fadd2_rn(v, make_float2(g[2 * pp], g[2 * pp + 1]));
                 o[2 * pp] = v.x;
