@@ -21,6 +21,7 @@ from ._binding import (ENGRAM_BF16, ENGRAM_CONV_NORM, ENGRAM_CONV_RESIDUAL, ENGR
                        engram_hash_gather_slice, engram_host_floor_mod, engram_ple_short_conv,
                        engram_ple_short_conv_backward,
                        engram_ple_short_conv_backward_workspace_size, engram_sparse_adam,
+                       engram_owner_bucket, engram_owner_bucket_workspace_size,
                        engram_launch_count, lib, make_params, status_string)
 
 __all__ = [
@@ -34,6 +35,6 @@ __all__ = [
     "engram_gather", "engram_get_device_error", "engram_hash", "engram_hash_gather",
     "engram_hash_gather_slice", "engram_grouped_rms_norm", "engram_ple_short_conv",
     "engram_ple_short_conv_backward", "engram_ple_short_conv_backward_workspace_size",
-    "engram_sparse_adam",
+    "engram_sparse_adam", "engram_owner_bucket", "engram_owner_bucket_workspace_size",
     "engram_host_floor_mod", "engram_launch_count", "lib", "make_params", "status_string",
 ]

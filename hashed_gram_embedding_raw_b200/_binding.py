@@ -35,6 +35,7 @@ EXPORTED = (
     "engram_host_floor_mod", "engram_backward_noalloc", "engram_hash_gather_slice",
     "engram_ple_short_conv", "engram_grouped_rms_norm", "engram_sparse_adam",
     "engram_ple_short_conv_backward", "engram_ple_short_conv_backward_workspace_size",
+    "engram_owner_bucket", "engram_owner_bucket_workspace_size",
 )
 
 ENGRAM_NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -142,6 +143,8 @@ def _load():
         "engram_ple_short_conv_backward": [P, P, i32, P, i32, i64, P, P, P, P, i32, P, P, P, P,
                                            P, sz, P],
         "engram_ple_short_conv_backward_workspace_size": [P, i64, ctypes.POINTER(sz)],
+        "engram_owner_bucket": [P, i64, i64, i32, P, P, P, P, P, sz, P],
+        "engram_owner_bucket_workspace_size": [i64, i32, ctypes.POINTER(sz)],
     }
     for name, args in sig.items():
         fn = getattr(L, name)
@@ -497,6 +500,44 @@ def engram_ple_short_conv_backward(x: torch.Tensor, conv_weight: torch.Tensor,
         _ptr(dconv_weight), _ptr(dconv_bias), _ptr(workspace), workspace.numel(),
         _stream(stream)), "engram_ple_short_conv_backward")
     return dx, dnorm_weight, dconv_weight, dconv_bias
+
+
+def engram_owner_bucket_workspace_size(n: int, owners: int) -> int:
+    nbytes = ctypes.c_size_t(0)
+    _check(lib.engram_owner_bucket_workspace_size(int(n), int(owners), ctypes.byref(nbytes)),
+           "engram_owner_bucket_workspace_size")
+    return nbytes.value
+
+
+def engram_owner_bucket(rows: torch.Tensor, rows_per_owner: int, owners: int, send_rows=None,
+                        src_pos=None, dst_pos=None, counts=None, workspace=None, stream=None):
+    """Stable grouping of lookups by owner rank (rows // rows_per_owner):
+    returns (send_rows [n] owner-local rows in owner order, src_pos [n] the
+    lookup of each grouped position, dst_pos [n] the grouped position of each
+    lookup, counts [owners] int32 on the device)."""
+    _cuda(rows, "rows", torch.int32)
+    n = rows.numel()
+    dev = rows.device
+
+    def buf(t, name, size):
+        t = torch.empty(size, dtype=torch.int32, device=dev) if t is None else t
+        _cuda(t, name, torch.int32)
+        if t.numel() != size:
+            raise ValueError(f"{name} must hold {size} elements")
+        return t
+
+    send_rows, src_pos, dst_pos = (buf(send_rows, "send_rows", n), buf(src_pos, "src_pos", n),
+                                   buf(dst_pos, "dst_pos", n))
+    counts = buf(counts, "counts", int(owners))
+    if workspace is None:
+        workspace = torch.empty(max(16, engram_owner_bucket_workspace_size(n, owners)),
+                                dtype=torch.uint8, device=dev)
+    _cuda(workspace, "workspace", torch.uint8)
+    _check(lib.engram_owner_bucket(_ptr(rows), n, int(rows_per_owner), int(owners),
+                                   _ptr(send_rows), _ptr(src_pos), _ptr(dst_pos), _ptr(counts),
+                                   _ptr(workspace), workspace.numel(), _stream(stream)),
+           "engram_owner_bucket")
+    return send_rows, src_pos, dst_pos, counts
 
 
 def engram_grouped_rms_norm(x: torch.Tensor, group_size: int, weight=None, eps: float = 1e-6,

@@ -23,6 +23,7 @@
 #include "ple_conv_reg.cuh"
 #include "ple_conv_bwd.cuh"
 #include "optim.cuh"
+#include "owner.cuh"
 #include "norm.cuh"
 
 using namespace engram;
@@ -1184,6 +1185,67 @@ int engram_sparse_adam(const engram_adam_params_t *params, void *table, int32_t 
         break;
     }
     return after_launch();
+}
+
+} // extern "C"
+
+// ------------------------------------------------------ owner routing
+
+extern "C" {
+
+int engram_owner_bucket_workspace_size(int64_t n, int32_t owners, size_t *bytes)
+{
+    if (bytes == nullptr || n < 0 || n > INT32_MAX || owners < 1 || owners > owner::kMaxOwners)
+        return ENGRAM_EINVAL;
+    const int64_t ntiles = std::max<int64_t>(1, ceil_div(n, owner::kTile));
+    *bytes = (size_t)2 * ntiles * owners * sizeof(uint32_t);
+    return ENGRAM_OK;
+}
+
+int engram_owner_bucket(const int32_t *rows, int64_t n, int64_t rows_per_owner, int32_t owners,
+                        int32_t *send_rows, int32_t *src_pos, int32_t *dst_pos, int32_t *counts,
+                        void *workspace, size_t workspace_bytes, engram_stream_t stream)
+{
+    size_t need = 0;
+    ENGRAM_TRY(engram_owner_bucket_workspace_size(n, owners, &need));
+    if (rows_per_owner < 1 || counts == nullptr)
+        return ENGRAM_EINVAL;
+    if (n > 0 && (rows == nullptr || send_rows == nullptr || src_pos == nullptr ||
+                  dst_pos == nullptr || workspace == nullptr))
+        return ENGRAM_EINVAL;
+    const size_t nb = (size_t)n * sizeof(int32_t);
+    if (overlaps(rows, nb, send_rows, nb) || overlaps(rows, nb, src_pos, nb) ||
+        overlaps(rows, nb, dst_pos, nb) || overlaps(send_rows, nb, src_pos, nb) ||
+        overlaps(send_rows, nb, dst_pos, nb) || overlaps(src_pos, nb, dst_pos, nb))
+        return ENGRAM_EINVAL;
+    if (workspace_bytes < need)
+        return ENGRAM_ENOSPC;
+    owner::OwnerArgs a;
+    a.rows = rows;
+    a.n = n;
+    a.rows_per_owner = rows_per_owner;
+    a.owners = owners;
+    a.ntiles = (int32_t)std::max<int64_t>(1, ceil_div(n, owner::kTile));
+    a.tile_cnt = static_cast<uint32_t *>(workspace);
+    a.tile_off = a.tile_cnt + (size_t)a.ntiles * owners;
+    a.counts = counts;
+    a.send_rows = send_rows;
+    a.src_pos = src_pos;
+    a.dst_pos = dst_pos;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (n > 0) {
+        owner::owner_count<<<a.ntiles, owner::kThreads, 0, s>>>(a);
+        ENGRAM_TRY(after_launch());
+    }
+    if (n == 0)
+        a.ntiles = 0;  // counts only: all zero
+    owner::owner_scan<<<1, owner::kThreads, 0, s>>>(a);
+    ENGRAM_TRY(after_launch());
+    if (n > 0) {
+        owner::owner_scatter<<<a.ntiles, owner::kThreads, 0, s>>>(a);
+        ENGRAM_TRY(after_launch());
+    }
+    return ENGRAM_OK;
 }
 
 } // extern "C"

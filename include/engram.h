@@ -402,6 +402,45 @@ ENGRAM_API int engram_sparse_adam(const engram_adam_params_t *params, void *tabl
                                   const int32_t *num_unique, int64_t max_rows,
                                   engram_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * Owner-sharded table (Qwen3_8_FlashNextOwnerShardedEmbedding, engram page):
+ * rank r of an owner group of `owners` ranks holds rows
+ * [r * rows_per_owner, (r + 1) * rows_per_owner) of the table. A requesting
+ * rank groups its lookups by owner, sends the owner-local rows in the first
+ * All-to-All, the owners look them up (engram_gather on their shard), and the
+ * second All-to-All brings the values back in the same grouping; in the
+ * backward the row gradients travel the reverse way and only the owner
+ * accumulates them (engram_backward on its shard). The collectives themselves
+ * are the caller's (NCCL through torch.distributed in the Python package);
+ * this call is the routing step on the requesting rank.
+ * ------------------------------------------------------------------------ */
+
+/*
+ * engram_owner_bucket -- stable grouping of n lookups by owner
+ * o = rows[i] / rows_per_owner. For the lookup i placed at grouped position p
+ * (owners in ascending order, each owner's lookups in ascending i):
+ *   send_rows[p] = rows[i] - o * rows_per_owner   (owner-local row)
+ *   src_pos[p]   = i
+ *   dst_pos[i]   = p
+ *   counts[o]    = lookups of owner o (device, int32 [owners])
+ * so engram_gather(values, dst_pos) restores request order from values that
+ * came back grouped, and engram_gather(dout, src_pos) groups the gradients.
+ * A row outside [0, owners * rows_per_owner) goes to the last owner with
+ * local row -1 (which that owner's lookup rejects) and sets
+ * ENGRAM_DEVERR_ROW_RANGE.
+ *   rows       device, int32 [n] (e.g. engram_hash's [T, H] output)
+ *   send_rows, src_pos, dst_pos  device, int32 [n], not overlapping rows
+ *   workspace  device, >= engram_owner_bucket_workspace_size bytes
+ * Limits: 1 <= owners <= 256, rows_per_owner >= 1, 0 <= n < 2^31. Three
+ * launches.
+ */
+ENGRAM_API int engram_owner_bucket(const int32_t *rows, int64_t n, int64_t rows_per_owner,
+                                   int32_t owners, int32_t *send_rows, int32_t *src_pos,
+                                   int32_t *dst_pos, int32_t *counts, void *workspace,
+                                   size_t workspace_bytes, engram_stream_t stream);
+
+ENGRAM_API int engram_owner_bucket_workspace_size(int64_t n, int32_t owners, size_t *bytes);
+
 /*
  * engram_get_device_error -- copy the current device's error word
  * (ENGRAM_DEVERR_* bits set since the last call) into *flags and clear it.

@@ -254,3 +254,30 @@ def test_package_import_fails_loudly_without_library(tmp_path):
     mod = importlib.util.module_from_spec(spec)
     with pytest.raises(ImportError, match="not found"):
         spec.loader.exec_module(mod)
+
+
+def test_host_rejects_bad_owner_bucket_args(E):
+    L = E.lib
+    a, b, c, d, e = (ctypes.c_void_p(v << 20) for v in (1, 2, 3, 4, 5))
+    ws = ctypes.c_void_p(6 << 20)
+    sz = ctypes.c_size_t(0)
+
+    def call(rows=a, n=100, rpo=10, owners=4, send=b, src=c, dst=d, counts=e, work=ws,
+             nbytes=1 << 20):
+        return L.engram_owner_bucket(rows, n, rpo, owners, send, src, dst, counts, work,
+                                     nbytes, None)
+
+    assert L.engram_owner_bucket_workspace_size(100, 0, ctypes.byref(sz)) == E.ENGRAM_EINVAL
+    assert L.engram_owner_bucket_workspace_size(100, 257, ctypes.byref(sz)) == E.ENGRAM_EINVAL
+    assert L.engram_owner_bucket_workspace_size(-1, 4, ctypes.byref(sz)) == E.ENGRAM_EINVAL
+    assert L.engram_owner_bucket_workspace_size(4096, 4, ctypes.byref(sz)) == E.ENGRAM_OK
+    assert sz.value == 2 * 2 * 4 * 4
+    assert call(owners=0) == E.ENGRAM_EINVAL
+    assert call(rpo=0) == E.ENGRAM_EINVAL
+    assert call(n=-1) == E.ENGRAM_EINVAL
+    assert call(counts=None) == E.ENGRAM_EINVAL
+    assert call(rows=None) == E.ENGRAM_EINVAL
+    assert call(work=None) == E.ENGRAM_EINVAL
+    assert call(send=ctypes.c_void_p((1 << 20) + 64)) == E.ENGRAM_EINVAL   # overlaps rows
+    assert call(dst=c) == E.ENGRAM_EINVAL                                  # src = dst
+    assert call(nbytes=8) == E.ENGRAM_ENOSPC

@@ -1,0 +1,157 @@
+"""Owner-sharded routing (hashed_gram_embedding_raw_b200.owner) on the CPU.
+
+The routing generators run with host stand-ins for the device steps (defined
+here: the oracle's hash, gather and backward, and a stable argsort for the
+grouping), first as ranks emulated in one process, then as two gloo ranks with
+real all-to-alls. What they pin is the exchange logic of the page's
+Qwen3_8_FlashNextOwnerShardedEmbedding: counts, split sizes, the grouping by
+owner, putting values back in request order and sending gradients back to
+the owner, which alone accumulates its rows. Every rank's output must equal
+the oracle's lookup in the whole table, and every owner's row gradients the
+oracle's backward over all ranks' lookups restricted to its rows.
+"""
+
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from workloads import head_params, host_dout, host_table, token_stream
+
+
+class HostOps:
+    """Host stand-ins for the device steps (test only)."""
+
+    def __init__(self, cfg):
+        self.cfg = cfg
+
+    def hash(self, params, ids, cu):
+        idx = oracle.hash_ids(ids.numpy(), None if cu is None else cu.numpy(), self.cfg)
+        return torch.from_numpy(idx.astype(np.int32))
+
+    def bucket(self, rows, rpo, owners):
+        r = rows.numpy().astype(np.int64)
+        o = r // rpo
+        order = np.argsort(o, kind="stable")
+        dst = np.empty_like(order)
+        dst[order] = np.arange(len(order))
+        return (torch.from_numpy((r[order] - o[order] * rpo).astype(np.int32)),
+                torch.from_numpy(order.astype(np.int32)), torch.from_numpy(dst.astype(np.int32)),
+                torch.from_numpy(np.bincount(o, minlength=owners).astype(np.int32)))
+
+    def gather(self, table, idx):
+        return table[idx.long()]
+
+    def backward(self, idx, dout, table_rows):
+        u, g = oracle.backward(idx.numpy(), dout.numpy(), oracle.F32)
+        return torch.from_numpy(u), torch.from_numpy(g), torch.tensor([len(u)], dtype=torch.int32)
+
+
+def split_stream(ids, W):
+    """W equal token chunks of the tiny stream, one sequence each."""
+    T = len(ids) // W
+    return [(torch.from_numpy(ids[r * T:(r + 1) * T].copy()),
+             torch.tensor([0, T], dtype=torch.int32)) for r in range(W)]
+
+
+def expected(cfg, table, parts, douts, W):
+    rpo = cfg["table_rows"] // W
+    outs, all_idx = [], []
+    for ids, cu in parts:
+        idx = oracle.hash_ids(ids.numpy(), cu.numpy(), cfg)
+        outs.append(oracle.gather(table, idx).reshape(len(ids), -1))
+        all_idx.append(idx.reshape(-1))
+    idx = np.concatenate(all_idx)
+    dout = np.concatenate([d.numpy() for d in douts])
+    owners = []
+    for r in range(W):
+        keep = (idx // rpo) == r
+        u, g = oracle.backward(idx[keep] - r * rpo, dout[keep], oracle.F32)
+        owners.append((u, g))
+    return outs, owners
+
+
+def run_rank(E_owner, params, cfg, table, W, r, ids, cu, dout, runner):
+    rpo = cfg["table_rows"] // W
+    shard = torch.from_numpy(table[r * rpo:(r + 1) * rpo].copy())
+    ops = HostOps(cfg)
+    out, routing = runner(E_owner.forward_steps(params, shard, W, ids, cu, ops=ops))
+    u, g, nu = runner(E_owner.backward_steps(params, W, routing, dout, ops=ops))
+    return out, u, g, nu
+
+
+@pytest.mark.parametrize("W", [1, 2, 4])
+def test_lockstep_emulated_ranks(W):
+    from hashed_gram_embedding_raw_b200 import make_params, owner
+    cfg = head_params("tiny")
+    params = make_params(cfg)
+    table = host_table("tiny")
+    ids, _ = token_stream("tiny")
+    parts = split_stream(ids, W)
+    H, D = params.heads, cfg["dim"]
+    douts = [host_dout("tiny", len(p[0]) * H, D, "f32", seed_offset=r) for r, p in
+             enumerate(parts)]
+    rpo = cfg["table_rows"] // W
+    ops = HostOps(cfg)
+    shards = [torch.from_numpy(table[r * rpo:(r + 1) * rpo].copy()) for r in range(W)]
+    fwd = owner.run_lockstep([owner.forward_steps(params, shards[r], W, *parts[r], ops=ops)
+                              for r in range(W)])
+    bwd = owner.run_lockstep([owner.backward_steps(params, W, fwd[r][1], douts[r], ops=ops)
+                              for r in range(W)])
+    outs, owners = expected(cfg, table, parts, douts, W)
+    for r in range(W):
+        assert np.array_equal(fwd[r][0].numpy(), outs[r])
+        u, g, nu = bwd[r]
+        assert int(nu[0]) == len(owners[r][0])
+        assert np.array_equal(u.numpy(), owners[r][0]) and np.array_equal(g.numpy(), owners[r][1])
+
+
+def test_rows_must_divide_among_owners():
+    from hashed_gram_embedding_raw_b200 import make_params, owner
+    cfg = dict(head_params("tiny"))
+    cfg["table_rows"] += 1
+    with pytest.raises(ValueError):
+        owner.rows_per_owner(make_params(cfg), 2)
+
+
+def _gloo_rank(rank, world, port, result_dir):
+    import datetime
+    import torch.distributed as dist
+    from hashed_gram_embedding_raw_b200 import make_params, owner
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        cfg = head_params("tiny")
+        params = make_params(cfg)
+        table = host_table("tiny")
+        ids, _ = token_stream("tiny")
+        parts = split_stream(ids, world)
+        H, D = params.heads, cfg["dim"]
+        douts = [host_dout("tiny", len(p[0]) * H, D, "f32", seed_offset=r)
+                 for r, p in enumerate(parts)]
+        out, u, g, nu = run_rank(owner, params, cfg, table, world, rank, *parts[rank],
+                                 douts[rank], lambda gen: owner.run_collective(gen))
+        outs, owners = expected(cfg, table, parts, douts, world)
+        ok = (np.array_equal(out.numpy(), outs[rank]) and int(nu[0]) == len(owners[rank][0])
+              and np.array_equal(u.numpy(), owners[rank][0])
+              and np.array_equal(g.numpy(), owners[rank][1]))
+        with open(os.path.join(result_dir, f"rank{rank}"), "w") as f:
+            f.write("ok" if ok else "mismatch")
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks(tmp_path):
+    import torch.multiprocessing as mp
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    mp.start_processes(_gloo_rank, args=(2, port, str(tmp_path)), nprocs=2, join=True,
+                       start_method="spawn")
+    for r in range(2):
+        assert (tmp_path / f"rank{r}").read_text() == "ok"
