@@ -9,6 +9,7 @@ gradients) over one batch of the named workload, all inputs resident in HBM.
     python bench.py --impl reference ...   # the CPU oracle, timed on this host
     python bench.py --stage ple ...        # the PLE tail kernel on its own workload
     python bench.py --stage ple_bwd ...    # the PLE tail's backward on the same workload
+    python bench.py --stage owner ...      # the owner-sharded table (NCCL all-to-alls)
     python bench.py --stage adam ...       # the sparse optimizer step on a table shard
 
 Multi-GPU (torchrun, one rank per GPU): every rank holds its own table
@@ -932,6 +933,107 @@ def run_adam(args):
     return 0
 
 
+# ------------------------------------------------- owner-sharded stage
+
+OWNER_METRIC = ("Engram tokens/s through the owner-sharded table (hash, owner grouping, "
+                "all-to-all of rows and values, owner lookup, request-order restore; backward "
+                "routed to the owners and reduced there)")
+
+
+def run_owner(args):
+    """--stage owner: the page's owner-sharded lookup and backward on the full
+    workload, every rank holding 1/N of the 320,001,536-row table and
+    requesting its own 16 x 4,096-token batch; the exchanges are NCCL
+    all-to-alls (a group of one rank when N = 1)."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    import hashed_gram_embedding_raw_b200 as E
+    from hashed_gram_embedding_raw_b200 import owner
+    from workloads import WORKLOADS, fill_device_table, head_params, host_dout, token_stream
+
+    rank, local_rank, world = rank_env()
+    assert torch.cuda.is_available(), "bench.py needs a CUDA device"
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=device,
+                                timeout=datetime.timedelta(seconds=300))
+    else:
+        import socket
+        with socket.socket() as sk:
+            sk.bind(("127.0.0.1", 0))
+            port = sk.getsockname()[1]
+        store = dist.TCPStore("127.0.0.1", port, 1, True,
+                              timeout=datetime.timedelta(seconds=60))
+        dist.init_process_group("nccl", store=store, rank=0, world_size=1, device_id=device,
+                                timeout=datetime.timedelta(seconds=300))
+    name = args.workload
+    w = WORKLOADS[name]
+    cfg = head_params(name)
+    params = E.make_params(cfg)
+    R, D, H = cfg["table_rows"], cfg["dim"], params.heads
+    rpo = owner.rows_per_owner(params, world)
+    tdtype = {"bf16": torch.bfloat16, "f32": torch.float32}[w.dtype]
+    shard = torch.empty((rpo, D), dtype=tdtype, device=device)
+    fill_device_table(shard, w.seed + rank)
+    ids_np, cu_np = token_stream(name)
+    T = len(ids_np)
+    ids = torch.from_numpy(ids_np.copy()).to(device)
+    cu = torch.from_numpy(cu_np.copy()).to(device)
+    dout = host_dout(name, T * H, D, w.dtype, seed_offset=rank).to(device)
+
+    def step():
+        out, routing = owner.run_collective(owner.forward_steps(params, shard, world, ids, cu))
+        return owner.run_collective(owner.backward_steps(params, world, routing, dout))
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    if E.engram_get_device_error():
+        raise RuntimeError("device error flag set during warm-up")
+    K = args.steps
+    stream = torch.cuda.current_stream(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = E.engram_launch_count()
+    barrier(device)
+    torch.cuda.synchronize(device)
+    with ClockSampler(gpu_smi_id(torch, device)) as clk:
+        e0.record(stream)
+        for _ in range(K):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+    barrier(device)
+    launches = E.engram_launch_count() - launches0
+    total_ms = max_over_ranks(e0.elapsed_time(e1), device)
+    if E.engram_get_device_error():
+        raise RuntimeError("device error flag set during timing")
+    esize = 2 if w.dtype == "bf16" else 4
+    line = {
+        "metric": OWNER_METRIC, "value": world * T * K / (total_ms / 1e3), "unit": UNIT,
+        "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": total_ms / K,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic",
+        "config": {"workload": name + "_owner", "tokens_per_step_per_gpu": T,
+                   "owners": world, "rows_per_owner": rpo,
+                   "exchange": "NCCL all_to_all_single, uneven splits",
+                   "all_to_all_bytes_per_step_per_gpu": T * H * (4 + 2 * D * esize),
+                   "l2": "inputs larger than L2"},
+        "gpu_launches": launches,
+        "clocks": clk.summary(),
+        "cpu_baseline": None,
+        "note": ("eager launches: the grouping counts cross to the host before each "
+                 "exchange, so the step cannot be one CUDA graph"),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -954,11 +1056,13 @@ def main(argv=None):
                     help="time the step as a replayed CUDA graph (default)")
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="time eager launches instead")
-    ap.add_argument("--stage", choices=["all", "bwd", "ple", "ple_bwd", "adam"], default="all",
+    ap.add_argument("--stage", choices=["all", "bwd", "ple", "ple_bwd", "adam", "owner"],
+                    default="all",
                     help="all: forward + backward (the step); bwd: the backward alone "
                          "(indices from engram_hash, no table allocated); ple: the PLE "
                          "tail (norm + short conv) on its own workload; ple_bwd: its "
-                         "backward on the same workload; adam: the sparse "
+                         "backward on the same workload; owner: the owner-sharded table "
+                         "with all-to-all exchanges; adam: the sparse "
                          "optimizer step on an 8-way owner shard of the table")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)      # at least 3 untimed warm-up steps
@@ -968,6 +1072,8 @@ def main(argv=None):
         return run_ple(args)
     if args.stage == "ple_bwd":
         return run_ple(args, backward=True)
+    if args.stage == "owner":
+        return run_owner(args)
     if args.stage == "adam":
         return run_adam(args)
     return run_ours(args)
