@@ -709,8 +709,8 @@ def run_ple(args, backward: bool = False):
         tname = "short_conv_bwd_kernel"
     else:
         alg = T * C * 2 * 2 + C * (K + 2) * 2 + cu.numel() * 4
-        kname = "short_conv_reg_kernel<bf16,bf16,4,3>"
-        tname = "short_conv_reg_kernel"
+        kname = "short_conv_cls_kernel<bf16,bf16,4>"
+        tname = "short_conv_cls_kernel"
     achieved = alg / kern_ms / 1e6
     line = {
         "metric": PLE_BWD_METRIC if backward else PLE_METRIC,

@@ -22,6 +22,7 @@
 #include "ple_conv.cuh"
 #include "ple_conv_reg.cuh"
 #include "ple_conv_bwd.cuh"
+#include "ple_conv_cls.cuh"
 #include "optim.cuh"
 #include "owner.cuh"
 #include "norm.cuh"
@@ -649,6 +650,7 @@ struct ConvPlan {
     size_t smem = 0;
     int grid = 0, threads = 0, chan = 4;
     bool reg = false;  // kernel width 4, dilation 3: history in registers
+    bool cls = false;  // kernel width <= 4, one residue class per block
 };
 
 bool overlaps(const void *a, size_t na, const void *b, size_t nb)
@@ -714,6 +716,21 @@ int conv_plan(const engram_conv_params_t *p, int32_t dtype, int32_t out_dtype, i
         P->threads = 32 * ((a.nth + 31) / 32 + ple::kRegRmsWarps);
         P->smem = ple::reg_smem_bytes(bufs, 9, pitch_reg);
     }
+    // kernel widths up to 4 on branches up to 2,560 channels (4 per thread):
+    // one residue class per block, batches of 8 rows in shared memory
+    const int cls_bufs = (int)std::min<size_t>(
+        ple::kClsMaxBufs,
+        (ple::kSmemLimit - ple::kClsDataOffset) / ((size_t)ple::kClsRows * pitch_reg));
+    P->cls = K <= ple::kClsTaps && G / 4 <= 32 * ple::kClsMaxConvWarps && cls_bufs >= 2;
+    if (P->cls) {
+        P->reg = false;
+        P->chan = 4;
+        a.nth = G / P->chan;
+        a.reg_bufs = cls_bufs;
+        a.pitch = pitch_reg;
+        P->threads = 32 * ((a.nth + 31) / 32 + ple::kClsStatWarps);
+        P->smem = ple::cls_smem_bytes(cls_bufs, pitch_reg);
+    }
     return ENGRAM_OK;
 }
 
@@ -723,6 +740,20 @@ int conv_grid(ConvPlan *P)
     int sms = 0;
     ENGRAM_TRY(device_sms(&sms));
     const int groups = P->a.C / P->a.G;
+    if (P->cls) {
+        // branches x residues x chunks, about one block per SM
+        const int classes = (int)std::max<int64_t>(1, std::min<int64_t>(P->a.dil, P->a.T));
+        const int64_t rows = std::max<int64_t>(1, ceil_div(P->a.T, P->a.dil));
+        int64_t chunks = std::max<int64_t>(1, sms / ((int64_t)groups * classes));
+        chunks = std::min<int64_t>(chunks, std::max<int64_t>(1, ceil_div(rows, 32)));
+        const int64_t grid = (int64_t)groups * classes * chunks;
+        if (grid > INT32_MAX)
+            return ENGRAM_EINVAL;
+        P->a.classes = classes;
+        P->a.bpg = (int32_t)chunks;
+        P->grid = (int)grid;
+        return ENGRAM_OK;
+    }
     int64_t bpg = std::max(1, sms / groups);
     bpg = std::min<int64_t>(bpg, std::max<int64_t>(1, ceil_div(P->a.T, 64)));
     if ((int64_t)groups * bpg > INT32_MAX)
@@ -760,6 +791,12 @@ int allow_smem(F fn)
 template <typename XT, typename OT>
 int launch_conv_t(const ConvPlan &P, cudaStream_t s)
 {
+    if (P.cls) {
+        auto fc = ple::short_conv_cls_kernel<XT, OT, 4>;
+        ENGRAM_TRY(allow_smem(fc));
+        fc<<<P.grid, P.threads, P.smem, s>>>(P.a);
+        return after_launch();
+    }
     if (P.reg) {
         auto fr = ple::short_conv_reg_kernel<XT, OT, 4, 3>;
         ENGRAM_TRY(allow_smem(fr));

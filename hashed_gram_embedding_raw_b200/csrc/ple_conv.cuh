@@ -61,8 +61,9 @@ struct ConvArgs {
     int32_t K, dil, halo;
     int32_t norm_slots; // rows of the private normalised history (halo + kRows)
     uint32_t flags;     // ENGRAM_CONV_* bits
-    int32_t reg_bufs;   // register-history kernel: row buffers of one block each
-    int32_t pitch;      // register-history kernel: bytes per buffered row
+    int32_t reg_bufs;   // register-history kernels: row buffers of one block each
+    int32_t pitch;      // register-history kernels: bytes per buffered row
+    int32_t classes;    // residue-class kernel: residues with rows, min(dil, T)
 };
 
 // Shared memory: inverse RMS [2][kChunk] float and history-tap counts
