@@ -975,7 +975,7 @@ int conv_bwd_plan(const engram_conv_params_t *p, int32_t dtype, int32_t grad_dty
         return ENGRAM_EINVAL;
     const int C = p->channels, G = p->group_size, K = p->kernel_size, d = p->dilation;
     if (C < 1 || G < 8 || C % G != 0 || G % 8 != 0 ||
-        G / 8 > ple::kBwdThreads * ple::kBwdMaxCluster)
+        G / 4 > ple::kBwdThreads * ple::kBwdMaxCluster)
         return ENGRAM_EINVAL;
     if (K < 1 || K > ple::kBwdTaps || d < 1 || d > 4096 || p->reserved != 0)
         return ENGRAM_EINVAL;
@@ -983,11 +983,9 @@ int conv_bwd_plan(const engram_conv_params_t *p, int32_t dtype, int32_t grad_dty
         return ENGRAM_EINVAL;
     if (T < 0 || T > INT32_MAX)
         return ENGRAM_EINVAL;
-    // branches wider than one block's 160 threads x 8 channels: two blocks of a
-    // cluster, one half each (G / 2 stays a multiple of 8)
-    const int csize = G / 8 > ple::kBwdThreads ? 2 : 1;
-    if (G % (8 * csize) != 0)
-        return ENGRAM_EINVAL;
+    // branches wider than one block's 320 threads x 4 channels: two blocks of a
+    // cluster, one half each (G / 2 stays a multiple of 4)
+    const int csize = G / 4 > ple::kBwdThreads ? 2 : 1;
     const int gc = G / csize;
     const int pitch_x = (gc * ex + 127) / 128 * 128, pitch_g = (gc * eg + 127) / 128 * 128;
     const int fit = (int)((ple::kSmemLimit - ple::kBwdDataOffset) / (size_t)(pitch_x + pitch_g));
@@ -1000,7 +998,7 @@ int conv_bwd_plan(const engram_conv_params_t *p, int32_t dtype, int32_t grad_dty
     a.T = T;
     a.C = C;
     a.G = G;
-    a.nth = gc / 8;
+    a.nth = gc / 4;
     a.dil = d;
     a.K = K;
     a.wdtype = p->weight_dtype;

@@ -17,14 +17,15 @@
 // The convolution only couples rows of one residue modulo d, so a unit of
 // work is one branch, one residue r and a range [ja, jb) of that residue's
 // rows j (token t = r + j d): along them the convolution has dilation 1. A
-// thread owns 8 channels and keeps about 250 registers of state (the dy ring,
-// weights, weight-gradient sums), so a block has at most 5 warps (two per
-// scheduler) and a branch wider than 1,280 channels is split between the two
-// blocks of a cluster, which exchange their per-row partial sums through
-// distributed shared memory. The unit walks its rows in batches of B = 4,
+// thread owns 4 channels and keeps their state in registers (the dy ring of 7
+// rows, weights, weight-gradient sums: at 8 channels this needed ~250
+// registers, five warps per SM), 168 registers at ten warps per block; a
+// branch wider than 1,280 channels is split between the two blocks of a
+// cluster, which exchange their per-row partial sums through distributed
+// shared memory. The unit walks its rows in batches of B = 4,
 // with the kernel width fixed at 4 (narrower kernels run with zero taps) so
 // that the lag of the transposed convolution is 3 rows:
-//   stage 1  every thread sums the squares of its 8 channels of the batch's
+//   stage 1  every thread sums the squares of its 4 channels of the batch's
 //            rows (one warp sum for four rows); warps post partial sums to
 //            both blocks;
 //   barrier (over the cluster)
@@ -54,16 +55,16 @@ namespace ple {
 constexpr int kBwdRows = 4;                    // rows per batch
 constexpr int kBwdTaps = 4;                    // kernel widths 1..4
 constexpr int kBwdLag = kBwdTaps - 1;
-constexpr int kBwdCtaWarps = 5;                // per block of a cluster
-constexpr int kBwdThreads = 32 * kBwdCtaWarps; // 8 channels per thread
+constexpr int kBwdCtaWarps = 10;               // per block of a cluster
+constexpr int kBwdThreads = 32 * kBwdCtaWarps; // 4 channels per thread
 constexpr int kBwdMaxCluster = 2;              // blocks sharing a branch: G <= 2560
-constexpr int kBwdPartStride = 12;             // per-row partials, padded for float4 reads
+constexpr int kBwdPartStride = 24;             // per-row partials (20 warps), padded for float4
 constexpr int kBwdMaxSlots = 32;
 constexpr int kBwdBars = 8;
 constexpr int kBwdQuantities = kBwdTaps + 2;   // weight taps, bias, norm scale
 
-// Shared memory: square-sum and dot partials [B][12] float each (column
-// rank * 5 + warp; the pads stay zero), inverse RMS
+// Shared memory: square-sum and dot partials [B][24] float each (column
+// rank * 10 + warp; the pads stay zero), inverse RMS
 // [32] float and tap counts [32] int32 per row slot, mbarriers [8]; then the
 // row slots of x [slots][pitch_x] and of dout [slots][pitch_g].
 constexpr int kBwdOffDot = kBwdRows * kBwdPartStride * 4;
@@ -120,36 +121,45 @@ __device__ __forceinline__ void st_cluster(const float *local, uint32_t rank, fl
     asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(remote), "f"(v) : "memory");
 }
 
-// 8 channels of one row in a shared-memory slot, as floats.
+// 4 channels of one row in a shared-memory slot (8 or 16 bytes), as floats.
 template <typename T>
-__device__ __forceinline__ void load_slot8(const unsigned char *p, float *f)
+__device__ __forceinline__ void load_slot4(const unsigned char *p, float *f)
 {
-    constexpr int W = 8 * (int)sizeof(T) / 4;
-    uint32_t w[W];
-#pragma unroll
-    for (int q = 0; q < W / 4; ++q) {
-        const uint4 u = reinterpret_cast<const uint4 *>(p)[q];
-        w[4 * q] = u.x;
-        w[4 * q + 1] = u.y;
-        w[4 * q + 2] = u.z;
-        w[4 * q + 3] = u.w;
+    uint32_t w[4];
+    if constexpr (sizeof(T) == 2) {
+        const uint2 u = *reinterpret_cast<const uint2 *>(p);
+        w[0] = u.x;
+        w[1] = u.y;
+    } else {
+        const uint4 u = *reinterpret_cast<const uint4 *>(p);
+        w[0] = u.x;
+        w[1] = u.y;
+        w[2] = u.z;
+        w[3] = u.w;
     }
-    Elem<T>::template unpack<8>(w, f);
+    Elem<T>::template unpack<4>(w, f);
 }
 
-// sum over 12 padded per-warp partials of row i
-__device__ __forceinline__ float sum_parts(const float *part, int i)
+// The totals of the four rows' padded per-warp partials, in every lane: lane
+// l adds columns l % 8, +8, +16 of row l / 8, the eight lanes of a row combine
+// by shuffles, and each row's total is broadcast from its first lane.
+__device__ __forceinline__ void sum_parts4(const float *part, int lane, float (&tot)[4])
 {
-    const float4 *p = reinterpret_cast<const float4 *>(part + i * kBwdPartStride);
-    const float4 a = p[0], b = p[1], c = p[2];
-    return ((a.x + a.y) + (a.z + a.w)) + ((b.x + b.y) + (b.z + b.w)) +
-           ((c.x + c.y) + (c.z + c.w));
+    static_assert(kBwdPartStride == 24 && kBwdRows == 4, "lane layout");
+    const float *p = part + (lane >> 3) * kBwdPartStride + (lane & 7);
+    float v = (p[0] + p[8]) + p[16];
+    v += __shfl_xor_sync(kFull, v, 4);
+    v += __shfl_xor_sync(kFull, v, 2);
+    v += __shfl_xor_sync(kFull, v, 1);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        tot[i] = __shfl_sync(kFull, v, 8 * i);
 }
 
 template <typename XT, typename GT>
 __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const ConvBwdArgs a)
 {
-    constexpr int B = kBwdRows, L = kBwdLag, KT = kBwdTaps, CH = 8, NP = CH / 2;
+    constexpr int B = kBwdRows, L = kBwdLag, KT = kBwdTaps, CH = 4, NP = CH / 2;
     constexpr int RING = L + B;
     extern __shared__ __align__(128) unsigned char smem[];
     float *ss_part = reinterpret_cast<float *>(smem);
@@ -184,10 +194,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
     if (ja >= jb) {  // no rows: the block's partials are zero
         if (active)
 #pragma unroll
-            for (int q = 0; q < kBwdQuantities; ++q) {
-                reinterpret_cast<float4 *>(part + (size_t)q * a.C)[0] = make_float4(0, 0, 0, 0);
-                reinterpret_cast<float4 *>(part + (size_t)q * a.C)[1] = make_float4(0, 0, 0, 0);
-            }
+            for (int q = 0; q < kBwdQuantities; ++q)
+                *reinterpret_cast<float4 *>(part + (size_t)q * a.C) = make_float4(0, 0, 0, 0);
         return;
     }
     const int64_t js = ja - L > 0 ? ja - L : 0;
@@ -323,7 +331,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
     // x of ring row q (rows j0 - L .. j0 + B - 1) of the batch, normalised
     auto load_xh = [&](int slot, float iv, float2 *xh) {
         float f[CH];
-        load_slot8<XT>(xs + (size_t)slot * a.pitch_x + xoff, f);
+        load_slot4<XT>(xs + (size_t)slot * a.pitch_x + xoff, f);
         const float2 iv2 = make_float2(iv, iv);
 #pragma unroll
         for (int pp = 0; pp < NP; ++pp)
@@ -353,7 +361,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
                 float2 acc = zero2;
                 if (active && j0 + i < je) {
                     float f[CH];
-                    load_slot8<XT>(xs + (size_t)slot[L + i] * a.pitch_x + xoff, f);
+                    load_slot4<XT>(xs + (size_t)slot[L + i] * a.pitch_x + xoff, f);
 #pragma unroll
                     for (int pp = 0; pp < NP; ++pp) {
                         const float2 x2 = make_float2(f[2 * pp], f[2 * pp + 1]);
@@ -373,11 +381,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
 #pragma unroll
         for (int q = 0; q < L; ++q)
             inv[q] = inv_s[slot[q]];
+        {
+            float tot[B];
+            if (do_norm)
+                sum_parts4(ss_part, lane, tot);
 #pragma unroll
-        for (int i = 0; i < B; ++i) {
-            inv[L + i] = do_norm ? rsqrtf(fmaf(sum_parts(ss_part, i), a.inv_G, a.eps)) : 1.f;
-            if (tid == 0)
-                inv_s[slot[L + i]] = inv[L + i];
+            for (int i = 0; i < B; ++i) {
+                inv[L + i] = do_norm ? rsqrtf(fmaf(tot[i], a.inv_G, a.eps)) : 1.f;
+                if (tid == 0)
+                    inv_s[slot[L + i]] = inv[L + i];
+            }
         }
         // taps: a row of the ring feeds rows i = q - L + k of the batch, tap k
         int back[B];
@@ -421,7 +434,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
             const bool need = active && j < je && j >= ja;
             float g[CH];
             if (need)
-                load_slot8<GT>(gs + (size_t)slot[L + i] * a.pitch_g + goff, g);
+                load_slot4<GT>(gs + (size_t)slot[L + i] * a.pitch_g + goff, g);
 #pragma unroll
             for (int pp = 0; pp < NP; ++pp) {
                 const float2 y = __ffma2_rn(sc[pp], acc[i][pp], bias[pp]);
@@ -482,17 +495,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
         sync_all();
 
         // ---- stage 4: dx of the lagged rows
+        float means[B];
+        if (do_norm)
+            sum_parts4(dot_part, lane, means);
 #pragma unroll
         for (int i = 0; i < B; ++i) {
             const int64_t jj = j0 - L + i;
             if (!active || jj < ja || jj >= jb)
                 continue;
-            const float mean = do_norm ? sum_parts(dot_part, i) * a.inv_G : 0.f;
+            const float mean = do_norm ? means[i] * a.inv_G : 0.f;
             float g[CH], o[CH];
             float2 xh[NP];
             load_xh(slot[i], inv[i], xh);
             if (do_res)
-                load_slot8<GT>(gs + (size_t)slot[i] * a.pitch_g + goff, g);
+                load_slot4<GT>(gs + (size_t)slot[i] * a.pitch_g + goff, g);
             const float2 ij2 = make_float2(inv[i], inv[i]), mean2 = make_float2(-mean, -mean);
 #pragma unroll
             for (int pp = 0; pp < NP; ++pp) {
@@ -526,9 +542,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
     // partials of this block: s * dw per tap, dbias, dnorm_w (zero without the norm)
     if (active) {
         auto put = [&](int q, const float2 *v) {
-            float4 *dst = reinterpret_cast<float4 *>(part + (size_t)q * a.C);
-            dst[0] = make_float4(v[0].x, v[0].y, v[1].x, v[1].y);
-            dst[1] = make_float4(v[2].x, v[2].y, v[3].x, v[3].y);
+            *reinterpret_cast<float4 *>(part + (size_t)q * a.C) =
+                make_float4(v[0].x, v[0].y, v[1].x, v[1].y);
         };
 #pragma unroll
         for (int k = 0; k < KT; ++k) {
