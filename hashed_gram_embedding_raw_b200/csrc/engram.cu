@@ -990,7 +990,7 @@ int conv_bwd_plan(const engram_conv_params_t *p, int32_t dtype, int32_t grad_dty
     const int pitch_x = (gc * ex + 127) / 128 * 128, pitch_g = (gc * eg + 127) / 128 * 128;
     const int fit = (int)((ple::kSmemLimit - ple::kBwdDataOffset) / (size_t)(pitch_x + pitch_g));
     const int slots_max = std::min(fit, ple::kBwdMaxSlots);
-    const int ahead = std::min((slots_max - ple::kBwdLag) / ple::kBwdRows - 1, ple::kBwdBars - 2);
+    const int ahead = std::min((slots_max - ple::kBwdLag) / ple::kBwdRows - 2, ple::kBwdBars - 2);
     if (ahead < 1)
         return ENGRAM_EINVAL;
     ple::ConvBwdArgs &a = P->a;
@@ -1006,7 +1006,7 @@ int conv_bwd_plan(const engram_conv_params_t *p, int32_t dtype, int32_t grad_dty
     a.inv_G = 1.f / (float)G;
     a.flags = p->flags;
     a.ahead = ahead;
-    a.slots = ple::kBwdLag + (ahead + 1) * ple::kBwdRows;
+    a.slots = ple::kBwdLag + (ahead + 2) * ple::kBwdRows;
     a.pitch_x = pitch_x;
     a.pitch_g = pitch_g;
     a.csize = csize;

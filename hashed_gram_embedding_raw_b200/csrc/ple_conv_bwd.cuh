@@ -28,14 +28,16 @@
 //   stage 1  every thread sums the squares of its 4 channels of the batch's
 //            rows (one warp sum for four rows); warps post partial sums to
 //            both blocks;
-//   barrier (over the cluster)
 //   stage 2  inverse RMS of the four rows; every row of the ring (j0 - 3 ..
 //            j0 + 3) is read and normalised once and added into the y of the
 //            batch rows it is a tap of; dy into a register ring;
 //   stage 3  for the lagged rows j0 - 3 .. j0: dn from the ring, the weight
 //            gradients, and partials of sum(s dn xh), posted to both blocks;
-//   barrier (over the cluster)
 //   stage 4  dx of the lagged rows (streaming stores), then the ring shifts.
+// Stages 1 and 3 post partial sums that stages 2 and 4 need complete; the
+// batches are software-pipelined so that one barrier (over the cluster)
+// serves both: iteration b runs stage 4 of batch b - 1, stages 2 and 3 of
+// batch b and stage 1 of batch b + 1, then the barrier.
 // Rows whose taps all stay inside their sequence (nearly all) take a path
 // without per-tap masks. Rows reach shared memory through a ring of row
 // slots filled by cp.async.bulk (one copy per row of x and of dout, issued
@@ -63,13 +65,14 @@ constexpr int kBwdMaxSlots = 32;
 constexpr int kBwdBars = 8;
 constexpr int kBwdQuantities = kBwdTaps + 2;   // weight taps, bias, norm scale
 
-// Shared memory: square-sum and dot partials [B][24] float each (column
-// rank * 10 + warp; the pads stay zero), inverse RMS
-// [32] float and tap counts [32] int32 per row slot, mbarriers [8]; then the
-// row slots of x [slots][pitch_x] and of dout [slots][pitch_g].
-constexpr int kBwdOffDot = kBwdRows * kBwdPartStride * 4;
-constexpr int kBwdOffInv = 2 * kBwdOffDot;
-constexpr int kBwdOffMeta = kBwdOffInv + kBwdMaxSlots * 4;
+// Shared memory: square-sum and dot partials [2][B][24] float each (by batch
+// parity; column rank * 10 + warp; the pads stay zero), tap counts [32] int32
+// per row slot, mbarriers [8]; then the row slots of x [slots][pitch_x] and
+// of dout [slots][pitch_g]. With batches in flight from the one being
+// finished (its window reaches 3 rows back) to `ahead` past the next,
+// slots = 3 + (ahead + 2) * 4.
+constexpr int kBwdOffDot = 2 * kBwdRows * kBwdPartStride * 4;  // two buffers each
+constexpr int kBwdOffMeta = 2 * kBwdOffDot;
 constexpr int kBwdOffBars = kBwdOffMeta + kBwdMaxSlots * 4;
 constexpr int kBwdHeader = kBwdOffBars + kBwdBars * 8;
 constexpr int kBwdDataOffset = (kBwdHeader + 127) / 128 * 128;
@@ -164,7 +167,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
     extern __shared__ __align__(128) unsigned char smem[];
     float *ss_part = reinterpret_cast<float *>(smem);
     float *dot_part = reinterpret_cast<float *>(smem + kBwdOffDot);
-    float *inv_s = reinterpret_cast<float *>(smem + kBwdOffInv);
     int32_t *meta_s = reinterpret_cast<int32_t *>(smem + kBwdOffMeta);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kBwdOffBars);
     unsigned char *xs = smem + kBwdDataOffset;
@@ -225,12 +227,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
             mbar_init(bars + b, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    for (int i = tid; i < 2 * B * kBwdPartStride; i += blockDim.x)
+    for (int i = tid; i < 4 * B * kBwdPartStride; i += blockDim.x)
         ss_part[i] = 0.f;  // (and dot_part) pads of absent warps stay zero
-    for (int i = tid; i < kBwdMaxSlots; i += blockDim.x) {
-        inv_s[i] = 0.f;
+    for (int i = tid; i < kBwdMaxSlots; i += blockDim.x)
         meta_s[i] = 0;
-    }
     // (every block of the cluster has started and zeroed its partials before
     // any block writes into another's)
     auto sync_all = [&]() {
@@ -338,10 +338,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
             xh[pp] = __fmul2_rn(make_float2(f[2 * pp], f[2 * pp + 1]), iv2);
     };
 
-    for (int b = 0; b < nbatch; ++b) {
-        const int64_t j0 = js + (int64_t)b * B;
-        // slots of ring rows j0 - L .. j0 + B - 1
-        int slot[RING];
+    // slots of the ring rows j0 - L .. j0 + B - 1 of the batch starting at j0
+    auto window_slots = [&](int64_t j0, int (&slot)[RING]) {
         slot[L] = (int)((j0 - js) % S);
 #pragma unroll
         for (int q = L - 1; q >= 0; --q)
@@ -349,48 +347,125 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
 #pragma unroll
         for (int q = L + 1; q < RING; ++q)
             slot[q] = slot[q - 1] + 1 == S ? 0 : slot[q - 1] + 1;
+    };
+    constexpr int PB = B * kBwdPartStride;  // one buffer of partials
+
+    // ---- stage 1 of batch b: wait for its rows, post the squares of its rows
+    auto stage1 = [&](int b) {
+        const int64_t j0 = js + (int64_t)b * B;
         if (j0 < je && !timed_out &&
             !mbar_wait(bars + b % kBwdBars, (uint32_t)(b / kBwdBars) & 1u))
             timed_out = true;
-
-        // ---- stage 1: squares of the batch's rows
-        if (do_norm) {
-            float ss[B];
+        if (!do_norm)
+            return;
+        int sl = (int)((j0 - js) % S);
+        float ss[B];
 #pragma unroll
-            for (int i = 0; i < B; ++i) {
-                float2 acc = zero2;
-                if (active && j0 + i < je) {
-                    float f[CH];
-                    load_slot4<XT>(xs + (size_t)slot[L + i] * a.pitch_x + xoff, f);
+        for (int i = 0; i < B; ++i, sl = sl + 1 == S ? 0 : sl + 1) {
+            float2 acc = zero2;
+            if (active && j0 + i < je) {
+                float f[CH];
+                load_slot4<XT>(xs + (size_t)sl * a.pitch_x + xoff, f);
 #pragma unroll
-                    for (int pp = 0; pp < NP; ++pp) {
-                        const float2 x2 = make_float2(f[2 * pp], f[2 * pp + 1]);
-                        acc = __ffma2_rn(x2, x2, acc);
-                    }
+                for (int pp = 0; pp < NP; ++pp) {
+                    const float2 x2 = make_float2(f[2 * pp], f[2 * pp + 1]);
+                    acc = __ffma2_rn(x2, x2, acc);
                 }
-                ss[i] = acc.x + acc.y;
             }
-            post(ss_part, warp_sum4(ss[0], ss[1], ss[2], ss[3], lane));
+            ss[i] = acc.x + acc.y;
         }
-        sync_all();
-        if (wid == 0 && b + a.ahead < nbatch)
-            issue(b + a.ahead);
+        post(ss_part + (b & 1) * PB, warp_sum4(ss[0], ss[1], ss[2], ss[3], lane));
+    };
+
+    float inv[RING];  // inverse RMS of the ring rows
+#pragma unroll
+    for (int q = 0; q < RING; ++q)
+        inv[q] = 0.f;
+
+    // ---- stage 4 of batch b: dx of its lagged rows (ring rows 0 .. B - 1),
+    // once the dot partials it posted are complete
+    auto stage4 = [&](int b) {
+        const int64_t j0 = js + (int64_t)b * B;
+        int slot[RING];
+        window_slots(j0, slot);
+        int fwd[B];
+        bool full_fwd = j0 - L >= ja && j0 - L + B <= jb;
+#pragma unroll
+        for (int i = 0; i < B; ++i) {
+            fwd[i] = meta_s[slot[i]] >> 8;
+            full_fwd = full_fwd && fwd[i] == L;
+        }
+        float means[B];
+        if (do_norm)
+            sum_parts4(dot_part + (b & 1) * PB, lane, means);
+#pragma unroll
+        for (int i = 0; i < B; ++i) {
+            const int64_t jj = j0 - L + i;
+            if (!active || jj < ja || jj >= jb)
+                continue;
+            const float mean = do_norm ? means[i] * a.inv_G : 0.f;
+            float g[CH], o[CH];
+            float2 xh[NP];
+            load_xh(slot[i], inv[i], xh);
+            if (do_res)
+                load_slot4<GT>(gs + (size_t)slot[i] * a.pitch_g + goff, g);
+            const float2 ij2 = make_float2(inv[i], inv[i]), mean2 = make_float2(-mean, -mean);
+#pragma unroll
+            for (int pp = 0; pp < NP; ++pp) {
+                float2 dn = zero2;
+#pragma unroll
+                for (int k = 0; k < KT; ++k)
+                    dn = __ffma2_rn(w[k][pp], full_fwd || k <= fwd[i] ? dy[i + k][pp] : zero2,
+                                    dn);
+                float2 v = do_norm ? __fmul2_rn(ij2, __ffma2_rn(xh[pp], mean2,
+                                                                __fmul2_rn(sc[pp], dn)))
+                                   : dn;
+                if (do_res)
+                    v = __fadd2_rn(v, make_float2(g[2 * pp], g[2 * pp + 1]));
+                o[2 * pp] = v.x;
+                o[2 * pp + 1] = v.y;
+            }
+            constexpr int OW = CH * (int)sizeof(GT) / 4;
+            uint32_t ow[OW];
+            Elem<GT>::template pack<CH>(o, ow);
+            const int64_t t = r + jj * d;
+            store_words<OW * 4>(dxb + t * grow, ow);
+        }
+    };
+
+    // The batches are pipelined so that one barrier separates them: iteration
+    // b finishes batch b - 1 (stage 4), computes batch b (stages 2 and 3) and
+    // posts the squares of batch b + 1 (stage 1); partials are double-buffered
+    // by batch parity, so a warp that runs ahead never overwrites partials
+    // another warp still reads.
+    stage1(0);
+    sync_all();
+    if (wid == 0 && a.ahead < nbatch)
+        issue(a.ahead);
+    for (int b = 0; b < nbatch; ++b) {
+        const int64_t j0 = js + (int64_t)b * B;
+        if (b > 0) {
+            stage4(b - 1);
+            // the ring moves on by one batch
+#pragma unroll
+            for (int i = 0; i < L; ++i) {
+                inv[i] = inv[i + B];
+#pragma unroll
+                for (int pp = 0; pp < NP; ++pp)
+                    dy[i][pp] = dy[i + B][pp];
+            }
+        }
+        int slot[RING];
+        window_slots(j0, slot);
 
         // ---- stage 2: inverse RMS, y and dy of the batch's rows
-        float inv[RING];  // of the ring rows: earlier batches' from shared memory
-#pragma unroll
-        for (int q = 0; q < L; ++q)
-            inv[q] = inv_s[slot[q]];
         {
             float tot[B];
             if (do_norm)
-                sum_parts4(ss_part, lane, tot);
+                sum_parts4(ss_part + (b & 1) * PB, lane, tot);
 #pragma unroll
-            for (int i = 0; i < B; ++i) {
+            for (int i = 0; i < B; ++i)
                 inv[L + i] = do_norm ? rsqrtf(fmaf(tot[i], a.inv_G, a.eps)) : 1.f;
-                if (tid == 0)
-                    inv_s[slot[L + i]] = inv[L + i];
-            }
         }
         // taps: a row of the ring feeds rows i = q - L + k of the batch, tap k
         int back[B];
@@ -490,54 +565,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
                 dotv[i] = accd.x + accd.y;
             }
             if (do_norm)
-                post(dot_part, warp_sum4(dotv[0], dotv[1], dotv[2], dotv[3], lane));
+                post(dot_part + (b & 1) * PB,
+                     warp_sum4(dotv[0], dotv[1], dotv[2], dotv[3], lane));
         }
+        if (b + 1 < nbatch)
+            stage1(b + 1);
         sync_all();
-
-        // ---- stage 4: dx of the lagged rows
-        float means[B];
-        if (do_norm)
-            sum_parts4(dot_part, lane, means);
-#pragma unroll
-        for (int i = 0; i < B; ++i) {
-            const int64_t jj = j0 - L + i;
-            if (!active || jj < ja || jj >= jb)
-                continue;
-            const float mean = do_norm ? means[i] * a.inv_G : 0.f;
-            float g[CH], o[CH];
-            float2 xh[NP];
-            load_xh(slot[i], inv[i], xh);
-            if (do_res)
-                load_slot4<GT>(gs + (size_t)slot[i] * a.pitch_g + goff, g);
-            const float2 ij2 = make_float2(inv[i], inv[i]), mean2 = make_float2(-mean, -mean);
-#pragma unroll
-            for (int pp = 0; pp < NP; ++pp) {
-                float2 dn = zero2;
-#pragma unroll
-                for (int k = 0; k < KT; ++k)
-                    dn = __ffma2_rn(w[k][pp], full_fwd || k <= fwd[i] ? dy[i + k][pp] : zero2,
-                                    dn);
-                float2 v = do_norm ? __fmul2_rn(ij2, __ffma2_rn(xh[pp], mean2,
-                                                                __fmul2_rn(sc[pp], dn)))
-                                   : dn;
-                if (do_res)
-                    v = __fadd2_rn(v, make_float2(g[2 * pp], g[2 * pp + 1]));
-                o[2 * pp] = v.x;
-                o[2 * pp + 1] = v.y;
-            }
-            constexpr int OW = CH * (int)sizeof(GT) / 4;
-            uint32_t ow[OW];
-            Elem<GT>::template pack<CH>(o, ow);
-            const int64_t t = r + jj * d;
-            store_words<OW * 4>(dxb + t * grow, ow);
-        }
-        // the ring moves on by one batch
-#pragma unroll
-        for (int i = 0; i < L; ++i)
-#pragma unroll
-            for (int pp = 0; pp < NP; ++pp)
-                dy[i][pp] = dy[i + B][pp];
+        if (wid == 0 && b + 1 + a.ahead < nbatch)
+            issue(b + 1 + a.ahead);
     }
+    if (nbatch > 0)
+        stage4(nbatch - 1);
 
     // partials of this block: s * dw per tap, dbias, dnorm_w (zero without the norm)
     if (active) {
