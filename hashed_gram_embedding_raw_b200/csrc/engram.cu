@@ -20,7 +20,6 @@
 #include "common.cuh"
 #include "hash_gather.cuh"
 #include "ple_conv.cuh"
-#include "ple_conv_reg.cuh"
 #include "ple_conv_bwd.cuh"
 #include "ple_conv_cls.cuh"
 #include "optim.cuh"
@@ -649,7 +648,6 @@ struct ConvPlan {
     ple::ConvArgs a;
     size_t smem = 0;
     int grid = 0, threads = 0, chan = 4;
-    bool reg = false;  // kernel width 4, dilation 3: history in registers
     bool cls = false;  // kernel width <= 4, one residue class per block
 };
 
@@ -704,18 +702,7 @@ int conv_plan(const engram_conv_params_t *p, int32_t dtype, int32_t out_dtype, i
     P->chan = chan;
     P->threads = (nth + 31) / 32 * 32;
     P->smem = ple::smem_bytes(norm_slots, nth, chan);
-    // kernel width 4, dilation 3: blocks of 9 rows buffered in shared memory
-    const int pitch_reg = (G * eb + 127) / 128 * 128;
-    const int bufs = (int)std::min<size_t>(
-        ple::kRegMaxBufs, (ple::kSmemLimit - ple::kRegDataOffset) / ((size_t)9 * pitch_reg));
-    P->reg = K == 4 && d == 3 && G / 8 <= 32 * ple::kRegMaxConvWarps && bufs >= 2;
-    if (P->reg) {
-        a.nth = G / 8;
-        a.reg_bufs = bufs;
-        a.pitch = pitch_reg;
-        P->threads = 32 * ((a.nth + 31) / 32 + ple::kRegRmsWarps);
-        P->smem = ple::reg_smem_bytes(bufs, 9, pitch_reg);
-    }
+    const int pitch_reg = (G * eb + 127) / 128 * 128;  // bytes per buffered row
     // kernel widths up to 4 on branches up to 2,560 channels (4 per thread):
     // one residue class per block, batches of 8 rows in shared memory
     const int cls_bufs = (int)std::min<size_t>(
@@ -723,7 +710,6 @@ int conv_plan(const engram_conv_params_t *p, int32_t dtype, int32_t out_dtype, i
         (ple::kSmemLimit - ple::kClsDataOffset) / ((size_t)ple::kClsRows * pitch_reg));
     P->cls = K <= ple::kClsTaps && G / 4 <= 32 * ple::kClsMaxConvWarps && cls_bufs >= 2;
     if (P->cls) {
-        P->reg = false;
         P->chan = 4;
         a.nth = G / P->chan;
         a.reg_bufs = cls_bufs;
@@ -784,10 +770,9 @@ int allow_smem(F fn)
     return ENGRAM_OK;
 }
 
-// The page's kernel width and dilation (4, 3) on branches up to 2,560
-// channels: the register-history kernel. Otherwise branches up to 2,560
-// channels take 4 channels per thread (kernel width 4 and the norm alone
-// specialised), wider branches 8.
+// Kernel widths up to 4 on branches up to 2,560 channels (the page's shape):
+// the residue-class kernel. Otherwise the chunked kernel, 4 channels per
+// thread up to 2,560 channels, 8 beyond.
 template <typename XT, typename OT>
 int launch_conv_t(const ConvPlan &P, cudaStream_t s)
 {
@@ -797,16 +782,8 @@ int launch_conv_t(const ConvPlan &P, cudaStream_t s)
         fc<<<P.grid, P.threads, P.smem, s>>>(P.a);
         return after_launch();
     }
-    if (P.reg) {
-        auto fr = ple::short_conv_reg_kernel<XT, OT, 4, 3>;
-        ENGRAM_TRY(allow_smem(fr));
-        fr<<<P.grid, P.threads, P.smem, s>>>(P.a);
-        return after_launch();
-    }
-    auto fn = P.chan == 8      ? ple::short_conv_kernel<XT, OT, 0, 8>
-              : P.a.K == 4 ? ple::short_conv_kernel<XT, OT, 4, 4>
-              : P.a.K == 1 ? ple::short_conv_kernel<XT, OT, 1, 4>
-                           : ple::short_conv_kernel<XT, OT, 0, 4>;
+    auto fn = P.chan == 8 ? ple::short_conv_kernel<XT, OT, 0, 8>
+                          : ple::short_conv_kernel<XT, OT, 0, 4>;
     ENGRAM_TRY(allow_smem(fn));
     fn<<<P.grid, P.threads, P.smem, s>>>(P.a);
     return after_launch();

@@ -61,8 +61,8 @@ struct ConvArgs {
     int32_t K, dil, halo;
     int32_t norm_slots; // rows of the private normalised history (halo + kRows)
     uint32_t flags;     // ENGRAM_CONV_* bits
-    int32_t reg_bufs;   // register-history kernels: row buffers of one block each
-    int32_t pitch;      // register-history kernels: bytes per buffered row
+    int32_t reg_bufs;   // residue-class kernel: row buffers (of 8 rows each)
+    int32_t pitch;      // residue-class kernel: bytes per buffered row
     int32_t classes;    // residue-class kernel: residues with rows, min(dil, T)
 };
 

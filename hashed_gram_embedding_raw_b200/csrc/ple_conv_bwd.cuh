@@ -49,7 +49,8 @@
 // timing.
 #pragma once
 
-#include "ple_conv_reg.cuh"
+#include "async_copy.cuh"
+#include "ple_conv.cuh"
 
 namespace engram {
 namespace ple {

@@ -31,7 +31,8 @@
 // The 3 rows before a range are read for history only.
 #pragma once
 
-#include "ple_conv_reg.cuh"
+#include "async_copy.cuh"
+#include "ple_conv.cuh"
 
 namespace engram {
 namespace ple {
