@@ -125,23 +125,25 @@ __device__ __forceinline__ void st_cluster(const float *local, uint32_t rank, fl
     asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(remote), "f"(v) : "memory");
 }
 
-// 4 channels of one row in a shared-memory slot (8 or 16 bytes), as floats.
+// 4 channels of one row in a shared-memory slot (8 or 16 bytes at the
+// shared-window address `addr`), as floats.
 template <typename T>
-__device__ __forceinline__ void load_slot4(const unsigned char *p, float *f)
+__device__ __forceinline__ void load_slot4(uint32_t addr, float *f)
 {
     uint32_t w[4];
-    if constexpr (sizeof(T) == 2) {
-        const uint2 u = *reinterpret_cast<const uint2 *>(p);
-        w[0] = u.x;
-        w[1] = u.y;
-    } else {
-        const uint4 u = *reinterpret_cast<const uint4 *>(p);
-        w[0] = u.x;
-        w[1] = u.y;
-        w[2] = u.z;
-        w[3] = u.w;
-    }
+    if constexpr (sizeof(T) == 2)
+        asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(w[0]), "=r"(w[1]) : "r"(addr));
+    else
+        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                     : "r"(addr));
     Elem<T>::template unpack<4>(w, f);
+}
+
+// Number of taps k in 1..3 with k * d <= span (span < 0 counts as 0).
+__device__ __forceinline__ int taps_within(int32_t span, int32_t d)
+{
+    return (span >= d) + (span >= 2 * d) + (span >= 3 * d);
 }
 
 // The totals of the four rows' padded per-warp partials, in every lane: lane
@@ -186,8 +188,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
     const int m = unit / per_branch;
     const int rem = unit - m * per_branch;
     const int r = rem / a.chunks, p = rem - r * a.chunks;
-    const int64_t nr = a.T > r ? (a.T - r + d - 1) / d : 0;  // rows of residue r
-    const int64_t ja = nr * p / a.chunks, jb = nr * (p + 1) / a.chunks;
+    // row indices fit 32 bits (T < 2^31)
+    const int32_t nr = a.T > r ? (int32_t)((a.T - r + d - 1) / d) : 0;  // rows of residue r
+    const int32_t ja = (int32_t)((int64_t)nr * p / a.chunks);
+    const int32_t jb = (int32_t)((int64_t)nr * (p + 1) / a.chunks);
     const int gc = a.G / a.csize;                               // channels of this block
     const int64_t cb = (int64_t)m * a.G + (int64_t)q_cta * gc;  // first channel of this block
     const int64_t c0 = cb + (int64_t)tid * CH;                  // first channel of this thread
@@ -201,8 +205,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
                 *reinterpret_cast<float4 *>(part + (size_t)q * a.C) = make_float4(0, 0, 0, 0);
         return;
     }
-    const int64_t js = ja - L > 0 ? ja - L : 0;
-    const int64_t je = min64(nr, jb + L);
+    const int32_t js = ja - L > 0 ? ja - L : 0;
+    const int32_t je = min(nr, jb + L);
     const int nbatch = (int)((jb + L - js + B - 1) / B);
     const int S = a.slots;
     const uint32_t xbytes = (uint32_t)gc * sizeof(XT), gbytes = (uint32_t)gc * sizeof(GT);
@@ -216,9 +220,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
     // warp 0, lane i < B: rows j0 + i of every batch; each such lane keeps
     // the bounds [seq_lo, seq_hi) of the sequence holding its last row
     int32_t seq = 0;
-    int64_t seq_lo = 0, seq_hi = a.T;
+    int32_t seq_lo = 0, seq_hi = (int32_t)a.T;
     if (wid == 0 && lane < B && a.cu != nullptr) {
-        const int64_t t = r + min64(js + lane, nr - 1) * d;
+        const int32_t t = r + min(js + lane, nr - 1) * d;
         seq = find_sequence(a.cu, a.nseq, t);
         seq_lo = __ldg(a.cu + seq);
         seq_hi = __ldg(a.cu + seq + 1);
@@ -251,10 +255,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
     };
     sync_all();
 
-    // warp 0: rows of batch b into their slots (lane i: row j0 + i), and
-    // their in-sequence tap counts
-    auto issue = [&](int b) {
-        const int64_t j0 = js + (int64_t)b * B;
+    // warp 0: rows of batch b (first slot s0) into their slots (lane i: row
+    // j0 + i), and their in-sequence tap counts
+    const uint32_t xs_u = smem_u32(xs), gs_u = smem_u32(gs);
+    auto issue = [&](int b, int s0) {
+        const int32_t j0 = js + b * B;
         if (j0 >= je)
             return;
         uint64_t *bar = bars + b % kBwdBars;
@@ -270,28 +275,33 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
                          : "memory");
         }
         __syncwarp();
-        const int64_t j = j0 + lane;
+        const int32_t j = j0 + lane;
         if (lane < B && j < je) {
-            const int slot = (int)((j - js) % S);
-            const int64_t t = r + j * d;
-            bulk_load(xs + (size_t)slot * a.pitch_x, xb + t * xrow, xbytes, bar);
+            const int slot = s0 + lane >= S ? s0 + lane - S : s0 + lane;
+            const int32_t t = r + j * d;
+            bulk_load(xs + (size_t)slot * a.pitch_x, xb + (int64_t)t * xrow, xbytes, bar);
             if (j >= ja)
-                bulk_load(gs + (size_t)slot * a.pitch_g, gb + t * grow, gbytes, bar);
+                bulk_load(gs + (size_t)slot * a.pitch_g, gb + (int64_t)t * grow, gbytes, bar);
             if (a.cu != nullptr)
                 while (t >= seq_hi && seq + 1 < a.nseq) {
                     ++seq;
                     seq_lo = seq_hi;
                     seq_hi = __ldg(a.cu + seq + 1);
                 }
-            const int64_t back = (t - seq_lo) / d, fwd = (seq_hi - 1 - t) / d;
-            const int nb = back <= 0 ? 0 : back >= L ? L : (int)back;
-            const int nf = fwd <= 0 ? 0 : fwd >= L ? L : (int)fwd;
-            meta_s[slot] = nb | nf << 8;
+            meta_s[slot] = taps_within(t - seq_lo, d) | taps_within(seq_hi - 1 - t, d) << 8;
         }
     };
+    // first slot of batch b + n from that of batch b (n * B < S)
+    auto slot_ahead = [&](int s0, int n) {
+        const int v = s0 + n * B;
+        return v >= S ? v - S : v;
+    };
+    int s_issue = 0;  // first slot of the next batch to issue
     if (wid == 0)
-        for (int b = 0; b < a.ahead && b < nbatch; ++b)
-            issue(b);
+        for (int b = 0; b < a.ahead && b < nbatch; ++b) {
+            issue(b, s_issue);
+            s_issue = slot_ahead(s_issue, 1);
+        }
 
     // this thread's weights, norm scale and bias, in channel pairs
     float2 w[KT][NP], sc[NP], bias[NP];
@@ -325,23 +335,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
         dnw[pp] = zero2;
     }
 
-    const size_t xoff = (size_t)tid * CH * sizeof(XT), goff = (size_t)tid * CH * sizeof(GT);
+    const uint32_t xoff = (uint32_t)tid * CH * sizeof(XT), goff = (uint32_t)tid * CH * sizeof(GT);
+    const uint32_t xs_t = xs_u + xoff, gs_t = gs_u + goff;  // this thread's channels, slot 0
+    const uint32_t px = (uint32_t)a.pitch_x, pg = (uint32_t)a.pitch_g;
     char *dxb = static_cast<char *>(a.dx) + cb * sizeof(GT) + goff;
     bool timed_out = false;
 
     // x of ring row q (rows j0 - L .. j0 + B - 1) of the batch, normalised
     auto load_xh = [&](int slot, float iv, float2 *xh) {
         float f[CH];
-        load_slot4<XT>(xs + (size_t)slot * a.pitch_x + xoff, f);
+        load_slot4<XT>(xs_t + (uint32_t)slot * px, f);
         const float2 iv2 = make_float2(iv, iv);
 #pragma unroll
         for (int pp = 0; pp < NP; ++pp)
             xh[pp] = __fmul2_rn(make_float2(f[2 * pp], f[2 * pp + 1]), iv2);
     };
 
-    // slots of the ring rows j0 - L .. j0 + B - 1 of the batch starting at j0
-    auto window_slots = [&](int64_t j0, int (&slot)[RING]) {
-        slot[L] = (int)((j0 - js) % S);
+    // slots of the ring rows j0 - L .. j0 + B - 1 of the batch whose first
+    // row is in slot s0
+    auto window_slots = [&](int s0, int (&slot)[RING]) {
+        slot[L] = s0;
 #pragma unroll
         for (int q = L - 1; q >= 0; --q)
             slot[q] = slot[q + 1] == 0 ? S - 1 : slot[q + 1] - 1;
@@ -351,22 +364,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
     };
     constexpr int PB = B * kBwdPartStride;  // one buffer of partials
 
-    // ---- stage 1 of batch b: wait for its rows, post the squares of its rows
-    auto stage1 = [&](int b) {
-        const int64_t j0 = js + (int64_t)b * B;
+    // ---- stage 1 of batch b (first slot s0): wait for its rows, post the
+    // squares of its rows
+    auto stage1 = [&](int b, int s0) {
+        const int32_t j0 = js + b * B;
         if (j0 < je && !timed_out &&
             !mbar_wait(bars + b % kBwdBars, (uint32_t)(b / kBwdBars) & 1u))
             timed_out = true;
         if (!do_norm)
             return;
-        int sl = (int)((j0 - js) % S);
+        int sl = s0;
         float ss[B];
 #pragma unroll
         for (int i = 0; i < B; ++i, sl = sl + 1 == S ? 0 : sl + 1) {
             float2 acc = zero2;
             if (active && j0 + i < je) {
                 float f[CH];
-                load_slot4<XT>(xs + (size_t)sl * a.pitch_x + xoff, f);
+                load_slot4<XT>(xs_t + (uint32_t)sl * px, f);
 #pragma unroll
                 for (int pp = 0; pp < NP; ++pp) {
                     const float2 x2 = make_float2(f[2 * pp], f[2 * pp + 1]);
@@ -383,12 +397,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
     for (int q = 0; q < RING; ++q)
         inv[q] = 0.f;
 
-    // ---- stage 4 of batch b: dx of its lagged rows (ring rows 0 .. B - 1),
-    // once the dot partials it posted are complete
-    auto stage4 = [&](int b) {
-        const int64_t j0 = js + (int64_t)b * B;
+    // ---- stage 4 of batch b (first slot s0): dx of its lagged rows (ring
+    // rows 0 .. B - 1), once the dot partials it posted are complete
+    auto stage4 = [&](int b, int s0) {
+        const int32_t j0 = js + b * B;
         int slot[RING];
-        window_slots(j0, slot);
+        window_slots(s0, slot);
         int fwd[B];
         bool full_fwd = j0 - L >= ja && j0 - L + B <= jb;
 #pragma unroll
@@ -401,7 +415,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
             sum_parts4(dot_part + (b & 1) * PB, lane, means);
 #pragma unroll
         for (int i = 0; i < B; ++i) {
-            const int64_t jj = j0 - L + i;
+            const int32_t jj = j0 - L + i;
             if (!active || jj < ja || jj >= jb)
                 continue;
             const float mean = do_norm ? means[i] * a.inv_G : 0.f;
@@ -409,7 +423,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
             float2 xh[NP];
             load_xh(slot[i], inv[i], xh);
             if (do_res)
-                load_slot4<GT>(gs + (size_t)slot[i] * a.pitch_g + goff, g);
+                load_slot4<GT>(gs_t + (uint32_t)slot[i] * pg, g);
             const float2 ij2 = make_float2(inv[i], inv[i]), mean2 = make_float2(-mean, -mean);
 #pragma unroll
             for (int pp = 0; pp < NP; ++pp) {
@@ -429,8 +443,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
             constexpr int OW = CH * (int)sizeof(GT) / 4;
             uint32_t ow[OW];
             Elem<GT>::template pack<CH>(o, ow);
-            const int64_t t = r + jj * d;
-            store_words<OW * 4>(dxb + t * grow, ow);
+            const int32_t t = r + jj * d;
+            store_words<OW * 4>(dxb + (int64_t)t * grow, ow);
         }
     };
 
@@ -439,14 +453,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
     // posts the squares of batch b + 1 (stage 1); partials are double-buffered
     // by batch parity, so a warp that runs ahead never overwrites partials
     // another warp still reads.
-    stage1(0);
+    stage1(0, 0);
     sync_all();
-    if (wid == 0 && a.ahead < nbatch)
-        issue(a.ahead);
+    if (wid == 0 && a.ahead < nbatch) {
+        issue(a.ahead, s_issue);
+        s_issue = slot_ahead(s_issue, 1);
+    }
+    int s_cur = 0, s_prev = S - B;  // first slots of batches b and b - 1
     for (int b = 0; b < nbatch; ++b) {
-        const int64_t j0 = js + (int64_t)b * B;
+        const int32_t j0 = js + b * B;
         if (b > 0) {
-            stage4(b - 1);
+            stage4(b - 1, s_prev);
             // the ring moves on by one batch
 #pragma unroll
             for (int i = 0; i < L; ++i) {
@@ -457,7 +474,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
             }
         }
         int slot[RING];
-        window_slots(j0, slot);
+        window_slots(s_cur, slot);
 
         // ---- stage 2: inverse RMS, y and dy of the batch's rows
         {
@@ -486,7 +503,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
         if (active) {
 #pragma unroll
             for (int q = 0; q < RING; ++q) {
-                const int64_t jr = j0 - L + q;
+                const int32_t jr = j0 - L + q;
                 if (jr < js || jr >= je)
                     continue;  // not loaded (no batch row reads it: its tap is out of range)
                 float2 xh[NP];
@@ -506,11 +523,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
         }
 #pragma unroll
         for (int i = 0; i < B; ++i) {
-            const int64_t j = j0 + i;
+            const int32_t j = j0 + i;
             const bool need = active && j < je && j >= ja;
             float g[CH];
             if (need)
-                load_slot4<GT>(gs + (size_t)slot[L + i] * a.pitch_g + goff, g);
+                load_slot4<GT>(gs_t + (uint32_t)slot[L + i] * pg, g);
 #pragma unroll
             for (int pp = 0; pp < NP; ++pp) {
                 const float2 y = __ffma2_rn(sc[pp], acc[i][pp], bias[pp]);
@@ -544,7 +561,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
             float dotv[B];
 #pragma unroll
             for (int i = 0; i < B; ++i) {
-                const int64_t jj = j0 - L + i;
+                const int32_t jj = j0 - L + i;
                 float2 accd = zero2;
                 if (active && jj >= ja && jj < jb) {
                     float2 xh[NP];
@@ -569,14 +586,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
                 post(dot_part + (b & 1) * PB,
                      warp_sum4(dotv[0], dotv[1], dotv[2], dotv[3], lane));
         }
+        const int s_next = slot_ahead(s_cur, 1);
         if (b + 1 < nbatch)
-            stage1(b + 1);
+            stage1(b + 1, s_next);
         sync_all();
-        if (wid == 0 && b + 1 + a.ahead < nbatch)
-            issue(b + 1 + a.ahead);
+        if (wid == 0 && b + 1 + a.ahead < nbatch) {
+            issue(b + 1 + a.ahead, s_issue);
+            s_issue = slot_ahead(s_issue, 1);
+        }
+        s_prev = s_cur;
+        s_cur = s_next;
     }
     if (nbatch > 0)
-        stage4(nbatch - 1);
+        stage4(nbatch - 1, s_prev);
 
     // partials of this block: s * dw per tap, dbias, dnorm_w (zero without the norm)
     if (active) {

@@ -59,27 +59,30 @@ __host__ __device__ constexpr size_t cls_smem_bytes(int bufs, int pitch)
     return (size_t)kClsDataOffset + (size_t)bufs * kClsRows * pitch;
 }
 
-// N (4 or 8) consecutive elements of T at p (8, 16 or 32 bytes) as floats.
+// N (4 or 8) consecutive elements of T (8, 16 or 32 bytes) at the
+// shared-window address `addr`, as floats.
 template <typename T, int N>
-__device__ __forceinline__ void load_n(const unsigned char *p, float *f)
+__device__ __forceinline__ void load_n(uint32_t addr, float *f)
 {
     constexpr int W = N * (int)sizeof(T) / 4;
     uint32_t w[W];
     if constexpr (W == 2) {
-        const uint2 u = *reinterpret_cast<const uint2 *>(p);
-        w[0] = u.x;
-        w[1] = u.y;
+        asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(w[0]), "=r"(w[1]) : "r"(addr));
     } else {
 #pragma unroll
-        for (int q = 0; q < W / 4; ++q) {
-            const uint4 u = reinterpret_cast<const uint4 *>(p)[q];
-            w[4 * q] = u.x;
-            w[4 * q + 1] = u.y;
-            w[4 * q + 2] = u.z;
-            w[4 * q + 3] = u.w;
-        }
+        for (int q = 0; q < W / 4; ++q)
+            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(w[4 * q]), "=r"(w[4 * q + 1]), "=r"(w[4 * q + 2]),
+                           "=r"(w[4 * q + 3])
+                         : "r"(addr + 16u * q));
     }
     Elem<T>::template unpack<N>(w, f);
+}
+
+// Number of taps k in 1..3 with k * d <= span (span < 0 counts as 0).
+__device__ __forceinline__ int cls_taps_within(int32_t span, int32_t d)
+{
+    return (span >= d) + (span >= 2 * d) + (span >= 3 * d);
 }
 
 // ConvArgs fields used: x, out, cu, nseq, T, C, G, bpg (chunks per residue),
@@ -110,11 +113,13 @@ __global__ void __maxnreg__(CH == 4 ? 80 : 128)
     const int m = blockIdx.x / per_branch;
     const int rem = blockIdx.x - m * per_branch;
     const int r = rem / a.bpg, p = rem - r * a.bpg;
-    const int64_t nr = a.T > r ? (a.T - r + d - 1) / d : 0;  // rows of residue r
-    const int64_t ja = nr * p / a.bpg, jb = nr * (p + 1) / a.bpg;
+    // row indices fit 32 bits (T < 2^31)
+    const int32_t nr = a.T > r ? (int32_t)((a.T - r + d - 1) / d) : 0;  // rows of residue r
+    const int32_t ja = (int32_t)((int64_t)nr * p / a.bpg);
+    const int32_t jb = (int32_t)((int64_t)nr * (p + 1) / a.bpg);
     if (ja >= jb)
         return;
-    const int64_t js = ja - H > 0 ? ja - H : 0;
+    const int32_t js = ja - H > 0 ? ja - H : 0;
     const int nbatch = (int)((jb - js + B - 1) / B);
     const int NB = a.reg_bufs;
     const uint32_t row_bytes = (uint32_t)a.G * sizeof(XT);
@@ -141,8 +146,8 @@ __global__ void __maxnreg__(CH == 4 ? 80 : 128)
         const bool do_norm = a.flags & ENGRAM_CONV_NORM;
         // lane i of stat warp 0 loads row i of batch c into buffer c % NB
         auto load_batch = [&](int c) {
-            const int64_t j0 = js + (int64_t)c * B;
-            const int rc = (int)min64(B, jb - j0);
+            const int32_t j0 = js + c * B;
+            const int rc = min(B, jb - j0);
             const int b = c % NB;
             if (lane == 0)
                 asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(
@@ -152,13 +157,13 @@ __global__ void __maxnreg__(CH == 4 ? 80 : 128)
             __syncwarp();
             if (lane < rc)
                 bulk_load(data + (size_t)(b * B + lane) * pitch,
-                          xbranch + (r + (j0 + lane) * d) * xrow, row_bytes, tma_bar + b);
+                          xbranch + (int64_t)(r + (j0 + lane) * d) * xrow, row_bytes, tma_bar + b);
         };
         // the sequence holding this lane's row, tracked from row to row
         int32_t seq = 0;
-        int64_t seq_lo = 0, seq_hi = a.T;
+        int32_t seq_lo = 0, seq_hi = (int32_t)a.T;
         if (sw == 1 && lane < B && a.cu != nullptr) {
-            seq = find_sequence(a.cu, a.nseq, r + min64(js + lane, nr - 1) * d);
+            seq = find_sequence(a.cu, a.nseq, r + min(js + lane, nr - 1) * d);
             seq_lo = __ldg(a.cu + seq);
             seq_hi = __ldg(a.cu + seq + 1);
         }
@@ -167,11 +172,11 @@ __global__ void __maxnreg__(CH == 4 ? 80 : 128)
                 load_batch(c);
         for (int c = 0; c < nbatch; ++c) {
             const int b = c % NB;
-            const int64_t j0 = js + (int64_t)c * B;
-            const int rc = (int)min64(B, jb - j0);
+            const int32_t j0 = js + c * B;
+            const int rc = min(B, jb - j0);
             if (!mbar_wait(tma_bar + b, (uint32_t)(c / NB) & 1u))
                 timed_out = true;
-            const unsigned char *buf = data + (size_t)b * B * pitch;
+            const uint32_t buf = smem_u32(data) + (uint32_t)(b * B) * pitch;
             for (int i = sw; i < rc; i += kClsStatWarps) {
                 float2 ss[EV / 2];
 #pragma unroll
@@ -179,9 +184,10 @@ __global__ void __maxnreg__(CH == 4 ? 80 : 128)
                     ss[e] = make_float2(0.f, 0.f);
 #pragma unroll 5
                 for (int v = lane; v < nvec; v += 32) {
-                    const uint4 q = *reinterpret_cast<const uint4 *>(buf + (size_t)i * pitch +
-                                                                     (size_t)v * 16);
-                    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+                    uint32_t w[4];
+                    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                                 : "r"(buf + (uint32_t)i * pitch + (uint32_t)v * 16u));
                     float f[EV];
                     Elem<XT>::template unpack<EV>(w, f);
 #pragma unroll
@@ -202,17 +208,16 @@ __global__ void __maxnreg__(CH == 4 ? 80 : 128)
             }
             if (sw == 1) {
                 int nv = 0;
-                const int64_t j = j0 + lane;
+                const int32_t j = j0 + lane;
                 if (lane < rc) {
-                    const int64_t t = r + j * d;
+                    const int32_t t = r + j * d;
                     if (a.cu != nullptr)
                         while (t >= seq_hi && seq + 1 < a.nseq) {
                             ++seq;
                             seq_lo = seq_hi;
                             seq_hi = __ldg(a.cu + seq + 1);
                         }
-                    const int64_t back = (t - seq_lo) / d;
-                    nv = back >= H ? H : back <= 0 ? 0 : (int)back;
+                    nv = cls_taps_within(t - seq_lo, d);
                     nv_s[b * B + lane] = nv;
                 }
                 const bool row_full = lane >= B || (lane < rc && j >= ja && nv == H);
@@ -268,14 +273,15 @@ __global__ void __maxnreg__(CH == 4 ? 80 : 128)
             hist[h][pp] = zero2;
 
     char *out = static_cast<char *>(a.out) + ((int64_t)m * a.G + (int64_t)tid * CH) * sizeof(OT);
-    const size_t xoff = (size_t)tid * CH * sizeof(XT);
+    const uint32_t xoff = (uint32_t)tid * CH * sizeof(XT);
+    const int64_t orow = (int64_t)a.C * sizeof(OT);
     for (int c = 0; c < nbatch; ++c) {
         const int b = c % NB;
-        const int64_t j0 = js + (int64_t)c * B;
-        const int rc = (int)min64(B, jb - j0);
+        const int32_t j0 = js + c * B;
+        const int rc = min(B, jb - j0);
         if (!timed_out && !mbar_wait(full_bar + b, (uint32_t)(c / NB) & 1u))
             timed_out = true;
-        const unsigned char *buf = data + (size_t)b * B * pitch + xoff;
+        const uint32_t buf = smem_u32(data) + (uint32_t)(b * B) * pitch + xoff;
         auto run = [&](auto fast_tag) {
             constexpr bool FAST = decltype(fast_tag)::value;
 #pragma unroll
@@ -284,7 +290,7 @@ __global__ void __maxnreg__(CH == 4 ? 80 : 128)
                     break;
                 float xv[CH];
                 if (active)
-                    load_n<XT, CH>(buf + (size_t)i * pitch, xv);
+                    load_n<XT, CH>(buf + (uint32_t)i * pitch, xv);
                 else
 #pragma unroll
                     for (int e = 0; e < CH; ++e)
@@ -325,7 +331,7 @@ __global__ void __maxnreg__(CH == 4 ? 80 : 128)
                     for (int pp = 0; pp < NP; ++pp)
                         y[pp] = __fadd2_rn(y[pp], make_float2(xv[2 * pp], xv[2 * pp + 1]));
                 }
-                const int64_t j = j0 + i;
+                const int32_t j = j0 + i;
                 if (active && (FAST || j >= ja)) {
                     float o[CH];
 #pragma unroll
@@ -336,7 +342,7 @@ __global__ void __maxnreg__(CH == 4 ? 80 : 128)
                     constexpr int OW = CH * (int)sizeof(OT) / 4;
                     uint32_t w[OW];
                     Elem<OT>::template pack<CH>(o, w);
-                    store_words<OW * 4>(out + (r + j * d) * (int64_t)a.C * sizeof(OT), w);
+                    store_words<OW * 4>(out + (int64_t)(r + j * d) * orow, w);
                 }
             }
         };
