@@ -413,39 +413,48 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
         float means[B];
         if (do_norm)
             sum_parts4(dot_part + (b & 1) * PB, lane, means);
+        // FAST: every lagged row has its output and all its taps in-sequence
+        auto rows = [&](auto fast_tag) {
+            constexpr bool FAST = decltype(fast_tag)::value;
 #pragma unroll
-        for (int i = 0; i < B; ++i) {
-            const int32_t jj = j0 - L + i;
-            if (!active || jj < ja || jj >= jb)
-                continue;
-            const float mean = do_norm ? means[i] * a.inv_G : 0.f;
-            float g[CH], o[CH];
-            float2 xh[NP];
-            load_xh(slot[i], inv[i], xh);
-            if (do_res)
-                load_slot4<GT>(gs_t + (uint32_t)slot[i] * pg, g);
-            const float2 ij2 = make_float2(inv[i], inv[i]), mean2 = make_float2(-mean, -mean);
-#pragma unroll
-            for (int pp = 0; pp < NP; ++pp) {
-                float2 dn = zero2;
-#pragma unroll
-                for (int k = 0; k < KT; ++k)
-                    dn = __ffma2_rn(w[k][pp], full_fwd || k <= fwd[i] ? dy[i + k][pp] : zero2,
-                                    dn);
-                float2 v = do_norm ? __fmul2_rn(ij2, __ffma2_rn(xh[pp], mean2,
-                                                                __fmul2_rn(sc[pp], dn)))
-                                   : dn;
+            for (int i = 0; i < B; ++i) {
+                const int32_t jj = j0 - L + i;
+                if (!FAST && (!active || jj < ja || jj >= jb))
+                    continue;
+                const float mean = do_norm ? means[i] * a.inv_G : 0.f;
+                float g[CH], o[CH];
+                float2 xh[NP];
+                load_xh(slot[i], inv[i], xh);
                 if (do_res)
-                    v = __fadd2_rn(v, make_float2(g[2 * pp], g[2 * pp + 1]));
-                o[2 * pp] = v.x;
-                o[2 * pp + 1] = v.y;
+                    load_slot4<GT>(gs_t + (uint32_t)slot[i] * pg, g);
+                const float2 ij2 = make_float2(inv[i], inv[i]);
+                const float2 mean2 = make_float2(-mean, -mean);
+#pragma unroll
+                for (int pp = 0; pp < NP; ++pp) {
+                    float2 dn = zero2;
+#pragma unroll
+                    for (int k = 0; k < KT; ++k)
+                        if (FAST || k <= fwd[i])
+                            dn = __ffma2_rn(w[k][pp], dy[i + k][pp], dn);
+                    float2 v = do_norm ? __fmul2_rn(ij2, __ffma2_rn(xh[pp], mean2,
+                                                                    __fmul2_rn(sc[pp], dn)))
+                                       : dn;
+                    if (do_res)
+                        v = __fadd2_rn(v, make_float2(g[2 * pp], g[2 * pp + 1]));
+                    o[2 * pp] = v.x;
+                    o[2 * pp + 1] = v.y;
+                }
+                constexpr int OW = CH * (int)sizeof(GT) / 4;
+                uint32_t ow[OW];
+                Elem<GT>::template pack<CH>(o, ow);
+                const int32_t t = r + jj * d;
+                store_words<OW * 4>(dxb + (int64_t)t * grow, ow);
             }
-            constexpr int OW = CH * (int)sizeof(GT) / 4;
-            uint32_t ow[OW];
-            Elem<GT>::template pack<CH>(o, ow);
-            const int32_t t = r + jj * d;
-            store_words<OW * 4>(dxb + (int64_t)t * grow, ow);
-        }
+        };
+        if (full_fwd && active)
+            rows(std::true_type{});
+        else
+            rows(std::false_type{});
     };
 
     // The batches are pipelined so that one barrier separates them: iteration
@@ -500,11 +509,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
 #pragma unroll
             for (int pp = 0; pp < NP; ++pp)
                 acc[i][pp] = zero2;
-        if (active) {
+        // FAST: every row of the batch has its output and all its taps
+        auto taps = [&](auto fast_tag) {
+            constexpr bool FAST = decltype(fast_tag)::value;
 #pragma unroll
             for (int q = 0; q < RING; ++q) {
                 const int32_t jr = j0 - L + q;
-                if (jr < js || jr >= je)
+                if (!FAST && (jr < js || jr >= je))
                     continue;  // not loaded (no batch row reads it: its tap is out of range)
                 float2 xh[NP];
                 load_xh(slot[q], inv[q], xh);
@@ -513,13 +524,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
                     const int k = L + i - q;
                     if (k < 0 || k >= KT)
                         continue;
-                    if (full_back || k <= back[i]) {
+                    if (FAST || k <= back[i]) {
 #pragma unroll
                         for (int pp = 0; pp < NP; ++pp)
                             acc[i][pp] = __ffma2_rn(w[k][pp], xh[pp], acc[i][pp]);
                     }
                 }
             }
+        };
+        if (active) {
+            if (full_back)
+                taps(std::true_type{});
+            else
+                taps(std::false_type{});
         }
 #pragma unroll
         for (int i = 0; i < B; ++i) {
@@ -559,29 +576,37 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
         }
         {
             float dotv[B];
+            // FAST: every lagged row has its output and all its taps in-sequence
+            auto rows = [&](auto fast_tag) {
+                constexpr bool FAST = decltype(fast_tag)::value;
 #pragma unroll
-            for (int i = 0; i < B; ++i) {
-                const int32_t jj = j0 - L + i;
-                float2 accd = zero2;
-                if (active && jj >= ja && jj < jb) {
-                    float2 xh[NP];
-                    load_xh(slot[i], inv[i], xh);
+                for (int i = 0; i < B; ++i) {
+                    const int32_t jj = j0 - L + i;
+                    float2 accd = zero2;
+                    if (FAST || (active && jj >= ja && jj < jb)) {
+                        float2 xh[NP];
+                        load_xh(slot[i], inv[i], xh);
 #pragma unroll
-                    for (int pp = 0; pp < NP; ++pp) {
-                        float2 dn = zero2;
+                        for (int pp = 0; pp < NP; ++pp) {
+                            float2 dn = zero2;
 #pragma unroll
-                        for (int k = 0; k < KT; ++k) {
-                            const float2 g = full_fwd || k <= fwd[i] ? dy[i + k][pp] : zero2;
-                            dn = __ffma2_rn(w[k][pp], g, dn);
-                            dw[k][pp] = __ffma2_rn(xh[pp], g, dw[k][pp]);
+                            for (int k = 0; k < KT; ++k)
+                                if (FAST || k <= fwd[i]) {
+                                    dn = __ffma2_rn(w[k][pp], dy[i + k][pp], dn);
+                                    dw[k][pp] = __ffma2_rn(xh[pp], dy[i + k][pp], dw[k][pp]);
+                                }
+                            db[pp] = __fadd2_rn(db[pp], dy[i][pp]);
+                            dnw[pp] = __ffma2_rn(dn, xh[pp], dnw[pp]);
+                            accd = __ffma2_rn(__fmul2_rn(sc[pp], dn), xh[pp], accd);
                         }
-                        db[pp] = __fadd2_rn(db[pp], dy[i][pp]);
-                        dnw[pp] = __ffma2_rn(dn, xh[pp], dnw[pp]);
-                        accd = __ffma2_rn(__fmul2_rn(sc[pp], dn), xh[pp], accd);
                     }
+                    dotv[i] = accd.x + accd.y;
                 }
-                dotv[i] = accd.x + accd.y;
-            }
+            };
+            if (full_fwd && active)
+                rows(std::true_type{});
+            else
+                rows(std::false_type{});
             if (do_norm)
                 post(dot_part + (b & 1) * PB,
                      warp_sum4(dotv[0], dotv[1], dotv[2], dotv[3], lane));
