@@ -683,7 +683,16 @@ int conv_plan(const engram_conv_params_t *p, int32_t dtype, int32_t out_dtype, i
     const int chan = G / 4 <= ple::kNarrowThreads ? 4 : 8;  // channels per thread
     const int nth = G / chan;
     const int norm_slots = halo + ple::kRows;
-    if (ple::smem_bytes(norm_slots, nth, chan) > ple::kSmemLimit)
+    // kernel widths up to 4 on branches up to 2,560 channels (4 per thread):
+    // one residue class per block, batches of 8 rows in shared memory, any
+    // dilation; otherwise the chunked kernel, whose private history rings
+    // must fit shared memory
+    const int pitch_reg = (G * eb + 127) / 128 * 128;  // bytes per buffered row
+    const int cls_bufs = (int)std::min<size_t>(
+        ple::kClsMaxBufs,
+        (ple::kSmemLimit - ple::kClsDataOffset) / ((size_t)ple::kClsRows * pitch_reg));
+    P->cls = K <= ple::kClsTaps && G / 4 <= 32 * ple::kClsMaxConvWarps && cls_bufs >= 2;
+    if (!P->cls && ple::smem_bytes(norm_slots, nth, chan) > ple::kSmemLimit)
         return ENGRAM_EINVAL;
     ple::ConvArgs &a = P->a;
     std::memset(&a, 0, sizeof(a));
@@ -702,13 +711,6 @@ int conv_plan(const engram_conv_params_t *p, int32_t dtype, int32_t out_dtype, i
     P->chan = chan;
     P->threads = (nth + 31) / 32 * 32;
     P->smem = ple::smem_bytes(norm_slots, nth, chan);
-    const int pitch_reg = (G * eb + 127) / 128 * 128;  // bytes per buffered row
-    // kernel widths up to 4 on branches up to 2,560 channels (4 per thread):
-    // one residue class per block, batches of 8 rows in shared memory
-    const int cls_bufs = (int)std::min<size_t>(
-        ple::kClsMaxBufs,
-        (ple::kSmemLimit - ple::kClsDataOffset) / ((size_t)ple::kClsRows * pitch_reg));
-    P->cls = K <= ple::kClsTaps && G / 4 <= 32 * ple::kClsMaxConvWarps && cls_bufs >= 2;
     if (P->cls) {
         P->chan = 4;
         a.nth = G / P->chan;

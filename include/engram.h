@@ -289,9 +289,9 @@ typedef struct engram_conv_params {
  *   conv_bias   device, [C] of weight_dtype, or NULL
  *   out         device, [T, C] of out_dtype (dtype or ENGRAM_F32), 16-byte
  *               aligned, not overlapping x
- * Limits (else ENGRAM_EINVAL): those of engram_conv_params_t and
- * 4 * G * ((K - 1) * d + 4) + 1152 <= 227 KB of shared memory per block (the
- * page's shape, G = 2560, K = 4, d = 3: 134 KB).
+ * Limits (else ENGRAM_EINVAL): those of engram_conv_params_t; and unless
+ * K <= 4 and G <= 2560 (the page's shape: any dilation), also
+ * 4 * G * ((K - 1) * d + 4) + 1152 <= 227 KB of shared memory per block.
  */
 ENGRAM_API int engram_ple_short_conv(const engram_conv_params_t *params, const void *x,
                                      int32_t dtype, const int32_t *cu_seqlens, int32_t nseq,

@@ -111,7 +111,7 @@ def test_flag_combinations(E, flags):
 
 
 @pytest.mark.parametrize("K,d", [(1, 1), (2, 1), (3, 5), (4, 1), (4, 3), (5, 7), (8, 2),
-                                 (8, 9)])
+                                 (8, 9), (4, 257)])
 def test_kernel_widths_and_dilations(E, K, d):
     T, C, G = 611, 256, 64
     x, nw, w, b = small_inputs("bf16", "f32", T, C, K, 30 + K + d)
@@ -132,8 +132,8 @@ def test_weight_dtypes(E, wdt):
 
 @pytest.mark.parametrize("G", [8, 16, 24, 3376])
 def test_narrow_and_widest_branches(E, G):
-    # G = 8: one active thread per block; G = 24: a partial warp; G = 3376: the
-    # widest bf16 branch whose kernel-4, dilation-3 history fits shared memory
+    # G = 8: one active thread per block; G = 24: a partial warp; G = 3376: a
+    # branch wider than 2,560 (the chunked kernel, 8 channels per thread)
     C = 2 * G if G < 1000 else G
     T = 97 if G < 1000 else 61
     x, nw, w, b = small_inputs("bf16", "f32", T, C, 4, 50 + G)
