@@ -1009,6 +1009,7 @@ int conv_bwd_grid(ConvBwdPlan *P)
     if (grid > INT32_MAX)
         return ENGRAM_EINVAL;
     a.chunks = (int32_t)chunks;
+    a.classes = classes;
     P->grid = (int)grid;
     P->npart = (int)(classes * chunks);
     P->ws = (size_t)P->npart * ple::kBwdQuantities * (size_t)a.C * sizeof(float);

@@ -92,6 +92,7 @@ struct ConvBwdArgs {
     int64_t T;
     int32_t C, G, nth;      // nth = G / 8 active threads
     int32_t dil, K, chunks; // chunks: blocks per (branch, residue)
+    int32_t classes;        // residues holding rows, min(dil, T): the grid's residue extent
     const void *norm_w, *conv_w, *bias;
     int32_t wdtype;
     float eps, inv_G;
@@ -184,7 +185,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
     const bool pair = a.csize == 2;
     const uint32_t q_cta = pair ? cluster_rank() : 0u;  // half of the branch slice
     const int unit = blockIdx.x / a.csize;
-    const int per_branch = d * a.chunks;
+    const int per_branch = a.classes * a.chunks;
     const int m = unit / per_branch;
     const int rem = unit - m * per_branch;
     const int r = rem / a.chunks, p = rem - r * a.chunks;

@@ -263,3 +263,13 @@ def test_page_shape_benchmark_size_sampled(E):
                            dilation=s.dilation)[-1]
         got = out[t].float().cpu().numpy().astype(np.float64)
         assert_close(got, want, "bf16", f"token {t}")
+
+
+@pytest.mark.parametrize("T,d", [(1, 3), (5, 9), (8, 4)])
+def test_fewer_tokens_than_residues(E, T, d):
+    # some residues of the dilation hold no token at all
+    C, G = 128, 64
+    x, nw, w, b = small_inputs("bf16", "f32", T, C, 4, 400 + T + d)
+    got = run_conv(E, x, w, nw, b, None, dt="bf16", wdt="f32", out_dt="f32", group=G, dilation=d)
+    want = oracle_conv(x, w, nw, b, None, dt="bf16", wdt="f32", group=G, dilation=d)
+    assert_close(got, want, "f32", f"T={T} d={d}")

@@ -320,3 +320,42 @@ def test_page_shape_benchmark_size_sampled(E):
     assert_wgrad(host(db)[chans], dbn, "dbias")
     # dn is the no-norm run's input gradient; dnorm_w = sum dn * xh = sum dn * n / (1 + w)
     assert_wgrad(host(dnw)[chans], (dxn * n).sum(0) / scale, "dnorm_w")
+
+
+@pytest.mark.parametrize("T,d", [(1, 3), (5, 9), (8, 4)])
+def test_fewer_tokens_than_residues(E, T, d):
+    # some residues of the dilation hold no token at all
+    C, G = 128, 64
+    x, nw, w, b, dout = inputs("bf16", "f32", "f32", T, C, 4, 300 + T + d)
+    got, want = run_both(E, x, w, nw, b, dout, None, dt="bf16", gdt="f32", wdt="f32", group=G,
+                         dilation=d)
+    check(got, want, "f32", f"T={T} d={d}")
+
+
+def test_replays_in_a_graph(E):
+    T, C, G = 4096, 5120, 2560
+    x, nw, w, b, dout = inputs("bf16", "bf16", "bf16", T, C, 4, 310)
+    xt, wt, gt = dev(x, "bf16"), dev(w, "bf16"), dev(dout, "bf16")
+    kw = dict(dilation=3, group_size=G, norm_weight=dev(nw, "bf16"), conv_bias=dev(b, "bf16"),
+              cu_seqlens=torch.tensor([0, 1000, 4096], dtype=torch.int32, device="cuda"))
+    ws = torch.empty(E.engram_ple_short_conv_backward_workspace_size(C, G, 4, 3, T),
+                     dtype=torch.uint8, device="cuda")
+    outs = [(torch.empty_like(gt), torch.empty(C, device="cuda"),
+             torch.empty((C, 4), device="cuda"), torch.empty(C, device="cuda")) for _ in range(2)]
+
+    def call(o):
+        E.engram_ple_short_conv_backward(xt, wt, gt, dx=o[0], dnorm_weight=o[1],
+                                         dconv_weight=o[2], dconv_bias=o[3], workspace=ws, **kw)
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        call(outs[0])
+    torch.cuda.current_stream().wait_stream(s)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        call(outs[1])
+    graph.replay()
+    torch.cuda.synchronize()
+    for a_, b_ in zip(outs[0], outs[1]):
+        assert torch.equal(a_, b_)
