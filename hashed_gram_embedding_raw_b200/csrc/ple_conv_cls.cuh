@@ -42,7 +42,6 @@ constexpr int kClsHist = kClsTaps - 1;
 constexpr int kClsRows = 8;                // rows per batch
 constexpr int kClsStatWarps = 4;
 constexpr int kClsMaxConvWarps = 20;       // 4 channels per thread: G <= 2560
-constexpr int kClsThreads = 32 * (kClsMaxConvWarps + kClsStatWarps);
 constexpr int kClsMaxBufs = 6;
 
 // Shared memory: inverse RMS [6][8] float, tap counts [6][8] int32, fast
