@@ -124,23 +124,26 @@ def test_emulated_group_tiny_vs_oracle(E, W):
     assert E.engram_get_device_error() == 0
 
 
-@pytest.mark.parametrize("W", [2, 8])
-def test_emulated_group_b4x4096_vs_unsharded(E, W):
-    cfg = head_params("b4x4096")
+@pytest.mark.parametrize("name,W", [("b4x4096", 2), ("b4x4096", 8), ("thd64k", 8)])
+def test_emulated_group_vs_unsharded(E, name, W):
+    # thd64k: Zipf IDs, so hot rows load some owners far more than others
+    cfg = head_params(name)
     params = E.make_params(cfg)
     R, D, H = cfg["table_rows"], cfg["dim"], params.heads
     table = torch.empty((R, D), dtype=torch.bfloat16, device="cuda")
     fill_device_table(table, 1)
-    ids, _ = token_stream("b4x4096")
+    ids, _ = token_stream(name)
     parts = split(ids, W)
-    douts = [host_dout("b4x4096", len(p[0]) * H, D, "bf16", seed_offset=r).cuda()
+    douts = [host_dout(name, len(p[0]) * H, D, "bf16", seed_offset=r).cuda()
              for r, p in enumerate(parts)]
     fwd, bwd = run_group(E, params, table, W, parts, douts)
     idx_all = []
+    counts = []
     for r, (ids_r, cu_r) in enumerate(parts):
         out, idx = E.engram_hash_gather(params, ids_r, table, cu_seqlens=cu_r)
         assert torch.equal(fwd[r][0], out)
         idx_all.append(idx.view(-1))
+        counts.append(fwd[r][1].send_counts)
     idx = torch.cat(idx_all)
     dout = torch.cat(douts)
     u, g, nu = E.engram_backward(idx, dout, R)
@@ -156,6 +159,10 @@ def test_emulated_group_b4x4096_vs_unsharded(E, W):
         assert torch.equal(gu[:Ur].long(), u[keep] - r * rpo)
         torch.testing.assert_close(gg[:Ur], g[keep], rtol=1e-6, atol=1e-6)
     assert E.engram_get_device_error() == 0
+    per_owner = np.asarray(counts).sum(0)
+    assert per_owner.sum() == idx.numel()
+    if name == "thd64k":
+        assert per_owner.max() > 1.5 * per_owner.min()   # the splits really are uneven
 
 
 def test_nccl_group_of_one(E):
