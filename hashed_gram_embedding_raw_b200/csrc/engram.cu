@@ -189,10 +189,48 @@ int launch_hash_gather(const HashArgs &a, const int32_t *ids, const int32_t *cu,
 // --------------------------------------------------------------- backward
 
 struct BwdPlan {
-    int passes = 0, ntiles = 0, ngroups = 0, wmax = 0, GF = 0;
+    int passes = 0, items = 0, ntiles = 0, ngroups = 0, wmax = 0, GF = 0;
     size_t a = 0, b = 0, tile_cnt = 0, ctl = 0, ctl_bytes = 0, group_cnt = 0, barrier = 0;
     size_t wcount = 0, bcount = 0, pb = 0, pe = 0, meta = 0, total = 0;
 };
+
+template <int I> int sort_resident_blocks(int64_t *blocks)
+{
+    int64_t warps = 0;
+    ENGRAM_TRY(resident_warps(bwd::radix_sort_coop<I>, bwd::kSortThreads, 0, &warps));
+    *blocks = warps / (bwd::kSortThreads / 32);
+    return ENGRAM_OK;
+}
+
+// Pairs per thread of the sort's tiles (4..8). Among the sizes that keep every
+// tile resident at once (the one-launch sort then holds a block's items in
+// registers across the grid barrier), take the one whose busiest SM holds the
+// fewest pairs -- 512 tiles of 2048 on 148 SMs leave 68 SMs with four tiles
+// and 80 with three; 586 tiles of 1792 give nearly all of them four smaller
+// ones. With none resident, the largest tiles.
+int sort_items(int64_t n, int sms, int *items)
+{
+    int64_t res[bwd::kSortItemsMax + 1] = {};
+    ENGRAM_TRY(sort_resident_blocks<4>(&res[4]));
+    ENGRAM_TRY(sort_resident_blocks<5>(&res[5]));
+    ENGRAM_TRY(sort_resident_blocks<6>(&res[6]));
+    ENGRAM_TRY(sort_resident_blocks<7>(&res[7]));
+    ENGRAM_TRY(sort_resident_blocks<8>(&res[8]));
+    int best = bwd::kSortItemsMax;
+    int64_t best_load = INT64_MAX;
+    for (int I = bwd::kSortItemsMax; I >= 4; --I) {
+        const int64_t tiles = std::max<int64_t>(1, ceil_div(n, (int64_t)bwd::kSortThreads * I));
+        if (tiles > res[I])
+            continue;
+        const int64_t load = ceil_div(tiles, (int64_t)sms) * I;
+        if (load < best_load) {
+            best = I;
+            best_load = load;
+        }
+    }
+    *items = best;
+    return ENGRAM_OK;
+}
 
 int bwd_plan(int64_t n, int64_t rows, int32_t dim, BwdPlan *P)
 {
@@ -203,9 +241,10 @@ int bwd_plan(int64_t n, int64_t rows, int32_t dim, BwdPlan *P)
     while ((int64_t(1) << bits) < rows)
         ++bits;
     P->passes = std::max(1, (bits + bwd::kRadixBits - 1) / bwd::kRadixBits);
-    P->ntiles = (int)std::max<int64_t>(1, ceil_div(n, bwd::kSortTile));
     int sms = 0;
     ENGRAM_TRY(device_sms(&sms));
+    ENGRAM_TRY(sort_items(n, sms, &P->items));
+    P->ntiles = (int)std::max<int64_t>(1, ceil_div(n, (int64_t)bwd::kSortThreads * P->items));
     P->wmax = sms * 32; // upper bound on resident warps of seg_reduce
     P->GF = (dim / 4 + 31) / 32;
     size_t off = 0;
@@ -223,7 +262,7 @@ int bwd_plan(int64_t n, int64_t rows, int32_t dim, BwdPlan *P)
     P->tile_cnt = take((size_t)bwd::kRadix * P->ntiles * 4);
     P->ctl = off;
     P->group_cnt = take((size_t)P->passes * bwd::kRadix * P->ngroups * 4);
-    P->barrier = take(2 * sizeof(unsigned)); // grid barrier of the one-launch sort
+    P->barrier = take(sizeof(unsigned)); // grid-barrier counter of the one-launch sort
     P->ctl_bytes = off - P->ctl;
     P->wcount = take((size_t)P->wmax * 4);
     P->bcount = take((size_t)ceil_div(P->wmax, bwd::kSegWarps) * 4);
@@ -243,8 +282,9 @@ int check_workspace(const BwdPlan &P, void *ws, size_t ws_bytes)
     return ENGRAM_OK;
 }
 
-int launch_sort(const int32_t *idx, int64_t n, int64_t rows, const BwdPlan &P, char *ws,
-                cudaStream_t stream)
+template <int I>
+int launch_sort_t(const int32_t *idx, int64_t n, int64_t rows, const BwdPlan &P, char *ws,
+                  cudaStream_t stream)
 {
     using namespace bwd;
     auto *A = (unsigned long long *)(ws + P.a);
@@ -261,12 +301,12 @@ int launch_sort(const int32_t *idx, int64_t n, int64_t rows, const BwdPlan &P, c
         cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) == cudaSuccess &&
         coop) {
         int64_t res = 0;
-        ENGRAM_TRY(resident_warps(radix_sort_coop, kSortThreads, 0, &res));
+        ENGRAM_TRY(resident_warps(radix_sort_coop<I>, kSortThreads, 0, &res));
         const int grid = (int)std::min<int64_t>(P.ntiles, res / (kSortThreads / 32));
         SortArgs args{idx, A, B, n, (uint32_t)rows, P.passes, P.ntiles, P.ngroups,
                       tile_cnt, group_cnt, (unsigned *)(ws + P.barrier)};
         void *params[] = {&args};
-        if (cudaLaunchCooperativeKernel((const void *)radix_sort_coop, dim3(grid),
+        if (cudaLaunchCooperativeKernel((const void *)radix_sort_coop<I>, dim3(grid),
                                         dim3(kSortThreads), params, 0, stream) == cudaSuccess) {
             g_launches.fetch_add(1, std::memory_order_relaxed);
             return ENGRAM_OK;
@@ -280,22 +320,35 @@ int launch_sort(const int32_t *idx, int64_t n, int64_t rows, const BwdPlan &P, c
         uint32_t *gc = group_cnt + (size_t)pass * kRadix * P.ngroups;
         const int shift = pass * kRadixBits;
         if (pass == 0) {
-            radix_count<true><<<P.ntiles, kSortThreads, 0, stream>>>(src, n, shift,
+            radix_count<true, I><<<P.ntiles, kSortThreads, 0, stream>>>(src, n, shift,
                                                                     (uint32_t)rows, tile_cnt, gc);
             ENGRAM_TRY(after_launch());
-            radix_scatter<true><<<P.ntiles, kSortThreads, 0, stream>>>(src, dst, n, shift,
+            radix_scatter<true, I><<<P.ntiles, kSortThreads, 0, stream>>>(src, dst, n, shift,
                                                                       tile_cnt, gc, P.ngroups);
         } else {
-            radix_count<false><<<P.ntiles, kSortThreads, 0, stream>>>(src, n, shift,
+            radix_count<false, I><<<P.ntiles, kSortThreads, 0, stream>>>(src, n, shift,
                                                                      (uint32_t)rows, tile_cnt, gc);
             ENGRAM_TRY(after_launch());
-            radix_scatter<false><<<P.ntiles, kSortThreads, 0, stream>>>(src, dst, n, shift,
+            radix_scatter<false, I><<<P.ntiles, kSortThreads, 0, stream>>>(src, dst, n, shift,
                                                                        tile_cnt, gc, P.ngroups);
         }
         ENGRAM_TRY(after_launch());
         src = dst;
     }
     return ENGRAM_OK;
+}
+
+int launch_sort(const int32_t *idx, int64_t n, int64_t rows, const BwdPlan &P, char *ws,
+                cudaStream_t stream)
+{
+    switch (P.items) {
+    case 4: return launch_sort_t<4>(idx, n, rows, P, ws, stream);
+    case 5: return launch_sort_t<5>(idx, n, rows, P, ws, stream);
+    case 6: return launch_sort_t<6>(idx, n, rows, P, ws, stream);
+    case 7: return launch_sort_t<7>(idx, n, rows, P, ws, stream);
+    case 8: return launch_sort_t<8>(idx, n, rows, P, ws, stream);
+    default: return ENGRAM_EINVAL;
+    }
 }
 
 template <int DT, int GF, int RVT>

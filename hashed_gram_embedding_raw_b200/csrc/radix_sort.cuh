@@ -5,7 +5,9 @@
 // items start in j order and every pass is stable, equal keys end up in
 // ascending j.
 //
-// Each pass has two phases over 2048-item tiles:
+// Each pass has two phases over tiles of 256 * ITEMS items (ITEMS <= 8 pairs
+// per thread, chosen per sort by the host so that the busiest SM holds as few
+// pairs as possible):
 //   count    a tile's digit counts are stored (tile-major, tile_cnt[tile][d])
 //            and added into per-group sums (group_cnt[group][d], 32 tiles per
 //            group; the adds commute, so the sums are deterministic);
@@ -22,8 +24,8 @@
 //
 // radix_sort_coop runs every phase of every pass in one cooperative launch:
 // each resident block takes tiles blockIdx.x, blockIdx.x + gridDim.x, ... and
-// the phases are separated by a grid barrier (bounded wait; a timeout raises
-// ENGRAM_DEVERR_SORT_TIMEOUT instead of hanging). Data written by other blocks
+// the phases are separated by a grid barrier on one arrival counter (bounded
+// wait; a timeout raises ENGRAM_DEVERR_SORT_TIMEOUT instead of hanging). Data written by other blocks
 // in the same launch is read through L2 (ld.global.cg), never through the
 // non-coherent load path. radix_count / radix_scatter run the same phases as
 // separate launches where cooperative launch is unavailable.
@@ -35,8 +37,7 @@ namespace engram {
 namespace bwd {
 
 constexpr int kSortThreads = 256;
-constexpr int kSortItems = 8;
-constexpr int kSortTile = kSortThreads * kSortItems; // 2048 pairs per tile
+constexpr int kSortItemsMax = 8; // pairs per thread of the largest tile (2048 pairs)
 constexpr int kRadixBits = 8;
 constexpr int kRadix = 1 << kRadixBits;
 constexpr int kMaxPasses = 4; // keys below 2^32
@@ -47,14 +48,15 @@ static_assert(kRadix == kSortThreads, "one thread per digit");
 
 __device__ __forceinline__ uint32_t item_key(uint64_t it) { return (uint32_t)(it >> 32); }
 
-struct SortSmem {
+template <int ITEMS> struct SortSmem {
+    static constexpr int kTile = kSortThreads * ITEMS;
     uint32_t whist[kSortWarps][kRadix];
     uint32_t tstart[kRadix];
     uint32_t gbase[kRadix];
     uint32_t cnt[kRadix];
     uint32_t warp[32];
     unsigned long long warp2[32];
-    unsigned long long items[kSortTile];
+    unsigned long long items[kTile];
     int flag;
 };
 
@@ -93,24 +95,24 @@ __device__ __forceinline__ uint32_t digit_peers(uint32_t dg, bool valid)
 }
 
 // Count phase of one tile. Pass 0 also flags keys outside [0, rows).
-template <bool COHERENT>
-__device__ __forceinline__ void count_tile(SortSmem &sm, const void *src, bool first, int64_t n,
+template <bool COHERENT, int ITEMS>
+__device__ __forceinline__ void count_tile(SortSmem<ITEMS> &sm, const void *src, bool first, int64_t n,
                                            int shift, uint32_t rows, int tile,
                                            uint32_t *tile_cnt, uint32_t *group_cnt)
 {
     const int tid = threadIdx.x, lane = tid & 31;
     sm.cnt[tid] = 0;
     __syncthreads();
-    const int64_t base = (int64_t)tile * kSortTile;
-    uint32_t key[kSortItems];
+    const int64_t base = (int64_t)tile * SortSmem<ITEMS>::kTile;
+    uint32_t key[ITEMS];
 #pragma unroll
-    for (int r = 0; r < kSortItems; ++r) {
+    for (int r = 0; r < ITEMS; ++r) {
         const int64_t i = base + r * kSortThreads + tid;
         key[r] = i < n ? item_key(load_item<COHERENT>(src, first, i)) : 0u;
     }
     bool bad = false;
 #pragma unroll
-    for (int r = 0; r < kSortItems; ++r) {
+    for (int r = 0; r < ITEMS; ++r) {
         const bool valid = base + r * kSortThreads + tid < n;
         if (first && valid && key[r] >= rows)
             bad = true;
@@ -134,26 +136,25 @@ __device__ __forceinline__ void count_tile(SortSmem &sm, const void *src, bool f
 // Loads the tile's items and ranks them stably: rank[r] is item r's position
 // among the items of its digit in its warp, and sm.whist[w][d] ends up as the
 // number of items of digit d in warp w. Pass 0 also flags keys outside the table.
-template <bool COHERENT>
-__device__ __forceinline__ void rank_tile(SortSmem &sm, const void *src, bool first, int64_t n,
-                                          int shift, uint32_t rows, int tile,
-                                          uint64_t (&it)[kSortItems],
-                                          uint32_t (&rank)[kSortItems])
+template <bool COHERENT, int ITEMS>
+__device__ __forceinline__ void rank_tile(SortSmem<ITEMS> &sm, const void *src, bool first,
+                                          int64_t n, int shift, uint32_t rows, int tile,
+                                          uint64_t (&it)[ITEMS], uint32_t (&rank)[ITEMS])
 {
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     for (int k = tid; k < kSortWarps * kRadix; k += kSortThreads)
         (&sm.whist[0][0])[k] = 0;
-    const int64_t wbase = (int64_t)tile * kSortTile + (int64_t)wid * (32 * kSortItems);
+    const int64_t wbase = (int64_t)tile * SortSmem<ITEMS>::kTile + (int64_t)wid * (32 * ITEMS);
     const uint32_t lt = lanemask_lt();
 #pragma unroll
-    for (int r = 0; r < kSortItems; ++r) {
+    for (int r = 0; r < ITEMS; ++r) {
         const int64_t i = wbase + r * 32 + lane;
         it[r] = i < n ? load_item<COHERENT>(src, first, i) : 0ull;
     }
     __syncthreads(); // whist zeroed
     bool bad = false;
 #pragma unroll
-    for (int r = 0; r < kSortItems; ++r) {
+    for (int r = 0; r < ITEMS; ++r) {
         const bool valid = wbase + r * 32 + lane < n;
         if (first && valid && item_key(it[r]) >= rows)
             bad = true;
@@ -176,7 +177,7 @@ __device__ __forceinline__ void rank_tile(SortSmem &sm, const void *src, bool fi
 
 // Thread d: turns sm.whist[.][d] into per-warp exclusive offsets and returns
 // the tile's count of digit d.
-__device__ __forceinline__ uint32_t tile_digit_count(SortSmem &sm)
+template <int ITEMS> __device__ __forceinline__ uint32_t tile_digit_count(SortSmem<ITEMS> &sm)
 {
     const int d = threadIdx.x;
     uint32_t tcount = 0;
@@ -201,11 +202,11 @@ __device__ __forceinline__ void publish_counts(int tile, uint32_t tcount, uint32
 
 // Writes a ranked tile to its sorted positions, once every tile of the pass
 // has published its counts. tcount is digit threadIdx.x's count in the tile.
-template <bool COHERENT>
-__device__ __forceinline__ void place_tile(SortSmem &sm, unsigned long long *dst, int64_t n,
-                                           int shift, int tile, uint32_t tcount,
-                                           const uint64_t (&it)[kSortItems],
-                                           const uint32_t (&rank)[kSortItems],
+template <bool COHERENT, int ITEMS>
+__device__ __forceinline__ void place_tile(SortSmem<ITEMS> &sm, unsigned long long *dst,
+                                           int64_t n, int shift, int tile, uint32_t tcount,
+                                           const uint64_t (&it)[ITEMS],
+                                           const uint32_t (&rank)[ITEMS],
                                            const uint32_t *tile_cnt, const uint32_t *group_cnt,
                                            int ngroups)
 {
@@ -251,17 +252,17 @@ __device__ __forceinline__ void place_tile(SortSmem &sm, unsigned long long *dst
     sm.gbase[d] = dbase + excl - tstart;
     __syncthreads();
 
-    const int64_t wbase = (int64_t)tile * kSortTile + (int64_t)wid * (32 * kSortItems);
+    const int64_t wbase = (int64_t)tile * SortSmem<ITEMS>::kTile + (int64_t)wid * (32 * ITEMS);
 #pragma unroll
-    for (int r = 0; r < kSortItems; ++r) {
+    for (int r = 0; r < ITEMS; ++r) {
         if (wbase + r * 32 + lane < n) {
             const uint32_t dg = (item_key(it[r]) >> shift) & (kRadix - 1);
             sm.items[sm.tstart[dg] + sm.whist[wid][dg] + rank[r]] = it[r];
         }
     }
     __syncthreads();
-    const int64_t base = (int64_t)tile * kSortTile;
-    const int tile_n = (int)min64(kSortTile, n - base);
+    const int64_t base = (int64_t)tile * SortSmem<ITEMS>::kTile;
+    const int tile_n = (int)min64(SortSmem<ITEMS>::kTile, n - base);
     for (int p = tid; p < tile_n; p += kSortThreads) {
         const unsigned long long x = sm.items[p];
         const uint32_t dg = (item_key(x) >> shift) & (kRadix - 1);
@@ -271,14 +272,14 @@ __device__ __forceinline__ void place_tile(SortSmem &sm, unsigned long long *dst
 }
 
 // Scatter phase of one tile after a separate count phase: rank, then place.
-template <bool COHERENT>
-__device__ __forceinline__ void scatter_tile(SortSmem &sm, const void *src, bool first,
+template <bool COHERENT, int ITEMS>
+__device__ __forceinline__ void scatter_tile(SortSmem<ITEMS> &sm, const void *src, bool first,
                                              unsigned long long *dst, int64_t n, int shift,
                                              int tile, const uint32_t *tile_cnt,
                                              const uint32_t *group_cnt, int ngroups)
 {
-    uint64_t it[kSortItems];
-    uint32_t rank[kSortItems];
+    uint64_t it[ITEMS];
+    uint32_t rank[ITEMS];
     // (the count phase has already checked the keys against the table)
     rank_tile<COHERENT>(sm, src, first, n, shift, 0xffffffffu, tile, it, rank);
     const uint32_t tcount = tile_digit_count(sm);
@@ -288,22 +289,22 @@ __device__ __forceinline__ void scatter_tile(SortSmem &sm, const void *src, bool
 
 // ----------------------------------------------- one launch per phase
 
-template <bool FIRST>
+template <bool FIRST, int ITEMS>
 __global__ void __launch_bounds__(kSortThreads)
     radix_count(const void *__restrict__ src, int64_t n, int shift, uint32_t rows,
                 uint32_t *__restrict__ tile_cnt, uint32_t *__restrict__ group_cnt)
 {
-    __shared__ SortSmem sm;
+    __shared__ SortSmem<ITEMS> sm;
     count_tile<false>(sm, src, FIRST, n, shift, rows, blockIdx.x, tile_cnt, group_cnt);
 }
 
-template <bool FIRST>
+template <bool FIRST, int ITEMS>
 __global__ void __launch_bounds__(kSortThreads)
     radix_scatter(const void *__restrict__ src, unsigned long long *__restrict__ dst,
                   int64_t n, int shift, const uint32_t *__restrict__ tile_cnt,
                   const uint32_t *__restrict__ group_cnt, int ngroups)
 {
-    __shared__ SortSmem sm;
+    __shared__ SortSmem<ITEMS> sm;
     scatter_tile<false>(sm, src, FIRST, dst, n, shift, blockIdx.x, tile_cnt, group_cnt,
                         ngroups);
 }
@@ -318,26 +319,30 @@ struct SortArgs {
     int passes, ntiles, ngroups;
     uint32_t *tile_cnt;  // [ntiles][256], rewritten every pass
     uint32_t *group_cnt; // [passes][ngroups][256], zero on entry
-    unsigned *barrier;   // [2]: arrival count, generation; zero on entry
+    unsigned *barrier;   // grid-barrier arrival counter; zero on entry
 };
 
-// Grid-wide barrier among co-resident blocks. The last block to arrive resets
-// the count and advances the generation; the others poll it with a bound.
-// Returns false (and raises ENGRAM_DEVERR_SORT_TIMEOUT) if the wait gave up.
+// Grid-wide barrier among co-resident blocks on one arrival counter that only
+// grows: barrier k of the launch is passed once the counter reaches
+// k * gridDim.x. Thread 0 of each block arrives with one acquire-release add
+// and, unless it was the last to arrive, polls the counter with acquire loads
+// (bounded; giving up raises ENGRAM_DEVERR_SORT_TIMEOUT and returns false).
+// The block's other threads wait at __syncthreads, which orders their later
+// reads after thread 0's acquire. The counter is zero at launch.
 __device__ __forceinline__ bool grid_barrier(unsigned *bar, unsigned &gen, int &flag)
 {
     __syncthreads();
     if (threadIdx.x == 0) {
-        const unsigned target = gen + 1;
+        const unsigned target = (gen + 1) * gridDim.x;
+        unsigned before;
+        asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;"
+                     : "=r"(before)
+                     : "l"(bar)
+                     : "memory");
         bool ok = true;
-        __threadfence();
-        if (atomicAdd(&bar[0], 1u) == gridDim.x - 1) {
-            atomicExch(&bar[0], 0u);
-            __threadfence();
-            atomicExch(&bar[1], target);
-        } else {
+        if (before + 1 < target) {
             uint32_t spins = 0;
-            while (ld_acquire_u32(&bar[1]) != target) {
+            while (ld_acquire_u32(bar) < target) {
                 if (++spins > kBarrierSpin) {
                     raise_device_error(ENGRAM_DEVERR_SORT_TIMEOUT);
                     ok = false;
@@ -346,7 +351,6 @@ __device__ __forceinline__ bool grid_barrier(unsigned *bar, unsigned &gen, int &
                 __nanosleep(64);
             }
         }
-        __threadfence();
         flag = ok;
     }
     __syncthreads();
@@ -354,10 +358,11 @@ __device__ __forceinline__ bool grid_barrier(unsigned *bar, unsigned &gen, int &
     return flag != 0;
 }
 
-// Four blocks per SM keep 592 tiles (1.2M pairs) resident on a 148-SM B200.
-__global__ void __launch_bounds__(kSortThreads, 4) radix_sort_coop(SortArgs a)
+// Four blocks per SM keep 592 tiles (1.2M pairs at ITEMS = 8) resident on a
+// 148-SM B200.
+template <int ITEMS> __global__ void __launch_bounds__(kSortThreads, 4) radix_sort_coop(SortArgs a)
 {
-    __shared__ SortSmem sm;
+    __shared__ SortSmem<ITEMS> sm;
     unsigned gen = 0;
     if (a.ntiles <= (int)gridDim.x) {
         // One tile per block: rank once, keep the items and their ranks in
@@ -371,8 +376,8 @@ __global__ void __launch_bounds__(kSortThreads, 4) radix_sort_coop(SortArgs a)
             unsigned long long *dst = pass % 2 == 0 ? a.a : a.b;
             uint32_t *gc = a.group_cnt + (size_t)pass * a.ngroups * kRadix;
             const int shift = pass * kRadixBits;
-            uint64_t it[kSortItems];
-            uint32_t rank[kSortItems];
+            uint64_t it[ITEMS];
+            uint32_t rank[ITEMS];
             uint32_t tcount = 0;
             if (has) {
                 rank_tile<true>(sm, src, first, a.n, shift, a.rows, tile, it, rank);
