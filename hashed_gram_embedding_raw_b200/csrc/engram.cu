@@ -282,73 +282,85 @@ int check_workspace(const BwdPlan &P, void *ws, size_t ws_bytes)
     return ENGRAM_OK;
 }
 
+// The one-launch sort at I pairs per thread; *launched is false where the
+// device or the launch refuses a cooperative grid (nothing ran).
 template <int I>
-int launch_sort_t(const int32_t *idx, int64_t n, int64_t rows, const BwdPlan &P, char *ws,
-                  cudaStream_t stream)
+int launch_sort_coop(const int32_t *idx, int64_t n, int64_t rows, const BwdPlan &P, char *ws,
+                     cudaStream_t stream, bool *launched)
 {
     using namespace bwd;
-    auto *A = (unsigned long long *)(ws + P.a);
-    auto *B = (unsigned long long *)(ws + P.b);
-    auto *tile_cnt = (uint32_t *)(ws + P.tile_cnt);
-    auto *group_cnt = (uint32_t *)(ws + P.group_cnt);
-    if (cudaMemsetAsync(ws + P.ctl, 0, P.ctl_bytes, stream) != cudaSuccess)
-        return ENGRAM_ECUDA;
-
-    // One cooperative launch for every pass when the device supports it: the
-    // grid is at most the co-resident blocks, which the launch itself checks.
+    *launched = false;
     int dev = 0, coop = 0;
-    if (cudaGetDevice(&dev) == cudaSuccess &&
-        cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) == cudaSuccess &&
-        coop) {
-        int64_t res = 0;
-        ENGRAM_TRY(resident_warps(radix_sort_coop<I>, kSortThreads, 0, &res));
-        const int grid = (int)std::min<int64_t>(P.ntiles, res / (kSortThreads / 32));
-        SortArgs args{idx, A, B, n, (uint32_t)rows, P.passes, P.ntiles, P.ngroups,
-                      tile_cnt, group_cnt, (unsigned *)(ws + P.barrier)};
-        void *params[] = {&args};
-        if (cudaLaunchCooperativeKernel((const void *)radix_sort_coop<I>, dim3(grid),
-                                        dim3(kSortThreads), params, 0, stream) == cudaSuccess) {
-            g_launches.fetch_add(1, std::memory_order_relaxed);
-            return ENGRAM_OK;
-        }
-        (void)cudaGetLastError(); // not launched: run the phases as separate launches
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess || !coop)
+        return ENGRAM_OK;
+    // the grid is at most the co-resident blocks, which the launch itself checks
+    int64_t res = 0;
+    ENGRAM_TRY(resident_warps(radix_sort_coop<I>, kSortThreads, 0, &res));
+    const int grid = (int)std::min<int64_t>(P.ntiles, res / (kSortThreads / 32));
+    SortArgs args{idx, (unsigned long long *)(ws + P.a), (unsigned long long *)(ws + P.b), n,
+                  (uint32_t)rows, P.passes, P.ntiles, P.ngroups, (uint32_t *)(ws + P.tile_cnt),
+                  (uint32_t *)(ws + P.group_cnt), (unsigned *)(ws + P.barrier)};
+    void *params[] = {&args};
+    if (cudaLaunchCooperativeKernel((const void *)radix_sort_coop<I>, dim3(grid),
+                                    dim3(kSortThreads), params, 0, stream) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return ENGRAM_OK;
     }
-
-    const void *src = idx;
-    for (int pass = 0; pass < P.passes; ++pass) {
-        unsigned long long *dst = (pass % 2 == 0) ? A : B;
-        uint32_t *gc = group_cnt + (size_t)pass * kRadix * P.ngroups;
-        const int shift = pass * kRadixBits;
-        if (pass == 0) {
-            radix_count<true, I><<<P.ntiles, kSortThreads, 0, stream>>>(src, n, shift,
-                                                                    (uint32_t)rows, tile_cnt, gc);
-            ENGRAM_TRY(after_launch());
-            radix_scatter<true, I><<<P.ntiles, kSortThreads, 0, stream>>>(src, dst, n, shift,
-                                                                      tile_cnt, gc, P.ngroups);
-        } else {
-            radix_count<false, I><<<P.ntiles, kSortThreads, 0, stream>>>(src, n, shift,
-                                                                     (uint32_t)rows, tile_cnt, gc);
-            ENGRAM_TRY(after_launch());
-            radix_scatter<false, I><<<P.ntiles, kSortThreads, 0, stream>>>(src, dst, n, shift,
-                                                                       tile_cnt, gc, P.ngroups);
-        }
-        ENGRAM_TRY(after_launch());
-        src = dst;
-    }
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    *launched = true;
     return ENGRAM_OK;
 }
 
 int launch_sort(const int32_t *idx, int64_t n, int64_t rows, const BwdPlan &P, char *ws,
                 cudaStream_t stream)
 {
+    using namespace bwd;
+    if (cudaMemsetAsync(ws + P.ctl, 0, P.ctl_bytes, stream) != cudaSuccess)
+        return ENGRAM_ECUDA;
+    bool launched = false;
     switch (P.items) {
-    case 4: return launch_sort_t<4>(idx, n, rows, P, ws, stream);
-    case 5: return launch_sort_t<5>(idx, n, rows, P, ws, stream);
-    case 6: return launch_sort_t<6>(idx, n, rows, P, ws, stream);
-    case 7: return launch_sort_t<7>(idx, n, rows, P, ws, stream);
-    case 8: return launch_sort_t<8>(idx, n, rows, P, ws, stream);
+    case 4: ENGRAM_TRY(launch_sort_coop<4>(idx, n, rows, P, ws, stream, &launched)); break;
+    case 5: ENGRAM_TRY(launch_sort_coop<5>(idx, n, rows, P, ws, stream, &launched)); break;
+    case 6: ENGRAM_TRY(launch_sort_coop<6>(idx, n, rows, P, ws, stream, &launched)); break;
+    case 7: ENGRAM_TRY(launch_sort_coop<7>(idx, n, rows, P, ws, stream, &launched)); break;
+    case 8: ENGRAM_TRY(launch_sort_coop<8>(idx, n, rows, P, ws, stream, &launched)); break;
     default: return ENGRAM_EINVAL;
     }
+    if (launched)
+        return ENGRAM_OK;
+
+    // Without a cooperative launch: two launches per pass, on the largest
+    // tiles (2,048 pairs; their counts take no more workspace than the plan's).
+    constexpr int I = kSortItemsMax;
+    const int ntiles = (int)std::max<int64_t>(1, ceil_div(n, (int64_t)kSortThreads * I));
+    const int ngroups = (int)ceil_div(ntiles, kTilesPerGroup);
+    auto *A = (unsigned long long *)(ws + P.a);
+    auto *B = (unsigned long long *)(ws + P.b);
+    auto *tile_cnt = (uint32_t *)(ws + P.tile_cnt);
+    auto *group_cnt = (uint32_t *)(ws + P.group_cnt);
+    const void *src = idx;
+    for (int pass = 0; pass < P.passes; ++pass) {
+        unsigned long long *dst = (pass % 2 == 0) ? A : B;
+        uint32_t *gc = group_cnt + (size_t)pass * kRadix * ngroups;
+        const int shift = pass * kRadixBits;
+        if (pass == 0) {
+            radix_count<true, I><<<ntiles, kSortThreads, 0, stream>>>(src, n, shift,
+                                                                     (uint32_t)rows, tile_cnt, gc);
+            ENGRAM_TRY(after_launch());
+            radix_scatter<true, I><<<ntiles, kSortThreads, 0, stream>>>(src, dst, n, shift,
+                                                                       tile_cnt, gc, ngroups);
+        } else {
+            radix_count<false, I><<<ntiles, kSortThreads, 0, stream>>>(src, n, shift,
+                                                                      (uint32_t)rows, tile_cnt, gc);
+            ENGRAM_TRY(after_launch());
+            radix_scatter<false, I><<<ntiles, kSortThreads, 0, stream>>>(src, dst, n, shift,
+                                                                        tile_cnt, gc, ngroups);
+        }
+        ENGRAM_TRY(after_launch());
+        src = dst;
+    }
+    return ENGRAM_OK;
 }
 
 template <int DT, int GF, int RVT>

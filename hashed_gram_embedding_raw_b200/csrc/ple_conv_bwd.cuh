@@ -397,6 +397,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
 #pragma unroll
     for (int q = 0; q < RING; ++q)
         inv[q] = 0.f;
+    // normalised x of the lagged rows (ring rows 0 .. B - 1), kept from stage
+    // 2 of a batch for its stage 3 and, across the barrier, its stage 4
+    float2 xl[B][NP];
+#pragma unroll
+    for (int i = 0; i < B; ++i)
+#pragma unroll
+        for (int pp = 0; pp < NP; ++pp)
+            xl[i][pp] = zero2;
 
     // ---- stage 4 of batch b (first slot s0): dx of its lagged rows (ring
     // rows 0 .. B - 1), once the dot partials it posted are complete
@@ -424,8 +432,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
                     continue;
                 const float mean = do_norm ? means[i] * a.inv_G : 0.f;
                 float g[CH], o[CH];
-                float2 xh[NP];
-                load_xh(slot[i], inv[i], xh);
+                const float2 *xh = xl[i];
                 if (do_res)
                     load_slot4<GT>(gs_t + (uint32_t)slot[i] * pg, g);
                 const float2 ij2 = make_float2(inv[i], inv[i]);
@@ -520,6 +527,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
                     continue;  // not loaded (no batch row reads it: its tap is out of range)
                 float2 xh[NP];
                 load_xh(slot[q], inv[q], xh);
+                if (q < B)
+#pragma unroll
+                    for (int pp = 0; pp < NP; ++pp)
+                        xl[q][pp] = xh[pp];
 #pragma unroll
                 for (int i = 0; i < B; ++i) {
                     const int k = L + i - q;
@@ -585,8 +596,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
                     const int32_t jj = j0 - L + i;
                     float2 accd = zero2;
                     if (FAST || (active && jj >= ja && jj < jb)) {
-                        float2 xh[NP];
-                        load_xh(slot[i], inv[i], xh);
+                        const float2 *xh = xl[i];
 #pragma unroll
                         for (int pp = 0; pp < NP; ++pp) {
                             float2 dn = zero2;
