@@ -274,6 +274,7 @@ __global__ void __maxnreg__(CH == 4 ? 80 : 128)
     char *out = static_cast<char *>(a.out) + ((int64_t)m * a.G + (int64_t)tid * CH) * sizeof(OT);
     const uint32_t xoff = (uint32_t)tid * CH * sizeof(XT);
     const int64_t orow = (int64_t)a.C * sizeof(OT);
+    const int64_t ostep = (int64_t)d * orow;  // from one row of the residue to the next
     for (int c = 0; c < nbatch; ++c) {
         const int b = c % NB;
         const int32_t j0 = js + c * B;
@@ -281,6 +282,24 @@ __global__ void __maxnreg__(CH == 4 ? 80 : 128)
         if (!timed_out && !mbar_wait(full_bar + b, (uint32_t)(c / NB) & 1u))
             timed_out = true;
         const uint32_t buf = smem_u32(data) + (uint32_t)(b * B) * pitch + xoff;
+        // the batch's inverse RMS values in two 16-byte loads, and the output
+        // row advanced by one stride per row (the conv warps are close to
+        // issue-bound, so per-row address and load instructions count)
+        static_assert(B == 8, "two float4 of inverse RMS per batch");
+        float invb[B];
+        {
+            const float4 lo = *reinterpret_cast<const float4 *>(inv_s + b * B);
+            const float4 hi = *reinterpret_cast<const float4 *>(inv_s + b * B + 4);
+            invb[0] = lo.x;
+            invb[1] = lo.y;
+            invb[2] = lo.z;
+            invb[3] = lo.w;
+            invb[4] = hi.x;
+            invb[5] = hi.y;
+            invb[6] = hi.z;
+            invb[7] = hi.w;
+        }
+        char *orow_p = out + (int64_t)(r + j0 * d) * orow;
         auto run = [&](auto fast_tag) {
             constexpr bool FAST = decltype(fast_tag)::value;
 #pragma unroll
@@ -294,7 +313,7 @@ __global__ void __maxnreg__(CH == 4 ? 80 : 128)
 #pragma unroll
                     for (int e = 0; e < CH; ++e)
                         xv[e] = 0.f;
-                const float inv = inv_s[b * B + i];
+                const float inv = invb[i];
                 const float2 inv2 = make_float2(inv, inv);
                 int nv = H;
                 if constexpr (!FAST)
@@ -341,8 +360,9 @@ __global__ void __maxnreg__(CH == 4 ? 80 : 128)
                     constexpr int OW = CH * (int)sizeof(OT) / 4;
                     uint32_t w[OW];
                     Elem<OT>::template pack<CH>(o, w);
-                    store_words<OW * 4>(out + (int64_t)(r + j * d) * orow, w);
+                    store_words<OW * 4>(orow_p, w);
                 }
+                orow_p += ostep;
             }
         };
         if (fast_s[b])
