@@ -268,6 +268,19 @@ def test_backward_radix_pass_counts(E, rows):
     check_backward(E, idx, dout, rows, oracle.F32)
 
 
+@pytest.mark.parametrize("n", [151_552, 180_000, 200_000, 900_000])
+def test_backward_sort_tile_sizes(E, n):
+    """The sort picks its tile (256 x I pairs, I = 4..8) per call from n and the
+    SM count; on a 148-SM part these n select I = 4, 5, 6 and 8 with every
+    tile resident (the workloads above reach only 4, 7 and 8 non-resident).
+    Half the lookups hit a few hot rows, so segments cross tiles."""
+    rng = np.random.Generator(np.random.PCG64(n))
+    rows = 320_001_536
+    idx = np.where(rng.random(n) < 0.5, rng.integers(0, 40, n), rng.integers(0, rows, n))
+    dout = torch.randn(n, 16, generator=torch.Generator().manual_seed(n % 997))
+    check_backward(E, idx.astype(np.int64), dout, rows, oracle.F32)
+
+
 def test_backward_empty(E):
     uniq, grads, nu = E.engram_backward(torch.empty(0, dtype=torch.int32, device="cuda"),
                                         torch.empty(0, 160, device="cuda"), 100)
