@@ -132,7 +132,7 @@ def test_backward_then_step_end_to_end(E):
     n = len(ids) * params.heads
     dout = host_dout("tiny", n, D, "f32")
     tab_d = torch.from_numpy(table.copy()).cuda()
-    ids_d, cu_d = torch.from_numpy(ids).cuda(), torch.from_numpy(cu).cuda()
+    ids_d, cu_d = torch.from_numpy(ids.copy()).cuda(), torch.from_numpy(cu.copy()).cuda()
     _, idx = E.engram_hash_gather(params, ids_d, tab_d, cu_seqlens=cu_d)
     uniq, grads, nu = E.engram_backward(idx.view(-1), dout.cuda(), R)
     m = torch.zeros((R, D), device="cuda")
