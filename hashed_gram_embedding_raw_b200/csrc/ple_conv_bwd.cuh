@@ -35,9 +35,12 @@
 //            gradients, and partials of sum(s dn xh), posted to both blocks;
 //   stage 4  dx of the lagged rows (streaming stores), then the ring shifts.
 // Stages 1 and 3 post partial sums that stages 2 and 4 need complete; the
-// batches are software-pipelined so that one barrier (over the cluster)
-// serves both: iteration b runs stage 4 of batch b - 1, stages 2 and 3 of
-// batch b and stage 1 of batch b + 1, then the barrier.
+// batches are software-pipelined so that one synchronisation serves both:
+// iteration b runs stage 4 of batch b - 1, stages 2 and 3 of batch b and
+// stage 1 of batch b + 1, then a block barrier and a wait for the partner
+// block's posts (asynchronous stores into this block's shared memory that
+// complete on an mbarrier), so no cluster-scope release has to wait for the
+// dx stores of stage 4.
 // Rows whose taps all stay inside their sequence (nearly all) take a path
 // without per-tap masks. Rows reach shared memory through a ring of row
 // slots filled by cp.async.bulk (one copy per row of x and of dout, issued
@@ -63,19 +66,20 @@ constexpr int kBwdThreads = 32 * kBwdCtaWarps; // 4 channels per thread
 constexpr int kBwdMaxCluster = 2;              // blocks sharing a branch: G <= 2560
 constexpr int kBwdPartStride = 24;             // per-row partials (20 warps), padded for float4
 constexpr int kBwdMaxSlots = 32;
-constexpr int kBwdBars = 8;
+constexpr int kBwdBars = 8;                    // row-copy barriers (batch % 8)
+constexpr int kBwdPartBars = 2;                // partner-partial barriers (phase % 2)
 constexpr int kBwdQuantities = kBwdTaps + 2;   // weight taps, bias, norm scale
 
 // Shared memory: square-sum and dot partials [2][B][24] float each (by batch
 // parity; column rank * 10 + warp; the pads stay zero), tap counts [32] int32
-// per row slot, mbarriers [8]; then the row slots of x [slots][pitch_x] and
+// per row slot, mbarriers [8 + 2]; then the row slots of x [slots][pitch_x] and
 // of dout [slots][pitch_g]. With batches in flight from the one being
 // finished (its window reaches 3 rows back) to `ahead` past the next,
 // slots = 3 + (ahead + 2) * 4.
 constexpr int kBwdOffDot = 2 * kBwdRows * kBwdPartStride * 4;  // two buffers each
 constexpr int kBwdOffMeta = 2 * kBwdOffDot;
 constexpr int kBwdOffBars = kBwdOffMeta + kBwdMaxSlots * 4;
-constexpr int kBwdHeader = kBwdOffBars + kBwdBars * 8;
+constexpr int kBwdHeader = kBwdOffBars + (kBwdBars + kBwdPartBars) * 8;
 constexpr int kBwdDataOffset = (kBwdHeader + 127) / 128 * 128;
 
 __host__ __device__ constexpr size_t bwd_smem_bytes(int slots, int pitch_x, int pitch_g)
@@ -117,13 +121,23 @@ __device__ __forceinline__ void cluster_barrier()
                  "barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-// A float into the same offset of block `rank`'s shared memory.
-__device__ __forceinline__ void st_cluster(const float *local, uint32_t rank, float v)
+// A float into the same offset of block `rank`'s shared memory, stored
+// asynchronously: the store completes 4 bytes of transaction count on the
+// mbarrier at `bar`'s offset in that block, and a thread there that sees the
+// barrier's phase complete sees the value. No fence: the storing thread's
+// earlier global stores are not waited for.
+__device__ __forceinline__ void st_async_cluster(const float *local, uint32_t rank, float v,
+                                                 const uint64_t *bar)
 {
-    uint32_t remote;
+    uint32_t remote, rbar;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)),
                  "r"(rank));
-    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(remote), "f"(v) : "memory");
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(rbar) : "r"(smem_u32(bar)),
+                 "r"(rank));
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.f32 [%0], %1, [%2];" ::"r"(
+                     remote),
+                 "f"(v), "r"(rbar)
+                 : "memory");
 }
 
 // 4 channels of one row in a shared-memory slot (8 or 16 bytes at the
@@ -173,6 +187,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
     float *dot_part = reinterpret_cast<float *>(smem + kBwdOffDot);
     int32_t *meta_s = reinterpret_cast<int32_t *>(smem + kBwdOffMeta);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kBwdOffBars);
+    uint64_t *pbars = bars + kBwdBars;  // the partner's partials of phase k land on pbars[k % 2]
     unsigned char *xs = smem + kBwdDataOffset;
     unsigned char *gs = xs + (size_t)a.slots * a.pitch_x;
 
@@ -229,7 +244,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
         seq_hi = __ldg(a.cu + seq + 1);
     }
     if (tid == 0) {
-        for (int b = 0; b < kBwdBars; ++b)
+        for (int b = 0; b < kBwdBars + kBwdPartBars; ++b)
             mbar_init(bars + b, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -237,24 +252,50 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
         ss_part[i] = 0.f;  // (and dot_part) pads of absent warps stay zero
     for (int i = tid; i < kBwdMaxSlots; i += blockDim.x)
         meta_s[i] = 0;
-    // (every block of the cluster has started and zeroed its partials before
-    // any block writes into another's)
-    auto sync_all = [&]() {
-        if (pair)
-            cluster_barrier();
-        else
-            __syncthreads();
-    };
-    // one row sum of each warp, into this block's and the partner's partials
+    // Partial sums are posted in phases: phase 0 before the batch loop,
+    // phase b + 1 in iteration b. Each post is one row sum per warp and row,
+    // stored by 4 lanes into this block's partials and, in a pair, into the
+    // partner's with asynchronous stores that complete on the partner's
+    // pbars[phase % 2].
+    bool timed_out = false;  // a bounded wait gave up (the result is then not valid)
+    uint32_t phase = 0;
     auto post = [&](float *partials, float tot) {
         if ((lane & 7) == 0) {
             float *dst = partials + (lane >> 3) * kBwdPartStride + pslot;
             *dst = tot;
             if (pair)
-                st_cluster(dst, q_cta ^ 1u, tot);
+                st_async_cluster(dst, q_cta ^ 1u, tot, pbars + (phase & 1));
         }
     };
-    sync_all();
+    // End of a phase with `nposts` posts: this block's partials are complete
+    // after a block barrier (which also orders the ring slots for reuse), the
+    // partner's once their bytes (4 lanes x 4 B per warp and post) have landed
+    // on pbars[phase % 2]; no cluster-scope release, so the global dx stores
+    // are not waited for. The double-buffered partials cannot be overwritten
+    // early: a block posts phase k + 2 only after the partner's phase k + 1
+    // posts, which the partner makes after it has read phase k's.
+    auto end_phase = [&](int nposts) {
+        if (pair) {
+            uint64_t *pb = pbars + (phase & 1);
+            if (tid == 0)
+                asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(
+                                 smem_u32(pb)),
+                             "r"((uint32_t)nposts * 16u * (blockDim.x >> 5))
+                             : "memory");
+            __syncthreads();
+            if (!timed_out && !mbar_wait(pb, (phase >> 1) & 1u))
+                timed_out = true;
+        } else {
+            __syncthreads();
+        }
+        ++phase;
+    };
+    // every block of the cluster has started, initialised its barriers and
+    // zeroed its partials before any block writes into another's
+    if (pair)
+        cluster_barrier();
+    else
+        __syncthreads();
 
     // warp 0: rows of batch b (first slot s0) into their slots (lane i: row
     // j0 + i), and their in-sequence tap counts
@@ -340,7 +381,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
     const uint32_t xs_t = xs_u + xoff, gs_t = gs_u + goff;  // this thread's channels, slot 0
     const uint32_t px = (uint32_t)a.pitch_x, pg = (uint32_t)a.pitch_g;
     char *dxb = static_cast<char *>(a.dx) + cb * sizeof(GT) + goff;
-    bool timed_out = false;
 
     // x of ring row q (rows j0 - L .. j0 + B - 1) of the batch, normalised
     auto load_xh = [&](int slot, float iv, float2 *xh) {
@@ -471,7 +511,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
     // by batch parity, so a warp that runs ahead never overwrites partials
     // another warp still reads.
     stage1(0, 0);
-    sync_all();
+    end_phase(do_norm ? 1 : 0);
     if (wid == 0 && a.ahead < nbatch) {
         issue(a.ahead, s_issue);
         s_issue = slot_ahead(s_issue, 1);
@@ -625,7 +665,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
         const int s_next = slot_ahead(s_cur, 1);
         if (b + 1 < nbatch)
             stage1(b + 1, s_next);
-        sync_all();
+        end_phase(do_norm ? (b + 1 < nbatch ? 2 : 1) : 0);
         if (wid == 0 && b + 1 + a.ahead < nbatch) {
             issue(b + 1 + a.ahead, s_issue);
             s_issue = slot_ahead(s_issue, 1);
@@ -659,6 +699,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
     }
     if (timed_out && lane == 0)
         raise_device_error(ENGRAM_DEVERR_COPY_TIMEOUT);
+    // a block leaves only once the partner has received everything it stored
+    // into the partner's shared memory
+    if (pair)
+        cluster_barrier();
 }
 
 // Sums the blocks' partials in block order (fp64) into the weight gradients:
