@@ -200,21 +200,18 @@ __device__ __forceinline__ void publish_counts(int tile, uint32_t tcount, uint32
         atomicAdd(&group_cnt[(size_t)(tile / kTilesPerGroup) * kRadix + d], tcount);
 }
 
-// Writes a ranked tile to its sorted positions, once every tile of the pass
-// has published its counts. tcount is digit threadIdx.x's count in the tile.
+// Once every tile of the pass has published its counts: sm.tstart[d] = the
+// start of digit d = threadIdx.x in the tile, sm.gbase[d] = its global start
+// minus that. tcount is digit d's count in the tile.
 template <bool COHERENT, int ITEMS>
-__device__ __forceinline__ void place_tile(SortSmem<ITEMS> &sm, unsigned long long *dst,
-                                           int64_t n, int shift, int tile, uint32_t tcount,
-                                           const uint64_t (&it)[ITEMS],
-                                           const uint32_t (&rank)[ITEMS],
-                                           const uint32_t *tile_cnt, const uint32_t *group_cnt,
-                                           int ngroups)
+__device__ __forceinline__ void tile_offsets(SortSmem<ITEMS> &sm, int tile, uint32_t tcount,
+                                             const uint32_t *tile_cnt,
+                                             const uint32_t *group_cnt, int ngroups)
 {
-    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    // Global offset of digit d = tid for this tile. Counts are tile- and
-    // group-major, so each load instruction reads 32 consecutive digits; the
-    // loops are unrolled so the loads are in flight together.
-    const int d = tid;
+    // Counts are tile- and group-major, so each load instruction reads 32
+    // consecutive digits; the loops are unrolled so the loads are in flight
+    // together.
+    const int d = threadIdx.x;
     const int grp = tile / kTilesPerGroup;
     uint32_t excl = 0, total = 0;
     for (int g0 = 0; g0 < ngroups; g0 += 8) {
@@ -251,6 +248,20 @@ __device__ __forceinline__ void place_tile(SortSmem<ITEMS> &sm, unsigned long lo
     sm.tstart[d] = tstart;
     sm.gbase[d] = dbase + excl - tstart;
     __syncthreads();
+}
+
+// Writes a ranked tile to its sorted positions, once every tile of the pass
+// has published its counts. tcount is digit threadIdx.x's count in the tile.
+template <bool COHERENT, int ITEMS>
+__device__ __forceinline__ void place_tile(SortSmem<ITEMS> &sm, unsigned long long *dst,
+                                           int64_t n, int shift, int tile, uint32_t tcount,
+                                           const uint64_t (&it)[ITEMS],
+                                           const uint32_t (&rank)[ITEMS],
+                                           const uint32_t *tile_cnt, const uint32_t *group_cnt,
+                                           int ngroups)
+{
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    tile_offsets<COHERENT>(sm, tile, tcount, tile_cnt, group_cnt, ngroups);
 
     const int64_t wbase = (int64_t)tile * SortSmem<ITEMS>::kTile + (int64_t)wid * (32 * ITEMS);
 #pragma unroll
@@ -285,6 +296,64 @@ __device__ __forceinline__ void scatter_tile(SortSmem<ITEMS> &sm, const void *sr
     const uint32_t tcount = tile_digit_count(sm);
     place_tile<COHERENT>(sm, dst, n, shift, tile, tcount, it, rank, tile_cnt, group_cnt,
                          ngroups);
+}
+
+// Count phase of the one-launch sort when tiles outnumber the resident
+// blocks (a block cannot keep its tiles' items and ranks across the barrier):
+// ranks the tile, publishes its digit counts and writes it back ordered by
+// digit, stably, into its own region of `ordered`, so that the place phase
+// need not rank it again. `ordered` may be `src` itself (the tile region is
+// read before it is written, by this block alone).
+template <int ITEMS>
+__device__ __forceinline__ void count_order_tile(SortSmem<ITEMS> &sm, const void *src, bool first,
+                                                 int64_t n, int shift, uint32_t rows, int tile,
+                                                 uint32_t *tile_cnt, uint32_t *group_cnt,
+                                                 unsigned long long *ordered)
+{
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    uint64_t it[ITEMS];
+    uint32_t rank[ITEMS];
+    rank_tile<true>(sm, src, first, n, shift, rows, tile, it, rank);
+    const uint32_t tcount = tile_digit_count(sm);
+    publish_counts(tile, tcount, tile_cnt, group_cnt);
+    sm.tstart[tid] = block_exclusive_scan(tcount, sm.warp, nullptr);
+    __syncthreads();
+    const int64_t base = (int64_t)tile * SortSmem<ITEMS>::kTile;
+    const int64_t wbase = base + (int64_t)wid * (32 * ITEMS);
+#pragma unroll
+    for (int r = 0; r < ITEMS; ++r) {
+        if (wbase + r * 32 + lane < n) {
+            const uint32_t dg = (item_key(it[r]) >> shift) & (kRadix - 1);
+            sm.items[sm.tstart[dg] + sm.whist[wid][dg] + rank[r]] = it[r];
+        }
+    }
+    __syncthreads();
+    const int tile_n = (int)min64(SortSmem<ITEMS>::kTile, n - base);
+    for (int q = tid; q < tile_n; q += kSortThreads)
+        ordered[base + q] = sm.items[q];
+    __syncthreads(); // shared memory free for the next tile
+}
+
+// Place phase for a tile that count_order_tile left ordered by digit: each
+// run of one digit goes to that digit's global offsets.
+template <int ITEMS>
+__device__ __forceinline__ void place_ordered_tile(SortSmem<ITEMS> &sm,
+                                                   const unsigned long long *ordered,
+                                                   unsigned long long *dst, int64_t n, int shift,
+                                                   int tile, const uint32_t *tile_cnt,
+                                                   const uint32_t *group_cnt, int ngroups)
+{
+    const int tid = threadIdx.x;
+    const uint32_t tcount = __ldcg(tile_cnt + (size_t)tile * kRadix + tid);
+    tile_offsets<true>(sm, tile, tcount, tile_cnt, group_cnt, ngroups);
+    const int64_t base = (int64_t)tile * SortSmem<ITEMS>::kTile;
+    const int tile_n = (int)min64(SortSmem<ITEMS>::kTile, n - base);
+    for (int q = tid; q < tile_n; q += kSortThreads) {
+        const unsigned long long x = __ldcg(ordered + base + q);
+        const uint32_t dg = (item_key(x) >> shift) & (kRadix - 1);
+        dst[(uint32_t)(sm.gbase[dg] + (uint32_t)q)] = x;
+    }
+    __syncthreads(); // shared memory free for the next tile
 }
 
 // ----------------------------------------------- one launch per phase
@@ -394,19 +463,23 @@ template <int ITEMS> __global__ void __launch_bounds__(kSortThreads, 4) radix_so
         }
         return;
     }
+    // More tiles than resident blocks: each tile is ranked once, in the count
+    // phase, and left ordered by digit in `ordered` (the pass's own input from
+    // the second pass on; the other item buffer on the first, whose input is
+    // idx), from where the place phase moves it.
     for (int pass = 0; pass < a.passes; ++pass) {
         const bool first = pass == 0;
         const void *src = first ? (const void *)a.idx : (pass % 2 == 1 ? a.a : a.b);
         unsigned long long *dst = pass % 2 == 0 ? a.a : a.b;
+        unsigned long long *ordered = first ? a.b : (pass % 2 == 1 ? a.a : a.b);
         uint32_t *gc = a.group_cnt + (size_t)pass * a.ngroups * kRadix;
         const int shift = pass * kRadixBits;
         for (int tile = blockIdx.x; tile < a.ntiles; tile += gridDim.x)
-            count_tile<true>(sm, src, first, a.n, shift, a.rows, tile, a.tile_cnt, gc);
+            count_order_tile(sm, src, first, a.n, shift, a.rows, tile, a.tile_cnt, gc, ordered);
         if (!grid_barrier(a.barrier, gen, sm.flag))
             return;
         for (int tile = blockIdx.x; tile < a.ntiles; tile += gridDim.x)
-            scatter_tile<true>(sm, src, first, dst, a.n, shift, tile, a.tile_cnt, gc,
-                               a.ngroups);
+            place_ordered_tile(sm, ordered, dst, a.n, shift, tile, a.tile_cnt, gc, a.ngroups);
         if (pass + 1 < a.passes && !grid_barrier(a.barrier, gen, sm.flag))
             return;
     }

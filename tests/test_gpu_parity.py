@@ -268,12 +268,13 @@ def test_backward_radix_pass_counts(E, rows):
     check_backward(E, idx, dout, rows, oracle.F32)
 
 
-@pytest.mark.parametrize("n", [151_552, 180_000, 200_000, 900_000])
+@pytest.mark.parametrize("n", [151_552, 180_000, 200_000, 900_000, 2_000_003])
 def test_backward_sort_tile_sizes(E, n):
     """The sort picks its tile (256 x I pairs, I = 4..8) per call from n and the
     SM count; on a 148-SM part these n select I = 4, 5, 6 and 8 with every
-    tile resident (the workloads above reach only 4, 7 and 8 non-resident).
-    Half the lookups hit a few hot rows, so segments cross tiles."""
+    tile resident, and 2,000,003 pairs (more tiles than resident blocks) take
+    the path that ranks each tile once and moves it from its digit-ordered
+    copy. Half the lookups hit a few hot rows, so segments cross tiles."""
     rng = np.random.Generator(np.random.PCG64(n))
     rows = 320_001_536
     idx = np.where(rng.random(n) < 0.5, rng.integers(0, 40, n), rng.integers(0, rows, n))
