@@ -8,6 +8,7 @@
 #include <atomic>
 #include <climits>
 #include <cmath>
+#include <cstdlib>
 #include <cstring>
 #include <map>
 #include <mutex>
@@ -312,6 +313,18 @@ int launch_sort_coop(const int32_t *idx, int64_t n, int64_t rows, const BwdPlan 
     return ENGRAM_OK;
 }
 
+// ENGRAM_SORT_SEPARATE_LAUNCHES=1 in the environment (read once per process)
+// makes the sort take its two-launches-per-pass form, the one devices without
+// cooperative launch get, so that it can be checked on a device that has it.
+bool sort_separate_launches()
+{
+    static const bool v = [] {
+        const char *e = std::getenv("ENGRAM_SORT_SEPARATE_LAUNCHES");
+        return e != nullptr && e[0] == '1';
+    }();
+    return v;
+}
+
 int launch_sort(const int32_t *idx, int64_t n, int64_t rows, const BwdPlan &P, char *ws,
                 cudaStream_t stream)
 {
@@ -319,7 +332,8 @@ int launch_sort(const int32_t *idx, int64_t n, int64_t rows, const BwdPlan &P, c
     if (cudaMemsetAsync(ws + P.ctl, 0, P.ctl_bytes, stream) != cudaSuccess)
         return ENGRAM_ECUDA;
     bool launched = false;
-    switch (P.items) {
+    switch (sort_separate_launches() ? 0 : P.items) {
+    case 0: break;
     case 4: ENGRAM_TRY(launch_sort_coop<4>(idx, n, rows, P, ws, stream, &launched)); break;
     case 5: ENGRAM_TRY(launch_sort_coop<5>(idx, n, rows, P, ws, stream, &launched)); break;
     case 6: ENGRAM_TRY(launch_sort_coop<6>(idx, n, rows, P, ws, stream, &launched)); break;

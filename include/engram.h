@@ -200,7 +200,10 @@ ENGRAM_API int engram_backward(const int32_t *idx, int64_t n, int64_t table_rows
                     float *row_grads, int32_t *num_unique, void *workspace,
                     size_t workspace_bytes, engram_stream_t stream);
 
-/* First stage: stable LSD radix sort of the (idx[j], j) pairs into the workspace. */
+/* First stage: stable LSD radix sort of the (idx[j], j) pairs into the workspace.
+ * One cooperative launch where the device supports it, else two launches per
+ * radix pass; ENGRAM_SORT_SEPARATE_LAUNCHES=1 in the environment (read once per
+ * process) forces the second form. Both give the same result. */
 ENGRAM_API int engram_backward_sort(const int32_t *idx, int64_t n, int64_t table_rows, int32_t dim,
                          void *workspace, size_t workspace_bytes, engram_stream_t stream);
 

@@ -1,0 +1,56 @@
+"""The backward sort's separate-launch form -- what a device without
+cooperative launch runs: two launches per pass on 2,048-pair tiles -- forced
+with ENGRAM_SORT_SEPARATE_LAUNCHES=1 in a child process, against the
+one-launch sort in another child on the same inputs. A stable sort has one
+result, so the distinct rows and their fp32 sums must be identical bit for
+bit. The sizes cover one tile, a ragged single tile, many resident tiles and
+more tiles than resident blocks; half the lookups hit a few hot rows.
+"""
+
+import os
+import subprocess
+import sys
+
+import numpy as np
+import pytest
+
+pytestmark = pytest.mark.gpu
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+CHILD = r"""
+import sys
+import numpy as np
+import torch
+sys.path.insert(0, sys.argv[1])
+import hashed_gram_embedding_raw_b200 as E
+rows = 320_001_536
+out = {}
+for n in (1, 1000, 250_007, 2_000_003):
+    rng = np.random.Generator(np.random.PCG64(n))
+    idx = np.where(rng.random(n) < 0.5, rng.integers(0, 40, n),
+                   rng.integers(0, rows, n)).astype(np.int32)
+    dout = torch.randn(n, 16, generator=torch.Generator().manual_seed(n % 997))
+    u, g, nu = E.engram_backward(torch.from_numpy(idx).cuda(), dout.cuda(), rows)
+    U = int(nu.item())
+    assert E.engram_get_device_error() == 0
+    out["u%d" % n] = u[:U].cpu().numpy()
+    out["g%d" % n] = g[:U].cpu().numpy()
+np.savez(sys.argv[2], **out)
+"""
+
+
+def run_child(tmp_path, separate: bool):
+    path = tmp_path / ("separate.npz" if separate else "one_launch.npz")
+    env = dict(os.environ, ENGRAM_SORT_SEPARATE_LAUNCHES="1" if separate else "0")
+    subprocess.run([sys.executable, "-c", CHILD, ROOT, str(path)], env=env, check=True,
+                   timeout=600)
+    return np.load(path)
+
+
+def test_separate_launch_sort_matches_one_launch(tmp_path):
+    split = run_child(tmp_path, True)
+    coop = run_child(tmp_path, False)
+    assert sorted(split.files) == sorted(coop.files)
+    for k in coop.files:
+        assert np.array_equal(split[k], coop[k]), k
