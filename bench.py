@@ -7,6 +7,9 @@ gradients) over one batch of the named workload, all inputs resident in HBM.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload full]
     python bench.py --impl reference ...   # the CPU oracle, timed on this host
+    python bench.py --stage hash ...       # engram_hash alone (L2 flushed between launches)
+    python bench.py --stage gather ...     # engram_gather alone on the hash's indices
+    python bench.py --stage bwd ...        # the backward alone (sort + reduce)
     python bench.py --stage ple ...        # the PLE tail kernel on its own workload
     python bench.py --stage ple_bwd ...    # the PLE tail's backward on the same workload
     python bench.py --stage owner ...      # the owner-sharded table (NCCL all-to-alls)
@@ -79,14 +82,18 @@ def hbm_peak():
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+    """nvidia-smi clock / throttle-reason samples, every `interval_ms`, from
+    before the warm-up to the end of the last measured pass. Each sample carries
+    nvidia-smi's own timestamp, so the samples inside the timed region can be
+    counted apart (mark_timed records its host-clock bounds)."""
 
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    QUERY = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_id: str, interval_ms: int = 50):
+    def __init__(self, gpu_id: str, interval_ms: int = 10):
         self.gpu_id, self.interval_ms, self.proc = gpu_id, interval_ms, None
+        self.lines, self.timed = [], []
 
     def __enter__(self):
         try:
@@ -94,9 +101,14 @@ class ClockSampler:
                 ["nvidia-smi", f"--id={self.gpu_id}", f"--query-gpu={self.QUERY}",
                  "--format=csv,noheader,nounits", f"-lms={self.interval_ms}"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            time.sleep(0.5)        # let the sampler come up before the measured work
         except OSError:
             self.proc = None
         return self
+
+    def mark_timed(self, t0: float, t1: float):
+        """Host wall-clock bounds (time.time()) of a timed region."""
+        self.timed.append((t0, t1))
 
     def __exit__(self, *exc):
         self.lines = []
@@ -110,23 +122,43 @@ class ClockSampler:
             self.lines = [ln for ln in out.splitlines() if ln.strip()]
         return False
 
+    @staticmethod
+    def _stamp(s: str):
+        import datetime
+        for fmt in ("%Y/%m/%d %H:%M:%S.%f", "%Y/%m/%d %H:%M:%S"):
+            try:
+                return datetime.datetime.strptime(s, fmt).timestamp()
+            except ValueError:
+                pass
+        return None
+
     def summary(self):
-        sm, mx, reasons = [], None, set()
+        sm, mx, reasons, in_timed, sm_timed = [], None, set(), 0, []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in getattr(self, "lines", []):
+        for ln in self.lines:
             f = [x.strip() for x in ln.split(",")]
-            if len(f) < 9:
+            if len(f) < 10:
                 continue
             try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
+                mhz = float(f[2])
+                mx = float(f[3])
             except ValueError:
                 continue
-            for nm, v in zip(names, f[5:9]):
+            sm.append(mhz)
+            ts = self._stamp(f[0])
+            if ts is not None and any(a - 0.02 <= ts <= b + 0.02 for a, b in self.timed):
+                in_timed += 1
+                sm_timed.append(mhz)
+            for nm, v in zip(names, f[6:10]):
                 if v.lower() == "active":
                     reasons.add(nm)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_mhz_min": min(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm),
+                "samples_in_timed_region": in_timed,
+                "sm_mhz_timed_region": statistics.median(sm_timed) if sm_timed else None,
+                "interval_ms": self.interval_ms,
+                "window": "from before the warm-up to the end of the last measured pass"}
 
 
 def gpu_smi_id(torch, device) -> str:
@@ -154,8 +186,10 @@ def source_digest(files) -> str:
 
 def committed_traffic(kernel: str, units: float):
     """DRAM bytes per launch from profiles/dram_traffic.json, scaled to `units`
-    (lookups or tokens), or None if absent or taken on other kernel sources
-    (each record carries the digest of the sources its kernel is built from)."""
+    (lookups or tokens): {"total", "read", "write", "read_overfetch"}, where
+    read_overfetch = DRAM bytes read / algorithmic bytes read. None if absent or
+    taken on other kernel sources (each record carries the digest of the
+    sources its kernel is built from)."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
     try:
         with open(path) as f:
@@ -163,17 +197,98 @@ def committed_traffic(kernel: str, units: float):
         k = rec["kernels"][kernel]
         if k["digest"] != source_digest(k["sources"]):
             return None
-    except (OSError, ValueError, KeyError):
+        out = {"total": k["dram_bytes_per_unit"] * units, "read": None, "write": None,
+               "read_overfetch": None}
+        if "read_bytes_per_unit" in k:
+            out["read"] = k["read_bytes_per_unit"] * units
+            out["write"] = k["write_bytes_per_unit"] * units
+        if k.get("alg_read_bytes_per_unit"):
+            out["read_overfetch"] = k["read_bytes_per_unit"] / k["alg_read_bytes_per_unit"]
+        return out
+    except (OSError, ValueError, KeyError, TypeError):
         return None
-    return k["dram_bytes_per_unit"] * units
+
+
+def traffic_fields(kernel: str, units: float) -> dict:
+    """The roofline's traffic keys for a kernel (nulls when no current record)."""
+    t = committed_traffic(kernel, units)
+    return {"traffic": t["total"] if t else None,
+            "traffic_read": t["read"] if t else None,
+            "traffic_write": t["write"] if t else None,
+            "read_overfetch": t["read_overfetch"] if t else None}
+
+
+# ------------------------------------------------------ host, workload config
+
+def host_info() -> dict:
+    """This host's CPU, as the CPU-baseline figures report it."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.lower().startswith("model name"):
+                    model = ln.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    try:
+        usable = len(os.sched_getaffinity(0))
+    except AttributeError:
+        usable = os.cpu_count()
+    return {"host_nproc": usable, "host_logical_cpus": os.cpu_count(), "cpu_model": model}
+
+
+def head_constants_record(name: str) -> dict:
+    """Where the workload's hash constants come from, with their values."""
+    from workloads import WORKLOADS, constants, head_params
+    w, cfg = WORKLOADS[name], head_params(name)
+    rec = {"multipliers": list(cfg["multipliers"]), "vocab_sizes": list(cfg["vocab_sizes"]),
+           "eos_id": cfg["eos_id"], "fill_id": cfg["fill_id"]}
+    if w.heads == "page":
+        rec["source"] = ("page: multipliers, padded rows and the first 8 vocab sizes and "
+                         "offsets printed; vocab sizes of heads 8-15 inferred (the next 8 "
+                         "consecutive primes), offsets their running sums")
+        rec["printed_heads"] = len(constants.PRINTED_VOCAB_SIZES)
+        rec["inferred_heads"] = len(constants.INFERRED_VOCAB_SIZES)
+    else:
+        rec["source"] = (f"seeded stand-in: 16 distinct primes drawn from "
+                         f"[{w.prime_range[0]}, {w.prime_range[1]}) by NumPy PCG64 seed "
+                         f"{1000 + w.seed}, sorted, offsets their running sums; page multipliers")
+        rec["prime_seed"] = 1000 + w.seed
+    return rec
+
+
+def workload_config(name: str, world: int, stage: str = "forward + backward") -> dict:
+    """The `config` of a bench line: identical on the GPU arm and the reference
+    arm of the same workload and stage."""
+    from workloads import WORKLOADS, head_params, token_stream
+    w, cfg = WORKLOADS[name], head_params(name)
+    T = len(token_stream(name)[0])
+    R = cfg["table_rows"]
+    return {"workload": name, "stage": stage, "tokens_per_step": T,
+            "tokens_per_step_per_gpu": T, "heads": 16, "dim": cfg["dim"], "table_rows": R,
+            "table_dtype": w.dtype,
+            "parallelism": f"replicas x{world} (own table and batch per GPU)",
+            "l2": ("inputs larger than L2 (102.4 GB table; 336 MB out and dout)" if R > 1e8
+                   else "per-step working set vs 126 MB L2: see table_rows"),
+            "input_seed": w.seed, "inputs": w.description,
+            "head_constants": head_constants_record(name)}
 
 
 # ------------------------------------------------------------ CPU oracle leg
 
-def oracle_run(name: str, S: int, reps_seconds: float = 0.0, max_reps: int = 1):
-    """Time the CPU oracle on the first S tokens of a workload: hash, gather from
-    a host table holding the rows those lookups touch (staged untimed), and the
-    row-gradient backward. Returns (tokens/s, seconds, reps, description)."""
+STAGE_NAMES = {"all": "forward + backward", "bwd": "backward only",
+               "hash": "hash only (engram_hash)", "gather": "gather only (engram_gather)"}
+ORACLE_PARTS = {"all": ("hash", "gather", "backward"), "bwd": ("backward",),
+                "hash": ("hash",), "gather": ("gather",)}
+
+
+def oracle_run(name: str, S: int, reps_seconds: float = 0.0, max_reps: int = 1,
+               parts=("hash", "gather", "backward")):
+    """Time the CPU oracle on the first S tokens of a workload (S is capped at
+    the workload's length): the named parts of hash, gather from a host table
+    holding the rows those lookups touch (staged untimed), and the row-gradient
+    backward. Returns (tokens/s, seconds, reps, description, tokens per rep)."""
     import torch
     import oracle
     from workloads import WORKLOADS, head_params, host_dout, token_stream
@@ -192,69 +307,93 @@ def oracle_run(name: str, S: int, reps_seconds: float = 0.0, max_reps: int = 1):
     esize = 4 if w.dtype == "f32" else 2
     compact = rng.integers(0, 2 ** 16, size=(len(uniq), D * esize // 2), dtype=np.uint16)
     remap = np.searchsorted(uniq, idx0.reshape(-1))
-    dout = host_dout(name, S * H, D, w.dtype)
-    dout_raw = dout.numpy() if w.dtype == "f32" else \
-        dout.view(torch.int16).numpy().view(np.uint16)
+    dout_raw = None
+    if "backward" in parts:
+        dout = host_dout(name, S * H, D, w.dtype)
+        dout_raw = dout.numpy() if w.dtype == "f32" else \
+            dout.view(torch.int16).numpy().view(np.uint16)
     code = oracle.F32 if w.dtype == "f32" else oracle.BF16
     oracle.lib()
     reps, t0 = 0, time.perf_counter()
     while True:
-        idx = oracle.hash_ids(ids, cu, cfg)
-        out = oracle.gather(compact, remap)
-        u, g = oracle.backward(idx.reshape(-1), dout_raw, code)
+        idx = oracle.hash_ids(ids, cu, cfg) if "hash" in parts else idx0
+        if "gather" in parts:
+            out = oracle.gather(compact, remap)
+            assert out.shape[0] == S * H
+        if "backward" in parts:
+            u, _ = oracle.backward(idx.reshape(-1), dout_raw, code)
+            assert len(u) == len(uniq)
         reps += 1
         el = time.perf_counter() - t0
         if reps >= max_reps or el >= reps_seconds:
             break
-    assert out.shape[0] == S * H and len(u) == len(uniq)
+    what = " + ".join(parts)
     desc = (f"first {S} of {len(token_stream(name)[0])} tokens of workload '{name}' "
-            f"x {reps} rep(s); gather from a host table of the {len(uniq)} rows the "
-            f"sample touches (staged before timing); single-threaded C oracle")
-    return S * reps / el, el, reps, desc
+            f"x {reps} rep(s), timed: {what}"
+            + ("; gather from a host table of the "
+               f"{len(uniq)} rows the sample touches (staged before timing)"
+               if "gather" in parts else "")
+            + "; single-threaded C oracle")
+    return S * reps / el, el, reps, desc, S
 
 
 def run_reference(args):
-    """--impl reference: the oracle, as it stands, on this host's cores."""
+    """--impl reference: the oracle, as it stands, on this host's cores, on the
+    GPU arm's metric, unit and config. Each step times a bounded sample of the
+    step's work (the whole step when it fits the time budget); value = units
+    processed / time, and ms_per_step = the time one whole step takes at that
+    rate."""
     rank, _, world = rank_env()
     if rank != 0:
         return 0
-    name = args.workload
-    ple, adam = args.stage in ("ple", "ple_bwd"), args.stage == "adam"
-    ple_bwd = args.stage == "ple_bwd"
-    if adam:
-        run = adam_oracle_run
-    elif ple:
-        run = lambda S: ple_oracle_run(S, backward=ple_bwd)  # noqa: E731
+    name, stage = args.workload, args.stage
+    if stage == "adam":
+        run, small, unit = adam_oracle_run, 2048, "rows/s"
+        full = args.adam_touched
+        config, metric, dtype = adam_config(args.adam_rows, args.adam_touched), ADAM_METRIC, "f64"
+    elif stage in ("ple", "ple_bwd"):
+        bwd = stage == "ple_bwd"
+        run = lambda S: ple_oracle_run(S, backward=bwd)  # noqa: E731
+        small, unit = 256, UNIT
+        config = ple_config(args, world, bwd)
+        full = config["tokens_per_step_per_gpu"]
+        metric, dtype = (PLE_BWD_METRIC if bwd else PLE_METRIC), "f64"
+    elif stage in ORACLE_PARTS:
+        parts = ORACLE_PARTS[stage]
+        run = lambda S: oracle_run(name, S, parts=parts)  # noqa: E731
+        small, unit = 4096, UNIT
+        config = workload_config(name, world, STAGE_NAMES[stage])
+        full = config["tokens_per_step"]
+        metric, dtype = STAGE_METRICS.get(stage, METRIC), "int64/f64"
     else:
-        run = lambda S: oracle_run(name, S)  # noqa: E731
-    # calibrate, then size each step's sample so W + K steps take ~2 minutes
-    rate, _, _, _ = run(256 if ple else 4096)
+        print(json.dumps({"impl": "reference", "unavailable":
+                          f"stage {stage} has no oracle arm (its exchanges need several ranks)"}))
+        return 0
+    # calibrate, then size each step's sample so W + K steps take about the budget
+    rate = run(small)[0]
     budget = float(os.environ.get("ENGRAM_REFERENCE_BUDGET_S", "120"))
-    S = int(max(256, min(65536 * 4, rate * budget / max(1, args.steps + args.warmup))))
+    S = int(max(small, min(full, rate * budget / max(1, args.steps + args.warmup))))
     for _ in range(args.warmup):
         run(S)
-    times = []
+    times, desc, done = [], "", 0
     for _ in range(args.steps):
-        _, el, _, desc = run(S)
+        _, el, _, desc, got = run(S)
         times.append(el)
+        done += got
     total = sum(times)
-    value = S * len(times) / total
-    if ple:
-        name = "ple_full_bwd" if ple_bwd else "ple_full"
-    if adam:
-        name = "adam_shard"
-    metric = (ADAM_METRIC if adam else PLE_BWD_METRIC if ple_bwd else PLE_METRIC if ple
-              else METRIC)
+    value = done / total
+    cores = 1
     line = {
-        "impl": "reference", "metric": metric,
-        "value": value, "unit": "rows/s" if adam else UNIT,
+        "impl": "reference", "metric": metric, "value": value, "unit": unit,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": 1e3 * total / len(times), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64" if ple or adam else "int64/f64",
-        "data": "synthetic", "config": {"workload": name, "tokens_per_step": S},
-        "cpu_baseline": {"value": value, "unit": "rows/s" if adam else UNIT, "cores": 1,
-                         "kind": "oracle", "sample": desc},
-        "e2e": {"value": value, "unit": "rows/s" if adam else UNIT, "h2d_bytes_per_step": 0,
+        "ms_per_step": 1e3 * full / value, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": dtype, "data": "synthetic",
+        "config": config,
+        "sample_per_step": {"units": done // len(times), "of": full,
+                            "ms": 1e3 * total / len(times)},
+        "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
+                         "sample": desc, **host_info()},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -263,7 +402,21 @@ def run_reference(args):
 
 # ------------------------------------------------------------------- GPU leg
 
+STAGE_METRICS = {
+    "hash": ("Engram hash tokens/s (engram_hash alone: raw token IDs to 16 head row "
+             "indices per token); achieved HBM GB/s vs peak"),
+    "gather": ("Engram gather tokens/s (engram_gather alone: 16 row lookups of 160 bf16 "
+               "per token from the hash's indices); achieved HBM GB/s vs peak"),
+}
+L2_FLUSH_BYTES = 256 << 20     # twice the B200's 126 MB L2
+
+
 def run_ours(args):
+    """The GPU arm. --stage all (default): the step = engram_hash_gather +
+    engram_backward_sort + engram_backward_reduce, captured once as a CUDA
+    graph and replayed; bwd: the backward alone; hash / gather: engram_hash or
+    engram_gather alone, each launch timed by its own events (the hash's
+    working set fits in L2, so L2 is flushed between its launches)."""
     import torch
     import torch.distributed as dist
 
@@ -279,6 +432,7 @@ def run_ours(args):
         dist.init_process_group("nccl", device_id=device,
                                 timeout=datetime.timedelta(seconds=300))
 
+    stage = args.stage
     name = args.workload
     w = WORKLOADS[name]
     cfg = head_params(name)
@@ -288,34 +442,41 @@ def run_ours(args):
     n = T * H
     tdtype = {"bf16": torch.bfloat16, "f32": torch.float32}[w.dtype]
     esize = 2 if w.dtype == "bf16" else 4
+    fwd, bwd = stage == "all", stage in ("all", "bwd")
+    gathers = stage in ("all", "gather")
 
-    # inputs resident in HBM; two sets of per-step buffers for the e2e pipeline
-    fwd = args.stage == "all"
     table = None
-    if fwd:
+    if gathers:
         table = torch.empty(R, D, dtype=tdtype, device=device)
         fill_device_table(table, w.seed)
-    dout_h = host_dout(name, n, D, w.dtype).pin_memory()
-    ws = torch.empty(E.engram_backward_workspace_size(n, R, D), dtype=torch.uint8,
-                     device=device)
-    nbuf = 2 if fwd else 1
+    dout_h = host_dout(name, n, D, w.dtype).pin_memory() if bwd else None
+    ws = (torch.empty(E.engram_backward_workspace_size(n, R, D), dtype=torch.uint8,
+                      device=device) if bwd else None)
+    flush = (torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+             if stage == "hash" else None)
     bufs = [{
         "ids": torch.from_numpy(ids_np.copy()).to(device),
         "cu": torch.from_numpy(cu_np.copy()).to(device),
-        "dout": dout_h.to(device),
-        "out": torch.empty(T, H * D, dtype=tdtype, device=device) if fwd else None,
+        "dout": dout_h.to(device) if bwd else None,
+        "out": torch.empty(T, H * D, dtype=tdtype, device=device) if gathers else None,
         "idx": torch.empty(T, H, dtype=torch.int32, device=device),
-        "uniq": torch.empty(n, dtype=torch.int32, device=device),
-        "grads": torch.empty(n, D, dtype=torch.float32, device=device),
+        "uniq": torch.empty(n, dtype=torch.int32, device=device) if bwd else None,
+        "grads": torch.empty(n, D, dtype=torch.float32, device=device) if bwd else None,
         "nu": torch.empty(1, dtype=torch.int32, device=device),
-    } for _ in range(nbuf)]
+    } for _ in range(2)]
     stream = torch.cuda.Stream(device)
-    if not fwd:  # backward alone: the indices come from the hash, no table needed
-        E.engram_hash(params, bufs[0]["ids"], bufs[0]["cu"], out_idx=bufs[0]["idx"],
-                      stream=stream)
+    if not fwd:   # the backward and the gather alone take the hash's indices
+        for b in bufs:
+            E.engram_hash(params, b["ids"], b["cu"], out_idx=b["idx"], stream=stream)
 
     def step(ev=None, b=None):
         b = bufs[0] if b is None else b
+        if stage == "hash":
+            E.engram_hash(params, b["ids"], b["cu"], out_idx=b["idx"], stream=stream)
+            return
+        if stage == "gather":
+            E.engram_gather(table, b["idx"].view(-1), out=b["out"].view(n, D), stream=stream)
+            return
         if ev is not None:
             ev[0].record(stream)
         if fwd:
@@ -330,116 +491,154 @@ def run_ours(args):
                                  stream=stream)
         if ev is not None:
             ev[3].record(stream)
-    nu = bufs[0]["nu"]
 
+    def flush_l2():
+        if flush is not None:
+            with torch.cuda.stream(stream):
+                flush.fill_(1)
+
+    clk = ClockSampler(gpu_smi_id(torch, device))
+    clk.__enter__()
     for _ in range(args.warmup):
+        flush_l2()
         step()
     torch.cuda.synchronize(device)
     if E.engram_get_device_error(stream):
         raise RuntimeError("device error flag set during warm-up")
-    U = int(nu.item())
+    U = int(bufs[0]["nu"].item()) if bwd else None
 
     K = args.steps
-    # the timed steps: one step captured as a CUDA graph and replayed (the
-    # library's calls need no host synchronisation), or eager launches
-    if args.graph:
-        graph = torch.cuda.CUDAGraph()
-        c0 = E.engram_launch_count()
-        with torch.cuda.graph(graph, stream=stream):
+    per_launch = stage in ("hash", "gather")
+    graph, launches_per_step = None, None
+    if per_launch:
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(K)]
+        launches0 = E.engram_launch_count()
+        barrier(device)
+        torch.cuda.synchronize(device)
+        h0 = time.time()
+        for e in evs:
+            flush_l2()
+            e[0].record(stream)
             step()
-        launches_per_step = E.engram_launch_count() - c0
-
-        def timed_step():
-            with torch.cuda.stream(stream):
-                graph.replay()
+            e[1].record(stream)
+        torch.cuda.synchronize(device)
+        clk.mark_timed(h0, time.time())
+        barrier(device)
+        launches = E.engram_launch_count() - launches0
+        per = [e[0].elapsed_time(e[1]) for e in evs]
+        local_ms = sum(per)
+        timed_as = ("sum of per-launch CUDA-event times, eager launches"
+                    + ("; L2 flushed by a 256 MB write between launches (not timed)"
+                       if flush is not None else "; inputs larger than L2"))
     else:
-        graph, launches_per_step, timed_step = None, None, step
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    timed_step()                       # first replay uploads the graph
-    torch.cuda.synchronize(device)
-    launches0 = E.engram_launch_count()
-    barrier(device)
-    torch.cuda.synchronize(device)
-    with ClockSampler(gpu_smi_id(torch, device)) as clk:
+        # one step captured as a CUDA graph and replayed (the library's calls
+        # need no host synchronisation), or eager launches
+        if args.graph:
+            graph = torch.cuda.CUDAGraph()
+            c0 = E.engram_launch_count()
+            with torch.cuda.graph(graph, stream=stream):
+                step()
+            launches_per_step = E.engram_launch_count() - c0
+
+            def timed_step():
+                with torch.cuda.stream(stream):
+                    graph.replay()
+        else:
+            timed_step = step
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        timed_step()                       # first replay uploads the graph
+        torch.cuda.synchronize(device)
+        launches0 = E.engram_launch_count()
+        barrier(device)
+        torch.cuda.synchronize(device)
+        h0 = time.time()
         t_start.record(stream)
         for k in range(K):
             timed_step()
         t_end.record(stream)
         torch.cuda.synchronize(device)
-    barrier(device)
-    launches = (launches_per_step * K if args.graph
-                else E.engram_launch_count() - launches0)
-    local_ms = t_start.elapsed_time(t_end)
+        clk.mark_timed(h0, time.time())
+        barrier(device)
+        launches = (launches_per_step * K if args.graph
+                    else E.engram_launch_count() - launches0)
+        local_ms = t_start.elapsed_time(t_end)
+        per = None
+        timed_as = ("CUDA graph of one step, replayed" if args.graph else "eager launches")
     total_ms = max_over_ranks(local_ms, device)
-    # per-stage times: a separate eager pass with events between the stages
-    # (kept out of the timed steps above)
-    KS = max(1, min(K, 50))
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(KS)]
-    for k in range(KS):
-        step(evs[k])
-    torch.cuda.synchronize(device)
-    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
-    sort_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
-    red_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+
+    # per-stage times of the step: a separate eager pass with events between
+    # the stages (kept out of the timed steps above)
+    if not per_launch:
+        KS = max(1, min(K, 50))
+        sevs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(KS)]
+        for k in range(KS):
+            step(sevs[k])
+        torch.cuda.synchronize(device)
+        fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in sevs)
+        sort_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in sevs)
+        red_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in sevs)
 
     # ---- end to end through the public API with host buffers: every step
-    # copies its inputs in from pinned host memory and its results out. Three
-    # streams pipeline consecutive steps (copy-in, compute, copy-out, with two
-    # sets of device buffers), so step k's results travel to the host while
-    # step k+1 computes and PCIe carries both directions at once.
-    def run_e2e(full_readback: bool):
-        """End to end through the public API with host buffers: every step
-        copies its inputs (ids, cu_seqlens, dout) in from pinned host memory
-        and reads its result back: num_unique (the step's metric) or, with
-        full_readback, also out, uniq_rows[:U] and row_grads[:U]. Three
-        streams pipeline consecutive steps (copy-in, compute, copy-out, two
-        sets of device buffers)."""
+    # copies its inputs in from pinned host memory and its results back out.
+    # Three streams pipeline consecutive steps (copy-in, compute, copy-out,
+    # two sets of device buffers), so step k's results travel to the host
+    # while step k+1 computes and PCIe carries both directions at once.
+    in_names = {"all": ["ids", "cu", "dout"], "bwd": ["idx", "dout"],
+                "hash": ["ids", "cu"], "gather": ["idx"]}[stage]
+    out_fixed = {"all": ["out", "nu"], "bwd": ["nu"], "hash": ["idx"], "gather": ["out"]}[stage]
+
+    def run_e2e(resident_rows: bool):
+        """resident_rows (stage all only): read back num_unique alone and leave
+        out and the row gradients on the device."""
         e2e_steps = max(1, min(K, args.e2e_steps))
-        ids_h = torch.from_numpy(ids_np.copy()).pin_memory()
-        cu_h = torch.from_numpy(cu_np.copy()).pin_memory()
-        host = [{"out": torch.empty(T, H * D, dtype=tdtype).pin_memory() if full_readback
-                 else None,
-                 "uniq": torch.empty(n, dtype=torch.int32).pin_memory() if full_readback
-                 else None,
-                 "grads": torch.empty(n, D, dtype=torch.float32).pin_memory() if full_readback
-                 else None,
-                 "nu": torch.empty(1, dtype=torch.int32).pin_memory()} for _ in range(2)]
+        src = {"ids": torch.from_numpy(ids_np.copy()), "cu": torch.from_numpy(cu_np.copy()),
+               "dout": dout_h, "idx": bufs[0]["idx"].cpu()}
+        host_in = {k: src[k] if src[k].is_pinned() else src[k].pin_memory() for k in in_names}
+        outs = ["nu"] if resident_rows else out_fixed
+        host = [{k: torch.empty_like(bufs[0][k], device="cpu").pin_memory() for k in outs}
+                for _ in range(2)]
+        if bwd and not resident_rows:
+            for hb in host:
+                hb["uniq"] = torch.empty(n, dtype=torch.int32).pin_memory()
+                hb["grads"] = torch.empty(n, D, dtype=torch.float32).pin_memory()
         s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
         ev = lambda: torch.cuda.Event()  # noqa: E731
         in_done = [ev() for _ in range(e2e_steps)]
         comp_done = [ev() for _ in range(e2e_steps)]
-        nu_done = [ev() for _ in range(e2e_steps)]
+        fixed_done = [ev() for _ in range(e2e_steps)]
         out_done = [ev() for _ in range(e2e_steps)]
-        h2d = ids_h.numel() * 4 + cu_h.numel() * 4 + dout_h.numel() * esize
-        d2h_bytes = [4] * e2e_steps
+        h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+        d2h_bytes = [0] * e2e_steps
 
         def drain(k):
-            # rows of step k: the host needs num_unique before copying them out
-            nu_done[k].synchronize()
-            if not full_readback:
-                with torch.cuda.stream(s_out):
-                    out_done[k].record(s_out)
-                return
+            # step k's rows: the host needs num_unique before copying them out
             hb, b = host[k % 2], bufs[k % 2]
-            u = int(hb["nu"].item())
+            d2h = sum(hb[x].numel() * hb[x].element_size() for x in outs)
+            if bwd and not resident_rows:
+                fixed_done[k].synchronize()
+                u = int(hb["nu"].item())
+                with torch.cuda.stream(s_out):
+                    hb["uniq"][:u].copy_(b["uniq"][:u], non_blocking=True)
+                    hb["grads"][:u].copy_(b["grads"][:u], non_blocking=True)
+                d2h += u * 4 + u * D * 4
             with torch.cuda.stream(s_out):
-                hb["uniq"][:u].copy_(b["uniq"][:u], non_blocking=True)
-                hb["grads"][:u].copy_(b["grads"][:u], non_blocking=True)
                 out_done[k].record(s_out)
-            d2h_bytes[k] = hb["out"].numel() * esize + 4 + u * 4 + u * D * 4
+            d2h_bytes[k] = d2h
 
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         barrier(device)
         torch.cuda.synchronize(device)
+        h0 = time.time()
         e0.record(s_in)
         for k in range(e2e_steps):
             b, hb = bufs[k % 2], host[k % 2]
             with torch.cuda.stream(s_in):
                 if k >= 2:
                     s_in.wait_event(comp_done[k - 2])  # inputs of buffer set k%2 free
-                b["ids"].copy_(ids_h, non_blocking=True)
-                b["cu"].copy_(cu_h, non_blocking=True)
-                b["dout"].copy_(dout_h, non_blocking=True)
+                for x in in_names:
+                    b[x].copy_(host_in[x], non_blocking=True)
                 in_done[k].record(s_in)
             stream.wait_event(in_done[k])
             if k >= 2:
@@ -448,29 +647,27 @@ def run_ours(args):
             comp_done[k].record(stream)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(comp_done[k])
-                if full_readback:
-                    hb["out"].copy_(b["out"], non_blocking=True)
-                hb["nu"].copy_(b["nu"], non_blocking=True)
-                nu_done[k].record(s_out)
+                for x in outs:
+                    hb[x].copy_(b[x], non_blocking=True)
+                fixed_done[k].record(s_out)
             if k >= 1:
                 drain(k - 1)
         drain(e2e_steps - 1)
         e1.record(s_out)
         torch.cuda.synchronize(device)
+        clk.mark_timed(h0, time.time())
         e2e_ms = max_over_ranks(e0.elapsed_time(e1), device)
         barrier(device)
+        rb = outs + (["uniq_rows[:U]", "row_grads[:U]"] if bwd and not resident_rows else [])
         return {"value": world * T * e2e_steps / (e2e_ms / 1e3), "unit": UNIT,
                 "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": int(statistics.mean(d2h_bytes)),
-                "steps": e2e_steps,
-                "readback": "out, uniq_rows[:U], row_grads[:U], num_unique" if full_readback
-                else "num_unique (the step's metric; out and the row gradients stay resident)",
+                "steps": e2e_steps, "inputs": in_names, "readback": rb,
                 "pipeline": "copy-in / compute / copy-out streams, two buffer sets"}
 
-    e2e = e2e_full = None
-    if fwd:
-        e2e = run_e2e(False)
-        e2e_full = run_e2e(True)
+    e2e = run_e2e(False)
+    e2e_resident = run_e2e(True) if fwd else None
+    clk.__exit__(None, None, None)
 
     if E.engram_get_device_error(stream):
         raise RuntimeError("device error flag set during timing")
@@ -479,61 +676,63 @@ def run_ours(args):
     value = world * T * K / (total_ms / 1e3)
     peak, peak_kind = hbm_peak()
     fwd_bytes = T * (4 + 2 * H * D * esize + H * 4)
-    red_bytes = n * D * esize + U * (4 + D * 4)
-    bwd_bytes = n * 4 + red_bytes
-    stages = {
-        "fwd_hash_gather": {"ms": fwd_ms, "alg_bytes": fwd_bytes,
-                            "gbs": fwd_bytes / max(fwd_ms, 1e-9) / 1e6,
-                            "frac": fwd_bytes / max(fwd_ms, 1e-9) / 1e6 / peak},
-        "bwd_sort": {"ms": sort_ms, "kernels": None},
-        "bwd_reduce": {"ms": red_ms, "alg_bytes": red_bytes,
-                       "gbs": red_bytes / red_ms / 1e6,
-                       "frac": red_bytes / red_ms / 1e6 / peak},
-        "bwd_total": {"ms": sort_ms + red_ms, "alg_bytes": bwd_bytes,
-                      "gbs": bwd_bytes / (sort_ms + red_ms) / 1e6,
-                      "frac": bwd_bytes / (sort_ms + red_ms) / 1e6 / peak},
-        "num_unique": U,
-    }
-    # dominant kernel: the fused forward unless the reduce stage takes longer
-    if fwd and fwd_ms >= red_ms:
-        dom, dom_ms, dom_bytes, tkey, tunits = ("hash_gather_kernel", fwd_ms, fwd_bytes,
-                                               "hash_gather_kernel", T)
+    hash_bytes = T * (4 + H * 4) + cu_np.size * 4
+    gather_bytes = n * (4 + 2 * D * esize)
+    stages = {}
+    if per_launch:
+        kname = "hash_kernel<3, 8>" if stage == "hash" else "gather_kernel<20>"
+        dom_bytes = hash_bytes if stage == "hash" else gather_bytes
+        dom_ms = statistics.mean(per)
+        stages[stage] = {"ms": dom_ms, "ms_min": min(per), "ms_max": max(per),
+                         "alg_bytes": dom_bytes, "gbs": dom_bytes / dom_ms / 1e6,
+                         "frac": dom_bytes / dom_ms / 1e6 / peak}
+        dom, tkey, tunits = kname, kname.split("<")[0], (T if stage == "hash" else n)
     else:
-        dom, dom_ms, dom_bytes, tkey, tunits = ("segment reduce stage (seg_count + seg_reduce "
-                                               "+ seg_fixup; seg_reduce dominates)", red_ms,
-                                               red_bytes, "seg_reduce", n)
-    if not fwd:
-        stages.pop("fwd_hash_gather")
+        red_bytes = n * D * esize + U * (4 + D * 4)
+        bwd_bytes = n * 4 + red_bytes
+        if fwd:
+            stages["fwd_hash_gather"] = {"ms": fwd_ms, "alg_bytes": fwd_bytes,
+                                         "gbs": fwd_bytes / max(fwd_ms, 1e-9) / 1e6,
+                                         "frac": fwd_bytes / max(fwd_ms, 1e-9) / 1e6 / peak}
+        stages["bwd_sort"] = {"ms": sort_ms}
+        stages["bwd_reduce"] = {"ms": red_ms, "alg_bytes": red_bytes,
+                                "gbs": red_bytes / red_ms / 1e6,
+                                "frac": red_bytes / red_ms / 1e6 / peak}
+        stages["bwd_total"] = {"ms": sort_ms + red_ms, "alg_bytes": bwd_bytes,
+                               "gbs": bwd_bytes / (sort_ms + red_ms) / 1e6,
+                               "frac": bwd_bytes / (sort_ms + red_ms) / 1e6 / peak}
+        stages["num_unique"] = U
+        # dominant kernel: the fused forward unless the reduce stage takes longer
+        if fwd and fwd_ms >= red_ms:
+            dom, dom_ms, dom_bytes, tkey, tunits = ("hash_gather_kernel<3, 8, 20>", fwd_ms,
+                                                   fwd_bytes, "hash_gather_kernel", T)
+        else:
+            dom, dom_ms, dom_bytes, tkey, tunits = (
+                "segment reduce stage (seg_count + seg_reduce + seg_fixup; seg_reduce "
+                "dominates)", red_ms, red_bytes, "seg_reduce", n)
     achieved = dom_bytes / dom_ms / 1e6
-    clocks = clk.summary()
+    config = workload_config(name, world, STAGE_NAMES[stage])
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
-        "warmup": args.warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-        "config": {"workload": name, "stage": "forward + backward" if fwd else "backward only",
-                   "timed_as": "CUDA graph of one step, replayed" if args.graph
-                   else "eager launches",
-                   "tokens_per_step_per_gpu": T, "heads": H, "dim": D,
-                   "table_rows": R, "table_dtype": w.dtype, "num_unique": U,
-                   "parallelism": f"replicas x{world} (own table and batch per GPU)",
-                   "l2": "inputs larger than L2 (102.4 GB table; 336 MB out and dout)"
-                   if R > 1e8 else "per-step working set vs 126 MB L2: see table_rows",
-                   "head_constants": "page" if w.heads == "page" else "seeded primes"},
+        "metric": STAGE_METRICS.get(stage, METRIC), "value": value, "unit": UNIT,
+        "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": total_ms / K,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic", "config": config, "timed_as": timed_as,
         "roofline": {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": committed_traffic(tkey, tunits)},
+                     "alg_bytes_per_launch": dom_bytes, **traffic_fields(tkey, tunits)},
         "stages": stages,
         "e2e": e2e,
-        "e2e_full_readback": e2e_full,
+        "e2e_resident_outputs": e2e_resident,
         "gpu_launches": launches,
-        "clocks": clocks,
     }
-    if world == 1 and fwd and not args.no_cpu_baseline:
-        v, el, reps, desc = oracle_run(name, T, reps_seconds=args.cpu_seconds, max_reps=8)
+    if world == 1 and not args.no_cpu_baseline:
+        v, el, reps, desc, _ = oracle_run(name, T, reps_seconds=args.cpu_seconds, max_reps=8,
+                                          parts=ORACLE_PARTS[stage])
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
-                                "sample": desc, "seconds": el}
+                                "sample": desc, "seconds": el, **host_info()}
     else:
         line["cpu_baseline"] = None
+    line["clocks"] = clk.summary()
     if rank == 0:
         print(json.dumps(line), flush=True)
     graph = None  # no graph outlives the process group
@@ -582,7 +781,39 @@ def ple_oracle_run(S: int, reps_seconds: float = 0.0, max_reps: int = 1,
     desc = (f"{S} tokens x {s.channels} channels (one sequence, the page's 4 x 2,560 "
             f"branches, kernel {s.kernel}, dilation {s.dilation}) x {reps} rep(s); "
             f"single-threaded C oracle in fp64{' (backward)' if backward else ''}")
-    return S * reps / el, el, reps, desc
+    return S * reps / el, el, reps, desc, S
+
+
+def ple_shape(args):
+    """(shape, tokens, rows) of the PLE stages: the full workload's batch, or
+    --ple-tokens worth of whole 4,096-token rows."""
+    from workloads import PLE_SHAPES
+    s = PLE_SHAPES["ple_full"]
+    batch = max(1, args.ple_tokens // s.seq_len) if args.ple_tokens else s.batch
+    return s, batch * s.seq_len, batch
+
+
+def ple_config(args, world: int, backward: bool) -> dict:
+    """`config` of the PLE stages, identical on both arms."""
+    s, T, batch = ple_shape(args)
+    C = s.channels
+    return {"workload": "ple_full_bwd" if backward else "ple_full",
+            "tokens_per_step": T, "tokens_per_step_per_gpu": T, "channels": C,
+            "branches": s.branches, "group": s.group, "kernel": s.kernel,
+            "dilation": s.dilation, "flags": "norm + silu + residual",
+            "cu_seqlens": f"{batch} rows", "input_seed": 5000 + s.seed,
+            "parallelism": f"replicas x{world} (own batch per GPU)",
+            "l2": (f"inputs larger than L2 ({T * C * 2 * (2 if backward else 1) / 1e9:.2f} "
+                   f"GB in, {T * C * 2 / 1e9:.2f} GB out)")}
+
+
+def adam_config(R: int, U: int) -> dict:
+    """`config` of the optimizer stage, identical on both arms."""
+    return {"workload": "adam_shard" if (R, U) == (ADAM_ROWS, ADAM_TOUCHED)
+            else f"adam_{R}x{ADAM_DIM}_touch{U}", "table_rows": R, "dim": ADAM_DIM,
+            "touched_rows": U, "table_dtype": "bf16", "moments": "f32", "lr": 1e-3,
+            "weight_decay": 0.01,
+            "l2": "inputs larger than L2 (12.8 GB table, 51.2 GB moments, random rows)"}
 
 
 def run_ple(args, backward: bool = False):
@@ -593,7 +824,7 @@ def run_ple(args, backward: bool = False):
     import torch
 
     import hashed_gram_embedding_raw_b200 as E
-    from workloads import PLE_SHAPES, ple_inputs, row_bounds
+    from workloads import ple_inputs, row_bounds
 
     rank, local_rank, world = rank_env()
     assert torch.cuda.is_available(), "bench.py needs a CUDA device"
@@ -604,12 +835,8 @@ def run_ple(args, backward: bool = False):
         import torch.distributed as dist
         dist.init_process_group("nccl", device_id=device,
                                 timeout=datetime.timedelta(seconds=300))
-    s = PLE_SHAPES["ple_full"]
-    T, C, G, K, d = s.tokens, s.channels, s.group, s.kernel, s.dilation
-    batch = s.batch
-    if args.ple_tokens:      # a smaller case of the same shape (whole rows), for profiling
-        batch = max(1, args.ple_tokens // s.seq_len)
-        T = batch * s.seq_len
+    s, T, batch = ple_shape(args)
+    C, G, K, d = s.channels, s.group, s.kernel, s.dilation
     g = torch.Generator(device=device).manual_seed(5000 + s.seed)
     x = torch.randn((T, C), generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
     _, nw_h, w_h, b_h = ple_inputs(1, C, K, s.seed, s.dtype)
@@ -638,6 +865,8 @@ def run_ple(args, backward: bool = False):
             E.engram_ple_short_conv(xx, w, dilation=d, group_size=G, cu_seqlens=cu,
                                     norm_weight=nw, conv_bias=b, out=oo, stream=stream)
 
+    clk = ClockSampler(gpu_smi_id(torch, device))
+    clk.__enter__()
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(device)
@@ -649,12 +878,13 @@ def run_ple(args, backward: bool = False):
     launches0 = E.engram_launch_count()
     barrier(device)
     torch.cuda.synchronize(device)
-    with ClockSampler(gpu_smi_id(torch, device)) as clk:
-        for e in evs:
-            e[0].record(stream)
-            step()
-            e[1].record(stream)
-        torch.cuda.synchronize(device)
+    h0 = time.time()
+    for e in evs:
+        e[0].record(stream)
+        step()
+        e[1].record(stream)
+    torch.cuda.synchronize(device)
+    clk.mark_timed(h0, time.time())
     barrier(device)
     launches = E.engram_launch_count() - launches0
     per = [e[0].elapsed_time(e[1]) for e in evs]
@@ -662,12 +892,14 @@ def run_ple(args, backward: bool = False):
     kern_ms = statistics.mean(per)
 
     # end to end through the public call with host buffers: x (and dout) in
-    # from pinned memory, out (dx) back, copy-in / compute / copy-out overlapped
-    # on three streams
+    # from pinned memory, out (dx and the weight gradients) back, copy-in /
+    # compute / copy-out overlapped on three streams
     e2e_steps = max(1, min(Ksteps, args.e2e_steps))
     x_h = x.cpu().pin_memory()
     g_h = dout.cpu().pin_memory() if backward else None
     out_h = [torch.empty_like(x_h).pin_memory() for _ in range(2)]
+    wg_d = [dnw, dw, db] if backward else []
+    wg_h = [[torch.empty_like(t, device="cpu").pin_memory() for t in wg_d] for _ in range(2)]
     xd = [x, torch.empty_like(x)]
     gd = [dout, torch.empty_like(dout)] if backward else [None, None]
     od = [out, torch.empty_like(out)]
@@ -678,6 +910,7 @@ def run_ple(args, backward: bool = False):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(device)
     torch.cuda.synchronize(device)
+    h0 = time.time()
     e0.record(s_in)
     for k in range(e2e_steps):
         with torch.cuda.stream(s_in):
@@ -695,9 +928,13 @@ def run_ple(args, backward: bool = False):
         with torch.cuda.stream(s_out):
             s_out.wait_event(comp_done[k])
             out_h[k % 2].copy_(od[k % 2], non_blocking=True)
+            for hh, dd in zip(wg_h[k % 2], wg_d):
+                hh.copy_(dd, non_blocking=True)
             out_done[k].record(s_out)
     e1.record(s_out)
     torch.cuda.synchronize(device)
+    clk.mark_timed(h0, time.time())
+    clk.__exit__(None, None, None)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), device)
     if E.engram_get_device_error(stream):
         raise RuntimeError("device error flag set during timing")
@@ -718,35 +955,31 @@ def run_ple(args, backward: bool = False):
         "n_gpus": world, "steps": Ksteps, "warmup": args.warmup,
         "ms_per_step": total_ms / Ksteps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": "ple_full_bwd" if backward else "ple_full",
-                   "tokens_per_step_per_gpu": T, "channels": C,
-                   "branches": s.branches, "group": G, "kernel": K, "dilation": d,
-                   "flags": "norm + silu + residual", "cu_seqlens": f"{batch} rows",
-                   "l2": (f"inputs larger than L2 ({T * C * 2 * (2 if backward else 1) / 1e9:.2f} "
-                          f"GB in, {T * C * 2 / 1e9:.2f} GB out)")},
+        "config": ple_config(args, world, backward),
+        "timed_as": "per-launch CUDA events, eager launches back to back",
         "roofline": {"kernel": kname, "bound": "hbm",
                      "achieved": achieved, "peak": peak, "peak_kind": peak_kind,
                      "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": committed_traffic(tname, T)},
+                     "alg_bytes_per_launch": alg, **traffic_fields(tname, T)},
         "stages": {("ple_short_conv_backward" if backward else "ple_short_conv"): {
             "ms": kern_ms, "alg_bytes": alg, "gbs": achieved, "frac": achieved / peak,
             "ms_min": min(per), "ms_max": max(per)}},
         "e2e": {"value": world * T * e2e_steps / (e2e_ms / 1e3), "unit": UNIT,
                 "h2d_bytes_per_step": x_h.numel() * 2 * (2 if backward else 1),
-                "d2h_bytes_per_step": x_h.numel() * 2,
+                "d2h_bytes_per_step": x_h.numel() * 2 + sum(t.numel() * 4 for t in wg_d),
                 "steps": e2e_steps,
                 "pipeline": "copy-in / compute / copy-out streams, two buffer sets"},
         "gpu_launches": launches,
-        "clocks": clk.summary(),
     }
     if world == 1 and not args.no_cpu_baseline:
-        rate, _, _, _ = ple_oracle_run(256, backward=backward)
+        rate = ple_oracle_run(256, backward=backward)[0]
         S = int(max(256, min(16384, rate * args.cpu_seconds)))
-        v, el, reps, desc = ple_oracle_run(S, backward=backward)
+        v, el, reps, desc, _ = ple_oracle_run(S, backward=backward)
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
-                                "sample": desc, "seconds": el}
+                                "sample": desc, "seconds": el, **host_info()}
     else:
         line["cpu_baseline"] = None
+    line["clocks"] = clk.summary()
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -786,7 +1019,7 @@ def adam_oracle_run(U: int, reps_seconds: float = 0.0, max_reps: int = 1):
             break
     desc = (f"{U} rows x {ADAM_DIM} columns, all touched, x {reps} rep(s) (array copies "
             f"included); single-threaded C oracle in fp64")
-    return U * reps / el, el, reps, desc
+    return U * reps / el, el, reps, desc, U
 
 
 def run_adam(args):
@@ -827,6 +1060,8 @@ def run_adam(args):
         E.engram_sparse_adam(table, m, v, rr, gg, n, lr=1e-3, weight_decay=0.01,
                              step=step_no[0], stream=stream)
 
+    clk = ClockSampler(gpu_smi_id(torch, device))
+    clk.__enter__()
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(device)
@@ -838,12 +1073,13 @@ def run_adam(args):
     launches0 = E.engram_launch_count()
     barrier(device)
     torch.cuda.synchronize(device)
-    with ClockSampler(gpu_smi_id(torch, device)) as clk:
-        for e in evs:
-            e[0].record(stream)
-            step()
-            e[1].record(stream)
-        torch.cuda.synchronize(device)
+    h0 = time.time()
+    for e in evs:
+        e[0].record(stream)
+        step()
+        e[1].record(stream)
+    torch.cuda.synchronize(device)
+    clk.mark_timed(h0, time.time())
     barrier(device)
     launches = E.engram_launch_count() - launches0
     per = [e[0].elapsed_time(e[1]) for e in evs]
@@ -866,6 +1102,7 @@ def run_adam(args):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(device)
     torch.cuda.synchronize(device)
+    h0 = time.time()
     e0.record(s_in)
     for k in range(e2e_steps):
         b = k % 2
@@ -887,6 +1124,8 @@ def run_adam(args):
             out_done[k].record(s_out)
     e1.record(s_out)
     torch.cuda.synchronize(device)
+    clk.mark_timed(h0, time.time())
+    clk.__exit__(None, None, None)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), device)
     if E.engram_get_device_error(stream):
         raise RuntimeError("device error flag set during timing")
@@ -899,14 +1138,12 @@ def run_adam(args):
         "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": total_ms / K,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16/f32",
         "data": "synthetic",
-        "config": {"workload": "adam_shard" if (R, U) == (ADAM_ROWS, ADAM_TOUCHED)
-                   else f"adam_{R}x{D}_touch{U}", "table_rows": R, "dim": D, "touched_rows": U,
-                   "table_dtype": "bf16", "moments": "f32", "lr": 1e-3, "weight_decay": 0.01,
-                   "l2": "inputs larger than L2 (12.8 GB table, 51.2 GB moments, random rows)"},
+        "config": adam_config(R, U),
+        "timed_as": "per-launch CUDA events, eager launches back to back",
         "roofline": {"kernel": "sparse_adam_kernel<bf16,40>", "bound": "hbm",
                      "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": achieved / peak,
-                     "traffic": committed_traffic("sparse_adam_kernel", U)},
+                     "alg_bytes_per_launch": alg, **traffic_fields("sparse_adam_kernel", U)},
         "stages": {"sparse_adam": {"ms": kern_ms, "alg_bytes": alg, "gbs": achieved,
                                    "frac": achieved / peak, "ms_min": min(per),
                                    "ms_max": max(per)}},
@@ -915,16 +1152,16 @@ def run_adam(args):
                 "d2h_bytes_per_step": U * D * 2, "steps": e2e_steps,
                 "pipeline": "copy-in / step + gather of the updated rows / copy-out streams"},
         "gpu_launches": launches,
-        "clocks": clk.summary(),
     }
     if world == 1 and not args.no_cpu_baseline:
-        rate, _, _, _ = adam_oracle_run(2048)
+        rate = adam_oracle_run(2048)[0]
         n = int(max(2048, min(1 << 18, rate * args.cpu_seconds)))
-        val, el, reps, desc = adam_oracle_run(n)
+        val, el, reps, desc, _ = adam_oracle_run(n)
         line["cpu_baseline"] = {"value": val, "unit": "rows/s", "cores": 1, "kind": "oracle",
-                                "sample": desc, "seconds": el}
+                                "sample": desc, "seconds": el, **host_info()}
     else:
         line["cpu_baseline"] = None
+    line["clocks"] = clk.summary()
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -1001,11 +1238,13 @@ def run_owner(args):
     barrier(device)
     torch.cuda.synchronize(device)
     with ClockSampler(gpu_smi_id(torch, device)) as clk:
+        h0 = time.time()
         e0.record(stream)
         for _ in range(K):
             step()
         e1.record(stream)
         torch.cuda.synchronize(device)
+        clk.mark_timed(h0, time.time())
     barrier(device)
     launches = E.engram_launch_count() - launches0
     total_ms = max_over_ranks(e0.elapsed_time(e1), device)
@@ -1056,10 +1295,13 @@ def main(argv=None):
                     help="time the step as a replayed CUDA graph (default)")
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="time eager launches instead")
-    ap.add_argument("--stage", choices=["all", "bwd", "ple", "ple_bwd", "adam", "owner"],
+    ap.add_argument("--stage",
+                    choices=["all", "bwd", "hash", "gather", "ple", "ple_bwd", "adam", "owner"],
                     default="all",
                     help="all: forward + backward (the step); bwd: the backward alone "
-                         "(indices from engram_hash, no table allocated); ple: the PLE "
+                         "(indices from engram_hash, no table allocated); hash: "
+                         "engram_hash alone; gather: engram_gather alone on the hash's "
+                         "indices; ple: the PLE "
                          "tail (norm + short conv) on its own workload; ple_bwd: its "
                          "backward on the same workload; owner: the owner-sharded table "
                          "with all-to-all exchanges; adam: the sparse "

@@ -29,9 +29,10 @@ __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t b
         : "memory");
 }
 
-// Waits (bounded by kCopyWaitNs) for phase `parity` of `bar`; false on timeout.
+// Waits (bounded by limit_ns) for phase `parity` of `bar`; false on timeout.
 // The clock is read once every 64 polls, so a poll costs little issue time.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
+                                          uint64_t limit_ns = kCopyWaitNs)
 {
     const uint32_t addr = smem_u32(bar);
     uint64_t t0 = 0;
@@ -50,7 +51,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
             asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(now));
             if (spin == 0)
                 t0 = now;
-            else if (now - t0 > kCopyWaitNs)
+            else if (now - t0 > limit_ns)
                 return false;
         }
     }

@@ -246,7 +246,9 @@ int bwd_plan(int64_t n, int64_t rows, int32_t dim, BwdPlan *P)
     ENGRAM_TRY(device_sms(&sms));
     ENGRAM_TRY(sort_items(n, sms, &P->items));
     P->ntiles = (int)std::max<int64_t>(1, ceil_div(n, (int64_t)bwd::kSortThreads * P->items));
-    P->wmax = sms * 32; // upper bound on resident warps of seg_reduce
+    // warps of seg_reduce: at most 32 per SM (its resident limit) and one per
+    // 32 lookups, so the fp64 partials below shrink with small n
+    P->wmax = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)sms * 32, ceil_div(n, 32)));
     P->GF = (dim / 4 + 31) / 32;
     size_t off = 0;
     auto take = [&](size_t bytes) {
@@ -283,6 +285,8 @@ int check_workspace(const BwdPlan &P, void *ws, size_t ws_bytes)
     return ENGRAM_OK;
 }
 
+uint32_t barrier_spin_limit();
+
 // The one-launch sort at I pairs per thread; *launched is false where the
 // device or the launch refuses a cooperative grid (nothing ran).
 template <int I>
@@ -301,7 +305,8 @@ int launch_sort_coop(const int32_t *idx, int64_t n, int64_t rows, const BwdPlan 
     const int grid = (int)std::min<int64_t>(P.ntiles, res / (kSortThreads / 32));
     SortArgs args{idx, (unsigned long long *)(ws + P.a), (unsigned long long *)(ws + P.b), n,
                   (uint32_t)rows, P.passes, P.ntiles, P.ngroups, (uint32_t *)(ws + P.tile_cnt),
-                  (uint32_t *)(ws + P.group_cnt), (unsigned *)(ws + P.barrier)};
+                  (uint32_t *)(ws + P.group_cnt), (unsigned *)(ws + P.barrier),
+                  barrier_spin_limit()};
     void *params[] = {&args};
     if (cudaLaunchCooperativeKernel((const void *)radix_sort_coop<I>, dim3(grid),
                                     dim3(kSortThreads), params, 0, stream) != cudaSuccess) {
@@ -322,6 +327,37 @@ bool sort_separate_launches()
         const char *e = std::getenv("ENGRAM_SORT_SEPARATE_LAUNCHES");
         return e != nullptr && e[0] == '1';
     }();
+    return v;
+}
+
+// Test hooks for the bounded waits: ENGRAM_TEST_BARRIER_SPIN=<polls> caps the
+// sort's grid-barrier polls and ENGRAM_TEST_CROSS_WAIT_NS=<ns> the PLE tail
+// kernel's waits on other warps (both read once per process). Small values
+// make a wait run out in a test -- the call then ends with the matching
+// ENGRAM_DEVERR_* bit set instead of the result; unset, the waits keep their
+// normal bounds (about 0.3 s and 0.5 s).
+uint64_t env_u64(const char *name, uint64_t fallback)
+{
+    const char *e = std::getenv(name);
+    if (e == nullptr || e[0] == '\0')
+        return fallback;
+    char *end = nullptr;
+    const unsigned long long v = std::strtoull(e, &end, 10);
+    return (end != nullptr && *end == '\0') ? (uint64_t)v : fallback;
+}
+
+uint32_t barrier_spin_limit()
+{
+    static const uint32_t v = (uint32_t)std::min<uint64_t>(
+        env_u64("ENGRAM_TEST_BARRIER_SPIN", bwd::kBarrierSpin), bwd::kBarrierSpin);
+    return v;
+}
+
+uint64_t cross_wait_ns()
+{
+    static const uint64_t v =
+        std::min<uint64_t>(env_u64("ENGRAM_TEST_CROSS_WAIT_NS", ple::kCopyWaitNs),
+                           ple::kCopyWaitNs);
     return v;
 }
 
@@ -787,6 +823,7 @@ int conv_plan(const engram_conv_params_t *p, int32_t dtype, int32_t out_dtype, i
     a.halo = halo;
     a.norm_slots = norm_slots;
     a.flags = p->flags;
+    a.cross_wait_ns = cross_wait_ns();
     P->chan = chan;
     P->threads = (nth + 31) / 32 * 32;
     P->smem = ple::smem_bytes(norm_slots, nth, chan);

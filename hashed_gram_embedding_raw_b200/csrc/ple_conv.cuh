@@ -64,6 +64,7 @@ struct ConvArgs {
     int32_t reg_bufs;   // residue-class kernel: row buffers (of 8 rows each)
     int32_t pitch;      // residue-class kernel: bytes per buffered row
     int32_t classes;    // residue-class kernel: residues with rows, min(dil, T)
+    uint64_t cross_wait_ns; // residue-class kernel: bound of a wait on other warps
 };
 
 // Shared memory: inverse RMS [2][kChunk] float and history-tap counts

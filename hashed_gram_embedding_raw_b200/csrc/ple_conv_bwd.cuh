@@ -409,8 +409,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
     // squares of its rows
     auto stage1 = [&](int b, int s0) {
         const int32_t j0 = js + b * B;
-        if (j0 < je && !timed_out &&
-            !mbar_wait(bars + b % kBwdBars, (uint32_t)(b / kBwdBars) & 1u))
+        // (the block's own copies are waited for even after a timeout, so
+        // that none is still in flight when the block ends)
+        if (j0 < je && !mbar_wait(bars + b % kBwdBars, (uint32_t)(b / kBwdBars) & 1u))
             timed_out = true;
         if (!do_norm)
             return;

@@ -27,7 +27,9 @@
 // No barrier spans the block inside the loop, so conv warps drift apart by up
 // to the ring depth. Every wait is bounded in time: one that runs out raises
 // ENGRAM_DEVERR_COPY_TIMEOUT and the thread skips its later waits on other
-// warps (not those on its own copies), so the kernel always ends promptly.
+// warps (not those on its own copies, which it always waits for before the
+// block ends), so the kernel always ends promptly. Waits on other warps are
+// bounded by ConvArgs::cross_wait_ns, waits on copies by kCopyWaitNs.
 // The 3 rows before a range are read for history only.
 #pragma once
 
@@ -231,7 +233,8 @@ __global__ void __maxnreg__(CH == 4 ? 80 : 128)
             // warp is done with it
             if (sw == 0 && c >= 1 && c - 1 + NB < nbatch) {
                 const int pb = (c - 1) % NB;
-                if (!timed_out && !mbar_wait(empty_bar + pb, (uint32_t)((c - 1) / NB) & 1u))
+                if (!timed_out && !mbar_wait(empty_bar + pb, (uint32_t)((c - 1) / NB) & 1u,
+                                             a.cross_wait_ns))
                     timed_out = true;
                 load_batch(c - 1 + NB);
             }
@@ -279,7 +282,7 @@ __global__ void __maxnreg__(CH == 4 ? 80 : 128)
         const int b = c % NB;
         const int32_t j0 = js + c * B;
         const int rc = min(B, jb - j0);
-        if (!timed_out && !mbar_wait(full_bar + b, (uint32_t)(c / NB) & 1u))
+        if (!timed_out && !mbar_wait(full_bar + b, (uint32_t)(c / NB) & 1u, a.cross_wait_ns))
             timed_out = true;
         const uint32_t buf = smem_u32(data) + (uint32_t)(b * B) * pitch + xoff;
         // the batch's inverse RMS values in two 16-byte loads, and the output
@@ -365,7 +368,9 @@ __global__ void __maxnreg__(CH == 4 ? 80 : 128)
                 orow_p += ostep;
             }
         };
-        if (fast_s[b])
+        // (rc == B keeps the full-batch path inside the block's rows even
+        // when a wait on the statistics warps ran out and fast_s is stale)
+        if (fast_s[b] && rc == B)
             run(std::true_type{});
         else
             run(std::false_type{});

@@ -389,6 +389,7 @@ struct SortArgs {
     uint32_t *tile_cnt;  // [ntiles][256], rewritten every pass
     uint32_t *group_cnt; // [passes][ngroups][256], zero on entry
     unsigned *barrier;   // grid-barrier arrival counter; zero on entry
+    uint32_t spin_limit; // polls before a grid-barrier wait gives up (<= kBarrierSpin)
 };
 
 // Grid-wide barrier among co-resident blocks on one arrival counter that only
@@ -398,7 +399,8 @@ struct SortArgs {
 // (bounded; giving up raises ENGRAM_DEVERR_SORT_TIMEOUT and returns false).
 // The block's other threads wait at __syncthreads, which orders their later
 // reads after thread 0's acquire. The counter is zero at launch.
-__device__ __forceinline__ bool grid_barrier(unsigned *bar, unsigned &gen, int &flag)
+__device__ __forceinline__ bool grid_barrier(unsigned *bar, unsigned &gen, int &flag,
+                                             uint32_t spin_limit)
 {
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -412,7 +414,7 @@ __device__ __forceinline__ bool grid_barrier(unsigned *bar, unsigned &gen, int &
         if (before + 1 < target) {
             uint32_t spins = 0;
             while (ld_acquire_u32(bar) < target) {
-                if (++spins > kBarrierSpin) {
+                if (++spins > spin_limit) {
                     raise_device_error(ENGRAM_DEVERR_SORT_TIMEOUT);
                     ok = false;
                     break;
@@ -453,12 +455,12 @@ template <int ITEMS> __global__ void __launch_bounds__(kSortThreads, 4) radix_so
                 tcount = tile_digit_count(sm);
                 publish_counts(tile, tcount, a.tile_cnt, gc);
             }
-            if (!grid_barrier(a.barrier, gen, sm.flag))
+            if (!grid_barrier(a.barrier, gen, sm.flag, a.spin_limit))
                 return;
             if (has)
                 place_tile<true>(sm, dst, a.n, shift, tile, tcount, it, rank, a.tile_cnt, gc,
                                  a.ngroups);
-            if (pass + 1 < a.passes && !grid_barrier(a.barrier, gen, sm.flag))
+            if (pass + 1 < a.passes && !grid_barrier(a.barrier, gen, sm.flag, a.spin_limit))
                 return;
         }
         return;
@@ -476,11 +478,11 @@ template <int ITEMS> __global__ void __launch_bounds__(kSortThreads, 4) radix_so
         const int shift = pass * kRadixBits;
         for (int tile = blockIdx.x; tile < a.ntiles; tile += gridDim.x)
             count_order_tile(sm, src, first, a.n, shift, a.rows, tile, a.tile_cnt, gc, ordered);
-        if (!grid_barrier(a.barrier, gen, sm.flag))
+        if (!grid_barrier(a.barrier, gen, sm.flag, a.spin_limit))
             return;
         for (int tile = blockIdx.x; tile < a.ntiles; tile += gridDim.x)
             place_ordered_tile(sm, ordered, dst, a.n, shift, tile, a.tile_cnt, gc, a.ngroups);
-        if (pass + 1 < a.passes && !grid_barrier(a.barrier, gen, sm.flag))
+        if (pass + 1 < a.passes && !grid_barrier(a.barrier, gen, sm.flag, a.spin_limit))
             return;
     }
 }

@@ -6,9 +6,10 @@ workspace, or a path that must not call cudaMalloc because it can synchronise
 the device). It keeps its scratch in one fixed array inside the library, so
 these tests call it through the C ABI twice in a row -- the second call
 starts from whatever the first left in that array -- and compare each result
-with the workspace-based entry point on the same input, within the
-tolerance the other backward tests use. This file is collected last so that a
-run stopping at the first failure has run every other test already.
+with the workspace-based entry point on the same input and with the CPU
+oracle, within the tolerance the other backward tests use. This file is
+collected last so that a run stopping at the first failure has run every
+other test already.
 """
 
 import ctypes
@@ -16,6 +17,8 @@ import ctypes
 import numpy as np
 import pytest
 import torch
+
+import oracle
 
 pytestmark = pytest.mark.gpu
 
@@ -56,6 +59,11 @@ def _noalloc_via_abi(E, idx, dout, rows):
     return uniq, grads, nu
 
 
+def _close(got, want):
+    err = (got.double() - want.double()).abs()
+    return bool((err <= ATOL + RTOL * want.double().abs()).all())
+
+
 def _compare(E, idx, dout, rows):
     ref_u, ref_g, ref_nu = E.engram_backward(idx, dout, rows)
     u, g, nu = _noalloc_via_abi(E, idx, dout, rows)
@@ -63,10 +71,18 @@ def _compare(E, idx, dout, rows):
     U = int(ref_nu.item())
     assert int(nu.item()) == U
     assert torch.equal(u[:U], ref_u[:U])
-    want = ref_g[:U].double()
-    err = (g[:U].double() - want).abs()
-    assert bool((err <= ATOL + RTOL * want.abs()).all())
+    assert _close(g[:U], ref_g[:U])
     assert E.engram_get_device_error() == 0
+    # and against the oracle
+    d = dout.cpu()
+    raw = d.numpy() if d.dtype == torch.float32 else \
+        d.view(torch.int16).numpy().view(np.uint16)
+    code = {torch.float32: oracle.F32, torch.bfloat16: oracle.BF16,
+            torch.float16: oracle.F16}[d.dtype]
+    want_u, want_g = oracle.backward(idx.cpu().numpy(), raw, code)
+    assert len(want_u) == U
+    np.testing.assert_array_equal(u[:U].cpu().numpy(), want_u)
+    assert _close(g[:U].cpu(), torch.from_numpy(want_g))
 
 
 def test_noalloc_two_calls_in_a_row_match_workspace_entry(E):
@@ -76,6 +92,15 @@ def test_noalloc_two_calls_in_a_row_match_workspace_entry(E):
     # second call, different shape and dtype, on top of the first's leftovers
     idx, dout = _case(2, 70_001, 5_000, 96, torch.float32)
     _compare(E, idx, dout, 5_000)
+
+
+def test_noalloc_wide_rows_small_batch(E):
+    # 512-wide rows: the scratch the reduction needs grows with the lookups,
+    # so a small batch fits the array
+    idx, dout = _case(3, 5_000, 70_000, 512, torch.bfloat16)
+    _compare(E, idx, dout, 70_000)
+    idx, dout = _case(4, 1, 10, 512, torch.float32)
+    _compare(E, idx, dout, 10)
 
 
 def test_noalloc_rejects_sizes_beyond_its_array(E):
