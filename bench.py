@@ -2,13 +2,15 @@
 
 One step = the fused hash+gather forward (engram_hash_gather, writing the
 [T, 16*160] rows and the [T, 16] indices) followed by the compact backward
-(engram_backward_sort + engram_backward_reduce: distinct rows and fp32 row
-gradients) over one batch of the named workload, all inputs resident in HBM.
+(engram_backward_sort_heads + engram_backward_reduce: distinct rows and fp32
+row gradients) over one batch of the named workload, all inputs resident in
+HBM.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload full]
     python bench.py --impl reference ...   # the CPU oracle, timed on this host
     python bench.py --stage hash ...       # engram_hash alone (L2 flushed between launches)
     python bench.py --stage gather ...     # engram_gather alone on the hash's indices
+    python bench.py --stage fwd ...        # engram_hash_gather alone
     python bench.py --stage bwd ...        # the backward alone (sort + reduce)
     python bench.py --stage ple ...        # the PLE tail kernel on its own workload
     python bench.py --stage ple_bwd ...    # the PLE tail's backward on the same workload
@@ -278,9 +280,10 @@ def workload_config(name: str, world: int, stage: str = "forward + backward") ->
 # ------------------------------------------------------------ CPU oracle leg
 
 STAGE_NAMES = {"all": "forward + backward", "bwd": "backward only",
-               "hash": "hash only (engram_hash)", "gather": "gather only (engram_gather)"}
+               "hash": "hash only (engram_hash)", "gather": "gather only (engram_gather)",
+               "fwd": "fused forward only (engram_hash_gather)"}
 ORACLE_PARTS = {"all": ("hash", "gather", "backward"), "bwd": ("backward",),
-                "hash": ("hash",), "gather": ("gather",)}
+                "hash": ("hash",), "gather": ("gather",), "fwd": ("hash", "gather")}
 
 
 def oracle_run(name: str, S: int, reps_seconds: float = 0.0, max_reps: int = 1,
@@ -407,6 +410,8 @@ STAGE_METRICS = {
              "indices per token); achieved HBM GB/s vs peak"),
     "gather": ("Engram gather tokens/s (engram_gather alone: 16 row lookups of 160 bf16 "
                "per token from the hash's indices); achieved HBM GB/s vs peak"),
+    "fwd": ("Engram forward tokens/s (engram_hash_gather alone: hash and 16 row lookups "
+            "per token, rows and indices written); achieved HBM GB/s vs peak"),
 }
 L2_FLUSH_BYTES = 256 << 20     # twice the B200's 126 MB L2
 
@@ -443,7 +448,7 @@ def run_ours(args):
     tdtype = {"bf16": torch.bfloat16, "f32": torch.float32}[w.dtype]
     esize = 2 if w.dtype == "bf16" else 4
     fwd, bwd = stage == "all", stage in ("all", "bwd")
-    gathers = stage in ("all", "gather")
+    gathers = stage in ("all", "gather", "fwd")
 
     table = None
     if gathers:
@@ -452,8 +457,9 @@ def run_ours(args):
     dout_h = host_dout(name, n, D, w.dtype).pin_memory() if bwd else None
     ws = (torch.empty(E.engram_backward_workspace_size(n, R, D), dtype=torch.uint8,
                       device=device) if bwd else None)
-    flush = (torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
-             if stage == "hash" else None)
+    per_launch = stage in ("hash", "gather", "fwd")
+    flush = (torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+             if per_launch else None)
     bufs = [{
         "ids": torch.from_numpy(ids_np.copy()).to(device),
         "cu": torch.from_numpy(cu_np.copy()).to(device),
@@ -465,7 +471,7 @@ def run_ours(args):
         "nu": torch.empty(1, dtype=torch.int32, device=device),
     } for _ in range(2)]
     stream = torch.cuda.Stream(device)
-    if not fwd:   # the backward and the gather alone take the hash's indices
+    if stage in ("bwd", "gather"):   # these take the hash's indices
         for b in bufs:
             E.engram_hash(params, b["ids"], b["cu"], out_idx=b["idx"], stream=stream)
 
@@ -477,6 +483,10 @@ def run_ours(args):
         if stage == "gather":
             E.engram_gather(table, b["idx"].view(-1), out=b["out"].view(n, D), stream=stream)
             return
+        if stage == "fwd":
+            E.engram_hash_gather(params, b["ids"], table, cu_seqlens=b["cu"], out=b["out"],
+                                 out_idx=b["idx"], stream=stream)
+            return
         if ev is not None:
             ev[0].record(stream)
         if fwd:
@@ -484,7 +494,10 @@ def run_ours(args):
                                  out_idx=b["idx"], stream=stream)
         if ev is not None:
             ev[1].record(stream)
-        E.engram_backward_sort(b["idx"].view(-1), R, D, ws, stream=stream)
+        if args.bwd_sort == "heads":
+            E.engram_backward_sort_heads(params, b["idx"], ws, stream=stream)
+        else:
+            E.engram_backward_sort(b["idx"].view(-1), R, D, ws, stream=stream)
         if ev is not None:
             ev[2].record(stream)
         E.engram_backward_reduce(n, R, b["dout"], b["uniq"], b["grads"], b["nu"], ws,
@@ -493,9 +506,12 @@ def run_ours(args):
             ev[3].record(stream)
 
     def flush_l2():
+        # a read of twice the L2's size: the lines it leaves are clean, so the
+        # next launch neither finds its inputs in L2 nor pays for writing back
+        # another kernel's dirty lines
         if flush is not None:
             with torch.cuda.stream(stream):
-                flush.fill_(1)
+                flush.sum()
 
     clk = ClockSampler(gpu_smi_id(torch, device))
     clk.__enter__()
@@ -508,7 +524,6 @@ def run_ours(args):
     U = int(bufs[0]["nu"].item()) if bwd else None
 
     K = args.steps
-    per_launch = stage in ("hash", "gather")
     graph, launches_per_step = None, None
     if per_launch:
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -528,9 +543,9 @@ def run_ours(args):
         launches = E.engram_launch_count() - launches0
         per = [e[0].elapsed_time(e[1]) for e in evs]
         local_ms = sum(per)
-        timed_as = ("sum of per-launch CUDA-event times, eager launches"
-                    + ("; L2 flushed by a 256 MB write between launches (not timed)"
-                       if flush is not None else "; inputs larger than L2"))
+        timed_as = ("sum of per-launch CUDA-event times, eager launches; L2 flushed "
+                    "between launches by a 256 MB read (not timed), which also writes "
+                    "back the previous launch's dirty lines outside the timed region")
     else:
         # one step captured as a CUDA graph and replayed (the library's calls
         # need no host synchronisation), or eager launches
@@ -586,8 +601,9 @@ def run_ours(args):
     # two sets of device buffers), so step k's results travel to the host
     # while step k+1 computes and PCIe carries both directions at once.
     in_names = {"all": ["ids", "cu", "dout"], "bwd": ["idx", "dout"],
-                "hash": ["ids", "cu"], "gather": ["idx"]}[stage]
-    out_fixed = {"all": ["out", "nu"], "bwd": ["nu"], "hash": ["idx"], "gather": ["out"]}[stage]
+                "hash": ["ids", "cu"], "gather": ["idx"], "fwd": ["ids", "cu"]}[stage]
+    out_fixed = {"all": ["out", "nu"], "bwd": ["nu"], "hash": ["idx"], "gather": ["out"],
+                 "fwd": ["out", "idx"]}[stage]
 
     def run_e2e(resident_rows: bool):
         """resident_rows (stage all only): read back num_unique alone and leave
@@ -680,13 +696,14 @@ def run_ours(args):
     gather_bytes = n * (4 + 2 * D * esize)
     stages = {}
     if per_launch:
-        kname = "hash_kernel<3, 8>" if stage == "hash" else "gather_kernel<20>"
-        dom_bytes = hash_bytes if stage == "hash" else gather_bytes
+        kname = {"hash": "hash_kernel<3, 8>", "gather": "gather_kernel<20>",
+                 "fwd": "hash_gather_kernel<3, 8, 20>"}[stage]
+        dom_bytes = {"hash": hash_bytes, "gather": gather_bytes, "fwd": fwd_bytes}[stage]
         dom_ms = statistics.mean(per)
         stages[stage] = {"ms": dom_ms, "ms_min": min(per), "ms_max": max(per),
                          "alg_bytes": dom_bytes, "gbs": dom_bytes / dom_ms / 1e6,
                          "frac": dom_bytes / dom_ms / 1e6 / peak}
-        dom, tkey, tunits = kname, kname.split("<")[0], (T if stage == "hash" else n)
+        dom, tkey, tunits = kname, kname.split("<")[0], (n if stage == "gather" else T)
     else:
         red_bytes = n * D * esize + U * (4 + D * 4)
         bwd_bytes = n * 4 + red_bytes
@@ -717,6 +734,9 @@ def run_ours(args):
         "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": total_ms / K,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
         "data": "synthetic", "config": config, "timed_as": timed_as,
+        "backward_sort": (None if not bwd else
+                          "by head (engram_backward_sort_heads)" if args.bwd_sort == "heads"
+                          else "whole row range (engram_backward_sort)"),
         "roofline": {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                      "alg_bytes_per_launch": dom_bytes, **traffic_fields(tkey, tunits)},
@@ -1289,6 +1309,9 @@ def main(argv=None):
     ap.add_argument("--ple-tokens", type=int, default=0,
                     help="--stage ple / ple_bwd: whole 4,096-token rows to use instead of "
                          "the workload's 16 (a smaller case for profiling)")
+    ap.add_argument("--bwd-sort", choices=["heads", "plain"], default="heads",
+                    help="backward sort: by head (engram_backward_sort_heads, the default) "
+                         "or over the whole row range (engram_backward_sort)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--graph", dest="graph", action="store_true", default=True,
@@ -1296,10 +1319,12 @@ def main(argv=None):
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="time eager launches instead")
     ap.add_argument("--stage",
-                    choices=["all", "bwd", "hash", "gather", "ple", "ple_bwd", "adam", "owner"],
+                    choices=["all", "bwd", "fwd", "hash", "gather", "ple", "ple_bwd", "adam",
+                             "owner"],
                     default="all",
                     help="all: forward + backward (the step); bwd: the backward alone "
-                         "(indices from engram_hash, no table allocated); hash: "
+                         "(indices from engram_hash, no table allocated); fwd: "
+                         "engram_hash_gather alone; hash: "
                          "engram_hash alone; gather: engram_gather alone on the hash's "
                          "indices; ple: the PLE "
                          "tail (norm + short conv) on its own workload; ple_bwd: its "

@@ -10,12 +10,13 @@ has not been built (`python hashed_gram_embedding_raw_b200/build.py`).
 
 from ._binding import (ENGRAM_BF16, ENGRAM_CONV_NORM, ENGRAM_CONV_RESIDUAL, ENGRAM_CONV_SILU,
                        ENGRAM_DEVERR_COPY_TIMEOUT, ENGRAM_DEVERR_CU_SEQLENS,
-                       ENGRAM_DEVERR_ROW_RANGE,
+                       ENGRAM_DEVERR_ROW_RANGE, ENGRAM_DEVERR_SORT_TIMEOUT,
                        ENGRAM_EINVAL, ENGRAM_ECUDA, ENGRAM_ENOSPC, ENGRAM_F16, ENGRAM_F32,
                        ENGRAM_NOALLOC_SCRATCH_BYTES, ENGRAM_OK, EXPORTED, LIB_PATH,
                        AdamParams, ConvParams, EngramError, EngramParams, engram_abi_version,
-                       engram_backward,
+                       engram_backward, engram_backward_heads,
                        engram_backward_noalloc, engram_backward_reduce, engram_backward_sort,
+                       engram_backward_sort_heads,
                        engram_backward_workspace_size, engram_gather, engram_get_device_error,
                        engram_grouped_rms_norm, engram_hash, engram_hash_gather,
                        engram_hash_gather_slice, engram_host_floor_mod, engram_ple_short_conv,
@@ -27,11 +28,13 @@ from ._binding import (ENGRAM_BF16, ENGRAM_CONV_NORM, ENGRAM_CONV_RESIDUAL, ENGR
 __all__ = [
     "ENGRAM_BF16", "ENGRAM_CONV_NORM", "ENGRAM_CONV_RESIDUAL", "ENGRAM_CONV_SILU",
     "ENGRAM_DEVERR_COPY_TIMEOUT", "ENGRAM_DEVERR_CU_SEQLENS", "ENGRAM_DEVERR_ROW_RANGE",
-    "ENGRAM_EINVAL",
+    "ENGRAM_DEVERR_SORT_TIMEOUT", "ENGRAM_EINVAL",
     "ENGRAM_ECUDA", "ENGRAM_ENOSPC", "ENGRAM_F16", "ENGRAM_F32",
     "ENGRAM_NOALLOC_SCRATCH_BYTES", "ENGRAM_OK", "EXPORTED", "LIB_PATH", "AdamParams", "ConvParams",
-    "EngramError", "EngramParams", "engram_abi_version", "engram_backward", "engram_backward_noalloc",
-    "engram_backward_reduce", "engram_backward_sort", "engram_backward_workspace_size",
+    "EngramError", "EngramParams", "engram_abi_version", "engram_backward",
+    "engram_backward_heads", "engram_backward_noalloc",
+    "engram_backward_reduce", "engram_backward_sort", "engram_backward_sort_heads",
+    "engram_backward_workspace_size",
     "engram_gather", "engram_get_device_error", "engram_hash", "engram_hash_gather",
     "engram_hash_gather_slice", "engram_grouped_rms_norm", "engram_ple_short_conv",
     "engram_ple_short_conv_backward", "engram_ple_short_conv_backward_workspace_size",

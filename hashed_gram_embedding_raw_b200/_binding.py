@@ -36,6 +36,7 @@ EXPORTED = (
     "engram_ple_short_conv", "engram_grouped_rms_norm", "engram_sparse_adam",
     "engram_ple_short_conv_backward", "engram_ple_short_conv_backward_workspace_size",
     "engram_owner_bucket", "engram_owner_bucket_workspace_size",
+    "engram_backward_heads", "engram_backward_sort_heads",
 )
 
 ENGRAM_NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -145,6 +146,8 @@ def _load():
         "engram_ple_short_conv_backward_workspace_size": [P, i64, ctypes.POINTER(sz)],
         "engram_owner_bucket": [P, i64, i64, i32, P, P, P, P, P, sz, P],
         "engram_owner_bucket_workspace_size": [i64, i32, ctypes.POINTER(sz)],
+        "engram_backward_heads": [P, P, i64, P, i32, P, P, P, P, sz, P],
+        "engram_backward_sort_heads": [P, P, i64, P, sz, P],
     }
     for name, args in sig.items():
         fn = getattr(L, name)
@@ -375,6 +378,38 @@ def engram_backward_sort(idx: torch.Tensor, table_rows: int, dim: int, workspace
     _cuda(workspace, "workspace", torch.uint8)
     _check(lib.engram_backward_sort(_ptr(idx), idx.numel(), table_rows, dim, _ptr(workspace),
                                     workspace.numel(), _stream(stream)), "engram_backward_sort")
+
+
+def engram_backward_heads(params: EngramParams, idx: torch.Tensor, dout: torch.Tensor,
+                          uniq_rows=None, row_grads=None, num_unique=None, workspace=None,
+                          stream=None):
+    """engram_backward for the hash's lookups idx [T, H] (head h's lookups in
+    its own slice), sorted by head: same results, fewer radix passes."""
+    _cuda(idx, "idx", torch.int32)
+    _cuda(dout, "dout")
+    H, dim, rows = params.heads, params.dim, params.table_rows
+    n = idx.numel()
+    if n % H != 0 or dout.numel() != n * dim:
+        raise ValueError("idx must be [T, H] and dout [T * H, dim]")
+    uniq_rows, row_grads, num_unique, workspace = _bwd_buffers(
+        n, dim, idx.device, uniq_rows, row_grads, num_unique, workspace, rows)
+    _check(lib.engram_backward_heads(ctypes.byref(params), _ptr(idx), n // H, _ptr(dout),
+                                     _dtype_code(dout), _ptr(uniq_rows), _ptr(row_grads),
+                                     _ptr(num_unique), _ptr(workspace), workspace.numel(),
+                                     _stream(stream)), "engram_backward_heads")
+    return uniq_rows, row_grads, num_unique
+
+
+def engram_backward_sort_heads(params: EngramParams, idx: torch.Tensor, workspace,
+                               stream=None) -> None:
+    _cuda(idx, "idx", torch.int32)
+    _cuda(workspace, "workspace", torch.uint8)
+    H = params.heads
+    if idx.numel() % H != 0:
+        raise ValueError("idx must be [T, H]")
+    _check(lib.engram_backward_sort_heads(ctypes.byref(params), _ptr(idx), idx.numel() // H,
+                                          _ptr(workspace), workspace.numel(), _stream(stream)),
+           "engram_backward_sort_heads")
 
 
 def engram_backward_reduce(n: int, table_rows: int, dout: torch.Tensor, uniq_rows, row_grads,

@@ -185,6 +185,26 @@ __device__ __forceinline__ int32_t find_sequence(const int32_t *__restrict__ cu,
     return lo;
 }
 
+// find_sequence for a t shared by the whole warp: each round the 32 lanes probe
+// 32 evenly spaced bounds at once, so nseq <= 32 takes one round of loads
+// and 1,024 two, instead of a chain of log2(nseq) dependent loads.
+__device__ __forceinline__ int32_t find_sequence_warp(const int32_t *__restrict__ cu,
+                                                      int32_t nseq, int64_t t)
+{
+    const int lane = threadIdx.x & 31;
+    int32_t lo = 0, hi = nseq - 1; // the answer lies in [lo, hi]; cu[lo] <= t
+    while (lo < hi) {
+        const int32_t step = (hi - lo + 32) / 32; // ceil((hi - lo + 1) / 32)
+        const int32_t p = lo + lane * step;
+        const bool le = p <= hi && (p == lo || __ldg(cu + p) <= t);
+        const uint32_t m = __ballot_sync(kFull, le);
+        const int32_t k = 31 - __clz(m); // lane 0 always qualifies
+        lo = lo + k * step;
+        hi = min(hi, lo + step - 1);
+    }
+    return lo;
+}
+
 // Flags malformed cu_seqlens (not 0 .. T, or decreasing). Grid-strided.
 __device__ __forceinline__ void check_cu_seqlens(const int32_t *__restrict__ cu, int32_t nseq,
                                                  int64_t T)

@@ -189,67 +189,30 @@ int launch_hash_gather(const HashArgs &a, const int32_t *ids, const int32_t *cu,
 
 // --------------------------------------------------------------- backward
 
+// Workspace layout of the backward for n lookups: large enough for the sort
+// of either form (one segment, or one per head) at any tile size.
 struct BwdPlan {
-    int passes = 0, items = 0, ntiles = 0, ngroups = 0, wmax = 0, GF = 0;
+    int wmax = 0, GF = 0, tiles_max = 0, groups_max = 0;
     size_t a = 0, b = 0, tile_cnt = 0, ctl = 0, ctl_bytes = 0, group_cnt = 0, barrier = 0;
     size_t wcount = 0, bcount = 0, pb = 0, pe = 0, meta = 0, total = 0;
 };
-
-template <int I> int sort_resident_blocks(int64_t *blocks)
-{
-    int64_t warps = 0;
-    ENGRAM_TRY(resident_warps(bwd::radix_sort_coop<I>, bwd::kSortThreads, 0, &warps));
-    *blocks = warps / (bwd::kSortThreads / 32);
-    return ENGRAM_OK;
-}
-
-// Pairs per thread of the sort's tiles (4..8). Among the sizes that keep every
-// tile resident at once (the one-launch sort then holds a block's items in
-// registers across the grid barrier), take the one whose busiest SM holds the
-// fewest pairs -- 512 tiles of 2048 on 148 SMs leave 68 SMs with four tiles
-// and 80 with three; 586 tiles of 1792 give nearly all of them four smaller
-// ones. With none resident, the largest tiles.
-int sort_items(int64_t n, int sms, int *items)
-{
-    int64_t res[bwd::kSortItemsMax + 1] = {};
-    ENGRAM_TRY(sort_resident_blocks<4>(&res[4]));
-    ENGRAM_TRY(sort_resident_blocks<5>(&res[5]));
-    ENGRAM_TRY(sort_resident_blocks<6>(&res[6]));
-    ENGRAM_TRY(sort_resident_blocks<7>(&res[7]));
-    ENGRAM_TRY(sort_resident_blocks<8>(&res[8]));
-    int best = bwd::kSortItemsMax;
-    int64_t best_load = INT64_MAX;
-    for (int I = bwd::kSortItemsMax; I >= 4; --I) {
-        const int64_t tiles = std::max<int64_t>(1, ceil_div(n, (int64_t)bwd::kSortThreads * I));
-        if (tiles > res[I])
-            continue;
-        const int64_t load = ceil_div(tiles, (int64_t)sms) * I;
-        if (load < best_load) {
-            best = I;
-            best_load = load;
-        }
-    }
-    *items = best;
-    return ENGRAM_OK;
-}
 
 int bwd_plan(int64_t n, int64_t rows, int32_t dim, BwdPlan *P)
 {
     if (n < 0 || n > INT32_MAX || rows < 1 || rows > (int64_t(1) << 31) || dim < 8 ||
         dim % 8 != 0 || dim > 512)
         return ENGRAM_EINVAL;
-    int bits = 0;
-    while ((int64_t(1) << bits) < rows)
-        ++bits;
-    P->passes = std::max(1, (bits + bwd::kRadixBits - 1) / bwd::kRadixBits);
     int sms = 0;
     ENGRAM_TRY(device_sms(&sms));
-    ENGRAM_TRY(sort_items(n, sms, &P->items));
-    P->ntiles = (int)std::max<int64_t>(1, ceil_div(n, (int64_t)bwd::kSortThreads * P->items));
     // warps of seg_reduce: at most 32 per SM (its resident limit) and one per
     // 32 lookups, so the fp64 partials below shrink with small n
     P->wmax = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)sms * 32, ceil_div(n, 32)));
     P->GF = (dim / 4 + 31) / 32;
+    // the smallest tiles, plus one short tile per segment at most
+    P->tiles_max = (int)(ceil_div(std::max<int64_t>(n, 1),
+                                  (int64_t)bwd::kSortThreads * bwd::kSortItemsMin) +
+                         bwd::kMaxSegments);
+    P->groups_max = (int)(ceil_div(P->tiles_max, bwd::kTilesPerGroup) + bwd::kMaxSegments);
     size_t off = 0;
     auto take = [&](size_t bytes) {
         const size_t at = off;
@@ -261,10 +224,9 @@ int bwd_plan(int64_t n, int64_t rows, int32_t dim, BwdPlan *P)
     P->b = take(nn * 8);
     // per-tile digit counts (rewritten by every pass), and per-group digit
     // sums of every pass (accumulated with atomic adds, zeroed once per sort)
-    P->ngroups = (int)ceil_div(P->ntiles, bwd::kTilesPerGroup);
-    P->tile_cnt = take((size_t)bwd::kRadix * P->ntiles * 4);
+    P->tile_cnt = take((size_t)bwd::kRadixMax * P->tiles_max * 4);
     P->ctl = off;
-    P->group_cnt = take((size_t)P->passes * bwd::kRadix * P->ngroups * 4);
+    P->group_cnt = take((size_t)bwd::kMaxPasses * bwd::kRadixMax * P->groups_max * 4);
     P->barrier = take(sizeof(unsigned)); // grid-barrier counter of the one-launch sort
     P->ctl_bytes = off - P->ctl;
     P->wcount = take((size_t)P->wmax * 4);
@@ -285,12 +247,146 @@ int check_workspace(const BwdPlan &P, void *ws, size_t ws_bytes)
     return ENGRAM_OK;
 }
 
+// What one sort orders: S segments of L lookups; segment s holds keys
+// off[s] .. off[s] + size[s] - 1 and is sorted by key - off[s].
+struct SortShape {
+    int S = 1;
+    int64_t L = 0;
+    int32_t off[bwd::kMaxSegments] = {};
+    uint32_t size[bwd::kMaxSegments] = {};
+};
+
+int bit_width(uint64_t v) // bits needed for 0 .. v
+{
+    int b = 0;
+    while (b < 64 && (v >> b) != 0)
+        ++b;
+    return b;
+}
+
+// The plain sort: one segment of all n lookups over the whole table.
+SortShape plain_shape(int64_t n, int64_t rows)
+{
+    SortShape sh;
+    sh.S = 1;
+    sh.L = n;
+    sh.off[0] = 0;
+    sh.size[0] = (uint32_t)std::min<int64_t>(rows, UINT32_MAX);
+    return sh;
+}
+
+// The sort by head: lookup j = t * H + h of T tokens lies in head h's slice.
+// Needs ascending, disjoint slices inside the table; otherwise the plain sort.
+SortShape head_shape(const engram_params_t *p, int64_t T)
+{
+    const int H = (p->ngram_size - 1) * p->heads_per_ngram;
+    bool ok = H >= 1 && H <= bwd::kMaxSegments;
+    for (int h = 0; ok && h < H; ++h) {
+        const int64_t o = p->offsets[h], v = p->vocab_sizes[h];
+        ok = v >= 1 && o >= 0 && o + v <= p->table_rows && o <= INT32_MAX &&
+             (h == 0 || o >= p->offsets[h - 1] + p->vocab_sizes[h - 1]);
+    }
+    if (!ok)
+        return plain_shape(T * std::max(H, 1), p->table_rows);
+    SortShape sh;
+    sh.S = H;
+    sh.L = T;
+    for (int h = 0; h < H; ++h) {
+        sh.off[h] = (int32_t)p->offsets[h];
+        sh.size[h] = (uint32_t)p->vocab_sizes[h];
+    }
+    return sh;
+}
+
+template <int I> int sort_resident_blocks(int64_t *blocks)
+{
+    int64_t warps = 0;
+    ENGRAM_TRY(resident_warps(bwd::radix_sort_coop<I>, bwd::kSortThreads, 0, &warps));
+    *blocks = warps / (bwd::kSortThreads / 32);
+    return ENGRAM_OK;
+}
+
+int64_t shape_tiles(const SortShape &sh, int items)
+{
+    return sh.S * std::max<int64_t>(1, ceil_div(sh.L, (int64_t)bwd::kSortThreads * items));
+}
+
+// Pairs per thread of the sort's tiles (4..8). Among the sizes that keep every
+// tile resident at once (the one-launch sort then holds a block's items in
+// registers across the grid barrier), take the one whose busiest SM holds the
+// fewest pairs -- 512 tiles of 2048 on 148 SMs leave 68 SMs with four tiles
+// and 80 with three; 592 tiles of 1792 give every SM four smaller ones. With
+// none resident, the largest tiles.
+int sort_items(const SortShape &sh, int sms, int *items)
+{
+    int64_t res[bwd::kSortItemsMax + 1] = {};
+    ENGRAM_TRY(sort_resident_blocks<4>(&res[4]));
+    ENGRAM_TRY(sort_resident_blocks<5>(&res[5]));
+    ENGRAM_TRY(sort_resident_blocks<6>(&res[6]));
+    ENGRAM_TRY(sort_resident_blocks<7>(&res[7]));
+    ENGRAM_TRY(sort_resident_blocks<8>(&res[8]));
+    int best = bwd::kSortItemsMax;
+    int64_t best_load = INT64_MAX;
+    for (int I = bwd::kSortItemsMax; I >= bwd::kSortItemsMin; --I) {
+        const int64_t tiles = shape_tiles(sh, I);
+        if (tiles > res[I])
+            continue;
+        const int64_t load = ceil_div(tiles, (int64_t)sms) * I;
+        if (load < best_load) {
+            best = I;
+            best_load = load;
+        }
+    }
+    *items = best;
+    return ENGRAM_OK;
+}
+
 uint32_t barrier_spin_limit();
+
+// Kernel arguments of a sort of `sh` on tiles of 256 * items pairs, inside
+// the workspace laid out by P.
+int sort_args(const int32_t *idx, const SortShape &sh, int items, const BwdPlan &P, char *ws,
+              bwd::SortArgs *out)
+{
+    using namespace bwd;
+    SortArgs &a = *out;
+    std::memset(&a, 0, sizeof(a));
+    int key_bits = 1;
+    for (int s = 0; s < sh.S; ++s)
+        key_bits = std::max(key_bits, bit_width((uint64_t)sh.size[s] - 1));
+    a.passes = (key_bits + kDigitBitsMax - 1) / kDigitBitsMax;
+    if (a.passes > kMaxPasses)
+        return ENGRAM_EINVAL;
+    for (int q = 0; q < a.passes; ++q) // spread the bits evenly, wider digits first
+        a.bits[q] = key_bits / a.passes + (q < key_bits % a.passes ? 1 : 0);
+    const int64_t tile = (int64_t)kSortThreads * items;
+    a.idx = idx;
+    a.a = (unsigned long long *)(ws + P.a);
+    a.b = (unsigned long long *)(ws + P.b);
+    a.S = sh.S;
+    a.L = sh.L;
+    a.n = (int64_t)sh.S * sh.L;
+    a.tps = (int)std::max<int64_t>(1, ceil_div(sh.L, tile));
+    a.gps = (int)ceil_div(a.tps, kTilesPerGroup);
+    a.ntiles = a.S * a.tps;
+    a.ngroups = a.S * a.gps;
+    if (a.ntiles > P.tiles_max || a.ngroups > P.groups_max)
+        return ENGRAM_EINVAL;
+    a.tile_cnt = (uint32_t *)(ws + P.tile_cnt);
+    a.group_cnt = (uint32_t *)(ws + P.group_cnt);
+    a.barrier = (unsigned *)(ws + P.barrier);
+    a.spin_limit = barrier_spin_limit();
+    for (int s = 0; s < sh.S; ++s) {
+        a.off[s] = sh.off[s];
+        a.size[s] = sh.size[s];
+    }
+    return ENGRAM_OK;
+}
 
 // The one-launch sort at I pairs per thread; *launched is false where the
 // device or the launch refuses a cooperative grid (nothing ran).
 template <int I>
-int launch_sort_coop(const int32_t *idx, int64_t n, int64_t rows, const BwdPlan &P, char *ws,
+int launch_sort_coop(const int32_t *idx, const SortShape &sh, const BwdPlan &P, char *ws,
                      cudaStream_t stream, bool *launched)
 {
     using namespace bwd;
@@ -299,14 +395,12 @@ int launch_sort_coop(const int32_t *idx, int64_t n, int64_t rows, const BwdPlan 
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess || !coop)
         return ENGRAM_OK;
+    SortArgs args;
+    ENGRAM_TRY(sort_args(idx, sh, I, P, ws, &args));
     // the grid is at most the co-resident blocks, which the launch itself checks
     int64_t res = 0;
     ENGRAM_TRY(resident_warps(radix_sort_coop<I>, kSortThreads, 0, &res));
-    const int grid = (int)std::min<int64_t>(P.ntiles, res / (kSortThreads / 32));
-    SortArgs args{idx, (unsigned long long *)(ws + P.a), (unsigned long long *)(ws + P.b), n,
-                  (uint32_t)rows, P.passes, P.ntiles, P.ngroups, (uint32_t *)(ws + P.tile_cnt),
-                  (uint32_t *)(ws + P.group_cnt), (unsigned *)(ws + P.barrier),
-                  barrier_spin_limit()};
+    const int grid = (int)std::min<int64_t>(args.ntiles, res / (kSortThreads / 32));
     void *params[] = {&args};
     if (cudaLaunchCooperativeKernel((const void *)radix_sort_coop<I>, dim3(grid),
                                     dim3(kSortThreads), params, 0, stream) != cudaSuccess) {
@@ -361,54 +455,42 @@ uint64_t cross_wait_ns()
     return v;
 }
 
-int launch_sort(const int32_t *idx, int64_t n, int64_t rows, const BwdPlan &P, char *ws,
+// Sorts the pairs of `sh` into buffer a of the workspace.
+int launch_sort(const int32_t *idx, const SortShape &sh, const BwdPlan &P, char *ws,
                 cudaStream_t stream)
 {
     using namespace bwd;
     if (cudaMemsetAsync(ws + P.ctl, 0, P.ctl_bytes, stream) != cudaSuccess)
         return ENGRAM_ECUDA;
     bool launched = false;
-    switch (sort_separate_launches() ? 0 : P.items) {
+    int items = 0;
+    if (!sort_separate_launches()) {
+        int sms = 0;
+        ENGRAM_TRY(device_sms(&sms));
+        ENGRAM_TRY(sort_items(sh, sms, &items));
+    }
+    switch (items) {
     case 0: break;
-    case 4: ENGRAM_TRY(launch_sort_coop<4>(idx, n, rows, P, ws, stream, &launched)); break;
-    case 5: ENGRAM_TRY(launch_sort_coop<5>(idx, n, rows, P, ws, stream, &launched)); break;
-    case 6: ENGRAM_TRY(launch_sort_coop<6>(idx, n, rows, P, ws, stream, &launched)); break;
-    case 7: ENGRAM_TRY(launch_sort_coop<7>(idx, n, rows, P, ws, stream, &launched)); break;
-    case 8: ENGRAM_TRY(launch_sort_coop<8>(idx, n, rows, P, ws, stream, &launched)); break;
+    case 4: ENGRAM_TRY(launch_sort_coop<4>(idx, sh, P, ws, stream, &launched)); break;
+    case 5: ENGRAM_TRY(launch_sort_coop<5>(idx, sh, P, ws, stream, &launched)); break;
+    case 6: ENGRAM_TRY(launch_sort_coop<6>(idx, sh, P, ws, stream, &launched)); break;
+    case 7: ENGRAM_TRY(launch_sort_coop<7>(idx, sh, P, ws, stream, &launched)); break;
+    case 8: ENGRAM_TRY(launch_sort_coop<8>(idx, sh, P, ws, stream, &launched)); break;
     default: return ENGRAM_EINVAL;
     }
     if (launched)
         return ENGRAM_OK;
 
     // Without a cooperative launch: two launches per pass, on the largest
-    // tiles (2,048 pairs; their counts take no more workspace than the plan's).
+    // tiles (2,048 pairs).
     constexpr int I = kSortItemsMax;
-    const int ntiles = (int)std::max<int64_t>(1, ceil_div(n, (int64_t)kSortThreads * I));
-    const int ngroups = (int)ceil_div(ntiles, kTilesPerGroup);
-    auto *A = (unsigned long long *)(ws + P.a);
-    auto *B = (unsigned long long *)(ws + P.b);
-    auto *tile_cnt = (uint32_t *)(ws + P.tile_cnt);
-    auto *group_cnt = (uint32_t *)(ws + P.group_cnt);
-    const void *src = idx;
-    for (int pass = 0; pass < P.passes; ++pass) {
-        unsigned long long *dst = (pass % 2 == 0) ? A : B;
-        uint32_t *gc = group_cnt + (size_t)pass * kRadix * ngroups;
-        const int shift = pass * kRadixBits;
-        if (pass == 0) {
-            radix_count<true, I><<<ntiles, kSortThreads, 0, stream>>>(src, n, shift,
-                                                                     (uint32_t)rows, tile_cnt, gc);
-            ENGRAM_TRY(after_launch());
-            radix_scatter<true, I><<<ntiles, kSortThreads, 0, stream>>>(src, dst, n, shift,
-                                                                       tile_cnt, gc, ngroups);
-        } else {
-            radix_count<false, I><<<ntiles, kSortThreads, 0, stream>>>(src, n, shift,
-                                                                      (uint32_t)rows, tile_cnt, gc);
-            ENGRAM_TRY(after_launch());
-            radix_scatter<false, I><<<ntiles, kSortThreads, 0, stream>>>(src, dst, n, shift,
-                                                                        tile_cnt, gc, ngroups);
-        }
+    SortArgs args;
+    ENGRAM_TRY(sort_args(idx, sh, I, P, ws, &args));
+    for (int pass = 0; pass < args.passes; ++pass) {
+        radix_count<I><<<args.ntiles, kSortThreads, 0, stream>>>(args, pass);
         ENGRAM_TRY(after_launch());
-        src = dst;
+        radix_scatter<I><<<args.ntiles, kSortThreads, 0, stream>>>(args, pass);
+        ENGRAM_TRY(after_launch());
     }
     return ENGRAM_OK;
 }
@@ -476,7 +558,7 @@ int launch_reduce(int64_t n, int32_t dim, const void *dout, int32_t dtype, int32
             return ENGRAM_ECUDA;
         return ENGRAM_OK;
     }
-    const auto *items = (const unsigned long long *)(ws + ((P.passes % 2 == 1) ? P.a : P.b));
+    const auto *items = (const unsigned long long *)(ws + P.a); // the sort's last pass wrote a
     switch (dtype) {
     case ENGRAM_F32:
         return launch_seg_dt<ENGRAM_F32>(items, n, P, dout, dim, uniq, grads, num_unique, ws,
@@ -498,6 +580,17 @@ int check_reduce_args(int64_t n, const void *dout, int32_t dtype, int32_t *uniq,
     if (n > 0 && (dout == nullptr || uniq == nullptr || grads == nullptr ||
                   !aligned16(dout) || !aligned16(grads)))
         return ENGRAM_EINVAL;
+    return ENGRAM_OK;
+}
+
+// The hash's lookups: n = T * H, lookup t * H + h in head h's slice.
+int heads_args(const engram_params_t *params, int64_t T, int64_t *n)
+{
+    HashArgs a;
+    ENGRAM_TRY(make_hash_args(params, &a));
+    if (T < 0 || T * a.H > INT32_MAX)
+        return ENGRAM_EINVAL;
+    *n = T * a.H;
     return ENGRAM_OK;
 }
 
@@ -611,7 +704,8 @@ int engram_backward_sort(const int32_t *idx, int64_t n, int64_t table_rows, int3
         return ENGRAM_OK;
     if (idx == nullptr)
         return ENGRAM_EINVAL;
-    return launch_sort(idx, n, table_rows, P, (char *)workspace, (cudaStream_t)stream);
+    return launch_sort(idx, plain_shape(n, table_rows), P, (char *)workspace,
+                       (cudaStream_t)stream);
 }
 
 int engram_backward_reduce(int64_t n, int64_t table_rows, int32_t dim, const void *dout,
@@ -640,8 +734,43 @@ int engram_backward(const int32_t *idx, int64_t n, int64_t table_rows, int32_t d
         return ENGRAM_EINVAL;
     cudaStream_t s = (cudaStream_t)stream;
     if (n > 0)
-        ENGRAM_TRY(launch_sort(idx, n, table_rows, P, (char *)workspace, s));
+        ENGRAM_TRY(launch_sort(idx, plain_shape(n, table_rows), P, (char *)workspace, s));
     return launch_reduce(n, dim, dout, dtype, uniq_rows, row_grads, num_unique, P,
+                         (char *)workspace, s);
+}
+
+int engram_backward_sort_heads(const engram_params_t *params, const int32_t *idx, int64_t T,
+                               void *workspace, size_t workspace_bytes, engram_stream_t stream)
+{
+    int64_t n = 0;
+    ENGRAM_TRY(heads_args(params, T, &n));
+    BwdPlan P;
+    ENGRAM_TRY(bwd_plan(n, params->table_rows, params->dim, &P));
+    ENGRAM_TRY(check_workspace(P, workspace, workspace_bytes));
+    if (n == 0)
+        return ENGRAM_OK;
+    if (idx == nullptr)
+        return ENGRAM_EINVAL;
+    return launch_sort(idx, head_shape(params, T), P, (char *)workspace, (cudaStream_t)stream);
+}
+
+int engram_backward_heads(const engram_params_t *params, const int32_t *idx, int64_t T,
+                          const void *dout, int32_t dtype, int32_t *uniq_rows, float *row_grads,
+                          int32_t *num_unique, void *workspace, size_t workspace_bytes,
+                          engram_stream_t stream)
+{
+    int64_t n = 0;
+    ENGRAM_TRY(heads_args(params, T, &n));
+    BwdPlan P;
+    ENGRAM_TRY(bwd_plan(n, params->table_rows, params->dim, &P));
+    ENGRAM_TRY(check_workspace(P, workspace, workspace_bytes));
+    ENGRAM_TRY(check_reduce_args(n, dout, dtype, uniq_rows, row_grads, num_unique));
+    if (n > 0 && idx == nullptr)
+        return ENGRAM_EINVAL;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (n > 0)
+        ENGRAM_TRY(launch_sort(idx, head_shape(params, T), P, (char *)workspace, s));
+    return launch_reduce(n, params->dim, dout, dtype, uniq_rows, row_grads, num_unique, P,
                          (char *)workspace, s);
 }
 
@@ -696,7 +825,7 @@ int engram_backward_noalloc(const int32_t *idx, int64_t n, int64_t table_rows, i
     cudaStream_t s = (cudaStream_t)stream;
     // launch_sort clears the sort's control block in the array on every call
     if (n > 0)
-        ENGRAM_TRY(launch_sort(idx, n, table_rows, P, ws, s));
+        ENGRAM_TRY(launch_sort(idx, plain_shape(n, table_rows), P, ws, s));
     return launch_reduce(n, dim, dout, dtype, uniq_rows, row_grads, num_unique, P, ws, s);
 }
 

@@ -156,7 +156,7 @@ __global__ void __launch_bounds__(kHashThreads)
         return;
     int64_t tb, te;
     warp_range(T, w, nwarps, tb, te);
-    int32_t s = cu != nullptr ? find_sequence(cu, nseq, tb) : 0;
+    int32_t s = cu != nullptr ? find_sequence_warp(cu, nseq, tb) : 0;
     for (int64_t t0 = tb; t0 < te; t0 += 32) {
         hash_chunk<NT, KT>(a, ids, cu, nseq, T, t0, te, s, s_idx, HP, lane);
         __syncwarp();
@@ -195,7 +195,8 @@ __global__ void __launch_bounds__(kHashThreads)
     warp_range(MAPPED ? nlog : T, w, nwarps, tb, te);
     if (tb >= te)
         return;
-    int32_t s = cu != nullptr ? find_sequence(cu, nseq, MAPPED ? slice_token(m, tb) : tb) : 0;
+    int32_t s = cu != nullptr ? find_sequence_warp(cu, nseq, MAPPED ? slice_token(m, tb) : tb)
+                              : 0;
 
     for (int64_t t0 = tb; t0 < te; t0 += 32) {
         hash_chunk<NT, KT, MAPPED>(a, ids, cu, nseq, T, t0, te, s, s_idx, HP, lane, m);
@@ -256,7 +257,7 @@ __global__ void __launch_bounds__(kHashThreads)
 // 32 x V chunk, taking each vector's row index from the owning lane by
 // shuffle, so stores stay fully coalesced for any V.
 template <int VT>
-__global__ void __launch_bounds__(kHashThreads)
+__global__ void __launch_bounds__(kHashThreads, 2)
     gather_kernel(const uint4 *__restrict__ table, int64_t rows, int v_rt,
                   const int32_t *__restrict__ idx, int64_t n, int64_t nwarps,
                   uint4 *__restrict__ out)

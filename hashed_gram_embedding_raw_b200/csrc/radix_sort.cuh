@@ -1,34 +1,50 @@
 // radix_sort.cuh -- stable LSD radix sort of the backward's (row, lookup) pairs.
 //
 // The pairs (idx[j], j) are packed as 64-bit items key << 32 | j and sorted by
-// key, 8 bits per pass, ceil(bits(table_rows - 1) / 8) passes. Because the
-// items start in j order and every pass is stable, equal keys end up in
-// ascending j.
+// key. Because the items enter each pass in ascending j and every pass is
+// stable, equal keys end up in ascending j.
 //
-// Each pass has two phases over tiles of 256 * ITEMS items (ITEMS <= 8 pairs
-// per thread, chosen per sort by the host so that the busiest SM holds as few
-// pairs as possible):
-//   count    a tile's digit counts are stored (tile-major, tile_cnt[tile][d])
-//            and added into per-group sums (group_cnt[group][d], 32 tiles per
-//            group; the adds commute, so the sums are deterministic);
-//   scatter  a tile ranks its items stably in shared memory (per-warp digit
+// Segments. A sort covers S segments of L positions each (n = S * L) and
+// sorts every segment on its own; the segments are laid out one after the
+// other. The plain sort is one segment holding all n lookups. The sort by
+// head uses the structure of the hash's output (engram API page,
+// Qwen3_8_FlashNextNGramEmbedding._hash_input_ids): lookup j = t * H + h of
+// token t and head h always lies in head h's own slice [o_h, o_h + p_h) of the
+// table, the slices are disjoint and ascend with h, and every head holds
+// exactly T lookups. So segment h takes head h's lookups (position h * T + t
+// holds lookup t * H + h), its keys are sorted as key - o_h, which needs only
+// bits(p_h - 1) bits (25 on the page's table, against 29 for the whole key),
+// and the concatenated segments are the whole sort. The last pass adds o_h
+// back, so both forms leave the same items.
+//
+// Passes take digits of up to 9 bits (the key's bits spread evenly over the
+// fewest passes), least significant first. Each pass has two phases over
+// tiles of 256 * ITEMS items (ITEMS = 4..8, chosen per sort by the host);
+// a tile never spans two segments:
+//   count    a tile's digit counts are stored (tile_cnt[tile][d]) and added
+//            into per-group sums (group_cnt[pass][group][d], groups of 32
+//            tiles inside one segment; the adds commute, so the sums are
+//            deterministic);
+//   place    a tile ranks its items stably in shared memory (per-warp digit
 //            counters, peers found with one ballot per digit bit), takes each
-//            digit's global offset as
-//              sum of all earlier digits' totals
+//            digit's position in its segment as
+//              sum of the earlier digits' totals in the segment
 //              + that digit's group sums before the tile's group
 //              + that digit's tile counts earlier in the group
-//            (a few dozen independent, coalesced loads per thread), and writes
-//            the tile out in contiguous runs staged through shared memory.
+//            (independent, coalesced loads), and writes the tile out in
+//            contiguous runs staged through shared memory.
 // No tile ever waits on another tile's result, so there is no serial prefix
-// chain across tiles.
+// chain across tiles. The last pass always writes buffer `a`, so the reduce
+// finds the sorted items in one place whatever the number of passes.
 //
 // radix_sort_coop runs every phase of every pass in one cooperative launch:
 // each resident block takes tiles blockIdx.x, blockIdx.x + gridDim.x, ... and
 // the phases are separated by a grid barrier on one arrival counter (bounded
-// wait; a timeout raises ENGRAM_DEVERR_SORT_TIMEOUT instead of hanging). Data written by other blocks
-// in the same launch is read through L2 (ld.global.cg), never through the
-// non-coherent load path. radix_count / radix_scatter run the same phases as
-// separate launches where cooperative launch is unavailable.
+// wait; a timeout raises ENGRAM_DEVERR_SORT_TIMEOUT instead of hanging). Data
+// written by other blocks in the same launch is read through L2
+// (ld.global.cg), never through the non-coherent load path. radix_count /
+// radix_scatter run the same phases as separate launches where cooperative
+// launch is unavailable.
 #pragma once
 
 #include "common.cuh"
@@ -37,41 +53,115 @@ namespace engram {
 namespace bwd {
 
 constexpr int kSortThreads = 256;
-constexpr int kSortItemsMax = 8; // pairs per thread of the largest tile (2048 pairs)
-constexpr int kRadixBits = 8;
-constexpr int kRadix = 1 << kRadixBits;
-constexpr int kMaxPasses = 4; // keys below 2^32
+constexpr int kSortItemsMin = 4;
+constexpr int kSortItemsMax = 8;   // pairs per thread of the largest tile (2048 pairs)
+constexpr int kDigitBitsMax = 9;
+constexpr int kRadixMax = 1 << kDigitBitsMax;
+constexpr int kMaxPasses = 4;      // keys below 2^32 at <= 9 bits per pass
 constexpr int kSortWarps = kSortThreads / 32;
 constexpr int kTilesPerGroup = 32;
+constexpr int kMaxSegments = ENGRAM_MAX_HEADS;
 constexpr uint32_t kBarrierSpin = 1u << 22; // polls (~64 ns apart) before a barrier gives up
-static_assert(kRadix == kSortThreads, "one thread per digit");
+static_assert(kRadixMax == 2 * kSortThreads, "at most two digits per thread");
+
+struct SortArgs {
+    const int32_t *idx;
+    unsigned long long *a, *b; // ping-pong item buffers; the last pass writes a
+    int64_t n;                 // S * L
+    int64_t L;                 // positions per segment
+    int S;                     // segments
+    int passes;
+    int bits[kMaxPasses];      // digit width of each pass, least significant first
+    int tps, gps;              // tiles and 32-tile groups per segment
+    int ntiles, ngroups;       // S * tps, S * gps
+    uint32_t *tile_cnt;        // [ntiles][kRadixMax], rewritten every pass
+    uint32_t *group_cnt;       // [passes][ngroups][kRadixMax], zero on entry
+    unsigned *barrier;         // grid-barrier arrival counter; zero on entry
+    uint32_t spin_limit;       // polls before a grid-barrier wait gives up
+    int32_t off[kMaxSegments]; // segment s holds keys off[s] .. off[s] + size[s] - 1
+    uint32_t size[kMaxSegments];
+};
 
 __device__ __forceinline__ uint32_t item_key(uint64_t it) { return (uint32_t)(it >> 32); }
 
+// One pass: its digit is bits [shift, shift + bits) of the (segment-relative) key.
+struct PassInfo {
+    int shift, bits, ndig, dpt; // dpt: digits per thread (1, or 2 above 8 bits)
+    bool first, last;
+};
+
+__device__ __forceinline__ PassInfo pass_info(const SortArgs &a, int p)
+{
+    PassInfo q;
+    q.shift = 0;
+    for (int k = 0; k < p; ++k)
+        q.shift += a.bits[k];
+    q.bits = a.bits[p];
+    q.ndig = 1 << q.bits;
+    q.dpt = q.ndig > kSortThreads ? 2 : 1;
+    q.first = p == 0;
+    q.last = p == a.passes - 1;
+    return q;
+}
+
+__device__ __forceinline__ uint32_t digit_of(uint64_t x, const PassInfo &P)
+{
+    return (item_key(x) >> P.shift) & (uint32_t)(P.ndig - 1);
+}
+
+// Pass p writes `out_buffer(a, p)` and reads the previous pass's output; the
+// parity is set so that the last pass writes a.
+__device__ __forceinline__ unsigned long long *out_buffer(const SortArgs &a, int p)
+{
+    return ((a.passes - 1 - p) & 1) == 0 ? a.a : a.b;
+}
+
+struct TileGeom {
+    int seg;       // segment of the tile
+    int k;         // tile index inside the segment
+    int64_t begin; // first position
+    int count;     // positions (the segment's last tile may be short)
+};
+
+__device__ __forceinline__ TileGeom tile_geom(const SortArgs &a, int tile, int tile_items)
+{
+    TileGeom g;
+    g.seg = tile / a.tps;
+    g.k = tile - g.seg * a.tps;
+    const int64_t lo = (int64_t)g.k * tile_items;
+    g.begin = (int64_t)g.seg * a.L + lo;
+    g.count = (int)min64(tile_items, a.L - lo);
+    return g;
+}
+
 template <int ITEMS> struct SortSmem {
     static constexpr int kTile = kSortThreads * ITEMS;
-    uint32_t whist[kSortWarps][kRadix];
-    uint32_t tstart[kRadix];
-    uint32_t gbase[kRadix];
-    uint32_t cnt[kRadix];
+    uint32_t whist[kSortWarps][kRadixMax];
+    uint32_t tstart[kRadixMax];
+    uint32_t gbase[kRadixMax];
+    uint32_t cnt[kRadixMax];
     uint32_t warp[32];
     unsigned long long warp2[32];
     unsigned long long items[kTile];
     int flag;
 };
 
-// Item i of a pass: pass 0 forms it from the int32 index, later passes read it.
+// Item at position i (0 <= i < count) of a tile. The first pass forms it from
+// the int32 index of lookup j = (k * TILE + i) * S + seg, keyed relative to
+// the segment's first row; later passes read the previous pass's output.
 // COHERENT loads go through L2 only (needed when another block of the same
-// launch wrote the data); otherwise the read-only path is used.
+// launch wrote the data).
 template <bool COHERENT>
-__device__ __forceinline__ uint64_t load_item(const void *__restrict__ src, bool first, int64_t i)
+__device__ __forceinline__ uint64_t load_item(const SortArgs &a, const void *__restrict__ src,
+                                              bool first, const TileGeom &g, int tile_items,
+                                              int i)
 {
     if (first) {
-        const int32_t *p = (const int32_t *)src + i;
-        const uint32_t key = (uint32_t)(COHERENT ? __ldcg(p) : __ldg(p));
-        return ((uint64_t)key << 32) | (uint32_t)i;
+        const int64_t j = ((int64_t)g.k * tile_items + i) * a.S + g.seg;
+        const uint32_t key = (uint32_t)__ldg(a.idx + j) - (uint32_t)a.off[g.seg];
+        return ((uint64_t)key << 32) | (uint32_t)j;
     }
-    const unsigned long long *p = (const unsigned long long *)src + i;
+    const unsigned long long *p = (const unsigned long long *)src + g.begin + i;
     return COHERENT ? __ldcg(p) : __ldg(p);
 }
 
@@ -81,85 +171,103 @@ __device__ __forceinline__ uint32_t load_u32(const uint32_t *p)
     return COHERENT ? __ldcg(p) : __ldg(p);
 }
 
-// Lanes of the warp whose digit equals this lane's (valid lanes only).
-__device__ __forceinline__ uint32_t digit_peers(uint32_t dg, bool valid)
+// Lanes of the warp whose digit equals this lane's (valid lanes only); `bits`
+// is the same on every lane.
+__device__ __forceinline__ uint32_t digit_peers(uint32_t dg, bool valid, int bits)
 {
     uint32_t peers = __ballot_sync(kFull, valid);
 #pragma unroll
-    for (int bit = 0; bit < kRadixBits; ++bit) {
-        const bool on = (dg >> bit) & 1u;
-        const uint32_t bal = __ballot_sync(kFull, on);
-        peers &= on ? bal : ~bal;
+    for (int bit = 0; bit < kDigitBitsMax; ++bit) {
+        if (bit < bits) {
+            const bool on = (dg >> bit) & 1u;
+            const uint32_t bal = __ballot_sync(kFull, on);
+            peers &= on ? bal : ~bal;
+        }
     }
     return peers;
 }
 
-// Count phase of one tile. Pass 0 also flags keys outside [0, rows).
-template <bool COHERENT, int ITEMS>
-__device__ __forceinline__ void count_tile(SortSmem<ITEMS> &sm, const void *src, bool first, int64_t n,
-                                           int shift, uint32_t rows, int tile,
-                                           uint32_t *tile_cnt, uint32_t *group_cnt)
+// Digit d of this thread's slot e (digits tid * dpt + e, consecutive per thread).
+__device__ __forceinline__ int my_digit(const PassInfo &P, int e)
 {
+    return threadIdx.x * P.dpt + e;
+}
+
+// Count phase of one tile (separate-launch form). The first pass also flags
+// keys outside their segment's rows.
+template <int ITEMS>
+__device__ __forceinline__ void count_tile(SortSmem<ITEMS> &sm, const SortArgs &a,
+                                           const void *src, const PassInfo &P, int tile,
+                                           uint32_t *gc)
+{
+    constexpr int TILE = SortSmem<ITEMS>::kTile;
     const int tid = threadIdx.x, lane = tid & 31;
-    sm.cnt[tid] = 0;
+    const TileGeom g = tile_geom(a, tile, TILE);
+    for (int d = tid; d < P.ndig; d += kSortThreads)
+        sm.cnt[d] = 0;
     __syncthreads();
-    const int64_t base = (int64_t)tile * SortSmem<ITEMS>::kTile;
     uint32_t key[ITEMS];
 #pragma unroll
     for (int r = 0; r < ITEMS; ++r) {
-        const int64_t i = base + r * kSortThreads + tid;
-        key[r] = i < n ? item_key(load_item<COHERENT>(src, first, i)) : 0u;
+        const int i = r * kSortThreads + tid;
+        key[r] = i < g.count ? item_key(load_item<false>(a, src, P.first, g, TILE, i)) : 0u;
     }
     bool bad = false;
 #pragma unroll
     for (int r = 0; r < ITEMS; ++r) {
-        const bool valid = base + r * kSortThreads + tid < n;
-        if (first && valid && key[r] >= rows)
+        const bool valid = r * kSortThreads + tid < g.count;
+        if (P.first && valid && key[r] >= a.size[g.seg])
             bad = true;
         // one shared-memory add per distinct digit in the warp, so runs of a
         // hot key do not serialise on one counter
-        const uint32_t dg = (key[r] >> shift) & (kRadix - 1);
-        const uint32_t peers = digit_peers(dg, valid);
+        const uint32_t dg = (key[r] >> P.shift) & (uint32_t)(P.ndig - 1);
+        const uint32_t peers = digit_peers(dg, valid, P.bits);
         if (valid && lane == __ffs(peers) - 1)
             atomicAdd(&sm.cnt[dg], (uint32_t)__popc(peers));
     }
     if (bad)
         raise_device_error(ENGRAM_DEVERR_ROW_RANGE);
     __syncthreads();
-    const uint32_t c = sm.cnt[tid];
-    tile_cnt[(size_t)tile * kRadix + tid] = c;
-    if (c)
-        atomicAdd(&group_cnt[(size_t)(tile / kTilesPerGroup) * kRadix + tid], c);
+    const int grp = g.seg * a.gps + g.k / kTilesPerGroup;
+    for (int d = tid; d < P.ndig; d += kSortThreads) {
+        const uint32_t c = sm.cnt[d];
+        a.tile_cnt[(size_t)tile * kRadixMax + d] = c;
+        if (c)
+            atomicAdd(&gc[(size_t)grp * kRadixMax + d], c);
+    }
     __syncthreads(); // sm.cnt free for the next tile
 }
 
 // Loads the tile's items and ranks them stably: rank[r] is item r's position
 // among the items of its digit in its warp, and sm.whist[w][d] ends up as the
-// number of items of digit d in warp w. Pass 0 also flags keys outside the table.
+// number of items of digit d in warp w. The first pass also flags keys outside
+// their segment's rows (check_keys).
 template <bool COHERENT, int ITEMS>
-__device__ __forceinline__ void rank_tile(SortSmem<ITEMS> &sm, const void *src, bool first,
-                                          int64_t n, int shift, uint32_t rows, int tile,
-                                          uint64_t (&it)[ITEMS], uint32_t (&rank)[ITEMS])
+__device__ __forceinline__ void rank_tile(SortSmem<ITEMS> &sm, const SortArgs &a,
+                                          const void *src, const PassInfo &P, const TileGeom &g,
+                                          bool check_keys, uint64_t (&it)[ITEMS],
+                                          uint32_t (&rank)[ITEMS])
 {
+    constexpr int TILE = SortSmem<ITEMS>::kTile;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    for (int k = tid; k < kSortWarps * kRadix; k += kSortThreads)
-        (&sm.whist[0][0])[k] = 0;
-    const int64_t wbase = (int64_t)tile * SortSmem<ITEMS>::kTile + (int64_t)wid * (32 * ITEMS);
+    for (int k = tid; k < (kSortWarps << P.bits); k += kSortThreads)
+        sm.whist[k >> P.bits][k & (P.ndig - 1)] = 0;
+    const int wbase = wid * (32 * ITEMS);
     const uint32_t lt = lanemask_lt();
 #pragma unroll
     for (int r = 0; r < ITEMS; ++r) {
-        const int64_t i = wbase + r * 32 + lane;
-        it[r] = i < n ? load_item<COHERENT>(src, first, i) : 0ull;
+        const int i = wbase + r * 32 + lane;
+        it[r] = i < g.count ? load_item<COHERENT>(a, src, P.first, g, TILE, i) : 0ull;
     }
     __syncthreads(); // whist zeroed
     bool bad = false;
 #pragma unroll
     for (int r = 0; r < ITEMS; ++r) {
-        const bool valid = wbase + r * 32 + lane < n;
-        if (first && valid && item_key(it[r]) >= rows)
+        const bool valid = wbase + r * 32 + lane < g.count;
+        if (check_keys && valid && item_key(it[r]) >= a.size[g.seg])
             bad = true;
-        const uint32_t dg = (item_key(it[r]) >> shift) & (kRadix - 1);
-        const uint32_t peers = digit_peers(dg, valid);
+        const uint32_t dg = digit_of(it[r], P);
+        const uint32_t peers = digit_peers(dg, valid, P.bits);
         const int leader = valid ? __ffs(peers) - 1 : lane;
         uint32_t cnt = 0;
         if (valid && lane == leader) {
@@ -175,230 +283,275 @@ __device__ __forceinline__ void rank_tile(SortSmem<ITEMS> &sm, const void *src, 
     __syncthreads();
 }
 
-// Thread d: turns sm.whist[.][d] into per-warp exclusive offsets and returns
-// the tile's count of digit d.
-template <int ITEMS> __device__ __forceinline__ uint32_t tile_digit_count(SortSmem<ITEMS> &sm)
+// For this thread's digits: turns sm.whist[.][d] into per-warp exclusive
+// offsets and returns the tile's count of each digit in tcount[e].
+template <int ITEMS>
+__device__ __forceinline__ void tile_digit_count(SortSmem<ITEMS> &sm, const PassInfo &P,
+                                                 uint32_t (&tcount)[2])
 {
-    const int d = threadIdx.x;
-    uint32_t tcount = 0;
 #pragma unroll
-    for (int w = 0; w < kSortWarps; ++w) {
-        const uint32_t c = sm.whist[w][d];
-        sm.whist[w][d] = tcount;
-        tcount += c;
+    for (int e = 0; e < 2; ++e) {
+        const int d = my_digit(P, e);
+        uint32_t run = 0;
+        if (e < P.dpt && d < P.ndig) {
+#pragma unroll
+            for (int w = 0; w < kSortWarps; ++w) {
+                const uint32_t c = sm.whist[w][d];
+                sm.whist[w][d] = run;
+                run += c;
+            }
+        }
+        tcount[e] = run;
     }
-    return tcount;
 }
 
-// Stores a tile's digit counts (tile-major) and adds them into its group's sums.
-__device__ __forceinline__ void publish_counts(int tile, uint32_t tcount, uint32_t *tile_cnt,
-                                               uint32_t *group_cnt)
+// Stores a tile's digit counts and adds them into its group's sums.
+__device__ __forceinline__ void publish_counts(const SortArgs &a, const PassInfo &P, int tile,
+                                               const TileGeom &g, const uint32_t (&tcount)[2],
+                                               uint32_t *gc)
 {
-    const int d = threadIdx.x;
-    tile_cnt[(size_t)tile * kRadix + d] = tcount;
-    if (tcount)
-        atomicAdd(&group_cnt[(size_t)(tile / kTilesPerGroup) * kRadix + d], tcount);
+    const int grp = g.seg * a.gps + g.k / kTilesPerGroup;
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+        const int d = my_digit(P, e);
+        if (e < P.dpt && d < P.ndig) {
+            a.tile_cnt[(size_t)tile * kRadixMax + d] = tcount[e];
+            if (tcount[e])
+                atomicAdd(&gc[(size_t)grp * kRadixMax + d], tcount[e]);
+        }
+    }
 }
 
-// Once every tile of the pass has published its counts: sm.tstart[d] = the
-// start of digit d = threadIdx.x in the tile, sm.gbase[d] = its global start
-// minus that. tcount is digit d's count in the tile.
+// Tile-local start of each of this thread's digits into sm.tstart (an
+// exclusive scan of the tile's digit counts over the block).
+template <int ITEMS>
+__device__ __forceinline__ void local_starts(SortSmem<ITEMS> &sm, const PassInfo &P,
+                                             const uint32_t (&tcount)[2])
+{
+    uint32_t tstart = block_exclusive_scan(tcount[0] + tcount[1], sm.warp, nullptr);
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+        const int d = my_digit(P, e);
+        if (e < P.dpt && d < P.ndig) {
+            sm.tstart[d] = tstart;
+            tstart += tcount[e];
+        }
+    }
+    __syncthreads();
+}
+
+// Ranks a tile, counts its digits (publishing the counts when `gc` is not
+// null) and leaves its items in sm.items ordered by digit, stably; tcount[e]
+// is the tile's count of this thread's digit e. Only the counts stay in
+// registers afterwards.
 template <bool COHERENT, int ITEMS>
-__device__ __forceinline__ void tile_offsets(SortSmem<ITEMS> &sm, int tile, uint32_t tcount,
-                                             const uint32_t *tile_cnt,
-                                             const uint32_t *group_cnt, int ngroups)
+__device__ __forceinline__ void stage_tile(SortSmem<ITEMS> &sm, const SortArgs &a,
+                                           const void *src, const PassInfo &P, int tile,
+                                           const TileGeom &g, bool check_keys, uint32_t *gc,
+                                           uint32_t (&tcount)[2])
+{
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    uint64_t it[ITEMS];
+    uint32_t rank[ITEMS];
+    rank_tile<COHERENT>(sm, a, src, P, g, check_keys, it, rank);
+    tile_digit_count(sm, P, tcount);
+    if (gc != nullptr)
+        publish_counts(a, P, tile, g, tcount, gc);
+    local_starts(sm, P, tcount);
+    const int wbase = wid * (32 * ITEMS);
+#pragma unroll
+    for (int r = 0; r < ITEMS; ++r) {
+        if (wbase + r * 32 + lane < g.count) {
+            const uint32_t dg = digit_of(it[r], P);
+            sm.items[sm.tstart[dg] + sm.whist[wid][dg] + rank[r]] = it[r];
+        }
+    }
+    __syncthreads();
+}
+
+// Once every tile of the pass has published its counts: sm.gbase[d] = the
+// position in the output of digit d's first item in the tile, minus
+// sm.tstart[d] (which WITH_TSTART computes here from tcount; otherwise
+// local_starts already has). tcount[e] is the tile's count of this thread's
+// digit e.
+template <bool COHERENT, bool WITH_TSTART, int ITEMS>
+__device__ __forceinline__ void tile_offsets(SortSmem<ITEMS> &sm, const SortArgs &a,
+                                             const PassInfo &P, const TileGeom &g,
+                                             const uint32_t (&tcount)[2], const uint32_t *gc)
 {
     // Counts are tile- and group-major, so each load instruction reads 32
     // consecutive digits; the loops are unrolled so the loads are in flight
     // together.
-    const int d = threadIdx.x;
-    const int grp = tile / kTilesPerGroup;
-    uint32_t excl = 0, total = 0;
-    for (int g0 = 0; g0 < ngroups; g0 += 8) {
-        uint32_t c[8];
+    const int kg = g.k / kTilesPerGroup;
+    const uint32_t *segg = gc + (size_t)g.seg * a.gps * kRadixMax;
+    const uint32_t *segt = a.tile_cnt + (size_t)g.seg * a.tps * kRadixMax;
+    uint32_t total[2] = {0u, 0u}, excl[2] = {0u, 0u};
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
-            c[q] = g0 + q < ngroups
-                       ? load_u32<COHERENT>(group_cnt + (size_t)(g0 + q) * kRadix + d)
-                       : 0u;
+    for (int e = 0; e < 2; ++e) {
+        const int d = my_digit(P, e);
+        if (e < P.dpt && d < P.ndig) {
+            for (int g0 = 0; g0 < a.gps; g0 += 8) {
+                uint32_t c[8];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            total += c[q];
-            if (g0 + q < grp)
-                excl += c[q];
+                for (int q = 0; q < 8; ++q)
+                    c[q] = g0 + q < a.gps
+                               ? load_u32<COHERENT>(segg + (size_t)(g0 + q) * kRadixMax + d)
+                               : 0u;
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    total[e] += c[q];
+                    if (g0 + q < kg)
+                        excl[e] += c[q];
+                }
+            }
+            const int t0 = kg * kTilesPerGroup;
+            for (int q0 = 0; q0 < kTilesPerGroup; q0 += 16) {
+                uint32_t c[16];
+#pragma unroll
+                for (int q = 0; q < 16; ++q)
+                    c[q] = t0 + q0 + q < g.k
+                               ? load_u32<COHERENT>(segt + (size_t)(t0 + q0 + q) * kRadixMax + d)
+                               : 0u;
+#pragma unroll
+                for (int q = 0; q < 16; ++q)
+                    excl[e] += c[q];
+            }
         }
     }
-    {
-        const int t0 = grp * kTilesPerGroup;
-        uint32_t c[kTilesPerGroup];
-#pragma unroll
-        for (int q = 0; q < kTilesPerGroup; ++q)
-            c[q] = t0 + q < tile ? load_u32<COHERENT>(tile_cnt + (size_t)(t0 + q) * kRadix + d)
-                                 : 0u;
-#pragma unroll
-        for (int q = 0; q < kTilesPerGroup; ++q)
-            excl += c[q];
-    }
 
-    // One scan over digits gives both the tile-local start (low half) and the
-    // start of the digit among all digits (high half).
-    const unsigned long long both = block_exclusive_scan64(
-        ((unsigned long long)total << 32) | tcount, (unsigned long long *)sm.warp2);
-    const uint32_t tstart = (uint32_t)both, dbase = (uint32_t)(both >> 32);
-    sm.tstart[d] = tstart;
-    sm.gbase[d] = dbase + excl - tstart;
+    // The start of each digit in the segment is a scan over the threads'
+    // digits; with WITH_TSTART the same scan also gives the tile-local start
+    // (low half).
+    const uint32_t seg_base = (uint32_t)(g.seg * a.L);
+    uint32_t dbase, tstart = 0;
+    if constexpr (WITH_TSTART) {
+        const unsigned long long both = block_exclusive_scan64(
+            ((unsigned long long)(total[0] + total[1]) << 32) | (tcount[0] + tcount[1]),
+            (unsigned long long *)sm.warp2);
+        tstart = (uint32_t)both;
+        dbase = (uint32_t)(both >> 32);
+    } else {
+        dbase = block_exclusive_scan(total[0] + total[1], sm.warp, nullptr);
+    }
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+        const int d = my_digit(P, e);
+        if (e < P.dpt && d < P.ndig) {
+            if constexpr (WITH_TSTART) {
+                sm.tstart[d] = tstart;
+                tstart += tcount[e];
+            }
+            sm.gbase[d] = seg_base + dbase + excl[e] - sm.tstart[d];
+            dbase += total[e];
+        }
+    }
     __syncthreads();
 }
 
-// Writes a ranked tile to its sorted positions, once every tile of the pass
-// has published its counts. tcount is digit threadIdx.x's count in the tile.
-template <bool COHERENT, int ITEMS>
-__device__ __forceinline__ void place_tile(SortSmem<ITEMS> &sm, unsigned long long *dst,
-                                           int64_t n, int shift, int tile, uint32_t tcount,
-                                           const uint64_t (&it)[ITEMS],
-                                           const uint32_t (&rank)[ITEMS],
-                                           const uint32_t *tile_cnt, const uint32_t *group_cnt,
-                                           int ngroups)
+// The item as the pass writes it: the last pass turns the segment-relative
+// key back into the row.
+__device__ __forceinline__ unsigned long long out_item(unsigned long long x, const SortArgs &a,
+                                                      const PassInfo &P, int seg)
 {
-    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    tile_offsets<COHERENT>(sm, tile, tcount, tile_cnt, group_cnt, ngroups);
+    return P.last ? x + ((unsigned long long)(uint32_t)a.off[seg] << 32) : x;
+}
 
-    const int64_t wbase = (int64_t)tile * SortSmem<ITEMS>::kTile + (int64_t)wid * (32 * ITEMS);
-#pragma unroll
-    for (int r = 0; r < ITEMS; ++r) {
-        if (wbase + r * 32 + lane < n) {
-            const uint32_t dg = (item_key(it[r]) >> shift) & (kRadix - 1);
-            sm.items[sm.tstart[dg] + sm.whist[wid][dg] + rank[r]] = it[r];
-        }
-    }
-    __syncthreads();
-    const int64_t base = (int64_t)tile * SortSmem<ITEMS>::kTile;
-    const int tile_n = (int)min64(SortSmem<ITEMS>::kTile, n - base);
-    for (int p = tid; p < tile_n; p += kSortThreads) {
+// Writes a staged tile (sm.items, ordered by digit) to its sorted positions,
+// once every tile of the pass has published its counts.
+template <bool COHERENT, int ITEMS>
+__device__ __forceinline__ void place_staged_tile(SortSmem<ITEMS> &sm, const SortArgs &a,
+                                                  const PassInfo &P, unsigned long long *dst,
+                                                  const TileGeom &g,
+                                                  const uint32_t (&tcount)[2],
+                                                  const uint32_t *gc)
+{
+    tile_offsets<COHERENT, false>(sm, a, P, g, tcount, gc);
+    for (int p = threadIdx.x; p < g.count; p += kSortThreads) {
         const unsigned long long x = sm.items[p];
-        const uint32_t dg = (item_key(x) >> shift) & (kRadix - 1);
-        dst[(uint32_t)(sm.gbase[dg] + (uint32_t)p)] = x;
+        dst[(uint32_t)(sm.gbase[digit_of(x, P)] + (uint32_t)p)] = out_item(x, a, P, g.seg);
     }
     __syncthreads(); // shared memory free for the next tile
 }
 
-// Scatter phase of one tile after a separate count phase: rank, then place.
-template <bool COHERENT, int ITEMS>
-__device__ __forceinline__ void scatter_tile(SortSmem<ITEMS> &sm, const void *src, bool first,
-                                             unsigned long long *dst, int64_t n, int shift,
-                                             int tile, const uint32_t *tile_cnt,
-                                             const uint32_t *group_cnt, int ngroups)
-{
-    uint64_t it[ITEMS];
-    uint32_t rank[ITEMS];
-    // (the count phase has already checked the keys against the table)
-    rank_tile<COHERENT>(sm, src, first, n, shift, 0xffffffffu, tile, it, rank);
-    const uint32_t tcount = tile_digit_count(sm);
-    place_tile<COHERENT>(sm, dst, n, shift, tile, tcount, it, rank, tile_cnt, group_cnt,
-                         ngroups);
-}
-
 // Count phase of the one-launch sort when tiles outnumber the resident
-// blocks (a block cannot keep its tiles' items and ranks across the barrier):
-// ranks the tile, publishes its digit counts and writes it back ordered by
-// digit, stably, into its own region of `ordered`, so that the place phase
-// need not rank it again. `ordered` may be `src` itself (the tile region is
-// read before it is written, by this block alone).
+// blocks (a block cannot keep its tiles across the barrier): stages the tile
+// and writes it back ordered by digit into its own region of `ordered`, so
+// that the place phase need not rank it again. `ordered` may be `src` itself
+// (the tile region is read before it is written, by this block alone).
 template <int ITEMS>
-__device__ __forceinline__ void count_order_tile(SortSmem<ITEMS> &sm, const void *src, bool first,
-                                                 int64_t n, int shift, uint32_t rows, int tile,
-                                                 uint32_t *tile_cnt, uint32_t *group_cnt,
-                                                 unsigned long long *ordered)
+__device__ __forceinline__ void count_order_tile(SortSmem<ITEMS> &sm, const SortArgs &a,
+                                                 const void *src, const PassInfo &P, int tile,
+                                                 uint32_t *gc, unsigned long long *ordered)
 {
-    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    uint64_t it[ITEMS];
-    uint32_t rank[ITEMS];
-    rank_tile<true>(sm, src, first, n, shift, rows, tile, it, rank);
-    const uint32_t tcount = tile_digit_count(sm);
-    publish_counts(tile, tcount, tile_cnt, group_cnt);
-    sm.tstart[tid] = block_exclusive_scan(tcount, sm.warp, nullptr);
-    __syncthreads();
-    const int64_t base = (int64_t)tile * SortSmem<ITEMS>::kTile;
-    const int64_t wbase = base + (int64_t)wid * (32 * ITEMS);
-#pragma unroll
-    for (int r = 0; r < ITEMS; ++r) {
-        if (wbase + r * 32 + lane < n) {
-            const uint32_t dg = (item_key(it[r]) >> shift) & (kRadix - 1);
-            sm.items[sm.tstart[dg] + sm.whist[wid][dg] + rank[r]] = it[r];
-        }
-    }
-    __syncthreads();
-    const int tile_n = (int)min64(SortSmem<ITEMS>::kTile, n - base);
-    for (int q = tid; q < tile_n; q += kSortThreads)
-        ordered[base + q] = sm.items[q];
+    const TileGeom g = tile_geom(a, tile, SortSmem<ITEMS>::kTile);
+    uint32_t tcount[2];
+    stage_tile<true>(sm, a, src, P, tile, g, P.first, gc, tcount);
+    for (int q = threadIdx.x; q < g.count; q += kSortThreads)
+        ordered[g.begin + q] = sm.items[q];
     __syncthreads(); // shared memory free for the next tile
 }
 
 // Place phase for a tile that count_order_tile left ordered by digit: each
-// run of one digit goes to that digit's global offsets.
+// run of one digit goes to that digit's positions.
 template <int ITEMS>
-__device__ __forceinline__ void place_ordered_tile(SortSmem<ITEMS> &sm,
+__device__ __forceinline__ void place_ordered_tile(SortSmem<ITEMS> &sm, const SortArgs &a,
+                                                   const PassInfo &P,
                                                    const unsigned long long *ordered,
-                                                   unsigned long long *dst, int64_t n, int shift,
-                                                   int tile, const uint32_t *tile_cnt,
-                                                   const uint32_t *group_cnt, int ngroups)
+                                                   unsigned long long *dst, int tile,
+                                                   const uint32_t *gc)
 {
-    const int tid = threadIdx.x;
-    const uint32_t tcount = __ldcg(tile_cnt + (size_t)tile * kRadix + tid);
-    tile_offsets<true>(sm, tile, tcount, tile_cnt, group_cnt, ngroups);
-    const int64_t base = (int64_t)tile * SortSmem<ITEMS>::kTile;
-    const int tile_n = (int)min64(SortSmem<ITEMS>::kTile, n - base);
-    for (int q = tid; q < tile_n; q += kSortThreads) {
-        const unsigned long long x = __ldcg(ordered + base + q);
-        const uint32_t dg = (item_key(x) >> shift) & (kRadix - 1);
-        dst[(uint32_t)(sm.gbase[dg] + (uint32_t)q)] = x;
+    const TileGeom g = tile_geom(a, tile, SortSmem<ITEMS>::kTile);
+    uint32_t tcount[2] = {0u, 0u};
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+        const int d = my_digit(P, e);
+        if (e < P.dpt && d < P.ndig)
+            tcount[e] = __ldcg(a.tile_cnt + (size_t)tile * kRadixMax + d);
+    }
+    tile_offsets<true, true>(sm, a, P, g, tcount, gc);
+    for (int q = threadIdx.x; q < g.count; q += kSortThreads) {
+        const unsigned long long x = __ldcg(ordered + g.begin + q);
+        dst[(uint32_t)(sm.gbase[digit_of(x, P)] + (uint32_t)q)] = out_item(x, a, P, g.seg);
     }
     __syncthreads(); // shared memory free for the next tile
 }
 
 // ----------------------------------------------- one launch per phase
 
-template <bool FIRST, int ITEMS>
-__global__ void __launch_bounds__(kSortThreads)
-    radix_count(const void *__restrict__ src, int64_t n, int shift, uint32_t rows,
-                uint32_t *__restrict__ tile_cnt, uint32_t *__restrict__ group_cnt)
+template <int ITEMS>
+__global__ void __launch_bounds__(kSortThreads) radix_count(SortArgs a, int pass)
 {
     __shared__ SortSmem<ITEMS> sm;
-    count_tile<false>(sm, src, FIRST, n, shift, rows, blockIdx.x, tile_cnt, group_cnt);
+    const PassInfo P = pass_info(a, pass);
+    const void *src = P.first ? nullptr : out_buffer(a, pass - 1);
+    count_tile(sm, a, src, P, blockIdx.x, a.group_cnt + (size_t)pass * a.ngroups * kRadixMax);
 }
 
-template <bool FIRST, int ITEMS>
-__global__ void __launch_bounds__(kSortThreads)
-    radix_scatter(const void *__restrict__ src, unsigned long long *__restrict__ dst,
-                  int64_t n, int shift, const uint32_t *__restrict__ tile_cnt,
-                  const uint32_t *__restrict__ group_cnt, int ngroups)
+template <int ITEMS>
+__global__ void __launch_bounds__(kSortThreads) radix_scatter(SortArgs a, int pass)
 {
     __shared__ SortSmem<ITEMS> sm;
-    scatter_tile<false>(sm, src, FIRST, dst, n, shift, blockIdx.x, tile_cnt, group_cnt,
-                        ngroups);
+    const PassInfo P = pass_info(a, pass);
+    const void *src = P.first ? nullptr : out_buffer(a, pass - 1);
+    const TileGeom g = tile_geom(a, blockIdx.x, SortSmem<ITEMS>::kTile);
+    uint32_t tcount[2];
+    // (the count phase has already published the counts and checked the keys)
+    stage_tile<false>(sm, a, src, P, blockIdx.x, g, false, nullptr, tcount);
+    place_staged_tile<false>(sm, a, P, out_buffer(a, pass), g, tcount,
+                             a.group_cnt + (size_t)pass * a.ngroups * kRadixMax);
 }
 
 // ------------------------------------------------ one cooperative launch
-
-struct SortArgs {
-    const int32_t *idx;
-    unsigned long long *a, *b; // ping-pong item buffers; pass p writes (p even ? a : b)
-    int64_t n;
-    uint32_t rows;
-    int passes, ntiles, ngroups;
-    uint32_t *tile_cnt;  // [ntiles][256], rewritten every pass
-    uint32_t *group_cnt; // [passes][ngroups][256], zero on entry
-    unsigned *barrier;   // grid-barrier arrival counter; zero on entry
-    uint32_t spin_limit; // polls before a grid-barrier wait gives up (<= kBarrierSpin)
-};
 
 // Grid-wide barrier among co-resident blocks on one arrival counter that only
 // grows: barrier k of the launch is passed once the counter reaches
 // k * gridDim.x. Thread 0 of each block arrives with one acquire-release add
 // and, unless it was the last to arrive, polls the counter with acquire loads
-// (bounded; giving up raises ENGRAM_DEVERR_SORT_TIMEOUT and returns false).
-// The block's other threads wait at __syncthreads, which orders their later
-// reads after thread 0's acquire. The counter is zero at launch.
+// (at most spin_limit polls; giving up raises ENGRAM_DEVERR_SORT_TIMEOUT and
+// returns false). The block's other threads wait at __syncthreads, which
+// orders their later reads after thread 0's acquire. The counter is zero at
+// launch. A block reaches barrier k only after passing barrier k - 1, so a
+// block that passes barrier k sees every block's writes before it.
 __device__ __forceinline__ bool grid_barrier(unsigned *bar, unsigned &gen, int &flag,
                                              uint32_t spin_limit)
 {
@@ -429,60 +582,51 @@ __device__ __forceinline__ bool grid_barrier(unsigned *bar, unsigned &gen, int &
     return flag != 0;
 }
 
-// Four blocks per SM keep 592 tiles (1.2M pairs at ITEMS = 8) resident on a
-// 148-SM B200.
+// Four blocks per SM keep 592 tiles resident on a 148-SM B200.
 template <int ITEMS> __global__ void __launch_bounds__(kSortThreads, 4) radix_sort_coop(SortArgs a)
 {
     __shared__ SortSmem<ITEMS> sm;
+    constexpr int TILE = SortSmem<ITEMS>::kTile;
     unsigned gen = 0;
     if (a.ntiles <= (int)gridDim.x) {
-        // One tile per block: rank once, keep the items and their ranks in
-        // registers (and the per-warp offsets in shared memory) across the
-        // barrier, then place them.
+        // One tile per block: rank it once and keep it staged in shared
+        // memory, ordered by digit, across the barrier; then place it.
         const int tile = blockIdx.x;
         const bool has = tile < a.ntiles;
+        const TileGeom g = tile_geom(a, has ? tile : 0, TILE);
         for (int pass = 0; pass < a.passes; ++pass) {
-            const bool first = pass == 0;
-            const void *src = first ? (const void *)a.idx : (pass % 2 == 1 ? a.a : a.b);
-            unsigned long long *dst = pass % 2 == 0 ? a.a : a.b;
-            uint32_t *gc = a.group_cnt + (size_t)pass * a.ngroups * kRadix;
-            const int shift = pass * kRadixBits;
-            uint64_t it[ITEMS];
-            uint32_t rank[ITEMS];
-            uint32_t tcount = 0;
-            if (has) {
-                rank_tile<true>(sm, src, first, a.n, shift, a.rows, tile, it, rank);
-                tcount = tile_digit_count(sm);
-                publish_counts(tile, tcount, a.tile_cnt, gc);
-            }
+            const PassInfo P = pass_info(a, pass);
+            const void *src = P.first ? nullptr : out_buffer(a, pass - 1);
+            uint32_t *gc = a.group_cnt + (size_t)pass * a.ngroups * kRadixMax;
+            uint32_t tcount[2] = {0u, 0u};
+            if (has)
+                stage_tile<true>(sm, a, src, P, tile, g, P.first, gc, tcount);
             if (!grid_barrier(a.barrier, gen, sm.flag, a.spin_limit))
                 return;
             if (has)
-                place_tile<true>(sm, dst, a.n, shift, tile, tcount, it, rank, a.tile_cnt, gc,
-                                 a.ngroups);
-            if (pass + 1 < a.passes && !grid_barrier(a.barrier, gen, sm.flag, a.spin_limit))
+                place_staged_tile<true>(sm, a, P, out_buffer(a, pass), g, tcount, gc);
+            if (!P.last && !grid_barrier(a.barrier, gen, sm.flag, a.spin_limit))
                 return;
         }
         return;
     }
     // More tiles than resident blocks: each tile is ranked once, in the count
     // phase, and left ordered by digit in `ordered` (the pass's own input from
-    // the second pass on; the other item buffer on the first, whose input is
-    // idx), from where the place phase moves it.
+    // the second pass on; on the first, whose input is idx, the buffer the
+    // pass does not write), from where the place phase moves it.
     for (int pass = 0; pass < a.passes; ++pass) {
-        const bool first = pass == 0;
-        const void *src = first ? (const void *)a.idx : (pass % 2 == 1 ? a.a : a.b);
-        unsigned long long *dst = pass % 2 == 0 ? a.a : a.b;
-        unsigned long long *ordered = first ? a.b : (pass % 2 == 1 ? a.a : a.b);
-        uint32_t *gc = a.group_cnt + (size_t)pass * a.ngroups * kRadix;
-        const int shift = pass * kRadixBits;
+        const PassInfo P = pass_info(a, pass);
+        unsigned long long *dst = out_buffer(a, pass);
+        unsigned long long *src = P.first ? nullptr : out_buffer(a, pass - 1);
+        unsigned long long *ordered = P.first ? (dst == a.a ? a.b : a.a) : src;
+        uint32_t *gc = a.group_cnt + (size_t)pass * a.ngroups * kRadixMax;
         for (int tile = blockIdx.x; tile < a.ntiles; tile += gridDim.x)
-            count_order_tile(sm, src, first, a.n, shift, a.rows, tile, a.tile_cnt, gc, ordered);
+            count_order_tile(sm, a, src, P, tile, gc, ordered);
         if (!grid_barrier(a.barrier, gen, sm.flag, a.spin_limit))
             return;
         for (int tile = blockIdx.x; tile < a.ntiles; tile += gridDim.x)
-            place_ordered_tile(sm, ordered, dst, a.n, shift, tile, a.tile_cnt, gc, a.ngroups);
-        if (pass + 1 < a.passes && !grid_barrier(a.barrier, gen, sm.flag, a.spin_limit))
+            place_ordered_tile(sm, a, P, ordered, dst, tile, gc);
+        if (!P.last && !grid_barrier(a.barrier, gen, sm.flag, a.spin_limit))
             return;
     }
 }

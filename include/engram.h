@@ -36,7 +36,7 @@
 extern "C" {
 #endif
 
-#define ENGRAM_ABI_VERSION 1
+#define ENGRAM_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define ENGRAM_API __attribute__((visibility("default")))
@@ -208,11 +208,52 @@ ENGRAM_API int engram_backward_sort(const int32_t *idx, int64_t n, int64_t table
                          void *workspace, size_t workspace_bytes, engram_stream_t stream);
 
 /* Second stage: distinct rows and segmented fp32 sums from the sorted pairs
- * that engram_backward_sort left in the workspace. */
+ * that engram_backward_sort (or engram_backward_sort_heads) left in the
+ * workspace. */
 ENGRAM_API int engram_backward_reduce(int64_t n, int64_t table_rows, int32_t dim, const void *dout,
                            int32_t dtype, int32_t *uniq_rows, float *row_grads,
                            int32_t *num_unique, void *workspace, size_t workspace_bytes,
                            engram_stream_t stream);
+
+/*
+ * engram_backward_heads -- engram_backward for the lookups the hash produced
+ * (engram API page, Qwen3_8_FlashNextNGramEmbedding._hash_input_ids and the
+ * owner-side gradient accumulation of Qwen3_8_FlashNextOwnerShardedEmbedding),
+ * with the same results, computed faster by using their structure: lookup
+ * j = t * H + h of token t and head h lies in head h's slice
+ * [offsets[h], offsets[h] + vocab_sizes[h]) of the table, and the heads'
+ * slices ascend without overlapping. The sort then orders each head's T
+ * lookups by row - offsets[h] (bits(vocab_sizes[h] - 1) bits: 25 on the
+ * page's table, against 29 for the whole row, so 3 radix passes instead of 4)
+ * and lays the heads out in order.
+ *   params     the hash's parameters (H = (ngram_size - 1) * heads_per_ngram
+ *              heads, table_rows, dim)
+ *   idx        device, int32 [T, H] as engram_hash / engram_hash_gather wrote
+ *              it; a value outside its head's slice sets
+ *              ENGRAM_DEVERR_ROW_RANGE (results are then unspecified, memory
+ *              accesses stay in bounds)
+ *   T          tokens, n = T * H < 2^31
+ *   dout, dtype, uniq_rows, row_grads, num_unique   as engram_backward with
+ *              n = T * H lookups of width params->dim
+ *   workspace  >= engram_backward_workspace_size(T * H, params->table_rows,
+ *              params->dim) bytes, 256-byte aligned
+ * Parameters whose slices do not ascend disjointly inside the table are
+ * sorted as engram_backward sorts (same results).
+ * engram_backward_heads = engram_backward_sort_heads followed by
+ * engram_backward_reduce(T * H, params->table_rows, params->dim, ...) with the
+ * same workspace.
+ */
+ENGRAM_API int engram_backward_heads(const engram_params_t *params, const int32_t *idx,
+                                     int64_t T, const void *dout, int32_t dtype,
+                                     int32_t *uniq_rows, float *row_grads, int32_t *num_unique,
+                                     void *workspace, size_t workspace_bytes,
+                                     engram_stream_t stream);
+
+/* First stage of engram_backward_heads: the sort by head into the workspace
+ * (one cooperative launch, or two launches per pass as engram_backward_sort). */
+ENGRAM_API int engram_backward_sort_heads(const engram_params_t *params, const int32_t *idx,
+                                          int64_t T, void *workspace, size_t workspace_bytes,
+                                          engram_stream_t stream);
 
 /* Size of the library's own device scratch array used by engram_backward_noalloc. */
 #define ENGRAM_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20) /* 32 MiB per device */

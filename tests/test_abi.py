@@ -50,7 +50,7 @@ def test_library_exports_every_declared_symbol(E):
 
 def test_params_layout_and_version(E):
     assert E.lib.engram_params_size() == ctypes.sizeof(E.EngramParams) == 576
-    assert E.engram_abi_version() == 1
+    assert E.engram_abi_version() == 2
     for rc in range(4):
         assert E.status_string(rc).startswith("ENGRAM_")
     assert "unknown" in E.status_string(99)

@@ -314,3 +314,104 @@ def test_backward_stages_equal_whole(E):
     U = int(nu1.item())
     assert U == int(nu2.item())
     assert torch.equal(u1[:U], u2[:U]) and torch.equal(g1[:U], g2[:U])
+
+
+# ============================================== backward sorted by head
+
+def check_backward_heads(E, cfg, idx_np, dout_t, dtype_code):
+    """engram_backward_heads on the hash's [T, H] lookups: the oracle's rows and
+    sums, and bit for bit what engram_backward gives on the same lookups."""
+    p = E.make_params(cfg)
+    H = p.heads
+    idx_t = dev(idx_np.reshape(-1, H).astype(np.int32))
+    n = idx_t.numel()
+    uniq, grads, nu = E.engram_backward_heads(p, idx_t, dout_t.cuda())
+    U = int(nu.item())
+    raw = dout_t.numpy() if dout_t.dtype == torch.float32 else bits16(dout_t)
+    want_u, want_g = oracle.backward(idx_np.reshape(-1), raw.reshape(n, -1), dtype_code)
+    assert U == len(want_u)
+    np.testing.assert_array_equal(uniq[:U].cpu().numpy(), want_u)
+    assert_grads_close(grads[:U].cpu().numpy(), want_g)
+    u2, g2, nu2 = E.engram_backward(idx_t.view(-1), dout_t.cuda(), cfg["table_rows"])
+    assert int(nu2.item()) == U
+    assert torch.equal(uniq[:U], u2[:U]) and torch.equal(grads[:U], g2[:U])
+    assert E.engram_get_device_error() == 0
+
+
+@pytest.mark.parametrize("name", list(WORKLOADS))
+def test_backward_heads_full_workloads(E, name):
+    cfg = head_params(name)
+    ids, cu = token_stream(name)
+    idx = oracle.hash_ids(ids, cu, cfg)
+    w = WORKLOADS[name]
+    dout = host_dout(name, idx.size, cfg["dim"], w.dtype)
+    check_backward_heads(E, cfg, idx, dout, oracle.F32 if w.dtype == "f32" else oracle.BF16)
+
+
+@pytest.mark.parametrize("N,K", [(3, 8), (2, 3), (4, 2), (2, 1), (2, 32)])
+@pytest.mark.parametrize("T", [1, 77, 5003, 40_000])
+def test_backward_heads_shapes(E, N, K, T):
+    """Head counts 1 to 32, tokens from one to several tiles per head with
+    ragged last tiles; small moduli, so rows repeat often."""
+    cfg = dict(small_params(seed=T % 13, N=N, K=K, eos=3), dim=32)
+    ids, cu = random_stream(T + N, T, 50, 3, 0.1, nseq=1 + T // 900)
+    idx = oracle.hash_ids(ids, cu, cfg)
+    dout = torch.randn(idx.size, 32, generator=torch.Generator().manual_seed(T))
+    check_backward_heads(E, cfg, idx, dout, oracle.F32)
+
+
+def test_backward_heads_page_rows_long_tiles(E):
+    """The page's table with more tiles than resident blocks (4M lookups): the
+    sort's digit-ordered path, per head."""
+    cfg = head_params("full")
+    ids, cu = random_stream(11, 262_144, 248_320, cfg["eos_id"], 1 / 512, nseq=64)
+    idx = oracle.hash_ids(ids, cu, cfg)
+    dout = torch.randn(idx.size, 160, generator=torch.Generator().manual_seed(2)).to(
+        torch.bfloat16)
+    check_backward_heads(E, cfg, idx, dout, oracle.BF16)
+
+
+def test_backward_heads_slices_out_of_order_sort_plainly(E):
+    """Slices that do not ascend with the head: the call sorts the lookups as
+    engram_backward does and gives the same results."""
+    cfg = dict(small_params(seed=5, N=3, K=4, eos=3), dim=16)
+    vocab, offs = list(cfg["vocab_sizes"]), list(cfg["offsets"])
+    offs[0], offs[-1] = offs[-1] - vocab[0] + vocab[-1], 0     # first and last swap places
+    vocab[0], vocab[-1] = vocab[-1], vocab[0]
+    cfg = dict(cfg, vocab_sizes=tuple(vocab), offsets=tuple(offs))
+    ids, cu = random_stream(5, 3000, 50, 3, 0.1, nseq=3)
+    idx = oracle.hash_ids(ids, cu, cfg)
+    dout = torch.randn(idx.size, 16, generator=torch.Generator().manual_seed(5))
+    check_backward_heads(E, cfg, idx, dout, oracle.F32)
+
+
+def test_backward_heads_empty_and_flags(E):
+    cfg = dict(small_params(seed=2, N=3, K=2, eos=3), dim=16)
+    p = E.make_params(cfg)
+    u, g, nu = E.engram_backward_heads(p, torch.empty(0, 4, dtype=torch.int32, device="cuda"),
+                                       torch.empty(0, 16, device="cuda"))
+    assert int(nu.item()) == 0
+    # a lookup outside its own head's slice (here: head 1's slice in head 0)
+    idx = np.array([[cfg["offsets"][1], cfg["offsets"][1], cfg["offsets"][2],
+                     cfg["offsets"][3]]], np.int32)
+    E.engram_backward_heads(p, dev(idx), torch.randn(4, 16, device="cuda"))
+    assert E.engram_get_device_error() & E.ENGRAM_DEVERR_ROW_RANGE
+
+
+def test_backward_heads_stages_equal_whole(E):
+    cfg = head_params("thd64k")
+    ids, cu = token_stream("thd64k")
+    idx = dev(oracle.hash_ids(ids, cu, cfg).astype(np.int32))
+    p = E.make_params(cfg)
+    n, D, R = idx.numel(), cfg["dim"], cfg["table_rows"]
+    dout = torch.randn(n, D, device="cuda").to(torch.bfloat16)
+    u1, g1, nu1 = E.engram_backward_heads(p, idx, dout)
+    ws = torch.empty(E.engram_backward_workspace_size(n, R, D), dtype=torch.uint8, device="cuda")
+    u2 = torch.empty(n, dtype=torch.int32, device="cuda")
+    g2 = torch.empty(n, D, device="cuda")
+    nu2 = torch.empty(1, dtype=torch.int32, device="cuda")
+    E.engram_backward_sort_heads(p, idx, ws)
+    E.engram_backward_reduce(n, R, dout, u2, g2, nu2, ws)
+    U = int(nu1.item())
+    assert U == int(nu2.item())
+    assert torch.equal(u1[:U], u2[:U]) and torch.equal(g1[:U], g2[:U])

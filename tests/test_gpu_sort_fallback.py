@@ -4,7 +4,9 @@ with ENGRAM_SORT_SEPARATE_LAUNCHES=1 in a child process, against the
 one-launch sort in another child on the same inputs. A stable sort has one
 result, so the distinct rows and their fp32 sums must be identical bit for
 bit. The sizes cover one tile, a ragged single tile, many resident tiles and
-more tiles than resident blocks; half the lookups hit a few hot rows.
+more tiles than resident blocks; half the lookups hit a few hot rows. The
+sort by head (engram_backward_heads) is compared the same way on the page's
+head constants.
 """
 
 import os
@@ -36,6 +38,19 @@ for n in (1, 1000, 250_007, 2_000_003):
     assert E.engram_get_device_error() == 0
     out["u%d" % n] = u[:U].cpu().numpy()
     out["g%d" % n] = g[:U].cpu().numpy()
+from workloads import head_params, random_stream
+import oracle
+cfg = dict(head_params("full"), dim=16)
+p = E.make_params(cfg)
+for T in (1, 63, 15_625, 131_072):
+    ids, cu = random_stream(T, T, 2000, cfg["eos_id"], 0.01, nseq=1 + T // 4096)
+    idx = oracle.hash_ids(ids, cu, cfg).astype(np.int32)
+    dout = torch.randn(idx.size, 16, generator=torch.Generator().manual_seed(T % 997))
+    u, g, nu = E.engram_backward_heads(p, torch.from_numpy(idx).cuda(), dout.cuda())
+    U = int(nu.item())
+    assert E.engram_get_device_error() == 0
+    out["hu%d" % T] = u[:U].cpu().numpy()
+    out["hg%d" % T] = g[:U].cpu().numpy()
 np.savez(sys.argv[2], **out)
 """
 
