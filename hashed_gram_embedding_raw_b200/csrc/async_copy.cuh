@@ -31,10 +31,21 @@ __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t b
 
 // Waits (bounded by limit_ns) for phase `parity` of `bar`; false on timeout.
 // The clock is read once every 64 polls, so a poll costs little issue time.
+// limit_ns == 0 tests the phase once without waiting (a test hook's bound).
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
                                           uint64_t limit_ns = kCopyWaitNs)
 {
     const uint32_t addr = smem_u32(bar);
+    if (limit_ns == 0) {
+        uint32_t done;
+        asm volatile("{\n\t.reg .pred p;\n\t"
+                     "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                     "selp.u32 %0, 1, 0, p;\n\t}"
+                     : "=r"(done)
+                     : "r"(addr), "r"(parity)
+                     : "memory");
+        return done != 0;
+    }
     uint64_t t0 = 0;
     for (uint32_t spin = 0;; ++spin) {
         uint32_t done;

@@ -100,7 +100,10 @@ __device__ __forceinline__ uint32_t lanemask_lt()
 
 // Exclusive scan of one value per thread over the block (blockDim.x a
 // multiple of 32, at most 1024). s_warp holds 32 words of shared scratch.
-// Every thread gets the block total in *total when total != nullptr.
+// Every thread gets the block total in *total when total != nullptr. TRAIL =
+// false leaves out the closing barrier that protects s_warp from the next
+// scan; the caller must then pass a block barrier before reusing s_warp.
+template <bool TRAIL = true>
 __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t *s_warp,
                                                          uint32_t *total)
 {
@@ -131,11 +134,13 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t *s
     const uint32_t before = wid ? s_warp[wid - 1] : 0u;
     if (total)
         *total = s_warp[nw - 1];
-    __syncthreads();
+    if constexpr (TRAIL)
+        __syncthreads();
     return before + x - v;
 }
 
 // The same scan over 64-bit values (no total); s_warp holds 32 words.
+template <bool TRAIL = true>
 __device__ __forceinline__ unsigned long long block_exclusive_scan64(unsigned long long v,
                                                                     unsigned long long *s_warp)
 {
@@ -164,7 +169,8 @@ __device__ __forceinline__ unsigned long long block_exclusive_scan64(unsigned lo
     }
     __syncthreads();
     const unsigned long long before = wid ? s_warp[wid - 1] : 0ull;
-    __syncthreads();
+    if constexpr (TRAIL)
+        __syncthreads();
     return before + x - v;
 }
 

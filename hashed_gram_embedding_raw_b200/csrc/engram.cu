@@ -194,7 +194,8 @@ int launch_hash_gather(const HashArgs &a, const int32_t *ids, const int32_t *cu,
 struct BwdPlan {
     int wmax = 0, GF = 0, tiles_max = 0, groups_max = 0;
     size_t a = 0, b = 0, tile_cnt = 0, ctl = 0, ctl_bytes = 0, group_cnt = 0, barrier = 0;
-    size_t wcount = 0, bcount = 0, pb = 0, pe = 0, meta = 0, total = 0;
+    size_t seg_status = 0, seg_ready = 0, seg_gen = 0, seg_done = 0;
+    size_t pb = 0, pe = 0, meta = 0, total = 0;
 };
 
 int bwd_plan(int64_t n, int64_t rows, int32_t dim, BwdPlan *P)
@@ -228,9 +229,12 @@ int bwd_plan(int64_t n, int64_t rows, int32_t dim, BwdPlan *P)
     P->ctl = off;
     P->group_cnt = take((size_t)bwd::kMaxPasses * bwd::kRadixMax * P->groups_max * 4);
     P->barrier = take(sizeof(unsigned)); // grid-barrier counter of the one-launch sort
+    // the reduce's look-back words, ready flags, generation and finish count
+    P->seg_status = take((size_t)P->wmax * 8);
+    P->seg_ready = take((size_t)P->wmax * 4);
+    P->seg_gen = take(sizeof(unsigned));
+    P->seg_done = take(sizeof(unsigned));
     P->ctl_bytes = off - P->ctl;
-    P->wcount = take((size_t)P->wmax * 4);
-    P->bcount = take((size_t)ceil_div(P->wmax, bwd::kSegWarps) * 4);
     P->pb = take((size_t)P->wmax * dim * 8);
     P->pe = take((size_t)P->wmax * dim * 8);
     P->meta = take((size_t)P->wmax * sizeof(bwd::SegMeta));
@@ -514,18 +518,13 @@ int launch_seg(const unsigned long long *items, int64_t n, const BwdPlan &P, con
     const int W = (int)std::max<int64_t>(
         1, std::min<int64_t>(std::min<int64_t>(res, P.wmax), ceil_div(n, 32)));
     const int blocks = (int)ceil_div(W, kSegWarps);
-    auto *wcount = (uint32_t *)(ws + P.wcount);
-    auto *bcount = (uint32_t *)(ws + P.bcount);
+    const SegSync sy{(unsigned long long *)(ws + P.seg_status), (unsigned *)(ws + P.seg_ready),
+                     (unsigned *)(ws + P.seg_gen), (unsigned *)(ws + P.seg_done)};
     auto *pb = (double *)(ws + P.pb);
     auto *pe = (double *)(ws + P.pe);
     auto *meta = (SegMeta *)(ws + P.meta);
-    seg_count<<<blocks, kSegThreads, 0, stream>>>(items, n, W, wcount, bcount);
-    ENGRAM_TRY(after_launch());
-    fn<<<blocks, kSegThreads, smem, stream>>>(items, n, W, wcount, bcount, dout, dim, batch,
-                                              stage_bytes, uniq, grads, pb, pe, meta,
-                                              num_unique);
-    ENGRAM_TRY(after_launch());
-    seg_fixup<GF><<<blocks, kSegThreads, 0, stream>>>(W, dim, pb, pe, meta, uniq, grads);
+    fn<<<blocks, kSegThreads, smem, stream>>>(items, n, W, sy, dout, dim, batch, stage_bytes,
+                                              uniq, grads, pb, pe, meta, num_unique);
     return after_launch();
 }
 

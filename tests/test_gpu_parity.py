@@ -415,3 +415,33 @@ def test_backward_heads_stages_equal_whole(E):
     U = int(nu1.item())
     assert U == int(nu2.item())
     assert torch.equal(u1[:U], u2[:U]) and torch.equal(g1[:U], g2[:U])
+
+
+@pytest.mark.parametrize("pattern", ["hot_and_cold", "one_row"])
+def test_backward_reduce_repeated_after_one_sort(E, pattern):
+    """engram_backward_reduce run three times on one sort's workspace, with
+    different output gradients: the reduce's published counts and pieces carry
+    the launch's generation, so every run stands on its own. one_row makes a
+    single segment cross every warp's range."""
+    rng = np.random.Generator(np.random.PCG64(3))
+    n, R, D = 300_007, 320_001_536, 160
+    if pattern == "one_row":
+        idx_np = np.full(n, 77, np.int64)
+    else:
+        idx_np = np.where(rng.random(n) < 0.3, rng.integers(0, 5, n), rng.integers(0, R, n))
+    idx = dev(idx_np.astype(np.int32))
+    ws = torch.empty(E.engram_backward_workspace_size(n, R, D), dtype=torch.uint8, device="cuda")
+    E.engram_backward_sort(idx, R, D, ws)
+    for k in range(3):
+        dout = torch.randn(n, D, generator=torch.Generator().manual_seed(10 + k)).to(
+            torch.bfloat16)
+        u = torch.empty(n, dtype=torch.int32, device="cuda")
+        g = torch.empty(n, D, device="cuda")
+        nu = torch.empty(1, dtype=torch.int32, device="cuda")
+        E.engram_backward_reduce(n, R, dout.cuda(), u, g, nu, ws)
+        U = int(nu.item())
+        want_u, want_g = oracle.backward(idx_np, bits16(dout).reshape(n, -1), oracle.BF16)
+        assert U == len(want_u)
+        np.testing.assert_array_equal(u[:U].cpu().numpy(), want_u)
+        assert_grads_close(g[:U].cpu().numpy(), want_g)
+    assert E.engram_get_device_error() == 0
