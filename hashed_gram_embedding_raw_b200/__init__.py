@@ -10,8 +10,7 @@ has not been built (`python hashed_gram_embedding_raw_b200/build.py`).
 
 from ._binding import (ENGRAM_BF16, ENGRAM_CONV_NORM, ENGRAM_CONV_RESIDUAL, ENGRAM_CONV_SILU,
                        ENGRAM_DEVERR_COPY_TIMEOUT, ENGRAM_DEVERR_CU_SEQLENS,
-                       ENGRAM_DEVERR_REDUCE_TIMEOUT, ENGRAM_DEVERR_ROW_RANGE,
-                       ENGRAM_DEVERR_SORT_TIMEOUT,
+                       ENGRAM_DEVERR_ROW_RANGE, ENGRAM_DEVERR_SORT_TIMEOUT,
                        ENGRAM_EINVAL, ENGRAM_ECUDA, ENGRAM_ENOSPC, ENGRAM_F16, ENGRAM_F32,
                        ENGRAM_NOALLOC_SCRATCH_BYTES, ENGRAM_OK, EXPORTED, LIB_PATH,
                        AdamParams, ConvParams, EngramError, EngramParams, engram_abi_version,
@@ -29,7 +28,7 @@ from ._binding import (ENGRAM_BF16, ENGRAM_CONV_NORM, ENGRAM_CONV_RESIDUAL, ENGR
 __all__ = [
     "ENGRAM_BF16", "ENGRAM_CONV_NORM", "ENGRAM_CONV_RESIDUAL", "ENGRAM_CONV_SILU",
     "ENGRAM_DEVERR_COPY_TIMEOUT", "ENGRAM_DEVERR_CU_SEQLENS", "ENGRAM_DEVERR_ROW_RANGE",
-    "ENGRAM_DEVERR_REDUCE_TIMEOUT", "ENGRAM_DEVERR_SORT_TIMEOUT", "ENGRAM_EINVAL",
+    "ENGRAM_DEVERR_SORT_TIMEOUT", "ENGRAM_EINVAL",
     "ENGRAM_ECUDA", "ENGRAM_ENOSPC", "ENGRAM_F16", "ENGRAM_F32",
     "ENGRAM_NOALLOC_SCRATCH_BYTES", "ENGRAM_OK", "EXPORTED", "LIB_PATH", "AdamParams", "ConvParams",
     "EngramError", "EngramParams", "engram_abi_version", "engram_backward",

@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(_PKG, "_lib", "libengram_b200.so")
 ENGRAM_OK, ENGRAM_EINVAL, ENGRAM_ENOSPC, ENGRAM_ECUDA = 0, 1, 2, 3
 ENGRAM_F32, ENGRAM_BF16, ENGRAM_F16 = 0, 1, 2
 ENGRAM_DEVERR_ROW_RANGE, ENGRAM_DEVERR_CU_SEQLENS, ENGRAM_DEVERR_SORT_TIMEOUT = 1, 2, 4
-ENGRAM_DEVERR_COPY_TIMEOUT, ENGRAM_DEVERR_REDUCE_TIMEOUT = 8, 16
+ENGRAM_DEVERR_COPY_TIMEOUT = 8
 ENGRAM_CONV_NORM, ENGRAM_CONV_SILU, ENGRAM_CONV_RESIDUAL = 1, 2, 4
 ENGRAM_MAX_NGRAM, ENGRAM_MAX_HEADS = 4, 32
 

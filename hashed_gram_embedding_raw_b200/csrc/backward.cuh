@@ -8,26 +8,19 @@
 //
 // Stage 1 (sort): radix_sort.cuh orders the (row, lookup) pairs by row.
 //
-// Stage 2 (reduce, one launch): the sorted items are cut into one contiguous
-// range per resident warp. A segment is a run of equal keys. Each warp counts
-// the segment heads in its range, publishes the count and looks back over the
-// earlier warps' published counts for its first segment index (a decoupled
-// look-back: a warp's count is out as soon as it is taken, and a warp that has
-// its total publishes that too, so later warps stop there). Meanwhile its
-// first dout rows are already on their way: the warp streams its rows through
+// Stage 2 (reduce): the sorted items are cut into one contiguous range per
+// resident warp. A segment is a run of equal keys. seg_count counts segment
+// heads per range and per block; seg_reduce turns those counts into each
+// range's first segment index, then streams the dout rows of its range through
 // a shared-memory ring filled by cp.async (several rows in flight per warp,
 // independent of registers) and sums each segment in fp64 (rounded once to
 // fp32 on output, so hot rows with thousands of terms stay at fp32-rounding
 // distance from the exact sum). Segments that start and end inside a range are
 // written directly, with each store instruction covering contiguous bytes; the
 // pieces of segments that cross range boundaries are written as fp64 partial
-// sums, and the warp holding a crossing segment's last piece adds the pieces
-// in range order once their owners have published them. No atomics touch the
-// sums, so the result is deterministic and hot rows spread over many warps.
-// Published words carry the launch's generation (advanced by the last warp of
-// each launch), so nothing has to be cleared between launches; the sort clears
-// them once. Every wait is bounded: one that runs out raises
-// ENGRAM_DEVERR_REDUCE_TIMEOUT and the warp skips the writes it cannot place.
+// sums and combined, in range order, by seg_fixup (one warp per crossing
+// segment). No atomics touch the sums, so the result is deterministic and hot
+// rows spread over many warps.
 #pragma once
 
 #include "common.cuh"
@@ -58,93 +51,45 @@ __device__ __forceinline__ void range_of(int64_t n, int64_t w, int64_t W, int64_
     b = n * (w + 1) / W;
 }
 
-// Look-back state of a reduce launch, in the workspace (cleared by the sort).
-struct SegSync {
-    unsigned long long *status; // [W]: per warp, tag << 32 | count (tag: generation, kind)
-    unsigned *ready;            // [W]: generation + 1 once the warp's partials are out
-    unsigned *gen;              // launch generation, advanced by each launch's last warp
-    unsigned *done;             // warps of the launch that have finished
-};
-
-constexpr uint32_t kSegSpin = 1u << 22; // polls (~64 ns apart) before a wait gives up
-
-__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long *p)
+// Segment heads (first item, or key differs from the previous one) per range
+// (wcount) and per block of kSegWarps ranges (bcount).
+__global__ void __launch_bounds__(kSegThreads)
+    seg_count(const unsigned long long *__restrict__ items, int64_t n, int W,
+              uint32_t *__restrict__ wcount, uint32_t *__restrict__ bcount)
 {
-    unsigned long long v;
-    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-    return v;
-}
-
-__device__ __forceinline__ void st_relaxed_u64(unsigned long long *p, unsigned long long v)
-{
-    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
-
-// Segment heads (first item, or key differs from the previous one) in [a, b).
-__device__ __forceinline__ uint32_t count_heads(const unsigned long long *__restrict__ items,
-                                                int64_t a, int64_t b, int lane)
-{
+    __shared__ uint32_t s_cnt[kSegWarps];
+    const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+    const int64_t w = (int64_t)blockIdx.x * kSegWarps + wib;
     uint32_t cnt = 0;
-    for (int64_t c0 = a; c0 < b; c0 += 128) {
-        uint32_t key[4], prev[4];
+    if (w < W) {
+        int64_t a, b;
+        range_of(n, w, W, a, b);
+        for (int64_t c0 = a; c0 < b; c0 += 128) {
+            uint32_t key[4], prev[4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int64_t i = c0 + 32 * q + lane;
-            key[q] = i < b ? item_key(__ldg(items + i)) : 0u;
-            prev[q] = (i < b && i > 0) ? item_key(__ldg(items + i - 1)) : ~key[q];
-        }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int64_t i = c0 + 32 * q + lane;
-            cnt += __popc(__ballot_sync(kFull, i < b && key[q] != prev[q]));
-        }
-    }
-    return cnt;
-}
-
-// Decoupled look-back: publishes warp w's head count `cnt` and returns the
-// number of heads before its range (false if a wait ran out). Tag of a word:
-// 2 * (generation + 1) + (1 if the value is the inclusive total up to that warp).
-__device__ __forceinline__ bool seg_lookback(const SegSync &sy, uint32_t G, int64_t w,
-                                             uint32_t cnt, int lane, uint32_t &excl)
-{
-    const uint32_t tag = 2u * (G + 1u);
-    if (lane == 0)
-        st_relaxed_u64(sy.status + w, ((unsigned long long)tag << 32) | cnt);
-    excl = 0;
-    int64_t base = w - 1;
-    uint32_t spins = 0;
-    while (base >= 0) {
-        const int64_t q = base - lane;
-        unsigned long long word = 0;
-        bool ok = false;
-        for (;;) {
-            if (q >= 0) {
-                word = ld_relaxed_u64(sy.status + q);
-                ok = (uint32_t)(word >> 33) == G + 1u;
-            } else {
-                word = ((unsigned long long)(tag | 1u) << 32); // before warp 0: total 0
-                ok = true;
+            for (int q = 0; q < 4; ++q) {
+                const int64_t i = c0 + 32 * q + lane;
+                key[q] = i < b ? item_key(__ldg(items + i)) : 0u;
+                prev[q] = (i < b && i > 0) ? item_key(__ldg(items + i - 1)) : ~key[q];
             }
-            if (__all_sync(kFull, ok))
-                break;
-            if (++spins > kSegSpin)
-                return false;
-            __nanosleep(64);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int64_t i = c0 + 32 * q + lane;
+                cnt += __popc(__ballot_sync(kFull, i < b && key[q] != prev[q]));
+            }
         }
-        const uint32_t incl = __ballot_sync(kFull, (word >> 32) & 1u);
-        const uint32_t v = (uint32_t)word;
-        if (incl) {
-            const int k = __ffs(incl) - 1; // the nearest inclusive total
-            excl += __reduce_add_sync(kFull, lane <= k ? v : 0u);
-            break;
-        }
-        excl += __reduce_add_sync(kFull, v);
-        base -= 32;
+        if (lane == 0)
+            wcount[w] = cnt;
     }
     if (lane == 0)
-        st_relaxed_u64(sy.status + w, ((unsigned long long)(tag | 1u) << 32) | (excl + cnt));
-    return true;
+        s_cnt[wib] = w < W ? cnt : 0u;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t t = 0;
+        for (int k = 0; k < kSegWarps; ++k)
+            t += s_cnt[k];
+        bcount[blockIdx.x] = t;
+    }
 }
 
 // Four consecutive columns (float4 group f) of one staged row, as fp32.
@@ -264,20 +209,35 @@ __device__ __forceinline__ void cp_async_wait()
 // Dynamic shared memory: kSegWarps * kSegStages * (stage bytes + batch items).
 template <int DT, int GF, int RVT>
 __global__ void __launch_bounds__(kSegThreads)
-    seg_reduce(const unsigned long long *__restrict__ items, int64_t n, int W, SegSync sy,
+    seg_reduce(const unsigned long long *__restrict__ items, int64_t n, int W,
+               const uint32_t *__restrict__ wcount, const uint32_t *__restrict__ bcount,
                const void *__restrict__ dout, int dim, int batch, int stage_bytes,
                int32_t *__restrict__ uniq, float *__restrict__ grads,
                double *__restrict__ pb, double *__restrict__ pe, SegMeta *__restrict__ meta,
                int32_t *__restrict__ num_unique)
 {
     extern __shared__ __align__(16) unsigned char smem[];
+    __shared__ uint32_t s_warp[32];
     const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
     const int64_t w = (int64_t)blockIdx.x * kSegWarps + wib;
     const int F = dim >> 2; // float4 groups per row
     const int rvec = RVT ? RVT : dim * (DT == ENGRAM_F32 ? 4 : 2) / 16;
+
+    // First segment index of each range: heads in earlier blocks + earlier warps.
+    uint32_t before = 0;
+    for (int k = threadIdx.x; k < (int)blockIdx.x; k += kSegThreads)
+        before += bcount[k];
+    uint32_t block_before;
+    (void)block_exclusive_scan(before, s_warp, &block_before);
+    uint32_t warp_before = 0;
+    for (int k = 0; k < wib; ++k) {
+        const int64_t wk = (int64_t)blockIdx.x * kSegWarps + k;
+        warp_before += wk < W ? wcount[wk] : 0u;
+    }
+    if (blockIdx.x == gridDim.x - 1 && threadIdx.x == 0)
+        *num_unique = (int32_t)(block_before + bcount[blockIdx.x]);
     if (w >= W)
         return;
-    const uint32_t G = *(volatile const unsigned *)sy.gen; // set before this launch
 
     int64_t a, b;
     range_of(n, w, W, a, b);
@@ -312,37 +272,9 @@ __global__ void __launch_bounds__(kSegThreads)
         cp_async_commit();
     };
 
-#pragma unroll
-    for (int k = 0; k < kSegStages; ++k)
-        issue(k);
-
-    // First segment index of the range, while the first rows are in flight.
-    const uint32_t cnt = count_heads(items, a, b, lane);
-    uint32_t excl = 0;
-    const bool placed = seg_lookback(sy, G, w, cnt, lane, excl);
-    if (w == W - 1 && lane == 0 && placed)
-        *num_unique = (int32_t)(excl + cnt);
-    if (!placed) {
-        if (lane == 0)
-            raise_device_error(ENGRAM_DEVERR_REDUCE_TIMEOUT);
-        cp_async_wait<0>();
-        // nothing of this range can be placed; let the launch finish
-        if (lane == 0) {
-            __threadfence();
-            *(volatile unsigned *)(sy.ready + w) = G + 1u;
-            if (atomicAdd(sy.done, 1u) == (unsigned)W - 1u) {
-                *(volatile unsigned *)sy.done = 0u;
-                __threadfence();
-                atomicAdd(sy.gen, 1u);
-            }
-        }
-        return;
-    }
-    const uint32_t first_key = item_key(__ldg(items + a));
-
     SegAcc<GF> sa;
     sa.cnt = 0;
-    int32_t u = (int32_t)excl - 1; // open segment's index
+    int32_t u = (int32_t)(block_before + warp_before) - 1; // open segment's index
     uint32_t cur_key = 0;
     uint32_t prev_key = a > 0 ? item_key(__ldg(items + a - 1)) : ~item_key(__ldg(items + a));
     bool open_here = false; // the open segment's head lies in this range
@@ -350,6 +282,9 @@ __global__ void __launch_bounds__(kSegThreads)
     int32_t pb_ends = 0;
 
     const int nb = (len + batch - 1) / batch;
+#pragma unroll
+    for (int k = 0; k < kSegStages; ++k)
+        issue(k);
     for (int k = 0; k < nb; ++k) {
         cp_async_wait<kSegStages - 1>();
         __syncwarp();
@@ -457,85 +392,57 @@ __global__ void __launch_bounds__(kSegThreads)
         store_partial<GF>(pb + (size_t)w * dim, sa, lane, F);
         pb_ends = cont ? 0 : 1;
     }
-    if (lane == 0) {
+    if (lane == 0)
         meta[w] = SegMeta{pe_valid, u, (int32_t)cur_key, pb_ends};
-        __threadfence();
-        *(volatile unsigned *)(sy.ready + w) = G + 1u; // this range's pieces are out
-    }
-    __syncwarp();
+}
 
-    // The range holds the last piece of a segment begun in an earlier range:
-    // find the range with its head piece (pe) and add the pieces in range
-    // order -- head piece, the earlier ranges' pieces, this range's (pb).
-    if (pb_ends) {
-        int64_t wh = -1;
-        uint32_t spins = 0;
-        for (int64_t base = w - 1; wh < 0 && base >= 0; base -= 32) {
-            const int64_t q = base - lane;
-            bool ok = q < 0;
-            while (!__all_sync(kFull, ok)) {
-                if (!ok)
-                    ok = *(volatile const unsigned *)(sy.ready + q) == G + 1u;
-                if (++spins > kSegSpin)
-                    break;
-                __nanosleep(64);
-            }
-            if (!__all_sync(kFull, ok)) {
-                wh = -2;
-                break;
-            }
-            __threadfence();
-            const bool head = q >= 0 && __ldcg(&meta[q].pe_valid) != 0;
-            const uint32_t hm = __ballot_sync(kFull, head);
-            if (hm)
-                wh = base - (__ffs(hm) - 1);
-        }
-        if (wh < 0) {
-            if (lane == 0)
-                raise_device_error(ENGRAM_DEVERR_REDUCE_TIMEOUT);
-        } else {
-            double acc[GF][4];
+// One warp per segment that crosses range boundaries: its head piece plus the
+// following ranges' pieces, in range order.
+template <int GF>
+__global__ void __launch_bounds__(kSegThreads)
+    seg_fixup(int W, int dim, const double *__restrict__ pb, const double *__restrict__ pe,
+              const SegMeta *__restrict__ meta, int32_t *__restrict__ uniq,
+              float *__restrict__ grads)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    if (w >= W)
+        return;
+    const SegMeta m = meta[w];
+    if (!m.pe_valid)
+        return;
+    const int F = dim >> 2;
+    double acc[GF][4];
 #pragma unroll
-            for (int g = 0; g < GF; ++g) {
-                const int f = lane + 32 * g;
+    for (int g = 0; g < GF; ++g) {
+        const int f = lane + 32 * g;
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            acc[g][q] = f < F ? pe[(size_t)w * dim + 4 * f + q] : 0.0;
+    }
+    for (int64_t w2 = w + 1; w2 < W; ++w2) {
+#pragma unroll
+        for (int g = 0; g < GF; ++g) {
+            const int f = lane + 32 * g;
+            if (f < F) {
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
-                    acc[g][q] = f < F ? __ldcg(pe + (size_t)wh * dim + 4 * f + q) : 0.0;
+                    acc[g][q] += pb[(size_t)w2 * dim + 4 * f + q];
             }
-            for (int64_t w2 = wh + 1; w2 <= w; ++w2) {
-#pragma unroll
-                for (int g = 0; g < GF; ++g) {
-                    const int f = lane + 32 * g;
-                    if (f < F) {
-#pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            acc[g][q] += __ldcg(pb + (size_t)w2 * dim + 4 * f + q);
-                    }
-                }
-            }
-            const int32_t uc = (int32_t)excl - 1; // the segment continued into this range
-#pragma unroll
-            for (int g = 0; g < GF; ++g) {
-                const int f = lane + 32 * g;
-                if (f < F)
-                    st_stream((float4 *)(grads + (size_t)uc * dim) + f,
-                              make_float4((float)acc[g][0], (float)acc[g][1], (float)acc[g][2],
-                                          (float)acc[g][3]));
-            }
-            if (lane == 0)
-                uniq[uc] = (int32_t)first_key;
         }
+        if (meta[w2].pb_ends)
+            break;
     }
-
-    // The launch's last warp advances the generation for the next launch.
-    if (lane == 0) {
-        __threadfence();
-        if (atomicAdd(sy.done, 1u) == (unsigned)W - 1u) {
-            *(volatile unsigned *)sy.done = 0u;
-            __threadfence();
-            atomicAdd(sy.gen, 1u);
-        }
+#pragma unroll
+    for (int g = 0; g < GF; ++g) {
+        const int f = lane + 32 * g;
+        if (f < F)
+            st_stream((float4 *)(grads + (size_t)m.pe_u * dim) + f,
+                      make_float4((float)acc[g][0], (float)acc[g][1], (float)acc[g][2],
+                                  (float)acc[g][3]));
     }
+    if (lane == 0)
+        uniq[m.pe_u] = m.pe_key;
 }
 
 } // namespace bwd

@@ -18,6 +18,7 @@
 #include "engram.h"
 
 #include "backward.cuh"
+#include "cluster_sort.cuh"
 #include "common.cuh"
 #include "hash_gather.cuh"
 #include "ple_conv.cuh"
@@ -194,8 +195,7 @@ int launch_hash_gather(const HashArgs &a, const int32_t *ids, const int32_t *cu,
 struct BwdPlan {
     int wmax = 0, GF = 0, tiles_max = 0, groups_max = 0;
     size_t a = 0, b = 0, tile_cnt = 0, ctl = 0, ctl_bytes = 0, group_cnt = 0, barrier = 0;
-    size_t seg_status = 0, seg_ready = 0, seg_gen = 0, seg_done = 0;
-    size_t pb = 0, pe = 0, meta = 0, total = 0;
+    size_t wcount = 0, bcount = 0, pb = 0, pe = 0, meta = 0, total = 0;
 };
 
 int bwd_plan(int64_t n, int64_t rows, int32_t dim, BwdPlan *P)
@@ -229,12 +229,9 @@ int bwd_plan(int64_t n, int64_t rows, int32_t dim, BwdPlan *P)
     P->ctl = off;
     P->group_cnt = take((size_t)bwd::kMaxPasses * bwd::kRadixMax * P->groups_max * 4);
     P->barrier = take(sizeof(unsigned)); // grid-barrier counter of the one-launch sort
-    // the reduce's look-back words, ready flags, generation and finish count
-    P->seg_status = take((size_t)P->wmax * 8);
-    P->seg_ready = take((size_t)P->wmax * 4);
-    P->seg_gen = take(sizeof(unsigned));
-    P->seg_done = take(sizeof(unsigned));
     P->ctl_bytes = off - P->ctl;
+    P->wcount = take((size_t)P->wmax * 4);
+    P->bcount = take((size_t)ceil_div(P->wmax, bwd::kSegWarps) * 4);
     P->pb = take((size_t)P->wmax * dim * 8);
     P->pe = take((size_t)P->wmax * dim * 8);
     P->meta = take((size_t)P->wmax * sizeof(bwd::SegMeta));
@@ -459,14 +456,83 @@ uint64_t cross_wait_ns()
     return v;
 }
 
-// Sorts the pairs of `sh` into buffer a of the workspace.
+// The on-chip sort (one cluster per segment, cluster_sort.cuh) where the
+// segments fit a cluster and the device runs such clusters; *launched is
+// false otherwise (nothing ran).
+int launch_sort_cluster(const int32_t *idx, const SortShape &sh, const BwdPlan &P, char *ws,
+                        cudaStream_t stream, bool *launched)
+{
+    using namespace bwd;
+    *launched = false;
+    if (sh.L < 1 || sh.L > kClusterMaxSegment)
+        return ENGRAM_OK;
+    SortArgs args;
+    ENGRAM_TRY(sort_args(idx, sh, kSortItemsMax, P, ws, &args));
+    const size_t smem = sizeof(ClusterSmem);
+    static std::once_flag once;
+    static cudaError_t attr_rc = cudaSuccess;
+    std::call_once(once, [&] {
+        attr_rc = cudaFuncSetAttribute(cluster_sort_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    });
+    if (attr_rc != cudaSuccess) {
+        (void)cudaGetLastError();
+        return ENGRAM_OK;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(sh.S * kClusterCtas));
+    cfg.blockDim = dim3(kClusterThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kClusterCtas;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, cluster_sort_kernel, &cfg) != cudaSuccess ||
+        clusters < 1) {
+        (void)cudaGetLastError();
+        return ENGRAM_OK;
+    }
+    if (cudaLaunchKernelEx(&cfg, cluster_sort_kernel, args) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return ENGRAM_OK;
+    }
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    *launched = true;
+    return ENGRAM_OK;
+}
+
+// ENGRAM_SORT_NO_CLUSTER=1 in the environment (read once per process) keeps
+// the sort off the on-chip cluster form, so that the grid-wide form can be
+// checked on shapes the cluster form would take.
+bool sort_no_cluster()
+{
+    static const bool v = [] {
+        const char *e = std::getenv("ENGRAM_SORT_NO_CLUSTER");
+        return e != nullptr && e[0] == '1';
+    }();
+    return v;
+}
+
+// Sorts the pairs of `sh` into buffer a of the workspace: on chip where a
+// segment fits one cluster, else the grid-wide sort in one cooperative
+// launch, else two launches per pass.
 int launch_sort(const int32_t *idx, const SortShape &sh, const BwdPlan &P, char *ws,
                 cudaStream_t stream)
 {
     using namespace bwd;
+    bool launched = false;
+    if (!sort_separate_launches() && !sort_no_cluster()) {
+        ENGRAM_TRY(launch_sort_cluster(idx, sh, P, ws, stream, &launched));
+        if (launched)
+            return ENGRAM_OK;
+    }
     if (cudaMemsetAsync(ws + P.ctl, 0, P.ctl_bytes, stream) != cudaSuccess)
         return ENGRAM_ECUDA;
-    bool launched = false;
     int items = 0;
     if (!sort_separate_launches()) {
         int sms = 0;
@@ -518,13 +584,18 @@ int launch_seg(const unsigned long long *items, int64_t n, const BwdPlan &P, con
     const int W = (int)std::max<int64_t>(
         1, std::min<int64_t>(std::min<int64_t>(res, P.wmax), ceil_div(n, 32)));
     const int blocks = (int)ceil_div(W, kSegWarps);
-    const SegSync sy{(unsigned long long *)(ws + P.seg_status), (unsigned *)(ws + P.seg_ready),
-                     (unsigned *)(ws + P.seg_gen), (unsigned *)(ws + P.seg_done)};
+    auto *wcount = (uint32_t *)(ws + P.wcount);
+    auto *bcount = (uint32_t *)(ws + P.bcount);
     auto *pb = (double *)(ws + P.pb);
     auto *pe = (double *)(ws + P.pe);
     auto *meta = (SegMeta *)(ws + P.meta);
-    fn<<<blocks, kSegThreads, smem, stream>>>(items, n, W, sy, dout, dim, batch, stage_bytes,
-                                              uniq, grads, pb, pe, meta, num_unique);
+    seg_count<<<blocks, kSegThreads, 0, stream>>>(items, n, W, wcount, bcount);
+    ENGRAM_TRY(after_launch());
+    fn<<<blocks, kSegThreads, smem, stream>>>(items, n, W, wcount, bcount, dout, dim, batch,
+                                              stage_bytes, uniq, grads, pb, pe, meta,
+                                              num_unique);
+    ENGRAM_TRY(after_launch());
+    seg_fixup<GF><<<blocks, kSegThreads, 0, stream>>>(W, dim, pb, pe, meta, uniq, grads);
     return after_launch();
 }
 

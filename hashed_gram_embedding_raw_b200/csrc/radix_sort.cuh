@@ -328,8 +328,7 @@ template <int ITEMS>
 __device__ __forceinline__ void local_starts(SortSmem<ITEMS> &sm, const PassInfo &P,
                                              const uint32_t (&tcount)[2])
 {
-    // (the barrier after the writes below protects sm.warp)
-    uint32_t tstart = block_exclusive_scan<false>(tcount[0] + tcount[1], sm.warp, nullptr);
+    uint32_t tstart = block_exclusive_scan(tcount[0] + tcount[1], sm.warp, nullptr);
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
         const int d = my_digit(P, e);
@@ -405,17 +404,18 @@ __device__ __forceinline__ void tile_offsets(SortSmem<ITEMS> &sm, const SortArgs
                         excl[e] += c[q];
                 }
             }
-            // the tile counts before this tile in its group, in one round of
-            // loads (only the needed ones are issued)
             const int t0 = kg * kTilesPerGroup;
-            uint32_t c[kTilesPerGroup];
+            for (int q0 = 0; q0 < kTilesPerGroup; q0 += 16) {
+                uint32_t c[16];
 #pragma unroll
-            for (int q = 0; q < kTilesPerGroup; ++q)
-                c[q] = t0 + q < g.k ? load_u32<COHERENT>(segt + (size_t)(t0 + q) * kRadixMax + d)
-                                    : 0u;
+                for (int q = 0; q < 16; ++q)
+                    c[q] = t0 + q0 + q < g.k
+                               ? load_u32<COHERENT>(segt + (size_t)(t0 + q0 + q) * kRadixMax + d)
+                               : 0u;
 #pragma unroll
-            for (int q = 0; q < kTilesPerGroup; ++q)
-                excl[e] += c[q];
+                for (int q = 0; q < 16; ++q)
+                    excl[e] += c[q];
+            }
         }
     }
 
@@ -425,13 +425,13 @@ __device__ __forceinline__ void tile_offsets(SortSmem<ITEMS> &sm, const SortArgs
     const uint32_t seg_base = (uint32_t)(g.seg * a.L);
     uint32_t dbase, tstart = 0;
     if constexpr (WITH_TSTART) {
-        const unsigned long long both = block_exclusive_scan64<false>(
+        const unsigned long long both = block_exclusive_scan64(
             ((unsigned long long)(total[0] + total[1]) << 32) | (tcount[0] + tcount[1]),
             (unsigned long long *)sm.warp2);
         tstart = (uint32_t)both;
         dbase = (uint32_t)(both >> 32);
     } else {
-        dbase = block_exclusive_scan<false>(total[0] + total[1], sm.warp, nullptr);
+        dbase = block_exclusive_scan(total[0] + total[1], sm.warp, nullptr);
     }
 #pragma unroll
     for (int e = 0; e < 2; ++e) {

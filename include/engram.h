@@ -65,9 +65,6 @@ extern "C" {
                                          (results of that call are invalid) */
 #define ENGRAM_DEVERR_COPY_TIMEOUT 8u /* a bulk copy into shared memory did not complete in
                                          time (results of that call are invalid) */
-#define ENGRAM_DEVERR_REDUCE_TIMEOUT 16u /* a warp of the backward reduce gave up waiting for
-                                            an earlier warp's segment count or partial sum
-                                            (results of that call are invalid) */
 /* Same type as cudaStream_t, without requiring the CUDA headers. */
 typedef struct CUstream_st *engram_stream_t;
 

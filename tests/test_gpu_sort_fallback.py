@@ -1,7 +1,9 @@
-"""The backward sort's separate-launch form -- what a device without
-cooperative launch runs: two launches per pass on 2,048-pair tiles -- forced
-with ENGRAM_SORT_SEPARATE_LAUNCHES=1 in a child process, against the
-one-launch sort in another child on the same inputs. A stable sort has one
+"""The backward sort's three forms on the same inputs, each in a child
+process, compared bit for bit: the on-chip cluster sort (segments of up to
+65,536 lookups, the default there), the grid-wide sort in one cooperative
+launch (forced with ENGRAM_SORT_NO_CLUSTER=1), and the separate-launch form --
+what a device without cooperative launch runs: two launches per pass on
+2,048-pair tiles -- forced with ENGRAM_SORT_SEPARATE_LAUNCHES=1. A stable sort has one
 result, so the distinct rows and their fp32 sums must be identical bit for
 bit. The sizes cover one tile, a ragged single tile, many resident tiles and
 more tiles than resident blocks; half the lookups hit a few hot rows. The
@@ -28,7 +30,7 @@ sys.path.insert(0, sys.argv[1])
 import hashed_gram_embedding_raw_b200 as E
 rows = 320_001_536
 out = {}
-for n in (1, 1000, 250_007, 2_000_003):
+for n in (1, 1000, 65_536, 250_007, 2_000_003):
     rng = np.random.Generator(np.random.PCG64(n))
     idx = np.where(rng.random(n) < 0.5, rng.integers(0, 40, n),
                    rng.integers(0, rows, n)).astype(np.int32)
@@ -42,7 +44,7 @@ from workloads import head_params, random_stream
 import oracle
 cfg = dict(head_params("full"), dim=16)
 p = E.make_params(cfg)
-for T in (1, 63, 15_625, 131_072):
+for T in (1, 63, 15_625, 65_536, 65_537, 131_072):
     ids, cu = random_stream(T, T, 2000, cfg["eos_id"], 0.01, nseq=1 + T // 4096)
     idx = oracle.hash_ids(ids, cu, cfg).astype(np.int32)
     dout = torch.randn(idx.size, 16, generator=torch.Generator().manual_seed(T % 997))
@@ -55,17 +57,19 @@ np.savez(sys.argv[2], **out)
 """
 
 
-def run_child(tmp_path, separate: bool):
-    path = tmp_path / ("separate.npz" if separate else "one_launch.npz")
-    env = dict(os.environ, ENGRAM_SORT_SEPARATE_LAUNCHES="1" if separate else "0")
+def run_child(tmp_path, form: str):
+    path = tmp_path / (form + ".npz")
+    env = dict(os.environ, ENGRAM_SORT_SEPARATE_LAUNCHES="1" if form == "separate" else "0",
+               ENGRAM_SORT_NO_CLUSTER="1" if form == "grid" else "0")
     subprocess.run([sys.executable, "-c", CHILD, ROOT, str(path)], env=env, check=True,
                    timeout=600)
     return np.load(path)
 
 
-def test_separate_launch_sort_matches_one_launch(tmp_path):
-    split = run_child(tmp_path, True)
-    coop = run_child(tmp_path, False)
-    assert sorted(split.files) == sorted(coop.files)
-    for k in coop.files:
-        assert np.array_equal(split[k], coop[k]), k
+def test_sort_forms_agree_bit_for_bit(tmp_path):
+    forms = {f: run_child(tmp_path, f) for f in ("default", "grid", "separate")}
+    base = forms["default"]
+    for name, got in forms.items():
+        assert sorted(got.files) == sorted(base.files), name
+        for k in base.files:
+            assert np.array_equal(got[k], base[k]), (name, k)
