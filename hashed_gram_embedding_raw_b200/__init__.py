@@ -9,7 +9,8 @@ has not been built (`python hashed_gram_embedding_raw_b200/build.py`).
 """
 
 from ._binding import (ENGRAM_BF16, ENGRAM_CONV_NORM, ENGRAM_CONV_RESIDUAL, ENGRAM_CONV_SILU,
-                       ENGRAM_DEVERR_COPY_TIMEOUT, ENGRAM_DEVERR_CU_SEQLENS,
+                       ENGRAM_DEVERR_CAPACITY, ENGRAM_DEVERR_COPY_TIMEOUT,
+                       ENGRAM_DEVERR_CU_SEQLENS,
                        ENGRAM_DEVERR_ROW_RANGE, ENGRAM_DEVERR_SORT_TIMEOUT,
                        ENGRAM_EINVAL, ENGRAM_ECUDA, ENGRAM_ENOSPC, ENGRAM_F16, ENGRAM_F32,
                        ENGRAM_NOALLOC_SCRATCH_BYTES, ENGRAM_OK, EXPORTED, LIB_PATH,
@@ -22,12 +23,14 @@ from ._binding import (ENGRAM_BF16, ENGRAM_CONV_NORM, ENGRAM_CONV_RESIDUAL, ENGR
                        engram_hash_gather_slice, engram_host_floor_mod, engram_ple_short_conv,
                        engram_ple_short_conv_backward,
                        engram_ple_short_conv_backward_workspace_size, engram_sparse_adam,
-                       engram_owner_bucket, engram_owner_bucket_workspace_size,
+                       engram_owner_bucket, engram_owner_bucket_padded,
+                       engram_owner_bucket_workspace_size,
                        engram_launch_count, lib, make_params, status_string)
 
 __all__ = [
     "ENGRAM_BF16", "ENGRAM_CONV_NORM", "ENGRAM_CONV_RESIDUAL", "ENGRAM_CONV_SILU",
-    "ENGRAM_DEVERR_COPY_TIMEOUT", "ENGRAM_DEVERR_CU_SEQLENS", "ENGRAM_DEVERR_ROW_RANGE",
+    "ENGRAM_DEVERR_CAPACITY", "ENGRAM_DEVERR_COPY_TIMEOUT", "ENGRAM_DEVERR_CU_SEQLENS",
+    "ENGRAM_DEVERR_ROW_RANGE",
     "ENGRAM_DEVERR_SORT_TIMEOUT", "ENGRAM_EINVAL",
     "ENGRAM_ECUDA", "ENGRAM_ENOSPC", "ENGRAM_F16", "ENGRAM_F32",
     "ENGRAM_NOALLOC_SCRATCH_BYTES", "ENGRAM_OK", "EXPORTED", "LIB_PATH", "AdamParams", "ConvParams",
@@ -38,6 +41,7 @@ __all__ = [
     "engram_gather", "engram_get_device_error", "engram_hash", "engram_hash_gather",
     "engram_hash_gather_slice", "engram_grouped_rms_norm", "engram_ple_short_conv",
     "engram_ple_short_conv_backward", "engram_ple_short_conv_backward_workspace_size",
-    "engram_sparse_adam", "engram_owner_bucket", "engram_owner_bucket_workspace_size",
+    "engram_sparse_adam", "engram_owner_bucket", "engram_owner_bucket_padded",
+    "engram_owner_bucket_workspace_size",
     "engram_host_floor_mod", "engram_launch_count", "lib", "make_params", "status_string",
 ]

@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(_PKG, "_lib", "libengram_b200.so")
 ENGRAM_OK, ENGRAM_EINVAL, ENGRAM_ENOSPC, ENGRAM_ECUDA = 0, 1, 2, 3
 ENGRAM_F32, ENGRAM_BF16, ENGRAM_F16 = 0, 1, 2
 ENGRAM_DEVERR_ROW_RANGE, ENGRAM_DEVERR_CU_SEQLENS, ENGRAM_DEVERR_SORT_TIMEOUT = 1, 2, 4
-ENGRAM_DEVERR_COPY_TIMEOUT = 8
+ENGRAM_DEVERR_COPY_TIMEOUT, ENGRAM_DEVERR_CAPACITY = 8, 16
 ENGRAM_CONV_NORM, ENGRAM_CONV_SILU, ENGRAM_CONV_RESIDUAL = 1, 2, 4
 ENGRAM_MAX_NGRAM, ENGRAM_MAX_HEADS = 4, 32
 
@@ -36,7 +36,7 @@ EXPORTED = (
     "engram_ple_short_conv", "engram_grouped_rms_norm", "engram_sparse_adam",
     "engram_ple_short_conv_backward", "engram_ple_short_conv_backward_workspace_size",
     "engram_owner_bucket", "engram_owner_bucket_workspace_size",
-    "engram_backward_heads", "engram_backward_sort_heads",
+    "engram_backward_heads", "engram_backward_sort_heads", "engram_owner_bucket_padded",
 )
 
 ENGRAM_NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -148,6 +148,7 @@ def _load():
         "engram_owner_bucket_workspace_size": [i64, i32, ctypes.POINTER(sz)],
         "engram_backward_heads": [P, P, i64, P, i32, P, P, P, P, sz, P],
         "engram_backward_sort_heads": [P, P, i64, P, sz, P],
+        "engram_owner_bucket_padded": [P, i64, i64, i32, i64, P, P, P, P, P, sz, P],
     }
     for name, args in sig.items():
         fn = getattr(L, name)
@@ -572,6 +573,38 @@ def engram_owner_bucket(rows: torch.Tensor, rows_per_owner: int, owners: int, se
                                    _ptr(send_rows), _ptr(src_pos), _ptr(dst_pos), _ptr(counts),
                                    _ptr(workspace), workspace.numel(), _stream(stream)),
            "engram_owner_bucket")
+    return send_rows, src_pos, dst_pos, counts
+
+
+def engram_owner_bucket_padded(rows: torch.Tensor, rows_per_owner: int, owners: int,
+                               capacity: int, send_rows=None, src_pos=None, dst_pos=None,
+                               counts=None, workspace=None, stream=None):
+    """engram_owner_bucket into fixed-capacity segments: (send_rows
+    [owners * capacity], src_pos [owners * capacity] with -1 padding, dst_pos
+    [n] (-1 for a lookup dropped past the capacity), counts [owners])."""
+    _cuda(rows, "rows", torch.int32)
+    n = rows.numel()
+    dev = rows.device
+    slots = int(owners) * int(capacity)
+
+    def buf(t, name, size):
+        t = torch.empty(size, dtype=torch.int32, device=dev) if t is None else t
+        _cuda(t, name, torch.int32)
+        if t.numel() != size:
+            raise ValueError(f"{name} must hold {size} elements")
+        return t
+
+    send_rows, src_pos = buf(send_rows, "send_rows", slots), buf(src_pos, "src_pos", slots)
+    dst_pos, counts = buf(dst_pos, "dst_pos", n), buf(counts, "counts", int(owners))
+    if workspace is None:
+        workspace = torch.empty(max(16, engram_owner_bucket_workspace_size(n, owners)),
+                                dtype=torch.uint8, device=dev)
+    _cuda(workspace, "workspace", torch.uint8)
+    _check(lib.engram_owner_bucket_padded(_ptr(rows), n, int(rows_per_owner), int(owners),
+                                          int(capacity), _ptr(send_rows), _ptr(src_pos),
+                                          _ptr(dst_pos), _ptr(counts), _ptr(workspace),
+                                          workspace.numel(), _stream(stream)),
+           "engram_owner_bucket_padded")
     return send_rows, src_pos, dst_pos, counts
 
 

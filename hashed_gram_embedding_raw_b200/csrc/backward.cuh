@@ -52,9 +52,11 @@ __device__ __forceinline__ void range_of(int64_t n, int64_t w, int64_t W, int64_
 }
 
 // Segment heads (first item, or key differs from the previous one) per range
-// (wcount) and per block of kSegWarps ranges (bcount).
+// (wcount) and per block of kSegWarps ranges (bcount). The run of key
+// `absent` (absent lookups; it sorts last) is not counted, so num_unique
+// leaves it out; its sum lands past the counted rows.
 __global__ void __launch_bounds__(kSegThreads)
-    seg_count(const unsigned long long *__restrict__ items, int64_t n, int W,
+    seg_count(const unsigned long long *__restrict__ items, int64_t n, int W, uint32_t absent,
               uint32_t *__restrict__ wcount, uint32_t *__restrict__ bcount)
 {
     __shared__ uint32_t s_cnt[kSegWarps];
@@ -75,7 +77,7 @@ __global__ void __launch_bounds__(kSegThreads)
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const int64_t i = c0 + 32 * q + lane;
-                cnt += __popc(__ballot_sync(kFull, i < b && key[q] != prev[q]));
+                cnt += __popc(__ballot_sync(kFull, i < b && key[q] != prev[q] && key[q] != absent));
             }
         }
         if (lane == 0)

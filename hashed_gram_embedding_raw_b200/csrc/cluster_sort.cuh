@@ -111,10 +111,7 @@ __global__ void __launch_bounds__(kClusterThreads, 1) cluster_sort_kernel(SortAr
             const int i = wbase + r * 32 + lane;
             if (i < cnt) {
                 if (P.first) {
-                    const int64_t j = (int64_t)(lo + i) * a.S + seg;
-                    const uint32_t key = (uint32_t)__ldg(a.idx + j) - (uint32_t)a.off[seg];
-                    bad |= key >= a.size[seg];
-                    it[r] = ((uint64_t)key << 32) | (uint32_t)j;
+                    it[r] = first_item(a, seg, (int64_t)(lo + i) * a.S + seg, bad);
                 } else {
                     it[r] = sm.buf[cur][i];
                 }

@@ -194,6 +194,7 @@ int launch_hash_gather(const HashArgs &a, const int32_t *ids, const int32_t *cu,
 // of either form (one segment, or one per head) at any tile size.
 struct BwdPlan {
     int wmax = 0, GF = 0, tiles_max = 0, groups_max = 0;
+    int64_t rows = 0;
     size_t a = 0, b = 0, tile_cnt = 0, ctl = 0, ctl_bytes = 0, group_cnt = 0, barrier = 0;
     size_t wcount = 0, bcount = 0, pb = 0, pe = 0, meta = 0, total = 0;
 };
@@ -205,6 +206,7 @@ int bwd_plan(int64_t n, int64_t rows, int32_t dim, BwdPlan *P)
         return ENGRAM_EINVAL;
     int sms = 0;
     ENGRAM_TRY(device_sms(&sms));
+    P->rows = rows;
     // warps of seg_reduce: at most 32 per SM (its resident limit) and one per
     // 32 lookups, so the fp64 partials below shrink with small n
     P->wmax = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)sms * 32, ceil_div(n, 32)));
@@ -255,6 +257,7 @@ struct SortShape {
     int64_t L = 0;
     int32_t off[bwd::kMaxSegments] = {};
     uint32_t size[bwd::kMaxSegments] = {};
+    bool pad = false; // negative indices are absent lookups, keyed size[s]
 };
 
 int bit_width(uint64_t v) // bits needed for 0 .. v
@@ -265,14 +268,16 @@ int bit_width(uint64_t v) // bits needed for 0 .. v
     return b;
 }
 
-// The plain sort: one segment of all n lookups over the whole table.
-SortShape plain_shape(int64_t n, int64_t rows)
+// The plain sort: one segment of all n lookups over the whole table; with
+// `pad`, a negative index is an absent lookup that sorts after every row.
+SortShape plain_shape(int64_t n, int64_t rows, bool pad)
 {
     SortShape sh;
     sh.S = 1;
     sh.L = n;
     sh.off[0] = 0;
     sh.size[0] = (uint32_t)std::min<int64_t>(rows, UINT32_MAX);
+    sh.pad = pad;
     return sh;
 }
 
@@ -288,7 +293,7 @@ SortShape head_shape(const engram_params_t *p, int64_t T)
              (h == 0 || o >= p->offsets[h - 1] + p->vocab_sizes[h - 1]);
     }
     if (!ok)
-        return plain_shape(T * std::max(H, 1), p->table_rows);
+        return plain_shape(T * std::max(H, 1), p->table_rows, false);
     SortShape sh;
     sh.S = H;
     sh.L = T;
@@ -352,9 +357,9 @@ int sort_args(const int32_t *idx, const SortShape &sh, int items, const BwdPlan 
     using namespace bwd;
     SortArgs &a = *out;
     std::memset(&a, 0, sizeof(a));
-    int key_bits = 1;
+    int key_bits = 1; // the largest key: size - 1, or size for an absent lookup
     for (int s = 0; s < sh.S; ++s)
-        key_bits = std::max(key_bits, bit_width((uint64_t)sh.size[s] - 1));
+        key_bits = std::max(key_bits, bit_width((uint64_t)sh.size[s] - (sh.pad ? 0 : 1)));
     a.passes = (key_bits + kDigitBitsMax - 1) / kDigitBitsMax;
     if (a.passes > kMaxPasses)
         return ENGRAM_EINVAL;
@@ -381,6 +386,7 @@ int sort_args(const int32_t *idx, const SortShape &sh, int items, const BwdPlan 
         a.off[s] = sh.off[s];
         a.size[s] = sh.size[s];
     }
+    a.pad = sh.pad;
     return ENGRAM_OK;
 }
 
@@ -491,12 +497,24 @@ int launch_sort_cluster(const int32_t *idx, const SortShape &sh, const BwdPlan &
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    int clusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&clusters, cluster_sort_kernel, &cfg) != cudaSuccess ||
-        clusters < 1) {
+    // whether the device runs such clusters at all: asked once per device (a
+    // query inside a stream capture could end the capture)
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128)
+        return ENGRAM_ECUDA;
+    static std::atomic<int> cluster_ok[128];
+    int ok = cluster_ok[dev].load(std::memory_order_relaxed);
+    if (ok == 0) {
+        int clusters = 0;
+        ok = cudaOccupancyMaxActiveClusters(&clusters, cluster_sort_kernel, &cfg) == cudaSuccess &&
+                     clusters >= 1
+                 ? 1
+                 : -1;
         (void)cudaGetLastError();
-        return ENGRAM_OK;
+        cluster_ok[dev].store(ok, std::memory_order_relaxed);
     }
+    if (ok < 0)
+        return ENGRAM_OK;
     if (cudaLaunchKernelEx(&cfg, cluster_sort_kernel, args) != cudaSuccess) {
         (void)cudaGetLastError();
         return ENGRAM_OK;
@@ -589,7 +607,9 @@ int launch_seg(const unsigned long long *items, int64_t n, const BwdPlan &P, con
     auto *pb = (double *)(ws + P.pb);
     auto *pe = (double *)(ws + P.pe);
     auto *meta = (SegMeta *)(ws + P.meta);
-    seg_count<<<blocks, kSegThreads, 0, stream>>>(items, n, W, wcount, bcount);
+    // an absent lookup's item has key table_rows: its run is no distinct row
+    seg_count<<<blocks, kSegThreads, 0, stream>>>(items, n, W, (uint32_t)P.rows, wcount,
+                                                  bcount);
     ENGRAM_TRY(after_launch());
     fn<<<blocks, kSegThreads, smem, stream>>>(items, n, W, wcount, bcount, dout, dim, batch,
                                               stage_bytes, uniq, grads, pb, pe, meta,
@@ -774,7 +794,7 @@ int engram_backward_sort(const int32_t *idx, int64_t n, int64_t table_rows, int3
         return ENGRAM_OK;
     if (idx == nullptr)
         return ENGRAM_EINVAL;
-    return launch_sort(idx, plain_shape(n, table_rows), P, (char *)workspace,
+    return launch_sort(idx, plain_shape(n, table_rows, true), P, (char *)workspace,
                        (cudaStream_t)stream);
 }
 
@@ -804,7 +824,7 @@ int engram_backward(const int32_t *idx, int64_t n, int64_t table_rows, int32_t d
         return ENGRAM_EINVAL;
     cudaStream_t s = (cudaStream_t)stream;
     if (n > 0)
-        ENGRAM_TRY(launch_sort(idx, plain_shape(n, table_rows), P, (char *)workspace, s));
+        ENGRAM_TRY(launch_sort(idx, plain_shape(n, table_rows, true), P, (char *)workspace, s));
     return launch_reduce(n, dim, dout, dtype, uniq_rows, row_grads, num_unique, P,
                          (char *)workspace, s);
 }
@@ -895,7 +915,7 @@ int engram_backward_noalloc(const int32_t *idx, int64_t n, int64_t table_rows, i
     cudaStream_t s = (cudaStream_t)stream;
     // launch_sort clears the sort's control block in the array on every call
     if (n > 0)
-        ENGRAM_TRY(launch_sort(idx, plain_shape(n, table_rows), P, ws, s));
+        ENGRAM_TRY(launch_sort(idx, plain_shape(n, table_rows, true), P, ws, s));
     return launch_reduce(n, dim, dout, dtype, uniq_rows, row_grads, num_unique, P, ws, s);
 }
 
@@ -1532,21 +1552,27 @@ int engram_owner_bucket_workspace_size(int64_t n, int32_t owners, size_t *bytes)
     return ENGRAM_OK;
 }
 
-int engram_owner_bucket(const int32_t *rows, int64_t n, int64_t rows_per_owner, int32_t owners,
-                        int32_t *send_rows, int32_t *src_pos, int32_t *dst_pos, int32_t *counts,
-                        void *workspace, size_t workspace_bytes, engram_stream_t stream)
+} // extern "C"
+
+namespace {
+
+int owner_bucket(const int32_t *rows, int64_t n, int64_t rows_per_owner, int32_t owners,
+                 int64_t cap, int32_t *send_rows, int32_t *src_pos, int32_t *dst_pos,
+                 int32_t *counts, void *workspace, size_t workspace_bytes, engram_stream_t stream)
 {
     size_t need = 0;
     ENGRAM_TRY(engram_owner_bucket_workspace_size(n, owners, &need));
-    if (rows_per_owner < 1 || counts == nullptr)
+    if (rows_per_owner < 1 || counts == nullptr || cap < 0 || cap > INT32_MAX ||
+        cap * owners > INT32_MAX)
         return ENGRAM_EINVAL;
-    if (n > 0 && (rows == nullptr || send_rows == nullptr || src_pos == nullptr ||
-                  dst_pos == nullptr || workspace == nullptr))
+    const int64_t slots = cap > 0 ? cap * owners : n; // grouped positions
+    if ((n > 0 && (rows == nullptr || dst_pos == nullptr || workspace == nullptr)) ||
+        (slots > 0 && (send_rows == nullptr || src_pos == nullptr)))
         return ENGRAM_EINVAL;
-    const size_t nb = (size_t)n * sizeof(int32_t);
-    if (overlaps(rows, nb, send_rows, nb) || overlaps(rows, nb, src_pos, nb) ||
-        overlaps(rows, nb, dst_pos, nb) || overlaps(send_rows, nb, src_pos, nb) ||
-        overlaps(send_rows, nb, dst_pos, nb) || overlaps(src_pos, nb, dst_pos, nb))
+    const size_t nb = (size_t)n * sizeof(int32_t), sb = (size_t)slots * sizeof(int32_t);
+    if (overlaps(rows, nb, send_rows, sb) || overlaps(rows, nb, src_pos, sb) ||
+        overlaps(rows, nb, dst_pos, nb) || overlaps(send_rows, sb, src_pos, sb) ||
+        overlaps(send_rows, sb, dst_pos, nb) || overlaps(src_pos, sb, dst_pos, nb))
         return ENGRAM_EINVAL;
     if (workspace_bytes < need)
         return ENGRAM_ENOSPC;
@@ -1562,20 +1588,46 @@ int engram_owner_bucket(const int32_t *rows, int64_t n, int64_t rows_per_owner, 
     a.send_rows = send_rows;
     a.src_pos = src_pos;
     a.dst_pos = dst_pos;
+    a.cap = cap;
     cudaStream_t s = (cudaStream_t)stream;
     if (n > 0) {
         owner::owner_count<<<a.ntiles, owner::kThreads, 0, s>>>(a);
         ENGRAM_TRY(after_launch());
     }
+    const int32_t ntiles = a.ntiles;
     if (n == 0)
         a.ntiles = 0;  // counts only: all zero
     owner::owner_scan<<<1, owner::kThreads, 0, s>>>(a);
     ENGRAM_TRY(after_launch());
-    if (n > 0) {
+    a.ntiles = ntiles;
+    if (n > 0 || slots > 0) {
         owner::owner_scatter<<<a.ntiles, owner::kThreads, 0, s>>>(a);
         ENGRAM_TRY(after_launch());
     }
     return ENGRAM_OK;
+}
+
+} // namespace
+
+extern "C" {
+
+int engram_owner_bucket(const int32_t *rows, int64_t n, int64_t rows_per_owner, int32_t owners,
+                        int32_t *send_rows, int32_t *src_pos, int32_t *dst_pos, int32_t *counts,
+                        void *workspace, size_t workspace_bytes, engram_stream_t stream)
+{
+    return owner_bucket(rows, n, rows_per_owner, owners, 0, send_rows, src_pos, dst_pos, counts,
+                        workspace, workspace_bytes, stream);
+}
+
+int engram_owner_bucket_padded(const int32_t *rows, int64_t n, int64_t rows_per_owner,
+                               int32_t owners, int64_t capacity, int32_t *send_rows,
+                               int32_t *src_pos, int32_t *dst_pos, int32_t *counts,
+                               void *workspace, size_t workspace_bytes, engram_stream_t stream)
+{
+    if (capacity < 1)
+        return ENGRAM_EINVAL;
+    return owner_bucket(rows, n, rows_per_owner, owners, capacity, send_rows, src_pos, dst_pos,
+                        counts, workspace, workspace_bytes, stream);
 }
 
 } // extern "C"

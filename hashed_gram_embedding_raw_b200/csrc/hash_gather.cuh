@@ -252,7 +252,8 @@ __global__ void __launch_bounds__(kHashThreads)
     }
 }
 
-// engram_gather: out[i] = table[idx[i]] for n lookups of V 16-byte vectors.
+// engram_gather: out[i] = table[idx[i]] for n lookups of V 16-byte vectors
+// (a zero row where idx[i] < 0).
 // A warp moves 32 rows at a time: lane l handles vectors l, l+32, ... of the
 // 32 x V chunk, taking each vector's row index from the owning lane by
 // shuffle, so stores stay fully coalesced for any V.
@@ -271,11 +272,13 @@ __global__ void __launch_bounds__(kHashThreads, 2)
     warp_range(n, w, nwarps, ib, ie);
     for (int64_t i0 = ib; i0 < ie; i0 += 32) {
         const int nrow = (int)min64(32, ie - i0);
+        // a negative index marks an absent lookup (padding): a zero row; an
+        // index past the table is an error, also answered with a zero row
         int32_t my = lane < nrow ? __ldg(idx + i0 + lane) : 0;
-        if (lane < nrow && (my < 0 || (int64_t)my >= rows)) {
+        if (lane < nrow && (int64_t)my >= rows)
             raise_device_error(ENGRAM_DEVERR_ROW_RANGE);
+        if (my < 0 || (int64_t)my >= rows)
             my = -1;
-        }
         uint4 *dst = out + (size_t)i0 * V;
         if constexpr (VT != 0) {
             constexpr int BATCH = VT < 20 ? VT : 20;   // vectors in flight per lane

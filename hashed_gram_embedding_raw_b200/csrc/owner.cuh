@@ -20,6 +20,12 @@
 // so lookups of one owner keep their original order. A row outside
 // [0, owners * rows_per_owner) is routed to the last owner with local row -1,
 // which that owner's lookup rejects, and raises ENGRAM_DEVERR_ROW_RANGE here.
+// In the fixed-capacity layout (the pages' _fixed_capacity_all_to_all: every
+// owner's segment padded to one capacity agreed ahead of time, so the
+// exchanges have static sizes and need no counts on the host), owner o's
+// lookups go to positions o * cap + rank, the rest of the segment is padding
+// (-1), and lookups past the capacity are dropped (dst_pos -1) with
+// ENGRAM_DEVERR_CAPACITY.
 #pragma once
 
 #include "common.cuh"
@@ -42,6 +48,7 @@ struct OwnerArgs {
     uint32_t *tile_off;   // [ntiles][owners] exclusive starts (owner start + earlier tiles)
     int32_t *counts;      // [owners]
     int32_t *send_rows, *src_pos, *dst_pos;
+    int64_t cap;          // > 0: fixed-capacity segments [owners][cap]; 0: compact
 };
 
 __device__ __forceinline__ int owner_of(int32_t row, const OwnerArgs &a, bool &bad)
@@ -105,15 +112,22 @@ __global__ void __launch_bounds__(kThreads) owner_scan(const OwnerArgs a)
                 }
         }
         total[o] = run;
-        a.counts[o] = (int32_t)run;
+        if (a.cap > 0 && (int64_t)run > a.cap)
+            raise_device_error(ENGRAM_DEVERR_CAPACITY);
+        a.counts[o] = (int32_t)(a.cap > 0 ? min64(run, a.cap) : run);
     }
     __syncthreads();
     if (o < a.owners) {
-        uint32_t start = 0;
-        for (int q = 0; q < o; ++q)
-            start += total[q];
+        // owner o's segment starts after the earlier owners' lookups, or at
+        // o * cap in the fixed-capacity layout
+        int64_t start = 0;
+        if (a.cap > 0)
+            start = (int64_t)o * a.cap;
+        else
+            for (int q = 0; q < o; ++q)
+                start += total[q];
         for (int t = 0; t < a.ntiles; ++t)
-            a.tile_off[(size_t)t * a.owners + o] += start;
+            a.tile_off[(size_t)t * a.owners + o] += (uint32_t)start;
     }
 }
 
@@ -165,9 +179,26 @@ __global__ void __launch_bounds__(kThreads) owner_scatter(const OwnerArgs a)
         const int64_t i = wbase + r * 32 + lane;
         if (i < a.n) {
             const uint32_t p = wcnt[wid][own[r]] + rank[r];
+            if (a.cap > 0 && (int64_t)p - (int64_t)own[r] * a.cap >= a.cap) {
+                a.dst_pos[i] = -1; // past the owner's capacity: dropped (flagged by the scan)
+                continue;
+            }
             a.send_rows[p] = local_row(row[r], own[r], a);
             a.src_pos[p] = (int32_t)i;
             a.dst_pos[i] = (int32_t)p;
+        }
+    }
+    // fixed-capacity layout: the unused slots of every owner's segment are
+    // padding (row -1, position -1), which the lookups and the backward skip
+    if (a.cap > 0) {
+        const int64_t slots = a.cap * a.owners;
+        for (int64_t k = (int64_t)blockIdx.x * kThreads + tid; k < slots;
+             k += (int64_t)gridDim.x * kThreads) {
+            const int o = (int)(k / a.cap);
+            if (k - (int64_t)o * a.cap >= a.counts[o]) {
+                a.send_rows[k] = -1;
+                a.src_pos[k] = -1;
+            }
         }
     }
 }

@@ -80,6 +80,7 @@ struct SortArgs {
     uint32_t spin_limit;       // polls before a grid-barrier wait gives up
     int32_t off[kMaxSegments]; // segment s holds keys off[s] .. off[s] + size[s] - 1
     uint32_t size[kMaxSegments];
+    bool pad;                  // a negative index is an absent lookup: key size[s], not an error
 };
 
 __device__ __forceinline__ uint32_t item_key(uint64_t it) { return (uint32_t)(it >> 32); }
@@ -151,16 +152,29 @@ template <int ITEMS> struct SortSmem {
 // the segment's first row; later passes read the previous pass's output.
 // COHERENT loads go through L2 only (needed when another block of the same
 // launch wrote the data).
+// The first pass's item of lookup j: its key relative to the segment, or the
+// segment's size for an absent lookup (negative index, when a.pad); `bad`
+// is set for an index outside the segment's rows.
+__device__ __forceinline__ uint64_t first_item(const SortArgs &a, int seg, int64_t j, bool &bad)
+{
+    const int32_t v = __ldg(a.idx + j);
+    uint32_t key;
+    if (a.pad && v < 0) {
+        key = a.size[seg];
+    } else {
+        key = (uint32_t)v - (uint32_t)a.off[seg];
+        bad |= key >= a.size[seg];
+    }
+    return ((uint64_t)key << 32) | (uint32_t)j;
+}
+
 template <bool COHERENT>
 __device__ __forceinline__ uint64_t load_item(const SortArgs &a, const void *__restrict__ src,
                                               bool first, const TileGeom &g, int tile_items,
-                                              int i)
+                                              int i, bool &bad)
 {
-    if (first) {
-        const int64_t j = ((int64_t)g.k * tile_items + i) * a.S + g.seg;
-        const uint32_t key = (uint32_t)__ldg(a.idx + j) - (uint32_t)a.off[g.seg];
-        return ((uint64_t)key << 32) | (uint32_t)j;
-    }
+    if (first)
+        return first_item(a, g.seg, ((int64_t)g.k * tile_items + i) * a.S + g.seg, bad);
     const unsigned long long *p = (const unsigned long long *)src + g.begin + i;
     return COHERENT ? __ldcg(p) : __ldg(p);
 }
@@ -207,17 +221,15 @@ __device__ __forceinline__ void count_tile(SortSmem<ITEMS> &sm, const SortArgs &
         sm.cnt[d] = 0;
     __syncthreads();
     uint32_t key[ITEMS];
-#pragma unroll
-    for (int r = 0; r < ITEMS; ++r) {
-        const int i = r * kSortThreads + tid;
-        key[r] = i < g.count ? item_key(load_item<false>(a, src, P.first, g, TILE, i)) : 0u;
-    }
     bool bad = false;
 #pragma unroll
     for (int r = 0; r < ITEMS; ++r) {
+        const int i = r * kSortThreads + tid;
+        key[r] = i < g.count ? item_key(load_item<false>(a, src, P.first, g, TILE, i, bad)) : 0u;
+    }
+#pragma unroll
+    for (int r = 0; r < ITEMS; ++r) {
         const bool valid = r * kSortThreads + tid < g.count;
-        if (P.first && valid && key[r] >= a.size[g.seg])
-            bad = true;
         // one shared-memory add per distinct digit in the warp, so runs of a
         // hot key do not serialise on one counter
         const uint32_t dg = (key[r] >> P.shift) & (uint32_t)(P.ndig - 1);
@@ -254,18 +266,17 @@ __device__ __forceinline__ void rank_tile(SortSmem<ITEMS> &sm, const SortArgs &a
         sm.whist[k >> P.bits][k & (P.ndig - 1)] = 0;
     const int wbase = wid * (32 * ITEMS);
     const uint32_t lt = lanemask_lt();
-#pragma unroll
-    for (int r = 0; r < ITEMS; ++r) {
-        const int i = wbase + r * 32 + lane;
-        it[r] = i < g.count ? load_item<COHERENT>(a, src, P.first, g, TILE, i) : 0ull;
-    }
-    __syncthreads(); // whist zeroed
     bool bad = false;
 #pragma unroll
     for (int r = 0; r < ITEMS; ++r) {
+        const int i = wbase + r * 32 + lane;
+        it[r] = i < g.count ? load_item<COHERENT>(a, src, P.first, g, TILE, i, bad) : 0ull;
+    }
+    bad = bad && check_keys;
+    __syncthreads(); // whist zeroed
+#pragma unroll
+    for (int r = 0; r < ITEMS; ++r) {
         const bool valid = wbase + r * 32 + lane < g.count;
-        if (check_keys && valid && item_key(it[r]) >= a.size[g.seg])
-            bad = true;
         const uint32_t dg = digit_of(it[r], P);
         const uint32_t peers = digit_peers(dg, valid, P.bits);
         const int leader = valid ? __ffs(peers) - 1 : lane;

@@ -1,28 +1,36 @@
-"""Owner-sharded Engram table over an owner group of ranks (engram page,
-Qwen3_8_FlashNextOwnerShardedEmbedding with _FixedCapacityAllToAll).
+"""Owner-sharded Engram table over an owner group of ranks (engram API page,
+Qwen3_8_FlashNextOwnerShardedEmbedding with _FixedCapacityAllToAll /
+_fixed_capacity_all_to_all).
 
 Rank r of W owners holds rows [r * R / W, (r + 1) * R / W) of the packed
 table (R divisible by W, as the page requires). A requesting rank hashes its
-tokens, groups the row lookups by owner (engram_owner_bucket), and
+tokens and groups the row lookups by owner into fixed-capacity segments
+(engram_owner_bucket_padded: W segments of `capacity` slots, the unused
+slots marked -1), then
 
-  1. exchanges the per-owner counts (a W-element all-to-all),
-  2. sends the owner-local rows to their owners (all-to-all of int32),
-  3. each owner gathers the rows from its shard (engram_gather),
-  4. the rows come back in the same grouping (all-to-all of rows) and are
-     put back in request order (engram_gather by each lookup's position).
+  1. sends every owner its segment (an equal-split all-to-all of int32 rows),
+  2. each owner gathers the rows from its shard (engram_gather; padding
+     slots give zero rows),
+  3. the rows come back in the same layout (an equal-split all-to-all) and
+     are put back in request order (engram_gather by each lookup's slot).
 
 The backward sends each lookup's gradient to the owner the row came from
-(engram_gather by grouped position, then the reverse all-to-all), and the
-owner reduces them into compact per-row gradients of its shard
-(engram_backward), ready for engram_sparse_adam on that shard: only the owner
-accumulates and updates a row's gradient.
+(engram_gather by grouped slot, then the same exchange), and the owner
+reduces them into compact per-row gradients of its shard (engram_backward,
+which leaves the padding slots out), ready for engram_sparse_adam on that
+shard: only the owner accumulates and updates a row's gradient.
+
+The capacity is agreed ahead of time, as the page's capacity is, so every
+exchange has the same size whatever the data: no counts cross to the host,
+nothing synchronises with it, and a whole step can be captured in a CUDA
+graph. capacity = n (the default) can never overflow; a smaller one that
+an owner's lookups exceed drops the excess and sets ENGRAM_DEVERR_CAPACITY.
 
 Every step on the device runs in the library's kernels; the exchanges are
-NCCL all-to-alls through torch.distributed (uneven splits, so no padding to a
-common capacity is needed). The routing is written as generators that yield
-at each exchange, so one code path serves a real process group
-(`run_collective`) and a group of ranks emulated in one process on one device
-(`run_lockstep`), where the exchange is a set of device copies.
+NCCL all-to-alls through torch.distributed. The routing is written as
+generators that yield at each exchange, so one code path serves a real
+process group (`run_collective`) and a group of ranks emulated in one process
+on one device (`run_lockstep`), where the exchange is a set of device copies.
 """
 
 from __future__ import annotations
@@ -35,27 +43,18 @@ from . import _binding as B
 
 
 @dataclass
-class Counts:
-    """Exchange request: every rank's per-owner counts [W] (int32, device)."""
-    counts: torch.Tensor
-
-
-@dataclass
 class AllToAll:
-    """Exchange request: send[sum(send_counts)] grouped by destination rank,
-    receive sum(recv_counts) rows grouped by source rank."""
+    """Exchange request: send [W * capacity, ...] holds one segment of
+    `capacity` rows per destination rank; the result holds one such segment
+    per source rank."""
     send: torch.Tensor
-    send_counts: list
-    recv_counts: list
 
 
 @dataclass
 class Routing:
     """What the backward needs from a forward."""
-    src_pos: torch.Tensor     # [n] lookup index of each grouped position
-    recv_rows: torch.Tensor   # [sum recv] owner-local rows this rank serves
-    send_counts: list
-    recv_counts: list
+    src_pos: torch.Tensor     # [W * capacity] lookup of each grouped slot, -1: padding
+    recv_rows: torch.Tensor   # [W * capacity] owner-local rows this rank serves, -1: padding
 
 
 class CudaOps:
@@ -66,9 +65,8 @@ class CudaOps:
         return B.engram_hash(params, ids, cu_seqlens)
 
     @staticmethod
-    def bucket(rows, rows_per_owner, owners):
-        send, src_pos, dst_pos, counts = B.engram_owner_bucket(rows, rows_per_owner, owners)
-        return send, src_pos, dst_pos, counts
+    def bucket(rows, rows_per_owner, owners, capacity):
+        return B.engram_owner_bucket_padded(rows, rows_per_owner, owners, capacity)
 
     @staticmethod
     def gather(table, idx):
@@ -86,23 +84,25 @@ def rows_per_owner(params, owners: int) -> int:
 
 
 def forward_steps(params, shard: torch.Tensor, owners: int, ids: torch.Tensor,
-                  cu_seqlens=None, ops=CudaOps):
-    """Generator: the owner-sharded forward of one rank. Yields Counts and
-    AllToAll requests and receives their results; returns (out [T, H * dim],
-    Routing)."""
+                  cu_seqlens=None, capacity=None, ops=CudaOps):
+    """Generator: the owner-sharded forward of one rank. Yields AllToAll
+    requests and receives their results; returns (out [T, H * dim], Routing).
+    `capacity` (slots per owner and requesting rank, the same on every rank)
+    defaults to this rank's lookups, T * H."""
     rpo = rows_per_owner(params, owners)
     if shard.shape[0] != rpo:
         raise ValueError("shard must hold table_rows / owners rows")
     idx = ops.hash(params, ids, cu_seqlens)                  # [T, H] global rows
     T, H = idx.shape
-    send, src_pos, dst_pos, counts = ops.bucket(idx.reshape(-1), rpo, owners)
-    recv_counts = yield Counts(counts)
-    sc, rc = [int(v) for v in counts.tolist()], [int(v) for v in recv_counts.tolist()]
-    recv_rows = yield AllToAll(send, sc, rc)                 # rows this rank serves
-    vals = ops.gather(shard, recv_rows)                      # [sum rc, dim]
-    back = yield AllToAll(vals, rc, sc)                      # [n, dim], grouped by owner
+    cap = T * H if capacity is None else int(capacity)
+    if cap < 1:
+        raise ValueError("capacity must be at least 1")
+    send, src_pos, dst_pos, _ = ops.bucket(idx.reshape(-1), rpo, owners, cap)
+    recv_rows = yield AllToAll(send)                         # rows this rank serves
+    vals = ops.gather(shard, recv_rows)                      # [W * cap, dim]
+    back = yield AllToAll(vals)                              # grouped by owner
     out = ops.gather(back, dst_pos)                          # request order
-    return out.reshape(T, H * shard.shape[1]), Routing(src_pos, recv_rows, sc, rc)
+    return out.reshape(T, H * shard.shape[1]), Routing(src_pos, recv_rows)
 
 
 def backward_steps(params, owners: int, routing: Routing, dout: torch.Tensor, ops=CudaOps):
@@ -112,25 +112,19 @@ def backward_steps(params, owners: int, routing: Routing, dout: torch.Tensor, op
     rpo = rows_per_owner(params, owners)
     dim = params.dim
     grouped = ops.gather(dout.reshape(-1, dim), routing.src_pos)   # grouped by owner
-    owner_dout = yield AllToAll(grouped, routing.send_counts, routing.recv_counts)
+    owner_dout = yield AllToAll(grouped)
     return ops.backward(routing.recv_rows, owner_dout, rpo)
 
 
 def run_collective(gen, group=None):
-    """Runs one rank's generator over a torch.distributed process group."""
+    """Runs one rank's generator over a torch.distributed process group; every
+    exchange is an equal-split all_to_all_single."""
     import torch.distributed as dist
     try:
         req = next(gen)
         while True:
-            if isinstance(req, Counts):
-                out = torch.empty_like(req.counts)
-                dist.all_to_all_single(out, req.counts, group=group)
-            else:
-                rows = sum(req.recv_counts)
-                out = torch.empty((rows,) + tuple(req.send.shape[1:]), dtype=req.send.dtype,
-                                  device=req.send.device)
-                dist.all_to_all_single(out, req.send, output_split_sizes=req.recv_counts,
-                                       input_split_sizes=req.send_counts, group=group)
+            out = torch.empty_like(req.send)
+            dist.all_to_all_single(out, req.send, group=group)
             req = gen.send(out)
     except StopIteration as stop:
         return stop.value
@@ -138,34 +132,18 @@ def run_collective(gen, group=None):
 
 def run_lockstep(gens):
     """Runs the generators of W ranks emulated in one process: every exchange
-    is performed as copies once all ranks have reached it."""
+    is performed as device copies once all ranks have reached it."""
     W = len(gens)
     reqs = [next(g) for g in gens]
     results = [None] * W
     done = [False] * W
     while not all(done):
-        kinds = {type(r) for r in reqs}
-        if len(kinds) != 1:
-            raise RuntimeError("ranks reached different exchanges")
-        if isinstance(reqs[0], Counts):
-            table = torch.stack([r.counts for r in reqs])            # [src, dst]
-            outs = [table[:, r].contiguous() for r in range(W)]
-        else:
-            starts = []
-            for r in reqs:
-                offs, o = [], 0
-                for c in r.send_counts:
-                    offs.append(o)
-                    o += c
-                starts.append(offs)
-            outs = []
-            for dst in range(W):
-                parts = [reqs[src].send[starts[src][dst]:starts[src][dst] +
-                                        reqs[src].send_counts[dst]] for src in range(W)]
-                got = torch.cat(parts) if parts else reqs[dst].send[:0]
-                if got.shape[0] != sum(reqs[dst].recv_counts):
-                    raise RuntimeError("receive counts disagree with the senders")
-                outs.append(got)
+        shape = reqs[0].send.shape
+        if any(r.send.shape != shape for r in reqs) or shape[0] % W:
+            raise RuntimeError("ranks disagree on the exchange's capacity")
+        cap = shape[0] // W
+        outs = [torch.cat([reqs[src].send[dst * cap:(dst + 1) * cap] for src in range(W)])
+                for dst in range(W)]
         for r, g in enumerate(gens):
             try:
                 reqs[r] = g.send(outs[r])

@@ -65,6 +65,8 @@ extern "C" {
                                          (results of that call are invalid) */
 #define ENGRAM_DEVERR_COPY_TIMEOUT 8u /* a bulk copy into shared memory did not complete in
                                          time (results of that call are invalid) */
+#define ENGRAM_DEVERR_CAPACITY 16u   /* an owner received more lookups than the exchange's
+                                         capacity; the extra ones were dropped */
 /* Same type as cudaStream_t, without requiring the CUDA headers. */
 typedef struct CUstream_st *engram_stream_t;
 
@@ -125,8 +127,9 @@ ENGRAM_API int engram_hash(const engram_params_t *params, const int32_t *ids,
  *          a multiple of 16 bytes
  *   idx    device, int32 [n]
  *   out    device, [n, dim] of dtype, 16-byte aligned
- * An index outside [0, table_rows) writes a zero row and sets
- * ENGRAM_DEVERR_ROW_RANGE.
+ * A negative index marks an absent lookup (the padding of a fixed-capacity
+ * exchange): its output row is zero. An index >= table_rows also writes a zero
+ * row and sets ENGRAM_DEVERR_ROW_RANGE.
  */
 ENGRAM_API int engram_gather(const void *table, int32_t dtype, int64_t table_rows, int32_t dim,
                   const int32_t *idx, int64_t n, void *out, engram_stream_t stream);
@@ -182,7 +185,9 @@ ENGRAM_API int engram_backward_workspace_size(int64_t n, int64_t table_rows, int
  *                     accumulated in fp64 and rounded once to fp32 (no
  *                     atomics; deterministic for a given device type)
  *   *num_unique     = U, the number of distinct rows
- *   idx        device, int32 [n], 0 <= n < 2^31; out-of-range values set
+ *   idx        device, int32 [n], 0 <= n < 2^31; a negative value marks an
+ *              absent lookup (the padding of a fixed-capacity exchange), left
+ *              out of the rows and sums; values >= table_rows set
  *              ENGRAM_DEVERR_ROW_RANGE (results are then unspecified, memory
  *              accesses stay in bounds)
  *   dout       device, [n, dim] of dtype, 16-byte aligned; dim % 8 == 0 and
@@ -484,6 +489,32 @@ ENGRAM_API int engram_owner_bucket(const int32_t *rows, int64_t n, int64_t rows_
                                    size_t workspace_bytes, engram_stream_t stream);
 
 ENGRAM_API int engram_owner_bucket_workspace_size(int64_t n, int32_t owners, size_t *bytes);
+
+/*
+ * engram_owner_bucket_padded -- engram_owner_bucket into the fixed-capacity
+ * layout of the engram API page's _FixedCapacityAllToAll /
+ * _fixed_capacity_all_to_all: every owner gets a segment of `capacity` slots,
+ * agreed ahead of time, so that both exchanges are equal-split all-to-alls
+ * whose sizes never depend on the data and the step needs no host
+ * synchronisation (it can be captured in a CUDA graph).
+ *   send_rows[o * capacity + k], src_pos[o * capacity + k]
+ *              owner o's k-th lookup (as engram_owner_bucket) for
+ *              k < counts[o]; -1 in the padding slots k >= counts[o]
+ *   dst_pos[i] o * capacity + k for lookup i, or -1 if owner o already had
+ *              `capacity` lookups (the lookup is dropped and
+ *              ENGRAM_DEVERR_CAPACITY is set)
+ *   counts[o]  min(lookups of owner o, capacity)
+ * The lookup (engram_gather) and the backward (engram_backward) treat the -1
+ * entries as absent: zero rows, left out of the gradient. capacity = n never
+ * drops a lookup. send_rows and src_pos hold owners * capacity int32 each
+ * (owners * capacity < 2^31); workspace as engram_owner_bucket.
+ */
+ENGRAM_API int engram_owner_bucket_padded(const int32_t *rows, int64_t n,
+                                          int64_t rows_per_owner, int32_t owners,
+                                          int64_t capacity, int32_t *send_rows,
+                                          int32_t *src_pos, int32_t *dst_pos, int32_t *counts,
+                                          void *workspace, size_t workspace_bytes,
+                                          engram_stream_t stream);
 
 /*
  * engram_get_device_error -- copy the current device's error word

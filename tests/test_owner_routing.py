@@ -4,11 +4,12 @@ The routing generators run with host stand-ins for the device steps (defined
 here: the oracle's hash, gather and backward, and a stable argsort for the
 grouping), first as ranks emulated in one process, then as two gloo ranks with
 real all-to-alls. What they pin is the exchange logic of the page's
-Qwen3_8_FlashNextOwnerShardedEmbedding: counts, split sizes, the grouping by
-owner, putting values back in request order and sending gradients back to
-the owner, which alone accumulates its rows. Every rank's output must equal
-the oracle's lookup in the whole table, and every owner's row gradients the
-oracle's backward over all ranks' lookups restricted to its rows.
+Qwen3_8_FlashNextOwnerShardedEmbedding with its fixed-capacity exchange: the
+grouping by owner into padded segments, putting values back in request order
+and sending gradients back to the owner, which alone accumulates its rows.
+Every rank's output must equal the oracle's lookup in the whole table, and
+every owner's row gradients the oracle's backward over all ranks' lookups
+restricted to its rows -- at the default capacity and at tight ones.
 """
 
 import os
@@ -32,21 +33,32 @@ class HostOps:
         idx = oracle.hash_ids(ids.numpy(), None if cu is None else cu.numpy(), self.cfg)
         return torch.from_numpy(idx.astype(np.int32))
 
-    def bucket(self, rows, rpo, owners):
+    def bucket(self, rows, rpo, owners, cap):
         r = rows.numpy().astype(np.int64)
         o = r // rpo
         order = np.argsort(o, kind="stable")
-        dst = np.empty_like(order)
-        dst[order] = np.arange(len(order))
-        return (torch.from_numpy((r[order] - o[order] * rpo).astype(np.int32)),
-                torch.from_numpy(order.astype(np.int32)), torch.from_numpy(dst.astype(np.int32)),
-                torch.from_numpy(np.bincount(o, minlength=owners).astype(np.int32)))
+        counts = np.bincount(o, minlength=owners)
+        send = np.full(owners * cap, -1, np.int32)
+        src = np.full(owners * cap, -1, np.int32)
+        dst = np.full(len(r), -1, np.int32)
+        start = np.concatenate([[0], np.cumsum(counts)])
+        for p, i in enumerate(order):
+            k = p - start[o[i]]
+            if k < cap:
+                slot = o[i] * cap + k
+                send[slot], src[slot], dst[i] = r[i] - o[i] * rpo, i, slot
+        return (torch.from_numpy(send), torch.from_numpy(src), torch.from_numpy(dst),
+                torch.from_numpy(np.minimum(counts, cap).astype(np.int32)))
 
     def gather(self, table, idx):
-        return table[idx.long()]
+        i = idx.long()
+        out = table[i.clamp(min=0)]
+        out[i < 0] = 0
+        return out
 
     def backward(self, idx, dout, table_rows):
-        u, g = oracle.backward(idx.numpy(), dout.numpy(), oracle.F32)
+        keep = idx.numpy() >= 0
+        u, g = oracle.backward(idx.numpy()[keep], dout.numpy()[keep], oracle.F32)
         return torch.from_numpy(u), torch.from_numpy(g), torch.tensor([len(u)], dtype=torch.int32)
 
 
@@ -83,8 +95,8 @@ def run_rank(E_owner, params, cfg, table, W, r, ids, cu, dout, runner):
     return out, u, g, nu
 
 
-@pytest.mark.parametrize("W", [1, 2, 4])
-def test_lockstep_emulated_ranks(W):
+@pytest.mark.parametrize("W,cap", [(1, None), (2, None), (4, None), (2, 1100), (4, 600)])
+def test_lockstep_emulated_ranks(W, cap):
     from hashed_gram_embedding_raw_b200 import make_params, owner
     cfg = head_params("tiny")
     params = make_params(cfg)
@@ -97,8 +109,8 @@ def test_lockstep_emulated_ranks(W):
     rpo = cfg["table_rows"] // W
     ops = HostOps(cfg)
     shards = [torch.from_numpy(table[r * rpo:(r + 1) * rpo].copy()) for r in range(W)]
-    fwd = owner.run_lockstep([owner.forward_steps(params, shards[r], W, *parts[r], ops=ops)
-                              for r in range(W)])
+    fwd = owner.run_lockstep([owner.forward_steps(params, shards[r], W, *parts[r],
+                                                  capacity=cap, ops=ops) for r in range(W)])
     bwd = owner.run_lockstep([owner.backward_steps(params, W, fwd[r][1], douts[r], ops=ops)
                               for r in range(W)])
     outs, owners = expected(cfg, table, parts, douts, W)
@@ -107,6 +119,34 @@ def test_lockstep_emulated_ranks(W):
         u, g, nu = bwd[r]
         assert int(nu[0]) == len(owners[r][0])
         assert np.array_equal(u.numpy(), owners[r][0]) and np.array_equal(g.numpy(), owners[r][1])
+
+
+def test_lockstep_capacity_overflow_drops_lookups():
+    """A capacity below some owner's lookups drops the excess: their rows come
+    back zero and their gradients are left out, nothing else changes."""
+    from hashed_gram_embedding_raw_b200 import make_params, owner
+    cfg = head_params("tiny")
+    params = make_params(cfg)
+    table = host_table("tiny")
+    ids, _ = token_stream("tiny")
+    W, cap = 2, 300
+    parts = split_stream(ids, W)
+    ops = HostOps(cfg)
+    rpo = cfg["table_rows"] // W
+    shards = [torch.from_numpy(table[r * rpo:(r + 1) * rpo].copy()) for r in range(W)]
+    fwd = owner.run_lockstep([owner.forward_steps(params, shards[r], W, *parts[r],
+                                                  capacity=cap, ops=ops) for r in range(W)])
+    for r in range(W):
+        idx = oracle.hash_ids(parts[r][0].numpy(), parts[r][1].numpy(), cfg).reshape(-1)
+        got = fwd[r][0].numpy().reshape(len(idx), -1)
+        # lookups kept: each owner's first `cap` lookups in request order
+        o = idx // rpo
+        kept = np.zeros(len(idx), bool)
+        for w in range(W):
+            kept[np.nonzero(o == w)[0][:cap]] = True
+        assert (~kept).any()
+        want = oracle.gather(table, idx)
+        assert np.array_equal(got[kept], want[kept]) and not got[~kept].any()
 
 
 def test_rows_must_divide_among_owners():
