@@ -18,7 +18,6 @@
 #include "engram.h"
 
 #include "backward.cuh"
-#include "cluster_sort.cuh"
 #include "common.cuh"
 #include "hash_gather.cuh"
 #include "ple_conv.cuh"
@@ -462,93 +461,13 @@ uint64_t cross_wait_ns()
     return v;
 }
 
-// The on-chip sort (one cluster per segment, cluster_sort.cuh) where the
-// segments fit a cluster and the device runs such clusters; *launched is
-// false otherwise (nothing ran).
-int launch_sort_cluster(const int32_t *idx, const SortShape &sh, const BwdPlan &P, char *ws,
-                        cudaStream_t stream, bool *launched)
-{
-    using namespace bwd;
-    *launched = false;
-    if (sh.L < 1 || sh.L > kClusterMaxSegment)
-        return ENGRAM_OK;
-    SortArgs args;
-    ENGRAM_TRY(sort_args(idx, sh, kSortItemsMax, P, ws, &args));
-    const size_t smem = sizeof(ClusterSmem);
-    static std::once_flag once;
-    static cudaError_t attr_rc = cudaSuccess;
-    std::call_once(once, [&] {
-        attr_rc = cudaFuncSetAttribute(cluster_sort_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    });
-    if (attr_rc != cudaSuccess) {
-        (void)cudaGetLastError();
-        return ENGRAM_OK;
-    }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(sh.S * kClusterCtas));
-    cfg.blockDim = dim3(kClusterThreads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = kClusterCtas;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    // whether the device runs such clusters at all: asked once per device (a
-    // query inside a stream capture could end the capture)
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128)
-        return ENGRAM_ECUDA;
-    static std::atomic<int> cluster_ok[128];
-    int ok = cluster_ok[dev].load(std::memory_order_relaxed);
-    if (ok == 0) {
-        int clusters = 0;
-        ok = cudaOccupancyMaxActiveClusters(&clusters, cluster_sort_kernel, &cfg) == cudaSuccess &&
-                     clusters >= 1
-                 ? 1
-                 : -1;
-        (void)cudaGetLastError();
-        cluster_ok[dev].store(ok, std::memory_order_relaxed);
-    }
-    if (ok < 0)
-        return ENGRAM_OK;
-    if (cudaLaunchKernelEx(&cfg, cluster_sort_kernel, args) != cudaSuccess) {
-        (void)cudaGetLastError();
-        return ENGRAM_OK;
-    }
-    g_launches.fetch_add(1, std::memory_order_relaxed);
-    *launched = true;
-    return ENGRAM_OK;
-}
-
-// ENGRAM_SORT_NO_CLUSTER=1 in the environment (read once per process) keeps
-// the sort off the on-chip cluster form, so that the grid-wide form can be
-// checked on shapes the cluster form would take.
-bool sort_no_cluster()
-{
-    static const bool v = [] {
-        const char *e = std::getenv("ENGRAM_SORT_NO_CLUSTER");
-        return e != nullptr && e[0] == '1';
-    }();
-    return v;
-}
-
-// Sorts the pairs of `sh` into buffer a of the workspace: on chip where a
-// segment fits one cluster, else the grid-wide sort in one cooperative
-// launch, else two launches per pass.
+// Sorts the pairs of `sh` into buffer a of the workspace: the grid-wide sort
+// in one cooperative launch, else two launches per pass.
 int launch_sort(const int32_t *idx, const SortShape &sh, const BwdPlan &P, char *ws,
                 cudaStream_t stream)
 {
     using namespace bwd;
     bool launched = false;
-    if (!sort_separate_launches() && !sort_no_cluster()) {
-        ENGRAM_TRY(launch_sort_cluster(idx, sh, P, ws, stream, &launched));
-        if (launched)
-            return ENGRAM_OK;
-    }
     if (cudaMemsetAsync(ws + P.ctl, 0, P.ctl_bytes, stream) != cudaSuccess)
         return ENGRAM_ECUDA;
     int items = 0;
