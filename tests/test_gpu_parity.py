@@ -445,3 +445,18 @@ def test_backward_reduce_repeated_after_one_sort(E, pattern):
         np.testing.assert_array_equal(u[:U].cpu().numpy(), want_u)
         assert_grads_close(g[:U].cpu().numpy(), want_g)
     assert E.engram_get_device_error() == 0
+
+
+@pytest.mark.parametrize("vocab", [3, 248_320])
+def test_backward_heads_page_table_hot_and_spread(E, vocab):
+    """The sort by head on the page's table and batch shape: token IDs from 3
+    values make a few rows take nearly all lookups, so some bucket of the
+    two-step sort overflows and the launch falls back to its LSD passes; IDs
+    over the whole vocabulary spread evenly and take the two-step form. Both
+    against the oracle."""
+    cfg = head_params("full")
+    ids, cu = random_stream(vocab, 65_536, vocab, cfg["eos_id"], 1 / 512, nseq=16)
+    idx = oracle.hash_ids(ids, cu, cfg)
+    dout = torch.randn(idx.size, 160, generator=torch.Generator().manual_seed(vocab)).to(
+        torch.bfloat16)
+    check_backward_heads(E, cfg, idx, dout, oracle.BF16)

@@ -1,8 +1,10 @@
-"""The backward sort's two forms on the same inputs, each in a child
-process, compared bit for bit: the grid-wide sort in one cooperative launch
-(the default) and the separate-launch form -- what a device without
-cooperative launch runs: two launches per pass on 2,048-pair tiles -- forced
-with ENGRAM_SORT_SEPARATE_LAUNCHES=1. A stable sort has one
+"""The backward sort's forms on the same inputs, each in a child process,
+compared bit for bit: the one cooperative launch (the default; a sort by head
+on evenly spread keys takes the two-step form there, buckets of the top bits
+then in-block sorts), the same launch held to its LSD passes
+(ENGRAM_SORT_ONE_STEP=1), and the separate-launch form -- what a device
+without cooperative launch runs: two launches per pass on 2,048-pair tiles --
+forced with ENGRAM_SORT_SEPARATE_LAUNCHES=1. A stable sort has one
 result, so the distinct rows and their fp32 sums must be identical bit for
 bit. The sizes cover one tile, a ragged single tile, many resident tiles and
 more tiles than resident blocks; half the lookups hit a few hot rows. The
@@ -43,29 +45,31 @@ from workloads import head_params, random_stream
 import oracle
 cfg = dict(head_params("full"), dim=16)
 p = E.make_params(cfg)
-for T in (1, 63, 15_625, 65_536, 65_537, 131_072):
-    ids, cu = random_stream(T, T, 2000, cfg["eos_id"], 0.01, nseq=1 + T // 4096)
+for T, vocab in ((1, 2000), (63, 2000), (15_625, 2000), (65_536, 2000), (65_536, 248_320),
+                 (40_000, 248_320), (65_537, 2000), (131_072, 2000)):
+    ids, cu = random_stream(T, T, vocab, cfg["eos_id"], 0.01, nseq=1 + T // 4096)
     idx = oracle.hash_ids(ids, cu, cfg).astype(np.int32)
     dout = torch.randn(idx.size, 16, generator=torch.Generator().manual_seed(T % 997))
     u, g, nu = E.engram_backward_heads(p, torch.from_numpy(idx).cuda(), dout.cuda())
     U = int(nu.item())
     assert E.engram_get_device_error() == 0
-    out["hu%d" % T] = u[:U].cpu().numpy()
-    out["hg%d" % T] = g[:U].cpu().numpy()
+    out["hu%d_%d" % (T, vocab)] = u[:U].cpu().numpy()
+    out["hg%d_%d" % (T, vocab)] = g[:U].cpu().numpy()
 np.savez(sys.argv[2], **out)
 """
 
 
 def run_child(tmp_path, form: str):
     path = tmp_path / (form + ".npz")
-    env = dict(os.environ, ENGRAM_SORT_SEPARATE_LAUNCHES="1" if form == "separate" else "0")
+    env = dict(os.environ, ENGRAM_SORT_SEPARATE_LAUNCHES="1" if form == "separate" else "0",
+               ENGRAM_SORT_ONE_STEP="1" if form == "one_step" else "0")
     subprocess.run([sys.executable, "-c", CHILD, ROOT, str(path)], env=env, check=True,
                    timeout=600)
     return np.load(path)
 
 
 def test_sort_forms_agree_bit_for_bit(tmp_path):
-    forms = {f: run_child(tmp_path, f) for f in ("default", "separate")}
+    forms = {f: run_child(tmp_path, f) for f in ("default", "one_step", "separate")}
     base = forms["default"]
     for name, got in forms.items():
         assert sorted(got.files) == sorted(base.files), name
