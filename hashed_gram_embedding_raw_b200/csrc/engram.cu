@@ -389,41 +389,6 @@ int sort_args(const int32_t *idx, const SortShape &sh, int items, const BwdPlan 
     return ENGRAM_OK;
 }
 
-bool two_step_sort_off();
-
-// The two-step sort's buckets (radix_sort.cuh), when a sort can use them:
-// segments without absent lookups, at most 3 LSD passes (the fourth pass's
-// group sums hold the buckets'), and buckets whose expected size -- keys
-// spread evenly over a segment's rows -- is at most half a tile, so that on
-// such traffic none overflows; then the largest bucket shift with at most two
-// 9-bit local passes and at most 256 buckets per segment.
-void bucket_plan(const SortShape &sh, int items, bwd::SortArgs *a)
-{
-    using namespace bwd;
-    a->bkt_shift = 0;
-    if (two_step_sort_off() || sh.pad || a->passes > kMaxPasses - 1 || a->passes < 2 || sh.L < 1)
-        return;
-    uint64_t smin = UINT64_MAX, smax = 0;
-    for (int s = 0; s < sh.S; ++s) {
-        smin = std::min<uint64_t>(smin, sh.size[s]);
-        smax = std::max<uint64_t>(smax, sh.size[s]);
-    }
-    const double half_tile = 0.5 * kSortThreads * items;
-    int bs = 0;
-    while (bs < 18 && (double)sh.L * (double)(1ull << (bs + 1)) / (double)smin <= half_tile)
-        ++bs;
-    if (bs == 0)
-        return;
-    const uint64_t nb = (smax + (1ull << bs) - 1) >> bs;
-    if (nb > 256)
-        return;
-    a->bkt_shift = bs;
-    a->bkt_nb = (int)nb;
-    a->bkt_bits = std::max(1, bit_width(nb - 1));
-    a->lbits[0] = std::min(9, bs);
-    a->lbits[1] = bs - a->lbits[0];
-}
-
 // The one-launch sort at I pairs per thread; *launched is false where the
 // device or the launch refuses a cooperative grid (nothing ran).
 template <int I>
@@ -442,8 +407,6 @@ int launch_sort_coop(const int32_t *idx, const SortShape &sh, const BwdPlan &P, 
     int64_t res = 0;
     ENGRAM_TRY(resident_warps(radix_sort_coop<I>, kSortThreads, 0, &res));
     const int grid = (int)std::min<int64_t>(args.ntiles, res / (kSortThreads / 32));
-    if (args.ntiles <= grid)
-        bucket_plan(sh, I, &args);
     void *params[] = {&args};
     if (cudaLaunchCooperativeKernel((const void *)radix_sort_coop<I>, dim3(grid),
                                     dim3(kSortThreads), params, 0, stream) != cudaSuccess) {
@@ -481,18 +444,6 @@ uint64_t env_u64(const char *name, uint64_t fallback)
     char *end = nullptr;
     const unsigned long long v = std::strtoull(e, &end, 10);
     return (end != nullptr && *end == '\0') ? (uint64_t)v : fallback;
-}
-
-// ENGRAM_SORT_ONE_STEP=1 in the environment (read once per process) keeps the
-// sort on its LSD passes, so that the two-step form can be checked against
-// them on the same device.
-bool two_step_sort_off()
-{
-    static const bool v = [] {
-        const char *e = std::getenv("ENGRAM_SORT_ONE_STEP");
-        return e != nullptr && e[0] == '1';
-    }();
-    return v;
 }
 
 uint32_t barrier_spin_limit()

@@ -81,11 +81,6 @@ struct SortArgs {
     int32_t off[kMaxSegments]; // segment s holds keys off[s] .. off[s] + size[s] - 1
     uint32_t size[kMaxSegments];
     bool pad;                  // a negative index is an absent lookup: key size[s], not an error
-    // two-step sort (0: off): bucket b = min(key >> bkt_shift, bkt_nb - 1) of
-    // each segment in one grid pass, then every bucket sorted by its low
-    // bkt_shift bits inside one block (local passes of lbits[0], lbits[1])
-    int bkt_shift, bkt_bits, bkt_nb;
-    int lbits[2];
 };
 
 __device__ __forceinline__ uint32_t item_key(uint64_t it) { return (uint32_t)(it >> 32); }
@@ -94,7 +89,6 @@ __device__ __forceinline__ uint32_t item_key(uint64_t it) { return (uint32_t)(it
 struct PassInfo {
     int shift, bits, ndig, dpt; // dpt: digits per thread (1, or 2 above 8 bits)
     bool first, last;
-    uint32_t dmax;              // digits above dmax count as dmax (the bucket pass)
 };
 
 __device__ __forceinline__ PassInfo pass_info(const SortArgs &a, int p)
@@ -108,14 +102,12 @@ __device__ __forceinline__ PassInfo pass_info(const SortArgs &a, int p)
     q.dpt = q.ndig > kSortThreads ? 2 : 1;
     q.first = p == 0;
     q.last = p == a.passes - 1;
-    q.dmax = 0xffffffffu;
     return q;
 }
 
 __device__ __forceinline__ uint32_t digit_of(uint64_t x, const PassInfo &P)
 {
-    const uint32_t d = item_key(x) >> P.shift;
-    return P.dmax != 0xffffffffu ? min(d, P.dmax) : d & (uint32_t)(P.ndig - 1);
+    return (item_key(x) >> P.shift) & (uint32_t)(P.ndig - 1);
 }
 
 // Pass p writes `out_buffer(a, p)` and reads the previous pass's output; the
@@ -535,136 +527,6 @@ __device__ __forceinline__ void place_ordered_tile(SortSmem<ITEMS> &sm, const So
     __syncthreads(); // shared memory free for the next tile
 }
 
-// ------------------------------------------------- two-step sort by head
-//
-// When each head's keys spread evenly over its slice (uniform traffic), one
-// grid pass can cut every segment into buckets of the key's top bits small
-// enough for one block, and each block then sorts whole buckets by their low
-// bits in shared memory, with no grid barrier between those passes: one
-// grid-wide pass in place of two or three. The grid pass is the LSD pass of
-// the bucket digit (stable, so a bucket keeps its lookups in ascending j);
-// the in-block passes are stable too, so equal rows keep ascending j. Before
-// committing, every block checks that no bucket exceeds a tile (the largest
-// bucket of a Zipf workload's hot rows can); if one does, the launch sorts by
-// the LSD passes instead.
-
-// Ranks `count` items held in registers (item i = wbase + r * 32 + lane) by
-// P's digit: rank[r] and sm.whist as rank_tile leaves them.
-template <int ITEMS>
-__device__ __forceinline__ void rank_loaded(SortSmem<ITEMS> &sm, const PassInfo &P, int count,
-                                            const uint64_t (&it)[ITEMS],
-                                            uint32_t (&rank)[ITEMS])
-{
-    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    for (int k = tid; k < (kSortWarps << P.bits); k += kSortThreads)
-        sm.whist[k >> P.bits][k & (P.ndig - 1)] = 0;
-    __syncthreads();
-    const int wbase = wid * (32 * ITEMS);
-    const uint32_t lt = lanemask_lt();
-#pragma unroll
-    for (int r = 0; r < ITEMS; ++r) {
-        const bool valid = wbase + r * 32 + lane < count;
-        const uint32_t dg = digit_of(it[r], P);
-        const uint32_t peers = digit_peers(dg, valid, P.bits);
-        const int leader = valid ? __ffs(peers) - 1 : lane;
-        uint32_t cnt = 0;
-        if (valid && lane == leader) {
-            cnt = sm.whist[wid][dg];
-            sm.whist[wid][dg] = cnt + __popc(peers);
-        }
-        cnt = __shfl_sync(kFull, cnt, leader);
-        rank[r] = cnt + __popc(peers & lt);
-        __syncwarp();
-    }
-    __syncthreads();
-}
-
-// Whether some bucket (its count summed over the segment's groups) holds
-// more than a tile; the same answer in every block.
-template <int ITEMS>
-__device__ __forceinline__ bool bucket_overflows(const SortArgs &a, const uint32_t *gc)
-{
-    uint32_t mx = 0;
-    for (int k = threadIdx.x; k < a.S * a.bkt_nb; k += kSortThreads) {
-        const int seg = k / a.bkt_nb, b = k - seg * a.bkt_nb;
-        uint32_t t = 0;
-        for (int g = 0; g < a.gps; ++g)
-            t += __ldcg(gc + (size_t)(seg * a.gps + g) * kRadixMax + b);
-        mx = max(mx, t);
-    }
-    return __syncthreads_or(mx > (uint32_t)SortSmem<ITEMS>::kTile) != 0;
-}
-
-// Sorts bucket b of segment seg (left in a.b by the bucket pass, bucket-major
-// inside the segment) by the low bkt_shift bits of its keys and writes it to
-// its final positions in a.a with the segment's first row added back.
-template <int ITEMS>
-__device__ __forceinline__ void sort_bucket(SortSmem<ITEMS> &sm, const SortArgs &a,
-                                            const uint32_t *gc, int seg, int b)
-{
-    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    // the bucket's start in the segment and its size
-    uint32_t tot = 0;
-    if (tid < a.bkt_nb)
-        for (int g = 0; g < a.gps; ++g)
-            tot += __ldcg(gc + (size_t)(seg * a.gps + g) * kRadixMax + tid);
-    const uint32_t excl = block_exclusive_scan(tot, sm.warp, nullptr);
-    if (tid == b) {
-        sm.cnt[0] = excl;
-        sm.cnt[1] = tot;
-    }
-    __syncthreads();
-    const uint32_t start = sm.cnt[0], size = sm.cnt[1];
-    __syncthreads();
-    if (size == 0)
-        return;
-    const int64_t base = (int64_t)seg * a.L + start;
-    const int wbase = wid * (32 * ITEMS);
-    uint64_t it[ITEMS];
-#pragma unroll
-    for (int r = 0; r < ITEMS; ++r) {
-        const int i = wbase + r * 32 + lane;
-        it[r] = i < (int)size ? __ldcg(a.b + base + i) : 0ull;
-    }
-    int shift = 0;
-#pragma unroll 1
-    for (int q = 0; q < 2; ++q) {
-        if (a.lbits[q] == 0)
-            continue;
-        PassInfo P;
-        P.shift = shift;
-        P.bits = a.lbits[q];
-        P.ndig = 1 << P.bits;
-        P.dpt = P.ndig > kSortThreads ? 2 : 1;
-        P.first = P.last = false;
-        P.dmax = 0xffffffffu;
-        shift += P.bits;
-        if (q == 1) { // the first local pass left the bucket in sm.items
-#pragma unroll
-            for (int r = 0; r < ITEMS; ++r) {
-                const int i = wbase + r * 32 + lane;
-                it[r] = i < (int)size ? sm.items[i] : 0ull;
-            }
-        }
-        uint32_t rank[ITEMS], tcount[2];
-        rank_loaded(sm, P, (int)size, it, rank);
-        tile_digit_count(sm, P, tcount);
-        local_starts(sm, P, tcount);
-#pragma unroll
-        for (int r = 0; r < ITEMS; ++r) {
-            if (wbase + r * 32 + lane < (int)size) {
-                const uint32_t dg = digit_of(it[r], P);
-                sm.items[sm.tstart[dg] + sm.whist[wid][dg] + rank[r]] = it[r];
-            }
-        }
-        __syncthreads();
-    }
-    const unsigned long long offhi = (unsigned long long)(uint32_t)a.off[seg] << 32;
-    for (int i = tid; i < (int)size; i += kSortThreads)
-        a.a[base + i] = sm.items[i] + offhi;
-    __syncthreads(); // shared memory free for the next bucket
-}
-
 // ----------------------------------------------- one launch per phase
 
 template <int ITEMS>
@@ -743,36 +605,6 @@ template <int ITEMS> __global__ void __launch_bounds__(kSortThreads, 4) radix_so
         const int tile = blockIdx.x;
         const bool has = tile < a.ntiles;
         const TileGeom g = tile_geom(a, has ? tile : 0, TILE);
-        if (a.bkt_shift > 0) {
-            // the two-step sort: buckets of the top bits into a.b, then each
-            // bucket sorted in one block (group sums in the spare pass slot)
-            PassInfo P;
-            P.shift = a.bkt_shift;
-            P.bits = a.bkt_bits;
-            P.ndig = 1 << P.bits;
-            P.dpt = P.ndig > kSortThreads ? 2 : 1;
-            P.first = true;
-            P.last = false;
-            P.dmax = (uint32_t)a.bkt_nb - 1u;
-            const uint32_t *gcb = a.group_cnt + (size_t)(kMaxPasses - 1) * a.ngroups * kRadixMax;
-            uint32_t tcount[2] = {0u, 0u};
-            if (has)
-                stage_tile<true>(sm, a, nullptr, P, tile, g, true,
-                                 const_cast<uint32_t *>(gcb), tcount);
-            if (!grid_barrier(a.barrier, gen, sm.flag, a.spin_limit))
-                return;
-            if (!bucket_overflows<ITEMS>(a, gcb)) {
-                if (has)
-                    place_staged_tile<true>(sm, a, P, a.b, g, tcount, gcb);
-                if (!grid_barrier(a.barrier, gen, sm.flag, a.spin_limit))
-                    return;
-                for (int bk = blockIdx.x; bk < a.S * a.bkt_nb; bk += gridDim.x)
-                    sort_bucket(sm, a, gcb, bk / a.bkt_nb, bk % a.bkt_nb);
-                return;
-            }
-            // some bucket is larger than a tile: the LSD passes, from the
-            // indices again
-        }
         for (int pass = 0; pass < a.passes; ++pass) {
             const PassInfo P = pass_info(a, pass);
             const void *src = P.first ? nullptr : out_buffer(a, pass - 1);

@@ -449,11 +449,9 @@ def test_backward_reduce_repeated_after_one_sort(E, pattern):
 
 @pytest.mark.parametrize("vocab", [3, 248_320])
 def test_backward_heads_page_table_hot_and_spread(E, vocab):
-    """The sort by head on the page's table and batch shape: token IDs from 3
-    values make a few rows take nearly all lookups, so some bucket of the
-    two-step sort overflows and the launch falls back to its LSD passes; IDs
-    over the whole vocabulary spread evenly and take the two-step form. Both
-    against the oracle."""
+    """The sort by head on the page's table and batch shape against the
+    oracle: token IDs from 3 values make a few rows take nearly all lookups;
+    IDs over the whole vocabulary spread them evenly over each head's slice."""
     cfg = head_params("full")
     ids, cu = random_stream(vocab, 65_536, vocab, cfg["eos_id"], 1 / 512, nseq=16)
     idx = oracle.hash_ids(ids, cu, cfg)

@@ -1,10 +1,8 @@
-"""The backward sort's forms on the same inputs, each in a child process,
-compared bit for bit: the one cooperative launch (the default; a sort by head
-on evenly spread keys takes the two-step form there, buckets of the top bits
-then in-block sorts), the same launch held to its LSD passes
-(ENGRAM_SORT_ONE_STEP=1), and the separate-launch form -- what a device
-without cooperative launch runs: two launches per pass on 2,048-pair tiles --
-forced with ENGRAM_SORT_SEPARATE_LAUNCHES=1. A stable sort has one
+"""The backward sort's two forms on the same inputs, each in a child
+process, compared bit for bit: the grid-wide sort in one cooperative launch
+(the default) and the separate-launch form -- what a device without
+cooperative launch runs: two launches per pass on 2,048-pair tiles -- forced
+with ENGRAM_SORT_SEPARATE_LAUNCHES=1. A stable sort has one
 result, so the distinct rows and their fp32 sums must be identical bit for
 bit. The sizes cover one tile, a ragged single tile, many resident tiles and
 more tiles than resident blocks; half the lookups hit a few hot rows. The
@@ -61,15 +59,14 @@ np.savez(sys.argv[2], **out)
 
 def run_child(tmp_path, form: str):
     path = tmp_path / (form + ".npz")
-    env = dict(os.environ, ENGRAM_SORT_SEPARATE_LAUNCHES="1" if form == "separate" else "0",
-               ENGRAM_SORT_ONE_STEP="1" if form == "one_step" else "0")
+    env = dict(os.environ, ENGRAM_SORT_SEPARATE_LAUNCHES="1" if form == "separate" else "0")
     subprocess.run([sys.executable, "-c", CHILD, ROOT, str(path)], env=env, check=True,
                    timeout=600)
     return np.load(path)
 
 
 def test_sort_forms_agree_bit_for_bit(tmp_path):
-    forms = {f: run_child(tmp_path, f) for f in ("default", "one_step", "separate")}
+    forms = {f: run_child(tmp_path, f) for f in ("default", "separate")}
     base = forms["default"]
     for name, got in forms.items():
         assert sorted(got.files) == sorted(base.files), name
