@@ -1242,8 +1242,11 @@ def run_owner(args):
     cu = torch.from_numpy(cu_np.copy()).to(device)
     dout = host_dout(name, T * H, D, w.dtype, seed_offset=rank).to(device)
 
+    capacity = owner.agree_capacity(params, world, ids, cu)
+
     def step():
-        out, routing = owner.run_collective(owner.forward_steps(params, shard, world, ids, cu))
+        out, routing = owner.run_collective(
+            owner.forward_steps(params, shard, world, ids, cu, capacity=capacity))
         return owner.run_collective(owner.backward_steps(params, world, routing, dout))
 
     for _ in range(args.warmup):
@@ -1278,14 +1281,16 @@ def run_owner(args):
         "data": "synthetic",
         "config": {"workload": name + "_owner", "tokens_per_step_per_gpu": T,
                    "owners": world, "rows_per_owner": rpo,
-                   "exchange": "NCCL all_to_all_single, uneven splits",
-                   "all_to_all_bytes_per_step_per_gpu": T * H * (4 + 2 * D * esize),
+                   "exchange": "NCCL all_to_all_single, equal splits of a fixed capacity",
+                   "capacity": capacity,
+                   "all_to_all_bytes_per_step_per_gpu": world * capacity * (4 + 2 * D * esize),
                    "l2": "inputs larger than L2"},
         "gpu_launches": launches,
         "clocks": clk.summary(),
         "cpu_baseline": None,
-        "note": ("eager launches: the grouping counts cross to the host before each "
-                 "exchange, so the step cannot be one CUDA graph"),
+        "note": ("eager launches; the capacity (the largest owner segment of this batch "
+                 "over all ranks, rounded up to 256) is agreed in a setup pass, so no count "
+                 "crosses to the host inside a step"),
     }
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -116,6 +116,26 @@ def backward_steps(params, owners: int, routing: Routing, dout: torch.Tensor, op
     return ops.backward(routing.recv_rows, owner_dout, rpo)
 
 
+def agree_capacity(params, owners: int, ids: torch.Tensor, cu_seqlens=None, group=None,
+                   multiple: int = 256, ops=CudaOps) -> int:
+    """A capacity for batches like this one, agreed once ahead of the steps:
+    the largest number of lookups any rank sends any owner (the page's global
+    maximum peer-segment row count), rounded up to `multiple`. This setup
+    call reads the counts on the host and, in a process group, takes their
+    maximum over the ranks with an all-reduce; the steps that then use the
+    capacity do neither."""
+    rpo = rows_per_owner(params, owners)
+    idx = ops.hash(params, ids, cu_seqlens).reshape(-1)
+    n = idx.numel()
+    _, _, _, counts = ops.bucket(idx, rpo, owners, max(n, 1))
+    top = counts.max().reshape(1).to(torch.int64)
+    if group is not None or owners > 1:
+        import torch.distributed as dist
+        dist.all_reduce(top, op=dist.ReduceOp.MAX, group=group)
+    cap = int(top.item())
+    return max(multiple, -(-cap // multiple) * multiple)
+
+
 def run_collective(gen, group=None):
     """Runs one rank's generator over a torch.distributed process group; every
     exchange is an equal-split all_to_all_single."""

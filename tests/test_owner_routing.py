@@ -86,11 +86,12 @@ def expected(cfg, table, parts, douts, W):
     return outs, owners
 
 
-def run_rank(E_owner, params, cfg, table, W, r, ids, cu, dout, runner):
+def run_rank(E_owner, params, cfg, table, W, r, ids, cu, dout, runner, capacity=None):
     rpo = cfg["table_rows"] // W
     shard = torch.from_numpy(table[r * rpo:(r + 1) * rpo].copy())
     ops = HostOps(cfg)
-    out, routing = runner(E_owner.forward_steps(params, shard, W, ids, cu, ops=ops))
+    out, routing = runner(E_owner.forward_steps(params, shard, W, ids, cu, capacity=capacity,
+                                                ops=ops))
     u, g, nu = runner(E_owner.backward_steps(params, W, routing, dout, ops=ops))
     return out, u, g, nu
 
@@ -174,10 +175,18 @@ def _gloo_rank(rank, world, port, result_dir):
         H, D = params.heads, cfg["dim"]
         douts = [host_dout("tiny", len(p[0]) * H, D, "f32", seed_offset=r)
                  for r, p in enumerate(parts)]
+        # the capacity agreed over both ranks: the largest owner segment of
+        # either rank's lookups, rounded up to 16
+        cap = owner.agree_capacity(params, world, *parts[rank], multiple=16, ops=HostOps(cfg))
+        rpo = cfg["table_rows"] // world
+        top = max(np.bincount(oracle.hash_ids(i.numpy(), c.numpy(), cfg).reshape(-1) // rpo,
+                              minlength=world).max() for i, c in parts)
         out, u, g, nu = run_rank(owner, params, cfg, table, world, rank, *parts[rank],
-                                 douts[rank], lambda gen: owner.run_collective(gen))
+                                 douts[rank], lambda gen: owner.run_collective(gen),
+                                 capacity=cap)
         outs, owners = expected(cfg, table, parts, douts, world)
-        ok = (np.array_equal(out.numpy(), outs[rank]) and int(nu[0]) == len(owners[rank][0])
+        ok = (cap == -(-top // 16) * 16 and cap < len(parts[rank][0]) * params.heads
+              and np.array_equal(out.numpy(), outs[rank]) and int(nu[0]) == len(owners[rank][0])
               and np.array_equal(u.numpy(), owners[rank][0])
               and np.array_equal(g.numpy(), owners[rank][1]))
         with open(os.path.join(result_dir, f"rank{rank}"), "w") as f:
@@ -187,6 +196,8 @@ def _gloo_rank(rank, world, port, result_dir):
 
 
 def test_two_gloo_ranks(tmp_path):
+    """Two gloo ranks with real all-to-alls at the capacity they agree on
+    (agree_capacity's all-reduce), below the default, with nothing dropped."""
     import torch.multiprocessing as mp
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))
