@@ -1192,12 +1192,18 @@ struct ConvBwdPlan {
     ple::ConvBwdArgs a;
     size_t smem = 0, ws = 0;
     int grid = 0, threads = 0, npart = 0;
+    int32_t dtype = 0, grad_dtype = 0;
 };
 
-// Checks the shape (host only) and sizes the launch: G / 8 threads, a ring of
-// row slots as deep as shared memory allows (at most 32, at least 11), and
-// one block per (branch, residue, chunk) with chunks chosen so that one wave
-// covers the multiprocessors.
+// Checks the shape (host only) and sizes the launch: a branch slice of G
+// channels on 1, 2 or 4 blocks of a cluster (at most 1,280 channels each, 640
+// with 4; 2 per thread; every block but the last a multiple of 8 channels so
+// that every row copy starts and ends on 16 bytes), the fewest blocks whose
+// rings of row slots leave a batch in flight ahead, the rings as deep as
+// shared memory allows with two blocks per multiprocessor (one, with deeper
+// rings, when two leave no batch ahead), and one block per (branch,
+// residue, chunk) with chunks chosen so that one wave of clusters covers the
+// device.
 int conv_bwd_plan(const engram_conv_params_t *p, int32_t dtype, int32_t grad_dtype, int64_t T,
                   ConvBwdPlan *P)
 {
@@ -1207,8 +1213,7 @@ int conv_bwd_plan(const engram_conv_params_t *p, int32_t dtype, int32_t grad_dty
     if (ex == 0 || eg == 0 || elem_bytes(p->weight_dtype) == 0)
         return ENGRAM_EINVAL;
     const int C = p->channels, G = p->group_size, K = p->kernel_size, d = p->dilation;
-    if (C < 1 || G < 8 || C % G != 0 || G % 8 != 0 ||
-        G / 4 > ple::kBwdThreads * ple::kBwdMaxCluster)
+    if (C < 1 || G < 8 || C % G != 0 || G % 8 != 0 || G > ple::kBwdMaxChannels)
         return ENGRAM_EINVAL;
     if (K < 1 || K > ple::kBwdTaps || d < 1 || d > 4096 || p->reserved != 0)
         return ENGRAM_EINVAL;
@@ -1216,14 +1221,28 @@ int conv_bwd_plan(const engram_conv_params_t *p, int32_t dtype, int32_t grad_dty
         return ENGRAM_EINVAL;
     if (T < 0 || T > INT32_MAX)
         return ENGRAM_EINVAL;
-    // branches wider than one block's 320 threads x 4 channels: two blocks of a
-    // cluster, one half each (G / 2 stays a multiple of 4)
-    const int csize = G / 4 > ple::kBwdThreads ? 2 : 1;
-    const int gc = G / csize;
-    const int pitch_x = (gc * ex + 127) / 128 * 128, pitch_g = (gc * eg + 127) / 128 * 128;
-    const int fit = (int)((ple::kSmemLimit - ple::kBwdDataOffset) / (size_t)(pitch_x + pitch_g));
-    const int slots_max = std::min(fit, ple::kBwdMaxSlots);
-    const int ahead = std::min((slots_max - ple::kBwdLag) / ple::kBwdRows - 2, ple::kBwdBars - 2);
+    int csize = 0, gca = 0, pitch_x = 0, pitch_g = 0, pitch_u = 0, ahead = 0;
+    for (int cs = 1; cs <= ple::kBwdMaxCluster && ahead < 1; cs *= 2) {
+        gca = (int)ceil_div(G, 8 * cs) * 8;
+        const int threads = (gca / ple::kBwdCh + 31) / 32 * 32;
+        if (gca > ple::kBwdBlockChannels || cs * (threads / 32) > ple::kBwdCols ||
+            G - (cs - 1) * gca < 8)
+            continue;
+        pitch_x = (gca * ex + 127) / 128 * 128;
+        pitch_g = (gca * eg + 127) / 128 * 128;
+        pitch_u = gca * (int)sizeof(float);
+        auto ahead_for = [&](size_t budget) {
+            const int most = std::min(ple::kBwdMaxSlots / ple::kBwdRows - 3, ple::kBwdBars - 2);
+            int n = 0;
+            while (n < most && ple::bwd_smem_bytes(n + 1, pitch_x, pitch_g, pitch_u) <= budget)
+                ++n;
+            return n;
+        };
+        ahead = ahead_for(ple::kBwdTwoBlockSmem);
+        if (ahead < 1)
+            ahead = ahead_for(ple::kSmemLimit);
+        csize = cs;
+    }
     if (ahead < 1)
         return ENGRAM_EINVAL;
     ple::ConvBwdArgs &a = P->a;
@@ -1231,7 +1250,7 @@ int conv_bwd_plan(const engram_conv_params_t *p, int32_t dtype, int32_t grad_dty
     a.T = T;
     a.C = C;
     a.G = G;
-    a.nth = gc / 4;
+    a.gca = gca;
     a.dil = d;
     a.K = K;
     a.wdtype = p->weight_dtype;
@@ -1239,12 +1258,91 @@ int conv_bwd_plan(const engram_conv_params_t *p, int32_t dtype, int32_t grad_dty
     a.inv_G = 1.f / (float)G;
     a.flags = p->flags;
     a.ahead = ahead;
-    a.slots = ple::kBwdLag + (ahead + 2) * ple::kBwdRows;
+    a.nbx = ahead + 3;
+    a.nbg = ahead + 2;
     a.pitch_x = pitch_x;
     a.pitch_g = pitch_g;
+    a.pitch_u = pitch_u;
     a.csize = csize;
-    P->smem = ple::bwd_smem_bytes(a.slots, pitch_x, pitch_g);
-    P->threads = (a.nth + 31) / 32 * 32;
+    P->smem = ple::bwd_smem_bytes(ahead, pitch_x, pitch_g, pitch_u);
+    P->threads = (gca / ple::kBwdCh + 31) / 32 * 32;
+    P->dtype = dtype;
+    P->grad_dtype = grad_dtype;
+    return ENGRAM_OK;
+}
+
+template <typename XT, typename GT>
+int conv_bwd_clusters_t(const ConvBwdPlan &P, int *clusters)
+{
+    auto fn = P.a.gca == ple::kBwdBlockChannels ? ple::short_conv_bwd_kernel<XT, GT, true>
+                                                : ple::short_conv_bwd_kernel<XT, GT, false>;
+    ENGRAM_TRY(allow_smem(fn));
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3((unsigned)P.a.csize);
+    cfg.blockDim = dim3((unsigned)P.threads);
+    cfg.dynamicSmemBytes = P.smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)P.a.csize;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(clusters, fn, &cfg) != cudaSuccess)
+        return ENGRAM_ECUDA;
+    return ENGRAM_OK;
+}
+
+template <typename XT>
+int conv_bwd_clusters_x(const ConvBwdPlan &P, int *clusters)
+{
+    switch (P.grad_dtype) {
+    case ENGRAM_F32:
+        return conv_bwd_clusters_t<XT, float>(P, clusters);
+    case ENGRAM_BF16:
+        return conv_bwd_clusters_t<XT, __nv_bfloat16>(P, clusters);
+    default:
+        return conv_bwd_clusters_t<XT, __half>(P, clusters);
+    }
+}
+
+// Clusters of a checked plan that are resident at once on the current
+// device, asked once per (device, element types, cluster size, shared memory).
+int conv_bwd_clusters(const ConvBwdPlan &P, int *clusters)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return ENGRAM_ECUDA;
+    static std::mutex mu;
+    static std::map<std::tuple<int, int, int, int, size_t, int>, int> known;
+    const auto key = std::make_tuple(dev, (int)P.dtype, (int)P.grad_dtype, P.a.csize, P.smem,
+                                     P.threads);
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        auto it = known.find(key);
+        if (it != known.end()) {
+            *clusters = it->second;
+            return ENGRAM_OK;
+        }
+    }
+    int n = 0;
+    switch (P.dtype) {
+    case ENGRAM_F32:
+        ENGRAM_TRY(conv_bwd_clusters_x<float>(P, &n));
+        break;
+    case ENGRAM_BF16:
+        ENGRAM_TRY(conv_bwd_clusters_x<__nv_bfloat16>(P, &n));
+        break;
+    default:
+        ENGRAM_TRY(conv_bwd_clusters_x<__half>(P, &n));
+        break;
+    }
+    if (n < 1)
+        return ENGRAM_ECUDA;
+    std::lock_guard<std::mutex> lock(mu);
+    known[key] = n;
+    *clusters = n;
     return ENGRAM_OK;
 }
 
@@ -1252,12 +1350,12 @@ int conv_bwd_plan(const engram_conv_params_t *p, int32_t dtype, int32_t grad_dty
 int conv_bwd_grid(ConvBwdPlan *P)
 {
     ple::ConvBwdArgs &a = P->a;
-    int sms = 0;
-    ENGRAM_TRY(device_sms(&sms));
+    int clusters = 0;
+    ENGRAM_TRY(conv_bwd_clusters(*P, &clusters));
     const int groups = a.C / a.G;
     const int classes = (int)std::max<int64_t>(1, std::min<int64_t>(a.dil, a.T));
     const int64_t rows = std::max<int64_t>(1, ceil_div(a.T, a.dil));  // rows of residue 0
-    int64_t chunks = std::max<int64_t>(1, sms / ((int64_t)groups * classes * a.csize));
+    int64_t chunks = std::max<int64_t>(1, clusters / ((int64_t)groups * classes));
     chunks = std::min<int64_t>(chunks, std::max<int64_t>(1, ceil_div(rows, 16)));
     const int64_t grid = (int64_t)groups * classes * chunks * a.csize;
     if (grid > INT32_MAX)
@@ -1273,7 +1371,8 @@ int conv_bwd_grid(ConvBwdPlan *P)
 template <typename XT, typename GT>
 int launch_conv_bwd_t(const ConvBwdPlan &P, cudaStream_t s)
 {
-    auto fn = ple::short_conv_bwd_kernel<XT, GT>;
+    auto fn = P.a.gca == ple::kBwdBlockChannels ? ple::short_conv_bwd_kernel<XT, GT, true>
+                                                : ple::short_conv_bwd_kernel<XT, GT, false>;
     ENGRAM_TRY(allow_smem(fn));
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof(cfg));

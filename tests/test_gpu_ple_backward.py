@@ -152,9 +152,12 @@ def test_weight_dtypes(E, wdt):
     check(got, want, "bf16", wdt)
 
 
-@pytest.mark.parametrize("G", [8, 16, 24, 2560])
+@pytest.mark.parametrize("G", [8, 16, 24, 648, 1288, 2552, 2560])
 def test_narrow_and_widest_branches(E, G):
-    # G = 8: one active thread per block; G = 24: a partial warp; G = 2560: ten full warps
+    # G = 8: four active threads in one warp; G = 24: a partial warp; 648: one
+    # block whose last warp is partial; 1288: a cluster of 2 blocks, the
+    # second narrower; 2552 and 2560 with this fp32 dout: 4 blocks of 640
+    # channels (the last narrower for 2552, which is not a multiple of 16)
     C = 2 * G
     T = 97 if G < 1000 else 61
     x, nw, w, b, dout = inputs("bf16", "f32", "f32", T, C, 4, 50 + G)
