@@ -82,8 +82,9 @@ constexpr size_t kBwdTwoBlockSmem = 112 * 1024;
 // Shared memory: square-sum and dot partials [2][B][40] float each (by batch
 // parity; column rank * warps + warp, at most 40 columns for 2 blocks of 20
 // warps or 4 of 10; columns of absent warps stay zero), tap counts [64] int32
-// and inverse RMS [64] float per x row slot, the dot means of the batch
-// stage 4 finishes next [8] float, mbarriers [8 + 2]; then u [B][pitch_u] (fp32, each thread its own channels), the x
+// and inverse RMS [64] float2 per x row slot, the dx coefficients -inv^2 mean
+// of the rows stage 4 finishes next [8] float2 (both as equal pairs, ready
+// for the packed f32x2 operations), mbarriers [8 + 2]; then u [B][pitch_u] (fp32, each thread its own channels), the x
 // ring [(ahead + 3) * B][pitch_x] and the dout ring [(ahead + 2) * B][pitch_g]
 // of row slots, B slots per batch. An x row is read until the stage 4 of the
 // batch that lags it, a dout row until its stage 3, and batches are issued
@@ -94,8 +95,8 @@ constexpr int kBwdPartBytes = 2 * kBwdRows * kBwdCols * 4;  // one kind, both pa
 constexpr int kBwdOffDot = kBwdPartBytes;
 constexpr int kBwdOffMeta = 2 * kBwdPartBytes;
 constexpr int kBwdOffInv = kBwdOffMeta + kBwdMaxSlots * 4;
-constexpr int kBwdOffMean = kBwdOffInv + kBwdMaxSlots * 4;
-constexpr int kBwdOffBars = kBwdOffMean + kBwdRows * 4;
+constexpr int kBwdOffCoef = kBwdOffInv + kBwdMaxSlots * 8;
+constexpr int kBwdOffBars = kBwdOffCoef + kBwdRows * 8;
 constexpr int kBwdHeader = kBwdOffBars + (kBwdBars + kBwdPartBars) * 8;
 constexpr int kBwdDataOffset = (kBwdHeader + 127) / 128 * 128;
 
@@ -247,17 +248,6 @@ __device__ __forceinline__ float row_total8(const float *part, int lane)
     return v;
 }
 
-// Eight floats at a 16-byte aligned shared-window address.
-__device__ __forceinline__ void load8(uint32_t addr, float (&v)[8])
-{
-    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-                 : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3])
-                 : "r"(addr));
-    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-                 : "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7])
-                 : "r"(addr + 16));
-}
-
 // SiLU'(y) = sg + y sg (1 - sg), sg = 1 / (1 + 2^(-y log2 e)), for a pair.
 __device__ __forceinline__ float2 silu_grad2(float2 y)
 {
@@ -283,8 +273,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
     float *ss_part = reinterpret_cast<float *>(smem);
     float *dot_part = reinterpret_cast<float *>(smem + kBwdOffDot);
     int32_t *meta_s = reinterpret_cast<int32_t *>(smem + kBwdOffMeta);
-    float *inv_s = reinterpret_cast<float *>(smem + kBwdOffInv);
-    float *mean_s = reinterpret_cast<float *>(smem + kBwdOffMean);
+    float2 *inv_s = reinterpret_cast<float2 *>(smem + kBwdOffInv);
+    float2 *coef_s = reinterpret_cast<float2 *>(smem + kBwdOffCoef);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kBwdOffBars);
     uint64_t *pbars = bars + kBwdBars;  // the partners' partials of phase k land on pbars[k % 2]
     unsigned char *us = smem + kBwdDataOffset;
@@ -353,7 +343,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
         ss_part[i] = 0.f;  // (and dot_part) columns of absent warps stay zero
     for (int i = tid; i < kBwdMaxSlots; i += blockDim.x) {
         meta_s[i] = 0;
-        inv_s[i] = 1.f;  // stays 1 without the norm
+        inv_s[i] = make_float2(1.f, 1.f);  // stays 1 without the norm
     }
     // Partial sums are posted in phases: phase 0 before the batch loop,
     // phase b + 1 in iteration b. Each post is one row sum per warp and row,
@@ -365,24 +355,29 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
         if ((lane & 3) == 0) {
             float *dst = partials + (lane >> 2) * kBwdCols + pslot;
             *dst = tot;
-            for (int k = 1; k < cs; ++k)
-                st_async_cluster(dst, (q_cta + (uint32_t)k) & (uint32_t)(cs - 1), tot,
-                                 pbars + (phase & 1));
+            uint64_t *pb = pbars + (phase & 1);
+            if (cs > 1)
+                st_async_cluster(dst, q_cta ^ 1u, tot, pb);
+            if (cs > 2) {
+                st_async_cluster(dst, q_cta ^ 2u, tot, pb);
+                st_async_cluster(dst, q_cta ^ 3u, tot, pb);
+            }
         }
     };
     // End of a phase whose posts were the squares of batch bs (rows in x
-    // slots from xs0) and the dot partials of batch bd (either absent: -1):
+    // slots from xs0) and the dot partials of batch bd (its lagged rows in x
+    // slots sd_lo + q for q < 3, sd_hi + q after; either batch absent: -1):
     // this block's partials are complete after a block barrier (which also
     // orders the ring slots for reuse), the partners' once their bytes (8
     // lanes x 4 B per warp, post and partner) have landed on pbars[phase %
     // 2]. Warp 0 waits for those (lane 0 polls), then sums the partials once
-    // for the block: the rows' inverse RMS into inv_s by slot, the dot means
-    // into mean_s; the others wait at a second barrier, after which they read
-    // them. No cluster-scope release, so the global dx stores are not waited
+    // for the block: the rows' inverse RMS into inv_s by slot, the lagged
+    // rows' dx coefficients into coef_s; the others wait at a second barrier,
+    // after which they read them. No cluster-scope release, so the global dx stores are not waited
     // for. The double-buffered partials cannot be overwritten early: a block
     // posts phase k + 2 only after every partner's phase k + 1 posts, which
     // each partner makes after its warp 0 has read phase k's.
-    auto end_phase = [&](int bs, int xs0, int bd) {
+    auto end_phase = [&](int bs, int xs0, int bd, int sd_lo, int sd_hi) {
         const int nposts = do_norm ? (bs >= 0) + (bd >= 0) : 0;
         if (cs > 1 && tid == 0) {
             asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(
@@ -399,13 +394,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
             }
             if (do_norm && bs >= 0) {
                 const float v = row_total8(ss_part + (bs & 1) * PB, lane);
-                if ((lane & 3) == 0)
-                    inv_s[xs0 + (lane >> 2)] = rsqrtf(fmaf(v, a.inv_G, a.eps));
+                if ((lane & 3) == 0) {
+                    const float iv = rsqrtf(fmaf(v, a.inv_G, a.eps));
+                    inv_s[xs0 + (lane >> 2)] = make_float2(iv, iv);
+                }
             }
             if (do_norm && bd >= 0) {
                 const float v = row_total8(dot_part + (bd & 1) * PB, lane);
-                if ((lane & 3) == 0)
-                    mean_s[lane >> 2] = v * a.inv_G;
+                if ((lane & 3) == 0) {
+                    const int q = lane >> 2;
+                    const float iv = inv_s[(q < L ? sd_lo : sd_hi) + q].x;
+                    const float cf = -(iv * iv) * (v * a.inv_G);
+                    coef_s[q] = make_float2(cf, cf);
+                }
             }
         }
         __syncthreads();
@@ -519,26 +520,29 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
         if (!do_norm)
             return;
         const uint32_t xa = xs_t + (uint32_t)(xc * B) * px;
-        float ss[B];
+        auto squares = [&](auto all_tag) {
+            constexpr bool ALL = decltype(all_tag)::value;  // every row loaded
+            float ss[B];
 #pragma unroll
-        for (int i = 0; i < B; ++i) {
-            float v = 0.f;
-            if (active && j0 + i < je) {
-                const float2 x = load_pair<XT>(xa + (uint32_t)i * px);
-                v = fmaf(x.x, x.x, x.y * x.y);
+            for (int i = 0; i < B; ++i) {
+                float v = 0.f;
+                if (ALL || (active && j0 + i < je)) {
+                    const float2 x = load_pair<XT>(xa + (uint32_t)i * px);
+                    v = fmaf(x.x, x.x, x.y * x.y);
+                }
+                ss[i] = v;
             }
-            ss[i] = v;
-        }
-        post(ss_part + (b & 1) * PB, warp_sum8(ss, lane));
+            return warp_sum8(ss, lane);
+        };
+        const float tot = active && j0 + B <= je ? squares(std::true_type{})
+                                                 : squares(std::false_type{});
+        post(ss_part + (b & 1) * PB, tot);
     };
 
     // ---- stage 4 of batch b (x ring batches xc of b, xp of b - 1): dx of its
     // lagged rows j0 - 3 + q, once the dot partials it posted are complete
     auto stage4 = [&](int b, int xc, int xp) {
         const int32_t j0 = js + b * B;
-        float mean[B];
-        if (do_norm)
-            load8(smem_u32(mean_s), mean);
         const int s_lo = xp * B + B - L, s_hi = xc * B - L;  // slot of lagged row q: + q
         auto rows = [&](auto all_tag) {
             constexpr bool ALL = decltype(all_tag)::value;
@@ -551,12 +555,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
                     continue;
                 const int sl = (q < L ? s_lo : s_hi) + q;
                 float2 u = load_u(us_t + (uint32_t)q * pu);
-                if (do_norm) {
-                    const float iv = inv_s[sl];
-                    const float cf = -(iv * iv) * mean[q];
-                    u = __ffma2_rn(load_pair<XT>(xs_t + (uint32_t)sl * px), make_float2(cf, cf),
-                                   u);
-                }
+                if (do_norm)
+                    u = __ffma2_rn(load_pair<XT>(xs_t + (uint32_t)sl * px), coef_s[q], u);
                 store_pair<GT>(ALL ? drow + q * dstep : dxb + (int64_t)(r + jj * d) * grow, u);
             }
         };
@@ -572,7 +572,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
     // lane / 4)
     auto stage23 = [&](int b, int xc, int xp, int gcur, int gprev) {
         const int32_t j0 = js + b * B;
-        const float *ivn = inv_s + xc * B;  // inverse RMS of the new rows
+        const float2 *ivn = inv_s + xc * B;  // inverse RMS of the new rows
         // slots of lagged row q: q < L in the previous batch, else in this one
         const int sx_lo = xp * B + B - L, sx_hi = xc * B - L;
         const int sg_lo = gprev * B + B - L, sg_hi = gcur * B - L;
@@ -595,8 +595,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
                 // new row: normalised x into the ring, then y and dy
                 float2 xh = zero2;
                 if (FAST || (active && jn < je))
-                    xh = __fmul2_rn(load_pair<XT>(xa + (uint32_t)q * px),
-                                    make_float2(ivn[q], ivn[q]));
+                    xh = __fmul2_rn(load_pair<XT>(xa + (uint32_t)q * px), ivn[q]);
                 xr[q & 3] = xh;
                 float2 dyv = zero2;
                 if (FAST || (active && jn < je && jn >= ja)) {
@@ -631,8 +630,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
                     const float2 st = __fmul2_rn(sc, t);
                     dv = st.x + st.y;
                     // (rows of the previous batch: their inverse RMS from its stage 2)
-                    const float il = inv_s[sxl];
-                    float2 u = __fmul2_rn(__fmul2_rn(sc, make_float2(il, il)), dn);
+                    float2 u = __fmul2_rn(__fmul2_rn(sc, inv_s[sxl]), dn);
                     if (do_res)
                         u = __fadd2_rn(
                             u, load_pair<GT>(gs_t + (uint32_t)((q < L ? sg_lo : sg_hi) + q) * pg));
@@ -651,7 +649,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
     // by batch parity, so a warp that runs ahead never overwrites partials
     // another warp still reads.
     stage1(0, 0);
-    end_phase(0, 0, -1);
+    end_phase(0, 0, -1, 0, 0);
     if (wid == 0 && a.ahead < nbatch)
         issue_next(a.ahead);
     // ring batches of batches b, b - 1 and b - 2 (those of batches before the
@@ -666,7 +664,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
         const int xn = x0 + 1 == nbx ? 0 : x0 + 1;
         if (b + 1 < nbatch)
             stage1(b + 1, xn);
-        end_phase(b + 1 < nbatch ? b + 1 : -1, xn * B, b);
+        end_phase(b + 1 < nbatch ? b + 1 : -1, xn * B, b, x1 * B + B - L, x0 * B - L);
         if (wid == 0 && b + 1 + a.ahead < nbatch)
             issue_next(b + 1 + a.ahead);
         x2 = x1;
