@@ -824,7 +824,10 @@ def ple_config(args, world: int, backward: bool) -> dict:
             "cu_seqlens": f"{batch} rows", "input_seed": 5000 + s.seed,
             "parallelism": f"replicas x{world} (own batch per GPU)",
             "l2": (f"inputs larger than L2 ({T * C * 2 * (2 if backward else 1) / 1e9:.2f} "
-                   f"GB in, {T * C * 2 / 1e9:.2f} GB out)")}
+                   f"GB in, {T * C * 2 / 1e9:.2f} GB out)"),
+            **({"inverse_rms": ("the forward's, saved (made before timing)"
+                                if getattr(args, "ple_inv", "computed") == "saved"
+                                else "computed by the backward")} if backward else {})}
 
 
 def adam_config(R: int, U: int) -> dict:
@@ -868,19 +871,26 @@ def run_ple(args, backward: bool = False):
     cu = torch.from_numpy(row_bounds(batch, s.seq_len)).to(device)
     out = torch.empty_like(x)
     stream = torch.cuda.Stream(device)
+    inv = None
     if backward:
         dout = torch.randn((T, C), generator=g, device=device).to(torch.bfloat16)
         dnw, db = torch.empty(C, device=device), torch.empty(C, device=device)
         dw = torch.empty((C, K), device=device)
         ws = torch.empty(E.engram_ple_short_conv_backward_workspace_size(C, G, K, d, T),
                          dtype=torch.uint8, device=device)
+        if args.ple_inv == "saved":
+            # the forward's saved inverse RMS, as training has it (untimed)
+            inv = torch.empty((T, C // G), device=device)
+            E.engram_ple_short_conv(x, w, dilation=d, group_size=G, cu_seqlens=cu,
+                                    norm_weight=nw, conv_bias=b, out=out, inv_rms=inv)
+            torch.cuda.synchronize(device)
 
     def step(xx=x, oo=out, gg=None):
         if backward:
             E.engram_ple_short_conv_backward(
                 xx, w, dout if gg is None else gg, dilation=d, group_size=G, cu_seqlens=cu,
                 norm_weight=nw, conv_bias=b, dx=oo, dnorm_weight=dnw, dconv_weight=dw,
-                dconv_bias=db, workspace=ws, stream=stream)
+                dconv_bias=db, workspace=ws, inv_rms=inv, stream=stream)
         else:
             E.engram_ple_short_conv(xx, w, dilation=d, group_size=G, cu_seqlens=cu,
                                     norm_weight=nw, conv_bias=b, out=oo, stream=stream)
@@ -962,6 +972,8 @@ def run_ple(args, backward: bool = False):
     peak, peak_kind = hbm_peak()
     if backward:   # x, dout in; dx out; weights in; fp32 weight gradients out
         alg = T * C * 2 * 3 + C * (K + 2) * 2 + C * (K + 2) * 4 + cu.numel() * 4
+        if inv is not None:
+            alg += inv.numel() * 4
         kname = "short_conv_bwd_kernel<bf16,bf16> + conv_bwd_reduce_kernel (one call)"
         tname = "short_conv_bwd_kernel"
     else:
@@ -1317,6 +1329,9 @@ def main(argv=None):
     ap.add_argument("--bwd-sort", choices=["heads", "plain"], default="heads",
                     help="backward sort: by head (engram_backward_sort_heads, the default) "
                          "or over the whole row range (engram_backward_sort)")
+    ap.add_argument("--ple-inv", choices=["saved", "computed"], default="saved",
+                    help="--stage ple_bwd: take the forward's saved inverse RMS (training's "
+                         "path, default) or compute it in the backward")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--graph", dest="graph", action="store_true", default=True,

@@ -37,6 +37,7 @@ EXPORTED = (
     "engram_ple_short_conv_backward", "engram_ple_short_conv_backward_workspace_size",
     "engram_owner_bucket", "engram_owner_bucket_workspace_size",
     "engram_backward_heads", "engram_backward_sort_heads", "engram_owner_bucket_padded",
+    "engram_ple_short_conv_save", "engram_ple_short_conv_backward_saved",
 )
 
 ENGRAM_NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -139,10 +140,13 @@ def _load():
         "engram_backward_noalloc": [P, i64, i64, i32, P, i32, P, P, P, P],
         "engram_hash_gather_slice": [P, P, P, i32, i64, i64, i64, i64, P, i32, P, P, P],
         "engram_ple_short_conv": [P, P, i32, P, i32, i64, P, P, P, P, i32, P],
+        "engram_ple_short_conv_save": [P, P, i32, P, i32, i64, P, P, P, P, i32, P, P],
         "engram_grouped_rms_norm": [P, i32, i64, i32, i32, P, i32, ctypes.c_float, P, i32, P],
         "engram_sparse_adam": [P, P, i32, i64, i32, P, P, P, P, P, i64, P],
         "engram_ple_short_conv_backward": [P, P, i32, P, i32, i64, P, P, P, P, i32, P, P, P, P,
                                            P, sz, P],
+        "engram_ple_short_conv_backward_saved": [P, P, i32, P, i32, i64, P, P, P, P, P, i32, P,
+                                                 P, P, P, P, sz, P],
         "engram_ple_short_conv_backward_workspace_size": [P, i64, ctypes.POINTER(sz)],
         "engram_owner_bucket": [P, i64, i64, i32, P, P, P, P, P, sz, P],
         "engram_owner_bucket_workspace_size": [i64, i32, ctypes.POINTER(sz)],
@@ -440,10 +444,12 @@ def engram_ple_short_conv(x: torch.Tensor, conv_weight: torch.Tensor, *, dilatio
                           group_size: int, cu_seqlens=None, norm_weight=None, conv_bias=None,
                           eps: float = 1e-6, norm: bool = True, silu: bool = True,
                           residual: bool = True, out=None, out_dtype=None,
-                          stream=None) -> torch.Tensor:
+                          inv_rms=None, stream=None) -> torch.Tensor:
     """PLE tail over x [T, C]: x + SiLU(causal depthwise conv(grouped RMS norm(x)))
     with each of norm, SiLU and residual optional; conv_weight is [C, K] (or
-    the conv1d layout [C, 1, K]); all weights share one dtype."""
+    the conv1d layout [C, 1, K]); all weights share one dtype. inv_rms, an
+    fp32 [T, C / group_size] tensor (norm on), receives every branch slice's
+    inverse RMS for engram_ple_short_conv_backward(..., inv_rms=...)."""
     _cuda(x, "x")
     if x.dim() != 2:
         raise ValueError("x must be [T, C]")
@@ -462,11 +468,25 @@ def engram_ple_short_conv(x: torch.Tensor, conv_weight: torch.Tensor, *, dilatio
     p = ConvParams(C, int(group_size), w.shape[1], int(dilation), float(eps),
                    (ENGRAM_CONV_NORM if norm else 0) | (ENGRAM_CONV_SILU if silu else 0)
                    | (ENGRAM_CONV_RESIDUAL if residual else 0), _dtype_code(w), 0)
-    _check(lib.engram_ple_short_conv(ctypes.byref(p), _ptr(x), _dtype_code(x), _ptr(cu), nseq,
-                                     T, _ptr(norm_weight), _ptr(w), _ptr(conv_bias), _ptr(out),
-                                     _dtype_code(out), _stream(stream)),
-           "engram_ple_short_conv")
+    if inv_rms is None:
+        _check(lib.engram_ple_short_conv(ctypes.byref(p), _ptr(x), _dtype_code(x), _ptr(cu),
+                                         nseq, T, _ptr(norm_weight), _ptr(w), _ptr(conv_bias),
+                                         _ptr(out), _dtype_code(out), _stream(stream)),
+               "engram_ple_short_conv")
+        return out
+    _inv_rms_arg(inv_rms, T, C, group_size)
+    _check(lib.engram_ple_short_conv_save(ctypes.byref(p), _ptr(x), _dtype_code(x), _ptr(cu),
+                                          nseq, T, _ptr(norm_weight), _ptr(w), _ptr(conv_bias),
+                                          _ptr(out), _dtype_code(out), _ptr(inv_rms),
+                                          _stream(stream)),
+           "engram_ple_short_conv_save")
     return out
+
+
+def _inv_rms_arg(inv_rms, T, C, group_size):
+    _cuda(inv_rms, "inv_rms", torch.float32)
+    if group_size < 1 or C % group_size or inv_rms.numel() != T * (C // group_size):
+        raise ValueError("inv_rms must hold T * C / group_size floats")
 
 
 def _conv_params(C, group_size, w, dilation, eps, norm, silu, residual):
@@ -494,11 +514,14 @@ def engram_ple_short_conv_backward(x: torch.Tensor, conv_weight: torch.Tensor,
                                    eps: float = 1e-6, norm: bool = True, silu: bool = True,
                                    residual: bool = True, dx=None, dnorm_weight=None,
                                    dconv_weight=None, dconv_bias=None, workspace=None,
-                                   stream=None):
+                                   inv_rms=None, stream=None):
     """Gradients of engram_ple_short_conv's output given dout [T, C]:
     returns (dx [T, C] of dout's dtype, dnorm_weight [C], dconv_weight [C, K],
     dconv_bias [C]), the weight gradients fp32. Optional outputs and the
-    workspace (uint8) may be passed in; they are allocated otherwise."""
+    workspace (uint8) may be passed in; they are allocated otherwise.
+    inv_rms: the forward's saved inverse RMS (engram_ple_short_conv(...,
+    inv_rms=...)) for the same x, which the backward then uses instead of
+    computing it (norm on)."""
     _cuda(x, "x")
     _cuda(dout, "dout")
     if x.dim() != 2 or dout.shape != x.shape:
@@ -530,11 +553,19 @@ def engram_ple_short_conv_backward(x: torch.Tensor, conv_weight: torch.Tensor,
         need = engram_ple_short_conv_backward_workspace_size(C, group_size, K, dilation, T)
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
     _cuda(workspace, "workspace", torch.uint8)
-    _check(lib.engram_ple_short_conv_backward(
+    if inv_rms is None:
+        _check(lib.engram_ple_short_conv_backward(
+            ctypes.byref(p), _ptr(x), _dtype_code(x), _ptr(cu), nseq, T, _ptr(norm_weight),
+            _ptr(w), _ptr(conv_bias), _ptr(dout), _dtype_code(dout), _ptr(dx),
+            _ptr(dnorm_weight), _ptr(dconv_weight), _ptr(dconv_bias), _ptr(workspace),
+            workspace.numel(), _stream(stream)), "engram_ple_short_conv_backward")
+        return dx, dnorm_weight, dconv_weight, dconv_bias
+    _inv_rms_arg(inv_rms, T, C, group_size)
+    _check(lib.engram_ple_short_conv_backward_saved(
         ctypes.byref(p), _ptr(x), _dtype_code(x), _ptr(cu), nseq, T, _ptr(norm_weight), _ptr(w),
-        _ptr(conv_bias), _ptr(dout), _dtype_code(dout), _ptr(dx), _ptr(dnorm_weight),
-        _ptr(dconv_weight), _ptr(dconv_bias), _ptr(workspace), workspace.numel(),
-        _stream(stream)), "engram_ple_short_conv_backward")
+        _ptr(conv_bias), _ptr(inv_rms), _ptr(dout), _dtype_code(dout), _ptr(dx),
+        _ptr(dnorm_weight), _ptr(dconv_weight), _ptr(dconv_bias), _ptr(workspace),
+        workspace.numel(), _stream(stream)), "engram_ple_short_conv_backward_saved")
     return dx, dnorm_weight, dconv_weight, dconv_bias
 
 

@@ -955,6 +955,7 @@ int conv_plan(const engram_conv_params_t *p, int32_t dtype, int32_t out_dtype, i
     a.nth = nth;
     a.wdtype = p->weight_dtype;
     a.eps = p->eps;
+    a.groups = C / G;
     a.inv_G = 1.f / (float)G;
     a.K = K;
     a.dil = d;
@@ -1033,13 +1034,17 @@ template <typename XT, typename OT>
 int launch_conv_t(const ConvPlan &P, cudaStream_t s)
 {
     if (P.cls) {
-        auto fc = ple::short_conv_cls_kernel<XT, OT, 4>;
+        auto fc = P.a.inv_out != nullptr ? ple::short_conv_cls_kernel<XT, OT, 4, true>
+                                         : ple::short_conv_cls_kernel<XT, OT, 4, false>;
         ENGRAM_TRY(allow_smem(fc));
         fc<<<P.grid, P.threads, P.smem, s>>>(P.a);
         return after_launch();
     }
-    auto fn = P.chan == 8 ? ple::short_conv_kernel<XT, OT, 0, 8>
-                          : ple::short_conv_kernel<XT, OT, 0, 4>;
+    const bool save = P.a.inv_out != nullptr;
+    auto fn = P.chan == 8 ? (save ? ple::short_conv_kernel<XT, OT, 0, 8, true>
+                                  : ple::short_conv_kernel<XT, OT, 0, 8, false>)
+                          : (save ? ple::short_conv_kernel<XT, OT, 0, 4, true>
+                                  : ple::short_conv_kernel<XT, OT, 0, 4, false>);
     ENGRAM_TRY(allow_smem(fn));
     fn<<<P.grid, P.threads, P.smem, s>>>(P.a);
     return after_launch();
@@ -1064,15 +1069,17 @@ int launch_conv(ConvPlan &P, int32_t dtype, int32_t out_dtype, cudaStream_t s)
 
 extern "C" {
 
-int engram_ple_short_conv(const engram_conv_params_t *params, const void *x, int32_t dtype,
-                          const int32_t *cu_seqlens, int32_t nseq, int64_t T,
-                          const void *norm_weight, const void *conv_weight,
-                          const void *conv_bias, void *out, int32_t out_dtype,
-                          engram_stream_t stream)
+int engram_ple_short_conv_save(const engram_conv_params_t *params, const void *x,
+                               int32_t dtype, const int32_t *cu_seqlens, int32_t nseq, int64_t T,
+                               const void *norm_weight, const void *conv_weight,
+                               const void *conv_bias, void *out, int32_t out_dtype,
+                               float *inv_rms, engram_stream_t stream)
 {
     ConvPlan P;
     ENGRAM_TRY(conv_plan(params, dtype, out_dtype, T, &P));
     if (cu_seqlens != nullptr && nseq < 1)
+        return ENGRAM_EINVAL;
+    if (inv_rms != nullptr && !(params->flags & ENGRAM_CONV_NORM))
         return ENGRAM_EINVAL;
     if (T == 0)
         return ENGRAM_OK;
@@ -1082,6 +1089,12 @@ int engram_ple_short_conv(const engram_conv_params_t *params, const void *x, int
     const size_t n = (size_t)T * params->channels;
     if (overlaps(x, n * elem_bytes(dtype), out, n * elem_bytes(out_dtype)))
         return ENGRAM_EINVAL;
+    if (inv_rms != nullptr) {
+        const size_t ni = (size_t)T * (params->channels / params->group_size) * sizeof(float);
+        if (((uintptr_t)inv_rms & 3) != 0 || overlaps(inv_rms, ni, x, n * elem_bytes(dtype)) ||
+            overlaps(inv_rms, ni, out, n * elem_bytes(out_dtype)))
+            return ENGRAM_EINVAL;
+    }
     P.a.x = x;
     P.a.out = out;
     P.a.cu = cu_seqlens;
@@ -1089,7 +1102,18 @@ int engram_ple_short_conv(const engram_conv_params_t *params, const void *x, int
     P.a.norm_w = norm_weight;
     P.a.conv_w = conv_weight;
     P.a.bias = conv_bias;
+    P.a.inv_out = inv_rms;
     return launch_conv(P, dtype, out_dtype, (cudaStream_t)stream);
+}
+
+int engram_ple_short_conv(const engram_conv_params_t *params, const void *x, int32_t dtype,
+                          const int32_t *cu_seqlens, int32_t nseq, int64_t T,
+                          const void *norm_weight, const void *conv_weight,
+                          const void *conv_bias, void *out, int32_t out_dtype,
+                          engram_stream_t stream)
+{
+    return engram_ple_short_conv_save(params, x, dtype, cu_seqlens, nseq, T, norm_weight,
+                                      conv_weight, conv_bias, out, out_dtype, nullptr, stream);
 }
 
 int engram_grouped_rms_norm(const void *x, int32_t dtype, int64_t rows, int32_t channels,
@@ -1255,6 +1279,7 @@ int conv_bwd_plan(const engram_conv_params_t *p, int32_t dtype, int32_t grad_dty
     a.K = K;
     a.wdtype = p->weight_dtype;
     a.eps = p->eps;
+    a.groups = C / G;
     a.inv_G = 1.f / (float)G;
     a.flags = p->flags;
     a.ahead = ahead;
@@ -1421,18 +1446,21 @@ int engram_ple_short_conv_backward_workspace_size(const engram_conv_params_t *pa
     return ENGRAM_OK;
 }
 
-int engram_ple_short_conv_backward(const engram_conv_params_t *params, const void *x,
-                                   int32_t dtype, const int32_t *cu_seqlens, int32_t nseq,
-                                   int64_t T, const void *norm_weight, const void *conv_weight,
-                                   const void *conv_bias, const void *dout, int32_t grad_dtype,
-                                   void *dx, float *dnorm_weight, float *dconv_weight,
-                                   float *dconv_bias, void *workspace, size_t workspace_bytes,
-                                   engram_stream_t stream)
+int engram_ple_short_conv_backward_saved(
+    const engram_conv_params_t *params, const void *x, int32_t dtype, const int32_t *cu_seqlens,
+    int32_t nseq, int64_t T, const void *norm_weight, const void *conv_weight,
+    const void *conv_bias, const float *inv_rms, const void *dout, int32_t grad_dtype, void *dx,
+    float *dnorm_weight, float *dconv_weight, float *dconv_bias, void *workspace,
+    size_t workspace_bytes, engram_stream_t stream)
 {
     ConvBwdPlan P;
     ENGRAM_TRY(conv_bwd_plan(params, dtype, grad_dtype, T, &P));
     if (cu_seqlens != nullptr && nseq < 1)
         return ENGRAM_EINVAL;
+    if (inv_rms != nullptr &&
+        (!(params->flags & ENGRAM_CONV_NORM) || ((uintptr_t)inv_rms & 3) != 0))
+        return ENGRAM_EINVAL;
+    P.a.inv_in = inv_rms;
     if (conv_weight == nullptr || dconv_weight == nullptr)
         return ENGRAM_EINVAL;
     const int C = params->channels, K = params->kernel_size;
@@ -1480,6 +1508,20 @@ int engram_ple_short_conv_backward(const engram_conv_params_t *params, const voi
         static_cast<const float *>(workspace), T > 0 ? P.npart : 0, C, K, dconv_weight,
         dconv_bias, dnorm_weight);
     return after_launch();
+}
+
+int engram_ple_short_conv_backward(const engram_conv_params_t *params, const void *x,
+                                   int32_t dtype, const int32_t *cu_seqlens, int32_t nseq,
+                                   int64_t T, const void *norm_weight, const void *conv_weight,
+                                   const void *conv_bias, const void *dout, int32_t grad_dtype,
+                                   void *dx, float *dnorm_weight, float *dconv_weight,
+                                   float *dconv_bias, void *workspace, size_t workspace_bytes,
+                                   engram_stream_t stream)
+{
+    return engram_ple_short_conv_backward_saved(params, x, dtype, cu_seqlens, nseq, T,
+                                                norm_weight, conv_weight, conv_bias, nullptr,
+                                                dout, grad_dtype, dx, dnorm_weight, dconv_weight,
+                                                dconv_bias, workspace, workspace_bytes, stream);
 }
 
 } // extern "C"

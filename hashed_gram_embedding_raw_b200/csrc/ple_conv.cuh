@@ -65,6 +65,8 @@ struct ConvArgs {
     int32_t pitch;      // residue-class kernel: bytes per buffered row
     int32_t classes;    // residue-class kernel: residues with rows, min(dil, T)
     uint64_t cross_wait_ns; // residue-class kernel: bound of a wait on other warps
+    float *inv_out;         // [T][C / G] inverse RMS of every branch slice, or null
+    int32_t groups;         // C / G
 };
 
 // Shared memory: inverse RMS [2][kChunk] float and history-tap counts
@@ -238,8 +240,9 @@ __device__ __forceinline__ float warp_sum4(float v0, float v1, float v2, float v
 // ------------------------------------------------------------------ kernel
 
 // XT: element type of x; OT: of out; KT: kernel width (0 = runtime, <= 8);
-// CH: channels per thread in pass 2 (4 or 8).
-template <typename XT, typename OT, int KT, int CH>
+// CH: channels per thread in pass 2 (4 or 8); SAVE: also store every output
+// row's inverse RMS to inv_out.
+template <typename XT, typename OT, int KT, int CH, bool SAVE>
 __global__ void __launch_bounds__(CH == 4 ? kNarrowThreads : kWideThreads, 1)
     short_conv_kernel(const ConvArgs a)
 {
@@ -352,8 +355,12 @@ __global__ void __launch_bounds__(CH == 4 ? kNarrowThreads : kWideThreads, 1)
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1)
                 tot += __shfl_xor_sync(kFull, tot, o);
-            if (lane == 0)
-                inv_s[buf * kChunk + r] = do_norm ? rsqrtf(fmaf(tot, a.inv_G, a.eps)) : 1.f;
+            if (lane == 0) {
+                const float iv = do_norm ? rsqrtf(fmaf(tot, a.inv_G, a.eps)) : 1.f;
+                inv_s[buf * kChunk + r] = iv;
+                if (SAVE && c0 + r >= ta)  // (halo rows belong to the block before)
+                    a.inv_out[(c0 + r) * a.groups + m] = iv;
+            }
         }
         // in-sequence history taps of every row of the chunk
         for (int r = tid; r < rc; r += blockDim.x) {

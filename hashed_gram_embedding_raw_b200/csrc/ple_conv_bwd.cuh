@@ -126,6 +126,8 @@ struct ConvBwdArgs {
     int32_t nbx, nbg;       // batches held by the x ring (ahead + 3) and the dout ring (ahead + 2)
     int32_t pitch_x, pitch_g, pitch_u;
     int32_t csize;          // blocks per cluster sharing one branch slice (1, 2 or 4)
+    const float *inv_in;    // [T][C / G] inverse RMS saved by the forward, or null
+    int32_t groups;         // C / G
 };
 
 __device__ __forceinline__ uint32_t cluster_rank()
@@ -323,6 +325,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
     const bool do_norm = a.flags & ENGRAM_CONV_NORM;
     const bool do_silu = a.flags & ENGRAM_CONV_SILU;
     const bool do_res = a.flags & ENGRAM_CONV_RESIDUAL;
+    // the forward's saved inverse RMS (the norm is on): no squares to sum
+    const bool saved = a.inv_in != nullptr;
 
     // warp 0, lane i < B: rows j0 + i of every batch; each such lane keeps
     // the bounds [seq_lo, seq_hi) of the sequence holding its last row
@@ -378,7 +382,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
     // posts phase k + 2 only after every partner's phase k + 1 posts, which
     // each partner makes after its warp 0 has read phase k's.
     auto end_phase = [&](int bs, int xs0, int bd, int sd_lo, int sd_hi) {
-        const int nposts = do_norm ? (bs >= 0) + (bd >= 0) : 0;
+        const int nposts = do_norm ? (bs >= 0 && !saved) + (bd >= 0) : 0;
         if (cs > 1 && tid == 0) {
             asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(
                              smem_u32(pbars + (phase & 1))),
@@ -392,7 +396,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
                     timed_out = true;
                 __syncwarp();
             }
-            if (do_norm && bs >= 0) {
+            if (do_norm && !saved && bs >= 0) {
                 const float v = row_total8(ss_part + (bs & 1) * PB, lane);
                 if ((lane & 3) == 0) {
                     const float iv = rsqrtf(fmaf(v, a.inv_G, a.eps));
@@ -427,6 +431,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
     // from (b mod nbg) * B of the dout ring; tap counts and inverse RMS are
     // kept per x slot. Warp 0 issues the copies of batch b (lane i: row j0 +
     // i) and notes the rows' in-sequence tap counts.
+    // With the saved inverse RMS, lane i also loads row j0 + i's value when it
+    // issues the row; the value is stored to the row's slot (as a pair) at
+    // once before the loop, and in the loop just before the next iteration's
+    // barrier, so the load has an iteration to land and the barrier makes the
+    // value visible before the row is computed (at least one batch ahead).
+    float inv_pend = 0.f;
+    int inv_pend_slot = -1;
+    auto store_pending = [&]() {
+        if (inv_pend_slot >= 0) {
+            inv_s[inv_pend_slot] = make_float2(inv_pend, inv_pend);
+            inv_pend_slot = -1;
+        }
+    };
     auto issue = [&](int b, int xs0, int gs0) {
         const int32_t j0 = js + b * B;
         if (j0 >= je)
@@ -457,6 +474,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
                     seq_hi = __ldg(a.cu + seq + 1);
                 }
             meta_s[xs0 + lane] = taps_within(t - seq_lo, d) | taps_within(seq_hi - 1 - t, d) << 8;
+            if (saved) {
+                inv_pend = __ldg(a.inv_in + (int64_t)t * a.groups + m);
+                inv_pend_slot = xs0 + lane;
+            }
         }
     };
     const int nbx = a.nbx, nbg = a.nbg;
@@ -467,8 +488,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
         ig = ig + 1 == nbg ? 0 : ig + 1;
     };
     if (wid == 0)
-        for (int b = 0; b < a.ahead && b < nbatch; ++b)
+        for (int b = 0; b < a.ahead && b < nbatch; ++b) {
             issue_next(b);
+            store_pending();
+        }
 
     // this thread's weights, norm scale and bias, as channel pairs
     float2 w[KT], sc, bias;
@@ -517,7 +540,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
         // that none is still in flight when the block ends)
         if (j0 < je && !mbar_wait(bars + b % kBwdBars, (uint32_t)(b / kBwdBars) & 1u))
             timed_out = true;
-        if (!do_norm)
+        if (!do_norm || saved)
             return;
         const uint32_t xa = xs_t + (uint32_t)(xc * B) * px;
         auto squares = [&](auto all_tag) {
@@ -664,6 +687,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
         const int xn = x0 + 1 == nbx ? 0 : x0 + 1;
         if (b + 1 < nbatch)
             stage1(b + 1, xn);
+        if (wid == 0)
+            store_pending();
         end_phase(b + 1 < nbatch ? b + 1 : -1, xn * B, b, x1 * B + B - L, x0 * B - L);
         if (wid == 0 && b + 1 + a.ahead < nbatch)
             issue_next(b + 1 + a.ahead);

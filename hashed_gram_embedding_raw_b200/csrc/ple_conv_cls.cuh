@@ -88,9 +88,10 @@ __device__ __forceinline__ int cls_taps_within(int32_t span, int32_t d)
 
 // ConvArgs fields used: x, out, cu, nseq, T, C, G, bpg (chunks per residue),
 // nth (= G / 4), norm_w, conv_w, bias, wdtype, eps, inv_G, K, dil, flags,
-// reg_bufs, pitch, classes; the grid is branches x classes x bpg blocks of
-// 32 * (ceil(nth / 32) + 2) threads.
-template <typename XT, typename OT, int CH>
+// reg_bufs, pitch, classes (and with SAVE: inv_out, groups); the grid is
+// branches x classes x bpg blocks of 32 * (ceil(nth / 32) + 2) threads.
+// SAVE: also store every output row's inverse RMS to inv_out.
+template <typename XT, typename OT, int CH, bool SAVE>
 __global__ void __maxnreg__(CH == 4 ? 80 : 128)
     short_conv_cls_kernel(const ConvArgs a)
 {
@@ -204,8 +205,12 @@ __global__ void __maxnreg__(CH == 4 ? 80 : 128)
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1)
                     tot += __shfl_xor_sync(kFull, tot, o);
-                if (lane == 0)
-                    inv_s[b * B + i] = do_norm ? rsqrtf(fmaf(tot, a.inv_G, a.eps)) : 1.f;
+                if (lane == 0) {
+                    const float iv = do_norm ? rsqrtf(fmaf(tot, a.inv_G, a.eps)) : 1.f;
+                    inv_s[b * B + i] = iv;
+                    if (SAVE && j0 + i >= ja)  // (history rows belong to the block before)
+                        a.inv_out[(int64_t)(r + (j0 + i) * d) * a.groups + m] = iv;
+                }
             }
             if (sw == 1) {
                 int nv = 0;

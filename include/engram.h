@@ -374,11 +374,9 @@ ENGRAM_API int engram_ple_short_conv(const engram_conv_params_t *params, const v
  *   dnorm_weight  device, fp32 [C], or NULL (not wanted)
  *   workspace     device, >= engram_ple_short_conv_backward_workspace_size
  *                 bytes, 16-byte aligned (per-block partial sums; overwritten)
- * Limits (else ENGRAM_EINVAL): those of engram_conv_params_t, K <= 4,
- * G <= 2560, and a ring of 11 row slots -- G elements of dtype plus G of
- * grad_dtype, each rounded up to 128 bytes -- within 227 KB of shared memory
- * (every dtype pair fits up to G = 2560). Two launches; T = 0 writes zero
- * weight gradients.
+ * Limits (else ENGRAM_EINVAL): those of engram_conv_params_t, K <= 4 and
+ * G <= 2560 (every pair of element types fits). Two launches; T = 0 writes
+ * zero weight gradients.
  */
 ENGRAM_API int engram_ple_short_conv_backward(
     const engram_conv_params_t *params, const void *x, int32_t dtype,
@@ -386,6 +384,34 @@ ENGRAM_API int engram_ple_short_conv_backward(
     const void *conv_weight, const void *conv_bias, const void *dout, int32_t grad_dtype,
     void *dx, float *dnorm_weight, float *dconv_weight, float *dconv_bias, void *workspace,
     size_t workspace_bytes, engram_stream_t stream);
+
+/*
+ * engram_ple_short_conv_save -- engram_ple_short_conv that also keeps what
+ * its backward needs from the norm, as an autograd norm keeps its rstd:
+ *   inv_rms  device, fp32 [T, C / G]: inv of every token's branch slices
+ *            (ENGRAM_CONV_NORM required, else ENGRAM_EINVAL)
+ * Same arguments, limits and output otherwise.
+ */
+ENGRAM_API int engram_ple_short_conv_save(const engram_conv_params_t *params, const void *x,
+                                          int32_t dtype, const int32_t *cu_seqlens,
+                                          int32_t nseq, int64_t T, const void *norm_weight,
+                                          const void *conv_weight, const void *conv_bias,
+                                          void *out, int32_t out_dtype, float *inv_rms,
+                                          engram_stream_t stream);
+
+/*
+ * engram_ple_short_conv_backward_saved -- engram_ple_short_conv_backward
+ * given the inv_rms [T, C / G] that engram_ple_short_conv_save wrote for the
+ * same x and params (the backward then skips computing it; it does not
+ * check the values). ENGRAM_CONV_NORM required, else ENGRAM_EINVAL. Same
+ * arguments, limits, workspace and outputs otherwise.
+ */
+ENGRAM_API int engram_ple_short_conv_backward_saved(
+    const engram_conv_params_t *params, const void *x, int32_t dtype,
+    const int32_t *cu_seqlens, int32_t nseq, int64_t T, const void *norm_weight,
+    const void *conv_weight, const void *conv_bias, const float *inv_rms, const void *dout,
+    int32_t grad_dtype, void *dx, float *dnorm_weight, float *dconv_weight, float *dconv_bias,
+    void *workspace, size_t workspace_bytes, engram_stream_t stream);
 
 /* Workspace bytes engram_ple_short_conv_backward needs for T tokens on the
  * current device (it depends on the device's multiprocessor count). */

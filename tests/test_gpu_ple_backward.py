@@ -362,3 +362,84 @@ def test_replays_in_a_graph(E):
     torch.cuda.synchronize()
     for a_, b_ in zip(outs[0], outs[1]):
         assert torch.equal(a_, b_)
+
+
+def run_saved(E, x, w, nw, b, dout, cu, *, dt, gdt, wdt, group, dilation, K_fwd=None):
+    """The forward saving every slice's inverse RMS, then the backward given
+    it, against the oracle; also returns the saved values and the forward's
+    outputs with and without saving."""
+    cu_t = None if cu is None else torch.from_numpy(np.asarray(cu, np.int32)).cuda()
+    T, C = x.shape
+    xt, wt = dev(x, dt), dev(w, wdt)
+    kw = dict(dilation=dilation, group_size=group, cu_seqlens=cu_t,
+              norm_weight=None if nw is None else dev(nw, wdt),
+              conv_bias=None if b is None else dev(b, wdt))
+    inv = torch.full((T, C // group), float("nan"), device="cuda")
+    out_saved = E.engram_ple_short_conv(xt, wt, inv_rms=inv, **kw)
+    out_plain = E.engram_ple_short_conv(xt, wt, **kw)
+    dx, dnw, dw, db = E.engram_ple_short_conv_backward(xt, wt, dev(dout, gdt), inv_rms=inv, **kw)
+    torch.cuda.synchronize()
+    assert E.engram_get_device_error() == 0
+    got = (host(dx), host(dnw), host(dw), host(db))
+    want = oracle.short_conv_backward(
+        x, ORACLE_DT[dt], cu, w, decode(dout, gdt), dilation=dilation, group=group,
+        norm_w=nw, bias=b, wdtype=ORACLE_DT[wdt])
+    return got, want, inv.cpu().numpy().astype(np.float64), out_saved, out_plain
+
+
+def oracle_inv_rms(x, dt, group):
+    """Each slice's inverse RMS from the oracle's norm without a scale:
+    normalised value over input at the slice's largest input."""
+    n = oracle.grouped_rms_norm(x, ORACLE_DT[dt], group)
+    xv = decode(x, dt)
+    T, C = xv.shape
+    xs = xv.reshape(T, C // group, group)
+    k = np.abs(xs).argmax(axis=2)[..., None]
+    return (np.take_along_axis(n.reshape(T, C // group, group), k, 2) /
+            np.take_along_axis(xs, k, 2))[..., 0]
+
+
+@pytest.mark.parametrize("dt,gdt,G,K", [("bf16", "bf16", 2560, 4), ("bf16", "f32", 2560, 4),
+                                         ("bf16", "bf16", 1288, 4), ("f16", "f16", 520, 3),
+                                         ("f32", "f32", 2560, 2), ("bf16", "bf16", 64, 1)])
+def test_backward_with_the_forwards_saved_inverse_rms(E, dt, gdt, G, K):
+    # clusters of 2 (bf16, 2,560 and 1,288 channels) and 4 blocks (fp32 dout
+    # or x at 2,560), single blocks for narrow branches; sequence edges
+    C, T = 2 * G, 301
+    x, nw, w, b, dout = inputs(dt, "bf16", gdt, T, C, K, 70 + G + K)
+    cu = [0, 1, 2, 40, 200, T]
+    got, want, inv, out_saved, out_plain = run_saved(E, x, w, nw, b, dout, cu, dt=dt, gdt=gdt,
+                                                     wdt="bf16", group=G, dilation=3)
+    check(got, want, gdt, f"G={G} K={K}")
+    # saving changes no output, and the saved values are the slices' inverse RMS
+    assert torch.equal(out_saved, out_plain)
+    ref = oracle_inv_rms(x, dt, G)
+    assert np.abs(inv - ref).max() <= 1e-5 * np.abs(ref).max()
+
+
+def test_saved_inverse_rms_by_the_general_forward(E):
+    # kernel width 6 takes the general forward kernel; its saved values feed
+    # a width-4 backward of the same x just as well (they depend on x alone)
+    T, C, G = 257, 256, 128
+    x, nw, w6, b, _ = inputs("bf16", "f32", "bf16", T, C, 6, 77)
+    xt = dev(x, "bf16")
+    inv = torch.full((T, C // G), float("nan"), device="cuda")
+    E.engram_ple_short_conv(xt, dev(w6, "f32"), dilation=2, group_size=G, inv_rms=inv)
+    torch.cuda.synchronize()
+    ref = oracle_inv_rms(x, "bf16", G)
+    got = inv.cpu().numpy().astype(np.float64)
+    assert np.abs(got - ref).max() <= 1e-5 * np.abs(ref).max()
+
+
+def test_saved_inverse_rms_needs_the_norm(E):
+    x = torch.zeros(8, 64, dtype=torch.bfloat16, device="cuda")
+    w = torch.zeros(64, 4, dtype=torch.bfloat16, device="cuda")
+    inv = torch.zeros(8, 1, device="cuda")
+    with pytest.raises(E.EngramError):
+        E.engram_ple_short_conv(x, w, dilation=3, group_size=64, norm=False, inv_rms=inv)
+    with pytest.raises(E.EngramError):
+        E.engram_ple_short_conv_backward(x, w, x.clone(), dilation=3, group_size=64, norm=False,
+                                         inv_rms=inv)
+    with pytest.raises(ValueError):
+        E.engram_ple_short_conv(x, w, dilation=3, group_size=64, inv_rms=torch.zeros(8, 2,
+                                                                                     device="cuda"))
