@@ -388,9 +388,11 @@ ENGRAM_API int engram_ple_short_conv_backward(
 /*
  * engram_ple_short_conv_save -- engram_ple_short_conv that also keeps what
  * its backward needs from the norm, as an autograd norm keeps its rstd:
- *   inv_rms  device, fp32 [T, C / G]: inv of every token's branch slices
- *            (ENGRAM_CONV_NORM required, else ENGRAM_EINVAL)
- * Same arguments, limits and output otherwise.
+ *   inv_rms  device, fp32 [T, C / G], 4-byte aligned, overlapping neither x
+ *            nor out: inv of every token's branch slices (ENGRAM_CONV_NORM
+ *            required, else ENGRAM_EINVAL); NULL keeps nothing (then this is
+ *            engram_ple_short_conv)
+ * Same arguments, limits and output otherwise; saving changes no output bit.
  */
 ENGRAM_API int engram_ple_short_conv_save(const engram_conv_params_t *params, const void *x,
                                           int32_t dtype, const int32_t *cu_seqlens,
@@ -403,8 +405,11 @@ ENGRAM_API int engram_ple_short_conv_save(const engram_conv_params_t *params, co
  * engram_ple_short_conv_backward_saved -- engram_ple_short_conv_backward
  * given the inv_rms [T, C / G] that engram_ple_short_conv_save wrote for the
  * same x and params (the backward then skips computing it; it does not
- * check the values). ENGRAM_CONV_NORM required, else ENGRAM_EINVAL. Same
- * arguments, limits, workspace and outputs otherwise.
+ * check the values; 4-byte aligned). ENGRAM_CONV_NORM required, else
+ * ENGRAM_EINVAL; NULL computes them (then this is
+ * engram_ple_short_conv_backward). Same arguments, limits, workspace and
+ * outputs otherwise; the results differ from the computing form only by
+ * rounding (the saved values were summed in another order).
  */
 ENGRAM_API int engram_ple_short_conv_backward_saved(
     const engram_conv_params_t *params, const void *x, int32_t dtype,
