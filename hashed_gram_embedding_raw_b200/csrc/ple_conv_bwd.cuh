@@ -48,7 +48,7 @@
 // Batches whose rows and taps all stay inside their sequence (nearly all)
 // take a path without per-tap masks. Rows reach shared memory through rings
 // of row slots filled by cp.async.bulk (one copy per row of x and of dout,
-// issued `ahead` batches early by eight lanes of warp 0, completion on a
+// issued `ahead` batches early by eight lanes of the last warp, completion on a
 // per-batch mbarrier waited on with a time bound). Halo rows (3 before ja for
 // history, 3 after jb for dy) are read but own no output. Each block writes
 // its weight-gradient partials to a workspace, [d * chunks][4 + 2][C] fp32,
@@ -328,11 +328,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
     // the forward's saved inverse RMS (the norm is on): no squares to sum
     const bool saved = a.inv_in != nullptr;
 
-    // warp 0, lane i < B: rows j0 + i of every batch; each such lane keeps
-    // the bounds [seq_lo, seq_hi) of the sequence holding its last row
+    // The last warp issues the row copies (warp 0 has the partial sums to add
+    // between the barriers): its lane i < B takes rows j0 + i of every batch
+    // and keeps the bounds [seq_lo, seq_hi) of the sequence holding its last row
+    const int iwarp = nwarps - 1;
     int32_t seq = 0;
     int32_t seq_lo = 0, seq_hi = (int32_t)a.T;
-    if (wid == 0 && lane < B && a.cu != nullptr) {
+    if (wid == iwarp && lane < B && a.cu != nullptr) {
         const int32_t t = r + min(js + lane, nr - 1) * d;
         seq = find_sequence(a.cu, a.nseq, t);
         seq_lo = __ldg(a.cu + seq);
@@ -429,7 +431,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
     const uint32_t pu = WIDE ? kBwdBlockChannels * sizeof(float) : (uint32_t)a.pitch_u;
     // Batch b's rows take the B slots from (b mod nbx) * B of the x ring and
     // from (b mod nbg) * B of the dout ring; tap counts and inverse RMS are
-    // kept per x slot. Warp 0 issues the copies of batch b (lane i: row j0 +
+    // kept per x slot. The last warp issues the copies of batch b (lane i: row j0 +
     // i) and notes the rows' in-sequence tap counts.
     // With the saved inverse RMS, lane i also loads row j0 + i's value when it
     // issues the row; the value is stored to the row's slot (as a pair) at
@@ -487,7 +489,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
         ix = ix + 1 == nbx ? 0 : ix + 1;
         ig = ig + 1 == nbg ? 0 : ig + 1;
     };
-    if (wid == 0)
+    if (wid == iwarp)
         for (int b = 0; b < a.ahead && b < nbatch; ++b) {
             issue_next(b);
             store_pending();
@@ -673,7 +675,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
     // another warp still reads.
     stage1(0, 0);
     end_phase(0, 0, -1, 0, 0);
-    if (wid == 0 && a.ahead < nbatch)
+    if (wid == iwarp && a.ahead < nbatch)
         issue_next(a.ahead);
     // ring batches of batches b, b - 1 and b - 2 (those of batches before the
     // first are never read: their rows precede js)
@@ -687,10 +689,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) short_conv_bwd_kernel(const Co
         const int xn = x0 + 1 == nbx ? 0 : x0 + 1;
         if (b + 1 < nbatch)
             stage1(b + 1, xn);
-        if (wid == 0)
+        if (wid == iwarp)
             store_pending();
         end_phase(b + 1 < nbatch ? b + 1 : -1, xn * B, b, x1 * B + B - L, x0 * B - L);
-        if (wid == 0 && b + 1 + a.ahead < nbatch)
+        if (wid == iwarp && b + 1 + a.ahead < nbatch)
             issue_next(b + 1 + a.ahead);
         x2 = x1;
         x1 = x0;
